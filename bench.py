@@ -1,0 +1,450 @@
+"""Benchmark: causal linear-attention forward tokens/s at N=16K, d=128 (plus
+decode and global legs), as a fraction of the B200 roofline.
+
+One step = one causal forward (linattn_fwd_causal) over the
+causal_decay_d128 workload: B=4 sequences x H=16 heads x N=16384 tokens,
+d_k = d_v = 128, bf16 q/k/v ~ N(0,1)/sqrt(128), per-head decay
+lambda_h = linspace(0.9, 0.999, 16), fp32 state, outputs y, S_final, z_final.
+Under torchrun every rank runs its own batch of that size (the batch axis is
+sharded: heads and sequences are independent, so there is no data-path
+collective; weak scaling).  Timing: W untimed steps, then K steps between a
+barrier + synchronize on both sides, CUDA events on the launch stream, max
+over ranks.  Inputs (805 MB per step) are larger than the 126 MB L2.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                  [--no-e2e] [--no-legs] [--no-cpu-baseline]
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from weight_state_recurrence_b200 import inputs  # noqa: E402
+
+METRIC = "causal linear-attn fwd tokens/s (N=16K,d=128) + decode tok/s, % roofline"
+WL = inputs.WORKLOADS["causal_decay_d128"]
+WL_DEC = inputs.WORKLOADS["decode_d128"]
+WL_GLB = inputs.WORKLOADS["global_d64"]
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, "fallback"
+
+
+def causal_bytes(B, H, N, dk, dv, es=2):
+    """Algorithmic HBM bytes of one causal forward: q, k, v read once, y
+    written once, S_final / z_final written once (fp32)."""
+    return B * H * N * (2 * dk + 2 * dv) * es + B * H * (dk * dv + dk) * 4
+
+
+def causal_mma_flops(B, H, N, dk, dv):
+    """MMA flops the tensor-core kernel executes per launch (C = 128, dv
+    sliced 64 per CTA): per 128-token chunk and slice, A 128x128x128, O
+    2 x 128x64x128, qz 128x16x128, dS 128x64x128, dz 128x16x128."""
+    C = 128
+    chunks = -(-N // C)
+    slices = dv // 64
+    per = 2 * (C * C * dk + 2 * C * 64 * dk + C * 16 * dk + dk * 64 * C + dk * 16 * C)
+    return B * H * slices * chunks * per
+
+
+def decode_bytes(B, H, dk, dv, es=2):
+    """Per step: S read + written (fp32), z read + written, q/k/v read, y written."""
+    return B * H * (2 * dk * dv * 4 + 2 * dk * 4 + (2 * dk + 2 * dv) * es)
+
+
+def global_bytes(B, H, N, dk, dv, es=2):
+    return B * H * N * (2 * dk + 2 * dv) * es + B * H * (dk * dv + dk) * 4
+
+
+def traffic_record(kernel):
+    """DRAM bytes per launch from the committed ncu summary, valid only while
+    the kernel source is unchanged (sha256 of the sources it was taken on)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)[kernel]
+    except Exception:
+        return None
+    h = hashlib.sha256()
+    for rel in rec.get("sources", []):
+        try:
+            with open(os.path.join(ROOT, rel), "rb") as f:
+                h.update(f.read())
+        except OSError:
+            return None
+    if h.hexdigest() != rec.get("sha256"):
+        return None
+    return rec.get("bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason sampling during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, val in zip(names, f[5:9]):
+                if val.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def time_steps(fn, steps, warmup, world, stream):
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    return max_over_ranks(e0.elapsed_time(e1), world)
+
+
+# ---------------------------------------------------------------- legs
+def causal_leg(lib, args, world, rank, stream, hbm, tc_peak):
+    B, H, N, d = WL.B, WL.H, WL.N, WL.d
+    dev = torch.device("cuda")
+    q, k, v = inputs.qkv((B, H, N, d), (B, H, N, d), WL.seed * 1000 + rank, WL.scale,
+                         WL.dtype, device=dev)
+    lam = inputs.decay(WL).to(dev)
+    out = torch.empty_like(v)
+    S = torch.empty(B, H, d, d, device=dev)
+    z = torch.empty(B, H, d, device=dev)
+
+    def step():
+        lib.linattn_fwd_causal(q, k, v, lam, WL.eps, out, S, z, stream)
+
+    with torch.cuda.stream(stream):
+        with ClockSampler(torch.cuda.current_device()) as clk:
+            ms = time_steps(step, args.steps, args.warmup, world, stream)
+    assert lib.linattn_device_status(clear=True, stream=stream) == 0, "device error flag set"
+    per_launch_s = ms / 1e3 / args.steps
+    tokens = B * N * world * args.steps
+    value = tokens / (ms / 1e3)
+    alg = causal_bytes(B, H, N, d, d)
+    flops = causal_mma_flops(B, H, N, d, d)
+    traffic = traffic_record("causal_tc_kernel")
+    roof = {"bound": "hbm", "achieved": alg / per_launch_s / 1e9, "peak": hbm, "unit": "GB/s",
+            "frac": alg / per_launch_s / 1e9 / hbm, "traffic": traffic,
+            "algorithmic_bytes_per_launch": alg, "kernel": "causal_tc_kernel",
+            "tensor": {"mma_tflops": flops / per_launch_s / 1e12, "peak": tc_peak,
+                       "frac": flops / per_launch_s / 1e12 / tc_peak,
+                       "mma_flops_per_launch": flops}}
+    res = {"ms_per_step": ms / args.steps, "value": value, "roofline": roof,
+           "clocks": clk.summary(), "gpu_launches": args.steps}
+
+    if args.e2e:
+        # through the public API with host buffers: pinned H2D of q, k, v,
+        # the call, D2H of y, S_final, z_final, every step
+        hq, hk, hv = (t.to("cpu").pin_memory() for t in (q, k, v))
+        hy = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+        hS = torch.empty(S.shape, dtype=S.dtype, pin_memory=True)
+        hz = torch.empty(z.shape, dtype=z.dtype, pin_memory=True)
+
+        def e2e_step():
+            q.copy_(hq, non_blocking=True)
+            k.copy_(hk, non_blocking=True)
+            v.copy_(hv, non_blocking=True)
+            lib.linattn_fwd_causal(q, k, v, lam, WL.eps, out, S, z, stream)
+            hy.copy_(out, non_blocking=True)
+            hS.copy_(S, non_blocking=True)
+            hz.copy_(z, non_blocking=True)
+
+        ksteps = max(1, min(args.steps, 5))
+        with torch.cuda.stream(stream):
+            ms_e = time_steps(e2e_step, ksteps, 1, world, stream)
+        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
+        d2h = sum(t.numel() * t.element_size() for t in (hy, hS, hz))
+        res["e2e"] = {"value": B * N * world * ksteps / (ms_e / 1e3), "unit": "tokens/s",
+                      "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                      "steps": ksteps, "ms_per_step": ms_e / ksteps}
+    del q, k, v, out
+    torch.cuda.empty_cache()
+    return res
+
+
+def decode_leg(lib, args, world, rank, stream, hbm):
+    """256 sequences x 32 heads, d=128, state from a 512-token prefill, then
+    1024 decode steps captured in one CUDA graph (inputs pre-staged)."""
+    w = WL_DEC
+    B, H, d, T = w.B, w.H, w.d, w.steps
+    dev = torch.device("cuda")
+    lam = inputs.decay(w).to(dev)
+    qp, kp, vp = inputs.qkv((B, H, w.N, d), (B, H, w.N, d), w.seed * 1000 + rank, w.scale,
+                            w.dtype, device=dev)
+    S = torch.empty(B, H, d, d, device=dev)
+    z = torch.empty(B, H, d, device=dev)
+    yp = torch.empty_like(vp)
+    lib.linattn_fwd_causal(qp, kp, vp, lam, w.eps, yp, S, z, stream)
+    del qp, kp, vp, yp
+    g = torch.Generator(device=dev)
+    g.manual_seed(inputs.STEP_SEED0 + rank)
+    qs = (torch.randn(T, B, H, d, generator=g, device=dev) * w.scale).to(w.dtype)
+    ks = (torch.randn(T, B, H, d, generator=g, device=dev) * w.scale).to(w.dtype)
+    vs = (torch.randn(T, B, H, d, generator=g, device=dev) * w.scale).to(w.dtype)
+    ys = torch.empty_like(vs)
+    torch.cuda.synchronize()
+
+    def all_steps():
+        for s in range(T):
+            lib.linattn_decode_step(qs[s], ks[s], vs[s], lam, w.eps, S, z, ys[s], stream)
+
+    with torch.cuda.stream(stream):
+        all_steps()  # warm-up outside capture
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            all_steps()
+        reps = 3
+        ms = time_steps(graph.replay, reps, 1, world, stream)
+    assert lib.linattn_device_status(clear=True, stream=stream) == 0
+    del graph
+    step_s = ms / 1e3 / (reps * T)
+    alg = decode_bytes(B, H, d, d)
+    state = B * H * (2 * d * d * 4 + 2 * d * 4)
+    res = {"value": B * world / step_s, "unit": "tokens/s", "ms_per_step": step_s * 1e3,
+           "steps_per_graph": T,
+           "roofline": {"bound": "hbm", "achieved": alg / step_s / 1e9, "peak": hbm,
+                        "unit": "GB/s", "frac": alg / step_s / 1e9 / hbm,
+                        "state_frac": state / step_s / 1e9 / hbm,
+                        "traffic": traffic_record("decode_step_kernel"),
+                        "algorithmic_bytes_per_launch": alg, "kernel": "decode_step_kernel"},
+           "gpu_launches": (reps + 1) * T}
+    del qs, ks, vs, ys, S, z
+    torch.cuda.empty_cache()
+    return res
+
+
+def global_leg(lib, args, world, rank, stream, hbm):
+    w = WL_GLB
+    B, H, N, d = w.B, w.H, w.N, w.d
+    dev = torch.device("cuda")
+    q, k, v = inputs.qkv((B, H, N, d), (B, H, N, d), w.seed * 1000 + rank, w.scale, w.dtype,
+                         device=dev)
+    out = torch.empty_like(v)
+    KV = torch.empty(B, H, d, d, device=dev)
+    ks = torch.empty(B, H, d, device=dev)
+
+    def step():
+        lib.linattn_fwd_global(q, k, v, w.eps, out, KV, ks, stream)
+
+    with torch.cuda.stream(stream):
+        ms = time_steps(step, args.steps, args.warmup, world, stream)
+    per = ms / 1e3 / args.steps
+    alg = global_bytes(B, H, N, d, d)
+    res = {"value": B * N * world / per, "unit": "tokens/s", "ms_per_step": per * 1e3,
+           "roofline": {"bound": "hbm", "achieved": alg / per / 1e9, "peak": hbm,
+                        "unit": "GB/s", "frac": alg / per / 1e9 / hbm,
+                        "algorithmic_bytes_per_launch": alg}}
+    del q, k, v, out
+    torch.cuda.empty_cache()
+    return res
+
+
+# ---------------------------------------------------------------- oracle
+def oracle_sample(target_s=12.0, heads=None):
+    """Times the fp64 oracle (as it stands) on a bounded sample of the causal
+    workload: one sequence, `heads` heads, a prefix of the sequence sized to
+    take about target_s seconds.  Returns (tokens/s, cores, description)."""
+    import oracle
+    cores = oracle.num_threads(0)
+    h = heads or max(1, min(WL.H, cores))
+    n = 256
+    q, k, v = inputs.causal_inputs(WL, B=1, N=n)
+    lam = inputs.decay(WL)
+    t0 = time.perf_counter()
+    oracle.causal(q[:, :h], k[:, :h], v[:, :h], lam[:h], WL.eps)
+    dt = time.perf_counter() - t0
+    n = int(min(WL.N, max(256, n * target_s / max(dt, 1e-3))))
+    q, k, v = inputs.causal_inputs(WL, B=1, N=n)
+    t0 = time.perf_counter()
+    oracle.causal(q[:, :h], k[:, :h], v[:, :h], lam[:h], WL.eps)
+    dt = time.perf_counter() - t0
+    # a token of the workload = one position of one sequence across all H heads
+    tok_s = n * (h / WL.H) / dt
+    used = min(cores, h)
+    desc = (f"oracle causal recurrence (fp64, {used} threads) on 1 sequence x {h}/{WL.H} heads"
+            f" x {n} tokens of causal_decay_d128; tokens/s scaled by {h}/{WL.H} heads")
+    return tok_s, used, desc, dt
+
+
+def reference_arm(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    steps = []
+    per_step_target = max(1.0, min(8.0, 150.0 / max(1, args.steps + args.warmup)))
+    for i in range(args.warmup + args.steps):
+        tok_s, cores, desc, dt = oracle_sample(target_s=per_step_target)
+        if i >= args.warmup:
+            steps.append((tok_s, dt))
+    value = statistics.median(t for t, _ in steps)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": statistics.median(dt for _, dt in steps) * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": "causal_decay_d128 (B=4,H=16,N=16384,d=128,lambda_h in "
+                               "[0.9,0.999]); each step a bounded sample on the host cores"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-e2e", dest="e2e", action="store_false")
+    ap.add_argument("--no-legs", dest="legs", action="store_false")
+    ap.add_argument("--no-cpu-baseline", dest="cpu", action="store_false")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return reference_arm(args)
+
+    world, rank, local = dist_setup()
+    from weight_state_recurrence_b200 import linattn as lib
+    lib.load()
+    hbm, tcp, peak_src = peaks()
+    stream = torch.cuda.Stream()
+
+    res = causal_leg(lib, args, world, rank, stream, hbm, tcp)
+    line = {
+        "metric": METRIC, "value": res["value"], "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": res["ms_per_step"],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded torch RNG on the device, N(0,1)/sqrt(d))",
+        "config": {"workload": "causal_decay_d128: B=4 x H=16 x N=16384, d_k=d_v=128, bf16 "
+                               "q/k/v, lambda_h=linspace(0.9,0.999,16), fp32 S/z, eps=1e-6",
+                   "global_batch": WL.B * world, "seq_len": WL.N, "heads": WL.H, "d": WL.d,
+                   "parallelism": f"dp{world} (batch sharded, no data-path collective)",
+                   "l2": "inputs larger than L2 (805 MB per step)"},
+        "roofline": res["roofline"], "clocks": res["clocks"],
+        "gpu_launches": res["gpu_launches"], "peaks": peak_src,
+    }
+    if "e2e" in res:
+        line["e2e"] = res["e2e"]
+    if args.legs:
+        line["decode"] = decode_leg(lib, args, world, rank, stream, hbm)
+        line["global"] = global_leg(lib, args, world, rank, stream, hbm)
+    if args.cpu and world == 1 and rank == 0:
+        tok_s, cores, desc, _ = oracle_sample()
+        line["cpu_baseline"] = {"value": tok_s, "unit": "tokens/s", "cores": cores,
+                                "kind": "oracle", "sample": desc}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

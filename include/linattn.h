@@ -1,0 +1,140 @@
+/*
+ * linattn — kernelised causal linear attention read as a fast-weight update,
+ * for NVIDIA B200 (sm_100a).  C ABI of liblinattn.so.
+ *
+ * The operation (sources by page title and section):
+ *   [FW]  "attention is also an FFN" fast-weight article (kwkr.cn/news/587576)
+ *   [LN]  linear-attention note (tqpw.cn/news/561043)
+ *   [BSA] "Beyond self-attention: what comes after the Transformer"
+ *         (datadaily.news, section on linear attention)
+ *
+ *   phi(x) = elu(x) + 1  (x + 1 for x > 0, exp(x) otherwise; ELU alpha = 1)
+ *                        [FW] §4.1, [LN] §4.1, [BSA] linear-attention code
+ *   S_i = lambda S_{i-1} + phi(k_i) v_i^T     [FW] §2.1 (recurrence), §3.2 (decay)
+ *   z_i = lambda z_{i-1} + phi(k_i)           [FW] §4.2 (normaliser, decayed)
+ *   y_i = phi(q_i)^T S_i / (phi(q_i)^T z_i + eps)   [FW] §4.2, [LN] §3
+ *
+ * Conventions shared by every entry point
+ *   - Layouts are contiguous row-major: q, k [B, H, N, dk]; v, out
+ *     [B, H, N, dv]; S [B, H, dk, dv] (S[k][v], the [FW] §2.1 / [LN] §3
+ *     orientation); z [B, H, dk].  Decode uses N = 1 and drops that axis.
+ *   - q, k, v and out share one element type (dims.dtype); S, z, KV and ksum
+ *     are always fp32 ([FW] §4.1: the accumulated state must stay fp32).
+ *   - q and k are passed raw: phi is applied inside the library.  Any
+ *     1/sqrt(d) scaling is part of the caller's data, not of the operation.
+ *   - lambda points to H fp32 values in device memory (one decay per head),
+ *     or is NULL for lambda = 1 (no decay).  Values are used as given; the
+ *     method assumes 0 <= lambda <= 1 ([FW] §3.2).  lambda = 0 is allowed
+ *     (each token then sees only itself: lambda^0 = 1).
+ *   - eps >= 0 is added to the denominator ([FW] §4.2, [LN] §4.1 1e-6).
+ *   - Every pointer is a device pointer, 16-byte aligned.  The caller owns
+ *     every buffer.  The library allocates no memory, keeps no per-call state
+ *     and never synchronises; work is queued on `stream` (NULL: the legacy
+ *     default stream).  Inputs must not alias outputs.
+ *   - Supported sizes: dk and dv in {16, 32, 64, 128}; B, H, N >= 0 with
+ *     B*H*N*max(dk,dv) < 2^31.  dtype LINATTN_BF16 or LINATTN_F32.
+ *
+ * Errors
+ *   Arguments are checked on the host before anything is queued; a bad call
+ *   returns LINATTN_ERR_INVALID / LINATTN_ERR_UNSUPPORTED and touches nothing.
+ *   LINATTN_ERR_CUDA means a launch was refused (cudaGetLastError).  Faults
+ *   inside a kernel surface at the caller's next synchronisation.  Kernels
+ *   never trap: a bounded wait that runs out records a flag readable with
+ *   linattn_device_status().  No C++ exception crosses this interface.
+ */
+#ifndef LINATTN_H
+#define LINATTN_H
+
+#if defined(__GNUC__)
+#define LINATTN_API __attribute__((visibility("default")))
+#else
+#define LINATTN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st *linattn_stream_t;
+
+typedef enum { LINATTN_BF16 = 0, LINATTN_F32 = 1 } linattn_dtype;
+
+typedef struct {
+    int B;      /* batch */
+    int H;      /* heads */
+    int N;      /* tokens per sequence (ignored by linattn_decode_step) */
+    int dk;     /* key / feature dimension */
+    int dv;     /* value dimension */
+    int dtype;  /* linattn_dtype of q, k, v and out */
+} linattn_dims;
+
+enum {
+    LINATTN_OK = 0,
+    LINATTN_ERR_INVALID = 1,     /* NULL, negative, misaligned or aliased argument */
+    LINATTN_ERR_UNSUPPORTED = 2, /* dk, dv, dtype or size outside the supported set */
+    LINATTN_ERR_CUDA = 3,        /* the CUDA runtime refused a launch */
+    LINATTN_ERR_DEVICE = 4       /* a kernel recorded a device-side error flag */
+};
+
+/*
+ * Causal (prefill / training) forward, chunk-parallel
+ * ([FW] §3.1 triangular-mask form, §4.1 and §5.2 blockwise accumulation;
+ *  recurrence [FW] §2.1, §3.2, §4.2).
+ *   q, k   [B, H, N, dk]  dtype      v [B, H, N, dv] dtype
+ *   lambda [H] fp32 or NULL          eps >= 0
+ *   out    [B, H, N, dv]  dtype      y_i for every token (token i included)
+ *   S_final [B, H, dk, dv] fp32 or NULL   state after the last token
+ *   z_final [B, H, dk]     fp32 or NULL   normaliser after the last token
+ * The starting state is zero ([FW] §4.1 init_state, [LN] §6 init_state).
+ * N = 0 writes zero S_final / z_final and nothing else.
+ */
+LINATTN_API int linattn_fwd_causal(const linattn_dims *dims, const void *q, const void *k,
+                       const void *v, const float *lambda, float eps, void *out,
+                       float *S_final, float *z_final, linattn_stream_t stream);
+
+/*
+ * Global (non-causal) forward ([LN] §3 after the sum swap and §6 forward;
+ * [BSA] linear-attention code, here with eps):
+ *   KV = sum_n phi(k_n) v_n^T, ksum = sum_n phi(k_n),
+ *   y_i = phi(q_i)^T KV / (phi(q_i)^T ksum + eps).  No decay: the sum has no order.
+ *   out  [B, H, N, dv] dtype
+ *   KV   [B, H, dk, dv] fp32, required (written)
+ *   ksum [B, H, dk]     fp32, required (written)
+ */
+LINATTN_API int linattn_fwd_global(const linattn_dims *dims, const void *q, const void *k,
+                       const void *v, float eps, void *out, float *KV, float *ksum,
+                       linattn_stream_t stream);
+
+/*
+ * One decode step for every (b, h) ([FW] §4.1 forward_step, §3.1 constant
+ * d x d cache; [LN] §5 O(1) per token, §6 forward_autoregressive):
+ *   S <- lambda S + phi(k) v^T;  z <- lambda z + phi(k);
+ *   out = phi(q)^T S / (phi(q)^T z + eps)       (updated state, token included)
+ *   q, k [B, H, dk] dtype    v [B, H, dv] dtype    out [B, H, dv] dtype
+ *   S [B, H, dk, dv] fp32 and z [B, H, dk] fp32 are read and updated in place.
+ * dims->N is ignored.  A state produced by linattn_fwd_causal (S_final,
+ * z_final) continues exactly where the prefill stopped.
+ */
+LINATTN_API int linattn_decode_step(const linattn_dims *dims, const void *q, const void *k,
+                        const void *v, const float *lambda, float eps, float *S,
+                        float *z, void *out, linattn_stream_t stream);
+
+/* Static English text for a status code (never NULL). */
+LINATTN_API const char *linattn_status_string(int status);
+
+/*
+ * Synchronises `stream`, then returns the device-side error word of the
+ * current device (0 = no kernel recorded an error; bit 0: a bounded wait
+ * ran out).  clear != 0 resets the word afterwards.  Returns -1 if CUDA
+ * itself reports an error.
+ */
+LINATTN_API int linattn_device_status(int clear, linattn_stream_t stream);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+LINATTN_API int linattn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* LINATTN_H */

@@ -1,0 +1,140 @@
+"""Host-side checks of the C ABI (no GPU needed).
+
+The library must load on a machine without a GPU, export every entry point
+that include/linattn.h declares, and reject bad arguments with the documented
+status code before anything is queued.  Only argument combinations that are
+rejected on the host are exercised here, so no kernel is ever launched.
+"""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from weight_state_recurrence_b200 import linattn
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "linattn.h")
+
+
+def declared():
+    txt = open(HEADER).read()
+    return sorted(set(re.findall(r"\b(linattn_[a-z_]+)\s*\(", txt)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return linattn.load()
+
+
+def test_header_declares_the_entry_points():
+    assert set(declared()) == set(linattn.ENTRY_POINTS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", linattn.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = {ln.split()[-1] for ln in out.splitlines() if " T " in ln}
+    for name in declared():
+        assert name in exported, name
+        assert getattr(lib, name) is not None
+    # nothing else leaks out of the library (hidden visibility)
+    extra = {e for e in exported if e.startswith("linattn_")} - set(declared())
+    assert not extra, extra
+
+
+def test_status_strings_and_version(lib):
+    for code in range(5):
+        s = linattn.status_string(code)
+        assert isinstance(s, str) and s
+    assert linattn.status_string(99) == "unknown status"
+    assert lib.linattn_version() >= 100
+
+
+def D(B=1, H=1, N=8, dk=64, dv=64, dtype=0):
+    return linattn.linattn_dims(B, H, N, dk, dv, dtype)
+
+
+P = ctypes.c_void_p
+FAKE = P(0x7F0000000000)   # never dereferenced: every call below fails validation
+FAKE2 = P(0x7F0000100000)
+FAKE3 = P(0x7F0000200000)
+FAKE4 = P(0x7F0000300000)
+MIS = P(0x7F0000400008)    # 8-byte aligned only
+
+
+def causal(lib, d, q=FAKE, k=FAKE2, v=FAKE3, lam=None, eps=1e-6, out=FAKE4, S=None, z=None):
+    return lib.linattn_fwd_causal(ctypes.byref(d) if d is not None else None, q, k, v, lam,
+                                  eps, out, S, z, None)
+
+
+def test_causal_rejects_bad_arguments(lib):
+    assert causal(lib, None) == linattn.LINATTN_ERR_INVALID
+    assert causal(lib, D(B=-1)) == linattn.LINATTN_ERR_INVALID
+    assert causal(lib, D(N=-3)) == linattn.LINATTN_ERR_INVALID
+    assert causal(lib, D(dk=48)) == linattn.LINATTN_ERR_UNSUPPORTED
+    assert causal(lib, D(dv=256)) == linattn.LINATTN_ERR_UNSUPPORTED
+    assert causal(lib, D(dtype=7)) == linattn.LINATTN_ERR_UNSUPPORTED
+    assert causal(lib, D(B=1 << 12, H=1 << 10, N=1 << 10)) == linattn.LINATTN_ERR_UNSUPPORTED
+    assert causal(lib, D(), eps=-1.0) == linattn.LINATTN_ERR_INVALID
+    assert causal(lib, D(), eps=float("nan")) == linattn.LINATTN_ERR_INVALID
+    assert causal(lib, D(), eps=float("inf")) == linattn.LINATTN_ERR_INVALID
+    assert causal(lib, D(), q=None) == linattn.LINATTN_ERR_INVALID
+    assert causal(lib, D(), out=None) == linattn.LINATTN_ERR_INVALID
+    assert causal(lib, D(), q=MIS) == linattn.LINATTN_ERR_INVALID
+    assert causal(lib, D(), S=MIS) == linattn.LINATTN_ERR_INVALID
+    assert causal(lib, D(), lam=MIS) == linattn.LINATTN_ERR_INVALID
+    # output aliasing an input
+    assert causal(lib, D(), out=FAKE3) == linattn.LINATTN_ERR_INVALID
+    assert causal(lib, D(), out=FAKE) == linattn.LINATTN_ERR_INVALID
+
+
+def test_empty_batch_is_a_no_op(lib):
+    # B*H == 0: nothing to do, nothing launched, even with NULL buffers
+    assert causal(lib, D(B=0), q=None, k=None, v=None, out=None) == linattn.LINATTN_OK
+    d = D(H=0)
+    assert lib.linattn_fwd_global(ctypes.byref(d), None, None, None, 1e-6, None, None, None,
+                                  None) == linattn.LINATTN_OK
+    assert lib.linattn_decode_step(ctypes.byref(d), None, None, None, None, 1e-6, None, None,
+                                   None, None) == linattn.LINATTN_OK
+
+
+def test_global_rejects_bad_arguments(lib):
+    d = D()
+    g = lambda **kw: lib.linattn_fwd_global(ctypes.byref(kw.get("d", d)), kw.get("q", FAKE),
+                                            FAKE2, FAKE3, kw.get("eps", 1e-6),
+                                            kw.get("out", FAKE4), kw.get("KV", P(0x7F0000500000)),
+                                            kw.get("ks", P(0x7F0000600000)), None)
+    assert g(KV=None) == linattn.LINATTN_ERR_INVALID
+    assert g(ks=None) == linattn.LINATTN_ERR_INVALID
+    assert g(KV=MIS) == linattn.LINATTN_ERR_INVALID
+    assert g(eps=-2.0) == linattn.LINATTN_ERR_INVALID
+    assert g(d=D(dk=12)) == linattn.LINATTN_ERR_UNSUPPORTED
+    assert g(out=FAKE2) == linattn.LINATTN_ERR_INVALID
+    assert g(KV=FAKE4) == linattn.LINATTN_ERR_INVALID
+
+
+def test_decode_rejects_bad_arguments(lib):
+    d = D()
+    S, z = P(0x7F0000500000), P(0x7F0000600000)
+    dec = lambda **kw: lib.linattn_decode_step(
+        ctypes.byref(kw.get("d", d)), kw.get("q", FAKE), FAKE2, FAKE3, kw.get("lam", None),
+        kw.get("eps", 1e-6), kw.get("S", S), kw.get("z", z), kw.get("out", FAKE4), None)
+    assert dec(S=None) == linattn.LINATTN_ERR_INVALID
+    assert dec(z=None) == linattn.LINATTN_ERR_INVALID
+    assert dec(q=None) == linattn.LINATTN_ERR_INVALID
+    assert dec(out=None) == linattn.LINATTN_ERR_INVALID
+    assert dec(S=MIS) == linattn.LINATTN_ERR_INVALID
+    assert dec(eps=float("nan")) == linattn.LINATTN_ERR_INVALID
+    assert dec(d=D(dv=100)) == linattn.LINATTN_ERR_UNSUPPORTED
+    assert dec(d=D(dtype=3)) == linattn.LINATTN_ERR_UNSUPPORTED
+    assert dec(z=S) == linattn.LINATTN_ERR_INVALID          # state buffers overlap
+    assert dec(out=S) == linattn.LINATTN_ERR_INVALID
+
+
+def test_python_binding_checks_shapes():
+    import torch
+    q = torch.zeros(1, 2, 4, 64)
+    with pytest.raises(ValueError):
+        linattn.linattn_fwd_causal(q, q, torch.zeros(1, 2, 5, 64), None, 1e-6, q)

@@ -1,0 +1,176 @@
+// Chunked causal forward on CUDA cores, fp32 arithmetic throughout.
+//
+// This is the path for fp32 inputs (whose 1e-4 accuracy target rules out
+// bf16/tf32 tensor-core operands) and for sizes the tensor-core kernel does
+// not cover.  It computes the same chunked form as the tensor-core kernel
+// (fast-weight article §3.1 triangular mask, §4.1/§5.2 blockwise
+// accumulation) with C = 32 tokens per chunk.  For a chunk starting after
+// state (S, z), token t (0-based, Cv valid tokens):
+//   A[t][s]  = lambda^(t-s) phi(q_t).phi(k_s)        for s <= t, else 0
+//   y_t      = (sum_s A[t][s] v_s + lambda^(t+1) phi(q_t)^T S)
+//              / (sum_s A[t][s] + lambda^(t+1) phi(q_t).z + eps)
+//   S       <- lambda^Cv S + sum_s lambda^(Cv-1-s) phi(k_s) v_s^T
+//   z       <- lambda^Cv z + sum_s lambda^(Cv-1-s) phi(k_s)
+// which unrolls the recurrence S_i = lambda S_{i-1} + phi(k_i) v_i^T exactly.
+// One CTA owns one (b, h) and a DVS-wide slice of dv; S for the slice lives in
+// shared memory for the whole sequence.
+#pragma once
+#include "common.cuh"
+
+namespace linattn {
+
+constexpr int kSimtChunk = 32;
+
+template <int DK, int DVS>
+constexpr int causal_simt_smem_floats() {
+  constexpr int C = kSimtChunk;
+  return 2 * C * (DK + 1) + C * DVS + C * (C + 1) + DK * DVS + DK + (C + 4) + C;
+}
+
+template <int DK, int DVS, typename T>
+__global__ void __launch_bounds__(256) causal_simt_kernel(
+    const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
+    const float *__restrict__ lam, float eps, T *__restrict__ out, float *__restrict__ S_final,
+    float *__restrict__ z_final, int H, int N, int DV) {
+  constexpr int C = kSimtChunk, NT = 256, QS = DK + 1;
+  static_assert(DVS % 4 == 0, "slice must be float4-divisible");
+  extern __shared__ __align__(16) float sm[];
+  float *sQ = sm;                  // [C][DK+1]  phi(q)
+  float *sK = sQ + C * QS;         // [C][DK+1]  phi(k)
+  float *sV = sK + C * QS;         // [C][DVS]   v slice (later decay-weighted)
+  float *sA = sV + C * DVS;        // [C][C+1]   masked, decayed scores
+  float *sS = sA + C * (C + 1);    // [DK][DVS]  state slice
+  float *sz = sS + DK * DVS;       // [DK]       normaliser
+  float *pw = sz + DK;             // [C+1]      lambda^i
+  float *sqz = pw + (C + 4);       // [C]        phi(q_t).z
+
+  const int nslices = DV / DVS;
+  const long pair = blockIdx.x / nslices;
+  const int j0 = (blockIdx.x % nslices) * DVS;
+  const int h = static_cast<int>(pair % H);
+  const int tid = threadIdx.x;
+  const float L = lam ? lam[h] : 1.f;
+
+  if (tid <= C) pw[tid] = pow_int(L, tid);
+  for (int i = tid; i < DK * DVS; i += NT) sS[i] = 0.f;
+  for (int i = tid; i < DK; i += NT) sz[i] = 0.f;
+
+  const T *qp = q + pair * static_cast<long>(N) * DK;
+  const T *kp = k + pair * static_cast<long>(N) * DK;
+  const T *vp = v + pair * static_cast<long>(N) * DV;
+  T *op = out + pair * static_cast<long>(N) * DV;
+
+  for (int c0 = 0; c0 < N; c0 += C) {
+    const int Cv = min(C, N - c0);
+    __syncthreads();
+    for (int i = tid; i < C * DK; i += NT) {
+      const int t = i / DK, a = i % DK;
+      float fq = 0.f, fk = 0.f;
+      if (t < Cv) {
+        fq = phi_f32(to_f32(qp[static_cast<long>(c0 + t) * DK + a]));
+        fk = phi_f32(to_f32(kp[static_cast<long>(c0 + t) * DK + a]));
+      }
+      sQ[t * QS + a] = fq;
+      sK[t * QS + a] = fk;
+    }
+    for (int i = tid; i < C * DVS; i += NT) {
+      const int t = i / DVS, j = i % DVS;
+      sV[i] = t < Cv ? to_f32(vp[static_cast<long>(c0 + t) * DV + j0 + j]) : 0.f;
+    }
+    __syncthreads();
+    // masked decayed scores and phi(q_t).z (z is still the state before the chunk)
+    for (int i = tid; i < C * C; i += NT) {
+      const int t = i / C, s = i % C;
+      float a = 0.f;
+      if (s <= t && t < Cv) {
+        float d = 0.f;
+#pragma unroll 8
+        for (int c = 0; c < DK; ++c) d = fmaf(sQ[t * QS + c], sK[s * QS + c], d);
+        a = pw[t - s] * d;
+      }
+      sA[t * (C + 1) + s] = a;
+    }
+    for (int t = tid; t < C; t += NT) {
+      float d = 0.f;
+      for (int c = 0; c < DK; ++c) d = fmaf(sQ[t * QS + c], sz[c], d);
+      sqz[t] = d;
+    }
+    __syncthreads();
+    // outputs: each thread one token and four columns of the slice
+    for (int i = tid; i < C * (DVS / 4); i += NT) {
+      const int t = i / (DVS / 4), j = 4 * (i % (DVS / 4));
+      if (t >= Cv) continue;
+      float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
+      float rs = 0.f;
+      for (int s = 0; s <= t; ++s) {
+        const float a = sA[t * (C + 1) + s];
+        const float4 vv = *reinterpret_cast<const float4 *>(&sV[s * DVS + j]);
+        num.x = fmaf(a, vv.x, num.x);
+        num.y = fmaf(a, vv.y, num.y);
+        num.z = fmaf(a, vv.z, num.z);
+        num.w = fmaf(a, vv.w, num.w);
+        rs += a;
+      }
+      float4 in = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int c = 0; c < DK; ++c) {
+        const float fq = sQ[t * QS + c];
+        const float4 ss = *reinterpret_cast<const float4 *>(&sS[c * DVS + j]);
+        in.x = fmaf(fq, ss.x, in.x);
+        in.y = fmaf(fq, ss.y, in.y);
+        in.z = fmaf(fq, ss.z, in.z);
+        in.w = fmaf(fq, ss.w, in.w);
+      }
+      const float g = pw[t + 1];
+      const float inv = 1.f / (rs + g * sqz[t] + eps);
+      T *o = op + static_cast<long>(c0 + t) * DV + j0 + j;
+      o[0] = from_f32<T>(fmaf(g, in.x, num.x) * inv);
+      o[1] = from_f32<T>(fmaf(g, in.y, num.y) * inv);
+      o[2] = from_f32<T>(fmaf(g, in.z, num.z) * inv);
+      o[3] = from_f32<T>(fmaf(g, in.w, num.w) * inv);
+    }
+    __syncthreads();
+    // weight value rows by lambda^(Cv-1-s) for the state update
+    for (int i = tid; i < C * DVS; i += NT) {
+      const int s = i / DVS;
+      sV[i] = s < Cv ? sV[i] * pw[Cv - 1 - s] : 0.f;
+    }
+    __syncthreads();
+    const float gC = pw[Cv];
+    for (int i = tid; i < DK * (DVS / 4); i += NT) {
+      const int c = i / (DVS / 4), j = 4 * (i % (DVS / 4));
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int s = 0; s < Cv; ++s) {
+        const float f = sK[s * QS + c];
+        const float4 vv = *reinterpret_cast<const float4 *>(&sV[s * DVS + j]);
+        acc.x = fmaf(f, vv.x, acc.x);
+        acc.y = fmaf(f, vv.y, acc.y);
+        acc.z = fmaf(f, vv.z, acc.z);
+        acc.w = fmaf(f, vv.w, acc.w);
+      }
+      float4 *sp = reinterpret_cast<float4 *>(&sS[c * DVS + j]);
+      float4 st = *sp;
+      st.x = fmaf(gC, st.x, acc.x);
+      st.y = fmaf(gC, st.y, acc.y);
+      st.z = fmaf(gC, st.z, acc.z);
+      st.w = fmaf(gC, st.w, acc.w);
+      *sp = st;
+    }
+    for (int c = tid; c < DK; c += NT) {
+      float a = 0.f;
+      for (int s = 0; s < Cv; ++s) a = fmaf(sK[s * QS + c], pw[Cv - 1 - s], a);
+      sz[c] = fmaf(gC, sz[c], a);
+    }
+  }
+  __syncthreads();
+  if (S_final) {
+    for (int i = tid; i < DK * DVS; i += NT) {
+      const int c = i / DVS, j = i % DVS;
+      S_final[(pair * DK + c) * DV + j0 + j] = sS[i];
+    }
+  }
+  if (z_final && j0 == 0) {
+    for (int c = tid; c < DK; c += NT) z_final[pair * DK + c] = sz[c];
+  }
+}
+
+}  // namespace linattn

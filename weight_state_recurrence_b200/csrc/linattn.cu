@@ -1,0 +1,371 @@
+// liblinattn.so: the C-ABI host layer (argument checks, kernel choice,
+// launch configuration) over the sm_100a kernels.  See include/linattn.h for
+// the contract of every entry point.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <set>
+#include <utility>
+
+#include "../../include/linattn.h"
+#include "sm100.cuh"
+#include "common.cuh"
+#include "decode.cuh"
+#include "causal_simt.cuh"
+#include "causal_tc.cuh"
+#include "global_simt.cuh"
+
+namespace linattn {
+namespace {
+
+constexpr int kVersion = 100;  // 0.1.0
+
+using bf16 = __nv_bfloat16;
+
+bool supported_dim(int d) { return d == 16 || d == 32 || d == 64 || d == 128; }
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool overlaps(const void *a, size_t na, const void *b, size_t nb) {
+  if (!a || !b || na == 0 || nb == 0) return false;
+  const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+  return a0 < b0 + nb && b0 < a0 + na;
+}
+
+size_t elem_size(int dtype) { return dtype == LINATTN_F32 ? 4 : 2; }
+
+// Common checks on the dims struct; returns a status code.
+int check_dims(const linattn_dims *d, bool use_n) {
+  if (!d) return LINATTN_ERR_INVALID;
+  if (d->B < 0 || d->H < 0 || (use_n && d->N < 0)) return LINATTN_ERR_INVALID;
+  if (d->dtype != LINATTN_BF16 && d->dtype != LINATTN_F32) return LINATTN_ERR_UNSUPPORTED;
+  if (!supported_dim(d->dk) || !supported_dim(d->dv)) return LINATTN_ERR_UNSUPPORTED;
+  const long long n = use_n ? d->N : 1;
+  const long long big = static_cast<long long>(d->B) * d->H * n *
+                        (d->dk > d->dv ? d->dk : d->dv);
+  if (big >= (1ll << 31)) return LINATTN_ERR_UNSUPPORTED;
+  if (static_cast<long long>(d->B) * d->H * d->dk * d->dv >= (1ll << 31))
+    return LINATTN_ERR_UNSUPPORTED;
+  return LINATTN_OK;
+}
+
+bool bad_eps(float eps) { return !(eps >= 0.f) || !std::isfinite(eps); }
+
+int launch_status() {
+  return cudaGetLastError() == cudaSuccess ? LINATTN_OK : LINATTN_ERR_CUDA;
+}
+
+// Opt a kernel in to more than 48 KB of dynamic shared memory, once per
+// (kernel, device).  Keyed by the kernel's address: instantiations that share
+// a signature are still distinct kernels.
+bool set_smem_impl(const void *kernel, int bytes) {
+  static std::mutex mu;
+  static std::set<std::pair<const void *, int>> done;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  std::lock_guard<std::mutex> lock(mu);
+  if (done.count({kernel, dev})) return true;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
+      cudaSuccess)
+    return false;
+  done.insert({kernel, dev});
+  return true;
+}
+
+template <typename F>
+bool set_smem(F *kernel, int bytes) {
+  return set_smem_impl(reinterpret_cast<const void *>(kernel), bytes);
+}
+
+// ------------------------------------------------------------ tensor maps
+using EncodeTiled = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                 const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                 const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                 CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiled encode_fn() {
+  static EncodeTiled fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiled>(p);
+  });
+  return fn;
+}
+
+// [planes, rows, inner] bf16 tensor; boxes of 64 x 128 x 1 with 128-byte
+// swizzle (64 bf16 = 128 bytes per box row).
+bool make_map_bf16(CUtensorMap *m, const void *ptr, int inner, int rows, int planes) {
+  EncodeTiled enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(rows),
+                              static_cast<cuuint64_t>(planes)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(inner) * 2,
+                                 static_cast<cuuint64_t>(inner) * rows * 2};
+  const cuuint32_t box[3] = {64, 128, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Which causal kernel: LINATTN_CAUSAL_KERNEL=simt forces the CUDA-core
+// kernel (a second opinion for tests); otherwise bf16 with d_k = 128 and dv
+// a multiple of 64 takes the tensor-core kernel.
+bool use_tc_causal(const linattn_dims *d) {
+  const char *e = std::getenv("LINATTN_CAUSAL_KERNEL");
+  if (e && std::strcmp(e, "simt") == 0) return false;
+  return d->dtype == LINATTN_BF16 && d->dk == tc::DK && d->dv % tc::DVS == 0;
+}
+
+// ------------------------------------------------------------ launchers
+template <int DK, int DV, typename T>
+int launch_decode(const linattn_dims *d, const void *q, const void *k, const void *v,
+                  const float *lam, float eps, float *S, float *z, void *out,
+                  cudaStream_t s) {
+  decode_step_kernel<DK, DV, T><<<d->B * d->H, 256, 0, s>>>(
+      static_cast<const T *>(q), static_cast<const T *>(k), static_cast<const T *>(v), lam, eps,
+      S, z, static_cast<T *>(out), d->H);
+  return launch_status();
+}
+
+template <int DK, typename T>
+int decode_dv(const linattn_dims *d, const void *q, const void *k, const void *v,
+              const float *lam, float eps, float *S, float *z, void *out, cudaStream_t s) {
+  switch (d->dv) {
+    case 16: return launch_decode<DK, 16, T>(d, q, k, v, lam, eps, S, z, out, s);
+    case 32: return launch_decode<DK, 32, T>(d, q, k, v, lam, eps, S, z, out, s);
+    case 64: return launch_decode<DK, 64, T>(d, q, k, v, lam, eps, S, z, out, s);
+    case 128: return launch_decode<DK, 128, T>(d, q, k, v, lam, eps, S, z, out, s);
+  }
+  return LINATTN_ERR_UNSUPPORTED;
+}
+
+template <typename T>
+int decode_dispatch(const linattn_dims *d, const void *q, const void *k, const void *v,
+                    const float *lam, float eps, float *S, float *z, void *out,
+                    cudaStream_t s) {
+  switch (d->dk) {
+    case 16: return decode_dv<16, T>(d, q, k, v, lam, eps, S, z, out, s);
+    case 32: return decode_dv<32, T>(d, q, k, v, lam, eps, S, z, out, s);
+    case 64: return decode_dv<64, T>(d, q, k, v, lam, eps, S, z, out, s);
+    case 128: return decode_dv<128, T>(d, q, k, v, lam, eps, S, z, out, s);
+  }
+  return LINATTN_ERR_UNSUPPORTED;
+}
+
+template <int DK, int DVS, typename T>
+int launch_causal_simt(const linattn_dims *d, const void *q, const void *k, const void *v,
+                       const float *lam, float eps, void *out, float *S_final, float *z_final,
+                       cudaStream_t s) {
+  auto *kern = causal_simt_kernel<DK, DVS, T>;
+  const int bytes = causal_simt_smem_floats<DK, DVS>() * 4;
+  if (!set_smem(kern, bytes)) return LINATTN_ERR_CUDA;
+  const int grid = d->B * d->H * (d->dv / DVS);
+  kern<<<grid, 256, bytes, s>>>(static_cast<const T *>(q), static_cast<const T *>(k),
+                                static_cast<const T *>(v), lam, eps, static_cast<T *>(out),
+                                S_final, z_final, d->H, d->N, d->dv);
+  return launch_status();
+}
+
+template <int DK, typename T>
+int causal_simt_dv(const linattn_dims *d, const void *q, const void *k, const void *v,
+                   const float *lam, float eps, void *out, float *S_final, float *z_final,
+                   cudaStream_t s) {
+  if (d->dv == 16)
+    return launch_causal_simt<DK, 16, T>(d, q, k, v, lam, eps, out, S_final, z_final, s);
+  return launch_causal_simt<DK, 32, T>(d, q, k, v, lam, eps, out, S_final, z_final, s);
+}
+
+template <typename T>
+int causal_simt_dispatch(const linattn_dims *d, const void *q, const void *k, const void *v,
+                         const float *lam, float eps, void *out, float *S_final, float *z_final,
+                         cudaStream_t s) {
+  switch (d->dk) {
+    case 16: return causal_simt_dv<16, T>(d, q, k, v, lam, eps, out, S_final, z_final, s);
+    case 32: return causal_simt_dv<32, T>(d, q, k, v, lam, eps, out, S_final, z_final, s);
+    case 64: return causal_simt_dv<64, T>(d, q, k, v, lam, eps, out, S_final, z_final, s);
+    case 128: return causal_simt_dv<128, T>(d, q, k, v, lam, eps, out, S_final, z_final, s);
+  }
+  return LINATTN_ERR_UNSUPPORTED;
+}
+
+int launch_causal_tc(const linattn_dims *d, const void *q, const void *k, const void *v,
+                     const float *lam, float eps, void *out, float *S_final, float *z_final,
+                     cudaStream_t s) {
+  const int BH = d->B * d->H;
+  CUtensorMap mq, mk, mv, my;
+  if (!make_map_bf16(&mq, q, d->dk, d->N, BH) || !make_map_bf16(&mk, k, d->dk, d->N, BH) ||
+      !make_map_bf16(&mv, v, d->dv, d->N, BH) || !make_map_bf16(&my, out, d->dv, d->N, BH))
+    return LINATTN_ERR_CUDA;
+  if (!set_smem(tc::causal_tc_kernel, static_cast<int>(tc::kSmemBytes))) return LINATTN_ERR_CUDA;
+  const int grid = BH * (d->dv / tc::DVS);
+  tc::causal_tc_kernel<<<grid, tc::NT, tc::kSmemBytes, s>>>(mq, mk, mv, my, lam, eps, S_final,
+                                                           z_final, d->H, d->N, d->dv);
+  return launch_status();
+}
+
+template <int DK, int DV, typename T>
+int launch_global_simt(const linattn_dims *d, const void *q, const void *k, const void *v,
+                       float eps, void *out, float *KV, float *ksum, cudaStream_t s) {
+  const int BH = d->B * d->H;
+  dim3 g1(BH, (d->N + kGlobalSplit - 1) / kGlobalSplit);
+  global_kv_simt_kernel<DK, DV, T><<<g1, 256, 0, s>>>(
+      static_cast<const T *>(k), static_cast<const T *>(v), KV, ksum, d->N);
+  if (cudaGetLastError() != cudaSuccess) return LINATTN_ERR_CUDA;
+  auto *kern = global_out_simt_kernel<DK, DV, T>;
+  const int bytes = (DK * DV + DK + kGlobalTile * (DK + 1) + kGlobalTile) * 4;
+  if (!set_smem(kern, bytes)) return LINATTN_ERR_CUDA;
+  dim3 g2(BH, (d->N + kGlobalTile - 1) / kGlobalTile);
+  kern<<<g2, 256, bytes, s>>>(static_cast<const T *>(q), KV, ksum, eps, static_cast<T *>(out),
+                              d->N);
+  return launch_status();
+}
+
+template <int DK, typename T>
+int global_dv(const linattn_dims *d, const void *q, const void *k, const void *v, float eps,
+              void *out, float *KV, float *ksum, cudaStream_t s) {
+  switch (d->dv) {
+    case 16: return launch_global_simt<DK, 16, T>(d, q, k, v, eps, out, KV, ksum, s);
+    case 32: return launch_global_simt<DK, 32, T>(d, q, k, v, eps, out, KV, ksum, s);
+    case 64: return launch_global_simt<DK, 64, T>(d, q, k, v, eps, out, KV, ksum, s);
+    case 128: return launch_global_simt<DK, 128, T>(d, q, k, v, eps, out, KV, ksum, s);
+  }
+  return LINATTN_ERR_UNSUPPORTED;
+}
+
+template <typename T>
+int global_dispatch(const linattn_dims *d, const void *q, const void *k, const void *v,
+                    float eps, void *out, float *KV, float *ksum, cudaStream_t s) {
+  switch (d->dk) {
+    case 16: return global_dv<16, T>(d, q, k, v, eps, out, KV, ksum, s);
+    case 32: return global_dv<32, T>(d, q, k, v, eps, out, KV, ksum, s);
+    case 64: return global_dv<64, T>(d, q, k, v, eps, out, KV, ksum, s);
+    case 128: return global_dv<128, T>(d, q, k, v, eps, out, KV, ksum, s);
+  }
+  return LINATTN_ERR_UNSUPPORTED;
+}
+
+}  // namespace
+}  // namespace linattn
+
+using namespace linattn;
+
+extern "C" int linattn_fwd_causal(const linattn_dims *d, const void *q, const void *k,
+                                  const void *v, const float *lambda, float eps, void *out,
+                                  float *S_final, float *z_final, linattn_stream_t stream) {
+  int rc = check_dims(d, true);
+  if (rc != LINATTN_OK) return rc;
+  if (bad_eps(eps)) return LINATTN_ERR_INVALID;
+  const size_t BH = static_cast<size_t>(d->B) * d->H;
+  if (BH == 0) return LINATTN_OK;
+  const size_t es = elem_size(d->dtype);
+  const size_t nq = BH * d->N * d->dk * es, nv = BH * d->N * d->dv * es;
+  const size_t nS = BH * d->dk * d->dv * 4, nz = BH * d->dk * 4;
+  if (d->N > 0 && (!q || !k || !v || !out)) return LINATTN_ERR_INVALID;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
+      !aligned16(S_final) || !aligned16(z_final) || !aligned16(lambda))
+    return LINATTN_ERR_INVALID;
+  if (overlaps(out, nv, q, nq) || overlaps(out, nv, k, nq) || overlaps(out, nv, v, nv) ||
+      overlaps(S_final, nS, out, nv) || overlaps(z_final, nz, out, nv) ||
+      overlaps(S_final, nS, z_final, nz))
+    return LINATTN_ERR_INVALID;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (d->N == 0) {
+    if (S_final && cudaMemsetAsync(S_final, 0, nS, s) != cudaSuccess) return LINATTN_ERR_CUDA;
+    if (z_final && cudaMemsetAsync(z_final, 0, nz, s) != cudaSuccess) return LINATTN_ERR_CUDA;
+    return LINATTN_OK;
+  }
+  if (use_tc_causal(d)) return launch_causal_tc(d, q, k, v, lambda, eps, out, S_final, z_final, s);
+  if (d->dtype == LINATTN_F32)
+    return causal_simt_dispatch<float>(d, q, k, v, lambda, eps, out, S_final, z_final, s);
+  return causal_simt_dispatch<bf16>(d, q, k, v, lambda, eps, out, S_final, z_final, s);
+}
+
+extern "C" int linattn_fwd_global(const linattn_dims *d, const void *q, const void *k,
+                                  const void *v, float eps, void *out, float *KV, float *ksum,
+                                  linattn_stream_t stream) {
+  int rc = check_dims(d, true);
+  if (rc != LINATTN_OK) return rc;
+  if (bad_eps(eps)) return LINATTN_ERR_INVALID;
+  const size_t BH = static_cast<size_t>(d->B) * d->H;
+  if (BH == 0) return LINATTN_OK;
+  if (!KV || !ksum) return LINATTN_ERR_INVALID;
+  const size_t es = elem_size(d->dtype);
+  const size_t nq = BH * d->N * d->dk * es, nv = BH * d->N * d->dv * es;
+  const size_t nS = BH * d->dk * d->dv * 4, nz = BH * d->dk * 4;
+  if (d->N > 0 && (!q || !k || !v || !out)) return LINATTN_ERR_INVALID;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(KV) ||
+      !aligned16(ksum))
+    return LINATTN_ERR_INVALID;
+  if (overlaps(out, nv, q, nq) || overlaps(out, nv, k, nq) || overlaps(out, nv, v, nv) ||
+      overlaps(KV, nS, out, nv) || overlaps(ksum, nz, out, nv) || overlaps(KV, nS, ksum, nz) ||
+      overlaps(KV, nS, k, nq) || overlaps(KV, nS, v, nv))
+    return LINATTN_ERR_INVALID;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(KV, 0, nS, s) != cudaSuccess) return LINATTN_ERR_CUDA;
+  if (cudaMemsetAsync(ksum, 0, nz, s) != cudaSuccess) return LINATTN_ERR_CUDA;
+  if (d->N == 0) return LINATTN_OK;
+  if (d->dtype == LINATTN_F32)
+    return global_dispatch<float>(d, q, k, v, eps, out, KV, ksum, s);
+  return global_dispatch<bf16>(d, q, k, v, eps, out, KV, ksum, s);
+}
+
+extern "C" int linattn_decode_step(const linattn_dims *d, const void *q, const void *k,
+                                   const void *v, const float *lambda, float eps, float *S,
+                                   float *z, void *out, linattn_stream_t stream) {
+  int rc = check_dims(d, false);
+  if (rc != LINATTN_OK) return rc;
+  if (bad_eps(eps)) return LINATTN_ERR_INVALID;
+  const size_t BH = static_cast<size_t>(d->B) * d->H;
+  if (BH == 0) return LINATTN_OK;
+  if (!q || !k || !v || !S || !z || !out) return LINATTN_ERR_INVALID;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(S) || !aligned16(z) ||
+      !aligned16(out) || !aligned16(lambda))
+    return LINATTN_ERR_INVALID;
+  const size_t es = elem_size(d->dtype);
+  const size_t nq = BH * d->dk * es, nv = BH * d->dv * es;
+  const size_t nS = BH * d->dk * d->dv * 4, nz = BH * d->dk * 4;
+  if (overlaps(out, nv, q, nq) || overlaps(out, nv, k, nq) || overlaps(out, nv, v, nv) ||
+      overlaps(S, nS, out, nv) || overlaps(z, nz, out, nv) || overlaps(S, nS, z, nz) ||
+      overlaps(S, nS, q, nq) || overlaps(S, nS, k, nq) || overlaps(S, nS, v, nv))
+    return LINATTN_ERR_INVALID;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (d->dtype == LINATTN_F32)
+    return decode_dispatch<float>(d, q, k, v, lambda, eps, S, z, out, s);
+  return decode_dispatch<bf16>(d, q, k, v, lambda, eps, S, z, out, s);
+}
+
+extern "C" const char *linattn_status_string(int status) {
+  switch (status) {
+    case LINATTN_OK: return "ok";
+    case LINATTN_ERR_INVALID: return "invalid argument (NULL, negative, misaligned or aliased)";
+    case LINATTN_ERR_UNSUPPORTED: return "unsupported size or dtype";
+    case LINATTN_ERR_CUDA: return "CUDA runtime error at launch";
+    case LINATTN_ERR_DEVICE: return "a kernel recorded a device-side error";
+  }
+  return "unknown status";
+}
+
+extern "C" int linattn_device_status(int clear, linattn_stream_t stream) {
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return -1;
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_status, sizeof(v)) != cudaSuccess) return -1;
+  if (clear) {
+    const unsigned int zero = 0;
+    if (cudaMemcpyToSymbol(g_status, &zero, sizeof(zero)) != cudaSuccess) return -1;
+  }
+  return static_cast<int>(v);
+}
+
+extern "C" int linattn_version(void) { return kVersion; }

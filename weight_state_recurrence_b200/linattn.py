@@ -1,0 +1,210 @@
+"""Thin ctypes binding over liblinattn.so (include/linattn.h).
+
+The functions named ``linattn_*`` mirror the C entry points one to one and do
+argument marshalling only: shapes and dtypes of torch tensors are turned into
+a ``linattn_dims`` struct, device pointers and the current CUDA stream.  Every
+step of the computation runs in the library's kernels.  There is no CPU or
+PyTorch fallback: if the library cannot be loaded, the call raises.
+
+``fwd_causal`` / ``fwd_global`` / ``decode_step`` are conveniences that
+allocate the outputs with torch and call the entry points.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "liblinattn.so")
+
+LINATTN_BF16, LINATTN_F32 = 0, 1
+LINATTN_OK = 0
+LINATTN_ERR_INVALID = 1
+LINATTN_ERR_UNSUPPORTED = 2
+LINATTN_ERR_CUDA = 3
+LINATTN_ERR_DEVICE = 4
+
+ENTRY_POINTS = ("linattn_fwd_causal", "linattn_fwd_global", "linattn_decode_step",
+                "linattn_status_string", "linattn_device_status", "linattn_version")
+
+
+class linattn_dims(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("N", ctypes.c_int),
+                ("dk", ctypes.c_int), ("dv", ctypes.c_int), ("dtype", ctypes.c_int)]
+
+
+class LinattnError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: status {code} ({status_string(code)})")
+
+
+_lib = None
+
+
+def load(build_if_missing: bool = True):
+    """Load liblinattn.so (building it with nvcc first if it is missing or
+    older than its sources)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if build_if_missing:
+        from . import build as _build
+        try:
+            _build.build()
+        except Exception:
+            if not os.path.exists(LIB_PATH):
+                raise
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"CUDA library missing: {LIB_PATH}")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, fp, i, f = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+    dp = ctypes.POINTER(linattn_dims)
+    lib.linattn_fwd_causal.argtypes = [dp, vp, vp, vp, fp, f, vp, fp, fp, vp]
+    lib.linattn_fwd_causal.restype = i
+    lib.linattn_fwd_global.argtypes = [dp, vp, vp, vp, f, vp, fp, fp, vp]
+    lib.linattn_fwd_global.restype = i
+    lib.linattn_decode_step.argtypes = [dp, vp, vp, vp, fp, f, fp, fp, vp, vp]
+    lib.linattn_decode_step.restype = i
+    lib.linattn_status_string.argtypes = [i]
+    lib.linattn_status_string.restype = ctypes.c_char_p
+    lib.linattn_device_status.argtypes = [i, vp]
+    lib.linattn_device_status.restype = i
+    lib.linattn_version.argtypes = []
+    lib.linattn_version.restype = i
+    _lib = lib
+    return lib
+
+
+def status_string(code: int) -> str:
+    return load().linattn_status_string(int(code)).decode()
+
+
+def _dtype_code(t: torch.dtype) -> int:
+    if t == torch.bfloat16:
+        return LINATTN_BF16
+    if t == torch.float32:
+        return LINATTN_F32
+    raise TypeError(f"unsupported dtype {t}")
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensor must live on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensor must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _check(code, where):
+    if code != LINATTN_OK:
+        raise LinattnError(code, where)
+
+
+def _f32(t, shape, name):
+    if t is None:
+        return
+    if t.dtype != torch.float32 or tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must be float32 with shape {tuple(shape)}")
+
+
+def linattn_fwd_causal(q, k, v, lam, eps, out, S_final=None, z_final=None, stream=None):
+    """Causal forward: q, k [B,H,N,dk], v/out [B,H,N,dv] (bf16 or fp32),
+    lam [H] fp32 or None, S_final [B,H,dk,dv] / z_final [B,H,dk] fp32 or None."""
+    B, H, N, dk = q.shape
+    dv = v.shape[-1]
+    if k.shape != q.shape or tuple(v.shape) != (B, H, N, dv) or out.shape != v.shape:
+        raise ValueError("shape mismatch among q, k, v, out")
+    if not (q.dtype == k.dtype == v.dtype == out.dtype):
+        raise ValueError("q, k, v, out must share one dtype")
+    _f32(lam, (H,), "lambda")
+    _f32(S_final, (B, H, dk, dv), "S_final")
+    _f32(z_final, (B, H, dk), "z_final")
+    d = linattn_dims(B, H, N, dk, dv, _dtype_code(q.dtype))
+    _check(load().linattn_fwd_causal(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), _ptr(lam),
+                                     float(eps), _ptr(out), _ptr(S_final), _ptr(z_final),
+                                     _stream(stream)), "linattn_fwd_causal")
+
+
+def linattn_fwd_global(q, k, v, eps, out, KV, ksum, stream=None):
+    """Global forward: q, k [B,H,N,dk], v/out [B,H,N,dv]; KV [B,H,dk,dv] and
+    ksum [B,H,dk] fp32 are written."""
+    B, H, N, dk = q.shape
+    dv = v.shape[-1]
+    if k.shape != q.shape or tuple(v.shape) != (B, H, N, dv) or out.shape != v.shape:
+        raise ValueError("shape mismatch among q, k, v, out")
+    if not (q.dtype == k.dtype == v.dtype == out.dtype):
+        raise ValueError("q, k, v, out must share one dtype")
+    _f32(KV, (B, H, dk, dv), "KV")
+    _f32(ksum, (B, H, dk), "ksum")
+    d = linattn_dims(B, H, N, dk, dv, _dtype_code(q.dtype))
+    _check(load().linattn_fwd_global(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), float(eps),
+                                     _ptr(out), _ptr(KV), _ptr(ksum), _stream(stream)),
+           "linattn_fwd_global")
+
+
+def linattn_decode_step(q, k, v, lam, eps, S, z, out, stream=None):
+    """One decode step: q, k [B,H,dk], v/out [B,H,dv]; S [B,H,dk,dv] and z
+    [B,H,dk] fp32 are updated in place."""
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    if k.shape != q.shape or tuple(v.shape) != (B, H, dv) or out.shape != v.shape:
+        raise ValueError("shape mismatch among q, k, v, out")
+    if not (q.dtype == k.dtype == v.dtype == out.dtype):
+        raise ValueError("q, k, v, out must share one dtype")
+    _f32(lam, (H,), "lambda")
+    _f32(S, (B, H, dk, dv), "S")
+    _f32(z, (B, H, dk), "z")
+    d = linattn_dims(B, H, 1, dk, dv, _dtype_code(q.dtype))
+    _check(load().linattn_decode_step(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), _ptr(lam),
+                                      float(eps), _ptr(S), _ptr(z), _ptr(out), _stream(stream)),
+           "linattn_decode_step")
+
+
+def linattn_status_string(code: int) -> str:
+    return status_string(code)
+
+
+def linattn_device_status(clear: bool = True, stream=None) -> int:
+    return load().linattn_device_status(int(bool(clear)), _stream(stream))
+
+
+def linattn_version() -> int:
+    return load().linattn_version()
+
+
+# ---------------------------------------------------------------- helpers
+def fwd_causal(q, k, v, lam=None, eps=1e-6, want_state=True, stream=None):
+    B, H, N, dk = q.shape
+    dv = v.shape[-1]
+    out = torch.empty_like(v)
+    S = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device) if want_state else None
+    z = torch.empty((B, H, dk), dtype=torch.float32, device=q.device) if want_state else None
+    linattn_fwd_causal(q, k, v, lam, eps, out, S, z, stream)
+    return out, S, z
+
+
+def fwd_global(q, k, v, eps=1e-6, stream=None):
+    B, H, N, dk = q.shape
+    dv = v.shape[-1]
+    out = torch.empty_like(v)
+    KV = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
+    ks = torch.empty((B, H, dk), dtype=torch.float32, device=q.device)
+    linattn_fwd_global(q, k, v, eps, out, KV, ks, stream)
+    return out, KV, ks
+
+
+def decode_step(q, k, v, S, z, lam=None, eps=1e-6, stream=None):
+    out = torch.empty_like(v)
+    linattn_decode_step(q, k, v, lam, eps, S, z, out, stream)
+    return out
