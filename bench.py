@@ -13,6 +13,10 @@ over ranks.  Inputs (805 MB per step) are larger than the 126 MB L2.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                   [--no-e2e] [--no-legs] [--no-cpu-baseline]
+                  [--only causal|decode|global] [--batch B] [--dec-batch B]
+                  [--dec-steps T]
+The last four options shrink or isolate a leg for profiler captures; the
+reported benchmark always uses the full workloads (their defaults).
 """
 from __future__ import annotations
 
@@ -57,12 +61,13 @@ def causal_bytes(B, H, N, dk, dv, es=2):
 
 def causal_mma_flops(B, H, N, dk, dv):
     """MMA flops the tensor-core kernel executes per launch (C = 128, dv
-    sliced 64 per CTA): per 128-token chunk and slice, A 128x128x128, O
-    2 x 128x64x128, qz 128x16x128, dS 128x64x128, dz 128x16x128."""
+    sliced 64 per CTA).  Per 128-token chunk and slice: scores 128x128xdk;
+    O_in, O_x and the state update 128x64x128 each; row sums, phi(q).z and
+    dz 128x16x128 each."""
     C = 128
     chunks = -(-N // C)
     slices = dv // 64
-    per = 2 * (C * C * dk + 2 * C * 64 * dk + C * 16 * dk + dk * 64 * C + dk * 16 * C)
+    per = 2 * (C * C * dk + 3 * C * 64 * 128 + 3 * C * 16 * 128)
     return B * H * slices * chunks * per
 
 
@@ -200,7 +205,7 @@ def time_steps(fn, steps, warmup, world, stream):
 
 # ---------------------------------------------------------------- legs
 def causal_leg(lib, args, world, rank, stream, hbm, tc_peak):
-    B, H, N, d = WL.B, WL.H, WL.N, WL.d
+    B, H, N, d = args.batch or WL.B, WL.H, WL.N, WL.d
     dev = torch.device("cuda")
     q, k, v = inputs.qkv((B, H, N, d), (B, H, N, d), WL.seed * 1000 + rank, WL.scale,
                          WL.dtype, device=dev)
@@ -265,7 +270,7 @@ def decode_leg(lib, args, world, rank, stream, hbm):
     """256 sequences x 32 heads, d=128, state from a 512-token prefill, then
     1024 decode steps captured in one CUDA graph (inputs pre-staged)."""
     w = WL_DEC
-    B, H, d, T = w.B, w.H, w.d, w.steps
+    B, H, d, T = args.dec_batch or w.B, w.H, w.d, args.dec_steps or w.steps
     dev = torch.device("cuda")
     lam = inputs.decay(w).to(dev)
     qp, kp, vp = inputs.qkv((B, H, w.N, d), (B, H, w.N, d), w.seed * 1000 + rank, w.scale,
@@ -403,6 +408,10 @@ def main():
     ap.add_argument("--no-e2e", dest="e2e", action="store_false")
     ap.add_argument("--no-legs", dest="legs", action="store_false")
     ap.add_argument("--no-cpu-baseline", dest="cpu", action="store_false")
+    ap.add_argument("--only", default="all", choices=["all", "causal", "decode", "global"])
+    ap.add_argument("--batch", type=int, default=0, help="causal leg batch (profiling)")
+    ap.add_argument("--dec-batch", type=int, default=0, help="decode sequences (profiling)")
+    ap.add_argument("--dec-steps", type=int, default=0, help="decode steps (profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -415,23 +424,32 @@ def main():
     hbm, tcp, peak_src = peaks()
     stream = torch.cuda.Stream()
 
+    if args.only in ("decode", "global"):
+        leg = decode_leg if args.only == "decode" else global_leg
+        line = {"metric": METRIC, "leg": args.only, "n_gpus": world,
+                args.only: leg(lib, args, world, rank, stream, hbm)}
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+        return 0
     res = causal_leg(lib, args, world, rank, stream, hbm, tcp)
+    B = args.batch or WL.B
     line = {
         "metric": METRIC, "value": res["value"], "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": res["ms_per_step"],
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded torch RNG on the device, N(0,1)/sqrt(d))",
-        "config": {"workload": "causal_decay_d128: B=4 x H=16 x N=16384, d_k=d_v=128, bf16 "
+        "config": {"workload": f"causal_decay_d128: B={B} x H=16 x N=16384, d_k=d_v=128, bf16 "
                                "q/k/v, lambda_h=linspace(0.9,0.999,16), fp32 S/z, eps=1e-6",
-                   "global_batch": WL.B * world, "seq_len": WL.N, "heads": WL.H, "d": WL.d,
+                   "global_batch": B * world, "seq_len": WL.N, "heads": WL.H, "d": WL.d,
                    "parallelism": f"dp{world} (batch sharded, no data-path collective)",
-                   "l2": "inputs larger than L2 (805 MB per step)"},
+                   "l2": f"inputs larger than L2 ({3 * B * WL.H * WL.N * WL.d * 2 / 1e6:.0f} MB "
+                         "per step)"},
         "roofline": res["roofline"], "clocks": res["clocks"],
         "gpu_launches": res["gpu_launches"], "peaks": peak_src,
     }
     if "e2e" in res:
         line["e2e"] = res["e2e"]
-    if args.legs:
+    if args.legs and args.only == "all":
         line["decode"] = decode_leg(lib, args, world, rank, stream, hbm)
         line["global"] = global_leg(lib, args, world, rank, stream, hbm)
     if args.cpu and world == 1 and rank == 0:

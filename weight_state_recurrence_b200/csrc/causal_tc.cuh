@@ -7,32 +7,39 @@
 // C = 128 tokens, t and s 0-based inside the chunk, Cv valid tokens, state
 // (S, z) carried from the previous chunk:
 //
-//   A        = (phi(Q) phi(K)^T) o M,   M[t][s] = lambda^(t-s) for s <= t, else 0
-//   O        = A V  +  (Lq phi(Q)) S,                  Lq = diag(lambda^(t+1))
-//   den      = rowsum(A) + (Lq phi(Q)) z + eps,        y = O / den
-//   S       <- lambda^Cv S + (Lk phi(K))^T V,          Lk = diag(lambda^(Cv-1-t))
-//   z       <- lambda^Cv z + (Lk phi(K))^T 1
+//   A      = (phi(Q) phi(K)^T) o M,       M[t][s] = lambda^(t-s) for s <= t, else 0
+//   O_in   = A V,                         rs = A 1
+//   O_x    = phi(Q) S,                    qz = phi(Q) z
+//   y_t    = (O_in[t] + lambda^(t+1) O_x[t]) / (rs[t] + lambda^(t+1) qz[t] + eps)
+//   S     <- lambda^Cv S + phi(K)^T (Lk V),   Lk = diag(lambda^(Cv-1-t))
+//   z     <- lambda^Cv z + phi(K)^T (Lk 1)
 //
-// Every product above is one tcgen05.mma chain issued by a single thread:
-//   A    : M=128 (t) x N=128 (s) x K=128 (d_k)   phi(Q) K-major, phi(K) K-major
-//   O    : M=128 x N=64 x K=128 (s)              A (bf16, K-major) x V (MN-major)
-//        + M=128 x N=64 x K=128 (d_k)            Lq phi(Q) (K-major) x S (bf16, MN-major)
-//   qz   : M=128 x N=16 x K=128 (d_k)            Lq phi(Q) x [z_hi; z_lo; 0...] (K-major)
-//   dS   : M=128 (d_k) x N=64 x K=128 (t)        (Lk phi(K))^T (MN-major) x V (MN-major)
-//   dz   : M=128 (d_k) x N=16 x K=128 (t)        (Lk phi(K))^T x [1; 0...] (K-major)
-// The fp32 state slice S (128 x 64) and z stay in registers of one
-// warpgroup for the whole sequence; after each chunk they are re-emitted as
-// bf16 operand tiles (z as a hi/lo bf16 pair so the denominator keeps ~16
-// bits).  The denominator sums exactly the bf16-rounded weights that the
-// numerator uses (row sums of the rounded A tile), so the output stays a
-// normalised average.
+// Every product is a tcgen05.mma chain issued by one thread (M = 128):
+//   A     N=128 K=128(d_k)  phi(Q) K-major x phi(K) K-major   -> TMEM (2 buffers)
+//   O_in  N=64  K=128(s)    A bf16 K-major x V MN-major
+//   rs    N=16  K=128(s)    A bf16 x W (row 0 = ones)
+//   O_x   N=64  K=128(d_k)  phi(Q) x S bf16 MN-major
+//   qz    N=16  K=128(d_k)  phi(Q) x Z (rows: z_hi, z_lo)
+//   S     N=64  K=128(t)    phi(K)^T MN-major x Lk V MN-major, accumulated onto
+//                           the fp32 state that stays in TMEM
+//   dz    N=16  K=128(t)    phi(K)^T x W (rows 1, 2: hi / lo of lambda^(Cv-1-t))
+// The fp32 state S never leaves the tensor memory between chunks: after each
+// chunk one warpgroup reads it, emits it as the bf16 operand of the next
+// chunk's O_x, and writes it back multiplied by lambda^Cv so that the next
+// S MMA accumulates onto the decayed state.  The denominator sums exactly
+// the bf16-rounded weights the numerator uses (rs comes from the same bf16 A
+// tile), so y stays a normalised average of values.
 //
-// Decay powers lambda^i are formed directly per exponent (never as ratios),
-// so lambda in [0, 1] including 0 is exact in form.
-//
-// Data movement: q, k, v tiles arrive by TMA (128B swizzle, out-of-range
-// rows of a ragged last chunk read as zeros) into a two-stage ring; y leaves
-// by TMA store from a swizzled staging tile (rows past N are clipped).
+// Warp roles (512 threads):
+//   warp 0      TMA producer: q, k, v tiles of a chunk into a 2-stage ring
+//   warp 1      TMEM owner and the single MMA-issuing thread
+//   warps 2-7   phi applied in place to q and k tiles (packed bf16x2), and
+//               the in-place decay weighting of V for the state update
+//   warps 8-11  masked, decayed score tile: TMEM -> registers -> bf16 SMEM
+//   warps 12-15 output (y = numerator / denominator, stored to HBM) and the
+//               state update
+// Every barrier wait is bounded (see sm100.cuh); a wait that runs out
+// records an error flag and every role leaves its loop.
 #pragma once
 #include "common.cuh"
 #include "sm100.cuh"
@@ -43,32 +50,54 @@ namespace tc {
 constexpr int C = 128;      // tokens per chunk
 constexpr int DK = 128;     // key dimension handled by this kernel
 constexpr int DVS = 64;     // dv columns per CTA
-constexpr int NT = 256;     // threads: warpgroup 0 = output side, warpgroup 1 = state side
+constexpr int NT = 512;
 
-constexpr uint32_t kPanel = C * 128;          // 128 rows x 128 bytes
-constexpr uint32_t kOffQ = 0;                 // per stage: phi(Q), 2 panels (d_k 0-63, 64-127)
-constexpr uint32_t kOffK = 2 * kPanel;        //            phi(K), 2 panels
-constexpr uint32_t kOffV = 4 * kPanel;        //            V slice, 1 panel
-constexpr uint32_t kStage = 5 * kPanel;
-constexpr uint32_t kOffA = 2 * kStage;        // masked scores, 2 panels; later the y staging tile
-constexpr uint32_t kOffS = kOffA + 2 * kPanel;  // S slice operand (bf16), 1 panel
-constexpr uint32_t kOffZ = kOffS + kPanel;      // [z_hi; z_lo; 0..] 16 x 128, 2 panels of 2 KB
-constexpr uint32_t kOffW = kOffZ + 4096;        // [1; 0..] 16 x 128, 2 panels of 2 KB
-constexpr uint32_t kOffMisc = kOffW + 4096;     // barriers, TMEM slot, flags, decay table
-constexpr uint32_t kMiscBytes = 2048;
+constexpr int kXformThreads = 192;  // warps 2-7
+constexpr int kBarXform = 1, kBarEpiA = 2, kBarOut = 3;  // named barrier ids
+
+// ---- shared memory (offsets from a 1024-byte aligned base)
+constexpr uint32_t kPanel = C * 128;            // 128 rows x 128 bytes
+constexpr uint32_t kOffQ = 0;                   // per stage: phi(Q), 2 panels (d_k 0-63, 64-127)
+constexpr uint32_t kOffK = 2 * kPanel;          //            phi(K), 2 panels
+constexpr uint32_t kOffV = 4 * kPanel;          //            V slice, 1 panel
+constexpr uint32_t kStage = 5 * kPanel;         // 80 KB
+constexpr uint32_t kOffA = 2 * kStage;          // bf16 score tile, 2 panels (keys 0-63, 64-127)
+constexpr uint32_t kOffS = kOffA + 2 * kPanel;  // bf16 S slice operand, 1 panel
+constexpr uint32_t kOffZ = kOffS + kPanel;      // [z_hi; z_lo; 0 ...] 16 x 128, 2 panels of 2 KB
+constexpr uint32_t kOffW = kOffZ + 4096;        // [1; w_hi; w_lo; 0 ...] for full chunks
+constexpr uint32_t kOffWt = kOffW + 4096;       // same for the last (ragged) chunk
+constexpr uint32_t kOffMisc = kOffWt + 4096;
+constexpr uint32_t kMiscBytes = 2560;
 constexpr uint32_t kSmemBytes = kOffMisc + kMiscBytes + 1024;  // + alignment slack
 constexpr uint32_t kStageTxBytes = 5 * kPanel;
 
-// TMEM columns (fp32, lane = row)
-constexpr uint32_t kTmA = 0, kTmO = 128, kTmDS = 192, kTmQZ = 256, kTmDZ = 272;
+// ---- barriers (8 bytes each, at kOffMisc)
+enum Bar {
+  kFull0 = 0, kFull1, kPhi0, kPhi1, kFree0, kFree1, kAFull0, kAFull1, kAFree0, kAFree1,
+  kAbfFull, kOvDone, kOxDone, kVsDone, kDsDone, kStateDone, kOutDone, kFinal, kNumBars
+};
+constexpr uint32_t kMiscTmem = 160, kMiscAbort = 164, kMiscConsumed = 168;
+constexpr uint32_t kMiscPw = 192;                    // lambda^i, i = 0..C      (132 floats)
+constexpr uint32_t kMiscQs = kMiscPw + 132 * 4;      // lambda^(t+1)           (128 floats)
+constexpr uint32_t kMiscVf = kMiscQs + 128 * 4;      // lambda^(C-1-t)         (128 floats)
+constexpr uint32_t kMiscVt = kMiscVf + 128 * 4;      // lambda^(Ct-1-t), 0 past Ct
+static_assert(kMiscVt + 128 * 4 <= kMiscBytes, "misc region overflow");
+
+// ---- tensor memory columns (fp32, lane = row)
+constexpr uint32_t kTmA = 0;      // two 128-column score buffers
+constexpr uint32_t kTmOI = 256;   // O_in  (64)
+constexpr uint32_t kTmOX = 320;   // O_x   (64)
+constexpr uint32_t kTmS = 384;    // state (64), lane = d_k row
+constexpr uint32_t kTmRS = 448;   // rs    (16)
+constexpr uint32_t kTmQZ = 464;   // qz    (16)
+constexpr uint32_t kTmDZ = 480;   // dz    (16), lane = d_k row
 constexpr uint32_t kTmCols = 512;
 
 constexpr uint32_t kIdA = idesc_bf16(128, 128, 0, 0);
-constexpr uint32_t kIdOV = idesc_bf16(128, 64, 0, 1);
-constexpr uint32_t kIdOS = idesc_bf16(128, 64, 0, 1);
-constexpr uint32_t kIdQZ = idesc_bf16(128, 16, 0, 0);
-constexpr uint32_t kIdDS = idesc_bf16(128, 64, 1, 1);
-constexpr uint32_t kIdDZ = idesc_bf16(128, 16, 1, 0);
+constexpr uint32_t kIdN64 = idesc_bf16(128, 64, 0, 1);    // K-major A, MN-major B
+constexpr uint32_t kIdN16 = idesc_bf16(128, 16, 0, 0);    // K-major A, K-major B
+constexpr uint32_t kIdS = idesc_bf16(128, 64, 1, 1);      // MN-major A, MN-major B
+constexpr uint32_t kIdDZ = idesc_bf16(128, 16, 1, 0);     // MN-major A, K-major B
 
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
@@ -78,319 +107,442 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<uint32_t *>(&p);
 }
 
-__device__ __forceinline__ float phi_fast(float x) { return x > 0.f ? x + 1.f : __expf(x); }
-
-// phi applied in place to a bf16 tile (layout-agnostic: elementwise).
-__device__ __forceinline__ void phi_tile_inplace(uint8_t *p, uint32_t bytes, int tid, int nthr) {
-  for (uint32_t o = static_cast<uint32_t>(tid) * 16u; o < bytes; o += static_cast<uint32_t>(nthr) * 16u) {
-    uint4 w = *reinterpret_cast<uint4 *>(p + o);
-    uint32_t *u = reinterpret_cast<uint32_t *>(&w);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) u[i] = pack_bf16(phi_fast(bf16lo(u[i])), phi_fast(bf16hi(u[i])));
-    *reinterpret_cast<uint4 *>(p + o) = w;
-  }
+// phi on a packed pair: max(x,0) + 2^(min(x,0) log2 e), in bf16x2 arithmetic.
+// log2 e is split into a bf16 head and tail so its rounding does not bias the
+// exponent; ex2 takes the bf16 argument (the result is bf16 either way).
+__device__ __forceinline__ uint32_t phi_bf16x2(uint32_t x) {
+  const uint32_t zero = 0u;
+  const uint32_t l2e_hi = 0x3FB93FB9u;   // bf16(log2 e) = 1.4453125, twice
+  const uint32_t l2e_lo = 0xBB2CBB2Cu;   // bf16(log2 e - 1.4453125) = -0.00262451, twice
+  uint32_t m, r, t, e, y;
+  asm("min.bf16x2 %0, %1, %2;" : "=r"(m) : "r"(x), "r"(zero));
+  asm("max.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(x), "r"(zero));
+  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(t) : "r"(m), "r"(l2e_hi));
+  asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(t) : "r"(m), "r"(l2e_lo), "r"(t));
+  asm("ex2.approx.ftz.bf16x2 %0, %1;" : "=r"(e) : "r"(t));
+  asm("add.rn.bf16x2 %0, %1, %2;" : "=r"(y) : "r"(r), "r"(e));
+  return y;
 }
 
-// Multiply every row r of a 2-panel swizzled tile (128 rows x 128 bf16) by
-// scale[r] (rows keep their place under the swizzle: row = offset / 128).
-__device__ __forceinline__ void scale_rows_inplace(uint8_t *p, const float *scale, int tid,
-                                                   int nthr) {
-  for (uint32_t o = static_cast<uint32_t>(tid) * 16u; o < 2 * kPanel;
-       o += static_cast<uint32_t>(nthr) * 16u) {
-    const float f = scale[(o % kPanel) >> 7];
-    uint4 w = *reinterpret_cast<uint4 *>(p + o);
-    uint32_t *u = reinterpret_cast<uint32_t *>(&w);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) u[i] = pack_bf16(bf16lo(u[i]) * f, bf16hi(u[i]) * f);
-    *reinterpret_cast<uint4 *>(p + o) = w;
-  }
+__device__ __forceinline__ uint32_t mul_bf16x2(uint32_t x, uint32_t s2) {
+  uint32_t y;
+  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(y) : "r"(x), "r"(s2));
+  return y;
+}
+
+// K-major operand tile [n rows x 128] with 128B swizzle, 2 panels of 64
+// columns, panel stride `panel_bytes`: byte offset of element (row, col).
+__device__ __forceinline__ uint32_t kmajor_off(uint32_t row, uint32_t col, uint32_t panel_bytes) {
+  return (col >> 6) * panel_bytes + sw128_offset(row, (col & 63) * 2);
 }
 
 __global__ void __launch_bounds__(NT, 1)
     causal_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                      const __grid_constant__ CUtensorMap tm_k,
-                     const __grid_constant__ CUtensorMap tm_v,
-                     const __grid_constant__ CUtensorMap tm_y, const float *__restrict__ lam,
-                     float eps, float *__restrict__ S_final, float *__restrict__ z_final, int H,
-                     int N, int DV) {
+                     const __grid_constant__ CUtensorMap tm_v, const float *__restrict__ lam,
+                     float eps, __nv_bfloat16 *__restrict__ out, float *__restrict__ S_final,
+                     float *__restrict__ z_final, int H, int N, int DV) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                             ~static_cast<uintptr_t>(1023));
   const uint32_t sb = smem_u32(sm);
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
+  const int lane = tid & 31;
   const int nslices = DV / DVS;
   const int pair = blockIdx.x / nslices;
   const int j0 = (blockIdx.x % nslices) * DVS;
   const int h = pair % H;
   const float L = lam ? lam[h] : 1.f;
+  const int nchunks = (N + C - 1) / C;
+  const int Ct = N - (nchunks - 1) * C;  // valid tokens of the last chunk
 
   uint8_t *misc = sm + kOffMisc;
-  const uint32_t bar_full0 = sb + kOffMisc + 0;   // stage 0 / 1 "data landed"
-  const uint32_t bar_mma = sb + kOffMisc + 16;    // "issued MMAs complete"
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(misc + 32);
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(misc + 36);
-  float *pw = reinterpret_cast<float *>(misc + 64);     // lambda^i, i = 0..C
-  float *qscale = pw + (C + 4);                         // lambda^(t+1)
-  float *kscale = qscale + C;                           // lambda^(Cv-1-t), 0 past Cv
+  auto bar = [&](int i) { return sb + kOffMisc + 8u * static_cast<uint32_t>(i); };
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(misc + kMiscTmem);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(misc + kMiscAbort);
+  volatile int *consumed = reinterpret_cast<volatile int *>(misc + kMiscConsumed);
+  float *pw = reinterpret_cast<float *>(misc + kMiscPw);
+  float *qs = reinterpret_cast<float *>(misc + kMiscQs);
+  float *vf = reinterpret_cast<float *>(misc + kMiscVf);
+  float *vt = reinterpret_cast<float *>(misc + kMiscVt);
 
+  // ------------------------------------------------------------ set-up
   if (tid == 0) {
-    mbar_init(bar_full0, 1);
-    mbar_init(bar_full0 + 8, 1);
-    mbar_init(bar_mma, 1);
+    for (int i = 0; i < kNumBars; ++i) mbar_init(bar(i), 1);
     *abort_flag = 0;
+    *consumed = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
-    tma_prefetch_desc(&tm_y);
   }
-  if (warp == 0) {
+  if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), kTmCols);
     tmem_relinquish();
   }
   if (tid <= C) pw[tid] = pow_int(L, tid);
-  // operand tiles that start as constants: S = 0, Z = 0, W = [1; 0...]
+  __syncthreads();
+  if (tid < C) {
+    qs[tid] = pw[tid + 1];
+    vf[tid] = pw[C - 1 - tid];
+    vt[tid] = tid < Ct ? pw[Ct - 1 - tid] : 0.f;
+  }
+  __syncthreads();
+  // constant operand tiles: S = 0, Z = 0, W / Wt = [1; w_hi; w_lo; 0 ...],
+  // and the score tile's blocks above the diagonal (always zero)
   for (uint32_t o = tid * 16u; o < kPanel; o += NT * 16u)
     *reinterpret_cast<uint4 *>(sm + kOffS + o) = make_uint4(0, 0, 0, 0);
-  for (uint32_t o = tid * 16u; o < 4096u; o += NT * 16u) {
+  for (uint32_t o = tid * 16u; o < 3 * 4096u; o += NT * 16u)
     *reinterpret_cast<uint4 *>(sm + kOffZ + o) = make_uint4(0, 0, 0, 0);
-    const bool row0 = ((o % 2048u) >> 7) == 0;     // row 0 of either panel
-    const uint32_t one2 = 0x3F803F80u;              // two bf16 ones
-    *reinterpret_cast<uint4 *>(sm + kOffW + o) =
-        row0 ? make_uint4(one2, one2, one2, one2) : make_uint4(0, 0, 0, 0);
+  for (uint32_t o = tid * 16u; o < 2 * kPanel; o += NT * 16u)
+    *reinterpret_cast<uint4 *>(sm + kOffA + o) = make_uint4(0, 0, 0, 0);
+  __syncthreads();
+  if (tid < C) {
+    const int t = tid;
+    const __nv_bfloat16 one = __float2bfloat16_rn(1.f);
+    const float wf = vf[t], wt = vt[t];
+    const __nv_bfloat16 fh = __float2bfloat16_rn(wf), th = __float2bfloat16_rn(wt);
+    const __nv_bfloat16 fl = __float2bfloat16_rn(wf - __bfloat162float(fh));
+    const __nv_bfloat16 tl = __float2bfloat16_rn(wt - __bfloat162float(th));
+    __nv_bfloat16 *W = reinterpret_cast<__nv_bfloat16 *>(sm + kOffW);
+    __nv_bfloat16 *Wt = reinterpret_cast<__nv_bfloat16 *>(sm + kOffWt);
+    W[kmajor_off(0, t, 2048) / 2] = one;
+    W[kmajor_off(1, t, 2048) / 2] = fh;
+    W[kmajor_off(2, t, 2048) / 2] = fl;
+    Wt[kmajor_off(0, t, 2048) / 2] = one;
+    Wt[kmajor_off(1, t, 2048) / 2] = th;
+    Wt[kmajor_off(2, t, 2048) / 2] = tl;
   }
   fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (tid <= C && tid >= 1) qscale[tid - 1] = pw[tid];
   const uint32_t tmem = *tmem_slot;
 
-  const int nchunks = (N + C - 1) / C;
-  auto issue_loads = [&](int c, int st) {
-    const uint32_t base = sb + st * kStage;
-    const uint32_t bar = bar_full0 + 8 * st;
-    mbar_arrive_expect_tx(bar, kStageTxBytes);
-    tma_load_3d(base + kOffQ, &tm_q, bar, 0, c * C, pair);
-    tma_load_3d(base + kOffQ + kPanel, &tm_q, bar, 64, c * C, pair);
-    tma_load_3d(base + kOffK, &tm_k, bar, 0, c * C, pair);
-    tma_load_3d(base + kOffK + kPanel, &tm_k, bar, 64, c * C, pair);
-    tma_load_3d(base + kOffV, &tm_v, bar, j0, c * C, pair);
-  };
-  if (tid == 0) {
-    for (int c = 0; c < nchunks && c < 2; ++c) issue_loads(c, c);
-  }
+  auto fail = [&]() { *abort_flag = 1; };
 
-  // warpgroup-local indices: row owned by this thread and its TMEM lane field
-  const int row = tid & 127;
-  const uint32_t lane_field = static_cast<uint32_t>((warp & 3) * 32) << 16;
-  float S_reg[DVS];
-#pragma unroll
-  for (int j = 0; j < DVS; ++j) S_reg[j] = 0.f;
-  float z_reg = 0.f;
-  float rowsum = 0.f;
-  uint32_t mma_phase = 0;
-  bool mma_in_flight = false;
-  int next_consume = 0;                        // chunks [next_consume, next_issue) in flight
-  int next_issue = nchunks < 2 ? nchunks : 2;
-
-  for (int c = 0; c < nchunks; ++c) {
-    const int st = c & 1;
-    const uint32_t stage = sb + st * kStage;
-    uint8_t *stage_p = sm + st * kStage;
-    const int Cv = min(C, N - c * C);
-
-    // ---- P1: inputs landed; apply phi in place to q and k
-    if (!mbar_wait(bar_full0 + 8 * st, (c >> 1) & 1)) *abort_flag = 1;
-    else next_consume = c + 1;
-    if (tid < C) kscale[tid] = tid < Cv ? pw[Cv - 1 - tid] : 0.f;
-    phi_tile_inplace(stage_p + kOffQ, 4 * kPanel, tid, NT);   // phi(Q) and phi(K) (adjacent)
-    fence_proxy_async_smem();
-    __syncthreads();
-    if (*abort_flag) break;
-
-    // ---- P2: A = phi(Q) phi(K)^T
-    if (tid == 0) {
-      tc_fence_after();
-#pragma unroll
-      for (int ks = 0; ks < DK / 16; ++ks) {
-        const uint32_t off = (ks >> 2) * kPanel + (ks & 3) * 32;
-        umma_bf16(tmem + kTmA, sdesc_sw128(stage + kOffQ + off, 16, 1024),
-                  sdesc_sw128(stage + kOffK + off, 16, 1024), kIdA, ks > 0);
+  if (warp == 0) {
+    // ------------------------------------------------------- TMA producer
+    int issued = 0;
+    if (lane == 0) {
+      for (int c = 0; c < nchunks && !*abort_flag; ++c) {
+        const int s = c & 1;
+        if (c >= 2 && !mbar_wait(bar(kFree0 + s), ((c - 2) >> 1) & 1)) {
+          fail();
+          break;
+        }
+        const uint32_t base = sb + s * kStage;
+        const uint32_t b = bar(kFull0 + s);
+        mbar_arrive_expect_tx(b, kStageTxBytes);
+        tma_load_3d(base + kOffQ, &tm_q, b, 0, c * C, pair);
+        tma_load_3d(base + kOffQ + kPanel, &tm_q, b, 64, c * C, pair);
+        tma_load_3d(base + kOffK, &tm_k, b, 0, c * C, pair);
+        tma_load_3d(base + kOffK + kPanel, &tm_k, b, 64, c * C, pair);
+        tma_load_3d(base + kOffV, &tm_v, b, j0, c * C, pair);
+        issued = c + 1;
       }
-      umma_commit(bar_mma);
+      if (*abort_flag) {
+        // let every copy this thread started land before the CTA exits
+        for (int c = *consumed; c < issued; ++c) mbar_wait(bar(kFull0 + (c & 1)), (c >> 1) & 1);
+      }
     }
-    if (!mbar_wait(bar_mma, mma_phase)) {
-      *abort_flag = 1;
-      mma_in_flight = true;
+    __syncwarp();
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      auto mma_scores = [&](int c) -> bool {
+        const int s = c & 1;
+        if (!mbar_wait(bar(kPhi0 + s), (c >> 1) & 1)) return false;
+        if (c >= 2 && !mbar_wait(bar(kAFree0 + s), ((c - 2) >> 1) & 1)) return false;
+        tc_fence_after();
+        const uint32_t st = sb + s * kStage;
+#pragma unroll
+        for (int ks = 0; ks < DK / 16; ++ks) {
+          const uint32_t off = (ks >> 2) * kPanel + (ks & 3) * 32;
+          umma_bf16(tmem + kTmA + s * 128, sdesc_sw128(st + kOffQ + off, 16, 1024),
+                    sdesc_sw128(st + kOffK + off, 16, 1024), kIdA, ks > 0);
+        }
+        umma_commit(bar(kAFull0 + s));
+        return true;
+      };
+      bool ok = nchunks > 0 && mma_scores(0);
+      for (int c = 0; ok && c < nchunks; ++c) {
+        const int s = c & 1;
+        const uint32_t st = sb + s * kStage;
+        const uint32_t w = sb + (c == nchunks - 1 ? kOffWt : kOffW);
+        if (*abort_flag) break;
+        if (c + 1 < nchunks && !(ok = mma_scores(c + 1))) break;
+        // O_x = phi(Q) S, qz = phi(Q) z   (state of the previous chunk)
+        if (c >= 1 && (!mbar_wait(bar(kStateDone), (c - 1) & 1) ||
+                       !mbar_wait(bar(kOutDone), (c - 1) & 1))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < DK / 16; ++ks) {
+          const uint32_t off = (ks >> 2) * kPanel + (ks & 3) * 32;
+          const uint64_t a = sdesc_sw128(st + kOffQ + off, 16, 1024);
+          umma_bf16(tmem + kTmOX, a, sdesc_sw128(sb + kOffS + ks * 2048, kPanel, 1024), kIdN64,
+                    ks > 0);
+          umma_bf16(tmem + kTmQZ, a,
+                    sdesc_sw128(sb + kOffZ + (ks >> 2) * 2048 + (ks & 3) * 32, 16, 1024), kIdN16,
+                    ks > 0);
+        }
+        umma_commit(bar(kOxDone));
+        // O_in = A V, rs = A 1
+        if (!mbar_wait(bar(kAbfFull), c & 1)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < C / 16; ++ks) {
+          const uint64_t a = sdesc_sw128(sb + kOffA + (ks >> 2) * kPanel + (ks & 3) * 32, 16, 1024);
+          umma_bf16(tmem + kTmOI, a, sdesc_sw128(st + kOffV + ks * 2048, kPanel, 1024), kIdN64,
+                    ks > 0);
+          umma_bf16(tmem + kTmRS, a, sdesc_sw128(w + (ks >> 2) * 2048 + (ks & 3) * 32, 16, 1024),
+                    kIdN16, ks > 0);
+        }
+        umma_commit(bar(kOvDone));
+        // S += phi(K)^T (Lk V), dz = phi(K)^T (Lk 1)
+        if (!mbar_wait(bar(kVsDone), c & 1)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < C / 16; ++ks) {
+          const uint64_t a = sdesc_sw128(st + kOffK + ks * 2048, kPanel, 1024);
+          umma_bf16(tmem + kTmS, a, sdesc_sw128(st + kOffV + ks * 2048, kPanel, 1024), kIdS,
+                    (c > 0 || ks > 0) ? 1u : 0u);
+          umma_bf16(tmem + kTmDZ, a, sdesc_sw128(w + (ks >> 2) * 2048 + (ks & 3) * 32, 16, 1024),
+                    kIdDZ, ks > 0);
+        }
+        umma_commit(bar(kDsDone));
+        umma_commit(bar(kFree0 + s));
+      }
+      if (!ok) fail();
+      // make sure nothing this thread issued is still running
+      umma_commit(bar(kFinal));
+      mbar_wait(bar(kFinal), 0);
     }
-    mma_phase ^= 1;
-    tc_fence_after();
-
-    // ---- P3: warpgroup 0 masks/decays A into bf16; warpgroup 1 rescales Q and K rows
-    if (warp < 4) {
-      const int t = row;
-      rowsum = 0.f;
-#pragma unroll 1
-      for (int blk = 0; blk < C / 32; ++blk) {
+    __syncwarp();
+  } else if (warp < 8) {
+    // ------------------------------------------- phi transform, V weighting
+    const int tt = tid - 64;
+    auto transform = [&](int c) -> bool {
+      const int s = c & 1;
+      if (!mbar_wait(bar(kFull0 + s), (c >> 1) & 1)) return false;
+      if (tt == 0) *consumed = c + 1;
+      uint8_t *p = sm + s * kStage + kOffQ;  // q and k tiles are adjacent (64 KB)
+      for (uint32_t o = tt * 16u; o < 4 * kPanel; o += kXformThreads * 16u) {
+        uint4 w = *reinterpret_cast<uint4 *>(p + o);
+        w.x = phi_bf16x2(w.x);
+        w.y = phi_bf16x2(w.y);
+        w.z = phi_bf16x2(w.z);
+        w.w = phi_bf16x2(w.w);
+        *reinterpret_cast<uint4 *>(p + o) = w;
+      }
+      fence_proxy_async_smem();
+      named_bar_sync(kBarXform, kXformThreads);
+      if (tt == 0) mbar_arrive(bar(kPhi0 + s));
+      return true;
+    };
+    auto weight_v = [&](int c) -> bool {
+      const int s = c & 1;
+      if (!mbar_wait(bar(kOvDone), c & 1)) return false;
+      const float *wv = c == nchunks - 1 ? vt : vf;
+      uint8_t *p = sm + s * kStage + kOffV;
+      for (uint32_t o = tt * 16u; o < kPanel; o += kXformThreads * 16u) {
+        const float f = wv[o >> 7];
+        const uint32_t f2 = pack_bf16(f, f);
+        uint4 w = *reinterpret_cast<uint4 *>(p + o);
+        w.x = mul_bf16x2(w.x, f2);
+        w.y = mul_bf16x2(w.y, f2);
+        w.z = mul_bf16x2(w.z, f2);
+        w.w = mul_bf16x2(w.w, f2);
+        *reinterpret_cast<uint4 *>(p + o) = w;
+      }
+      fence_proxy_async_smem();
+      named_bar_sync(kBarXform, kXformThreads);
+      if (tt == 0) mbar_arrive(bar(kVsDone));
+      return true;
+    };
+    bool ok = nchunks > 0 && transform(0);
+    for (int c = 0; ok && c < nchunks; ++c) {
+      if (*abort_flag) break;
+      if (c + 1 < nchunks && !(ok = transform(c + 1))) break;
+      ok = weight_v(c);
+    }
+    if (!ok) fail();
+  } else if (warp < 12) {
+    // ------------------------------------------------ masked score tile
+    const int wq = warp - 8;          // TMEM lane quarter and row block
+    const int t = wq * 32 + lane;     // query row inside the chunk
+    const uint32_t lane_field = static_cast<uint32_t>(wq * 32) << 16;
+    bool ok = true;
+    for (int c = 0; c < nchunks; ++c) {
+      const int b = c & 1;
+      if (*abort_flag) break;
+      if (!mbar_wait(bar(kAFull0 + b), (c >> 1) & 1) ||
+          (c >= 1 && !mbar_wait(bar(kOvDone), (c - 1) & 1))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      // only blocks at or below the diagonal change; the others stay zero
+      for (int blk = 0; blk <= wq; ++blk) {
         uint32_t r[32];
-        tmem_ld_32x32b_x32(tmem + lane_field + kTmA + blk * 32, r);
+        tmem_ld_32x32b_x32(tmem + lane_field + kTmA + b * 128 + blk * 32, r);
         tmem_wait_ld();
+        float f[32];
+        if (blk < wq) {
+          // whole block left of the diagonal: lambda^(t-s) from the last column back
+          float g = pw[t - (blk * 32 + 31)];
+#pragma unroll
+          for (int j = 31; j >= 0; --j) {
+            f[j] = g;
+            g *= L;
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) f[j] = j <= lane ? pw[max(lane - j, 0)] : 0.f;
+        }
         uint32_t pk[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int s0 = blk * 32 + 2 * i;
-          const int e0 = t - s0, e1 = t - s0 - 1;
-          const float f0 = (e0 >= 0 && s0 < Cv) ? pw[max(e0, 0)] : 0.f;
-          const float f1 = (e1 >= 0 && s0 + 1 < Cv) ? pw[max(e1, 0)] : 0.f;
-          pk[i] = pack_bf16(__uint_as_float(r[2 * i]) * f0, __uint_as_float(r[2 * i + 1]) * f1);
-          rowsum += bf16lo(pk[i]) + bf16hi(pk[i]);
-        }
+        for (int i = 0; i < 16; ++i)
+          pk[i] = pack_bf16(__uint_as_float(r[2 * i]) * f[2 * i],
+                            __uint_as_float(r[2 * i + 1]) * f[2 * i + 1]);
         uint8_t *pa = sm + kOffA + (blk >> 1) * kPanel;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const uint32_t byte = (blk & 1) * 64 + i * 16;
-          *reinterpret_cast<uint4 *>(pa + sw128_offset(t, byte)) =
+        for (int i = 0; i < 4; ++i)
+          *reinterpret_cast<uint4 *>(pa + sw128_offset(t, (blk & 1) * 64 + i * 16)) =
               make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+      }
+      tc_fence_before();
+      fence_proxy_async_smem();
+      named_bar_sync(kBarEpiA, 128);
+      if (t == 0) {
+        mbar_arrive(bar(kAFree0 + b));
+        mbar_arrive(bar(kAbfFull));
+      }
+    }
+    if (!ok) fail();
+  } else {
+    // ---------------------------------------------- output and state update
+    const int wq = warp - 12;
+    const int r = wq * 32 + lane;     // query row (output) and d_k row (state)
+    const uint32_t lane_field = static_cast<uint32_t>(wq * 32) << 16;
+    float z_reg = 0.f;
+    bool ok = true;
+    for (int c = 0; c < nchunks; ++c) {
+      if (*abort_flag) break;
+      const int Cv = c == nchunks - 1 ? Ct : C;
+      // -- y for the chunk's rows
+      if (!mbar_wait(bar(kOxDone), c & 1) || !mbar_wait(bar(kOvDone), c & 1)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      {
+        uint32_t rs[2], qz[2];
+        tmem_ld_32x32b_x2(tmem + lane_field + kTmRS, rs);
+        tmem_ld_32x32b_x2(tmem + lane_field + kTmQZ, qz);
+        tmem_wait_ld();
+        const float g = qs[r];
+        const float inv =
+            1.f / (__uint_as_float(rs[0]) + g * (__uint_as_float(qz[0]) + __uint_as_float(qz[1])) +
+                   eps);
+        const long row = static_cast<long>(c) * C + r;
+        uint4 *dst = reinterpret_cast<uint4 *>(out + (static_cast<long>(pair) * N + row) * DV + j0);
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          uint32_t oi[32], ox[32];
+          tmem_ld_32x32b_x32(tmem + lane_field + kTmOI + half * 32, oi);
+          tmem_ld_32x32b_x32(tmem + lane_field + kTmOX + half * 32, ox);
+          tmem_wait_ld();
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            pk[i] = pack_bf16(fmaf(g, __uint_as_float(ox[2 * i]), __uint_as_float(oi[2 * i])) * inv,
+                              fmaf(g, __uint_as_float(ox[2 * i + 1]), __uint_as_float(oi[2 * i + 1])) *
+                                  inv);
+          if (r < Cv) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              dst[half * 4 + i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+          }
         }
       }
-    } else {
-      scale_rows_inplace(stage_p + kOffQ, qscale, tid - 128, 128);
-      scale_rows_inplace(stage_p + kOffK, kscale, tid - 128, 128);
-    }
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-
-    // ---- P4: O = A V + (Lq phi(Q)) S ; qz ; dS ; dz
-    if (tid == 0) {
+      tc_fence_before();
+      named_bar_sync(kBarOut, 128);
+      if (r == 0) mbar_arrive(bar(kOutDone));
+      // -- state after the chunk
+      if (!mbar_wait(bar(kDsDone), c & 1)) {
+        ok = false;
+        break;
+      }
       tc_fence_after();
+      const bool last = c == nchunks - 1;
+      {
+        uint32_t dz[2];
+        tmem_ld_32x32b_x2(tmem + lane_field + kTmDZ + 1, dz);
+        tmem_wait_ld();
+        z_reg = fmaf(pw[Cv], z_reg, __uint_as_float(dz[0]) + __uint_as_float(dz[1]));
+        const float gnext = last ? 1.f : pw[c + 1 == nchunks - 1 ? Ct : C];
 #pragma unroll
-      for (int ks = 0; ks < C / 16; ++ks) {
-        const uint32_t off = (ks >> 2) * kPanel + (ks & 3) * 32;
-        umma_bf16(tmem + kTmO, sdesc_sw128(sb + kOffA + off, 16, 1024),
-                  sdesc_sw128(stage + kOffV + ks * 2048, kPanel, 1024), kIdOV, ks > 0);
-      }
+        for (int half = 0; half < 2; ++half) {
+          uint32_t sv[32];
+          tmem_ld_32x32b_x32(tmem + lane_field + kTmS + half * 32, sv);
+          tmem_wait_ld();
+          if (last) {
+            if (S_final) {
+              float4 *dst = reinterpret_cast<float4 *>(
+                  S_final + (static_cast<long>(pair) * DK + r) * DV + j0 + half * 32);
 #pragma unroll
-      for (int ks = 0; ks < DK / 16; ++ks) {
-        const uint32_t off = (ks >> 2) * kPanel + (ks & 3) * 32;
-        umma_bf16(tmem + kTmO, sdesc_sw128(stage + kOffQ + off, 16, 1024),
-                  sdesc_sw128(sb + kOffS + ks * 2048, kPanel, 1024), kIdOS, 1);
-      }
+              for (int i = 0; i < 8; ++i)
+                dst[i] = make_float4(__uint_as_float(sv[4 * i]), __uint_as_float(sv[4 * i + 1]),
+                                     __uint_as_float(sv[4 * i + 2]), __uint_as_float(sv[4 * i + 3]));
+            }
+          } else {
+            uint32_t pk[16];
 #pragma unroll
-      for (int ks = 0; ks < DK / 16; ++ks) {
-        const uint32_t off = (ks >> 2) * kPanel + (ks & 3) * 32;
-        const uint32_t offz = (ks >> 2) * 2048 + (ks & 3) * 32;
-        umma_bf16(tmem + kTmQZ, sdesc_sw128(stage + kOffQ + off, 16, 1024),
-                  sdesc_sw128(sb + kOffZ + offz, 16, 1024), kIdQZ, ks > 0);
-      }
+            for (int i = 0; i < 16; ++i)
+              pk[i] = pack_bf16(__uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1]));
 #pragma unroll
-      for (int ks = 0; ks < C / 16; ++ks) {
-        const uint64_t a = sdesc_sw128(stage + kOffK + ks * 2048, kPanel, 1024);
-        umma_bf16(tmem + kTmDS, a, sdesc_sw128(stage + kOffV + ks * 2048, kPanel, 1024), kIdDS,
-                  ks > 0);
-        const uint32_t offw = (ks >> 2) * 2048 + (ks & 3) * 32;
-        umma_bf16(tmem + kTmDZ, a, sdesc_sw128(sb + kOffW + offw, 16, 1024), kIdDZ, ks > 0);
-      }
-      umma_commit(bar_mma);
-    }
-    if (!mbar_wait(bar_mma, mma_phase)) {
-      *abort_flag = 1;
-      mma_in_flight = true;
-    }
-    mma_phase ^= 1;
-    tc_fence_after();
-
-    // ---- P5: warpgroup 0 writes y; warpgroup 1 advances the state
-    if (warp < 4) {
-      const int t = row;
-      uint32_t o[64];
-      uint32_t qz[2];
-      tmem_ld_32x32b_x32(tmem + lane_field + kTmO, *reinterpret_cast<uint32_t(*)[32]>(&o[0]));
-      tmem_ld_32x32b_x32(tmem + lane_field + kTmO + 32,
-                         *reinterpret_cast<uint32_t(*)[32]>(&o[32]));
-      tmem_ld_32x32b_x2(tmem + lane_field + kTmQZ, qz);
-      tmem_wait_ld();
-      const float inv = 1.f / (rowsum + (__uint_as_float(qz[0]) + __uint_as_float(qz[1])) + eps);
+            for (int i = 0; i < 4; ++i)
+              *reinterpret_cast<uint4 *>(sm + kOffS + sw128_offset(r, half * 64 + i * 16)) =
+                  make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        uint4 w;
-        w.x = pack_bf16(__uint_as_float(o[8 * i + 0]) * inv, __uint_as_float(o[8 * i + 1]) * inv);
-        w.y = pack_bf16(__uint_as_float(o[8 * i + 2]) * inv, __uint_as_float(o[8 * i + 3]) * inv);
-        w.z = pack_bf16(__uint_as_float(o[8 * i + 4]) * inv, __uint_as_float(o[8 * i + 5]) * inv);
-        w.w = pack_bf16(__uint_as_float(o[8 * i + 6]) * inv, __uint_as_float(o[8 * i + 7]) * inv);
-        *reinterpret_cast<uint4 *>(sm + kOffA + sw128_offset(t, i * 16)) = w;
+            for (int i = 0; i < 32; ++i) sv[i] = __float_as_uint(__uint_as_float(sv[i]) * gnext);
+            tmem_st_32x32b_x32(tmem + lane_field + kTmS + half * 32, sv);
+          }
+        }
+        if (last) {
+          if (z_final && j0 == 0) z_final[static_cast<long>(pair) * DK + r] = z_reg;
+        } else {
+          tmem_wait_st();
+          const __nv_bfloat16 zh = __float2bfloat16_rn(z_reg);
+          const __nv_bfloat16 zl = __float2bfloat16_rn(z_reg - __bfloat162float(zh));
+          __nv_bfloat16 *Z = reinterpret_cast<__nv_bfloat16 *>(sm + kOffZ);
+          Z[kmajor_off(0, r, 2048) / 2] = zh;
+          Z[kmajor_off(1, r, 2048) / 2] = zl;
+        }
       }
       fence_proxy_async_smem();
-      named_bar_sync(1, 128);
-      if (tid == 0) {
-        tma_store_3d(&tm_y, sb + kOffA, j0, c * C, pair);
-        tma_store_commit();
-      }
-    } else {
-      const int kk = row;
-      uint32_t d[64];
-      uint32_t dz[2];
-      tmem_ld_32x32b_x32(tmem + lane_field + kTmDS, *reinterpret_cast<uint32_t(*)[32]>(&d[0]));
-      tmem_ld_32x32b_x32(tmem + lane_field + kTmDS + 32,
-                         *reinterpret_cast<uint32_t(*)[32]>(&d[32]));
-      tmem_ld_32x32b_x2(tmem + lane_field + kTmDZ, dz);
-      tmem_wait_ld();
-      const float g = pw[Cv];
-#pragma unroll
-      for (int j = 0; j < DVS; ++j) S_reg[j] = fmaf(g, S_reg[j], __uint_as_float(d[j]));
-      z_reg = fmaf(g, z_reg, __uint_as_float(dz[0]));
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        uint4 w;
-        w.x = pack_bf16(S_reg[8 * i + 0], S_reg[8 * i + 1]);
-        w.y = pack_bf16(S_reg[8 * i + 2], S_reg[8 * i + 3]);
-        w.z = pack_bf16(S_reg[8 * i + 4], S_reg[8 * i + 5]);
-        w.w = pack_bf16(S_reg[8 * i + 6], S_reg[8 * i + 7]);
-        *reinterpret_cast<uint4 *>(sm + kOffS + sw128_offset(kk, i * 16)) = w;
-      }
-      const __nv_bfloat16 zh = __float2bfloat16_rn(z_reg);
-      const __nv_bfloat16 zl = __float2bfloat16_rn(z_reg - __bfloat162float(zh));
-      const uint32_t zb = (kk >> 6) * 2048u;
-      const uint32_t zbyte = (kk & 63) * 2;
-      *reinterpret_cast<__nv_bfloat16 *>(sm + kOffZ + zb + sw128_offset(0, zbyte)) = zh;
-      *reinterpret_cast<__nv_bfloat16 *>(sm + kOffZ + zb + sw128_offset(1, zbyte)) = zl;
-      fence_proxy_async_smem();
+      tc_fence_before();
+      named_bar_sync(kBarOut, 128);
+      if (r == 0) mbar_arrive(bar(kStateDone));
     }
-    tc_fence_before();
-    __syncthreads();
-    if (tid == 0) {
-      if (c + 2 < nchunks) issue_loads(c + 2, st);
-      tma_store_wait_read();   // the staging tile is rewritten by the next chunk's scores
-    }
-    __syncthreads();
-    next_issue = min(nchunks, c + 3);
-    if (*abort_flag) break;
+    if (!ok) fail();
   }
 
-  if (*abort_flag) {
-    // drain what this CTA still has in flight before releasing its resources
-    // (each wait is bounded; a second time-out leaves the flag set)
-    if (tid == 0) {
-      for (int cc = next_consume; cc < next_issue; ++cc)
-        mbar_wait(bar_full0 + 8 * (cc & 1), (cc >> 1) & 1);
-      if (mma_in_flight) mbar_wait(bar_mma, mma_phase ^ 1);
-    }
-  } else if (warp >= 4) {
-    const int kk = row;
-    if (S_final) {
-      float4 *dst = reinterpret_cast<float4 *>(S_final + (static_cast<long>(pair) * DK + kk) * DV + j0);
-#pragma unroll
-      for (int j = 0; j < DVS / 4; ++j)
-        dst[j] = make_float4(S_reg[4 * j], S_reg[4 * j + 1], S_reg[4 * j + 2], S_reg[4 * j + 3]);
-    }
-    if (z_final && j0 == 0) z_final[static_cast<long>(pair) * DK + kk] = z_reg;
-  }
-  if (tid == 0) tma_store_wait_all();
+  // ------------------------------------------------------------ teardown
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) {
+  if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmCols);
   }

@@ -129,13 +129,27 @@ bool use_tc_causal(const linattn_dims *d) {
 }
 
 // ------------------------------------------------------------ launchers
+int num_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return n;
+}
+
 template <int DK, int DV, typename T>
 int launch_decode(const linattn_dims *d, const void *q, const void *k, const void *v,
                   const float *lam, float eps, float *S, float *z, void *out,
                   cudaStream_t s) {
-  decode_step_kernel<DK, DV, T><<<d->B * d->H, 256, 0, s>>>(
+  auto *kern = decode_step_kernel<DK, DV, T>;
+  const int bytes = static_cast<int>(DecodeLayout<DK, DV, T>::kSmem);
+  if (!set_smem(kern, bytes)) return LINATTN_ERR_CUDA;
+  const int BH = d->B * d->H;
+  const int sms = num_sms();
+  if (sms <= 0) return LINATTN_ERR_CUDA;
+  const int grid = BH < sms ? BH : sms;
+  kern<<<grid, kDecodeThreads, bytes, s>>>(
       static_cast<const T *>(q), static_cast<const T *>(k), static_cast<const T *>(v), lam, eps,
-      S, z, static_cast<T *>(out), d->H);
+      S, z, static_cast<T *>(out), d->H, BH);
   return launch_status();
 }
 
@@ -204,14 +218,14 @@ int launch_causal_tc(const linattn_dims *d, const void *q, const void *k, const 
                      const float *lam, float eps, void *out, float *S_final, float *z_final,
                      cudaStream_t s) {
   const int BH = d->B * d->H;
-  CUtensorMap mq, mk, mv, my;
+  CUtensorMap mq, mk, mv;
   if (!make_map_bf16(&mq, q, d->dk, d->N, BH) || !make_map_bf16(&mk, k, d->dk, d->N, BH) ||
-      !make_map_bf16(&mv, v, d->dv, d->N, BH) || !make_map_bf16(&my, out, d->dv, d->N, BH))
+      !make_map_bf16(&mv, v, d->dv, d->N, BH))
     return LINATTN_ERR_CUDA;
   if (!set_smem(tc::causal_tc_kernel, static_cast<int>(tc::kSmemBytes))) return LINATTN_ERR_CUDA;
   const int grid = BH * (d->dv / tc::DVS);
-  tc::causal_tc_kernel<<<grid, tc::NT, tc::kSmemBytes, s>>>(mq, mk, mv, my, lam, eps, S_final,
-                                                           z_final, d->H, d->N, d->dv);
+  tc::causal_tc_kernel<<<grid, tc::NT, tc::kSmemBytes, s>>>(
+      mq, mk, mv, lam, eps, static_cast<bf16 *>(out), S_final, z_final, d->H, d->N, d->dv);
   return launch_status();
 }
 
