@@ -102,16 +102,17 @@ EncodeTiled encode_fn() {
   return fn;
 }
 
-// [planes, rows, inner] bf16 tensor; boxes of 64 x 128 x 1 with 128-byte
+// [planes, rows, inner] bf16 tensor; boxes of 64 x box_rows x 1 with 128-byte
 // swizzle (64 bf16 = 128 bytes per box row).
-bool make_map_bf16(CUtensorMap *m, const void *ptr, int inner, int rows, int planes) {
+bool make_map_bf16(CUtensorMap *m, const void *ptr, int inner, int rows, int planes,
+                   unsigned box_rows = 128) {
   EncodeTiled enc = encode_fn();
   if (!enc) return false;
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(rows),
                               static_cast<cuuint64_t>(planes)};
   const cuuint64_t strides[2] = {static_cast<cuuint64_t>(inner) * 2,
                                  static_cast<cuuint64_t>(inner) * rows * 2};
-  const cuuint32_t box[3] = {64, 128, 1};
+  const cuuint32_t box[3] = {64, box_rows, 1};
   const cuuint32_t estr[3] = {1, 1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides, box,
              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -218,14 +219,31 @@ int launch_causal_tc(const linattn_dims *d, const void *q, const void *k, const 
                      const float *lam, float eps, void *out, float *S_final, float *z_final,
                      cudaStream_t s) {
   const int BH = d->B * d->H;
+  // dv = 128: the two column halves of a head run as a 2-CTA cluster that
+  // shares the feature map (each CTA loads 64 rows of every q/k tile)
+  const bool paired = d->dv == 2 * tc::DVS;
+  const unsigned qk_rows = paired ? 64u : 128u;
   CUtensorMap mq, mk, mv;
-  if (!make_map_bf16(&mq, q, d->dk, d->N, BH) || !make_map_bf16(&mk, k, d->dk, d->N, BH) ||
-      !make_map_bf16(&mv, v, d->dv, d->N, BH))
+  if (!make_map_bf16(&mq, q, d->dk, d->N, BH, qk_rows) ||
+      !make_map_bf16(&mk, k, d->dk, d->N, BH, qk_rows) || !make_map_bf16(&mv, v, d->dv, d->N, BH))
     return LINATTN_ERR_CUDA;
-  if (!set_smem(tc::causal_tc_kernel, static_cast<int>(tc::kSmemBytes))) return LINATTN_ERR_CUDA;
-  const int grid = BH * (d->dv / tc::DVS);
-  tc::causal_tc_kernel<<<grid, tc::NT, tc::kSmemBytes, s>>>(
-      mq, mk, mv, lam, eps, static_cast<bf16 *>(out), S_final, z_final, d->H, d->N, d->dv);
+  auto *kern = paired ? tc::causal_tc_kernel<true> : tc::causal_tc_kernel<false>;
+  if (!set_smem(kern, static_cast<int>(tc::kSmemBytes))) return LINATTN_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(BH * (d->dv / tc::DVS));
+  cfg.blockDim = dim3(tc::NT);
+  cfg.dynamicSmemBytes = tc::kSmemBytes;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = paired ? 2 : 1;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, lam, eps, static_cast<bf16 *>(out), S_final,
+                         z_final, d->H, d->N, d->dv) != cudaSuccess)
+    return LINATTN_ERR_CUDA;
   return launch_status();
 }
 
