@@ -265,5 +265,31 @@ def test_convex_hull_on_gpu(cuda_lib):
     assert bool((y >= lo - slack).all()) and bool((y <= hi + slack).all())
 
 
+
+@pytest.mark.parametrize("N", [1, 100, 128, 129, 1111, 4096])
+def test_global_tc_edges(cuda_lib, N):
+    """Tensor-core global path (bf16, d = 64, even H): ragged and tiny N."""
+    q, k, v = inputs.random_case(300 + N, 2, 4, N, 64, 64, torch.bfloat16, scale=0.125)
+    out, KV, ks = cuda_lib.fwd_global(q.to(DEV), k.to(DEV), v.to(DEV), 1e-6)
+    torch.cuda.synchronize()
+    y_o, KV_o, ks_o = oracle.global_attn(q, k, v, 1e-6)
+    assert_close("y", out, y_o, 2e-2)
+    assert_close("KV", KV, KV_o, 2e-2)
+    assert_close("ksum", ks, ks_o, 2e-2)
+
+
+def test_global_simt_second_opinion(cuda_lib, monkeypatch):
+    q, k, v = inputs.random_case(17, 1, 6, 3000, 64, 64, torch.bfloat16, scale=0.125)
+    out_tc, KV_tc, _ = cuda_lib.fwd_global(q.to(DEV), k.to(DEV), v.to(DEV), 1e-6)
+    monkeypatch.setenv("LINATTN_GLOBAL_KERNEL", "simt")
+    out_s, KV_s, _ = cuda_lib.fwd_global(q.to(DEV), k.to(DEV), v.to(DEV), 1e-6)
+    torch.cuda.synchronize()
+    y_o, KV_o, _ = oracle.global_attn(q, k, v, 1e-6)
+    assert_close("y tc", out_tc, y_o, 2e-2)
+    assert_close("y simt", out_s, y_o, 2e-2)
+    assert_close("KV tc", KV_tc, KV_o, 2e-2)
+    assert_close("KV simt", KV_s, KV_o, 1e-4)
+
+
 def test_no_device_errors_recorded(cuda_lib):
     assert cuda_lib.linattn_device_status(clear=False) == 0

@@ -19,6 +19,7 @@
 #include "causal_simt.cuh"
 #include "causal_tc.cuh"
 #include "global_simt.cuh"
+#include "global_tc.cuh"
 
 namespace linattn {
 namespace {
@@ -264,6 +265,37 @@ int launch_global_simt(const linattn_dims *d, const void *q, const void *k, cons
   return launch_status();
 }
 
+// Tensor-core global path: bf16, d_k = d_v = 64, an even number of heads
+// (heads are paired in the KV kernel).  LINATTN_GLOBAL_KERNEL=simt forces the
+// CUDA-core kernels.
+bool use_tc_global(const linattn_dims *d) {
+  const char *e = std::getenv("LINATTN_GLOBAL_KERNEL");
+  if (e && std::strcmp(e, "simt") == 0) return false;
+  return d->dtype == LINATTN_BF16 && d->dk == gtc::D && d->dv == gtc::D && d->H % 2 == 0;
+}
+
+int launch_global_tc(const linattn_dims *d, const void *q, const void *k, const void *v, float eps,
+                     void *out, float *KV, float *ksum, cudaStream_t s) {
+  const int BH = d->B * d->H;
+  CUtensorMap mq, mk, mv, my;
+  if (!make_map_bf16(&mq, q, d->dk, d->N, BH) || !make_map_bf16(&mk, k, d->dk, d->N, BH) ||
+      !make_map_bf16(&mv, v, d->dv, d->N, BH) || !make_map_bf16(&my, out, d->dv, d->N, BH))
+    return LINATTN_ERR_CUDA;
+  const int sms = num_sms();
+  if (sms <= 0) return LINATTN_ERR_CUDA;
+  if (!set_smem(gtc::global_kv_tc_kernel, static_cast<int>(gtc::kv::kSmemBytes)) ||
+      !set_smem(gtc::global_out_tc_kernel, static_cast<int>(gtc::out::kSmemBytes)))
+    return LINATTN_ERR_CUDA;
+  const long chunks = (d->N + gtc::C - 1) / gtc::C;
+  const long u1 = static_cast<long>(BH / 2) * chunks, u2 = static_cast<long>(BH) * chunks;
+  gtc::global_kv_tc_kernel<<<static_cast<int>(u1 < sms ? u1 : sms), gtc::kv::NT,
+                             gtc::kv::kSmemBytes, s>>>(mk, mv, KV, ksum, BH / 2, d->N);
+  if (cudaGetLastError() != cudaSuccess) return LINATTN_ERR_CUDA;
+  gtc::global_out_tc_kernel<<<static_cast<int>(u2 < sms ? u2 : sms), gtc::out::NT,
+                              gtc::out::kSmemBytes, s>>>(mq, my, KV, ksum, eps, BH, d->N);
+  return launch_status();
+}
+
 template <int DK, typename T>
 int global_dv(const linattn_dims *d, const void *q, const void *k, const void *v, float eps,
               void *out, float *KV, float *ksum, cudaStream_t s) {
@@ -348,6 +380,7 @@ extern "C" int linattn_fwd_global(const linattn_dims *d, const void *q, const vo
   if (cudaMemsetAsync(KV, 0, nS, s) != cudaSuccess) return LINATTN_ERR_CUDA;
   if (cudaMemsetAsync(ksum, 0, nz, s) != cudaSuccess) return LINATTN_ERR_CUDA;
   if (d->N == 0) return LINATTN_OK;
+  if (use_tc_global(d)) return launch_global_tc(d, q, k, v, eps, out, KV, ksum, s);
   if (d->dtype == LINATTN_F32)
     return global_dispatch<float>(d, q, k, v, eps, out, KV, ksum, s);
   return global_dispatch<bf16>(d, q, k, v, eps, out, KV, ksum, s);
