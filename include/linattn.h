@@ -94,6 +94,29 @@ LINATTN_API int linattn_fwd_causal(const linattn_dims *dims, const void *q, cons
                        float *S_final, float *z_final, linattn_stream_t stream);
 
 /*
+ * The same forward continued from a given state: the recurrence of
+ * linattn_fwd_causal with S_0 = S_init, z_0 = z_init instead of zero
+ * ([FW] §4.1: the fast weights persist across calls; §6: a non-zero
+ * initial state), so that
+ *   y_i = phi(q_i)^T S_i / (phi(q_i)^T z_i + eps),
+ *   S_i = lambda^i S_init + sum_{j<=i} lambda^(i-j) phi(k_j) v_j^T,
+ *   z_i = lambda^i z_init + sum_{j<=i} lambda^(i-j) phi(k_j).
+ * A prefill of N1 tokens followed by this call on the next N2 tokens with
+ * the prefill's S_final / z_final gives the same y, S_final, z_final as one
+ * call on N1 + N2 tokens.
+ *   S_init [B, H, dk, dv] fp32, z_init [B, H, dk] fp32: both NULL (a zero
+ *   state, exactly linattn_fwd_causal) or both device pointers, 16-byte
+ *   aligned, owned by the caller, only read, and not overlapping out,
+ *   S_final or z_final (LINATTN_ERR_INVALID otherwise; to update a state in
+ *   place, alternate two buffers).
+ * N = 0 copies S_init / z_init to S_final / z_final.
+ */
+LINATTN_API int linattn_fwd_causal_from(const linattn_dims *dims, const void *q, const void *k,
+                       const void *v, const float *lambda, float eps,
+                       const float *S_init, const float *z_init, void *out,
+                       float *S_final, float *z_final, linattn_stream_t stream);
+
+/*
  * Global (non-causal) forward ([LN] §3 after the sum swap and §6 forward;
  * [BSA] linear-attention code, here with eps):
  *   KV = sum_n phi(k_n) v_n^T, ksum = sum_n phi(k_n),

@@ -90,6 +90,22 @@ def test_causal_rejects_bad_arguments(lib):
     assert causal(lib, D(), out=FAKE) == linattn.LINATTN_ERR_INVALID
 
 
+def test_causal_from_rejects_bad_state_arguments(lib):
+    S0, z0 = P(0x7F0000500000), P(0x7F0000600000)
+    Sf, zf = P(0x7F0000700000), P(0x7F0000800000)
+    cf = lambda **kw: lib.linattn_fwd_causal_from(
+        ctypes.byref(kw.get("d", D())), FAKE, FAKE2, FAKE3, None, 1e-6, kw.get("S0", S0),
+        kw.get("z0", z0), kw.get("out", FAKE4), kw.get("Sf", Sf), kw.get("zf", zf), None)
+    assert cf(z0=None) == linattn.LINATTN_ERR_INVALID        # one of the pair missing
+    assert cf(S0=None) == linattn.LINATTN_ERR_INVALID
+    assert cf(S0=MIS) == linattn.LINATTN_ERR_INVALID
+    assert cf(z0=MIS) == linattn.LINATTN_ERR_INVALID
+    assert cf(Sf=S0) == linattn.LINATTN_ERR_INVALID          # state read and written in place
+    assert cf(zf=z0) == linattn.LINATTN_ERR_INVALID
+    assert cf(out=S0) == linattn.LINATTN_ERR_INVALID
+    assert cf(d=D(dk=48)) == linattn.LINATTN_ERR_UNSUPPORTED
+
+
 def test_empty_batch_is_a_no_op(lib):
     # B*H == 0: nothing to do, nothing launched, even with NULL buffers
     assert causal(lib, D(B=0), q=None, k=None, v=None, out=None) == linattn.LINATTN_OK

@@ -224,6 +224,22 @@ def test_prefill_then_decode_equals_prefill():
     assert np.array_equal(S2, S) and np.array_equal(z2, z)
 
 
+def test_initial_state_single_token_closed_form():
+    """One token from a given (S0, z0): S1 = lam S0 + phi(k) v^T, z1 = lam z0 +
+    phi(k), y = phi(q) S1 / (phi(q) z1 + eps), written out with numpy."""
+    q, k, v = rand(13, 1, 1, 1, 6, 4)
+    rng = np.random.default_rng(14)
+    S0 = rng.standard_normal((1, 1, 6, 4))
+    z0 = rng.random((1, 1, 6)) + 0.5
+    lam, eps = 0.8, 1e-3
+    y, S, z = oracle.causal(q, k, v, np.array([lam]), eps=eps, S0=S0, z0=z0)
+    fq, fk = phi_np(q[0, 0, 0]), phi_np(k[0, 0, 0])
+    S1 = lam * S0[0, 0] + np.outer(fk, v[0, 0, 0])
+    z1 = lam * z0[0, 0] + fk
+    assert rel(S[0, 0], S1) < 1e-14 and rel(z[0, 0], z1) < 1e-14
+    assert rel(y[0, 0, 0], fq @ S1 / (fq @ z1 + eps)) < 1e-14
+
+
 def test_single_token_and_constant_values():
     q, k, v = rand(8, 1, 1, 1, 8, 4)
     eps = 1e-3

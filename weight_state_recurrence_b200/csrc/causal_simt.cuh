@@ -13,7 +13,8 @@
 //   z       <- lambda^Cv z + sum_s lambda^(Cv-1-s) phi(k_s)
 // which unrolls the recurrence S_i = lambda S_{i-1} + phi(k_i) v_i^T exactly.
 // One CTA owns one (b, h) and a DVS-wide slice of dv; S for the slice lives in
-// shared memory for the whole sequence.
+// shared memory for the whole sequence, starting from the caller's state if
+// one is given.
 #pragma once
 #include "common.cuh"
 
@@ -30,7 +31,8 @@ constexpr int causal_simt_smem_floats() {
 template <int DK, int DVS, typename T>
 __global__ void __launch_bounds__(256) causal_simt_kernel(
     const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
-    const float *__restrict__ lam, float eps, T *__restrict__ out, float *__restrict__ S_final,
+    const float *__restrict__ lam, float eps, const float *__restrict__ S_init,
+    const float *__restrict__ z_init, T *__restrict__ out, float *__restrict__ S_final,
     float *__restrict__ z_final, int H, int N, int DV) {
   constexpr int C = kSimtChunk, NT = 256, QS = DK + 1;
   static_assert(DVS % 4 == 0, "slice must be float4-divisible");
@@ -52,8 +54,10 @@ __global__ void __launch_bounds__(256) causal_simt_kernel(
   const float L = lam ? lam[h] : 1.f;
 
   if (tid <= C) pw[tid] = pow_int(L, tid);
-  for (int i = tid; i < DK * DVS; i += NT) sS[i] = 0.f;
-  for (int i = tid; i < DK; i += NT) sz[i] = 0.f;
+  // the state before the first token: the caller's (S_init, z_init), else zero
+  for (int i = tid; i < DK * DVS; i += NT)
+    sS[i] = S_init ? S_init[(pair * DK + i / DVS) * DV + j0 + i % DVS] : 0.f;
+  for (int i = tid; i < DK; i += NT) sz[i] = z_init ? z_init[pair * DK + i] : 0.f;
 
   const T *qp = q + pair * static_cast<long>(N) * DK;
   const T *kp = k + pair * static_cast<long>(N) * DK;

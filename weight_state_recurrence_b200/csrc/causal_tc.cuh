@@ -258,7 +258,8 @@ __global__ void __launch_bounds__(NT, 1)
     causal_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                      const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const float *__restrict__ lam,
-                     float eps, __nv_bfloat16 *__restrict__ out, float *__restrict__ S_final,
+                     float eps, const float *__restrict__ S_init, const float *__restrict__ z_init,
+                     __nv_bfloat16 *__restrict__ out, float *__restrict__ S_final,
                      float *__restrict__ z_final, int H, int N, int DV) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *sm = smem_raw;
@@ -337,6 +338,54 @@ __global__ void __launch_bounds__(NT, 1)
   if (kPair) cluster_sync_all();   // the peer's barriers are initialised before any remote use
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+
+  // A caller-supplied starting state: the state warpgroup puts lambda^Cv S_init
+  // (and z) into the TMEM state, where the first state MMA accumulates onto
+  // it, and S_init, z_init into the operands of the first O_x MMA.
+  const bool has_init = S_init != nullptr;
+  if (has_init) {
+    if (warp >= 12 && warp < 16) {
+      const int r = (warp - 12) * 32 + lane;   // d_k row
+      const uint32_t lane_field = static_cast<uint32_t>((warp - 12) * 32) << 16;
+      const float g0 = pw[nchunks == 1 ? Ct : C];   // decay of the first chunk
+      const float4 *src =
+          reinterpret_cast<const float4 *>(S_init + (static_cast<long>(pair) * DK + r) * DV + j0);
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint32_t sv[32], pk[16];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float4 f = src[half * 8 + i];
+          sv[4 * i] = __float_as_uint(f.x * g0);
+          sv[4 * i + 1] = __float_as_uint(f.y * g0);
+          sv[4 * i + 2] = __float_as_uint(f.z * g0);
+          sv[4 * i + 3] = __float_as_uint(f.w * g0);
+          pk[2 * i] = pack_bf16(f.x, f.y);
+          pk[2 * i + 1] = pack_bf16(f.z, f.w);
+        }
+        tmem_st_32x32b_x32(tmem + lane_field + kTmS + half * 32, sv);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          *reinterpret_cast<uint4 *>(sm + kOffS + sw128_offset(r, half * 64 + i * 16)) =
+              make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+      }
+      const float z0 = z_init[static_cast<long>(pair) * DK + r];
+      uint32_t zcol[16];
+      zcol[0] = __float_as_uint(z0 * g0);
+#pragma unroll
+      for (int i = 1; i < 16; ++i) zcol[i] = 0u;
+      tmem_st_32x32b_x16(tmem + lane_field + kTmS + 64, zcol);
+      tmem_wait_st();
+      const __nv_bfloat16 zh = __float2bfloat16_rn(z0);
+      const __nv_bfloat16 zl = __float2bfloat16_rn(z0 - __bfloat162float(zh));
+      *reinterpret_cast<__nv_bfloat16 *>(sm + kOffX + sw128_offset(r, 2)) = zh;
+      *reinterpret_cast<__nv_bfloat16 *>(sm + kOffX + sw128_offset(r, 4)) = zl;
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+  }
 
   auto fail = [&]() { *abort_flag = 1; };
   // Roles with several warps meet at a named barrier once per step.  A
@@ -430,7 +479,8 @@ __global__ void __launch_bounds__(NT, 1)
 #pragma unroll
         for (int ks = 0; ks < C / 16; ++ks)
           umma_bf16(tmem + kTmS, sdesc_sw128(st + kOffK + ks * 2048, kPanel, 1024),
-                    sdesc_sw128(va + ks * 2048, xa - va, 1024), kIdS, (c > 0 || ks > 0) ? 1u : 0u);
+                    sdesc_sw128(va + ks * 2048, xa - va, 1024), kIdS,
+                    (c > 0 || ks > 0 || has_init) ? 1u : 0u);
         umma_commit(bar(kDsDone));
         // [O_x | . | qz] = phi(Q) [S | 1, z_hi, z_lo]   (state before this chunk)
         if (c >= 1 && !mbar_wait(bar(kOutDone), (c - 1) & 1)) {

@@ -182,43 +182,45 @@ int decode_dispatch(const linattn_dims *d, const void *q, const void *k, const v
 
 template <int DK, int DVS, typename T>
 int launch_causal_simt(const linattn_dims *d, const void *q, const void *k, const void *v,
-                       const float *lam, float eps, void *out, float *S_final, float *z_final,
-                       cudaStream_t s) {
+                       const float *lam, float eps, const float *S_init, const float *z_init,
+                       void *out, float *S_final, float *z_final, cudaStream_t s) {
   auto *kern = causal_simt_kernel<DK, DVS, T>;
   const int bytes = causal_simt_smem_floats<DK, DVS>() * 4;
   if (!set_smem(kern, bytes)) return LINATTN_ERR_CUDA;
   const int grid = d->B * d->H * (d->dv / DVS);
   kern<<<grid, 256, bytes, s>>>(static_cast<const T *>(q), static_cast<const T *>(k),
-                                static_cast<const T *>(v), lam, eps, static_cast<T *>(out),
-                                S_final, z_final, d->H, d->N, d->dv);
+                                static_cast<const T *>(v), lam, eps, S_init, z_init,
+                                static_cast<T *>(out), S_final, z_final, d->H, d->N, d->dv);
   return launch_status();
 }
 
 template <int DK, typename T>
 int causal_simt_dv(const linattn_dims *d, const void *q, const void *k, const void *v,
-                   const float *lam, float eps, void *out, float *S_final, float *z_final,
-                   cudaStream_t s) {
+                   const float *lam, float eps, const float *S_init, const float *z_init,
+                   void *out, float *S_final, float *z_final, cudaStream_t s) {
   if (d->dv == 16)
-    return launch_causal_simt<DK, 16, T>(d, q, k, v, lam, eps, out, S_final, z_final, s);
-  return launch_causal_simt<DK, 32, T>(d, q, k, v, lam, eps, out, S_final, z_final, s);
+    return launch_causal_simt<DK, 16, T>(d, q, k, v, lam, eps, S_init, z_init, out, S_final,
+                                         z_final, s);
+  return launch_causal_simt<DK, 32, T>(d, q, k, v, lam, eps, S_init, z_init, out, S_final,
+                                       z_final, s);
 }
 
 template <typename T>
 int causal_simt_dispatch(const linattn_dims *d, const void *q, const void *k, const void *v,
-                         const float *lam, float eps, void *out, float *S_final, float *z_final,
-                         cudaStream_t s) {
+                         const float *lam, float eps, const float *S_init, const float *z_init,
+                         void *out, float *S_final, float *z_final, cudaStream_t s) {
   switch (d->dk) {
-    case 16: return causal_simt_dv<16, T>(d, q, k, v, lam, eps, out, S_final, z_final, s);
-    case 32: return causal_simt_dv<32, T>(d, q, k, v, lam, eps, out, S_final, z_final, s);
-    case 64: return causal_simt_dv<64, T>(d, q, k, v, lam, eps, out, S_final, z_final, s);
-    case 128: return causal_simt_dv<128, T>(d, q, k, v, lam, eps, out, S_final, z_final, s);
+    case 16: return causal_simt_dv<16, T>(d, q, k, v, lam, eps, S_init, z_init, out, S_final, z_final, s);
+    case 32: return causal_simt_dv<32, T>(d, q, k, v, lam, eps, S_init, z_init, out, S_final, z_final, s);
+    case 64: return causal_simt_dv<64, T>(d, q, k, v, lam, eps, S_init, z_init, out, S_final, z_final, s);
+    case 128: return causal_simt_dv<128, T>(d, q, k, v, lam, eps, S_init, z_init, out, S_final, z_final, s);
   }
   return LINATTN_ERR_UNSUPPORTED;
 }
 
 int launch_causal_tc(const linattn_dims *d, const void *q, const void *k, const void *v,
-                     const float *lam, float eps, void *out, float *S_final, float *z_final,
-                     cudaStream_t s) {
+                     const float *lam, float eps, const float *S_init, const float *z_init,
+                     void *out, float *S_final, float *z_final, cudaStream_t s) {
   const int BH = d->B * d->H;
   // dv = 128: the two column halves of a head run as a 2-CTA cluster that
   // shares the feature map (each CTA loads 64 rows of every q/k tile)
@@ -242,8 +244,9 @@ int launch_causal_tc(const linattn_dims *d, const void *q, const void *k, const 
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, lam, eps, static_cast<bf16 *>(out), S_final,
-                         z_final, d->H, d->N, d->dv) != cudaSuccess)
+  if (cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, lam, eps, S_init, z_init,
+                         static_cast<bf16 *>(out), S_final, z_final, d->H, d->N,
+                         d->dv) != cudaSuccess)
     return LINATTN_ERR_CUDA;
   return launch_status();
 }
@@ -325,9 +328,14 @@ int global_dispatch(const linattn_dims *d, const void *q, const void *k, const v
 
 using namespace linattn;
 
-extern "C" int linattn_fwd_causal(const linattn_dims *d, const void *q, const void *k,
-                                  const void *v, const float *lambda, float eps, void *out,
-                                  float *S_final, float *z_final, linattn_stream_t stream) {
+namespace linattn {
+namespace {
+
+// Both causal entry points: validation, then the tensor-core kernel (bf16,
+// d_k = 128, dv a multiple of 64) or the CUDA-core kernel.
+int fwd_causal_impl(const linattn_dims *d, const void *q, const void *k, const void *v,
+                    const float *lambda, float eps, const float *S_init, const float *z_init,
+                    void *out, float *S_final, float *z_final, cudaStream_t s) {
   int rc = check_dims(d, true);
   if (rc != LINATTN_OK) return rc;
   if (bad_eps(eps)) return LINATTN_ERR_INVALID;
@@ -337,23 +345,59 @@ extern "C" int linattn_fwd_causal(const linattn_dims *d, const void *q, const vo
   const size_t nq = BH * d->N * d->dk * es, nv = BH * d->N * d->dv * es;
   const size_t nS = BH * d->dk * d->dv * 4, nz = BH * d->dk * 4;
   if (d->N > 0 && (!q || !k || !v || !out)) return LINATTN_ERR_INVALID;
+  if ((S_init == nullptr) != (z_init == nullptr)) return LINATTN_ERR_INVALID;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
-      !aligned16(S_final) || !aligned16(z_final) || !aligned16(lambda))
+      !aligned16(S_final) || !aligned16(z_final) || !aligned16(lambda) || !aligned16(S_init) ||
+      !aligned16(z_init))
     return LINATTN_ERR_INVALID;
   if (overlaps(out, nv, q, nq) || overlaps(out, nv, k, nq) || overlaps(out, nv, v, nv) ||
       overlaps(S_final, nS, out, nv) || overlaps(z_final, nz, out, nv) ||
       overlaps(S_final, nS, z_final, nz))
     return LINATTN_ERR_INVALID;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  // the starting state is read while the outputs are written: no overlap
+  if (overlaps(S_init, nS, out, nv) || overlaps(S_init, nS, S_final, nS) ||
+      overlaps(S_init, nS, z_final, nz) || overlaps(z_init, nz, out, nv) ||
+      overlaps(z_init, nz, S_final, nS) || overlaps(z_init, nz, z_final, nz))
+    return LINATTN_ERR_INVALID;
   if (d->N == 0) {
-    if (S_final && cudaMemsetAsync(S_final, 0, nS, s) != cudaSuccess) return LINATTN_ERR_CUDA;
-    if (z_final && cudaMemsetAsync(z_final, 0, nz, s) != cudaSuccess) return LINATTN_ERR_CUDA;
+    // no token: the final state is the starting state
+    if (S_final) {
+      const cudaError_t e = S_init ? cudaMemcpyAsync(S_final, S_init, nS, cudaMemcpyDeviceToDevice, s)
+                                   : cudaMemsetAsync(S_final, 0, nS, s);
+      if (e != cudaSuccess) return LINATTN_ERR_CUDA;
+    }
+    if (z_final) {
+      const cudaError_t e = z_init ? cudaMemcpyAsync(z_final, z_init, nz, cudaMemcpyDeviceToDevice, s)
+                                   : cudaMemsetAsync(z_final, 0, nz, s);
+      if (e != cudaSuccess) return LINATTN_ERR_CUDA;
+    }
     return LINATTN_OK;
   }
-  if (use_tc_causal(d)) return launch_causal_tc(d, q, k, v, lambda, eps, out, S_final, z_final, s);
+  if (use_tc_causal(d))
+    return launch_causal_tc(d, q, k, v, lambda, eps, S_init, z_init, out, S_final, z_final, s);
   if (d->dtype == LINATTN_F32)
-    return causal_simt_dispatch<float>(d, q, k, v, lambda, eps, out, S_final, z_final, s);
-  return causal_simt_dispatch<bf16>(d, q, k, v, lambda, eps, out, S_final, z_final, s);
+    return causal_simt_dispatch<float>(d, q, k, v, lambda, eps, S_init, z_init, out, S_final,
+                                       z_final, s);
+  return causal_simt_dispatch<bf16>(d, q, k, v, lambda, eps, S_init, z_init, out, S_final,
+                                    z_final, s);
+}
+
+}  // namespace
+}  // namespace linattn
+
+extern "C" int linattn_fwd_causal(const linattn_dims *d, const void *q, const void *k,
+                                  const void *v, const float *lambda, float eps, void *out,
+                                  float *S_final, float *z_final, linattn_stream_t stream) {
+  return fwd_causal_impl(d, q, k, v, lambda, eps, nullptr, nullptr, out, S_final, z_final,
+                         reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" int linattn_fwd_causal_from(const linattn_dims *d, const void *q, const void *k,
+                                       const void *v, const float *lambda, float eps,
+                                       const float *S_init, const float *z_init, void *out,
+                                       float *S_final, float *z_final, linattn_stream_t stream) {
+  return fwd_causal_impl(d, q, k, v, lambda, eps, S_init, z_init, out, S_final, z_final,
+                         reinterpret_cast<cudaStream_t>(stream));
 }
 
 extern "C" int linattn_fwd_global(const linattn_dims *d, const void *q, const void *k,

@@ -26,7 +26,7 @@ LINATTN_ERR_UNSUPPORTED = 2
 LINATTN_ERR_CUDA = 3
 LINATTN_ERR_DEVICE = 4
 
-ENTRY_POINTS = ("linattn_fwd_causal", "linattn_fwd_global", "linattn_decode_step",
+ENTRY_POINTS = ("linattn_fwd_causal", "linattn_fwd_causal_from", "linattn_fwd_global", "linattn_decode_step",
                 "linattn_status_string", "linattn_device_status", "linattn_version")
 
 
@@ -64,6 +64,8 @@ def load(build_if_missing: bool = True):
     dp = ctypes.POINTER(linattn_dims)
     lib.linattn_fwd_causal.argtypes = [dp, vp, vp, vp, fp, f, vp, fp, fp, vp]
     lib.linattn_fwd_causal.restype = i
+    lib.linattn_fwd_causal_from.argtypes = [dp, vp, vp, vp, fp, f, fp, fp, vp, fp, fp, vp]
+    lib.linattn_fwd_causal_from.restype = i
     lib.linattn_fwd_global.argtypes = [dp, vp, vp, vp, f, vp, fp, fp, vp]
     lib.linattn_fwd_global.restype = i
     lib.linattn_decode_step.argtypes = [dp, vp, vp, vp, fp, f, fp, fp, vp, vp]
@@ -136,6 +138,28 @@ def linattn_fwd_causal(q, k, v, lam, eps, out, S_final=None, z_final=None, strea
                                      _stream(stream)), "linattn_fwd_causal")
 
 
+def linattn_fwd_causal_from(q, k, v, lam, eps, S_init, z_init, out, S_final=None, z_final=None,
+                            stream=None):
+    """Causal forward continued from (S_init [B,H,dk,dv], z_init [B,H,dk]) fp32,
+    both given or both None; the other arguments as linattn_fwd_causal."""
+    B, H, N, dk = q.shape
+    dv = v.shape[-1]
+    if k.shape != q.shape or tuple(v.shape) != (B, H, N, dv) or out.shape != v.shape:
+        raise ValueError("shape mismatch among q, k, v, out")
+    if not (q.dtype == k.dtype == v.dtype == out.dtype):
+        raise ValueError("q, k, v, out must share one dtype")
+    _f32(lam, (H,), "lambda")
+    _f32(S_init, (B, H, dk, dv), "S_init")
+    _f32(z_init, (B, H, dk), "z_init")
+    _f32(S_final, (B, H, dk, dv), "S_final")
+    _f32(z_final, (B, H, dk), "z_final")
+    d = linattn_dims(B, H, N, dk, dv, _dtype_code(q.dtype))
+    _check(load().linattn_fwd_causal_from(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), _ptr(lam),
+                                          float(eps), _ptr(S_init), _ptr(z_init), _ptr(out),
+                                          _ptr(S_final), _ptr(z_final), _stream(stream)),
+           "linattn_fwd_causal_from")
+
+
 def linattn_fwd_global(q, k, v, eps, out, KV, ksum, stream=None):
     """Global forward: q, k [B,H,N,dk], v/out [B,H,N,dv]; KV [B,H,dk,dv] and
     ksum [B,H,dk] fp32 are written."""
@@ -184,13 +208,17 @@ def linattn_version() -> int:
 
 
 # ---------------------------------------------------------------- helpers
-def fwd_causal(q, k, v, lam=None, eps=1e-6, want_state=True, stream=None):
+def fwd_causal(q, k, v, lam=None, eps=1e-6, want_state=True, S_init=None, z_init=None,
+               stream=None):
     B, H, N, dk = q.shape
     dv = v.shape[-1]
     out = torch.empty_like(v)
     S = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device) if want_state else None
     z = torch.empty((B, H, dk), dtype=torch.float32, device=q.device) if want_state else None
-    linattn_fwd_causal(q, k, v, lam, eps, out, S, z, stream)
+    if S_init is None and z_init is None:
+        linattn_fwd_causal(q, k, v, lam, eps, out, S, z, stream)
+    else:
+        linattn_fwd_causal_from(q, k, v, lam, eps, S_init, z_init, out, S, z, stream)
     return out, S, z
 
 
