@@ -117,6 +117,29 @@ LINATTN_API int linattn_fwd_causal_from(const linattn_dims *dims, const void *q,
                        float *S_final, float *z_final, linattn_stream_t stream);
 
 /*
+ * Backward of linattn_fwd_causal (zero starting state): the gradients of
+ * L = sum over all (b, h, i) of dy_i . y_i ([FW] §3.1 and §4.1 train the
+ * chunked forward; the gradients follow from the recurrence of [FW] §2.1,
+ * §3.2, §4.2 by the chain rule, with phi'(x) = 1 for x > 0 and e^x otherwise).
+ *   q, k, v, lambda, eps, dims: as given to the forward
+ *   dy      [B, H, N, dv] dtype     upstream gradient of out
+ *   dq, dk  [B, H, N, dk] dtype     written
+ *   dv      [B, H, N, dv] dtype     written
+ *   dlambda [H] fp32 or NULL        written (summed over the batch); with
+ *                                   lambda = NULL it is the gradient at 1
+ * Every output must overlap no input and no other output.  The forward is
+ * recomputed inside (nothing from it is needed).  fp32 arithmetic for both
+ * dtypes; dlambda is a sum of per-(b, h) fp32 atomics, so its last bits may
+ * vary from run to run.  Between its two passes the kernel keeps two fp32
+ * numbers per token in the first 8 bytes of that token's dk row, which it
+ * overwrites afterwards: dk must not be read before the call completes.
+ */
+LINATTN_API int linattn_bwd_causal(const linattn_dims *dims, const void *q, const void *k,
+                       const void *v, const float *lambda, float eps, const void *dy,
+                       void *dq, void *dk, void *dv, float *dlambda,
+                       linattn_stream_t stream);
+
+/*
  * Global (non-causal) forward ([LN] §3 after the sum swap and §6 forward;
  * [BSA] linear-attention code, here with eps):
  *   KV = sum_n phi(k_n) v_n^T, ksum = sum_n phi(k_n),

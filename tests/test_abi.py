@@ -106,6 +106,24 @@ def test_causal_from_rejects_bad_state_arguments(lib):
     assert cf(d=D(dk=48)) == linattn.LINATTN_ERR_UNSUPPORTED
 
 
+def test_bwd_rejects_bad_arguments(lib):
+    DY, DQ, DK, DV = (P(0x7F0000500000), P(0x7F0000600000), P(0x7F0000700000),
+                      P(0x7F0000800000))
+    bw = lambda **kw: lib.linattn_bwd_causal(
+        ctypes.byref(kw.get("d", D())), FAKE, FAKE2, FAKE3, kw.get("lam", None),
+        kw.get("eps", 1e-6), kw.get("dy", DY), kw.get("dq", DQ), kw.get("dk", DK),
+        kw.get("dv", DV), kw.get("dl", None), None)
+    assert bw(dy=None) == linattn.LINATTN_ERR_INVALID
+    assert bw(dq=None) == linattn.LINATTN_ERR_INVALID
+    assert bw(dk=MIS) == linattn.LINATTN_ERR_INVALID
+    assert bw(eps=-1.0) == linattn.LINATTN_ERR_INVALID
+    assert bw(d=D(dv=24)) == linattn.LINATTN_ERR_UNSUPPORTED
+    assert bw(dq=FAKE) == linattn.LINATTN_ERR_INVALID        # gradient over an input
+    assert bw(dv=DY) == linattn.LINATTN_ERR_INVALID
+    assert bw(dk=DQ) == linattn.LINATTN_ERR_INVALID          # two gradients overlap
+    assert bw(dl=MIS) == linattn.LINATTN_ERR_INVALID
+
+
 def test_empty_batch_is_a_no_op(lib):
     # B*H == 0: nothing to do, nothing launched, even with NULL buffers
     assert causal(lib, D(B=0), q=None, k=None, v=None, out=None) == linattn.LINATTN_OK

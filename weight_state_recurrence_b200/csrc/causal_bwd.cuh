@@ -1,0 +1,322 @@
+// Backward of the causal forward on CUDA cores, fp32 arithmetic throughout.
+//
+// For L = sum_i dy_i . y_i with y_i = num_i / den_i, num_i = phi(q_i)^T S_i,
+// den_i = phi(q_i)^T z_i + eps and the recurrence of the fast-weight article
+// (§2.1, §3.2, §4.2: S_i = lambda S_{i-1} + phi(k_i) v_i^T, z likewise):
+//   dnum_i = dy_i / den_i,   dden_i = -(dy_i . y_i) / den_i
+//   dphi(q_i) = S_i dnum_i + z_i dden_i
+//   R_j = sum_{i>=j} lambda^(i-j) phi(q_i) dnum_i^T,  r_j = sum_{i>=j} lambda^(i-j) phi(q_i) dden_i
+//   dphi(k_j) = R_j v_j + r_j,   dv_j = R_j^T phi(k_j)
+//   dlambda = sum_i phi(q_i)^T (S'_i dnum_i + z'_i dden_i),  S' = dS/dlambda
+//   dq = dphi(q) * phi'(q), phi'(x) = 1 (x > 0) else e^x = phi(x); dk likewise.
+// R and r obey the forward recurrence run backwards (R_j = lambda R_{j+1} +
+// phi(q_j) dnum_j^T), so the same chunked form applies in reverse (the §3.1
+// triangular mask, §5.2 blockwise accumulation), with C = 32 tokens a chunk.
+//
+// One CTA owns one (b, h) and all of dv (dq needs the whole S dnum).  Sweep 1
+// runs over the chunks in order: it rebuilds S, z (and S', z' when dlambda is
+// wanted), forms den, y, dnum, dden per token, writes dq, and keeps den_i and
+// c_i = dy_i . y_i in the first 8 bytes of row i of dk (dk is an output not
+// written before sweep 2).  Sweep 2 runs over the chunks in reverse: it reads
+// those two numbers back, carries R, r and writes dk and dv.  No memory
+// beyond the caller's buffers is used.  dlambda is accumulated with one
+// atomicAdd per CTA onto a buffer the host has zeroed.
+#pragma once
+#include "common.cuh"
+
+namespace linattn {
+
+constexpr int kBwdChunk = 32;
+constexpr int kBwdThreads = 256;
+
+template <int DK, int DV>
+constexpr int causal_bwd_smem_floats(bool with_dlam) {
+  constexpr int C = kBwdChunk;
+  return 2 * C * (DK + 1) + 2 * C * DV + 3 * C * (C + 1) + DK * DV + DK +
+         (with_dlam ? DK * DV + DK : 0) + 4 * C + 2 * (C + 4) + 8;
+}
+
+// the two fp32 numbers a token keeps between the sweeps, in the first 8 bytes of its dk row
+template <typename T>
+__device__ __forceinline__ void stash_put(T *row, float den, float c) {
+  float2 *p = reinterpret_cast<float2 *>(row);
+  *p = make_float2(den, c);
+}
+template <typename T>
+__device__ __forceinline__ float2 stash_get(const T *row) {
+  return *reinterpret_cast<const float2 *>(row);
+}
+
+template <int DK, int DV, typename T>
+__global__ void __launch_bounds__(kBwdThreads) causal_bwd_kernel(
+    const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
+    const T *__restrict__ dy, const float *__restrict__ lam, float eps, T *__restrict__ dq,
+    T *__restrict__ dk, T *__restrict__ dv, float *__restrict__ dlam, int H, int N) {
+  constexpr int C = kBwdChunk, NT = kBwdThreads, QS = DK + 1, AS = C + 1;
+  constexpr int W = DV / 4;   // threads that share one token in the per-column phases
+  static_assert(DV % 4 == 0 && W <= 32 && (32 % W) == 0, "dv must be 16..128");
+  extern __shared__ __align__(16) float sm[];
+  const bool with_dlam = dlam != nullptr;
+  float *sQ = sm;                  // [C][DK+1]  phi(q)
+  float *sK = sQ + C * QS;         // [C][DK+1]  phi(k)
+  float *sV = sK + C * QS;         // [C][DV]    v
+  float *sG = sV + C * DV;         // [C][DV]    dy, then dnum
+  float *sA = sG + C * DV;         // [C][C+1]   lambda^(t-s) phi(q_t).phi(k_s), s <= t
+  float *sB = sA + C * AS;         // [C][C+1]   lambda^(t-s) (dnum_t.v_s + dden_t), s <= t
+  float *sP = sB + C * AS;         // [C][C+1]   phi(q_t).phi(k_s) (for dlambda)
+  float *sS = sP + C * AS;         // [DK][DV]   S (sweep 1) / R (sweep 2)
+  float *sz = sS + DK * DV;        // [DK]       z / r
+  float *sS2 = sz + DK;            // [DK][DV]   S' (dlambda only)
+  float *sz2 = sS2 + (with_dlam ? DK * DV : 0);   // [DK] z'
+  float *sDen = sz2 + (with_dlam ? DK : 0);       // [C] den_t
+  float *sCc = sDen + C;           // [C] c_t = dy_t . y_t
+  float *sDd = sCc + C;            // [C] dden_t
+  float *pw = sDd + 2 * C;         // [C+4] lambda^i
+  float *dpw = pw + (C + 4);       // [C+4] i lambda^(i-1)
+  float *sRed = dpw + (C + 4);     // [8]   block reduction
+
+  const long pair = blockIdx.x;
+  const int h = static_cast<int>(pair % H);
+  const int tid = threadIdx.x;
+  const float L = lam ? lam[h] : 1.f;
+  if (tid < C + 4) pw[tid] = pow_int(L, tid);
+  __syncthreads();
+  if (tid < C + 4) dpw[tid] = tid == 0 ? 0.f : static_cast<float>(tid) * pw[tid - 1];
+  for (int i = tid; i < DK * DV; i += NT) {
+    sS[i] = 0.f;
+    if (with_dlam) sS2[i] = 0.f;
+  }
+  for (int i = tid; i < DK; i += NT) {
+    sz[i] = 0.f;
+    if (with_dlam) sz2[i] = 0.f;
+  }
+  const long qo = pair * static_cast<long>(N) * DK, vo = pair * static_cast<long>(N) * DV;
+  const int nchunks = (N + C - 1) / C;
+  float dl = 0.f;   // this thread's share of dlambda
+
+  // phi of a chunk's q and k rows, its v rows and dy rows; zero past the end
+  auto load_chunk = [&](int c0, int Cv) {
+    for (int i = tid; i < C * DK; i += NT) {
+      const int t = i / DK, a = i % DK;
+      float fq = 0.f, fk = 0.f;
+      if (t < Cv) {
+        fq = phi_f32(to_f32(q[qo + static_cast<long>(c0 + t) * DK + a]));
+        fk = phi_f32(to_f32(k[qo + static_cast<long>(c0 + t) * DK + a]));
+      }
+      sQ[t * QS + a] = fq;
+      sK[t * QS + a] = fk;
+    }
+    for (int i = tid; i < C * DV; i += NT) {
+      const int t = i / DV, j = i % DV;
+      const long o = vo + static_cast<long>(c0 + t) * DV + j;
+      sV[i] = t < Cv ? to_f32(v[o]) : 0.f;
+      sG[i] = t < Cv ? to_f32(dy[o]) : 0.f;
+    }
+  };
+  // masked decayed scores (and the raw ones for dlambda)
+  auto scores = [&](int Cv) {
+    for (int i = tid; i < C * C; i += NT) {
+      const int t = i / C, s = i % C;
+      float p = 0.f;
+      if (s <= t && t < Cv) {
+#pragma unroll 8
+        for (int a = 0; a < DK; ++a) p = fmaf(sQ[t * QS + a], sK[s * QS + a], p);
+      }
+      sA[t * AS + s] = s <= t && t < Cv ? pw[t - s] * p : 0.f;
+      sP[t * AS + s] = p;
+    }
+  };
+  // B_ts = lambda^(t-s) (dnum_t . v_s + dden_t); with dlambda also the
+  // intra-chunk term sum (t-s) lambda^(t-s-1) P_ts (dnum_t . v_s + dden_t)
+  auto scores_b = [&](int Cv, bool add_dlam) {
+    for (int i = tid; i < C * C; i += NT) {
+      const int t = i / C, s = i % C;
+      float b = 0.f;
+      if (s <= t && t < Cv) {
+        float e = sDd[t];
+#pragma unroll 8
+        for (int j = 0; j < DV; ++j) e = fmaf(sG[t * DV + j], sV[s * DV + j], e);
+        b = pw[t - s] * e;
+        if (add_dlam) dl = fmaf(dpw[t - s] * sP[t * AS + s], e, dl);
+      }
+      sB[t * AS + s] = b;
+    }
+  };
+
+  // ------------------------------------------------------------ sweep 1
+  for (int c = 0; c < nchunks; ++c) {
+    const int c0 = c * C, Cv = min(C, N - c0);
+    __syncthreads();
+    load_chunk(c0, Cv);
+    __syncthreads();
+    scores(Cv);
+    __syncthreads();
+    // den_t = sum_s A_ts + lambda^(t+1) phi(q_t).z + eps
+    if (tid < Cv) {
+      float rs = 0.f, qz = 0.f;
+      for (int s = 0; s <= tid; ++s) rs += sA[tid * AS + s];
+      for (int a = 0; a < DK; ++a) qz = fmaf(sQ[tid * QS + a], sz[a], qz);
+      sDen[tid] = rs + pw[tid + 1] * qz + eps;
+    }
+    __syncthreads();
+    // num_t, y_t = num/den, dnum_t = dy_t/den in place, c_t = dy_t . y_t
+    for (int i = tid; i < C * W; i += NT) {
+      const int t = i / W, j = 4 * (i % W);
+      float cpart = 0.f;
+      if (t < Cv) {
+        float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int s = 0; s <= t; ++s) {
+          const float a = sA[t * AS + s];
+          const float4 vv = *reinterpret_cast<const float4 *>(&sV[s * DV + j]);
+          num.x = fmaf(a, vv.x, num.x);
+          num.y = fmaf(a, vv.y, num.y);
+          num.z = fmaf(a, vv.z, num.z);
+          num.w = fmaf(a, vv.w, num.w);
+        }
+        float4 in = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int a = 0; a < DK; ++a) {
+          const float fq = sQ[t * QS + a];
+          const float4 ss = *reinterpret_cast<const float4 *>(&sS[a * DV + j]);
+          in.x = fmaf(fq, ss.x, in.x);
+          in.y = fmaf(fq, ss.y, in.y);
+          in.z = fmaf(fq, ss.z, in.z);
+          in.w = fmaf(fq, ss.w, in.w);
+        }
+        const float g = pw[t + 1], inv = 1.f / sDen[t];
+        float4 *gp = reinterpret_cast<float4 *>(&sG[t * DV + j]);
+        const float4 d = *gp;
+        const float y0 = fmaf(g, in.x, num.x) * inv, y1 = fmaf(g, in.y, num.y) * inv;
+        const float y2 = fmaf(g, in.z, num.z) * inv, y3 = fmaf(g, in.w, num.w) * inv;
+        cpart = d.x * y0 + d.y * y1 + d.z * y2 + d.w * y3;
+        *gp = make_float4(d.x * inv, d.y * inv, d.z * inv, d.w * inv);
+      }
+      // the W threads of one token are consecutive lanes of one warp
+#pragma unroll
+      for (int o = W / 2; o > 0; o >>= 1) cpart += __shfl_xor_sync(0xffffffffu, cpart, o, W);
+      if ((i % W) == 0 && t < Cv) {
+        sCc[t] = cpart;
+        sDd[t] = -cpart / sDen[t];
+        stash_put(dk + qo + static_cast<long>(c0 + t) * DK, sDen[t], cpart);
+      }
+    }
+    __syncthreads();
+    scores_b(Cv, with_dlam);
+    __syncthreads();
+    // dphi(q_t) = lambda^(t+1) (S dnum_t + z dden_t) + sum_s B_ts phi(k_s); dq
+    for (int i = tid; i < C * DK; i += NT) {
+      const int t = i / DK, a = i % DK;
+      if (t >= Cv) continue;
+      float gs = sz[a] * sDd[t];
+      for (int j = 0; j < DV; ++j) gs = fmaf(sS[a * DV + j], sG[t * DV + j], gs);
+      float intra = 0.f;
+      for (int s = 0; s <= t; ++s) intra = fmaf(sB[t * AS + s], sK[s * QS + a], intra);
+      const float fq = sQ[t * QS + a];
+      const float dphi = fmaf(pw[t + 1], gs, intra);
+      dq[qo + static_cast<long>(c0 + t) * DK + a] = from_f32<T>(dphi * (fq > 1.f ? 1.f : fq));
+      if (with_dlam) {
+        float gs2 = sz2[a] * sDd[t];
+        for (int j = 0; j < DV; ++j) gs2 = fmaf(sS2[a * DV + j], sG[t * DV + j], gs2);
+        dl = fmaf(fq, fmaf(dpw[t + 1], gs, pw[t + 1] * gs2), dl);
+      }
+    }
+    __syncthreads();
+    // state after the chunk: S' first (it needs the S before the chunk)
+    const float gC = pw[Cv], dgC = dpw[Cv];
+    for (int i = tid; i < DK * DV; i += NT) {
+      const int a = i / DV, j = i % DV;
+      float acc = 0.f, acc2 = 0.f;
+      for (int s = 0; s < Cv; ++s) {
+        const float kv = sK[s * QS + a] * sV[s * DV + j];
+        acc = fmaf(pw[Cv - 1 - s], kv, acc);
+        if (with_dlam) acc2 = fmaf(dpw[Cv - 1 - s], kv, acc2);
+      }
+      if (with_dlam) sS2[i] = fmaf(dgC, sS[i], fmaf(gC, sS2[i], acc2));
+      sS[i] = fmaf(gC, sS[i], acc);
+    }
+    for (int a = tid; a < DK; a += NT) {
+      float acc = 0.f, acc2 = 0.f;
+      for (int s = 0; s < Cv; ++s) {
+        acc = fmaf(pw[Cv - 1 - s], sK[s * QS + a], acc);
+        if (with_dlam) acc2 = fmaf(dpw[Cv - 1 - s], sK[s * QS + a], acc2);
+      }
+      if (with_dlam) sz2[a] = fmaf(dgC, sz[a], fmaf(gC, sz2[a], acc2));
+      sz[a] = fmaf(gC, sz[a], acc);
+    }
+  }
+
+  // ------------------------------------------------------------ sweep 2
+  __syncthreads();
+  for (int i = tid; i < DK * DV; i += NT) sS[i] = 0.f;   // R
+  for (int i = tid; i < DK; i += NT) sz[i] = 0.f;        // r
+  for (int c = nchunks - 1; c >= 0; --c) {
+    const int c0 = c * C, Cv = min(C, N - c0);
+    __syncthreads();
+    load_chunk(c0, Cv);
+    if (tid < Cv) {
+      const float2 st = stash_get(dk + qo + static_cast<long>(c0 + tid) * DK);
+      sDen[tid] = st.x;
+      sDd[tid] = -st.y / st.x;
+    }
+    __syncthreads();
+    for (int i = tid; i < C * DV; i += NT) {   // dnum = dy / den
+      const int t = i / DV;
+      if (t < Cv) sG[i] /= sDen[t];
+    }
+    scores(Cv);
+    __syncthreads();
+    scores_b(Cv, false);
+    __syncthreads();
+    // dphi(k_s) = lambda^(Cv-s) (R v_s + r) + sum_{t>=s} B_ts phi(q_t); dk
+    for (int i = tid; i < C * DK; i += NT) {
+      const int s = i / DK, a = i % DK;
+      if (s >= Cv) continue;
+      float rv = sz[a];
+      for (int j = 0; j < DV; ++j) rv = fmaf(sS[a * DV + j], sV[s * DV + j], rv);
+      float intra = 0.f;
+      for (int t = s; t < Cv; ++t) intra = fmaf(sB[t * AS + s], sQ[t * QS + a], intra);
+      const float fk = sK[s * QS + a];
+      dk[qo + static_cast<long>(c0 + s) * DK + a] =
+          from_f32<T>(fmaf(pw[Cv - s], rv, intra) * (fk > 1.f ? 1.f : fk));
+    }
+    // dv_s = lambda^(Cv-s) R^T phi(k_s) + sum_{t>=s} A_ts dnum_t
+    for (int i = tid; i < C * DV; i += NT) {
+      const int s = i / DV, j = i % DV;
+      if (s >= Cv) continue;
+      float rk = 0.f;
+      for (int a = 0; a < DK; ++a) rk = fmaf(sS[a * DV + j], sK[s * QS + a], rk);
+      float intra = 0.f;
+      for (int t = s; t < Cv; ++t) intra = fmaf(sA[t * AS + s], sG[t * DV + j], intra);
+      dv[vo + static_cast<long>(c0 + s) * DV + j] = from_f32<T>(fmaf(pw[Cv - s], rk, intra));
+    }
+    __syncthreads();
+    // R <- lambda^Cv R + sum_t lambda^t phi(q_t) dnum_t^T;  r likewise with dden
+    const float gC = pw[Cv];
+    for (int i = tid; i < DK * DV; i += NT) {
+      const int a = i / DV, j = i % DV;
+      float acc = 0.f;
+      for (int t = 0; t < Cv; ++t) acc = fmaf(pw[t] * sQ[t * QS + a], sG[t * DV + j], acc);
+      sS[i] = fmaf(gC, sS[i], acc);
+    }
+    for (int a = tid; a < DK; a += NT) {
+      float acc = 0.f;
+      for (int t = 0; t < Cv; ++t) acc = fmaf(pw[t] * sQ[t * QS + a], sDd[t], acc);
+      sz[a] = fmaf(gC, sz[a], acc);
+    }
+  }
+
+  // ------------------------------------------------------------ dlambda
+  if (with_dlam) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) dl += __shfl_xor_sync(0xffffffffu, dl, o);
+    __syncthreads();
+    if ((tid & 31) == 0) sRed[tid >> 5] = dl;
+    __syncthreads();
+    if (tid == 0) {
+      float tot = 0.f;
+      for (int w = 0; w < NT / 32; ++w) tot += sRed[w];
+      atomicAdd(dlam + h, tot);
+    }
+  }
+}
+
+}  // namespace linattn

@@ -18,6 +18,7 @@
 #include "decode.cuh"
 #include "causal_simt.cuh"
 #include "causal_tc.cuh"
+#include "causal_bwd.cuh"
 #include "global_simt.cuh"
 #include "global_tc.cuh"
 
@@ -323,6 +324,47 @@ int global_dispatch(const linattn_dims *d, const void *q, const void *k, const v
   return LINATTN_ERR_UNSUPPORTED;
 }
 
+template <int DK, int DV, typename T>
+int launch_causal_bwd(const linattn_dims *d, const void *q, const void *k, const void *v,
+                      const float *lam, float eps, const void *dy, void *dq, void *dk, void *dv,
+                      float *dlam, cudaStream_t s) {
+  auto *kern = causal_bwd_kernel<DK, DV, T>;
+  // the attribute covers the larger layout (with dlambda) once per kernel and device
+  if (!set_smem(kern, causal_bwd_smem_floats<DK, DV>(true) * 4)) return LINATTN_ERR_CUDA;
+  const int bytes = causal_bwd_smem_floats<DK, DV>(dlam != nullptr) * 4;
+  kern<<<d->B * d->H, kBwdThreads, bytes, s>>>(
+      static_cast<const T *>(q), static_cast<const T *>(k), static_cast<const T *>(v),
+      static_cast<const T *>(dy), lam, eps, static_cast<T *>(dq), static_cast<T *>(dk),
+      static_cast<T *>(dv), dlam, d->H, d->N);
+  return launch_status();
+}
+
+template <int DK, typename T>
+int causal_bwd_dv(const linattn_dims *d, const void *q, const void *k, const void *v,
+                  const float *lam, float eps, const void *dy, void *dq, void *dk, void *dv,
+                  float *dlam, cudaStream_t s) {
+  switch (d->dv) {
+    case 16: return launch_causal_bwd<DK, 16, T>(d, q, k, v, lam, eps, dy, dq, dk, dv, dlam, s);
+    case 32: return launch_causal_bwd<DK, 32, T>(d, q, k, v, lam, eps, dy, dq, dk, dv, dlam, s);
+    case 64: return launch_causal_bwd<DK, 64, T>(d, q, k, v, lam, eps, dy, dq, dk, dv, dlam, s);
+    case 128: return launch_causal_bwd<DK, 128, T>(d, q, k, v, lam, eps, dy, dq, dk, dv, dlam, s);
+  }
+  return LINATTN_ERR_UNSUPPORTED;
+}
+
+template <typename T>
+int causal_bwd_dispatch(const linattn_dims *d, const void *q, const void *k, const void *v,
+                        const float *lam, float eps, const void *dy, void *dq, void *dk, void *dv,
+                        float *dlam, cudaStream_t s) {
+  switch (d->dk) {
+    case 16: return causal_bwd_dv<16, T>(d, q, k, v, lam, eps, dy, dq, dk, dv, dlam, s);
+    case 32: return causal_bwd_dv<32, T>(d, q, k, v, lam, eps, dy, dq, dk, dv, dlam, s);
+    case 64: return causal_bwd_dv<64, T>(d, q, k, v, lam, eps, dy, dq, dk, dv, dlam, s);
+    case 128: return causal_bwd_dv<128, T>(d, q, k, v, lam, eps, dy, dq, dk, dv, dlam, s);
+  }
+  return LINATTN_ERR_UNSUPPORTED;
+}
+
 }  // namespace
 }  // namespace linattn
 
@@ -398,6 +440,41 @@ extern "C" int linattn_fwd_causal_from(const linattn_dims *d, const void *q, con
                                        float *S_final, float *z_final, linattn_stream_t stream) {
   return fwd_causal_impl(d, q, k, v, lambda, eps, S_init, z_init, out, S_final, z_final,
                          reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" int linattn_bwd_causal(const linattn_dims *d, const void *q, const void *k,
+                                  const void *v, const float *lambda, float eps, const void *dy,
+                                  void *dq, void *dk, void *dv, float *dlambda,
+                                  linattn_stream_t stream) {
+  int rc = check_dims(d, true);
+  if (rc != LINATTN_OK) return rc;
+  if (bad_eps(eps)) return LINATTN_ERR_INVALID;
+  const size_t BH = static_cast<size_t>(d->B) * d->H;
+  const size_t es = elem_size(d->dtype);
+  const size_t nq = BH * d->N * d->dk * es, nv = BH * d->N * d->dv * es;
+  const size_t nl = static_cast<size_t>(d->H) * 4;
+  if (BH > 0 && d->N > 0 && (!q || !k || !v || !dy || !dq || !dk || !dv))
+    return LINATTN_ERR_INVALID;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dy) || !aligned16(dq) ||
+      !aligned16(dk) || !aligned16(dv) || !aligned16(lambda) || !aligned16(dlambda))
+    return LINATTN_ERR_INVALID;
+  // every output overlaps no input and no other output
+  const void *in[5] = {q, k, v, dy, lambda};
+  const size_t nin[5] = {nq, nq, nv, nv, nl};
+  const void *outp[4] = {dq, dk, dv, dlambda};
+  const size_t nout[4] = {nq, nq, nv, nl};
+  for (int o = 0; o < 4; ++o) {
+    for (int i = 0; i < 5; ++i)
+      if (overlaps(outp[o], nout[o], in[i], nin[i])) return LINATTN_ERR_INVALID;
+    for (int o2 = o + 1; o2 < 4; ++o2)
+      if (overlaps(outp[o], nout[o], outp[o2], nout[o2])) return LINATTN_ERR_INVALID;
+  }
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (dlambda && cudaMemsetAsync(dlambda, 0, nl, s) != cudaSuccess) return LINATTN_ERR_CUDA;
+  if (BH == 0 || d->N == 0) return LINATTN_OK;
+  if (d->dtype == LINATTN_F32)
+    return causal_bwd_dispatch<float>(d, q, k, v, lambda, eps, dy, dq, dk, dv, dlambda, s);
+  return causal_bwd_dispatch<bf16>(d, q, k, v, lambda, eps, dy, dq, dk, dv, dlambda, s);
 }
 
 extern "C" int linattn_fwd_global(const linattn_dims *d, const void *q, const void *k,

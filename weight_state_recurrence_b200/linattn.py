@@ -26,7 +26,8 @@ LINATTN_ERR_UNSUPPORTED = 2
 LINATTN_ERR_CUDA = 3
 LINATTN_ERR_DEVICE = 4
 
-ENTRY_POINTS = ("linattn_fwd_causal", "linattn_fwd_causal_from", "linattn_fwd_global", "linattn_decode_step",
+ENTRY_POINTS = ("linattn_fwd_causal", "linattn_fwd_causal_from", "linattn_bwd_causal",
+                "linattn_fwd_global", "linattn_decode_step",
                 "linattn_status_string", "linattn_device_status", "linattn_version")
 
 
@@ -66,6 +67,8 @@ def load(build_if_missing: bool = True):
     lib.linattn_fwd_causal.restype = i
     lib.linattn_fwd_causal_from.argtypes = [dp, vp, vp, vp, fp, f, fp, fp, vp, fp, fp, vp]
     lib.linattn_fwd_causal_from.restype = i
+    lib.linattn_bwd_causal.argtypes = [dp, vp, vp, vp, fp, f, vp, vp, vp, vp, fp, vp]
+    lib.linattn_bwd_causal.restype = i
     lib.linattn_fwd_global.argtypes = [dp, vp, vp, vp, f, vp, fp, fp, vp]
     lib.linattn_fwd_global.restype = i
     lib.linattn_decode_step.argtypes = [dp, vp, vp, vp, fp, f, fp, fp, vp, vp]
@@ -160,6 +163,24 @@ def linattn_fwd_causal_from(q, k, v, lam, eps, S_init, z_init, out, S_final=None
            "linattn_fwd_causal_from")
 
 
+def linattn_bwd_causal(q, k, v, lam, eps, dy, dq, dk, dv, dlam=None, stream=None):
+    """Backward of the causal forward: dy like v; dq, dk like q; dv like v;
+    dlam [H] fp32 or None."""
+    B, H, N, dk_ = q.shape
+    dv_ = v.shape[-1]
+    if (k.shape != q.shape or tuple(v.shape) != (B, H, N, dv_) or dy.shape != v.shape or
+            dq.shape != q.shape or dk.shape != q.shape or dv.shape != v.shape):
+        raise ValueError("shape mismatch among q, k, v, dy, dq, dk, dv")
+    if len({t.dtype for t in (q, k, v, dy, dq, dk, dv)}) != 1:
+        raise ValueError("q, k, v, dy, dq, dk, dv must share one dtype")
+    _f32(lam, (H,), "lambda")
+    _f32(dlam, (H,), "dlambda")
+    d = linattn_dims(B, H, N, dk_, dv_, _dtype_code(q.dtype))
+    _check(load().linattn_bwd_causal(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), _ptr(lam),
+                                     float(eps), _ptr(dy), _ptr(dq), _ptr(dk), _ptr(dv),
+                                     _ptr(dlam), _stream(stream)), "linattn_bwd_causal")
+
+
 def linattn_fwd_global(q, k, v, eps, out, KV, ksum, stream=None):
     """Global forward: q, k [B,H,N,dk], v/out [B,H,N,dv]; KV [B,H,dk,dv] and
     ksum [B,H,dk] fp32 are written."""
@@ -220,6 +241,13 @@ def fwd_causal(q, k, v, lam=None, eps=1e-6, want_state=True, S_init=None, z_init
     else:
         linattn_fwd_causal_from(q, k, v, lam, eps, S_init, z_init, out, S, z, stream)
     return out, S, z
+
+
+def bwd_causal(q, k, v, dy, lam=None, eps=1e-6, want_dlam=False, stream=None):
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    dlam = (torch.empty(q.shape[1], dtype=torch.float32, device=q.device) if want_dlam else None)
+    linattn_bwd_causal(q, k, v, lam, eps, dy, dq, dk, dv, dlam, stream)
+    return dq, dk, dv, dlam
 
 
 def fwd_global(q, k, v, eps=1e-6, stream=None):
