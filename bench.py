@@ -45,6 +45,11 @@ WL_DEC = inputs.WORKLOADS["decode_d128"]
 WL_GLB = inputs.WORKLOADS["global_d64"]
 
 
+# fp32 FMA peak of the CUDA cores: 148 SMs x 128 FMA lanes x 2 flops x 1.965 GHz
+# (the nominal maximum SM clock), for kernels bound by plain ALU arithmetic
+ALU_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
 def peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -356,6 +361,54 @@ def global_leg(lib, args, world, rank, stream, hbm):
     return res
 
 
+def bwd_flops(B, H, N, dk, dv, with_dlam=True):
+    """fp32 FMA work of the backward kernel as written, 2 flops each: per
+    chunk of C = 32 tokens and head, both sweeps' score tiles (lower
+    triangle), the per-token forward rebuild, dphi(q), dphi(k), dv and the
+    state / reverse-state updates (plus S' and its use for dlambda)."""
+    C = 32
+    tri = C * (C + 1) / 2
+    per_chunk = (2 * tri * dk + 2 * tri * dv + C * (tri / C + dk) + C * dv * (tri / C + dk) +
+                 C * dk * (dv + tri / C) * 2 + C * dv * (dk + tri / C) + 2 * dk * dv * C)
+    if with_dlam:
+        per_chunk += C * dk * dv + dk * dv * C
+    return 2 * per_chunk * B * H * N / C
+
+
+def bwd_leg(lib, args, world, rank, stream, alu_peak):
+    """Backward (dq, dk, dv, dlambda) of the causal forward on the
+    causal_decay_d128 workload, a few steps (CUDA cores, fp32 arithmetic)."""
+    B, H, N, d = args.batch or WL.B, WL.H, WL.N, WL.d
+    dev = torch.device("cuda")
+    q, k, v = inputs.qkv((B, H, N, d), (B, H, N, d), WL.seed * 1000 + rank, WL.scale,
+                         WL.dtype, device=dev)
+    g = torch.Generator(device=dev)
+    g.manual_seed(WL.seed * 1000 + 500 + rank)
+    dy = torch.randn(B, H, N, d, generator=g, device=dev).to(WL.dtype)
+    lam = inputs.decay(WL).to(dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    dl = torch.empty(H, device=dev)
+
+    def step():
+        lib.linattn_bwd_causal(q, k, v, lam, WL.eps, dy, dq, dk, dv, dl, stream)
+
+    steps = max(1, min(args.steps, 3))
+    with torch.cuda.stream(stream):
+        ms = time_steps(step, steps, args.warmup, world, stream)
+    assert lib.linattn_device_status(clear=True, stream=stream) == 0
+    per = ms / 1e3 / steps
+    fl = bwd_flops(B, H, N, d, d)
+    res = {"value": B * N * world / per, "unit": "tokens/s", "ms_per_step": per * 1e3,
+           "steps": steps, "ctas": B * H,
+           "roofline": {"bound": "alu", "achieved": fl / per / 1e12, "peak": alu_peak,
+                        "unit": "TFLOP/s", "frac": fl / per / 1e12 / alu_peak,
+                        "flops_per_launch": fl, "kernel": "causal_bwd_kernel",
+                        "traffic": None}}
+    del q, k, v, dy, dq, dk, dv
+    torch.cuda.empty_cache()
+    return res
+
+
 # ---------------------------------------------------------------- oracle
 def oracle_sample(target_s=12.0, heads=None):
     """Times the fp64 oracle (as it stands) on a bounded sample of the causal
@@ -420,7 +473,8 @@ def main():
     ap.add_argument("--no-e2e", dest="e2e", action="store_false")
     ap.add_argument("--no-legs", dest="legs", action="store_false")
     ap.add_argument("--no-cpu-baseline", dest="cpu", action="store_false")
-    ap.add_argument("--only", default="all", choices=["all", "causal", "decode", "global"])
+    ap.add_argument("--only", default="all",
+                    choices=["all", "causal", "decode", "global", "backward"])
     ap.add_argument("--batch", type=int, default=0, help="causal leg batch (profiling)")
     ap.add_argument("--dec-batch", type=int, default=0, help="decode sequences (profiling)")
     ap.add_argument("--dec-steps", type=int, default=0, help="decode steps (profiling)")
@@ -436,10 +490,13 @@ def main():
     hbm, tcp, peak_src = peaks()
     stream = torch.cuda.Stream()
 
-    if args.only in ("decode", "global"):
-        leg = decode_leg if args.only == "decode" else global_leg
-        line = {"metric": METRIC, "leg": args.only, "n_gpus": world,
-                args.only: leg(lib, args, world, rank, stream, hbm)}
+    if args.only in ("decode", "global", "backward"):
+        if args.only == "backward":
+            r = bwd_leg(lib, args, world, rank, stream, ALU_PEAK_TFLOPS)
+        else:
+            leg = decode_leg if args.only == "decode" else global_leg
+            r = leg(lib, args, world, rank, stream, hbm)
+        line = {"metric": METRIC, "leg": args.only, "n_gpus": world, args.only: r}
         if rank == 0:
             print(json.dumps(line), flush=True)
         return 0
@@ -464,6 +521,7 @@ def main():
     if args.legs and args.only == "all":
         line["decode"] = decode_leg(lib, args, world, rank, stream, hbm)
         line["global"] = global_leg(lib, args, world, rank, stream, hbm)
+        line["backward"] = bwd_leg(lib, args, world, rank, stream, ALU_PEAK_TFLOPS)
     if args.cpu and world == 1 and rank == 0:
         tok_s, cores, desc, _ = oracle_sample()
         line["cpu_baseline"] = {"value": tok_s, "unit": "tokens/s", "cores": cores,
