@@ -32,8 +32,8 @@ constexpr int kBwdThreads = 256;
 template <int DK, int DV>
 constexpr int causal_bwd_smem_floats(bool with_dlam) {
   constexpr int C = kBwdChunk;
-  return 2 * C * (DK + 1) + 2 * C * DV + 3 * C * (C + 1) + DK * DV + DK +
-         (with_dlam ? DK * DV + DK : 0) + 4 * C + 2 * (C + 4) + 8;
+  return 2 * C * (DK + 1) + C * (DV + 1) + C * DV + 3 * C * (C + 1) + DK * (DV + 1) + DK +
+         (with_dlam ? DK * (DV + 1) + DK : 0) + 4 * C + 2 * (C + 4) + 8;
 }
 
 // the two fp32 numbers a token keeps between the sweeps, in the first 8 bytes of its dk row
@@ -52,22 +52,25 @@ __global__ void __launch_bounds__(kBwdThreads) causal_bwd_kernel(
     const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
     const T *__restrict__ dy, const float *__restrict__ lam, float eps, T *__restrict__ dq,
     T *__restrict__ dk, T *__restrict__ dv, float *__restrict__ dlam, int H, int N) {
-  constexpr int C = kBwdChunk, NT = kBwdThreads, QS = DK + 1, AS = C + 1;
+  // rows of phi(q), phi(k), v and of the states are padded by one float so that
+  // lanes walking different rows at the same column hit different banks
+  constexpr int C = kBwdChunk, NT = kBwdThreads, QS = DK + 1, AS = C + 1, VS = DV + 1,
+                SS = DV + 1;
   constexpr int W = DV / 4;   // threads that share one token in the per-column phases
   static_assert(DV % 4 == 0 && W <= 32 && (32 % W) == 0, "dv must be 16..128");
   extern __shared__ __align__(16) float sm[];
   const bool with_dlam = dlam != nullptr;
   float *sQ = sm;                  // [C][DK+1]  phi(q)
   float *sK = sQ + C * QS;         // [C][DK+1]  phi(k)
-  float *sV = sK + C * QS;         // [C][DV]    v
-  float *sG = sV + C * DV;         // [C][DV]    dy, then dnum
+  float *sV = sK + C * QS;         // [C][DV+1]  v
+  float *sG = sV + C * VS;         // [C][DV]    dy, then dnum
   float *sA = sG + C * DV;         // [C][C+1]   lambda^(t-s) phi(q_t).phi(k_s), s <= t
   float *sB = sA + C * AS;         // [C][C+1]   lambda^(t-s) (dnum_t.v_s + dden_t), s <= t
   float *sP = sB + C * AS;         // [C][C+1]   phi(q_t).phi(k_s) (for dlambda)
-  float *sS = sP + C * AS;         // [DK][DV]   S (sweep 1) / R (sweep 2)
-  float *sz = sS + DK * DV;        // [DK]       z / r
-  float *sS2 = sz + DK;            // [DK][DV]   S' (dlambda only)
-  float *sz2 = sS2 + (with_dlam ? DK * DV : 0);   // [DK] z'
+  float *sS = sP + C * AS;         // [DK][DV+1] S (sweep 1) / R (sweep 2)
+  float *sz = sS + DK * SS;        // [DK]       z / r
+  float *sS2 = sz + DK;            // [DK][DV+1] S' (dlambda only)
+  float *sz2 = sS2 + (with_dlam ? DK * SS : 0);   // [DK] z'
   float *sDen = sz2 + (with_dlam ? DK : 0);       // [C] den_t
   float *sCc = sDen + C;           // [C] c_t = dy_t . y_t
   float *sDd = sCc + C;            // [C] dden_t
@@ -82,7 +85,7 @@ __global__ void __launch_bounds__(kBwdThreads) causal_bwd_kernel(
   if (tid < C + 4) pw[tid] = pow_int(L, tid);
   __syncthreads();
   if (tid < C + 4) dpw[tid] = tid == 0 ? 0.f : static_cast<float>(tid) * pw[tid - 1];
-  for (int i = tid; i < DK * DV; i += NT) {
+  for (int i = tid; i < DK * SS; i += NT) {
     sS[i] = 0.f;
     if (with_dlam) sS2[i] = 0.f;
   }
@@ -109,7 +112,7 @@ __global__ void __launch_bounds__(kBwdThreads) causal_bwd_kernel(
     for (int i = tid; i < C * DV; i += NT) {
       const int t = i / DV, j = i % DV;
       const long o = vo + static_cast<long>(c0 + t) * DV + j;
-      sV[i] = t < Cv ? to_f32(v[o]) : 0.f;
+      sV[t * VS + j] = t < Cv ? to_f32(v[o]) : 0.f;
       sG[i] = t < Cv ? to_f32(dy[o]) : 0.f;
     }
   };
@@ -135,7 +138,7 @@ __global__ void __launch_bounds__(kBwdThreads) causal_bwd_kernel(
       if (s <= t && t < Cv) {
         float e = sDd[t];
 #pragma unroll 8
-        for (int j = 0; j < DV; ++j) e = fmaf(sG[t * DV + j], sV[s * DV + j], e);
+        for (int j = 0; j < DV; ++j) e = fmaf(sG[t * DV + j], sV[s * VS + j], e);
         b = pw[t - s] * e;
         if (add_dlam) dl = fmaf(dpw[t - s] * sP[t * AS + s], e, dl);
       }
@@ -159,41 +162,36 @@ __global__ void __launch_bounds__(kBwdThreads) causal_bwd_kernel(
       sDen[tid] = rs + pw[tid + 1] * qz + eps;
     }
     __syncthreads();
-    // num_t, y_t = num/den, dnum_t = dy_t/den in place, c_t = dy_t . y_t
+    // num_t, y_t = num/den, dnum_t = dy_t/den in place, c_t = dy_t . y_t; the W
+    // threads of a token take columns jj + W m (m = 0..3): consecutive lanes,
+    // consecutive columns
     for (int i = tid; i < C * W; i += NT) {
-      const int t = i / W, j = 4 * (i % W);
+      const int t = i / W, jj = i % W;
       float cpart = 0.f;
       if (t < Cv) {
-        float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
+        float num[4] = {0.f, 0.f, 0.f, 0.f}, in[4] = {0.f, 0.f, 0.f, 0.f};
         for (int s = 0; s <= t; ++s) {
           const float a = sA[t * AS + s];
-          const float4 vv = *reinterpret_cast<const float4 *>(&sV[s * DV + j]);
-          num.x = fmaf(a, vv.x, num.x);
-          num.y = fmaf(a, vv.y, num.y);
-          num.z = fmaf(a, vv.z, num.z);
-          num.w = fmaf(a, vv.w, num.w);
+#pragma unroll
+          for (int m = 0; m < 4; ++m) num[m] = fmaf(a, sV[s * VS + jj + W * m], num[m]);
         }
-        float4 in = make_float4(0.f, 0.f, 0.f, 0.f);
         for (int a = 0; a < DK; ++a) {
           const float fq = sQ[t * QS + a];
-          const float4 ss = *reinterpret_cast<const float4 *>(&sS[a * DV + j]);
-          in.x = fmaf(fq, ss.x, in.x);
-          in.y = fmaf(fq, ss.y, in.y);
-          in.z = fmaf(fq, ss.z, in.z);
-          in.w = fmaf(fq, ss.w, in.w);
+#pragma unroll
+          for (int m = 0; m < 4; ++m) in[m] = fmaf(fq, sS[a * SS + jj + W * m], in[m]);
         }
         const float g = pw[t + 1], inv = 1.f / sDen[t];
-        float4 *gp = reinterpret_cast<float4 *>(&sG[t * DV + j]);
-        const float4 d = *gp;
-        const float y0 = fmaf(g, in.x, num.x) * inv, y1 = fmaf(g, in.y, num.y) * inv;
-        const float y2 = fmaf(g, in.z, num.z) * inv, y3 = fmaf(g, in.w, num.w) * inv;
-        cpart = d.x * y0 + d.y * y1 + d.z * y2 + d.w * y3;
-        *gp = make_float4(d.x * inv, d.y * inv, d.z * inv, d.w * inv);
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          const float d = sG[t * DV + jj + W * m];
+          cpart = fmaf(d, fmaf(g, in[m], num[m]) * inv, cpart);
+          sG[t * DV + jj + W * m] = d * inv;
+        }
       }
       // the W threads of one token are consecutive lanes of one warp
 #pragma unroll
       for (int o = W / 2; o > 0; o >>= 1) cpart += __shfl_xor_sync(0xffffffffu, cpart, o, W);
-      if ((i % W) == 0 && t < Cv) {
+      if (jj == 0 && t < Cv) {
         sCc[t] = cpart;
         sDd[t] = -cpart / sDen[t];
         stash_put(dk + qo + static_cast<long>(c0 + t) * DK, sDen[t], cpart);
@@ -207,7 +205,7 @@ __global__ void __launch_bounds__(kBwdThreads) causal_bwd_kernel(
       const int t = i / DK, a = i % DK;
       if (t >= Cv) continue;
       float gs = sz[a] * sDd[t];
-      for (int j = 0; j < DV; ++j) gs = fmaf(sS[a * DV + j], sG[t * DV + j], gs);
+      for (int j = 0; j < DV; ++j) gs = fmaf(sS[a * SS + j], sG[t * DV + j], gs);
       float intra = 0.f;
       for (int s = 0; s <= t; ++s) intra = fmaf(sB[t * AS + s], sK[s * QS + a], intra);
       const float fq = sQ[t * QS + a];
@@ -215,7 +213,7 @@ __global__ void __launch_bounds__(kBwdThreads) causal_bwd_kernel(
       dq[qo + static_cast<long>(c0 + t) * DK + a] = from_f32<T>(dphi * (fq > 1.f ? 1.f : fq));
       if (with_dlam) {
         float gs2 = sz2[a] * sDd[t];
-        for (int j = 0; j < DV; ++j) gs2 = fmaf(sS2[a * DV + j], sG[t * DV + j], gs2);
+        for (int j = 0; j < DV; ++j) gs2 = fmaf(sS2[a * SS + j], sG[t * DV + j], gs2);
         dl = fmaf(fq, fmaf(dpw[t + 1], gs, pw[t + 1] * gs2), dl);
       }
     }
@@ -223,15 +221,15 @@ __global__ void __launch_bounds__(kBwdThreads) causal_bwd_kernel(
     // state after the chunk: S' first (it needs the S before the chunk)
     const float gC = pw[Cv], dgC = dpw[Cv];
     for (int i = tid; i < DK * DV; i += NT) {
-      const int a = i / DV, j = i % DV;
+      const int a = i / DV, j = i % DV, o = a * SS + j;
       float acc = 0.f, acc2 = 0.f;
       for (int s = 0; s < Cv; ++s) {
-        const float kv = sK[s * QS + a] * sV[s * DV + j];
+        const float kv = sK[s * QS + a] * sV[s * VS + j];
         acc = fmaf(pw[Cv - 1 - s], kv, acc);
         if (with_dlam) acc2 = fmaf(dpw[Cv - 1 - s], kv, acc2);
       }
-      if (with_dlam) sS2[i] = fmaf(dgC, sS[i], fmaf(gC, sS2[i], acc2));
-      sS[i] = fmaf(gC, sS[i], acc);
+      if (with_dlam) sS2[o] = fmaf(dgC, sS[o], fmaf(gC, sS2[o], acc2));
+      sS[o] = fmaf(gC, sS[o], acc);
     }
     for (int a = tid; a < DK; a += NT) {
       float acc = 0.f, acc2 = 0.f;
@@ -246,7 +244,7 @@ __global__ void __launch_bounds__(kBwdThreads) causal_bwd_kernel(
 
   // ------------------------------------------------------------ sweep 2
   __syncthreads();
-  for (int i = tid; i < DK * DV; i += NT) sS[i] = 0.f;   // R
+  for (int i = tid; i < DK * SS; i += NT) sS[i] = 0.f;   // R
   for (int i = tid; i < DK; i += NT) sz[i] = 0.f;        // r
   for (int c = nchunks - 1; c >= 0; --c) {
     const int c0 = c * C, Cv = min(C, N - c0);
@@ -271,7 +269,7 @@ __global__ void __launch_bounds__(kBwdThreads) causal_bwd_kernel(
       const int s = i / DK, a = i % DK;
       if (s >= Cv) continue;
       float rv = sz[a];
-      for (int j = 0; j < DV; ++j) rv = fmaf(sS[a * DV + j], sV[s * DV + j], rv);
+      for (int j = 0; j < DV; ++j) rv = fmaf(sS[a * SS + j], sV[s * VS + j], rv);
       float intra = 0.f;
       for (int t = s; t < Cv; ++t) intra = fmaf(sB[t * AS + s], sQ[t * QS + a], intra);
       const float fk = sK[s * QS + a];
@@ -283,7 +281,7 @@ __global__ void __launch_bounds__(kBwdThreads) causal_bwd_kernel(
       const int s = i / DV, j = i % DV;
       if (s >= Cv) continue;
       float rk = 0.f;
-      for (int a = 0; a < DK; ++a) rk = fmaf(sS[a * DV + j], sK[s * QS + a], rk);
+      for (int a = 0; a < DK; ++a) rk = fmaf(sS[a * SS + j], sK[s * QS + a], rk);
       float intra = 0.f;
       for (int t = s; t < Cv; ++t) intra = fmaf(sA[t * AS + s], sG[t * DV + j], intra);
       dv[vo + static_cast<long>(c0 + s) * DV + j] = from_f32<T>(fmaf(pw[Cv - s], rk, intra));
@@ -292,10 +290,10 @@ __global__ void __launch_bounds__(kBwdThreads) causal_bwd_kernel(
     // R <- lambda^Cv R + sum_t lambda^t phi(q_t) dnum_t^T;  r likewise with dden
     const float gC = pw[Cv];
     for (int i = tid; i < DK * DV; i += NT) {
-      const int a = i / DV, j = i % DV;
+      const int a = i / DV, j = i % DV, o = a * SS + j;
       float acc = 0.f;
       for (int t = 0; t < Cv; ++t) acc = fmaf(pw[t] * sQ[t * QS + a], sG[t * DV + j], acc);
-      sS[i] = fmaf(gC, sS[i], acc);
+      sS[o] = fmaf(gC, sS[o], acc);
     }
     for (int a = tid; a < DK; a += NT) {
       float acc = 0.f;
