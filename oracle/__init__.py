@@ -52,6 +52,8 @@ def _load():
         lib.oracle_decode_step.restype = i
         lib.oracle_global.argtypes = [i, i, i, i, i, _dp, _dp, _dp, d, _dp, _dp, _dp, i]
         lib.oracle_global.restype = i
+        lib.oracle_global_cross.argtypes = [i, i, i, i, i, i, _dp, _dp, _dp, d, _dp, _dp, _dp, i]
+        lib.oracle_global_cross.restype = i
         lib.oracle_feature_map.argtypes = [ctypes.c_long, _dp, _dp]
         lib.oracle_feature_map.restype = None
         lib.oracle_num_threads.argtypes = [i]
@@ -131,6 +133,22 @@ def decode_step(q, k, v, S, z, lam=None, eps=1e-6, nthreads=0):
     if rc != 0:
         raise ValueError("oracle_decode_step rejected its arguments")
     return y, S, z
+
+
+def global_cross(q, k, v, eps=1e-6, nthreads=0):
+    """Cross form: q ``[B,H,Nq,dk]`` attends to k ``[B,H,Nk,dk]``, v ``[B,H,Nk,dv]``.
+    Returns ``(y [B,H,Nq,dv], KV [B,H,dk,dv], ks [B,H,dk])``."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, H, Nq, dk = q.shape
+    Nk, dv = k.shape[2], v.shape[-1]
+    y = np.empty((B, H, Nq, dv))
+    KV = np.empty((B, H, dk, dv))
+    ks = np.empty((B, H, dk))
+    rc = _load().oracle_global_cross(B, H, Nq, Nk, dk, dv, _ptr(q), _ptr(k), _ptr(v),
+                                     float(eps), _ptr(y), _ptr(KV), _ptr(ks), int(nthreads))
+    if rc != 0:
+        raise ValueError("oracle_global_cross rejected its arguments")
+    return y, KV, ks
 
 
 def global_attn(q, k, v, eps=1e-6, nthreads=0):

@@ -195,7 +195,7 @@ int oracle_decode_step(int B, int H, int dk, int dv,
  *     y_i = phi(q_i)^T KV / (phi(q_i)^T ks + eps)
  * Every query sees every key; there is no decay (the sum has no order). */
 typedef struct {
-    int N, dk, dv;
+    int Nq, Nk, dk, dv;
     const double *q, *k, *v;
     double eps;
     double *y, *KV, *ks;
@@ -203,15 +203,15 @@ typedef struct {
 
 static void global_pair(void *vctx, long pair) {
     const global_ctx *c = (const global_ctx *)vctx;
-    const int N = c->N, dk = c->dk, dv = c->dv;
-    const double *q = c->q + (size_t)pair * N * dk;
-    const double *k = c->k + (size_t)pair * N * dk;
-    const double *v = c->v + (size_t)pair * N * dv;
+    const int Nq = c->Nq, Nk = c->Nk, dk = c->dk, dv = c->dv;
+    const double *q = c->q + (size_t)pair * Nq * dk;
+    const double *k = c->k + (size_t)pair * Nk * dk;
+    const double *v = c->v + (size_t)pair * Nk * dv;
     double *KV = (double *)calloc((size_t)dk * dv, sizeof(double));
     double *ks = (double *)calloc((size_t)dk, sizeof(double));
     double *f = (double *)malloc(sizeof(double) * dk);
 
-    for (int n = 0; n < N; ++n) {
+    for (int n = 0; n < Nk; ++n) {
         const double *kn = k + (size_t)n * dk;
         const double *vn = v + (size_t)n * dv;
         for (int a = 0; a < dk; ++a) f[a] = phi(kn[a]);
@@ -221,13 +221,13 @@ static void global_pair(void *vctx, long pair) {
         }
     }
     if (c->y) {
-        for (int i = 0; i < N; ++i) {
+        for (int i = 0; i < Nq; ++i) {
             const double *qi = q + (size_t)i * dk;
             for (int a = 0; a < dk; ++a) f[a] = phi(qi[a]);
             double den = 0.0;
             for (int a = 0; a < dk; ++a) den += f[a] * ks[a];
             den += c->eps;
-            double *yi = c->y + ((size_t)pair * N + i) * dv;
+            double *yi = c->y + ((size_t)pair * Nq + i) * dv;
             for (int b = 0; b < dv; ++b) {
                 double num = 0.0;
                 for (int a = 0; a < dk; ++a) num += f[a] * KV[(size_t)a * dv + b];
@@ -242,14 +242,23 @@ static void global_pair(void *vctx, long pair) {
     free(KV);
 }
 
+/* Cross form: Nq queries attend to Nk keys/values of another sequence
+ * (the linear-attention note's multi-head module, §6, takes target and source
+ * lengths); Nq = Nk = N is the self form above. */
+int oracle_global_cross(int B, int H, int Nq, int Nk, int dk, int dv,
+                        const double *q, const double *k, const double *v, double eps,
+                        double *y, double *KV, double *ks, int nthreads) {
+    if (B < 0 || H < 0 || Nq < 0 || Nk < 0 || dk <= 0 || dv <= 0) return -1;
+    if ((Nq > 0 && !q) || (Nk > 0 && (!k || !v))) return -1;
+    global_ctx c = {Nq, Nk, dk, dv, q, k, v, eps, y, KV, ks};
+    for_each_pair((long)B * H, nthreads, global_pair, &c);
+    return 0;
+}
+
 int oracle_global(int B, int H, int N, int dk, int dv,
                   const double *q, const double *k, const double *v, double eps,
                   double *y, double *KV, double *ks, int nthreads) {
-    if (B < 0 || H < 0 || N < 0 || dk <= 0 || dv <= 0) return -1;
-    if (N > 0 && (!q || !k || !v)) return -1;
-    global_ctx c = {N, dk, dv, q, k, v, eps, y, KV, ks};
-    for_each_pair((long)B * H, nthreads, global_pair, &c);
-    return 0;
+    return oracle_global_cross(B, H, N, N, dk, dv, q, k, v, eps, y, KV, ks, nthreads);
 }
 
 int oracle_num_threads(int nthreads) { return resolve_threads(nthreads); }

@@ -177,6 +177,25 @@ def test_global_closed_form_and_reorder():
             assert rel(ks[b, h], fk.sum(0)) < 1e-12
 
 
+def test_global_cross_brute_force():
+    """Nq queries against Nk keys of another sequence: the double sum
+    y_i = sum_j (phi(q_i).phi(k_j)) v_j / (sum_j phi(q_i).phi(k_j) + eps), and
+    Nq = Nk reduces to the self form."""
+    q, _, _ = rand(21, 2, 3, 7, 5, 4)
+    _, k, v = rand(22, 2, 3, 11, 5, 4)
+    eps = 1e-3
+    y, KV, ks = oracle.global_cross(q, k, v, eps)
+    fq, fk = phi_np(q), phi_np(k)
+    w = np.einsum("bhid,bhjd->bhij", fq, fk)
+    assert rel(y, np.einsum("bhij,bhjv->bhiv", w, v) / (w.sum(-1, keepdims=True) + eps)) < 1e-13
+    assert rel(KV, np.einsum("bhjd,bhjv->bhdv", fk, v)) < 1e-13 and rel(ks, fk.sum(2)) < 1e-13
+    y2, _, _ = oracle.global_cross(q, q, v[:, :, :7], eps)
+    y3, _, _ = oracle.global_attn(q, q, v[:, :, :7], eps)
+    assert np.array_equal(y2, y3)
+    y0, KV0, ks0 = oracle.global_cross(q, k[:, :, :0], v[:, :, :0], eps)
+    assert not y0.any() and not KV0.any() and not ks0.any()
+
+
 def test_causal_last_token_equals_global_without_decay():
     q, k, v = rand(5, 1, 3, 40, 8, 8)
     y, S, z = oracle.causal(q, k, v, None, eps=1e-6)
