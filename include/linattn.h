@@ -153,6 +153,20 @@ LINATTN_API int linattn_fwd_global(const linattn_dims *dims, const void *q, cons
                        linattn_stream_t stream);
 
 /*
+ * Cross form of the global forward: the d->N queries of one sequence attend
+ * to the Nk keys / values of another ([LN] §6: the multi-head module's target
+ * and source lengths; §3 with the sums over the source):
+ *   KV = sum_{n<Nk} phi(k_n) v_n^T,  ksum = sum_{n<Nk} phi(k_n),
+ *   y_i = phi(q_i)^T KV / (phi(q_i)^T ksum + eps),   i < d->N.
+ *   q [B, H, d->N, dk], out [B, H, d->N, dv], k [B, H, Nk, dk], v [B, H, Nk, dv]
+ *   dtype; KV, ksum as linattn_fwd_global (written).  Nk = 0 gives KV = 0,
+ *   ksum = 0 and y = 0.  linattn_fwd_global is this call with Nk = d->N.
+ */
+LINATTN_API int linattn_fwd_global_cross(const linattn_dims *dims, int Nk, const void *q,
+                       const void *k, const void *v, float eps, void *out, float *KV,
+                       float *ksum, linattn_stream_t stream);
+
+/*
  * One decode step for every (b, h) ([FW] §4.1 forward_step, §3.1 constant
  * d x d cache; [LN] §5 O(1) per token, §6 forward_autoregressive):
  *   S <- lambda S + phi(k) v^T;  z <- lambda z + phi(k);

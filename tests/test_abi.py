@@ -124,6 +124,19 @@ def test_bwd_rejects_bad_arguments(lib):
     assert bw(dl=MIS) == linattn.LINATTN_ERR_INVALID
 
 
+def test_global_cross_rejects_bad_arguments(lib):
+    KV, ks = P(0x7F0000500000), P(0x7F0000600000)
+    gc = lambda **kw: lib.linattn_fwd_global_cross(
+        ctypes.byref(kw.get("d", D())), kw.get("nk", 8), FAKE, FAKE2, FAKE3, 1e-6,
+        kw.get("out", FAKE4), kw.get("KV", KV), kw.get("ks", ks), None)
+    assert gc(nk=-1) == linattn.LINATTN_ERR_INVALID
+    assert gc(KV=None) == linattn.LINATTN_ERR_INVALID
+    assert gc(out=FAKE2) == linattn.LINATTN_ERR_INVALID      # output over the keys
+    assert gc(KV=FAKE) == linattn.LINATTN_ERR_INVALID        # KV over the queries
+    assert gc(nk=1 << 30) == linattn.LINATTN_ERR_UNSUPPORTED
+    assert gc(d=D(dk=20)) == linattn.LINATTN_ERR_UNSUPPORTED
+
+
 def test_empty_batch_is_a_no_op(lib):
     # B*H == 0: nothing to do, nothing launched, even with NULL buffers
     assert causal(lib, D(B=0), q=None, k=None, v=None, out=None) == linattn.LINATTN_OK

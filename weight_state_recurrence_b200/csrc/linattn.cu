@@ -253,19 +253,25 @@ int launch_causal_tc(const linattn_dims *d, const void *q, const void *k, const 
 }
 
 template <int DK, int DV, typename T>
-int launch_global_simt(const linattn_dims *d, const void *q, const void *k, const void *v,
-                       float eps, void *out, float *KV, float *ksum, cudaStream_t s) {
+int launch_global_simt(const linattn_dims *d, int Nk, const void *q, const void *k,
+                       const void *v, float eps, void *out, float *KV, float *ksum,
+                       cudaStream_t s) {
+  // KV, ksum over the Nk keys (none: they stay zero), then y for the d->N queries
   const int BH = d->B * d->H;
-  dim3 g1(BH, (d->N + kGlobalSplit - 1) / kGlobalSplit);
-  global_kv_simt_kernel<DK, DV, T><<<g1, 256, 0, s>>>(
-      static_cast<const T *>(k), static_cast<const T *>(v), KV, ksum, d->N);
-  if (cudaGetLastError() != cudaSuccess) return LINATTN_ERR_CUDA;
-  auto *kern = global_out_simt_kernel<DK, DV, T>;
-  const int bytes = (DK * DV + DK + kGlobalTile * (DK + 1) + kGlobalTile) * 4;
-  if (!set_smem(kern, bytes)) return LINATTN_ERR_CUDA;
-  dim3 g2(BH, (d->N + kGlobalTile - 1) / kGlobalTile);
-  kern<<<g2, 256, bytes, s>>>(static_cast<const T *>(q), KV, ksum, eps, static_cast<T *>(out),
-                              d->N);
+  if (Nk > 0) {
+    dim3 g1(BH, (Nk + kGlobalSplit - 1) / kGlobalSplit);
+    global_kv_simt_kernel<DK, DV, T><<<g1, 256, 0, s>>>(
+        static_cast<const T *>(k), static_cast<const T *>(v), KV, ksum, Nk);
+    if (cudaGetLastError() != cudaSuccess) return LINATTN_ERR_CUDA;
+  }
+  if (d->N > 0) {
+    auto *kern = global_out_simt_kernel<DK, DV, T>;
+    const int bytes = (DK * DV + DK + kGlobalTile * (DK + 1) + kGlobalTile) * 4;
+    if (!set_smem(kern, bytes)) return LINATTN_ERR_CUDA;
+    dim3 g2(BH, (d->N + kGlobalTile - 1) / kGlobalTile);
+    kern<<<g2, 256, bytes, s>>>(static_cast<const T *>(q), KV, ksum, eps,
+                                static_cast<T *>(out), d->N);
+  }
   return launch_status();
 }
 
@@ -278,48 +284,56 @@ bool use_tc_global(const linattn_dims *d) {
   return d->dtype == LINATTN_BF16 && d->dk == gtc::D && d->dv == gtc::D && d->H % 2 == 0;
 }
 
-int launch_global_tc(const linattn_dims *d, const void *q, const void *k, const void *v, float eps,
-                     void *out, float *KV, float *ksum, cudaStream_t s) {
+int launch_global_tc(const linattn_dims *d, int Nk, const void *q, const void *k,
+                     const void *v, float eps, void *out, float *KV, float *ksum,
+                     cudaStream_t s) {
+  // KV, ksum over the Nk keys (none: they stay zero), then y for the d->N queries
   const int BH = d->B * d->H;
-  CUtensorMap mq, mk, mv, my;
-  if (!make_map_bf16(&mq, q, d->dk, d->N, BH) || !make_map_bf16(&mk, k, d->dk, d->N, BH) ||
-      !make_map_bf16(&mv, v, d->dv, d->N, BH) || !make_map_bf16(&my, out, d->dv, d->N, BH))
-    return LINATTN_ERR_CUDA;
   const int sms = num_sms();
   if (sms <= 0) return LINATTN_ERR_CUDA;
   if (!set_smem(gtc::global_kv_tc_kernel, static_cast<int>(gtc::kv::kSmemBytes)) ||
       !set_smem(gtc::global_out_tc_kernel, static_cast<int>(gtc::out::kSmemBytes)))
     return LINATTN_ERR_CUDA;
-  const long chunks = (d->N + gtc::C - 1) / gtc::C;
-  const long u1 = static_cast<long>(BH / 2) * chunks, u2 = static_cast<long>(BH) * chunks;
-  gtc::global_kv_tc_kernel<<<static_cast<int>(u1 < sms ? u1 : sms), gtc::kv::NT,
-                             gtc::kv::kSmemBytes, s>>>(mk, mv, KV, ksum, BH / 2, d->N);
-  if (cudaGetLastError() != cudaSuccess) return LINATTN_ERR_CUDA;
-  gtc::global_out_tc_kernel<<<static_cast<int>(u2 < sms ? u2 : sms), gtc::out::NT,
-                              gtc::out::kSmemBytes, s>>>(mq, my, KV, ksum, eps, BH, d->N);
+  if (Nk > 0) {
+    CUtensorMap mk, mv;
+    if (!make_map_bf16(&mk, k, d->dk, Nk, BH) || !make_map_bf16(&mv, v, d->dv, Nk, BH))
+      return LINATTN_ERR_CUDA;
+    const long u1 = static_cast<long>(BH / 2) * ((Nk + gtc::C - 1) / gtc::C);
+    gtc::global_kv_tc_kernel<<<static_cast<int>(u1 < sms ? u1 : sms), gtc::kv::NT,
+                               gtc::kv::kSmemBytes, s>>>(mk, mv, KV, ksum, BH / 2, Nk);
+    if (cudaGetLastError() != cudaSuccess) return LINATTN_ERR_CUDA;
+  }
+  if (d->N > 0) {
+    CUtensorMap mq, my;
+    if (!make_map_bf16(&mq, q, d->dk, d->N, BH) || !make_map_bf16(&my, out, d->dv, d->N, BH))
+      return LINATTN_ERR_CUDA;
+    const long u2 = static_cast<long>(BH) * ((d->N + gtc::C - 1) / gtc::C);
+    gtc::global_out_tc_kernel<<<static_cast<int>(u2 < sms ? u2 : sms), gtc::out::NT,
+                                gtc::out::kSmemBytes, s>>>(mq, my, KV, ksum, eps, BH, d->N);
+  }
   return launch_status();
 }
 
 template <int DK, typename T>
-int global_dv(const linattn_dims *d, const void *q, const void *k, const void *v, float eps,
-              void *out, float *KV, float *ksum, cudaStream_t s) {
+int global_dv(const linattn_dims *d, int Nk, const void *q, const void *k, const void *v,
+              float eps, void *out, float *KV, float *ksum, cudaStream_t s) {
   switch (d->dv) {
-    case 16: return launch_global_simt<DK, 16, T>(d, q, k, v, eps, out, KV, ksum, s);
-    case 32: return launch_global_simt<DK, 32, T>(d, q, k, v, eps, out, KV, ksum, s);
-    case 64: return launch_global_simt<DK, 64, T>(d, q, k, v, eps, out, KV, ksum, s);
-    case 128: return launch_global_simt<DK, 128, T>(d, q, k, v, eps, out, KV, ksum, s);
+    case 16: return launch_global_simt<DK, 16, T>(d, Nk, q, k, v, eps, out, KV, ksum, s);
+    case 32: return launch_global_simt<DK, 32, T>(d, Nk, q, k, v, eps, out, KV, ksum, s);
+    case 64: return launch_global_simt<DK, 64, T>(d, Nk, q, k, v, eps, out, KV, ksum, s);
+    case 128: return launch_global_simt<DK, 128, T>(d, Nk, q, k, v, eps, out, KV, ksum, s);
   }
   return LINATTN_ERR_UNSUPPORTED;
 }
 
 template <typename T>
-int global_dispatch(const linattn_dims *d, const void *q, const void *k, const void *v,
+int global_dispatch(const linattn_dims *d, int Nk, const void *q, const void *k, const void *v,
                     float eps, void *out, float *KV, float *ksum, cudaStream_t s) {
   switch (d->dk) {
-    case 16: return global_dv<16, T>(d, q, k, v, eps, out, KV, ksum, s);
-    case 32: return global_dv<32, T>(d, q, k, v, eps, out, KV, ksum, s);
-    case 64: return global_dv<64, T>(d, q, k, v, eps, out, KV, ksum, s);
-    case 128: return global_dv<128, T>(d, q, k, v, eps, out, KV, ksum, s);
+    case 16: return global_dv<16, T>(d, Nk, q, k, v, eps, out, KV, ksum, s);
+    case 32: return global_dv<32, T>(d, Nk, q, k, v, eps, out, KV, ksum, s);
+    case 64: return global_dv<64, T>(d, Nk, q, k, v, eps, out, KV, ksum, s);
+    case 128: return global_dv<128, T>(d, Nk, q, k, v, eps, out, KV, ksum, s);
   }
   return LINATTN_ERR_UNSUPPORTED;
 }
@@ -477,34 +491,61 @@ extern "C" int linattn_bwd_causal(const linattn_dims *d, const void *q, const vo
   return causal_bwd_dispatch<bf16>(d, q, k, v, lambda, eps, dy, dq, dk, dv, dlambda, s);
 }
 
-extern "C" int linattn_fwd_global(const linattn_dims *d, const void *q, const void *k,
-                                  const void *v, float eps, void *out, float *KV, float *ksum,
-                                  linattn_stream_t stream) {
+namespace linattn {
+namespace {
+
+// Both global entry points: d->N queries against Nk keys/values.
+int fwd_global_impl(const linattn_dims *d, int Nk, const void *q, const void *k, const void *v,
+                    float eps, void *out, float *KV, float *ksum, cudaStream_t s) {
   int rc = check_dims(d, true);
   if (rc != LINATTN_OK) return rc;
+  if (Nk < 0) return LINATTN_ERR_INVALID;
+  if (Nk > 0) {
+    linattn_dims dk_ = *d;
+    dk_.N = Nk;
+    if ((rc = check_dims(&dk_, true)) != LINATTN_OK) return rc;
+  }
   if (bad_eps(eps)) return LINATTN_ERR_INVALID;
   const size_t BH = static_cast<size_t>(d->B) * d->H;
   if (BH == 0) return LINATTN_OK;
   if (!KV || !ksum) return LINATTN_ERR_INVALID;
   const size_t es = elem_size(d->dtype);
-  const size_t nq = BH * d->N * d->dk * es, nv = BH * d->N * d->dv * es;
+  const size_t nq = BH * d->N * d->dk * es, ny = BH * d->N * d->dv * es;
+  const size_t nk = BH * Nk * d->dk * es, nv = BH * Nk * d->dv * es;
   const size_t nS = BH * d->dk * d->dv * 4, nz = BH * d->dk * 4;
-  if (d->N > 0 && (!q || !k || !v || !out)) return LINATTN_ERR_INVALID;
+  if ((d->N > 0 && (!q || !out)) || (Nk > 0 && (!k || !v))) return LINATTN_ERR_INVALID;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(KV) ||
       !aligned16(ksum))
     return LINATTN_ERR_INVALID;
-  if (overlaps(out, nv, q, nq) || overlaps(out, nv, k, nq) || overlaps(out, nv, v, nv) ||
-      overlaps(KV, nS, out, nv) || overlaps(ksum, nz, out, nv) || overlaps(KV, nS, ksum, nz) ||
-      overlaps(KV, nS, k, nq) || overlaps(KV, nS, v, nv))
+  if (overlaps(out, ny, q, nq) || overlaps(out, ny, k, nk) || overlaps(out, ny, v, nv) ||
+      overlaps(KV, nS, out, ny) || overlaps(ksum, nz, out, ny) || overlaps(KV, nS, ksum, nz) ||
+      overlaps(KV, nS, k, nk) || overlaps(KV, nS, v, nv) || overlaps(KV, nS, q, nq) ||
+      overlaps(ksum, nz, q, nq) || overlaps(ksum, nz, k, nk) || overlaps(ksum, nz, v, nv))
     return LINATTN_ERR_INVALID;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(KV, 0, nS, s) != cudaSuccess) return LINATTN_ERR_CUDA;
   if (cudaMemsetAsync(ksum, 0, nz, s) != cudaSuccess) return LINATTN_ERR_CUDA;
-  if (d->N == 0) return LINATTN_OK;
-  if (use_tc_global(d)) return launch_global_tc(d, q, k, v, eps, out, KV, ksum, s);
+  if (d->N == 0 && Nk == 0) return LINATTN_OK;
+  if (use_tc_global(d)) return launch_global_tc(d, Nk, q, k, v, eps, out, KV, ksum, s);
   if (d->dtype == LINATTN_F32)
-    return global_dispatch<float>(d, q, k, v, eps, out, KV, ksum, s);
-  return global_dispatch<bf16>(d, q, k, v, eps, out, KV, ksum, s);
+    return global_dispatch<float>(d, Nk, q, k, v, eps, out, KV, ksum, s);
+  return global_dispatch<bf16>(d, Nk, q, k, v, eps, out, KV, ksum, s);
+}
+
+}  // namespace
+}  // namespace linattn
+
+extern "C" int linattn_fwd_global(const linattn_dims *d, const void *q, const void *k,
+                                  const void *v, float eps, void *out, float *KV, float *ksum,
+                                  linattn_stream_t stream) {
+  return fwd_global_impl(d, d ? d->N : 0, q, k, v, eps, out, KV, ksum,
+                         reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" int linattn_fwd_global_cross(const linattn_dims *d, int Nk, const void *q,
+                                        const void *k, const void *v, float eps, void *out,
+                                        float *KV, float *ksum, linattn_stream_t stream) {
+  return fwd_global_impl(d, Nk, q, k, v, eps, out, KV, ksum,
+                         reinterpret_cast<cudaStream_t>(stream));
 }
 
 extern "C" int linattn_decode_step(const linattn_dims *d, const void *q, const void *k,

@@ -27,7 +27,7 @@ LINATTN_ERR_CUDA = 3
 LINATTN_ERR_DEVICE = 4
 
 ENTRY_POINTS = ("linattn_fwd_causal", "linattn_fwd_causal_from", "linattn_bwd_causal",
-                "linattn_fwd_global", "linattn_decode_step",
+                "linattn_fwd_global", "linattn_fwd_global_cross", "linattn_decode_step",
                 "linattn_status_string", "linattn_device_status", "linattn_version")
 
 
@@ -71,6 +71,8 @@ def load(build_if_missing: bool = True):
     lib.linattn_bwd_causal.restype = i
     lib.linattn_fwd_global.argtypes = [dp, vp, vp, vp, f, vp, fp, fp, vp]
     lib.linattn_fwd_global.restype = i
+    lib.linattn_fwd_global_cross.argtypes = [dp, i, vp, vp, vp, f, vp, fp, fp, vp]
+    lib.linattn_fwd_global_cross.restype = i
     lib.linattn_decode_step.argtypes = [dp, vp, vp, vp, fp, f, fp, fp, vp, vp]
     lib.linattn_decode_step.restype = i
     lib.linattn_status_string.argtypes = [i]
@@ -198,6 +200,24 @@ def linattn_fwd_global(q, k, v, eps, out, KV, ksum, stream=None):
            "linattn_fwd_global")
 
 
+def linattn_fwd_global_cross(q, k, v, eps, out, KV, ksum, stream=None):
+    """Cross global forward: q/out [B,H,Nq,dk/dv], k/v [B,H,Nk,dk/dv];
+    KV [B,H,dk,dv] and ksum [B,H,dk] fp32 (written)."""
+    B, H, Nq, dk = q.shape
+    Nk, dv = k.shape[2], v.shape[-1]
+    if (tuple(k.shape) != (B, H, Nk, dk) or tuple(v.shape) != (B, H, Nk, dv) or
+            tuple(out.shape) != (B, H, Nq, dv)):
+        raise ValueError("shape mismatch among q, k, v, out")
+    if not (q.dtype == k.dtype == v.dtype == out.dtype):
+        raise ValueError("q, k, v, out must share one dtype")
+    _f32(KV, (B, H, dk, dv), "KV")
+    _f32(ksum, (B, H, dk), "ksum")
+    d = linattn_dims(B, H, Nq, dk, dv, _dtype_code(q.dtype))
+    _check(load().linattn_fwd_global_cross(ctypes.byref(d), int(Nk), _ptr(q), _ptr(k), _ptr(v),
+                                           float(eps), _ptr(out), _ptr(KV), _ptr(ksum),
+                                           _stream(stream)), "linattn_fwd_global_cross")
+
+
 def linattn_decode_step(q, k, v, lam, eps, S, z, out, stream=None):
     """One decode step: q, k [B,H,dk], v/out [B,H,dv]; S [B,H,dk,dv] and z
     [B,H,dk] fp32 are updated in place."""
@@ -257,6 +277,16 @@ def fwd_global(q, k, v, eps=1e-6, stream=None):
     KV = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
     ks = torch.empty((B, H, dk), dtype=torch.float32, device=q.device)
     linattn_fwd_global(q, k, v, eps, out, KV, ks, stream)
+    return out, KV, ks
+
+
+def fwd_global_cross(q, k, v, eps=1e-6, stream=None):
+    B, H, Nq, dk = q.shape
+    dv = v.shape[-1]
+    out = torch.empty((B, H, Nq, dv), dtype=v.dtype, device=v.device)
+    KV = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
+    ks = torch.empty((B, H, dk), dtype=torch.float32, device=q.device)
+    linattn_fwd_global_cross(q, k, v, eps, out, KV, ks, stream)
     return out, KV, ks
 
 
