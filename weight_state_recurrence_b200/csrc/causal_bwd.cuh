@@ -27,7 +27,7 @@
 namespace linattn {
 
 constexpr int kBwdChunk = 32;
-constexpr int kBwdThreads = 256;
+constexpr int kBwdThreads = 256;   // a 16 x 16 grid of output tiles
 
 template <int DK, int DV>
 constexpr int causal_bwd_smem_floats(bool with_dlam) {
@@ -56,8 +56,7 @@ __global__ void __launch_bounds__(kBwdThreads) causal_bwd_kernel(
   // lanes walking different rows at the same column hit different banks
   constexpr int C = kBwdChunk, NT = kBwdThreads, QS = DK + 1, AS = C + 1, VS = DV + 1,
                 SS = DV + 1;
-  constexpr int W = DV / 4;   // threads that share one token in the per-column phases
-  static_assert(DV % 4 == 0 && W <= 32 && (32 % W) == 0, "dv must be 16..128");
+  static_assert(DK % 16 == 0 && DV % 16 == 0 && C == 32, "tiles of 16 columns, chunks of 32");
   extern __shared__ __align__(16) float sm[];
   const bool with_dlam = dlam != nullptr;
   float *sQ = sm;                  // [C][DK+1]  phi(q)
@@ -116,34 +115,70 @@ __global__ void __launch_bounds__(kBwdThreads) causal_bwd_kernel(
       sG[i] = t < Cv ? to_f32(dy[o]) : 0.f;
     }
   };
-  // masked decayed scores (and the raw ones for dlambda)
+  // Every product below is a small matrix product over shared memory, tiled
+  // on a 16 x 16 thread grid: thread (ty, tx) owns the outputs at rows
+  // ty + 16 i and columns tx + 16 m, so one pass over the reduced index loads
+  // RI + CJ operands for RI x CJ fused multiply-adds; the odd row strides keep
+  // the loads of the 16 column threads in distinct banks.
+  const int ty = tid >> 4, tx = tid & 15;
+  constexpr int RC = C / 16, NK = DK / 16, NV = DV / 16;
+
+  // masked decayed scores A = lambda^(t-s) phi(q_t).phi(k_s) (s <= t), and the raw ones
   auto scores = [&](int Cv) {
-    for (int i = tid; i < C * C; i += NT) {
-      const int t = i / C, s = i % C;
-      float p = 0.f;
-      if (s <= t && t < Cv) {
-#pragma unroll 8
-        for (int a = 0; a < DK; ++a) p = fmaf(sQ[t * QS + a], sK[s * QS + a], p);
+    float acc[RC][RC] = {};
+#pragma unroll 4
+    for (int a = 0; a < DK; ++a) {
+      float x[RC], y[RC];
+#pragma unroll
+      for (int r = 0; r < RC; ++r) {
+        x[r] = sQ[(ty + 16 * r) * QS + a];
+        y[r] = sK[(tx + 16 * r) * QS + a];
       }
-      sA[t * AS + s] = s <= t && t < Cv ? pw[t - s] * p : 0.f;
-      sP[t * AS + s] = p;
+#pragma unroll
+      for (int r = 0; r < RC; ++r)
+#pragma unroll
+        for (int m = 0; m < RC; ++m) acc[r][m] = fmaf(x[r], y[m], acc[r][m]);
     }
+#pragma unroll
+    for (int r = 0; r < RC; ++r)
+#pragma unroll
+      for (int m = 0; m < RC; ++m) {
+        const int t = ty + 16 * r, u = tx + 16 * m;
+        const bool in = u <= t && t < Cv;
+        sA[t * AS + u] = in ? pw[t - u] * acc[r][m] : 0.f;
+        sP[t * AS + u] = in ? acc[r][m] : 0.f;
+      }
   };
-  // B_ts = lambda^(t-s) (dnum_t . v_s + dden_t); with dlambda also the
+  // B_ts = lambda^(t-s) (dnum_t . v_s + dden_t) (s <= t); with dlambda also the
   // intra-chunk term sum (t-s) lambda^(t-s-1) P_ts (dnum_t . v_s + dden_t)
   auto scores_b = [&](int Cv, bool add_dlam) {
-    for (int i = tid; i < C * C; i += NT) {
-      const int t = i / C, s = i % C;
-      float b = 0.f;
-      if (s <= t && t < Cv) {
-        float e = sDd[t];
-#pragma unroll 8
-        for (int j = 0; j < DV; ++j) e = fmaf(sG[t * DV + j], sV[s * VS + j], e);
-        b = pw[t - s] * e;
-        if (add_dlam) dl = fmaf(dpw[t - s] * sP[t * AS + s], e, dl);
+    float acc[RC][RC] = {};
+#pragma unroll 4
+    for (int jj = 0; jj < DV; ++jj) {
+      float x[RC], y[RC];
+#pragma unroll
+      for (int r = 0; r < RC; ++r) {
+        x[r] = sG[(ty + 16 * r) * DV + jj];
+        y[r] = sV[(tx + 16 * r) * VS + jj];
       }
-      sB[t * AS + s] = b;
+#pragma unroll
+      for (int r = 0; r < RC; ++r)
+#pragma unroll
+        for (int m = 0; m < RC; ++m) acc[r][m] = fmaf(x[r], y[m], acc[r][m]);
     }
+#pragma unroll
+    for (int r = 0; r < RC; ++r)
+#pragma unroll
+      for (int m = 0; m < RC; ++m) {
+        const int t = ty + 16 * r, u = tx + 16 * m;
+        float b = 0.f;
+        if (u <= t && t < Cv) {
+          const float e = acc[r][m] + sDd[t];
+          b = pw[t - u] * e;
+          if (add_dlam) dl = fmaf(dpw[t - u] * sP[t * AS + u], e, dl);
+        }
+        sB[t * AS + u] = b;
+      }
   };
 
   // ------------------------------------------------------------ sweep 1
@@ -157,85 +192,151 @@ __global__ void __launch_bounds__(kBwdThreads) causal_bwd_kernel(
     // den_t = sum_s A_ts + lambda^(t+1) phi(q_t).z + eps
     if (tid < Cv) {
       float rs = 0.f, qz = 0.f;
-      for (int s = 0; s <= tid; ++s) rs += sA[tid * AS + s];
+      for (int u = 0; u <= tid; ++u) rs += sA[tid * AS + u];
       for (int a = 0; a < DK; ++a) qz = fmaf(sQ[tid * QS + a], sz[a], qz);
       sDen[tid] = rs + pw[tid + 1] * qz + eps;
     }
     __syncthreads();
-    // num_t, y_t = num/den, dnum_t = dy_t/den in place, c_t = dy_t . y_t; the W
-    // threads of a token take columns jj + W m (m = 0..3): consecutive lanes,
-    // consecutive columns
-    for (int i = tid; i < C * W; i += NT) {
-      const int t = i / W, jj = i % W;
-      float cpart = 0.f;
-      if (t < Cv) {
-        float num[4] = {0.f, 0.f, 0.f, 0.f}, in[4] = {0.f, 0.f, 0.f, 0.f};
-        for (int s = 0; s <= t; ++s) {
-          const float a = sA[t * AS + s];
+    // num_t = A v + lambda^(t+1) phi(q_t)^T S; y_t = num/den; dnum_t = dy_t/den
+    // (in place); c_t = dy_t . y_t, summed over the 16 column threads of a row
+    {
+      float ni[RC][NV] = {}, ns[RC][NV] = {};
+      for (int u = 0; u < Cv; ++u) {   // A is zero above the diagonal
+        float x[RC], y[NV];
 #pragma unroll
-          for (int m = 0; m < 4; ++m) num[m] = fmaf(a, sV[s * VS + jj + W * m], num[m]);
-        }
-        for (int a = 0; a < DK; ++a) {
-          const float fq = sQ[t * QS + a];
+        for (int r = 0; r < RC; ++r) x[r] = sA[(ty + 16 * r) * AS + u];
 #pragma unroll
-          for (int m = 0; m < 4; ++m) in[m] = fmaf(fq, sS[a * SS + jj + W * m], in[m]);
-        }
-        const float g = pw[t + 1], inv = 1.f / sDen[t];
+        for (int m = 0; m < NV; ++m) y[m] = sV[u * VS + tx + 16 * m];
 #pragma unroll
-        for (int m = 0; m < 4; ++m) {
-          const float d = sG[t * DV + jj + W * m];
-          cpart = fmaf(d, fmaf(g, in[m], num[m]) * inv, cpart);
-          sG[t * DV + jj + W * m] = d * inv;
-        }
+        for (int r = 0; r < RC; ++r)
+#pragma unroll
+          for (int m = 0; m < NV; ++m) ni[r][m] = fmaf(x[r], y[m], ni[r][m]);
       }
-      // the W threads of one token are consecutive lanes of one warp
+#pragma unroll 4
+      for (int a = 0; a < DK; ++a) {
+        float x[RC], y[NV];
 #pragma unroll
-      for (int o = W / 2; o > 0; o >>= 1) cpart += __shfl_xor_sync(0xffffffffu, cpart, o, W);
-      if (jj == 0 && t < Cv) {
-        sCc[t] = cpart;
-        sDd[t] = -cpart / sDen[t];
-        stash_put(dk + qo + static_cast<long>(c0 + t) * DK, sDen[t], cpart);
+        for (int r = 0; r < RC; ++r) x[r] = sQ[(ty + 16 * r) * QS + a];
+#pragma unroll
+        for (int m = 0; m < NV; ++m) y[m] = sS[a * SS + tx + 16 * m];
+#pragma unroll
+        for (int r = 0; r < RC; ++r)
+#pragma unroll
+          for (int m = 0; m < NV; ++m) ns[r][m] = fmaf(x[r], y[m], ns[r][m]);
+      }
+#pragma unroll
+      for (int r = 0; r < RC; ++r) {
+        const int t = ty + 16 * r;
+        float cpart = 0.f;
+        if (t < Cv) {
+          const float g = pw[t + 1], inv = 1.f / sDen[t];
+#pragma unroll
+          for (int m = 0; m < NV; ++m) {
+            float *gp = &sG[t * DV + tx + 16 * m];
+            const float d = *gp;
+            cpart = fmaf(d, fmaf(g, ns[r][m], ni[r][m]) * inv, cpart);
+            *gp = d * inv;
+          }
+        }
+        // the 16 column threads of a row are 16 consecutive lanes of one warp
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1) cpart += __shfl_xor_sync(0xffffffffu, cpart, o, 16);
+        if (tx == 0 && t < Cv) {
+          sCc[t] = cpart;
+          sDd[t] = -cpart / sDen[t];
+          stash_put(dk + qo + static_cast<long>(c0 + t) * DK, sDen[t], cpart);
+        }
       }
     }
     __syncthreads();
     scores_b(Cv, with_dlam);
     __syncthreads();
     // dphi(q_t) = lambda^(t+1) (S dnum_t + z dden_t) + sum_s B_ts phi(k_s); dq
-    for (int i = tid; i < C * DK; i += NT) {
-      const int t = i / DK, a = i % DK;
-      if (t >= Cv) continue;
-      float gs = sz[a] * sDd[t];
-      for (int j = 0; j < DV; ++j) gs = fmaf(sS[a * SS + j], sG[t * DV + j], gs);
-      float intra = 0.f;
-      for (int s = 0; s <= t; ++s) intra = fmaf(sB[t * AS + s], sK[s * QS + a], intra);
-      const float fq = sQ[t * QS + a];
-      const float dphi = fmaf(pw[t + 1], gs, intra);
-      dq[qo + static_cast<long>(c0 + t) * DK + a] = from_f32<T>(dphi * (fq > 1.f ? 1.f : fq));
-      if (with_dlam) {
-        float gs2 = sz2[a] * sDd[t];
-        for (int j = 0; j < DV; ++j) gs2 = fmaf(sS2[a * SS + j], sG[t * DV + j], gs2);
-        dl = fmaf(fq, fmaf(dpw[t + 1], gs, pw[t + 1] * gs2), dl);
+    {
+      float g1[RC][NK] = {}, g2[RC][NK] = {}, in[RC][NK] = {};
+#pragma unroll 2
+      for (int jj = 0; jj < DV; ++jj) {
+        float x[RC], y[NK];
+#pragma unroll
+        for (int r = 0; r < RC; ++r) x[r] = sG[(ty + 16 * r) * DV + jj];
+#pragma unroll
+        for (int m = 0; m < NK; ++m) y[m] = sS[(tx + 16 * m) * SS + jj];
+#pragma unroll
+        for (int r = 0; r < RC; ++r)
+#pragma unroll
+          for (int m = 0; m < NK; ++m) g1[r][m] = fmaf(x[r], y[m], g1[r][m]);
+        if (with_dlam) {
+#pragma unroll
+          for (int m = 0; m < NK; ++m) y[m] = sS2[(tx + 16 * m) * SS + jj];
+#pragma unroll
+          for (int r = 0; r < RC; ++r)
+#pragma unroll
+            for (int m = 0; m < NK; ++m) g2[r][m] = fmaf(x[r], y[m], g2[r][m]);
+        }
+      }
+      for (int u = 0; u < Cv; ++u) {   // B is zero above the diagonal
+        float x[RC], y[NK];
+#pragma unroll
+        for (int r = 0; r < RC; ++r) x[r] = sB[(ty + 16 * r) * AS + u];
+#pragma unroll
+        for (int m = 0; m < NK; ++m) y[m] = sK[u * QS + tx + 16 * m];
+#pragma unroll
+        for (int r = 0; r < RC; ++r)
+#pragma unroll
+          for (int m = 0; m < NK; ++m) in[r][m] = fmaf(x[r], y[m], in[r][m]);
+      }
+#pragma unroll
+      for (int r = 0; r < RC; ++r) {
+        const int t = ty + 16 * r;
+        if (t >= Cv) continue;
+#pragma unroll
+        for (int m = 0; m < NK; ++m) {
+          const int a = tx + 16 * m;
+          const float gs = fmaf(sz[a], sDd[t], g1[r][m]);
+          const float fq = sQ[t * QS + a];
+          dq[qo + static_cast<long>(c0 + t) * DK + a] =
+              from_f32<T>(fmaf(pw[t + 1], gs, in[r][m]) * (fq > 1.f ? 1.f : fq));
+          if (with_dlam) {
+            const float gs2 = fmaf(sz2[a], sDd[t], g2[r][m]);
+            dl = fmaf(fq, fmaf(dpw[t + 1], gs, pw[t + 1] * gs2), dl);
+          }
+        }
       }
     }
     __syncthreads();
-    // state after the chunk: S' first (it needs the S before the chunk)
+    // state after the chunk: S' first (it needs the S before the chunk), then S
     const float gC = pw[Cv], dgC = dpw[Cv];
-    for (int i = tid; i < DK * DV; i += NT) {
-      const int a = i / DV, j = i % DV, o = a * SS + j;
-      float acc = 0.f, acc2 = 0.f;
-      for (int s = 0; s < Cv; ++s) {
-        const float kv = sK[s * QS + a] * sV[s * VS + j];
-        acc = fmaf(pw[Cv - 1 - s], kv, acc);
-        if (with_dlam) acc2 = fmaf(dpw[Cv - 1 - s], kv, acc2);
+    for (int pass = with_dlam ? 0 : 1; pass < 2; ++pass) {
+      const float *wt = pass == 0 ? dpw : pw;
+      float acc[NK][NV] = {};
+      for (int u = 0; u < Cv; ++u) {
+        const float w = wt[Cv - 1 - u];
+        float x[NK], y[NV];
+#pragma unroll
+        for (int r = 0; r < NK; ++r) x[r] = w * sK[u * QS + ty + 16 * r];
+#pragma unroll
+        for (int m = 0; m < NV; ++m) y[m] = sV[u * VS + tx + 16 * m];
+#pragma unroll
+        for (int r = 0; r < NK; ++r)
+#pragma unroll
+          for (int m = 0; m < NV; ++m) acc[r][m] = fmaf(x[r], y[m], acc[r][m]);
       }
-      if (with_dlam) sS2[o] = fmaf(dgC, sS[o], fmaf(gC, sS2[o], acc2));
-      sS[o] = fmaf(gC, sS[o], acc);
+#pragma unroll
+      for (int r = 0; r < NK; ++r)
+#pragma unroll
+        for (int m = 0; m < NV; ++m) {
+          const int o = (ty + 16 * r) * SS + tx + 16 * m;
+          if (pass == 0)
+            sS2[o] = fmaf(dgC, sS[o], fmaf(gC, sS2[o], acc[r][m]));
+          else
+            sS[o] = fmaf(gC, sS[o], acc[r][m]);
+        }
     }
     for (int a = tid; a < DK; a += NT) {
       float acc = 0.f, acc2 = 0.f;
-      for (int s = 0; s < Cv; ++s) {
-        acc = fmaf(pw[Cv - 1 - s], sK[s * QS + a], acc);
-        if (with_dlam) acc2 = fmaf(dpw[Cv - 1 - s], sK[s * QS + a], acc2);
+      for (int u = 0; u < Cv; ++u) {
+        acc = fmaf(pw[Cv - 1 - u], sK[u * QS + a], acc);
+        if (with_dlam) acc2 = fmaf(dpw[Cv - 1 - u], sK[u * QS + a], acc2);
       }
       if (with_dlam) sz2[a] = fmaf(dgC, sz[a], fmaf(gC, sz2[a], acc2));
       sz[a] = fmaf(gC, sz[a], acc);
@@ -265,35 +366,104 @@ __global__ void __launch_bounds__(kBwdThreads) causal_bwd_kernel(
     scores_b(Cv, false);
     __syncthreads();
     // dphi(k_s) = lambda^(Cv-s) (R v_s + r) + sum_{t>=s} B_ts phi(q_t); dk
-    for (int i = tid; i < C * DK; i += NT) {
-      const int s = i / DK, a = i % DK;
-      if (s >= Cv) continue;
-      float rv = sz[a];
-      for (int j = 0; j < DV; ++j) rv = fmaf(sS[a * SS + j], sV[s * VS + j], rv);
-      float intra = 0.f;
-      for (int t = s; t < Cv; ++t) intra = fmaf(sB[t * AS + s], sQ[t * QS + a], intra);
-      const float fk = sK[s * QS + a];
-      dk[qo + static_cast<long>(c0 + s) * DK + a] =
-          from_f32<T>(fmaf(pw[Cv - s], rv, intra) * (fk > 1.f ? 1.f : fk));
+    {
+      float rv[RC][NK] = {}, in[RC][NK] = {};
+#pragma unroll 2
+      for (int jj = 0; jj < DV; ++jj) {
+        float x[RC], y[NK];
+#pragma unroll
+        for (int r = 0; r < RC; ++r) x[r] = sV[(ty + 16 * r) * VS + jj];
+#pragma unroll
+        for (int m = 0; m < NK; ++m) y[m] = sS[(tx + 16 * m) * SS + jj];
+#pragma unroll
+        for (int r = 0; r < RC; ++r)
+#pragma unroll
+          for (int m = 0; m < NK; ++m) rv[r][m] = fmaf(x[r], y[m], rv[r][m]);
+      }
+      for (int t = 0; t < Cv; ++t) {   // B_ts is zero for s > t
+        float x[RC], y[NK];
+#pragma unroll
+        for (int r = 0; r < RC; ++r) x[r] = sB[t * AS + ty + 16 * r];
+#pragma unroll
+        for (int m = 0; m < NK; ++m) y[m] = sQ[t * QS + tx + 16 * m];
+#pragma unroll
+        for (int r = 0; r < RC; ++r)
+#pragma unroll
+          for (int m = 0; m < NK; ++m) in[r][m] = fmaf(x[r], y[m], in[r][m]);
+      }
+#pragma unroll
+      for (int r = 0; r < RC; ++r) {
+        const int u = ty + 16 * r;
+        if (u >= Cv) continue;
+#pragma unroll
+        for (int m = 0; m < NK; ++m) {
+          const int a = tx + 16 * m;
+          const float fk = sK[u * QS + a];
+          dk[qo + static_cast<long>(c0 + u) * DK + a] =
+              from_f32<T>(fmaf(pw[Cv - u], rv[r][m] + sz[a], in[r][m]) * (fk > 1.f ? 1.f : fk));
+        }
+      }
     }
     // dv_s = lambda^(Cv-s) R^T phi(k_s) + sum_{t>=s} A_ts dnum_t
-    for (int i = tid; i < C * DV; i += NT) {
-      const int s = i / DV, j = i % DV;
-      if (s >= Cv) continue;
-      float rk = 0.f;
-      for (int a = 0; a < DK; ++a) rk = fmaf(sS[a * SS + j], sK[s * QS + a], rk);
-      float intra = 0.f;
-      for (int t = s; t < Cv; ++t) intra = fmaf(sA[t * AS + s], sG[t * DV + j], intra);
-      dv[vo + static_cast<long>(c0 + s) * DV + j] = from_f32<T>(fmaf(pw[Cv - s], rk, intra));
+    {
+      float rk[RC][NV] = {}, in[RC][NV] = {};
+#pragma unroll 4
+      for (int a = 0; a < DK; ++a) {
+        float x[RC], y[NV];
+#pragma unroll
+        for (int r = 0; r < RC; ++r) x[r] = sK[(ty + 16 * r) * QS + a];
+#pragma unroll
+        for (int m = 0; m < NV; ++m) y[m] = sS[a * SS + tx + 16 * m];
+#pragma unroll
+        for (int r = 0; r < RC; ++r)
+#pragma unroll
+          for (int m = 0; m < NV; ++m) rk[r][m] = fmaf(x[r], y[m], rk[r][m]);
+      }
+      for (int t = 0; t < Cv; ++t) {   // A_ts is zero for s > t
+        float x[RC], y[NV];
+#pragma unroll
+        for (int r = 0; r < RC; ++r) x[r] = sA[t * AS + ty + 16 * r];
+#pragma unroll
+        for (int m = 0; m < NV; ++m) y[m] = sG[t * DV + tx + 16 * m];
+#pragma unroll
+        for (int r = 0; r < RC; ++r)
+#pragma unroll
+          for (int m = 0; m < NV; ++m) in[r][m] = fmaf(x[r], y[m], in[r][m]);
+      }
+#pragma unroll
+      for (int r = 0; r < RC; ++r) {
+        const int u = ty + 16 * r;
+        if (u >= Cv) continue;
+#pragma unroll
+        for (int m = 0; m < NV; ++m)
+          dv[vo + static_cast<long>(c0 + u) * DV + tx + 16 * m] =
+              from_f32<T>(fmaf(pw[Cv - u], rk[r][m], in[r][m]));
+      }
     }
     __syncthreads();
     // R <- lambda^Cv R + sum_t lambda^t phi(q_t) dnum_t^T;  r likewise with dden
     const float gC = pw[Cv];
-    for (int i = tid; i < DK * DV; i += NT) {
-      const int a = i / DV, j = i % DV, o = a * SS + j;
-      float acc = 0.f;
-      for (int t = 0; t < Cv; ++t) acc = fmaf(pw[t] * sQ[t * QS + a], sG[t * DV + j], acc);
-      sS[o] = fmaf(gC, sS[o], acc);
+    {
+      float acc[NK][NV] = {};
+      for (int t = 0; t < Cv; ++t) {
+        const float w = pw[t];
+        float x[NK], y[NV];
+#pragma unroll
+        for (int r = 0; r < NK; ++r) x[r] = w * sQ[t * QS + ty + 16 * r];
+#pragma unroll
+        for (int m = 0; m < NV; ++m) y[m] = sG[t * DV + tx + 16 * m];
+#pragma unroll
+        for (int r = 0; r < NK; ++r)
+#pragma unroll
+          for (int m = 0; m < NV; ++m) acc[r][m] = fmaf(x[r], y[m], acc[r][m]);
+      }
+#pragma unroll
+      for (int r = 0; r < NK; ++r)
+#pragma unroll
+        for (int m = 0; m < NV; ++m) {
+          const int o = (ty + 16 * r) * SS + tx + 16 * m;
+          sS[o] = fmaf(gC, sS[o], acc[r][m]);
+        }
     }
     for (int a = tid; a < DK; a += NT) {
       float acc = 0.f;
