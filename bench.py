@@ -361,6 +361,41 @@ def global_leg(lib, args, world, rank, stream, hbm):
     return res
 
 
+def seg_leg(lib, args, world, rank, stream, hbm):
+    """The causal_d64 workload (B=2, H=8, N=4096, d=64, bf16, no decay), which
+    the CUDA-core path serves with 32 CTAs: one sequential pass per head and
+    dv slice, against the segment-parallel form with its workspace."""
+    w = inputs.WORKLOADS["causal_d64"]
+    B, H, N, d = w.B, w.H, w.N, w.d
+    dev = torch.device("cuda")
+    q, k, v = inputs.qkv((B, H, N, d), (B, H, N, d), w.seed * 1000 + rank, w.scale, w.dtype,
+                         device=dev)
+    out = torch.empty_like(v)
+    S = torch.empty(B, H, d, d, device=dev)
+    z = torch.empty(B, H, d, device=dev)
+    need = lib.linattn_fwd_causal_workspace(B, H, N, d, d, w.dtype)
+    ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    res = {"workload": "causal_d64: B=2 x H=8 x N=4096, d=64, bf16, no decay",
+           "workspace_bytes": need}
+    alg = causal_bytes(B, H, N, d, d)
+    for name, fn in (("single_pass", lambda: lib.linattn_fwd_causal(q, k, v, None, w.eps, out, S,
+                                                                     z, stream)),
+                     ("segmented", lambda: lib.linattn_fwd_causal_ws(q, k, v, None, w.eps, None,
+                                                                     None, out, S, z, ws,
+                                                                     stream))):
+        with torch.cuda.stream(stream):
+            ms = time_steps(fn, args.steps, args.warmup, world, stream)
+        per = ms / 1e3 / args.steps
+        res[name] = {"value": B * N * world / per, "unit": "tokens/s", "ms_per_step": per * 1e3,
+                     "roofline": {"bound": "hbm", "achieved": alg / per / 1e9, "peak": hbm,
+                                  "unit": "GB/s", "frac": alg / per / 1e9 / hbm,
+                                  "algorithmic_bytes_per_launch": alg}}
+    assert lib.linattn_device_status(clear=True, stream=stream) == 0
+    del q, k, v, out, ws
+    torch.cuda.empty_cache()
+    return res
+
+
 def bwd_flops(B, H, N, dk, dv, with_dlam=True):
     """fp32 FMA work of the backward kernel as written, 2 flops each: per
     chunk of C = 32 tokens and head, both sweeps' score tiles (lower
@@ -474,7 +509,7 @@ def main():
     ap.add_argument("--no-legs", dest="legs", action="store_false")
     ap.add_argument("--no-cpu-baseline", dest="cpu", action="store_false")
     ap.add_argument("--only", default="all",
-                    choices=["all", "causal", "decode", "global", "backward"])
+                    choices=["all", "causal", "decode", "global", "backward", "segmented"])
     ap.add_argument("--batch", type=int, default=0, help="causal leg batch (profiling)")
     ap.add_argument("--dec-batch", type=int, default=0, help="decode sequences (profiling)")
     ap.add_argument("--dec-steps", type=int, default=0, help="decode steps (profiling)")
@@ -490,9 +525,11 @@ def main():
     hbm, tcp, peak_src = peaks()
     stream = torch.cuda.Stream()
 
-    if args.only in ("decode", "global", "backward"):
+    if args.only in ("decode", "global", "backward", "segmented"):
         if args.only == "backward":
             r = bwd_leg(lib, args, world, rank, stream, ALU_PEAK_TFLOPS)
+        elif args.only == "segmented":
+            r = seg_leg(lib, args, world, rank, stream, hbm)
         else:
             leg = decode_leg if args.only == "decode" else global_leg
             r = leg(lib, args, world, rank, stream, hbm)
@@ -522,6 +559,7 @@ def main():
         line["decode"] = decode_leg(lib, args, world, rank, stream, hbm)
         line["global"] = global_leg(lib, args, world, rank, stream, hbm)
         line["backward"] = bwd_leg(lib, args, world, rank, stream, ALU_PEAK_TFLOPS)
+        line["segmented"] = seg_leg(lib, args, world, rank, stream, hbm)
     if args.cpu and world == 1 and rank == 0:
         tok_s, cores, desc, _ = oracle_sample()
         line["cpu_baseline"] = {"value": tok_s, "unit": "tokens/s", "cores": cores,

@@ -51,6 +51,8 @@
 #define LINATTN_API
 #endif
 
+#include <stddef.h>
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -115,6 +117,31 @@ LINATTN_API int linattn_fwd_causal_from(const linattn_dims *dims, const void *q,
                        const void *v, const float *lambda, float eps,
                        const float *S_init, const float *z_init, void *out,
                        float *S_final, float *z_final, linattn_stream_t stream);
+
+/*
+ * Segment-parallel causal forward (the "parallel scan" alternative to one
+ * sequential pass, [FW] §4.1 note and §5.2, one level above the chunks).  When
+ * there are too few (b, h) to fill the GPU, each sequence is cut into G
+ * segments: every segment's own final state is computed from zero, the
+ * segments' starting states follow from one short scan over them
+ * (carry_{g+1} = lambda^len_g carry_g + dS_g), and all segments then run at
+ * once.  The result is the recurrence of linattn_fwd_causal_from, up to fp32
+ * summation order.
+ *
+ * linattn_fwd_causal_workspace: the bytes of workspace the segmented form
+ *   needs for these dims (0: the single pass is used; also for invalid dims).
+ *   Only the CUDA-core path (fp32 inputs, or d_k != 128) is segmented.
+ * linattn_fwd_causal_ws: linattn_fwd_causal_from with a caller-owned device
+ *   workspace (16-byte aligned, overlapping no other argument, contents
+ *   irrelevant and overwritten); with workspace_bytes below the size above,
+ *   or workspace = NULL, it runs the single pass.
+ */
+LINATTN_API size_t linattn_fwd_causal_workspace(const linattn_dims *dims);
+LINATTN_API int linattn_fwd_causal_ws(const linattn_dims *dims, const void *q, const void *k,
+                       const void *v, const float *lambda, float eps,
+                       const float *S_init, const float *z_init, void *out,
+                       float *S_final, float *z_final, void *workspace,
+                       size_t workspace_bytes, linattn_stream_t stream);
 
 /*
  * Backward of linattn_fwd_causal (zero starting state): the gradients of

@@ -33,7 +33,8 @@ __global__ void __launch_bounds__(256) causal_simt_kernel(
     const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
     const float *__restrict__ lam, float eps, const float *__restrict__ S_init,
     const float *__restrict__ z_init, T *__restrict__ out, float *__restrict__ S_final,
-    float *__restrict__ z_final, int H, int N, int DV) {
+    float *__restrict__ z_final, int H, int N, int DV, int seg_len,
+    const float *__restrict__ S_seg, const float *__restrict__ z_seg) {
   constexpr int C = kSimtChunk, NT = 256, QS = DK + 1;
   static_assert(DVS % 4 == 0, "slice must be float4-divisible");
   extern __shared__ __align__(16) float sm[];
@@ -54,18 +55,26 @@ __global__ void __launch_bounds__(256) causal_simt_kernel(
   const float L = lam ? lam[h] : 1.f;
 
   if (tid <= C) pw[tid] = pow_int(L, tid);
-  // the state before the first token: the caller's (S_init, z_init), else zero
+  // segment blockIdx.y of gridDim.y covers tokens [n0, n1); with segments its
+  // starting state is its slot of (S_seg, z_seg), otherwise the caller's
+  // (S_init, z_init) or zero
+  const int G = gridDim.y, g = blockIdx.y;
+  const int n0 = g * seg_len, n1 = min(N, n0 + seg_len);
+  const float *S0 = S_seg ? S_seg + (pair * G + g) * static_cast<long>(DK) * DV : S_init;
+  const float *z0 = z_seg ? z_seg + (pair * G + g) * static_cast<long>(DK) : z_init;
+  const long s0off = S_seg ? 0 : pair * static_cast<long>(DK) * DV;
+  const long z0off = z_seg ? 0 : pair * static_cast<long>(DK);
   for (int i = tid; i < DK * DVS; i += NT)
-    sS[i] = S_init ? S_init[(pair * DK + i / DVS) * DV + j0 + i % DVS] : 0.f;
-  for (int i = tid; i < DK; i += NT) sz[i] = z_init ? z_init[pair * DK + i] : 0.f;
+    sS[i] = S0 ? S0[s0off + (i / DVS) * static_cast<long>(DV) + j0 + i % DVS] : 0.f;
+  for (int i = tid; i < DK; i += NT) sz[i] = z0 ? z0[z0off + i] : 0.f;
 
   const T *qp = q + pair * static_cast<long>(N) * DK;
   const T *kp = k + pair * static_cast<long>(N) * DK;
   const T *vp = v + pair * static_cast<long>(N) * DV;
   T *op = out + pair * static_cast<long>(N) * DV;
 
-  for (int c0 = 0; c0 < N; c0 += C) {
-    const int Cv = min(C, N - c0);
+  for (int c0 = n0; c0 < n1; c0 += C) {
+    const int Cv = min(C, n1 - c0);
     __syncthreads();
     for (int i = tid; i < C * DK; i += NT) {
       const int t = i / DK, a = i % DK;
@@ -166,6 +175,7 @@ __global__ void __launch_bounds__(256) causal_simt_kernel(
     }
   }
   __syncthreads();
+  if (g != G - 1) return;   // only the last segment ends at the sequence's end
   if (S_final) {
     for (int i = tid; i < DK * DVS; i += NT) {
       const int c = i / DVS, j = i % DVS;
@@ -174,6 +184,108 @@ __global__ void __launch_bounds__(256) causal_simt_kernel(
   }
   if (z_final && j0 == 0) {
     for (int c = tid; c < DK; c += NT) z_final[pair * DK + c] = sz[c];
+  }
+}
+
+// ------------------------------------------------ segment-parallel form
+// For few (b, h) the sequence is cut into G segments of seg_len tokens
+// (blockwise accumulation of [FW] §4.1 note and §5.2, one level up: the
+// "parallel scan" alternative).  (1) Each segment but the last computes the
+// state it would end in from zero, dS_g = sum_{j in g} lambda^(end_g - j)
+// phi(k_j) v_j^T and dz_g likewise; (2) one pass per head turns them into the
+// starting state of every segment, carry_{g+1} = lambda^(len_g) carry_g + dS_g
+// with carry_0 the caller's starting state; (3) the chunked kernel above runs
+// all segments at once, each from its carry.  dS_g and carry_g share one slot
+// of the workspace ([B*H][G][DK][DV] fp32, then [B*H][G][DK] fp32).
+
+template <int DK, int DVS, typename T>
+__global__ void __launch_bounds__(256) causal_seg_state_kernel(
+    const T *__restrict__ k, const T *__restrict__ v, const float *__restrict__ lam,
+    float *__restrict__ ws_S, float *__restrict__ ws_z, int H, int N, int DV, int seg_len,
+    int G) {
+  constexpr int C = kSimtChunk, NT = 256, QS = DK + 1;
+  constexpr int NR = DK / 16, NCOL = DVS / 16;
+  __shared__ float sK[C * QS];      // lambda^(Cv-1-s) phi(k_s)
+  __shared__ float sV[C * (DVS + 1)];
+  __shared__ float pw[C + 4];
+  const int nslices = DV / DVS;
+  const long pair = blockIdx.x / nslices;
+  const int j0 = (blockIdx.x % nslices) * DVS;
+  const int g = blockIdx.y, tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
+  const float L = lam ? lam[pair % H] : 1.f;
+  if (tid < C + 4) pw[tid] = pow_int(L, tid);
+  const int n0 = g * seg_len, n1 = min(N, n0 + seg_len);
+  const T *kp = k + pair * static_cast<long>(N) * DK;
+  const T *vp = v + pair * static_cast<long>(N) * DV;
+  float acc[NR][NCOL] = {};
+  float zacc = 0.f;                 // thread a < DK: the normaliser's row a
+  for (int c0 = n0; c0 < n1; c0 += C) {
+    const int Cv = min(C, n1 - c0);
+    __syncthreads();
+    for (int i = tid; i < C * DK; i += NT) {
+      const int t = i / DK, a = i % DK;
+      sK[t * QS + a] = t < Cv ? pw[Cv - 1 - t] * phi_f32(to_f32(kp[static_cast<long>(c0 + t) * DK + a]))
+                              : 0.f;
+    }
+    for (int i = tid; i < C * DVS; i += NT) {
+      const int t = i / DVS, j = i % DVS;
+      sV[t * (DVS + 1) + j] = t < Cv ? to_f32(vp[static_cast<long>(c0 + t) * DV + j0 + j]) : 0.f;
+    }
+    __syncthreads();
+    const float gC = pw[Cv];
+#pragma unroll
+    for (int r = 0; r < NR; ++r)
+#pragma unroll
+      for (int m = 0; m < NCOL; ++m) acc[r][m] *= gC;
+    for (int t = 0; t < Cv; ++t) {
+      float x[NR], y[NCOL];
+#pragma unroll
+      for (int r = 0; r < NR; ++r) x[r] = sK[t * QS + ty + 16 * r];
+#pragma unroll
+      for (int m = 0; m < NCOL; ++m) y[m] = sV[t * (DVS + 1) + tx + 16 * m];
+#pragma unroll
+      for (int r = 0; r < NR; ++r)
+#pragma unroll
+        for (int m = 0; m < NCOL; ++m) acc[r][m] = fmaf(x[r], y[m], acc[r][m]);
+    }
+    if (tid < DK) {
+      zacc *= gC;
+      for (int t = 0; t < Cv; ++t) zacc += sK[t * QS + tid];
+    }
+  }
+  float *Sg = ws_S + (pair * G + g) * static_cast<long>(DK) * DV;
+#pragma unroll
+  for (int r = 0; r < NR; ++r)
+#pragma unroll
+    for (int m = 0; m < NCOL; ++m) Sg[(ty + 16 * r) * static_cast<long>(DV) + j0 + tx + 16 * m] = acc[r][m];
+  if (j0 == 0 && tid < DK) ws_z[(pair * G + g) * static_cast<long>(DK) + tid] = zacc;
+}
+
+// carry_0 = (S_init, z_init) or zero; carry_{g+1} = lambda^len_g carry_g + dS_g,
+// written over dS_g's slot; one CTA per (b, h), one element per thread step
+__global__ void __launch_bounds__(256) causal_seg_combine_kernel(
+    const float *__restrict__ lam, const float *__restrict__ S_init,
+    const float *__restrict__ z_init, float *__restrict__ ws_S, float *__restrict__ ws_z, int H,
+    int DK, int DV, int N, int seg_len, int G) {
+  __shared__ float decay[64];       // lambda^len_g
+  const long pair = blockIdx.x;
+  const float L = lam ? lam[pair % H] : 1.f;
+  for (int gg = threadIdx.x; gg < G; gg += blockDim.x)
+    decay[gg] = pow_int(L, min(seg_len, N - gg * seg_len));
+  __syncthreads();
+  const long per = static_cast<long>(DK) * DV;
+  for (long e = threadIdx.x; e < per + DK; e += blockDim.x) {
+    const bool isz = e >= per;
+    const long ei = isz ? e - per : e;
+    float *base = isz ? ws_z + pair * G * static_cast<long>(DK) : ws_S + pair * G * per;
+    const long stride = isz ? DK : per;
+    const float *init = isz ? z_init : S_init;
+    float run = init ? init[pair * stride + ei] : 0.f;
+    for (int gg = 0; gg < G; ++gg) {
+      const float d = gg < G - 1 ? base[gg * stride + ei] : 0.f;
+      base[gg * stride + ei] = run;
+      run = fmaf(decay[gg], run, d);
+    }
   }
 }
 

@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstdlib>
@@ -181,40 +182,90 @@ int decode_dispatch(const linattn_dims *d, const void *q, const void *k, const v
   return LINATTN_ERR_UNSUPPORTED;
 }
 
+// Segment-parallel plan for the CUDA-core causal kernel: G segments of len
+// tokens when (b, h, dv-slice) alone would leave most SMs idle; ws is the
+// workspace (G = 1: none, single pass).
+struct Segments {
+  int G = 1, len = 0;
+  float *ws = nullptr;
+};
+constexpr int kMaxSegments = 64;
+
+int simt_dv_slice(int dv) { return dv <= 16 ? 16 : 32; }
+
+Segments plan_segments(const linattn_dims *d) {
+  Segments sg;
+  sg.len = d->N;
+  if (use_tc_causal(d) || d->N < 256) return sg;
+  const long ctas = static_cast<long>(d->B) * d->H * (d->dv / simt_dv_slice(d->dv));
+  const int sms = num_sms();
+  if (sms <= 0 || ctas == 0 || ctas >= sms) return sg;
+  long G = (2L * sms + ctas - 1) / ctas;   // about two waves of CTAs
+  G = std::min<long>(G, d->N / 128);       // segments of at least 128 tokens
+  G = std::min<long>(G, kMaxSegments);
+  if (G < 2) return sg;
+  const int len = static_cast<int>(((d->N + G - 1) / G + 31) / 32 * 32);
+  sg.G = (d->N + len - 1) / len;
+  sg.len = len;
+  if (sg.G < 2) sg = Segments{1, d->N, nullptr};
+  return sg;
+}
+
+size_t segment_bytes(const linattn_dims *d, const Segments &sg) {
+  if (sg.G < 2) return 0;
+  return static_cast<size_t>(d->B) * d->H * sg.G * (static_cast<size_t>(d->dk) * d->dv + d->dk) * 4;
+}
+
 template <int DK, int DVS, typename T>
 int launch_causal_simt(const linattn_dims *d, const void *q, const void *k, const void *v,
                        const float *lam, float eps, const float *S_init, const float *z_init,
-                       void *out, float *S_final, float *z_final, cudaStream_t s) {
+                       void *out, float *S_final, float *z_final, const Segments &sg,
+                       cudaStream_t s) {
   auto *kern = causal_simt_kernel<DK, DVS, T>;
   const int bytes = causal_simt_smem_floats<DK, DVS>() * 4;
   if (!set_smem(kern, bytes)) return LINATTN_ERR_CUDA;
-  const int grid = d->B * d->H * (d->dv / DVS);
-  kern<<<grid, 256, bytes, s>>>(static_cast<const T *>(q), static_cast<const T *>(k),
-                                static_cast<const T *>(v), lam, eps, S_init, z_init,
-                                static_cast<T *>(out), S_final, z_final, d->H, d->N, d->dv);
+  const int ctas = d->B * d->H * (d->dv / DVS);
+  float *wsS = sg.ws, *wsz = sg.ws ? sg.ws + static_cast<long>(d->B) * d->H * sg.G * d->dk * d->dv
+                                   : nullptr;
+  if (sg.G > 1) {
+    // (1) each segment's own final state from zero, (2) the starting states
+    causal_seg_state_kernel<DK, DVS, T><<<dim3(ctas, sg.G - 1), 256, 0, s>>>(
+        static_cast<const T *>(k), static_cast<const T *>(v), lam, wsS, wsz, d->H, d->N, d->dv,
+        sg.len, sg.G);
+    if (cudaGetLastError() != cudaSuccess) return LINATTN_ERR_CUDA;
+    causal_seg_combine_kernel<<<d->B * d->H, 256, 0, s>>>(lam, S_init, z_init, wsS, wsz, d->H,
+                                                          d->dk, d->dv, d->N, sg.len, sg.G);
+    if (cudaGetLastError() != cudaSuccess) return LINATTN_ERR_CUDA;
+  }
+  kern<<<dim3(ctas, sg.G), 256, bytes, s>>>(
+      static_cast<const T *>(q), static_cast<const T *>(k), static_cast<const T *>(v), lam, eps,
+      S_init, z_init, static_cast<T *>(out), S_final, z_final, d->H, d->N, d->dv, sg.len,
+      sg.G > 1 ? wsS : nullptr, sg.G > 1 ? wsz : nullptr);
   return launch_status();
 }
 
 template <int DK, typename T>
 int causal_simt_dv(const linattn_dims *d, const void *q, const void *k, const void *v,
                    const float *lam, float eps, const float *S_init, const float *z_init,
-                   void *out, float *S_final, float *z_final, cudaStream_t s) {
+                   void *out, float *S_final, float *z_final, const Segments &sg,
+                   cudaStream_t s) {
   if (d->dv == 16)
     return launch_causal_simt<DK, 16, T>(d, q, k, v, lam, eps, S_init, z_init, out, S_final,
-                                         z_final, s);
+                                         z_final, sg, s);
   return launch_causal_simt<DK, 32, T>(d, q, k, v, lam, eps, S_init, z_init, out, S_final,
-                                       z_final, s);
+                                       z_final, sg, s);
 }
 
 template <typename T>
 int causal_simt_dispatch(const linattn_dims *d, const void *q, const void *k, const void *v,
                          const float *lam, float eps, const float *S_init, const float *z_init,
-                         void *out, float *S_final, float *z_final, cudaStream_t s) {
+                         void *out, float *S_final, float *z_final, const Segments &sg,
+                         cudaStream_t s) {
   switch (d->dk) {
-    case 16: return causal_simt_dv<16, T>(d, q, k, v, lam, eps, S_init, z_init, out, S_final, z_final, s);
-    case 32: return causal_simt_dv<32, T>(d, q, k, v, lam, eps, S_init, z_init, out, S_final, z_final, s);
-    case 64: return causal_simt_dv<64, T>(d, q, k, v, lam, eps, S_init, z_init, out, S_final, z_final, s);
-    case 128: return causal_simt_dv<128, T>(d, q, k, v, lam, eps, S_init, z_init, out, S_final, z_final, s);
+    case 16: return causal_simt_dv<16, T>(d, q, k, v, lam, eps, S_init, z_init, out, S_final, z_final, sg, s);
+    case 32: return causal_simt_dv<32, T>(d, q, k, v, lam, eps, S_init, z_init, out, S_final, z_final, sg, s);
+    case 64: return causal_simt_dv<64, T>(d, q, k, v, lam, eps, S_init, z_init, out, S_final, z_final, sg, s);
+    case 128: return causal_simt_dv<128, T>(d, q, k, v, lam, eps, S_init, z_init, out, S_final, z_final, sg, s);
   }
   return LINATTN_ERR_UNSUPPORTED;
 }
@@ -391,7 +442,8 @@ namespace {
 // d_k = 128, dv a multiple of 64) or the CUDA-core kernel.
 int fwd_causal_impl(const linattn_dims *d, const void *q, const void *k, const void *v,
                     const float *lambda, float eps, const float *S_init, const float *z_init,
-                    void *out, float *S_final, float *z_final, cudaStream_t s) {
+                    void *out, float *S_final, float *z_final, void *ws, size_t ws_bytes,
+                    cudaStream_t s) {
   int rc = check_dims(d, true);
   if (rc != LINATTN_OK) return rc;
   if (bad_eps(eps)) return LINATTN_ERR_INVALID;
@@ -431,12 +483,27 @@ int fwd_causal_impl(const linattn_dims *d, const void *q, const void *k, const v
   }
   if (use_tc_causal(d))
     return launch_causal_tc(d, q, k, v, lambda, eps, S_init, z_init, out, S_final, z_final, s);
+  // the segment-parallel form when it pays and the workspace holds it
+  Segments sg = plan_segments(d);
+  const size_t need = segment_bytes(d, sg);
+  if (sg.G > 1 && ws && ws_bytes >= need) {
+    if (!aligned16(ws)) return LINATTN_ERR_INVALID;
+    if (overlaps(ws, need, q, nq) || overlaps(ws, need, k, nq) || overlaps(ws, need, v, nv) ||
+        overlaps(ws, need, out, nv) || overlaps(ws, need, S_final, nS) ||
+        overlaps(ws, need, z_final, nz) || overlaps(ws, need, S_init, nS) ||
+        overlaps(ws, need, z_init, nz))
+      return LINATTN_ERR_INVALID;
+    sg.ws = static_cast<float *>(ws);
+  } else {
+    sg = Segments{1, d->N, nullptr};
+  }
   if (d->dtype == LINATTN_F32)
     return causal_simt_dispatch<float>(d, q, k, v, lambda, eps, S_init, z_init, out, S_final,
-                                       z_final, s);
+                                       z_final, sg, s);
   return causal_simt_dispatch<bf16>(d, q, k, v, lambda, eps, S_init, z_init, out, S_final,
-                                    z_final, s);
+                                    z_final, sg, s);
 }
+
 
 }  // namespace
 }  // namespace linattn
@@ -445,7 +512,7 @@ extern "C" int linattn_fwd_causal(const linattn_dims *d, const void *q, const vo
                                   const void *v, const float *lambda, float eps, void *out,
                                   float *S_final, float *z_final, linattn_stream_t stream) {
   return fwd_causal_impl(d, q, k, v, lambda, eps, nullptr, nullptr, out, S_final, z_final,
-                         reinterpret_cast<cudaStream_t>(stream));
+                         nullptr, 0, reinterpret_cast<cudaStream_t>(stream));
 }
 
 extern "C" int linattn_fwd_causal_from(const linattn_dims *d, const void *q, const void *k,
@@ -453,8 +520,23 @@ extern "C" int linattn_fwd_causal_from(const linattn_dims *d, const void *q, con
                                        const float *S_init, const float *z_init, void *out,
                                        float *S_final, float *z_final, linattn_stream_t stream) {
   return fwd_causal_impl(d, q, k, v, lambda, eps, S_init, z_init, out, S_final, z_final,
-                         reinterpret_cast<cudaStream_t>(stream));
+                         nullptr, 0, reinterpret_cast<cudaStream_t>(stream));
 }
+
+extern "C" size_t linattn_fwd_causal_workspace(const linattn_dims *d) {
+  if (check_dims(d, true) != LINATTN_OK || d->B == 0 || d->H == 0 || d->N == 0) return 0;
+  return segment_bytes(d, plan_segments(d));
+}
+
+extern "C" int linattn_fwd_causal_ws(const linattn_dims *d, const void *q, const void *k,
+                                     const void *v, const float *lambda, float eps,
+                                     const float *S_init, const float *z_init, void *out,
+                                     float *S_final, float *z_final, void *workspace,
+                                     size_t workspace_bytes, linattn_stream_t stream) {
+  return fwd_causal_impl(d, q, k, v, lambda, eps, S_init, z_init, out, S_final, z_final,
+                         workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
 
 extern "C" int linattn_bwd_causal(const linattn_dims *d, const void *q, const void *k,
                                   const void *v, const float *lambda, float eps, const void *dy,

@@ -26,7 +26,8 @@ LINATTN_ERR_UNSUPPORTED = 2
 LINATTN_ERR_CUDA = 3
 LINATTN_ERR_DEVICE = 4
 
-ENTRY_POINTS = ("linattn_fwd_causal", "linattn_fwd_causal_from", "linattn_bwd_causal",
+ENTRY_POINTS = ("linattn_fwd_causal", "linattn_fwd_causal_from", "linattn_fwd_causal_workspace",
+                "linattn_fwd_causal_ws", "linattn_bwd_causal",
                 "linattn_fwd_global", "linattn_fwd_global_cross", "linattn_decode_step",
                 "linattn_status_string", "linattn_device_status", "linattn_version")
 
@@ -67,6 +68,11 @@ def load(build_if_missing: bool = True):
     lib.linattn_fwd_causal.restype = i
     lib.linattn_fwd_causal_from.argtypes = [dp, vp, vp, vp, fp, f, fp, fp, vp, fp, fp, vp]
     lib.linattn_fwd_causal_from.restype = i
+    lib.linattn_fwd_causal_workspace.argtypes = [dp]
+    lib.linattn_fwd_causal_workspace.restype = ctypes.c_size_t
+    lib.linattn_fwd_causal_ws.argtypes = [dp, vp, vp, vp, fp, f, fp, fp, vp, fp, fp, vp,
+                                          ctypes.c_size_t, vp]
+    lib.linattn_fwd_causal_ws.restype = i
     lib.linattn_bwd_causal.argtypes = [dp, vp, vp, vp, fp, f, vp, vp, vp, vp, fp, vp]
     lib.linattn_bwd_causal.restype = i
     lib.linattn_fwd_global.argtypes = [dp, vp, vp, vp, f, vp, fp, fp, vp]
@@ -163,6 +169,38 @@ def linattn_fwd_causal_from(q, k, v, lam, eps, S_init, z_init, out, S_final=None
                                           float(eps), _ptr(S_init), _ptr(z_init), _ptr(out),
                                           _ptr(S_final), _ptr(z_final), _stream(stream)),
            "linattn_fwd_causal_from")
+
+
+def _causal_dims(q, k, v, out, S_final, z_final, lam):
+    B, H, N, dk = q.shape
+    dv = v.shape[-1]
+    if k.shape != q.shape or tuple(v.shape) != (B, H, N, dv) or out.shape != v.shape:
+        raise ValueError("shape mismatch among q, k, v, out")
+    if not (q.dtype == k.dtype == v.dtype == out.dtype):
+        raise ValueError("q, k, v, out must share one dtype")
+    _f32(lam, (H,), "lambda")
+    _f32(S_final, (B, H, dk, dv), "S_final")
+    _f32(z_final, (B, H, dk), "z_final")
+    return linattn_dims(B, H, N, dk, dv, _dtype_code(q.dtype))
+
+
+def linattn_fwd_causal_workspace(B, H, N, dk, dv, dtype) -> int:
+    """Workspace bytes the segment-parallel causal forward wants (0: none)."""
+    d = linattn_dims(B, H, N, dk, dv, _dtype_code(dtype))
+    return int(load().linattn_fwd_causal_workspace(ctypes.byref(d)))
+
+
+def linattn_fwd_causal_ws(q, k, v, lam, eps, S_init, z_init, out, S_final, z_final, workspace,
+                          stream=None):
+    """Causal forward (optionally from S_init, z_init) with a caller workspace:
+    a CUDA tensor of at least linattn_fwd_causal_workspace bytes, or None."""
+    d = _causal_dims(q, k, v, out, S_final, z_final, lam)
+    nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(load().linattn_fwd_causal_ws(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), _ptr(lam),
+                                        float(eps), _ptr(S_init), _ptr(z_init), _ptr(out),
+                                        _ptr(S_final), _ptr(z_final), _ptr(workspace),
+                                        ctypes.c_size_t(nbytes), _stream(stream)),
+           "linattn_fwd_causal_ws")
 
 
 def linattn_bwd_causal(q, k, v, lam, eps, dy, dq, dk, dv, dlam=None, stream=None):
