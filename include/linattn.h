@@ -144,6 +144,18 @@ LINATTN_API int linattn_fwd_causal_ws(const linattn_dims *dims, const void *q, c
                        size_t workspace_bytes, linattn_stream_t stream);
 
 /*
+ * linattn_fwd_causal (zero starting state) without a caller workspace: the
+ * segmented form uses a 16 MB device array that the library holds for every
+ * device it is loaded on, and falls back to the single pass when the
+ * workspace it needs is larger.  That array is shared by all calls of this
+ * entry point on one device, so those calls must be ordered (one stream, or
+ * streams ordered by events); it is the only memory the library owns.
+ */
+LINATTN_API int linattn_fwd_causal_noalloc(const linattn_dims *dims, const void *q, const void *k,
+                       const void *v, const float *lambda, float eps, void *out,
+                       float *S_final, float *z_final, linattn_stream_t stream);
+
+/*
  * Backward of linattn_fwd_causal (zero starting state): the gradients of
  * L = sum over all (b, h, i) of dy_i . y_i ([FW] §3.1 and §4.1 train the
  * chunked forward; the gradients follow from the recurrence of [FW] §2.1,

@@ -504,6 +504,21 @@ int fwd_causal_impl(const linattn_dims *d, const void *q, const void *k, const v
                                     z_final, sg, s);
 }
 
+// Scratch of the no-allocation entry point: a static device array (one per
+// device the library is loaded on), its address looked up once per device.
+constexpr size_t kScratchBytes = size_t(16) << 20;
+__device__ __align__(256) unsigned char g_causal_scratch[kScratchBytes];
+
+void *scratch_address() {
+  static void *addr[64] = {};
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev] && cudaGetSymbolAddress(&addr[dev], g_causal_scratch) != cudaSuccess)
+    addr[dev] = nullptr;
+  return addr[dev];
+}
 
 }  // namespace
 }  // namespace linattn
@@ -537,6 +552,14 @@ extern "C" int linattn_fwd_causal_ws(const linattn_dims *d, const void *q, const
                          workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
 }
 
+extern "C" int linattn_fwd_causal_noalloc(const linattn_dims *d, const void *q, const void *k,
+                                          const void *v, const float *lambda, float eps,
+                                          void *out, float *S_final, float *z_final,
+                                          linattn_stream_t stream) {
+  void *ws = scratch_address();
+  return fwd_causal_impl(d, q, k, v, lambda, eps, nullptr, nullptr, out, S_final, z_final, ws,
+                         ws ? kScratchBytes : 0, reinterpret_cast<cudaStream_t>(stream));
+}
 
 extern "C" int linattn_bwd_causal(const linattn_dims *d, const void *q, const void *k,
                                   const void *v, const float *lambda, float eps, const void *dy,

@@ -27,7 +27,7 @@ LINATTN_ERR_CUDA = 3
 LINATTN_ERR_DEVICE = 4
 
 ENTRY_POINTS = ("linattn_fwd_causal", "linattn_fwd_causal_from", "linattn_fwd_causal_workspace",
-                "linattn_fwd_causal_ws", "linattn_bwd_causal",
+                "linattn_fwd_causal_ws", "linattn_fwd_causal_noalloc", "linattn_bwd_causal",
                 "linattn_fwd_global", "linattn_fwd_global_cross", "linattn_decode_step",
                 "linattn_status_string", "linattn_device_status", "linattn_version")
 
@@ -73,6 +73,8 @@ def load(build_if_missing: bool = True):
     lib.linattn_fwd_causal_ws.argtypes = [dp, vp, vp, vp, fp, f, fp, fp, vp, fp, fp, vp,
                                           ctypes.c_size_t, vp]
     lib.linattn_fwd_causal_ws.restype = i
+    lib.linattn_fwd_causal_noalloc.argtypes = [dp, vp, vp, vp, fp, f, vp, fp, fp, vp]
+    lib.linattn_fwd_causal_noalloc.restype = i
     lib.linattn_bwd_causal.argtypes = [dp, vp, vp, vp, fp, f, vp, vp, vp, vp, fp, vp]
     lib.linattn_bwd_causal.restype = i
     lib.linattn_fwd_global.argtypes = [dp, vp, vp, vp, f, vp, fp, fp, vp]
@@ -201,6 +203,15 @@ def linattn_fwd_causal_ws(q, k, v, lam, eps, S_init, z_init, out, S_final, z_fin
                                         _ptr(S_final), _ptr(z_final), _ptr(workspace),
                                         ctypes.c_size_t(nbytes), _stream(stream)),
            "linattn_fwd_causal_ws")
+
+
+def linattn_fwd_causal_noalloc(q, k, v, lam, eps, out, S_final=None, z_final=None, stream=None):
+    """linattn_fwd_causal whose segment-parallel form uses the library's own scratch."""
+    d = _causal_dims(q, k, v, out, S_final, z_final, lam)
+    _check(load().linattn_fwd_causal_noalloc(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v),
+                                             _ptr(lam), float(eps), _ptr(out), _ptr(S_final),
+                                             _ptr(z_final), _stream(stream)),
+           "linattn_fwd_causal_noalloc")
 
 
 def linattn_bwd_causal(q, k, v, lam, eps, dy, dq, dk, dv, dlam=None, stream=None):
