@@ -87,6 +87,7 @@ constexpr int C = 128;      // tokens per chunk
 constexpr int DK = 128;     // key dimension handled by this kernel
 constexpr int DVS = 64;     // dv columns per CTA
 constexpr int NT = 768;
+constexpr int kPrefetch = 2;   // chunks ahead that the producers prefetch into L2
 
 // phi transform: warps 3-7 and 16-23
 constexpr int kXformThreads = 416;
@@ -418,11 +419,21 @@ __global__ void __launch_bounds__(NT, 1)
           tma_load_3d(base + kOffK + own_off, &tm_k, b, 0, y, pair);
           tma_load_3d(base + kOffQ + kPanel + own_off, &tm_q, b, 64, y, pair);
           tma_load_3d(base + kOffK + kPanel + own_off, &tm_k, b, 64, y, pair);
+          // the same rows two chunks ahead into L2, so that their load, issued
+          // when this stage frees up again, does not wait on HBM
+          if (c + kPrefetch < nchunks) {
+            const int yp = y + kPrefetch * C;
+            tma_prefetch_l2_3d(&tm_q, 0, yp, pair);
+            tma_prefetch_l2_3d(&tm_k, 0, yp, pair);
+            tma_prefetch_l2_3d(&tm_q, 64, yp, pair);
+            tma_prefetch_l2_3d(&tm_k, 64, yp, pair);
+          }
           LINATTN_TRACE_EVENT(c, 0);
         } else {
           const uint32_t b = bar(kFullV0 + s);
           mbar_arrive_expect_tx(b, kVTxBytes);
           tma_load_3d(base + kOffV, &tm_v, b, j0, c * C, pair);
+          if (c + kPrefetch < nchunks) tma_prefetch_l2_3d(&tm_v, j0, (c + kPrefetch) * C, pair);
         }
         issued = c + 1;
       }
