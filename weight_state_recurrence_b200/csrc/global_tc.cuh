@@ -145,6 +145,9 @@ __global__ void __launch_bounds__(kv::NT, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // the output kernel may start its CTAs on SMs this grid leaves (its q tiles
+  // and phi(q) do not depend on KV; it waits for this grid before reading KV)
+  grid_launch_dependents();
   // unit i of this CTA: pair u / nchunks, chunk u % nchunks; a segment is a run
   // of units of one pair; the accumulator is flushed at the end of a segment
   auto pair_of = [&](int i) { return static_cast<int>((u0 + i) / nchunks); };
@@ -238,6 +241,7 @@ __global__ void __launch_bounds__(kv::NT, 1)
         }
         tc_fence_after();
         if (ok && warp < 8) {
+          grid_dependency_wait();   // KV and ksum have been zeroed
           const int row = (warp - 4) * 32 + lane;
           const int hsel = row >> 6, kk = row & 63;
           const long bh = 2L * pair_of(i) + hsel;
@@ -407,7 +411,9 @@ __global__ void __launch_bounds__(out::NT, 1)
       const int d = i & 1;
       if (seg_start(i)) {
         // every earlier MMA has completed (its tile was consumed below), so
-        // the operand can be rewritten: KV rows = d_k (K), 64 columns (N)
+        // the operand can be rewritten: KV rows = d_k (K), 64 columns (N);
+        // KV and ksum are complete once the KV grid has finished
+        grid_dependency_wait();
         const long bh = head_of(i);
         if (r < D) {
           const float *src = KV + (bh * D + r) * D;
@@ -476,6 +482,22 @@ __global__ void __launch_bounds__(out::NT, 1)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmCols);
+  }
+}
+
+// KV and ksum to zero before the KV kernel accumulates into them (one launch
+// for both buffers; the KV kernel may start while this runs and waits for it
+// only before its first flush)
+__global__ void __launch_bounds__(256) zero2_kernel(float4 *__restrict__ a, long na4,
+                                                    float4 *__restrict__ b, long nb4) {
+  grid_launch_dependents();
+  const long stride = static_cast<long>(gridDim.x) * blockDim.x;
+  const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (long i = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x; i < na4 + nb4; i += stride) {
+    if (i < na4)
+      a[i] = z;
+    else
+      b[i - na4] = z;
   }
 }
 

@@ -335,6 +335,36 @@ bool use_tc_global(const linattn_dims *d) {
   return d->dtype == LINATTN_BF16 && d->dk == gtc::D && d->dv == gtc::D && d->H % 2 == 0;
 }
 
+// Launch configuration with programmatic stream serialization: the grid may
+// begin before the previous grid of the stream has finished, and orders
+// itself after it with griddepcontrol.wait where it reads that grid's output.
+struct ProgrammaticLaunch {
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  ProgrammaticLaunch(int grid, int block, size_t smem, cudaStream_t s) {
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  }
+};
+
+// KV and ksum to zero in one launch
+int zero_kv(float *KV, size_t nS, float *ksum, size_t nz, cudaStream_t s) {
+  const long n4 = static_cast<long>((nS + nz) / 16);
+  const int sms = num_sms();
+  const long blocks = std::min<long>((n4 + 255) / 256, 4L * (sms > 0 ? sms : 148));
+  if (blocks <= 0) return LINATTN_OK;
+  gtc::zero2_kernel<<<static_cast<int>(blocks), 256, 0, s>>>(
+      reinterpret_cast<float4 *>(KV), static_cast<long>(nS / 16), reinterpret_cast<float4 *>(ksum),
+      static_cast<long>(nz / 16));
+  return cudaGetLastError() == cudaSuccess ? LINATTN_OK : LINATTN_ERR_CUDA;
+}
+
 int launch_global_tc(const linattn_dims *d, int Nk, const void *q, const void *k,
                      const void *v, float eps, void *out, float *KV, float *ksum,
                      cudaStream_t s) {
@@ -350,17 +380,27 @@ int launch_global_tc(const linattn_dims *d, int Nk, const void *q, const void *k
     if (!make_map_bf16(&mk, k, d->dk, Nk, BH) || !make_map_bf16(&mv, v, d->dv, Nk, BH))
       return LINATTN_ERR_CUDA;
     const long u1 = static_cast<long>(BH / 2) * ((Nk + gtc::C - 1) / gtc::C);
-    gtc::global_kv_tc_kernel<<<static_cast<int>(u1 < sms ? u1 : sms), gtc::kv::NT,
-                               gtc::kv::kSmemBytes, s>>>(mk, mv, KV, ksum, BH / 2, Nk);
-    if (cudaGetLastError() != cudaSuccess) return LINATTN_ERR_CUDA;
+    // programmatic dependent launch: the KV grid may start while KV / ksum are
+    // being zeroed; it waits for that grid only before its first flush
+    const ProgrammaticLaunch pl(static_cast<int>(u1 < sms ? u1 : sms), gtc::kv::NT,
+                                gtc::kv::kSmemBytes, s);
+    if (cudaLaunchKernelEx(&pl.cfg, gtc::global_kv_tc_kernel, mk, mv, KV, ksum, BH / 2, Nk) !=
+        cudaSuccess)
+      return LINATTN_ERR_CUDA;
   }
   if (d->N > 0) {
     CUtensorMap mq, my;
     if (!make_map_bf16(&mq, q, d->dk, d->N, BH) || !make_map_bf16(&my, out, d->dv, d->N, BH))
       return LINATTN_ERR_CUDA;
     const long u2 = static_cast<long>(BH) * ((d->N + gtc::C - 1) / gtc::C);
-    gtc::global_out_tc_kernel<<<static_cast<int>(u2 < sms ? u2 : sms), gtc::out::NT,
-                                gtc::out::kSmemBytes, s>>>(mq, my, KV, ksum, eps, BH, d->N);
+    // the output grid loads q and applies phi while the KV grid drains; it
+    // waits for that grid only before reading KV and ksum
+    const ProgrammaticLaunch pl(static_cast<int>(u2 < sms ? u2 : sms), gtc::out::NT,
+                                gtc::out::kSmemBytes, s);
+    if (cudaLaunchKernelEx(&pl.cfg, gtc::global_out_tc_kernel, mq, my,
+                           static_cast<const float *>(KV), static_cast<const float *>(ksum), eps,
+                           BH, d->N) != cudaSuccess)
+      return LINATTN_ERR_CUDA;
   }
   return launch_status();
 }
@@ -627,8 +667,7 @@ int fwd_global_impl(const linattn_dims *d, int Nk, const void *q, const void *k,
       overlaps(KV, nS, k, nk) || overlaps(KV, nS, v, nv) || overlaps(KV, nS, q, nq) ||
       overlaps(ksum, nz, q, nq) || overlaps(ksum, nz, k, nk) || overlaps(ksum, nz, v, nv))
     return LINATTN_ERR_INVALID;
-  if (cudaMemsetAsync(KV, 0, nS, s) != cudaSuccess) return LINATTN_ERR_CUDA;
-  if (cudaMemsetAsync(ksum, 0, nz, s) != cudaSuccess) return LINATTN_ERR_CUDA;
+  if ((rc = zero_kv(KV, nS, ksum, nz, s)) != LINATTN_OK) return rc;
   if (d->N == 0 && Nk == 0) return LINATTN_OK;
   if (use_tc_global(d)) return launch_global_tc(d, Nk, q, k, v, eps, out, KV, ksum, s);
   if (d->dtype == LINATTN_F32)

@@ -102,6 +102,20 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_
       : "memory");
 }
 
+// ------------------------------------------------ programmatic dependent launch
+// Blocks until every grid this one depends on (launched before it with
+// programmatic stream serialization) has completed and its writes are
+// visible; returns at once for a grid launched without that dependency.
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// Lets the next grid of the stream (if launched with programmatic stream
+// serialization) start its CTAs as this grid's CTAs leave the SMs.
+__device__ __forceinline__ void grid_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ------------------------------------------------------------------ cluster
 __device__ __forceinline__ uint32_t cluster_ctarank() {
   uint32_t r;
