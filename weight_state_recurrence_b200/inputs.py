@@ -119,3 +119,59 @@ def decode_step_inputs(w: Workload, step: int, B=None, H=None, device="cpu"):
 def random_case(seed, B, H, N, dk, dv, dtype=torch.float32, scale=1.0, device="cpu"):
     """Generic seeded case for edge-shape tests (d_k may differ from d_v)."""
     return qkv((B, H, N, dk), (B, H, N, dv), seed, scale, dtype, device)
+
+
+# Performer workload: the fast-weight recurrence on random trig features
+# (linear-attention note §4.2) of q and k.  Raw q, k are N(0, 1/(4d)) (scale
+# 1/(2 sqrt d)), so |omega.(q-k)| stays near 0.7 rad and the m = 64 estimate of
+# the kernel is well conditioned; v is N(0, 1/d) like the other bf16 workloads.
+PERFORMER = {
+    "performer_d128": dict(B=4, H=16, N=16384, d=128, m=64, seed=6, lam_lo=0.9,
+                           lam_hi=0.999, dtype=torch.bfloat16),
+}
+
+
+def performer_omega(m, d, seed, orthogonal=True, dtype=torch.float32, device="cpu"):
+    """Projection ``[m, d]`` for the Performer feature map: every row is
+    marginally N(0, I_d) (linear-attention note §4.2: omega drawn from the
+    standard normal, with a fixed seed shared by all processes).
+
+    ``orthogonal`` draws the rows in blocks of d that are mutually orthogonal
+    (the note's orthogonalised omega): each block is Q^T of the QR factors of a
+    d x d Gaussian matrix, with Q's columns sign-fixed by diag(R) so the block
+    is Haar-distributed, and each row rescaled by the norm of an independent
+    N(0, I_d) vector.  The last block keeps its first m mod d rows.  The
+    result is rounded once to ``dtype``."""
+    gen = torch.Generator(device="cpu")
+    gen.manual_seed(int(seed))
+    if not orthogonal:
+        w = torch.randn((m, d), generator=gen, dtype=torch.float64)
+    else:
+        blocks = []
+        for _ in range((m + d - 1) // d):
+            G = torch.randn((d, d), generator=gen, dtype=torch.float64)
+            Q, R = torch.linalg.qr(G)
+            Q = Q * torch.sign(torch.diagonal(R))[None, :]
+            norms = torch.randn((d, d), generator=gen, dtype=torch.float64).norm(dim=1)
+            blocks.append(Q.T * norms[:, None])
+        w = torch.cat(blocks, 0)[:m]
+    return w.to(dtype).contiguous().to(device)
+
+
+def performer_inputs(name, B=None, H=None, N=None, device="cpu"):
+    """q, k ``[B, H, N, d]``, v ``[B, H, N, d]``, lambda ``[H]`` and omega
+    ``[m, d]`` (same dtype as q) of a Performer workload."""
+    p = PERFORMER[name]
+    B = p["B"] if B is None else B
+    H = p["H"] if H is None else H
+    N = p["N"] if N is None else N
+    d = p["d"]
+    gen = torch.Generator(device=device)
+    gen.manual_seed(int(p["seed"]))
+    shape = (B, H, N, d)
+    q = _draw(gen, shape, 0.5 / math.sqrt(d), p["dtype"], device)
+    k = _draw(gen, shape, 0.5 / math.sqrt(d), p["dtype"], device)
+    v = _draw(gen, shape, 1.0 / math.sqrt(d), p["dtype"], device)
+    lam = torch.linspace(p["lam_lo"], p["lam_hi"], H, dtype=torch.float32)
+    omega = performer_omega(p["m"], d, p["seed"] + 1, True, p["dtype"], device)
+    return q, k, v, lam, omega
