@@ -13,7 +13,8 @@ over ranks.  Inputs (805 MB per step) are larger than the 126 MB L2.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                   [--no-e2e] [--no-legs] [--no-cpu-baseline]
-                  [--only causal|decode|global] [--batch B] [--dec-batch B]
+                  [--only causal|decode|global|backward|segmented|performer]
+                  [--batch B] [--dec-batch B]
                   [--dec-steps T]
 The last four options shrink or isolate a leg for profiler captures; the
 reported benchmark always uses the full workloads (their defaults).
@@ -444,6 +445,70 @@ def bwd_leg(lib, args, world, rank, stream, alu_peak):
     return res
 
 
+def features_bytes(rows, d, m, es=2):
+    """Algorithmic HBM bytes of one feature launch: x read, 2m features written,
+    omega read once."""
+    return rows * (d + 2 * m) * es + m * d * es
+
+
+def performer_leg(lib, args, world, rank, stream, hbm):
+    """Causal attention on Performer random features (performer_d128: B=4 x
+    H=16 x N=16384, d=128, m=64 orthogonal features, bf16, decay): the
+    feature kernel on q and on k, then the causal forward in identity mode on
+    the 128 features.  The feature kernel is also timed alone."""
+    p = inputs.PERFORMER["performer_d128"]
+    B = args.batch or p["B"]
+    H, N, d, m = p["H"], p["N"], p["d"], p["m"]
+    dev = torch.device("cuda")
+    q, k, v, lam, w = inputs.performer_inputs("performer_d128", B=B, device=dev)
+    lam = lam.to(dev)
+    fq = torch.empty(B, H, N, 2 * m, dtype=q.dtype, device=dev)
+    fk = torch.empty_like(fq)
+    out = torch.empty_like(v)
+    S = torch.empty(B, H, 2 * m, d, device=dev)
+    z = torch.empty(B, H, 2 * m, device=dev)
+    K = lib.LINATTN_PERFORMER_SOFTMAX
+
+    def feat_q():
+        lib.linattn_performer_features(q, w, K, fq, stream)
+
+    def step():
+        lib.linattn_performer_features(q, w, K, fq, stream)
+        lib.linattn_performer_features(k, w, K, fk, stream)
+        lib.linattn_fwd_causal(fq, fk, v, lam, 1e-6, out, S, z, stream,
+                               phi=lib.LINATTN_PHI_IDENTITY)
+
+    def attn():
+        lib.linattn_fwd_causal(fq, fk, v, lam, 1e-6, out, S, z, stream,
+                               phi=lib.LINATTN_PHI_IDENTITY)
+
+    with torch.cuda.stream(stream):
+        ms = time_steps(step, args.steps, args.warmup, world, stream)
+        ms_f = time_steps(feat_q, args.steps, args.warmup, world, stream)
+        ms_a = time_steps(attn, args.steps, args.warmup, world, stream)
+    assert lib.linattn_device_status(clear=True, stream=stream) == 0
+    per, per_f, per_a = (x / 1e3 / args.steps for x in (ms, ms_f, ms_a))
+    fb = features_bytes(B * H * N, d, m)
+    ab = causal_bytes(B, H, N, 2 * m, d)
+    res = {"workload": f"performer_d128: B={B} x H={H} x N={N}, d={d}, m={m} orthogonal "
+                       "features (softmax kernel), bf16, lambda_h=linspace(0.9,0.999,16)",
+           "value": B * N * world / per, "unit": "tokens/s", "ms_per_step": per * 1e3,
+           "gpu_launches_per_step": 3,
+           "features": {"kernel": "performer_tc_kernel", "ms_per_launch": per_f * 1e3,
+                        "roofline": {"bound": "hbm", "achieved": fb / per_f / 1e9, "peak": hbm,
+                                     "unit": "GB/s", "frac": fb / per_f / 1e9 / hbm,
+                                     "algorithmic_bytes_per_launch": fb,
+                                     "traffic": traffic_record("performer_tc_kernel")}},
+           "attention": {"kernel": "causal_tc_kernel (identity features)",
+                         "ms_per_launch": per_a * 1e3,
+                         "roofline": {"bound": "hbm", "achieved": ab / per_a / 1e9, "peak": hbm,
+                                      "unit": "GB/s", "frac": ab / per_a / 1e9 / hbm,
+                                      "algorithmic_bytes_per_launch": ab}}}
+    del q, k, v, fq, fk, out
+    torch.cuda.empty_cache()
+    return res
+
+
 # ---------------------------------------------------------------- oracle
 def oracle_sample(target_s=12.0, heads=None):
     """Times the fp64 oracle (as it stands) on a bounded sample of the causal
@@ -509,7 +574,8 @@ def main():
     ap.add_argument("--no-legs", dest="legs", action="store_false")
     ap.add_argument("--no-cpu-baseline", dest="cpu", action="store_false")
     ap.add_argument("--only", default="all",
-                    choices=["all", "causal", "decode", "global", "backward", "segmented"])
+                    choices=["all", "causal", "decode", "global", "backward", "segmented",
+                             "performer"])
     ap.add_argument("--batch", type=int, default=0, help="causal leg batch (profiling)")
     ap.add_argument("--dec-batch", type=int, default=0, help="decode sequences (profiling)")
     ap.add_argument("--dec-steps", type=int, default=0, help="decode steps (profiling)")
@@ -525,8 +591,10 @@ def main():
     hbm, tcp, peak_src = peaks()
     stream = torch.cuda.Stream()
 
-    if args.only in ("decode", "global", "backward", "segmented"):
-        if args.only == "backward":
+    if args.only in ("decode", "global", "backward", "segmented", "performer"):
+        if args.only == "performer":
+            r = performer_leg(lib, args, world, rank, stream, hbm)
+        elif args.only == "backward":
             r = bwd_leg(lib, args, world, rank, stream, ALU_PEAK_TFLOPS)
         elif args.only == "segmented":
             r = seg_leg(lib, args, world, rank, stream, hbm)
@@ -560,6 +628,7 @@ def main():
         line["global"] = global_leg(lib, args, world, rank, stream, hbm)
         line["backward"] = bwd_leg(lib, args, world, rank, stream, ALU_PEAK_TFLOPS)
         line["segmented"] = seg_leg(lib, args, world, rank, stream, hbm)
+        line["performer"] = performer_leg(lib, args, world, rank, stream, hbm)
     if args.cpu and world == 1 and rank == 0:
         tok_s, cores, desc, _ = oracle_sample()
         line["cpu_baseline"] = {"value": tok_s, "unit": "tokens/s", "cores": cores,

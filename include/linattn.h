@@ -20,8 +20,11 @@
  *     orientation); z [B, H, dk].  Decode uses N = 1 and drops that axis.
  *   - q, k, v and out share one element type (dims.dtype); S, z, KV and ksum
  *     are always fp32 ([FW] §4.1: the accumulated state must stay fp32).
- *   - q and k are passed raw: phi is applied inside the library.  Any
- *     1/sqrt(d) scaling is part of the caller's data, not of the operation.
+ *   - q and k are passed raw: phi is applied inside the library (dims.phi =
+ *     LINATTN_PHI_ELU1), or they are feature vectors already
+ *     (LINATTN_PHI_IDENTITY; the backward then returns gradients with respect
+ *     to those features).  Any 1/sqrt(d) scaling is part of the caller's
+ *     data, not of the operation.
  *   - lambda points to H fp32 values in device memory (one decay per head),
  *     or is NULL for lambda = 1 (no decay).  Values are used as given; the
  *     method assumes 0 <= lambda <= 1 ([FW] §3.2).  lambda = 0 is allowed
@@ -62,6 +65,14 @@ typedef struct CUstream_st *linattn_stream_t;
 
 typedef enum { LINATTN_BF16 = 0, LINATTN_F32 = 1 } linattn_dtype;
 
+/* Feature map the attention calls apply to q and k. */
+typedef enum {
+    LINATTN_PHI_ELU1 = 0,     /* phi(x) = elu(x) + 1, elementwise (the default) */
+    LINATTN_PHI_IDENTITY = 1  /* q and k already hold feature vectors of length dk, e.g. the
+                                 random features of linattn_performer_features; they may be
+                                 negative, so the denominator may be too */
+} linattn_phi;
+
 typedef struct {
     int B;      /* batch */
     int H;      /* heads */
@@ -69,6 +80,7 @@ typedef struct {
     int dk;     /* key / feature dimension */
     int dv;     /* value dimension */
     int dtype;  /* linattn_dtype of q, k, v and out */
+    int phi;    /* linattn_phi; zero-initialised dims mean elu + 1 */
 } linattn_dims;
 
 enum {
@@ -220,6 +232,32 @@ LINATTN_API int linattn_decode_step(const linattn_dims *dims, const void *q, con
                         float *z, void *out, linattn_stream_t stream);
 
 /* Static English text for a status code (never NULL). */
+/*
+ * Performer random features ([LN] §4.2), the feature map to pair with
+ * dims.phi = LINATTN_PHI_IDENTITY.  For every row x of x:
+ *   out = g(x) / sqrt(m) [cos(omega_1.x) .. cos(omega_m.x), sin(omega_1.x) .. sin(omega_m.x)]
+ *   kernel LINATTN_PERFORMER_SOFTMAX:  g(x) = exp(|x|^2 / 2)   (h = 1; phi(x).phi(y)
+ *                                      is an unbiased estimate of exp(x.y))
+ *   kernel LINATTN_PERFORMER_GAUSSIAN: g(x) = 1   (h(x) = exp(-|x|^2/2), the note's example;
+ *                                      the estimate is of exp(-|x-y|^2 / 2))
+ *   x     [rows, d]   dtype   e.g. q or k of shape [B, H, N, d] with rows = B*H*N
+ *   omega [m, d]      dtype   the projection, drawn by the caller ([LN] §4.2: rows from
+ *                             N(0, I_d), optionally orthogonalised, one fixed seed shared by
+ *                             every process); the library draws no random numbers
+ *   out   [rows, 2m]  dtype   the m cosines, then the m sines
+ * d in {16, 32, 64, 128}; m in {8, 16, 32, 64}, so 2m is a supported dk of the attention
+ * calls; rows >= 0 with rows * max(d, 2m) < 2^31.  bf16 forms omega.x from the bf16 values
+ * with fp32 accumulation (tensor cores when d is 64 or 128 and m is 32 or 64) and rounds
+ * the features to bf16; fp32 computes in fp32.  With the softmax kernel g grows as
+ * exp(|x|^2 / 2) and overflows to inf for |x|^2 above about 177: keep x small (Performer
+ * scales q and k by d^-1/4 before the map).  out must not overlap x or omega; with rows = 0
+ * nothing is read or written and the pointers may be NULL.
+ */
+enum { LINATTN_PERFORMER_SOFTMAX = 0, LINATTN_PERFORMER_GAUSSIAN = 1 };
+LINATTN_API int linattn_performer_features(long long rows, int d, int m, int kernel, int dtype,
+                                           const void *x, const void *omega, void *out,
+                                           linattn_stream_t stream);
+
 LINATTN_API const char *linattn_status_string(int status);
 
 /*

@@ -16,6 +16,9 @@ with phi(x) = x + 1 for x > 0 and e^x otherwise (elu + 1).  torch autograd on
 that expression gives the gradients of L = sum(dy * y) with respect to q, k,
 v and the per-head lambda (summed over the batch).  The tests pin it with
 central differences of the C oracle's forward, which shares no code with it.
+With ``identity`` q and k are feature vectors already (phi is the identity,
+as for random features); that mode is pinned by central differences of the
+numpy recurrence on features in ``oracle/performer.py``.
 """
 from __future__ import annotations
 
@@ -41,24 +44,26 @@ def _decay_mask(lam: torch.Tensor, N: int) -> torch.Tensor:
     return torch.where((i[:, None] >= i[None, :])[None], W, torch.zeros((), dtype=lam.dtype))
 
 
-def causal_forward(q, k, v, lam, eps):
+def causal_forward(q, k, v, lam, eps, identity=False):
     """y [B, H, N, dv] of the masked form (torch float64, differentiable)."""
     N = q.shape[-2]
     W = _decay_mask(lam, N)[None]                     # [1, H, N, N]
-    A = (_phi(q) @ _phi(k).transpose(-1, -2)) * W
+    f = (lambda x: x) if identity else _phi
+    A = (f(q) @ f(k).transpose(-1, -2)) * W
     return (A @ v) / (A.sum(-1, keepdim=True) + eps)
 
 
-def causal_grad(q, k, v, lam, eps, dy):
+def causal_grad(q, k, v, lam, eps, dy, identity=False):
     """Returns numpy float64 (y, dq, dk, dv, dlam) for L = sum(dy * y).
-    ``lam`` [H] or None (no decay: dlam is then None)."""
+    ``lam`` [H] or None (no decay: dlam is then None); ``identity``: q and k
+    are feature vectors (no elu + 1)."""
     t = lambda a: torch.as_tensor(np.asarray(a, dtype=np.float64) if not torch.is_tensor(a)
                                   else a.detach().to(torch.float64).cpu().numpy())
     qd, kd, vd, dyd = (t(a).clone().requires_grad_(True) for a in (q, k, v, dy))
     H = qd.shape[1]
     want_lam = lam is not None
     lamd = t(lam).clone().requires_grad_(True) if want_lam else torch.ones(H, dtype=torch.float64)
-    y = causal_forward(qd, kd, vd, lamd, float(eps))
+    y = causal_forward(qd, kd, vd, lamd, float(eps), identity)
     (y * dyd.detach()).sum().backward()
     dlam = lamd.grad.numpy() if want_lam else None
     return (y.detach().numpy(), qd.grad.numpy(), kd.grad.numpy(), vd.grad.numpy(), dlam)

@@ -185,3 +185,44 @@ def test_python_binding_checks_shapes():
     q = torch.zeros(1, 2, 4, 64)
     with pytest.raises(ValueError):
         linattn.linattn_fwd_causal(q, q, torch.zeros(1, 2, 5, 64), None, 1e-6, q)
+
+
+def test_phi_field_is_checked(lib):
+    d = D()
+    d.phi = 2
+    assert causal(lib, d) == linattn.LINATTN_ERR_UNSUPPORTED
+    d.phi = -1
+    assert causal(lib, d) == linattn.LINATTN_ERR_UNSUPPORTED
+    # identity features still go through the other checks
+    d = D(dk=48)
+    d.phi = linattn.LINATTN_PHI_IDENTITY
+    assert causal(lib, d) == linattn.LINATTN_ERR_UNSUPPORTED
+    assert ctypes.sizeof(linattn.linattn_dims) == 7 * 4
+
+
+def feats(lib, rows=16, d=64, m=32, kernel=0, dtype=0, x=FAKE, w=FAKE2, out=FAKE3):
+    return lib.linattn_performer_features(rows, d, m, kernel, dtype, x, w, out, None)
+
+
+def test_performer_features_rejects_bad_arguments(lib):
+    E_INV, E_UNS = linattn.LINATTN_ERR_INVALID, linattn.LINATTN_ERR_UNSUPPORTED
+    assert feats(lib, rows=-1) == E_INV
+    assert feats(lib, d=48) == E_UNS
+    assert feats(lib, d=256) == E_UNS
+    assert feats(lib, m=128) == E_UNS          # 2m would exceed the attention's dk
+    assert feats(lib, m=12) == E_UNS
+    assert feats(lib, kernel=2) == E_UNS
+    assert feats(lib, dtype=5) == E_UNS
+    assert feats(lib, rows=1 << 25, d=128) == E_UNS
+    assert feats(lib, x=None) == E_INV
+    assert feats(lib, w=None) == E_INV
+    assert feats(lib, out=None) == E_INV
+    assert feats(lib, x=MIS) == E_INV
+    assert feats(lib, out=MIS) == E_INV
+    # out overlapping x or omega
+    assert feats(lib, out=P(FAKE.value + 64)) == E_INV
+    assert feats(lib, out=P(FAKE2.value - 64)) == E_INV
+
+
+def test_performer_features_zero_rows_is_a_no_op(lib):
+    assert feats(lib, rows=0, x=None, w=None, out=None) == linattn.LINATTN_OK

@@ -63,3 +63,32 @@ def test_zero_decay_has_finite_gradients():
     w = (og._phi(__import__("torch").tensor(q)) * og._phi(__import__("torch").tensor(k))).sum(-1)
     w = w.numpy()[..., None]
     assert np.abs(y - v * w / (w + 1e-3)).max() < 1e-13
+
+
+def test_identity_mode_gradients_match_central_differences_of_feature_recurrence():
+    """q and k as signed feature vectors: gradients of the masked form with phi =
+    identity equal central differences of oracle/performer.py's token-by-token
+    recurrence (numpy, no autograd)."""
+    from oracle import performer as P
+    q, k, v = rand(12, 1, 2, 6, 3), rand(13, 1, 2, 6, 3), rand(14, 1, 2, 6, 2)
+    q, k = q + 1.5, k + 1.5            # mostly positive scores, some signed features
+    dy = rand(15, 1, 2, 6, 2)
+    lam = np.array([0.8, 1.0])
+    eps = 0.5
+
+    def L(qq, kk, vv, ll):
+        return float((P.causal_feat(qq, kk, vv, ll, eps)[0] * dy).sum())
+
+    y, dq, dk, dv, dlam = og.causal_grad(q, k, v, lam, eps, dy, identity=True)
+    np.testing.assert_allclose(y, P.causal_feat(q, k, v, lam, eps)[0], rtol=1e-12)
+    h = 1e-6
+    for name, x, g in (("q", q, dq), ("k", k, dk), ("v", v, dv), ("lam", lam, dlam)):
+        fd = np.zeros_like(x)
+        for idx in np.ndindex(x.shape):
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += h
+            xm[idx] -= h
+            a = {"qq": q, "kk": k, "vv": v, "ll": lam}
+            key = {"q": "qq", "k": "kk", "v": "vv", "lam": "ll"}[name]
+            fd[idx] = (L(**{**a, key: xp}) - L(**{**a, key: xm})) / (2 * h)
+        assert np.abs(fd - g).max() <= 1e-6 * max(1.0, np.abs(g).max()), name

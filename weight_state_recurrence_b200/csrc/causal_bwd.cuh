@@ -9,6 +9,7 @@
 //   dphi(k_j) = R_j v_j + r_j,   dv_j = R_j^T phi(k_j)
 //   dlambda = sum_i phi(q_i)^T (S'_i dnum_i + z'_i dden_i),  S' = dS/dlambda
 //   dq = dphi(q) * phi'(q), phi'(x) = 1 (x > 0) else e^x = phi(x); dk likewise.
+//   With `ident` (q and k are feature vectors already) phi' = 1.
 // R and r obey the forward recurrence run backwards (R_j = lambda R_{j+1} +
 // phi(q_j) dnum_j^T), so the same chunked form applies in reverse (the §3.1
 // triangular mask, §5.2 blockwise accumulation), with C = 32 tokens a chunk.
@@ -51,7 +52,8 @@ template <int DK, int DV, typename T>
 __global__ void __launch_bounds__(kBwdThreads) causal_bwd_kernel(
     const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
     const T *__restrict__ dy, const float *__restrict__ lam, float eps, T *__restrict__ dq,
-    T *__restrict__ dk, T *__restrict__ dv, float *__restrict__ dlam, int H, int N) {
+    T *__restrict__ dk, T *__restrict__ dv, float *__restrict__ dlam, int H, int N,
+    bool ident) {
   // rows of phi(q), phi(k), v and of the states are padded by one float so that
   // lanes walking different rows at the same column hit different banks
   constexpr int C = kBwdChunk, NT = kBwdThreads, QS = DK + 1, AS = C + 1, VS = DV + 1,
@@ -102,8 +104,8 @@ __global__ void __launch_bounds__(kBwdThreads) causal_bwd_kernel(
       const int t = i / DK, a = i % DK;
       float fq = 0.f, fk = 0.f;
       if (t < Cv) {
-        fq = phi_f32(to_f32(q[qo + static_cast<long>(c0 + t) * DK + a]));
-        fk = phi_f32(to_f32(k[qo + static_cast<long>(c0 + t) * DK + a]));
+        fq = feat_f32(to_f32(q[qo + static_cast<long>(c0 + t) * DK + a]), ident);
+        fk = feat_f32(to_f32(k[qo + static_cast<long>(c0 + t) * DK + a]), ident);
       }
       sQ[t * QS + a] = fq;
       sK[t * QS + a] = fk;
@@ -295,7 +297,7 @@ __global__ void __launch_bounds__(kBwdThreads) causal_bwd_kernel(
           const float gs = fmaf(sz[a], sDd[t], g1[r][m]);
           const float fq = sQ[t * QS + a];
           dq[qo + static_cast<long>(c0 + t) * DK + a] =
-              from_f32<T>(fmaf(pw[t + 1], gs, in[r][m]) * (fq > 1.f ? 1.f : fq));
+              from_f32<T>(fmaf(pw[t + 1], gs, in[r][m]) * (ident || fq > 1.f ? 1.f : fq));
           if (with_dlam) {
             const float gs2 = fmaf(sz2[a], sDd[t], g2[r][m]);
             dl = fmaf(fq, fmaf(dpw[t + 1], gs, pw[t + 1] * gs2), dl);
@@ -400,7 +402,8 @@ __global__ void __launch_bounds__(kBwdThreads) causal_bwd_kernel(
           const int a = tx + 16 * m;
           const float fk = sK[u * QS + a];
           dk[qo + static_cast<long>(c0 + u) * DK + a] =
-              from_f32<T>(fmaf(pw[Cv - u], rv[r][m] + sz[a], in[r][m]) * (fk > 1.f ? 1.f : fk));
+              from_f32<T>(fmaf(pw[Cv - u], rv[r][m] + sz[a], in[r][m]) *
+                          (ident || fk > 1.f ? 1.f : fk));
         }
       }
     }

@@ -34,7 +34,7 @@ __global__ void __launch_bounds__(256) causal_simt_kernel(
     const float *__restrict__ lam, float eps, const float *__restrict__ S_init,
     const float *__restrict__ z_init, T *__restrict__ out, float *__restrict__ S_final,
     float *__restrict__ z_final, int H, int N, int DV, int seg_len,
-    const float *__restrict__ S_seg, const float *__restrict__ z_seg) {
+    const float *__restrict__ S_seg, const float *__restrict__ z_seg, bool ident) {
   constexpr int C = kSimtChunk, NT = 256, QS = DK + 1;
   static_assert(DVS % 4 == 0, "slice must be float4-divisible");
   extern __shared__ __align__(16) float sm[];
@@ -80,8 +80,8 @@ __global__ void __launch_bounds__(256) causal_simt_kernel(
       const int t = i / DK, a = i % DK;
       float fq = 0.f, fk = 0.f;
       if (t < Cv) {
-        fq = phi_f32(to_f32(qp[static_cast<long>(c0 + t) * DK + a]));
-        fk = phi_f32(to_f32(kp[static_cast<long>(c0 + t) * DK + a]));
+        fq = feat_f32(to_f32(qp[static_cast<long>(c0 + t) * DK + a]), ident);
+        fk = feat_f32(to_f32(kp[static_cast<long>(c0 + t) * DK + a]), ident);
       }
       sQ[t * QS + a] = fq;
       sK[t * QS + a] = fk;
@@ -202,7 +202,7 @@ template <int DK, int DVS, typename T>
 __global__ void __launch_bounds__(256) causal_seg_state_kernel(
     const T *__restrict__ k, const T *__restrict__ v, const float *__restrict__ lam,
     float *__restrict__ ws_S, float *__restrict__ ws_z, int H, int N, int DV, int seg_len,
-    int G) {
+    int G, bool ident) {
   constexpr int C = kSimtChunk, NT = 256, QS = DK + 1;
   constexpr int NR = DK / 16, NCOL = DVS / 16;
   __shared__ float sK[C * QS];      // lambda^(Cv-1-s) phi(k_s)
@@ -224,7 +224,7 @@ __global__ void __launch_bounds__(256) causal_seg_state_kernel(
     __syncthreads();
     for (int i = tid; i < C * DK; i += NT) {
       const int t = i / DK, a = i % DK;
-      sK[t * QS + a] = t < Cv ? pw[Cv - 1 - t] * phi_f32(to_f32(kp[static_cast<long>(c0 + t) * DK + a]))
+      sK[t * QS + a] = t < Cv ? pw[Cv - 1 - t] * feat_f32(to_f32(kp[static_cast<long>(c0 + t) * DK + a]), ident)
                               : 0.f;
     }
     for (int i = tid; i < C * DVS; i += NT) {

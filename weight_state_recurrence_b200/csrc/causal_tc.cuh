@@ -220,7 +220,8 @@ __device__ __forceinline__ void tile_pass(uint8_t *p, uint32_t block_bytes, uint
 template <int U>
 __device__ __forceinline__ void phi_pass(uint8_t *p, uint32_t own_bytes, uint32_t stride,
                                          int nblocks, int row0, const float *qsc,
-                                         const float *ksc, bool scaled, int tid, int nthr) {
+                                         const float *ksc, bool scaled, bool ident, int tid,
+                                         int nthr) {
   const uint32_t step = static_cast<uint32_t>(nthr) * 16u;
   const uint32_t total = own_bytes * static_cast<uint32_t>(nblocks);
   for (uint32_t o0 = static_cast<uint32_t>(tid) * 16u; o0 < total; o0 += U * step) {
@@ -234,10 +235,12 @@ __device__ __forceinline__ void phi_pass(uint8_t *p, uint32_t own_bytes, uint32_
     }
 #pragma unroll
     for (int i = 0; i < U; ++i) {
-      w[i].x = phi_bf16x2(w[i].x);
-      w[i].y = phi_bf16x2(w[i].y);
-      w[i].z = phi_bf16x2(w[i].z);
-      w[i].w = phi_bf16x2(w[i].w);
+      if (!ident) {
+        w[i].x = phi_bf16x2(w[i].x);
+        w[i].y = phi_bf16x2(w[i].y);
+        w[i].z = phi_bf16x2(w[i].z);
+        w[i].w = phi_bf16x2(w[i].w);
+      }
       if (scaled) {
         const uint32_t row = static_cast<uint32_t>(row0) + ((off[i] % kPanel) >> 7);
         const float f = (off[i] < 2 * kPanel ? qsc : ksc)[row];
@@ -261,7 +264,7 @@ __global__ void __launch_bounds__(NT, 1)
                      const __grid_constant__ CUtensorMap tm_v, const float *__restrict__ lam,
                      float eps, const float *__restrict__ S_init, const float *__restrict__ z_init,
                      __nv_bfloat16 *__restrict__ out, float *__restrict__ S_final,
-                     float *__restrict__ z_final, int H, int N, int DV) {
+                     float *__restrict__ z_final, int H, int N, int DV, bool ident) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *sm = smem_raw;
   const uint32_t sb = smem_u32(sm);
@@ -552,9 +555,9 @@ __global__ void __launch_bounds__(NT, 1)
       const bool tail = c == nchunks - 1;
       for (int g = 0; g < 2; ++g) {
         uint8_t *base = sm + s * kStage + kOffQ + g * kPanel;
-        if (!rf)
+        if (!rf && (factored || !ident))
           phi_pass<4>(base + own_off, own_bytes, 2 * kPanel, 2, row0, tail ? qt : qf,
-                      tail ? kt : kf, factored, tt, kXformThreads);
+                      tail ? kt : kf, factored, ident, tt, kXformThreads);
         fence_proxy_async_smem();
         named_bar_sync(kBarXform, kXformThreads);
         if (rf) return false;

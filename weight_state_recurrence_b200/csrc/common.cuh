@@ -28,6 +28,11 @@ __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
 // Fast-weight article §4.1 (feature_map); linear-attention note §4.1.
 __device__ __forceinline__ float phi_f32(float x) { return x > 0.f ? x + 1.f : expf(x); }
 
+// The feature applied to a q or k element: elu + 1, or none (`ident`) when q
+// and k already hold feature vectors, such as random features computed
+// beforehand.
+__device__ __forceinline__ float feat_f32(float x, bool ident) { return ident ? x : phi_f32(x); }
+
 // lambda^i for integer i >= 0 by binary exponentiation in fp32 (at most
 // 2*log2(i) roundings).  lambda^0 = 1 also for lambda = 0.  Powers are
 // always formed directly, never as a ratio lambda^a / lambda^b, which would

@@ -41,7 +41,7 @@ template <int DK, int DV, typename T>
 __global__ void __launch_bounds__(kDecodeThreads, 1) decode_step_kernel(
     const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
     const float *__restrict__ lam, float eps, float *__restrict__ S, float *__restrict__ z,
-    T *__restrict__ out, int H, int BH) {
+    T *__restrict__ out, int H, int BH, bool ident) {
   using Lay = DecodeLayout<DK, DV, T>;
   constexpr int NT = kDecodeThreads, TPR = Lay::TPR, RPP = Lay::RPP;
   constexpr int PASSES = (DK + RPP - 1) / RPP;
@@ -106,8 +106,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_step_kernel(
 
     float part = 0.f;
     if (tid < DK) {
-      const float fk = phi_f32(to_f32(sk[tid]));
-      const float fq = phi_f32(to_f32(sq[tid]));
+      const float fk = feat_f32(to_f32(sk[tid]), ident);
+      const float fq = feat_f32(to_f32(sq[tid]), ident);
       s_fk[tid] = fk;
       s_fq[tid] = fq;
       const float zn = fmaf(L, sz[tid], fk);

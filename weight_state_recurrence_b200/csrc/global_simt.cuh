@@ -19,7 +19,8 @@ template <int DK, int DV, typename T>
 __global__ void __launch_bounds__(256) global_kv_simt_kernel(const T *__restrict__ k,
                                                              const T *__restrict__ v,
                                                              float *__restrict__ KV,
-                                                             float *__restrict__ ksum, int N) {
+                                                             float *__restrict__ ksum, int N,
+                                                             bool ident) {
   constexpr int NT = 256, TT = kGlobalTile;
   constexpr int ENT = DK * DV;
   constexpr int PER = (ENT + NT - 1) / NT;
@@ -38,7 +39,7 @@ __global__ void __launch_bounds__(256) global_kv_simt_kernel(const T *__restrict
     __syncthreads();
     for (int i = tid; i < TT * DK; i += NT) {
       const int t = i / DK, a = i % DK;
-      sK[t][a] = t < tv ? phi_f32(to_f32(k[(pair * N + t0 + t) * DK + a])) : 0.f;
+      sK[t][a] = t < tv ? feat_f32(to_f32(k[(pair * N + t0 + t) * DK + a]), ident) : 0.f;
     }
     for (int i = tid; i < TT * DV; i += NT) {
       const int t = i / DV, b = i % DV;
@@ -71,7 +72,7 @@ __global__ void __launch_bounds__(256) global_out_simt_kernel(const T *__restric
                                                               const float *__restrict__ KV,
                                                               const float *__restrict__ ksum,
                                                               float eps, T *__restrict__ out,
-                                                              int N) {
+                                                              int N, bool ident) {
   constexpr int NT = 256, TT = kGlobalTile;
   extern __shared__ __align__(16) float gsm[];
   float *sKV = gsm;              // [DK][DV]
@@ -86,7 +87,7 @@ __global__ void __launch_bounds__(256) global_out_simt_kernel(const T *__restric
   for (int i = tid; i < DK; i += NT) sks[i] = ksum[pair * DK + i];
   for (int i = tid; i < TT * DK; i += NT) {
     const int t = i / DK, a = i % DK;
-    sQ[t * (DK + 1) + a] = t < tv ? phi_f32(to_f32(q[(pair * N + t0 + t) * DK + a])) : 0.f;
+    sQ[t * (DK + 1) + a] = t < tv ? feat_f32(to_f32(q[(pair * N + t0 + t) * DK + a]), ident) : 0.f;
   }
   __syncthreads();
   for (int t = tid; t < TT; t += NT) {

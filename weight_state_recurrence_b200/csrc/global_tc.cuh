@@ -54,7 +54,7 @@ __device__ __forceinline__ uint32_t phi2(uint32_t x) {
 // phi in place over `bytes` of swizzled tile rows (128 bytes per row); rows at
 // or past `valid` become 0 when zero_tail (rows the TMA filled with zeros).
 __device__ __forceinline__ void phi_tile(uint8_t *p, uint32_t bytes, int valid, bool zero_tail,
-                                         int tid, int nthr) {
+                                         bool ident, int tid, int nthr) {
   const uint32_t step = static_cast<uint32_t>(nthr) * 16u;
   for (uint32_t o0 = static_cast<uint32_t>(tid) * 16u; o0 < bytes; o0 += 4 * step) {
     uint4 w[4];
@@ -65,10 +65,10 @@ __device__ __forceinline__ void phi_tile(uint8_t *p, uint32_t bytes, int valid, 
     for (int i = 0; i < 4; ++i) {
       const uint32_t o = o0 + i * step;
       const bool dead = zero_tail && static_cast<int>((o % kPanel) >> 7) >= valid;
-      w[i].x = dead ? 0u : phi2(w[i].x);
-      w[i].y = dead ? 0u : phi2(w[i].y);
-      w[i].z = dead ? 0u : phi2(w[i].z);
-      w[i].w = dead ? 0u : phi2(w[i].w);
+      w[i].x = dead ? 0u : ident ? w[i].x : phi2(w[i].x);
+      w[i].y = dead ? 0u : ident ? w[i].y : phi2(w[i].y);
+      w[i].z = dead ? 0u : ident ? w[i].z : phi2(w[i].z);
+      w[i].w = dead ? 0u : ident ? w[i].w : phi2(w[i].w);
     }
 #pragma unroll
     for (int i = 0; i < 4; ++i)
@@ -100,7 +100,7 @@ constexpr uint32_t kMiscTmem = 128, kMiscFail = 132, kMiscRoleFail = 136;
 __global__ void __launch_bounds__(kv::NT, 1)
     global_kv_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, float *__restrict__ KV,
-                        float *__restrict__ ksum, int npairs, int N) {
+                        float *__restrict__ ksum, int npairs, int N, bool ident) {
   using namespace kv;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *sm = smem_raw;
@@ -227,7 +227,7 @@ __global__ void __launch_bounds__(kv::NT, 1)
       }
       const int c = chunk_of(i);
       const int valid = N - c * C;
-      if (!*rfail) phi_tile(sm + s * kStage, 2 * kPanel, valid, valid < C, tt, kXform);
+      if (!*rfail) phi_tile(sm + s * kStage, 2 * kPanel, valid, valid < C, ident, tt, kXform);
       fence_proxy_async_smem();
       named_bar_sync(1, kXform);
       if (*rfail) break;
@@ -297,7 +297,8 @@ constexpr uint32_t kMiscTmem = 256, kMiscFail = 260, kMiscXFail = 264, kMiscEFai
 __global__ void __launch_bounds__(out::NT, 1)
     global_out_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                          const __grid_constant__ CUtensorMap tm_y, const float *__restrict__ KV,
-                         const float *__restrict__ ksum, float eps, int BH, int N) {
+                         const float *__restrict__ ksum, float eps, int BH, int N,
+                         bool ident) {
   using namespace out;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *sm = smem_raw;
@@ -396,7 +397,7 @@ __global__ void __launch_bounds__(out::NT, 1)
         *xfail = 1;
         *fail = 1;
       }
-      if (!*xfail) phi_tile(sm + kOffQ + s * kPanel, kPanel, C, false, tt, kXform);
+      if (!*xfail && !ident) phi_tile(sm + kOffQ + s * kPanel, kPanel, C, false, false, tt, kXform);
       fence_proxy_async_smem();
       named_bar_sync(1, kXform);
       if (*xfail) break;

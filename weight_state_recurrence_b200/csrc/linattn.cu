@@ -22,6 +22,7 @@
 #include "causal_bwd.cuh"
 #include "global_simt.cuh"
 #include "global_tc.cuh"
+#include "performer.cuh"
 
 namespace linattn {
 namespace {
@@ -47,6 +48,7 @@ int check_dims(const linattn_dims *d, bool use_n) {
   if (!d) return LINATTN_ERR_INVALID;
   if (d->B < 0 || d->H < 0 || (use_n && d->N < 0)) return LINATTN_ERR_INVALID;
   if (d->dtype != LINATTN_BF16 && d->dtype != LINATTN_F32) return LINATTN_ERR_UNSUPPORTED;
+  if (d->phi != LINATTN_PHI_ELU1 && d->phi != LINATTN_PHI_IDENTITY) return LINATTN_ERR_UNSUPPORTED;
   if (!supported_dim(d->dk) || !supported_dim(d->dv)) return LINATTN_ERR_UNSUPPORTED;
   const long long n = use_n ? d->N : 1;
   const long long big = static_cast<long long>(d->B) * d->H * n *
@@ -56,6 +58,9 @@ int check_dims(const linattn_dims *d, bool use_n) {
     return LINATTN_ERR_UNSUPPORTED;
   return LINATTN_OK;
 }
+
+// q and k hold feature vectors already: the kernels apply no feature map
+bool ident(const linattn_dims *d) { return d->phi == LINATTN_PHI_IDENTITY; }
 
 bool bad_eps(float eps) { return !(eps >= 0.f) || !std::isfinite(eps); }
 
@@ -153,7 +158,7 @@ int launch_decode(const linattn_dims *d, const void *q, const void *k, const voi
   const int grid = BH < sms ? BH : sms;
   kern<<<grid, kDecodeThreads, bytes, s>>>(
       static_cast<const T *>(q), static_cast<const T *>(k), static_cast<const T *>(v), lam, eps,
-      S, z, static_cast<T *>(out), d->H, BH);
+      S, z, static_cast<T *>(out), d->H, BH, ident(d));
   return launch_status();
 }
 
@@ -231,7 +236,7 @@ int launch_causal_simt(const linattn_dims *d, const void *q, const void *k, cons
     // (1) each segment's own final state from zero, (2) the starting states
     causal_seg_state_kernel<DK, DVS, T><<<dim3(ctas, sg.G - 1), 256, 0, s>>>(
         static_cast<const T *>(k), static_cast<const T *>(v), lam, wsS, wsz, d->H, d->N, d->dv,
-        sg.len, sg.G);
+        sg.len, sg.G, ident(d));
     if (cudaGetLastError() != cudaSuccess) return LINATTN_ERR_CUDA;
     causal_seg_combine_kernel<<<d->B * d->H, 256, 0, s>>>(lam, S_init, z_init, wsS, wsz, d->H,
                                                           d->dk, d->dv, d->N, sg.len, sg.G);
@@ -240,7 +245,7 @@ int launch_causal_simt(const linattn_dims *d, const void *q, const void *k, cons
   kern<<<dim3(ctas, sg.G), 256, bytes, s>>>(
       static_cast<const T *>(q), static_cast<const T *>(k), static_cast<const T *>(v), lam, eps,
       S_init, z_init, static_cast<T *>(out), S_final, z_final, d->H, d->N, d->dv, sg.len,
-      sg.G > 1 ? wsS : nullptr, sg.G > 1 ? wsz : nullptr);
+      sg.G > 1 ? wsS : nullptr, sg.G > 1 ? wsz : nullptr, ident(d));
   return launch_status();
 }
 
@@ -297,8 +302,8 @@ int launch_causal_tc(const linattn_dims *d, const void *q, const void *k, const 
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   if (cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, lam, eps, S_init, z_init,
-                         static_cast<bf16 *>(out), S_final, z_final, d->H, d->N,
-                         d->dv) != cudaSuccess)
+                         static_cast<bf16 *>(out), S_final, z_final, d->H, d->N, d->dv,
+                         ident(d)) != cudaSuccess)
     return LINATTN_ERR_CUDA;
   return launch_status();
 }
@@ -312,7 +317,7 @@ int launch_global_simt(const linattn_dims *d, int Nk, const void *q, const void 
   if (Nk > 0) {
     dim3 g1(BH, (Nk + kGlobalSplit - 1) / kGlobalSplit);
     global_kv_simt_kernel<DK, DV, T><<<g1, 256, 0, s>>>(
-        static_cast<const T *>(k), static_cast<const T *>(v), KV, ksum, Nk);
+        static_cast<const T *>(k), static_cast<const T *>(v), KV, ksum, Nk, ident(d));
     if (cudaGetLastError() != cudaSuccess) return LINATTN_ERR_CUDA;
   }
   if (d->N > 0) {
@@ -321,7 +326,7 @@ int launch_global_simt(const linattn_dims *d, int Nk, const void *q, const void 
     if (!set_smem(kern, bytes)) return LINATTN_ERR_CUDA;
     dim3 g2(BH, (d->N + kGlobalTile - 1) / kGlobalTile);
     kern<<<g2, 256, bytes, s>>>(static_cast<const T *>(q), KV, ksum, eps,
-                                static_cast<T *>(out), d->N);
+                                static_cast<T *>(out), d->N, ident(d));
   }
   return launch_status();
 }
@@ -384,8 +389,8 @@ int launch_global_tc(const linattn_dims *d, int Nk, const void *q, const void *k
     // being zeroed; it waits for that grid only before its first flush
     const ProgrammaticLaunch pl(static_cast<int>(u1 < sms ? u1 : sms), gtc::kv::NT,
                                 gtc::kv::kSmemBytes, s);
-    if (cudaLaunchKernelEx(&pl.cfg, gtc::global_kv_tc_kernel, mk, mv, KV, ksum, BH / 2, Nk) !=
-        cudaSuccess)
+    if (cudaLaunchKernelEx(&pl.cfg, gtc::global_kv_tc_kernel, mk, mv, KV, ksum, BH / 2, Nk,
+                           ident(d)) != cudaSuccess)
       return LINATTN_ERR_CUDA;
   }
   if (d->N > 0) {
@@ -399,7 +404,7 @@ int launch_global_tc(const linattn_dims *d, int Nk, const void *q, const void *k
                                 gtc::out::kSmemBytes, s);
     if (cudaLaunchKernelEx(&pl.cfg, gtc::global_out_tc_kernel, mq, my,
                            static_cast<const float *>(KV), static_cast<const float *>(ksum), eps,
-                           BH, d->N) != cudaSuccess)
+                           BH, d->N, ident(d)) != cudaSuccess)
       return LINATTN_ERR_CUDA;
   }
   return launch_status();
@@ -440,7 +445,7 @@ int launch_causal_bwd(const linattn_dims *d, const void *q, const void *k, const
   kern<<<d->B * d->H, kBwdThreads, bytes, s>>>(
       static_cast<const T *>(q), static_cast<const T *>(k), static_cast<const T *>(v),
       static_cast<const T *>(dy), lam, eps, static_cast<T *>(dq), static_cast<T *>(dk),
-      static_cast<T *>(dv), dlam, d->H, d->N);
+      static_cast<T *>(dv), dlam, d->H, d->N, ident(d));
   return launch_status();
 }
 
@@ -715,6 +720,82 @@ extern "C" int linattn_decode_step(const linattn_dims *d, const void *q, const v
   if (d->dtype == LINATTN_F32)
     return decode_dispatch<float>(d, q, k, v, lambda, eps, S, z, out, s);
   return decode_dispatch<bf16>(d, q, k, v, lambda, eps, S, z, out, s);
+}
+
+// ------------------------------------------------------------ Performer features
+namespace {
+
+bool supported_features(int m) { return m == 8 || m == 16 || m == 32 || m == 64; }
+
+// bf16 with d in {64, 128} and m in {32, 64} takes the tensor-core kernel;
+// LINATTN_PERFORMER_KERNEL=simt forces the CUDA-core kernel.
+bool use_tc_features(int d, int m, int dtype) {
+  const char *e = std::getenv("LINATTN_PERFORMER_KERNEL");
+  if (e && std::strcmp(e, "simt") == 0) return false;
+  return dtype == LINATTN_BF16 && (d == 64 || d == 128) && (m == 32 || m == 64);
+}
+
+template <int D, int M>
+int launch_features_tc(long long rows, int kernel, const void *x, const void *omega, void *out,
+                       cudaStream_t s) {
+  using L = perf::Layout<D, M>;
+  auto *kern = performer_tc_kernel<D, M>;
+  if (!set_smem(kern, static_cast<int>(L::kSmem))) return LINATTN_ERR_CUDA;
+  const int sms = num_sms();
+  if (sms <= 0) return LINATTN_ERR_CUDA;
+  CUtensorMap mx, mw, my;
+  const int r = static_cast<int>(rows);
+  if (!make_map_bf16(&mx, x, D, r, 1) || !make_map_bf16(&mw, omega, D, M, 1, M) ||
+      !make_map_bf16(&my, out, 2 * M, r, 1))
+    return LINATTN_ERR_CUDA;
+  const long long tiles = (rows + perf::R - 1) / perf::R;
+  const int grid = static_cast<int>(tiles < sms ? tiles : sms);
+  kern<<<grid, perf::NT, L::kSmem, s>>>(mx, mw, my, static_cast<long>(rows), kernel);
+  return launch_status();
+}
+
+template <typename T>
+int launch_features_simt(long long rows, int d, int m, int kernel, const void *x,
+                         const void *omega, void *out, cudaStream_t s) {
+  const int sms = num_sms();
+  if (sms <= 0) return LINATTN_ERR_CUDA;
+  const int bytes = (m * (d + 1) + (kPerfSimtThreads / 32) * d) * 4;
+  const long long want = (rows + kPerfSimtThreads / 32 - 1) / (kPerfSimtThreads / 32);
+  const int grid = static_cast<int>(want < 8LL * sms ? want : 8LL * sms);
+  performer_simt_kernel<T><<<grid, kPerfSimtThreads, bytes, s>>>(
+      static_cast<const T *>(x), static_cast<const T *>(omega), static_cast<T *>(out),
+      static_cast<long>(rows), d, m, kernel);
+  return launch_status();
+}
+
+}  // namespace
+
+extern "C" int linattn_performer_features(long long rows, int d, int m, int kernel, int dtype,
+                                          const void *x, const void *omega, void *out,
+                                          linattn_stream_t stream) {
+  if (rows < 0) return LINATTN_ERR_INVALID;
+  if (dtype != LINATTN_BF16 && dtype != LINATTN_F32) return LINATTN_ERR_UNSUPPORTED;
+  if (kernel != LINATTN_PERFORMER_SOFTMAX && kernel != LINATTN_PERFORMER_GAUSSIAN)
+    return LINATTN_ERR_UNSUPPORTED;
+  if (!supported_dim(d) || !supported_features(m)) return LINATTN_ERR_UNSUPPORTED;
+  if (rows * (d > 2 * m ? d : 2 * m) >= (1LL << 31)) return LINATTN_ERR_UNSUPPORTED;
+  if (rows == 0) return LINATTN_OK;   // nothing to read or write: NULL buffers allowed
+  if (!x || !omega || !out) return LINATTN_ERR_INVALID;
+  if (!aligned16(x) || !aligned16(omega) || !aligned16(out)) return LINATTN_ERR_INVALID;
+  const size_t es = elem_size(dtype);
+  const size_t nx = static_cast<size_t>(rows) * d * es, nw = static_cast<size_t>(m) * d * es;
+  const size_t ny = static_cast<size_t>(rows) * 2 * m * es;
+  if (overlaps(out, ny, x, nx) || overlaps(out, ny, omega, nw)) return LINATTN_ERR_INVALID;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (use_tc_features(d, m, dtype)) {
+    if (d == 64) return m == 32 ? launch_features_tc<64, 32>(rows, kernel, x, omega, out, s)
+                                : launch_features_tc<64, 64>(rows, kernel, x, omega, out, s);
+    return m == 32 ? launch_features_tc<128, 32>(rows, kernel, x, omega, out, s)
+                   : launch_features_tc<128, 64>(rows, kernel, x, omega, out, s);
+  }
+  if (dtype == LINATTN_F32)
+    return launch_features_simt<float>(rows, d, m, kernel, x, omega, out, s);
+  return launch_features_simt<bf16>(rows, d, m, kernel, x, omega, out, s);
 }
 
 extern "C" const char *linattn_status_string(int status) {

@@ -25,16 +25,20 @@ LINATTN_ERR_INVALID = 1
 LINATTN_ERR_UNSUPPORTED = 2
 LINATTN_ERR_CUDA = 3
 LINATTN_ERR_DEVICE = 4
+LINATTN_PHI_ELU1, LINATTN_PHI_IDENTITY = 0, 1
+LINATTN_PERFORMER_SOFTMAX, LINATTN_PERFORMER_GAUSSIAN = 0, 1
 
 ENTRY_POINTS = ("linattn_fwd_causal", "linattn_fwd_causal_from", "linattn_fwd_causal_workspace",
                 "linattn_fwd_causal_ws", "linattn_fwd_causal_noalloc", "linattn_bwd_causal",
                 "linattn_fwd_global", "linattn_fwd_global_cross", "linattn_decode_step",
-                "linattn_status_string", "linattn_device_status", "linattn_version")
+                "linattn_performer_features", "linattn_status_string", "linattn_device_status",
+                "linattn_version")
 
 
 class linattn_dims(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("N", ctypes.c_int),
-                ("dk", ctypes.c_int), ("dv", ctypes.c_int), ("dtype", ctypes.c_int)]
+                ("dk", ctypes.c_int), ("dv", ctypes.c_int), ("dtype", ctypes.c_int),
+                ("phi", ctypes.c_int)]
 
 
 class LinattnError(RuntimeError):
@@ -83,6 +87,8 @@ def load(build_if_missing: bool = True):
     lib.linattn_fwd_global_cross.restype = i
     lib.linattn_decode_step.argtypes = [dp, vp, vp, vp, fp, f, fp, fp, vp, vp]
     lib.linattn_decode_step.restype = i
+    lib.linattn_performer_features.argtypes = [ctypes.c_longlong, i, i, i, i, vp, vp, vp, vp]
+    lib.linattn_performer_features.restype = i
     lib.linattn_status_string.argtypes = [i]
     lib.linattn_status_string.restype = ctypes.c_char_p
     lib.linattn_device_status.argtypes = [i, vp]
@@ -133,7 +139,8 @@ def _f32(t, shape, name):
         raise ValueError(f"{name} must be float32 with shape {tuple(shape)}")
 
 
-def linattn_fwd_causal(q, k, v, lam, eps, out, S_final=None, z_final=None, stream=None):
+def linattn_fwd_causal(q, k, v, lam, eps, out, S_final=None, z_final=None, stream=None, *,
+                       phi=LINATTN_PHI_ELU1):
     """Causal forward: q, k [B,H,N,dk], v/out [B,H,N,dv] (bf16 or fp32),
     lam [H] fp32 or None, S_final [B,H,dk,dv] / z_final [B,H,dk] fp32 or None."""
     B, H, N, dk = q.shape
@@ -145,14 +152,14 @@ def linattn_fwd_causal(q, k, v, lam, eps, out, S_final=None, z_final=None, strea
     _f32(lam, (H,), "lambda")
     _f32(S_final, (B, H, dk, dv), "S_final")
     _f32(z_final, (B, H, dk), "z_final")
-    d = linattn_dims(B, H, N, dk, dv, _dtype_code(q.dtype))
+    d = linattn_dims(B, H, N, dk, dv, _dtype_code(q.dtype), int(phi))
     _check(load().linattn_fwd_causal(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), _ptr(lam),
                                      float(eps), _ptr(out), _ptr(S_final), _ptr(z_final),
                                      _stream(stream)), "linattn_fwd_causal")
 
 
 def linattn_fwd_causal_from(q, k, v, lam, eps, S_init, z_init, out, S_final=None, z_final=None,
-                            stream=None):
+                            stream=None, *, phi=LINATTN_PHI_ELU1):
     """Causal forward continued from (S_init [B,H,dk,dv], z_init [B,H,dk]) fp32,
     both given or both None; the other arguments as linattn_fwd_causal."""
     B, H, N, dk = q.shape
@@ -166,14 +173,14 @@ def linattn_fwd_causal_from(q, k, v, lam, eps, S_init, z_init, out, S_final=None
     _f32(z_init, (B, H, dk), "z_init")
     _f32(S_final, (B, H, dk, dv), "S_final")
     _f32(z_final, (B, H, dk), "z_final")
-    d = linattn_dims(B, H, N, dk, dv, _dtype_code(q.dtype))
+    d = linattn_dims(B, H, N, dk, dv, _dtype_code(q.dtype), int(phi))
     _check(load().linattn_fwd_causal_from(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), _ptr(lam),
                                           float(eps), _ptr(S_init), _ptr(z_init), _ptr(out),
                                           _ptr(S_final), _ptr(z_final), _stream(stream)),
            "linattn_fwd_causal_from")
 
 
-def _causal_dims(q, k, v, out, S_final, z_final, lam):
+def _causal_dims(q, k, v, out, S_final, z_final, lam, phi=LINATTN_PHI_ELU1):
     B, H, N, dk = q.shape
     dv = v.shape[-1]
     if k.shape != q.shape or tuple(v.shape) != (B, H, N, dv) or out.shape != v.shape:
@@ -183,20 +190,20 @@ def _causal_dims(q, k, v, out, S_final, z_final, lam):
     _f32(lam, (H,), "lambda")
     _f32(S_final, (B, H, dk, dv), "S_final")
     _f32(z_final, (B, H, dk), "z_final")
-    return linattn_dims(B, H, N, dk, dv, _dtype_code(q.dtype))
+    return linattn_dims(B, H, N, dk, dv, _dtype_code(q.dtype), int(phi))
 
 
-def linattn_fwd_causal_workspace(B, H, N, dk, dv, dtype) -> int:
+def linattn_fwd_causal_workspace(B, H, N, dk, dv, dtype, phi=LINATTN_PHI_ELU1) -> int:
     """Workspace bytes the segment-parallel causal forward wants (0: none)."""
-    d = linattn_dims(B, H, N, dk, dv, _dtype_code(dtype))
+    d = linattn_dims(B, H, N, dk, dv, _dtype_code(dtype), int(phi))
     return int(load().linattn_fwd_causal_workspace(ctypes.byref(d)))
 
 
 def linattn_fwd_causal_ws(q, k, v, lam, eps, S_init, z_init, out, S_final, z_final, workspace,
-                          stream=None):
+                          stream=None, *, phi=LINATTN_PHI_ELU1):
     """Causal forward (optionally from S_init, z_init) with a caller workspace:
     a CUDA tensor of at least linattn_fwd_causal_workspace bytes, or None."""
-    d = _causal_dims(q, k, v, out, S_final, z_final, lam)
+    d = _causal_dims(q, k, v, out, S_final, z_final, lam, phi)
     nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(load().linattn_fwd_causal_ws(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), _ptr(lam),
                                         float(eps), _ptr(S_init), _ptr(z_init), _ptr(out),
@@ -205,16 +212,18 @@ def linattn_fwd_causal_ws(q, k, v, lam, eps, S_init, z_init, out, S_final, z_fin
            "linattn_fwd_causal_ws")
 
 
-def linattn_fwd_causal_noalloc(q, k, v, lam, eps, out, S_final=None, z_final=None, stream=None):
+def linattn_fwd_causal_noalloc(q, k, v, lam, eps, out, S_final=None, z_final=None, stream=None,
+                               *, phi=LINATTN_PHI_ELU1):
     """linattn_fwd_causal whose segment-parallel form uses the library's own scratch."""
-    d = _causal_dims(q, k, v, out, S_final, z_final, lam)
+    d = _causal_dims(q, k, v, out, S_final, z_final, lam, phi)
     _check(load().linattn_fwd_causal_noalloc(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v),
                                              _ptr(lam), float(eps), _ptr(out), _ptr(S_final),
                                              _ptr(z_final), _stream(stream)),
            "linattn_fwd_causal_noalloc")
 
 
-def linattn_bwd_causal(q, k, v, lam, eps, dy, dq, dk, dv, dlam=None, stream=None):
+def linattn_bwd_causal(q, k, v, lam, eps, dy, dq, dk, dv, dlam=None, stream=None, *,
+                       phi=LINATTN_PHI_ELU1):
     """Backward of the causal forward: dy like v; dq, dk like q; dv like v;
     dlam [H] fp32 or None."""
     B, H, N, dk_ = q.shape
@@ -226,13 +235,13 @@ def linattn_bwd_causal(q, k, v, lam, eps, dy, dq, dk, dv, dlam=None, stream=None
         raise ValueError("q, k, v, dy, dq, dk, dv must share one dtype")
     _f32(lam, (H,), "lambda")
     _f32(dlam, (H,), "dlambda")
-    d = linattn_dims(B, H, N, dk_, dv_, _dtype_code(q.dtype))
+    d = linattn_dims(B, H, N, dk_, dv_, _dtype_code(q.dtype), int(phi))
     _check(load().linattn_bwd_causal(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), _ptr(lam),
                                      float(eps), _ptr(dy), _ptr(dq), _ptr(dk), _ptr(dv),
                                      _ptr(dlam), _stream(stream)), "linattn_bwd_causal")
 
 
-def linattn_fwd_global(q, k, v, eps, out, KV, ksum, stream=None):
+def linattn_fwd_global(q, k, v, eps, out, KV, ksum, stream=None, *, phi=LINATTN_PHI_ELU1):
     """Global forward: q, k [B,H,N,dk], v/out [B,H,N,dv]; KV [B,H,dk,dv] and
     ksum [B,H,dk] fp32 are written."""
     B, H, N, dk = q.shape
@@ -243,13 +252,14 @@ def linattn_fwd_global(q, k, v, eps, out, KV, ksum, stream=None):
         raise ValueError("q, k, v, out must share one dtype")
     _f32(KV, (B, H, dk, dv), "KV")
     _f32(ksum, (B, H, dk), "ksum")
-    d = linattn_dims(B, H, N, dk, dv, _dtype_code(q.dtype))
+    d = linattn_dims(B, H, N, dk, dv, _dtype_code(q.dtype), int(phi))
     _check(load().linattn_fwd_global(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), float(eps),
                                      _ptr(out), _ptr(KV), _ptr(ksum), _stream(stream)),
            "linattn_fwd_global")
 
 
-def linattn_fwd_global_cross(q, k, v, eps, out, KV, ksum, stream=None):
+def linattn_fwd_global_cross(q, k, v, eps, out, KV, ksum, stream=None, *,
+                             phi=LINATTN_PHI_ELU1):
     """Cross global forward: q/out [B,H,Nq,dk/dv], k/v [B,H,Nk,dk/dv];
     KV [B,H,dk,dv] and ksum [B,H,dk] fp32 (written)."""
     B, H, Nq, dk = q.shape
@@ -261,13 +271,13 @@ def linattn_fwd_global_cross(q, k, v, eps, out, KV, ksum, stream=None):
         raise ValueError("q, k, v, out must share one dtype")
     _f32(KV, (B, H, dk, dv), "KV")
     _f32(ksum, (B, H, dk), "ksum")
-    d = linattn_dims(B, H, Nq, dk, dv, _dtype_code(q.dtype))
+    d = linattn_dims(B, H, Nq, dk, dv, _dtype_code(q.dtype), int(phi))
     _check(load().linattn_fwd_global_cross(ctypes.byref(d), int(Nk), _ptr(q), _ptr(k), _ptr(v),
                                            float(eps), _ptr(out), _ptr(KV), _ptr(ksum),
                                            _stream(stream)), "linattn_fwd_global_cross")
 
 
-def linattn_decode_step(q, k, v, lam, eps, S, z, out, stream=None):
+def linattn_decode_step(q, k, v, lam, eps, S, z, out, stream=None, *, phi=LINATTN_PHI_ELU1):
     """One decode step: q, k [B,H,dk], v/out [B,H,dv]; S [B,H,dk,dv] and z
     [B,H,dk] fp32 are updated in place."""
     B, H, dk = q.shape
@@ -279,10 +289,29 @@ def linattn_decode_step(q, k, v, lam, eps, S, z, out, stream=None):
     _f32(lam, (H,), "lambda")
     _f32(S, (B, H, dk, dv), "S")
     _f32(z, (B, H, dk), "z")
-    d = linattn_dims(B, H, 1, dk, dv, _dtype_code(q.dtype))
+    d = linattn_dims(B, H, 1, dk, dv, _dtype_code(q.dtype), int(phi))
     _check(load().linattn_decode_step(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), _ptr(lam),
                                       float(eps), _ptr(S), _ptr(z), _ptr(out), _stream(stream)),
            "linattn_decode_step")
+
+
+def linattn_performer_features(x, omega, kernel, out, stream=None):
+    """Performer random features: x [..., d] (rows = the product of the
+    leading dims), omega [m, d], out [..., 2m], one dtype; kernel
+    LINATTN_PERFORMER_SOFTMAX or LINATTN_PERFORMER_GAUSSIAN."""
+    d = x.shape[-1]
+    if omega.dim() != 2 or omega.shape[1] != d:
+        raise ValueError("omega must have shape [m, d]")
+    m = omega.shape[0]
+    if tuple(out.shape) != tuple(x.shape[:-1]) + (2 * m,):
+        raise ValueError("out must have shape x.shape[:-1] + (2m,)")
+    if not (x.dtype == omega.dtype == out.dtype):
+        raise ValueError("x, omega, out must share one dtype")
+    rows = x.numel() // d if d else 0
+    _check(load().linattn_performer_features(ctypes.c_longlong(rows), int(d), int(m), int(kernel),
+                                             _dtype_code(x.dtype), _ptr(x), _ptr(omega),
+                                             _ptr(out), _stream(stream)),
+           "linattn_performer_features")
 
 
 def linattn_status_string(code: int) -> str:
@@ -299,47 +328,64 @@ def linattn_version() -> int:
 
 # ---------------------------------------------------------------- helpers
 def fwd_causal(q, k, v, lam=None, eps=1e-6, want_state=True, S_init=None, z_init=None,
-               stream=None):
+               stream=None, phi=LINATTN_PHI_ELU1):
     B, H, N, dk = q.shape
     dv = v.shape[-1]
     out = torch.empty_like(v)
     S = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device) if want_state else None
     z = torch.empty((B, H, dk), dtype=torch.float32, device=q.device) if want_state else None
     if S_init is None and z_init is None:
-        linattn_fwd_causal(q, k, v, lam, eps, out, S, z, stream)
+        linattn_fwd_causal(q, k, v, lam, eps, out, S, z, stream, phi=phi)
     else:
-        linattn_fwd_causal_from(q, k, v, lam, eps, S_init, z_init, out, S, z, stream)
+        linattn_fwd_causal_from(q, k, v, lam, eps, S_init, z_init, out, S, z, stream, phi=phi)
     return out, S, z
 
 
-def bwd_causal(q, k, v, dy, lam=None, eps=1e-6, want_dlam=False, stream=None):
+def bwd_causal(q, k, v, dy, lam=None, eps=1e-6, want_dlam=False, stream=None,
+               phi=LINATTN_PHI_ELU1):
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     dlam = (torch.empty(q.shape[1], dtype=torch.float32, device=q.device) if want_dlam else None)
-    linattn_bwd_causal(q, k, v, lam, eps, dy, dq, dk, dv, dlam, stream)
+    linattn_bwd_causal(q, k, v, lam, eps, dy, dq, dk, dv, dlam, stream, phi=phi)
     return dq, dk, dv, dlam
 
 
-def fwd_global(q, k, v, eps=1e-6, stream=None):
+def fwd_global(q, k, v, eps=1e-6, stream=None, phi=LINATTN_PHI_ELU1):
     B, H, N, dk = q.shape
     dv = v.shape[-1]
     out = torch.empty_like(v)
     KV = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
     ks = torch.empty((B, H, dk), dtype=torch.float32, device=q.device)
-    linattn_fwd_global(q, k, v, eps, out, KV, ks, stream)
+    linattn_fwd_global(q, k, v, eps, out, KV, ks, stream, phi=phi)
     return out, KV, ks
 
 
-def fwd_global_cross(q, k, v, eps=1e-6, stream=None):
+def fwd_global_cross(q, k, v, eps=1e-6, stream=None, phi=LINATTN_PHI_ELU1):
     B, H, Nq, dk = q.shape
     dv = v.shape[-1]
     out = torch.empty((B, H, Nq, dv), dtype=v.dtype, device=v.device)
     KV = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
     ks = torch.empty((B, H, dk), dtype=torch.float32, device=q.device)
-    linattn_fwd_global_cross(q, k, v, eps, out, KV, ks, stream)
+    linattn_fwd_global_cross(q, k, v, eps, out, KV, ks, stream, phi=phi)
     return out, KV, ks
 
 
-def decode_step(q, k, v, S, z, lam=None, eps=1e-6, stream=None):
+def decode_step(q, k, v, S, z, lam=None, eps=1e-6, stream=None, phi=LINATTN_PHI_ELU1):
     out = torch.empty_like(v)
-    linattn_decode_step(q, k, v, lam, eps, S, z, out, stream)
+    linattn_decode_step(q, k, v, lam, eps, S, z, out, stream, phi=phi)
     return out
+
+
+def performer_features(x, omega, kernel=LINATTN_PERFORMER_SOFTMAX, stream=None):
+    out = torch.empty(tuple(x.shape[:-1]) + (2 * omega.shape[0],), dtype=x.dtype, device=x.device)
+    linattn_performer_features(x, omega, kernel, out, stream)
+    return out
+
+
+def performer_causal(q, k, v, omega, lam=None, eps=1e-6, kernel=LINATTN_PERFORMER_SOFTMAX,
+                     want_state=True, stream=None):
+    """Causal attention on Performer features: the features of q and k
+    ([B,H,N,2m]) from linattn_performer_features, then the causal forward in
+    identity mode.  Returns (out, S_final, z_final)."""
+    fq = performer_features(q, omega, kernel, stream)
+    fk = performer_features(k, omega, kernel, stream)
+    return fwd_causal(fq, fk, v, lam, eps, want_state, stream=stream, phi=LINATTN_PHI_IDENTITY)
