@@ -20,6 +20,11 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda:0"
 IDENT = 1
 KERNELS = {"softmax": 0, "gaussian": 1}
+# Features are bounded by their row's scale g(x)/sqrt(m) and rounded once to
+# bf16 (relative 2^-9); omega.x is accumulated in fp32 from the same bf16
+# values the oracle sees, and sin/cos are good to ~4e-7.  So the error of a
+# feature is a few 1e-3 of the row scale: gate 5e-3 of the largest feature.
+BF16_FEAT_TOL = 5e-3
 
 
 def draw(seed, shape, scale, dtype):
@@ -46,22 +51,24 @@ def check_features(lib, rows, d, m, kernel, dtype, scale, seed, tol, simt=False,
 def test_tensor_core_features(cuda_lib, d, m, kernel):
     # 1000 rows: 7 full tiles of 128 and a ragged tail of 104
     check_features(cuda_lib, 1000, d, m, kernel, torch.bfloat16, 0.5 / math.sqrt(d),
-                   2000 + d + m, 2e-2)
+                   2000 + d + m, BF16_FEAT_TOL)
 
 
-def test_tensor_core_features_large_arguments(cuda_lib):
-    # x ~ N(0, 1), d = 128: omega.x ~ N(0, 128), tens of radians
-    check_features(cuda_lib, 777, 128, 64, "gaussian", torch.bfloat16, 1.0, 2100, 2e-2)
+@pytest.mark.parametrize("scale", [1.0, 8.0])
+def test_tensor_core_features_large_arguments(cuda_lib, scale):
+    # d = 128: omega.x ~ N(0, 128 scale^2), tens (scale 1) to hundreds (scale 8)
+    # of radians, through every quadrant of the argument reduction
+    check_features(cuda_lib, 777, 128, 64, "gaussian", torch.bfloat16, scale, 2100, BF16_FEAT_TOL)
 
 
 def test_tensor_core_features_many_tiles(cuda_lib):
     # more tiles than CTAs: every CTA walks its range through the whole ring
     check_features(cuda_lib, 148 * 128 * 5 + 3, 128, 64, "softmax", torch.bfloat16,
-                   0.5 / math.sqrt(128), 2200, 2e-2)
+                   0.5 / math.sqrt(128), 2200, BF16_FEAT_TOL)
 
 
-@pytest.mark.parametrize("d,m,dtype,tol", [(32, 16, torch.bfloat16, 2e-2),
-                                           (128, 8, torch.bfloat16, 2e-2),
+@pytest.mark.parametrize("d,m,dtype,tol", [(32, 16, torch.bfloat16, BF16_FEAT_TOL),
+                                           (128, 8, torch.bfloat16, BF16_FEAT_TOL),
                                            (64, 64, torch.float32, 1e-4),
                                            (16, 32, torch.float32, 1e-4)])
 def test_cuda_core_features(cuda_lib, d, m, dtype, tol):
@@ -71,7 +78,7 @@ def test_cuda_core_features(cuda_lib, d, m, dtype, tol):
 
 def test_forced_cuda_core_features_bf16(cuda_lib, monkeypatch):
     check_features(cuda_lib, 500, 128, 64, "softmax", torch.bfloat16, 0.5 / math.sqrt(128), 2500,
-                   2e-2, simt=True, monkeypatch=monkeypatch)
+                   BF16_FEAT_TOL, simt=True, monkeypatch=monkeypatch)
 
 
 def test_zero_rows(cuda_lib):

@@ -746,7 +746,7 @@ int launch_features_tc(long long rows, int kernel, const void *x, const void *om
   CUtensorMap mx, mw, my;
   const int r = static_cast<int>(rows);
   if (!make_map_bf16(&mx, x, D, r, 1) || !make_map_bf16(&mw, omega, D, M, 1, M) ||
-      !make_map_bf16(&my, out, 2 * M, r, 1))
+      !make_map_bf16(&my, out, 2 * M, r, 1, 32))   // 32-row slabs, one per quadrant team
     return LINATTN_ERR_CUDA;
   const long long tiles = (rows + perf::R - 1) / perf::R;
   const int grid = static_cast<int>(tiles < sms ? tiles : sms);

@@ -10,9 +10,13 @@
 //                          is a dense contraction, so it runs on the tensor
 //                          cores: 128-row tiles of X arrive by TMA, one
 //                          M = 128, N = m, K = d chain per tile accumulates
-//                          in TMEM (two buffers), and eight epilogue warps
+//                          in TMEM (two buffers), and sixteen epilogue warps
 //                          turn U into cos/sin, scale by g/sqrt(m) and send
-//                          the bf16 tile out by TMA.  Persistent CTAs.
+//                          the bf16 tile out by TMA.  The four warps of a TMEM
+//                          lane quadrant own its 32 rows (a quarter of the
+//                          columns each) and work as an independent team:
+//                          they meet only at their own named barrier and store
+//                          their own 32-row slab.  Persistent CTAs.
 //   performer_simt_kernel  every other case, fp32 arithmetic with the
 //                          accurate sincosf/expf: one warp per row.
 #pragma once
@@ -23,16 +27,36 @@ namespace linattn {
 
 enum : int { kPerfSoftmax = 0, kPerfGaussian = 1 };
 
-// sin and cos of u for the bf16 path.  u is first reduced to [-pi, pi] by
-// Cody and Waite's two-constant method (2 pi = P1 + P2, P1 = 6.28125 has 8
-// significant bits, so k * P1 is exact for |k| < 2^16), then the hardware
-// approximations, accurate to about 2^-21 absolute on that interval, far below
-// the bf16 resolution of the result.
-__device__ __forceinline__ void sincos_reduced(float u, float *s, float *c) {
-  const float k = rintf(u * 0.159154943091895336f);   // u / (2 pi), rounded
-  float r = fmaf(-k, 6.28125f, u);
-  r = fmaf(-k, 1.93530717958647692e-3f, r);             // 2 pi - 6.28125
-  __sincosf(r, s, c);
+// sin and cos of u for the bf16 path, on the FMA pipe (the special-function
+// pipe, shared by the sin/cos approximations, float rounding and conversions,
+// is otherwise the bottleneck of the epilogue), scaled by sc:
+//   u = j pi + r:  j = u / pi rounded to nearest by adding 1.5 * 2^23 (the
+//     sum's lowest mantissa bit is then j's parity), r by Cody and Waite's
+//     two-constant reduction with pi = P1 + P2, P1 = 3.140625 (8 significant
+//     bits: j P1 is exact for |j| < 2^16, so |u| up to about 2e5 reduces
+//     accurately);
+//   sin r, cos r by their Taylor series through r^9 and r^8 on |r| <= pi/2
+//     (truncation errors below 4e-6 and 2.5e-5, against the 2^-9 relative
+//     rounding of the bf16 result);
+//   sin u = (-1)^j sin r, cos u = (-1)^j cos r: the sign goes into sc.
+__device__ __forceinline__ void sincos_poly(float u, float sc, float *sn, float *cs) {
+  const float kRound = 12582912.f;                            // 1.5 * 2^23
+  const float t = fmaf(u, 0.318309886183790672f, kRound);    // u / pi + 1.5 * 2^23
+  const float jf = t - kRound;
+  float r = fmaf(-jf, 3.140625f, u);
+  r = fmaf(-jf, 9.67653589793116e-4f, r);                    // pi - 3.140625
+  const float sg = __int_as_float(__float_as_int(sc) ^ (__float_as_int(t) << 31));
+  const float r2 = r * r;
+  float ps = fmaf(r2, 2.75573192239858907e-6f, -1.98412698412698413e-4f);   // 1/9!, -1/7!
+  ps = fmaf(r2, ps, 8.33333333333333333e-3f);                               // 1/5!
+  ps = fmaf(r2, ps, -0.166666666666666667f);                                // -1/3!
+  ps = fmaf(r2, ps, 1.0f);
+  float pc = fmaf(r2, 2.48015873015873016e-5f, -1.38888888888888889e-3f);   // 1/8!, -1/6!
+  pc = fmaf(r2, pc, 4.16666666666666667e-2f);                               // 1/4!
+  pc = fmaf(r2, pc, -0.5f);
+  pc = fmaf(r2, pc, 1.0f);
+  *sn = (r * sg) * ps;
+  *cs = sg * pc;
 }
 
 // ----------------------------------------------------------- CUDA cores
@@ -82,8 +106,9 @@ namespace perf {
 constexpr int R = 128;                   // rows per tile (the MMA's M)
 constexpr int kStages = 4;               // X tile ring
 constexpr uint32_t kPanel = R * 128;     // 128 rows x 64 bf16, 128B-swizzled
-constexpr int NT = 384;                  // warp 0 TMA, warp 1 MMA, warps 4-11 epilogue
-constexpr int kEpi = 256;                // epilogue threads: two per row
+constexpr int kGroups = 4;               // epilogue threads per row (warps per quadrant)
+constexpr int kEpi = kGroups * R;        // epilogue threads (warps 4 .. 4 + kEpi/32 - 1)
+constexpr int NT = 128 + kEpi;           // warp 0 TMA, warp 1 MMA, warps 2-3 idle
 enum { kXFull = 0, kXEmpty = kStages, kAccFull = 2 * kStages, kAccEmpty = kAccFull + 2,
        kWFull = kAccEmpty + 2, kFinal, kNumBars };
 
@@ -98,8 +123,9 @@ struct Layout {
   static constexpr uint32_t kYStage = (2 * M / 64) * kPanel;
   static constexpr uint32_t kOffMisc = kOffY + 2 * kYStage;
   static constexpr uint32_t kMiscTmem = 8 * kNumBars, kMiscFail = kMiscTmem + 4,
-                            kMiscEFail = kMiscTmem + 8;
-  static constexpr uint32_t kSmem = kOffMisc + 256;
+                            kMiscEFail = kMiscTmem + 8;   // 4 ints: one per row quadrant
+  static constexpr uint32_t kOffPart = kOffMisc + 256;              // [kGroups][R] |x|^2 parts
+  static constexpr uint32_t kSmem = kOffPart + kGroups * R * 4;
   static constexpr uint32_t kTmCols = 2 * M;                        // two accumulators
   static_assert(kOffW % 1024 == 0 && kOffY % 1024 == 0, "swizzled tiles need 1 KB alignment");
   static_assert(kSmem <= 227 * 1024, "shared memory");
@@ -140,9 +166,12 @@ __global__ void __launch_bounds__(perf::NT, 1)
   const int nmine = static_cast<int>(t1 - t0);
 
   if (tid == 0) {
-    for (int i = 0; i < kNumBars; ++i) mbar_init(bar(i), 1);
+    // the four quadrant teams each release an X stage and an accumulator
+    for (int i = 0; i < kNumBars; ++i)
+      mbar_init(bar(i), (i >= kXEmpty && i < kXEmpty + kStages) ||
+                                (i >= kAccEmpty && i < kAccEmpty + 2) ? 4 : 1);
     *fail = 0;
-    *efail = 0;
+    for (int q = 0; q < 4; ++q) efail[q] = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tm_x);
     tma_prefetch_desc(&tm_w);
@@ -211,65 +240,77 @@ __global__ void __launch_bounds__(perf::NT, 1)
     __syncwarp();
   } else if (warp >= 4) {
     // ------------------------------------------------ epilogue
-    // thread (row r, half h): TMEM lane quadrant warp % 4, columns of U
-    // [h M/2, (h+1) M/2) -> cos at those columns, sin at M + those columns
-    const int et = tid - 128;
-    const int h = (warp - 4) >> 2;
-    const int r = ((warp - 4) & 3) * 32 + lane;
-    const uint32_t lf = static_cast<uint32_t>(((warp - 4) & 3) * 32) << 16;
-    constexpr int HM = M / 2;
+    // quadrant team q = warp % 4 owns tile rows [32 q, 32 q + 32) (its TMEM
+    // lanes); thread (row r, group g) takes columns [g QM, (g+1) QM) of U ->
+    // cos at those columns, sin at M + those columns, and a quarter of |x_r|^2
+    const int q = warp & 3;
+    const int g = (warp - 4) >> 2;
+    const int r = q * 32 + lane;
+    const bool lead = g == 0 && lane == 0;     // the team's TMA-store / barrier thread
+    const uint32_t lf = static_cast<uint32_t>(q * 32) << 16;
+    constexpr int QM = M / kGroups;           // 16 or 8 columns of U per thread
+    constexpr int QC = D / kGroups / 8;       // 16-byte chunks of x per thread (4 or 2)
+    float *part = reinterpret_cast<float *>(sm + L::kOffPart);
     const float inv_sqrt_m = rsqrtf(static_cast<float>(M));
     for (int i = 0; i < nmine; ++i) {
       const int s = i % kStages, a = i & 1;
       const bool ok = !*fail && mbar_wait(bar(kAccFull + a), (i >> 1) & 1);
-      if (!ok) *efail = 1;
+      if (!ok) efail[q] = 1;
       tc_fence_after();
-      float sc = inv_sqrt_m;
       if (ok && kernel == kPerfSoftmax) {
-        // |x_r|^2 from the staged tile (the MMA has finished reading it)
+        // this thread's part of |x_r|^2 from the staged tile (the MMA has
+        // finished reading it)
         const uint8_t *xs = sm + L::kOffX + s * L::kXStage;
         float n2 = 0.f;
 #pragma unroll
-        for (int p = 0; p < D / 64; ++p)
+        for (int j = 0; j < QC; ++j) {
+          const int ch = g * QC + j;            // 16-byte chunk of the row
+          const uint4 w =
+              *reinterpret_cast<const uint4 *>(xs + (ch >> 3) * kPanel + sw128_offset(r, 16 * (ch & 7)));
+          const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const uint4 w = *reinterpret_cast<const uint4 *>(xs + p * kPanel + sw128_offset(r, 16 * j));
-            const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float lo = __uint_as_float(ww[e] << 16), hi = __uint_as_float(ww[e] & 0xffff0000u);
-              n2 = fmaf(lo, lo, n2);
-              n2 = fmaf(hi, hi, n2);
-            }
+          for (int e = 0; e < 4; ++e) {
+            const float lo = __uint_as_float(ww[e] << 16), hi = __uint_as_float(ww[e] & 0xffff0000u);
+            n2 = fmaf(lo, lo, n2);
+            n2 = fmaf(hi, hi, n2);
           }
+        }
+        part[g * R + r] = n2;
+      }
+      // the team's rows of staging tile a must be free: its store of tile i-2
+      // has read them
+      if (i >= 2 && lead) tma_store_wait_read_1();
+      named_bar_sync(1 + q, 32 * kGroups);
+      if (efail[q]) break;
+      if (lead) mbar_arrive(bar(kXEmpty + s));
+      float sc = inv_sqrt_m;
+      if (kernel == kPerfSoftmax) {
+        float n2 = 0.f;
+#pragma unroll
+        for (int p = 0; p < kGroups; ++p) n2 += part[p * R + r];
         sc *= expf(0.5f * n2);
       }
-      // staging tile a must be free: the store of tile i-2 has read it
-      if (i >= 2 && et == 0) tma_store_wait_read_1();
-      named_bar_sync(1, kEpi);
-      if (*efail) break;
-      if (et == 0) mbar_arrive(bar(kXEmpty + s));
-      uint32_t u[HM];
-      if constexpr (HM == 32) {
-        tmem_ld_32x32b_x32(tmem + lf + a * M + h * HM, u);
+      uint32_t u[QM];
+      if constexpr (QM == 16) {
+        tmem_ld_32x32b_x16(tmem + lf + a * M + g * QM, u);
       } else {
-        tmem_ld_32x32b_x16(tmem + lf + a * M + h * HM, u);
+        tmem_ld_32x32b_x8(tmem + lf + a * M + g * QM, u);
       }
       tmem_wait_ld();
       tc_fence_before();
       uint8_t *stg = sm + L::kOffY + a * L::kYStage;
 #pragma unroll
-      for (int j = 0; j < HM / 8; ++j) {
+      for (int j = 0; j < QM / 8; ++j) {
         uint32_t cw[4], sw[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           float s0, c0, s1, c1;
-          sincos_reduced(__uint_as_float(u[8 * j + 2 * e]), &s0, &c0);
-          sincos_reduced(__uint_as_float(u[8 * j + 2 * e + 1]), &s1, &c1);
-          cw[e] = pack_bf16x2(c0 * sc, c1 * sc);
-          sw[e] = pack_bf16x2(s0 * sc, s1 * sc);
+          sincos_poly(__uint_as_float(u[8 * j + 2 * e]), sc, &s0, &c0);
+          sincos_poly(__uint_as_float(u[8 * j + 2 * e + 1]), sc, &s1, &c1);
+          cw[e] = pack_bf16x2(c0, c1);
+          sw[e] = pack_bf16x2(s0, s1);
         }
-        const int cc = h * HM + 8 * j;    // cosine column; the sine is at M + cc
+        const int cc = g * QM + 8 * j;    // cosine column; the sine is at M + cc
         const int sc_col = M + cc;
         *reinterpret_cast<uint4 *>(stg + (cc >> 6) * kPanel + sw128_offset(r, (cc & 63) * 2)) =
             make_uint4(cw[0], cw[1], cw[2], cw[3]);
@@ -278,16 +319,18 @@ __global__ void __launch_bounds__(perf::NT, 1)
             make_uint4(sw[0], sw[1], sw[2], sw[3]);
       }
       fence_proxy_async_smem();
-      named_bar_sync(1, kEpi);
-      if (et == 0) {
+      named_bar_sync(1 + q, 32 * kGroups);
+      if (lead) {
         mbar_arrive(bar(kAccEmpty + a));
-        const int row0 = static_cast<int>((t0 + i) * R);
+        // the team's 32-row slab of every 64-column panel (4 KB, 1 KB aligned)
+        const int row0 = static_cast<int>((t0 + i) * R) + 32 * q;
         for (int p = 0; p < 2 * M / 64; ++p)
-          tma_store_3d(&tm_y, sb + L::kOffY + a * L::kYStage + p * kPanel, 64 * p, row0, 0);
+          tma_store_3d(&tm_y, sb + L::kOffY + a * L::kYStage + p * kPanel + 32 * q * 128, 64 * p,
+                       row0, 0);
         tma_store_commit();
       }
     }
-    if (et == 0) tma_store_wait_all();
+    if (lead) tma_store_wait_all();
   }
   tc_fence_before();
   __syncthreads();
