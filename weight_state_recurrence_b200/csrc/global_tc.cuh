@@ -82,6 +82,21 @@ __device__ __forceinline__ void red_add_v4(float *addr, float a, float b, float 
                : "memory");
 }
 
+// Position (group, index) of a CTA's work unit u0 + i, for units laid out as
+// groups of n consecutive indices, stepped one unit at a time: the loops need
+// no 64-bit division per unit.
+struct UnitCursor {
+  int group, index, n;
+  __device__ UnitCursor(long u0, int n_) : group(static_cast<int>(u0 / n_)),
+                                           index(static_cast<int>(u0 % n_)), n(n_) {}
+  __device__ void next() {
+    if (++index == n) {
+      index = 0;
+      ++group;
+    }
+  }
+};
+
 // ============================================================= KV, ksum
 namespace kv {
 constexpr int kStages = 3;
@@ -148,22 +163,22 @@ __global__ void __launch_bounds__(kv::NT, 1)
   // the output kernel may start its CTAs on SMs this grid leaves (its q tiles
   // and phi(q) do not depend on KV; it waits for this grid before reading KV)
   grid_launch_dependents();
-  // unit i of this CTA: pair u / nchunks, chunk u % nchunks; a segment is a run
-  // of units of one pair; the accumulator is flushed at the end of a segment
-  auto pair_of = [&](int i) { return static_cast<int>((u0 + i) / nchunks); };
-  auto chunk_of = [&](int i) { return static_cast<int>((u0 + i) % nchunks); };
-  auto seg_end = [&](int i) { return i + 1 == nmine || pair_of(i + 1) != pair_of(i); };
+  // unit u0 + i of this CTA: pair (u0 + i) / nchunks, chunk (u0 + i) % nchunks,
+  // tracked by a UnitCursor; a segment is a run of units of one pair, and the
+  // accumulator is flushed at its end (the last unit, or the pair's last chunk)
+  auto seg_end = [&](int i, const UnitCursor &u) { return i + 1 == nmine || u.index == nchunks - 1; };
 
   if (warp == 0) {
     if (lane == 0) {
       int issued = 0;
-      for (int i = 0; i < nmine && !*fail; ++i) {
+      UnitCursor u(u0, nchunks);
+      for (int i = 0; i < nmine && !*fail; ++i, u.next()) {
         const int s = i % kStages;
         if (i >= kStages && !mbar_wait(bar(kEmpty + s), ((i / kStages) - 1) & 1)) {
           *fail = 1;
           break;
         }
-        const int p = pair_of(i), c = chunk_of(i);
+        const int p = u.group, c = u.index;
         const uint32_t st = sb + s * kStage, b = bar(kFull + s);
         mbar_arrive_expect_tx(b, kStage);
         tma_load_3d(st, &tm_k, b, 0, c * C, 2 * p);
@@ -182,7 +197,8 @@ __global__ void __launch_bounds__(kv::NT, 1)
       const uint32_t idkv = idesc_bf16(128, 128, 1, 1), idks = idesc_bf16(128, 16, 1, 0);
       int seg = 0;
       bool first = true;
-      for (int i = 0; i < nmine; ++i) {
+      UnitCursor u(u0, nchunks);
+      for (int i = 0; i < nmine; ++i, u.next()) {
         const int s = i % kStages;
         if (*fail || !mbar_wait(bar(kPhi + s), (i / kStages) & 1)) {
           *fail = 1;
@@ -206,7 +222,7 @@ __global__ void __launch_bounds__(kv::NT, 1)
         }
         umma_commit(bar(kEmpty + s));
         first = false;
-        if (seg_end(i)) {
+        if (seg_end(i, u)) {
           umma_commit(bar(kFlushReady));
           ++seg;
           first = true;
@@ -219,32 +235,36 @@ __global__ void __launch_bounds__(kv::NT, 1)
   } else if (warp >= 4) {
     const int tt = tid - 128;   // 0..255
     int seg = 0;
-    for (int i = 0; i < nmine; ++i) {
+    UnitCursor u(u0, nchunks);
+    for (int i = 0; i < nmine; ++i, u.next()) {
       const int s = i % kStages;
       if (*fail || !mbar_wait(bar(kFull + s), (i / kStages) & 1)) {
         *rfail = 1;
         *fail = 1;
       }
-      const int c = chunk_of(i);
-      const int valid = N - c * C;
+      const int valid = N - u.index * C;
       if (!*rfail) phi_tile(sm + s * kStage, 2 * kPanel, valid, valid < C, ident, tt, kXform);
       fence_proxy_async_smem();
       named_bar_sync(1, kXform);
       if (*rfail) break;
       if (tt == 0) mbar_arrive(bar(kPhi + s));
-      if (seg_end(i)) {
-        // flush: lanes 0-63 are head 2p's d_k rows, 64-127 head 2p+1's
+      if (seg_end(i, u)) {
+        // flush: lanes 0-63 are head 2p's d_k rows, 64-127 head 2p+1's.  The
+        // verdict of the wait is shared through the barrier first, so that a
+        // warp reads TMEM with all its lanes or not at all.
         const bool ok = !*fail && mbar_wait(bar(kFlushReady), seg & 1);
         if (!ok) {
           *rfail = 1;
           *fail = 1;
         }
+        named_bar_sync(1, kXform);
+        if (*rfail) break;
         tc_fence_after();
-        if (ok && warp < 8) {
+        if (warp < 8) {
           grid_dependency_wait();   // KV and ksum have been zeroed
           const int row = (warp - 4) * 32 + lane;
           const int hsel = row >> 6, kk = row & 63;
-          const long bh = 2L * pair_of(i) + hsel;
+          const long bh = 2L * u.group + hsel;
           const uint32_t lf = static_cast<uint32_t>((warp - 4) * 32) << 16;
           uint32_t a[32], ksv[2];
           float *dst = KV + (bh * D + kk) * D;
@@ -286,11 +306,11 @@ constexpr uint32_t kOffX = kOffB + 8192;                // [ksum_hi, ksum_lo, 0 
 constexpr uint32_t kOffY = kOffX + 8192;                // 2 y staging tiles
 constexpr uint32_t kOffMisc = kOffY + 2 * kPanel;
 constexpr uint32_t kSmemBytes = kOffMisc + 512;
-constexpr int NT = 512;   // warp 0 TMA, 1 MMA, 4-7 epilogue, 8-15 phi
+constexpr int NT = 512;   // warp 0 TMA loads, 1 MMA, 2 TMA stores, 4-7 epilogue, 8-15 phi
 constexpr int kXform = 256;
 constexpr uint32_t kTmCols = 256;   // two 128-column accumulators (80 used each)
 enum { kFull = 0, kPhi = kStages, kEmpty = 2 * kStages, kDFull = 3 * kStages, kDEmpty = kDFull + 2,
-       kBReady = kDEmpty + 2, kFinal, kNumBars };
+       kBReady = kDEmpty + 2, kYFull, kYFree = kYFull + 2, kFinal = kYFree + 2, kNumBars };
 constexpr uint32_t kMiscTmem = 256, kMiscFail = 260, kMiscXFail = 264, kMiscEFail = 268;
 }  // namespace out
 
@@ -319,9 +339,9 @@ __global__ void __launch_bounds__(out::NT, 1)
   const long units = static_cast<long>(BH) * ntiles;
   const long u0 = units * blockIdx.x / gridDim.x, u1 = units * (blockIdx.x + 1) / gridDim.x;
   const int nmine = static_cast<int>(u1 - u0);
-  auto head_of = [&](int i) { return static_cast<int>((u0 + i) / ntiles); };
-  auto tile_of = [&](int i) { return static_cast<int>((u0 + i) % ntiles); };
-  auto seg_start = [&](int i) { return i == 0 || head_of(i) != head_of(i - 1); };
+  // unit u0 + i: head (u0 + i) / ntiles, tile (u0 + i) % ntiles, tracked by a
+  // UnitCursor; a new head starts at the CTA's first unit or at tile 0
+  auto seg_start = [&](int i, const UnitCursor &u) { return i == 0 || u.index == 0; };
 
   if (tid == 0) {
     for (int i = 0; i < kNumBars; ++i) mbar_init(bar(i), 1);
@@ -347,7 +367,8 @@ __global__ void __launch_bounds__(out::NT, 1)
   if (warp == 0) {
     if (lane == 0) {
       int issued = 0;
-      for (int i = 0; i < nmine && !*fail; ++i) {
+      UnitCursor u(u0, ntiles);
+      for (int i = 0; i < nmine && !*fail; ++i, u.next()) {
         const int s = i % kStages;
         if (i >= kStages && !mbar_wait(bar(kEmpty + s), ((i / kStages) - 1) & 1)) {
           *fail = 1;
@@ -355,7 +376,7 @@ __global__ void __launch_bounds__(out::NT, 1)
         }
         const uint32_t b = bar(kFull + s);
         mbar_arrive_expect_tx(b, kPanel);
-        tma_load_3d(sb + kOffQ + s * kPanel, &tm_q, b, 0, tile_of(i) * C, head_of(i));
+        tma_load_3d(sb + kOffQ + s * kPanel, &tm_q, b, 0, u.index * C, u.group);
         issued = i + 1;
       }
       if (*fail)   // let the copies still in flight land before the CTA exits
@@ -367,10 +388,11 @@ __global__ void __launch_bounds__(out::NT, 1)
     if (lane == 0) {
       const uint32_t id = idesc_bf16(128, 80, 0, 1);
       int seg = 0;
-      for (int i = 0; i < nmine; ++i) {
+      UnitCursor u(u0, ntiles);
+      for (int i = 0; i < nmine; ++i, u.next()) {
         const int s = i % kStages, d = i & 1;
         bool ok = !*fail && mbar_wait(bar(kPhi + s), (i / kStages) & 1);
-        if (ok && seg_start(i)) ok = mbar_wait(bar(kBReady), seg++ & 1);
+        if (ok && seg_start(i, u)) ok = mbar_wait(bar(kBReady), seg++ & 1);
         if (ok && i >= 2) ok = mbar_wait(bar(kDEmpty + d), ((i >> 1) - 1) & 1);
         if (!ok) {
           *fail = 1;
@@ -387,6 +409,27 @@ __global__ void __launch_bounds__(out::NT, 1)
       }
       umma_commit(bar(kFinal));
       mbar_wait(bar(kFinal), 0);
+    }
+    __syncwarp();
+  } else if (warp == 2) {
+    // y stores: issuing a 16 KB TMA store takes the issuing thread ~1 K
+    // cycles, so it happens here, off the epilogue's per-tile chain.  Staging
+    // tile d goes out once the epilogue has filled it, and is handed back once
+    // the copy has read it.
+    if (lane == 0) {
+      UnitCursor u(u0, ntiles);
+      for (int i = 0; i < nmine; ++i, u.next()) {
+        const int d = i & 1;
+        if (*fail || !mbar_wait(bar(kYFull + d), (i >> 1) & 1)) {
+          *fail = 1;
+          break;
+        }
+        tma_store_3d(&tm_y, sb + kOffY + d * kPanel, 0, u.index * C, u.group);
+        tma_store_commit();
+        tma_store_wait_read();
+        mbar_arrive(bar(kYFree + d));
+      }
+      tma_store_wait_all();
     }
     __syncwarp();
   } else if (warp >= 8) {
@@ -408,14 +451,15 @@ __global__ void __launch_bounds__(out::NT, 1)
     // every head, then turns each accumulator tile into y
     const int r = (warp - 4) * 32 + lane;
     const uint32_t lf = static_cast<uint32_t>((warp - 4) * 32) << 16;
-    for (int i = 0; i < nmine; ++i) {
+    UnitCursor u(u0, ntiles);
+    for (int i = 0; i < nmine; ++i, u.next()) {
       const int d = i & 1;
-      if (seg_start(i)) {
+      if (seg_start(i, u)) {
         // every earlier MMA has completed (its tile was consumed below), so
         // the operand can be rewritten: KV rows = d_k (K), 64 columns (N);
         // KV and ksum are complete once the KV grid has finished
         grid_dependency_wait();
-        const long bh = head_of(i);
+        const long bh = u.group;
         if (r < D) {
           const float *src = KV + (bh * D + r) * D;
 #pragma unroll
@@ -435,21 +479,24 @@ __global__ void __launch_bounds__(out::NT, 1)
         named_bar_sync(2, 128);
         if (r == 0) mbar_arrive(bar(kBReady));
       }
-      const bool ok = !*fail && mbar_wait(bar(kDFull + d), (i >> 1) & 1);
+      // every thread decides before the barrier and reads the verdict after
+      // it, so the whole warpgroup takes the same path
+      bool ok = !*fail && mbar_wait(bar(kDFull + d), (i >> 1) & 1);
+      // staging tile d must be free: the store of tile i-2 has read it
+      if (ok && i >= 2 && r == 0) ok = mbar_wait(bar(kYFree + d), ((i >> 1) - 1) & 1);
       if (!ok) {
         *efail = 1;
         *fail = 1;
       }
       tc_fence_after();
-      if (ok) {
+      named_bar_sync(2, 128);
+      if (*efail) break;
+      {
         uint32_t o[32], qz[2];
         tmem_ld_32x32b_x2(tmem + lf + d * 128 + 64, qz);
         tmem_ld_32x32b_x32(tmem + lf + d * 128, o);
         tmem_wait_ld();
         const float inv = 1.f / (__uint_as_float(qz[0]) + __uint_as_float(qz[1]) + eps);
-        // staging tile d must be free: its previous store has read it
-        if (i >= 2 && r == 0) tma_store_wait_read();
-        named_bar_sync(2, 128);
         uint8_t *stg = sm + kOffY + d * kPanel;
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
@@ -469,14 +516,11 @@ __global__ void __launch_bounds__(out::NT, 1)
       tc_fence_before();
       fence_proxy_async_smem();
       named_bar_sync(2, 128);
-      if (*efail) break;
       if (r == 0) {
         mbar_arrive(bar(kDEmpty + d));
-        tma_store_3d(&tm_y, sb + kOffY + d * kPanel, 0, tile_of(i) * C, head_of(i));
-        tma_store_commit();
+        mbar_arrive(bar(kYFull + d));
       }
     }
-    if (r == 0) tma_store_wait_all();
   }
   tc_fence_before();
   __syncthreads();

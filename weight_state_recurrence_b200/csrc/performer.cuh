@@ -137,10 +137,6 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t *>(&p);
 }
 
-__device__ __forceinline__ void tma_store_wait_read_1() {
-  asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
-}
-
 template <int D, int M>
 __global__ void __launch_bounds__(perf::NT, 1)
     performer_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
@@ -323,10 +319,13 @@ __global__ void __launch_bounds__(perf::NT, 1)
       if (lead) {
         mbar_arrive(bar(kAccEmpty + a));
         // the team's 32-row slab of every 64-column panel (4 KB, 1 KB aligned)
-        const int row0 = static_cast<int>((t0 + i) * R) + 32 * q;
-        for (int p = 0; p < 2 * M / 64; ++p)
-          tma_store_3d(&tm_y, sb + L::kOffY + a * L::kYStage + p * kPanel + 32 * q * 128, 64 * p,
-                       row0, 0);
+        // a slab wholly past the last row is not stored; its (empty) group is
+        // still committed so the group count per tile stays one
+        const long row0 = (t0 + i) * R + 32 * q;
+        if (row0 < rows)
+          for (int p = 0; p < 2 * M / 64; ++p)
+            tma_store_3d(&tm_y, sb + L::kOffY + a * L::kYStage + p * kPanel + 32 * q * 128,
+                         64 * p, static_cast<int>(row0), 0);
         tma_store_commit();
       }
     }
