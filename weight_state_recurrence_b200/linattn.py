@@ -389,3 +389,71 @@ def performer_causal(q, k, v, omega, lam=None, eps=1e-6, kernel=LINATTN_PERFORME
     fq = performer_features(q, omega, kernel, stream)
     fk = performer_features(k, omega, kernel, stream)
     return fwd_causal(fq, fk, v, lam, eps, want_state, stream=stream, phi=LINATTN_PHI_IDENTITY)
+
+
+def fwd_causal_host(q, k, v, lam=None, eps=1e-6, out=None, S_final=None, z_final=None,
+                    pieces=None, device=None):
+    """Causal forward on host-resident tensors (pinned for the copies to be
+    asynchronous).  Every (sequence, head) is independent, so the B*H heads are
+    cut into ``pieces`` runs of heads of one sequence (default: runs of 4
+    heads, or whole sequences when H is not a multiple of 4) whose
+    host-to-device copies, kernels and device-to-host copies run on three
+    streams: the copies of one piece overlap the kernels and copies of the
+    others, and the two copy directions overlap each other.  The device holds
+    two pieces at a time.  ``out`` [B,H,N,dv] (q's dtype), ``S_final``
+    [B,H,dk,dv] and ``z_final`` [B,H,dk] fp32 are host tensors, allocated
+    (pinned) when None.  Returns (out, S_final, z_final); on return every copy
+    has landed."""
+    B, H, N, dk = q.shape
+    dv = v.shape[-1]
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    pin = lambda shape, dt: torch.empty(shape, dtype=dt, pin_memory=True)
+    out = pin((B, H, N, dv), q.dtype) if out is None else out
+    S_final = pin((B, H, dk, dv), torch.float32) if S_final is None else S_final
+    z_final = pin((B, H, dk), torch.float32) if z_final is None else z_final
+    per_seq = max(1, (pieces or 4 * B) // max(B, 1))
+    hp = max(1, -(-H // per_seq))               # heads per piece
+    runs = [(b, h0, min(H, h0 + hp)) for b in range(B) for h0 in range(0, H, hp)]
+    lam_d = None if lam is None else lam.to(dev, non_blocking=True)
+    # one 16-byte aligned copy of lambda per head offset (the C ABI wants aligned pointers)
+    lam_runs = {} if lam_d is None else {h0: lam_d[h0:h1].clone() for _, h0, h1 in runs}
+    slots = [dict(q=torch.empty((hp, N, dk), dtype=q.dtype, device=dev),
+                  k=torch.empty((hp, N, dk), dtype=q.dtype, device=dev),
+                  v=torch.empty((hp, N, dv), dtype=q.dtype, device=dev),
+                  y=torch.empty((hp, N, dv), dtype=q.dtype, device=dev),
+                  S=torch.empty((hp, dk, dv), dtype=torch.float32, device=dev),
+                  z=torch.empty((hp, dk), dtype=torch.float32, device=dev),
+                  inputs_free=None, outputs_free=None) for _ in range(2)]
+    s_in, s_cmp, s_out = (torch.cuda.Stream(device=dev) for _ in range(3))
+    cur = torch.cuda.current_stream(dev)
+    for s in (s_in, s_cmp, s_out):
+        s.wait_stream(cur)          # lambda and the slots are ready
+    for p, (b, h0, h1) in enumerate(runs):
+        sl, nh = slots[p % 2], h1 - h0
+        with torch.cuda.stream(s_in):
+            if sl["inputs_free"] is not None:
+                s_in.wait_event(sl["inputs_free"])
+            sl["q"][:nh].copy_(q[b, h0:h1], non_blocking=True)
+            sl["k"][:nh].copy_(k[b, h0:h1], non_blocking=True)
+            sl["v"][:nh].copy_(v[b, h0:h1], non_blocking=True)
+            ready = torch.cuda.Event()
+            ready.record(s_in)
+        s_cmp.wait_event(ready)
+        if sl["outputs_free"] is not None:
+            s_cmp.wait_event(sl["outputs_free"])
+        view = lambda t: t[:nh].unsqueeze(0)   # [1, nh, ...]: one sequence, nh heads
+        linattn_fwd_causal(view(sl["q"]), view(sl["k"]), view(sl["v"]), lam_runs.get(h0), eps,
+                           view(sl["y"]), view(sl["S"]), view(sl["z"]), s_cmp)
+        done = torch.cuda.Event()
+        done.record(s_cmp)
+        sl["inputs_free"] = done
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(done)
+            out[b, h0:h1].copy_(sl["y"][:nh], non_blocking=True)
+            S_final[b, h0:h1].copy_(sl["S"][:nh], non_blocking=True)
+            z_final[b, h0:h1].copy_(sl["z"][:nh], non_blocking=True)
+            landed = torch.cuda.Event()
+            landed.record(s_out)
+        sl["outputs_free"] = landed
+    s_out.synchronize()
+    return out, S_final, z_final
