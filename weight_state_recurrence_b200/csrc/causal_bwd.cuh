@@ -98,23 +98,53 @@ __global__ void __launch_bounds__(kBwdThreads) causal_bwd_kernel(
   const int nchunks = (N + C - 1) / C;
   float dl = 0.f;   // this thread's share of dlambda
 
-  // phi of a chunk's q and k rows, its v rows and dy rows; zero past the end
+  // phi of a chunk's q and k rows, its v rows and dy rows; zero past the end.
+  // Eight elements per load, and every load of the chunk issued before the
+  // first shared-memory store, so the global latencies overlap.
   auto load_chunk = [&](int c0, int Cv) {
-    for (int i = tid; i < C * DK; i += NT) {
-      const int t = i / DK, a = i % DK;
-      float fq = 0.f, fk = 0.f;
-      if (t < Cv) {
-        fq = feat_f32(to_f32(q[qo + static_cast<long>(c0 + t) * DK + a]), ident);
-        fk = feat_f32(to_f32(k[qo + static_cast<long>(c0 + t) * DK + a]), ident);
+    constexpr int QI = (C * DK / 8 + NT - 1) / NT, VI = (C * DV / 8 + NT - 1) / NT;
+    float fq[QI][8], fk[QI][8], fv[VI][8], fg[VI][8];
+#pragma unroll
+    for (int u = 0; u < QI; ++u) {
+      const int i = tid + u * NT, t = i / (DK / 8), a = (i % (DK / 8)) * 8;
+      const bool live = i < C * DK / 8 && t < Cv;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) fq[u][e] = fk[u][e] = 0.f;
+      if (live) {
+        load8_f32(q + qo + static_cast<long>(c0 + t) * DK + a, fq[u]);
+        load8_f32(k + qo + static_cast<long>(c0 + t) * DK + a, fk[u]);
       }
-      sQ[t * QS + a] = fq;
-      sK[t * QS + a] = fk;
     }
-    for (int i = tid; i < C * DV; i += NT) {
-      const int t = i / DV, j = i % DV;
-      const long o = vo + static_cast<long>(c0 + t) * DV + j;
-      sV[t * VS + j] = t < Cv ? to_f32(v[o]) : 0.f;
-      sG[i] = t < Cv ? to_f32(dy[o]) : 0.f;
+#pragma unroll
+    for (int u = 0; u < VI; ++u) {
+      const int i = tid + u * NT, t = i / (DV / 8), j = (i % (DV / 8)) * 8;
+      const bool live = i < C * DV / 8 && t < Cv;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) fv[u][e] = fg[u][e] = 0.f;
+      if (live) {
+        load8_f32(v + vo + static_cast<long>(c0 + t) * DV + j, fv[u]);
+        load8_f32(dy + vo + static_cast<long>(c0 + t) * DV + j, fg[u]);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < QI; ++u) {
+      const int i = tid + u * NT, t = i / (DK / 8), a = (i % (DK / 8)) * 8;
+      if (i >= C * DK / 8) continue;
+      const bool live = t < Cv;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        sQ[t * QS + a + e] = live ? feat_f32(fq[u][e], ident) : 0.f;
+        sK[t * QS + a + e] = live ? feat_f32(fk[u][e], ident) : 0.f;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < VI; ++u) {
+      const int i = tid + u * NT, t = i / (DV / 8), j = (i % (DV / 8)) * 8;
+      if (i >= C * DV / 8) continue;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) sV[t * VS + j + e] = fv[u][e];
+      *reinterpret_cast<float4 *>(&sG[t * DV + j]) = make_float4(fg[u][0], fg[u][1], fg[u][2], fg[u][3]);
+      *reinterpret_cast<float4 *>(&sG[t * DV + j + 4]) = make_float4(fg[u][4], fg[u][5], fg[u][6], fg[u][7]);
     }
   };
   // Every product below is a small matrix product over shared memory, tiled

@@ -24,6 +24,28 @@ __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
   return __float2bfloat16_rn(x);
 }
 
+// Eight consecutive elements as fp32, from an address aligned to eight
+// elements (one 16-byte load for bf16, two for fp32).
+template <typename T>
+__device__ __forceinline__ void load8_f32(const T *p, float (&f)[8]);
+template <>
+__device__ __forceinline__ void load8_f32<float>(const float *p, float (&f)[8]) {
+  const float4 a = reinterpret_cast<const float4 *>(p)[0];
+  const float4 b = reinterpret_cast<const float4 *>(p)[1];
+  f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
+  f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+}
+template <>
+__device__ __forceinline__ void load8_f32<__nv_bfloat16>(const __nv_bfloat16 *p, float (&f)[8]) {
+  const uint4 w = *reinterpret_cast<const uint4 *>(p);
+  const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(ww[i] << 16);
+    f[2 * i + 1] = __uint_as_float(ww[i] & 0xffff0000u);
+  }
+}
+
 // phi(x) = elu(x) + 1 (alpha = 1): x + 1 for x > 0, exp(x) otherwise.
 // Fast-weight article §4.1 (feature_map); linear-attention note §4.1.
 __device__ __forceinline__ float phi_f32(float x) { return x > 0.f ? x + 1.f : expf(x); }
