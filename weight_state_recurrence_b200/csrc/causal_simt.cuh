@@ -76,19 +76,46 @@ __global__ void __launch_bounds__(256) causal_simt_kernel(
   for (int c0 = n0; c0 < n1; c0 += C) {
     const int Cv = min(C, n1 - c0);
     __syncthreads();
-    for (int i = tid; i < C * DK; i += NT) {
-      const int t = i / DK, a = i % DK;
-      float fq = 0.f, fk = 0.f;
-      if (t < Cv) {
-        fq = feat_f32(to_f32(qp[static_cast<long>(c0 + t) * DK + a]), ident);
-        fk = feat_f32(to_f32(kp[static_cast<long>(c0 + t) * DK + a]), ident);
+    {
+      // eight elements per load, every load of the chunk in flight before the
+      // first shared-memory store
+      constexpr int QI = (C * DK / 8 + NT - 1) / NT, VI = (C * DVS / 8 + NT - 1) / NT;
+      float fq[QI][8], fk[QI][8], fv[VI][8];
+#pragma unroll
+      for (int u = 0; u < QI; ++u) {
+        const int i = tid + u * NT, t = i / (DK / 8), a = (i % (DK / 8)) * 8;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) fq[u][e] = fk[u][e] = 0.f;
+        if (i < C * DK / 8 && t < Cv) {
+          load8_f32(qp + static_cast<long>(c0 + t) * DK + a, fq[u]);
+          load8_f32(kp + static_cast<long>(c0 + t) * DK + a, fk[u]);
+        }
       }
-      sQ[t * QS + a] = fq;
-      sK[t * QS + a] = fk;
-    }
-    for (int i = tid; i < C * DVS; i += NT) {
-      const int t = i / DVS, j = i % DVS;
-      sV[i] = t < Cv ? to_f32(vp[static_cast<long>(c0 + t) * DV + j0 + j]) : 0.f;
+#pragma unroll
+      for (int u = 0; u < VI; ++u) {
+        const int i = tid + u * NT, t = i / (DVS / 8), j = (i % (DVS / 8)) * 8;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) fv[u][e] = 0.f;
+        if (i < C * DVS / 8 && t < Cv) load8_f32(vp + static_cast<long>(c0 + t) * DV + j0 + j, fv[u]);
+      }
+#pragma unroll
+      for (int u = 0; u < QI; ++u) {
+        const int i = tid + u * NT, t = i / (DK / 8), a = (i % (DK / 8)) * 8;
+        if (i >= C * DK / 8) continue;
+        const bool live = t < Cv;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          sQ[t * QS + a + e] = live ? feat_f32(fq[u][e], ident) : 0.f;
+          sK[t * QS + a + e] = live ? feat_f32(fk[u][e], ident) : 0.f;
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < VI; ++u) {
+        const int i = tid + u * NT;
+        if (i >= C * DVS / 8) continue;
+        *reinterpret_cast<float4 *>(&sV[8 * i]) = make_float4(fv[u][0], fv[u][1], fv[u][2], fv[u][3]);
+        *reinterpret_cast<float4 *>(&sV[8 * i + 4]) = make_float4(fv[u][4], fv[u][5], fv[u][6], fv[u][7]);
+      }
     }
     __syncthreads();
     // masked decayed scores and phi(q_t).z (z is still the state before the chunk)
@@ -222,14 +249,40 @@ __global__ void __launch_bounds__(256) causal_seg_state_kernel(
   for (int c0 = n0; c0 < n1; c0 += C) {
     const int Cv = min(C, n1 - c0);
     __syncthreads();
-    for (int i = tid; i < C * DK; i += NT) {
-      const int t = i / DK, a = i % DK;
-      sK[t * QS + a] = t < Cv ? pw[Cv - 1 - t] * feat_f32(to_f32(kp[static_cast<long>(c0 + t) * DK + a]), ident)
-                              : 0.f;
-    }
-    for (int i = tid; i < C * DVS; i += NT) {
-      const int t = i / DVS, j = i % DVS;
-      sV[t * (DVS + 1) + j] = t < Cv ? to_f32(vp[static_cast<long>(c0 + t) * DV + j0 + j]) : 0.f;
+    {
+      // eight elements per load, every load of the chunk in flight before the
+      // first shared-memory store
+      constexpr int KI = (C * DK / 8 + NT - 1) / NT, VI = (C * DVS / 8 + NT - 1) / NT;
+      float fk[KI][8], fv[VI][8];
+#pragma unroll
+      for (int u = 0; u < KI; ++u) {
+        const int i = tid + u * NT, t = i / (DK / 8), a = (i % (DK / 8)) * 8;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) fk[u][e] = 0.f;
+        if (i < C * DK / 8 && t < Cv) load8_f32(kp + static_cast<long>(c0 + t) * DK + a, fk[u]);
+      }
+#pragma unroll
+      for (int u = 0; u < VI; ++u) {
+        const int i = tid + u * NT, t = i / (DVS / 8), j = (i % (DVS / 8)) * 8;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) fv[u][e] = 0.f;
+        if (i < C * DVS / 8 && t < Cv) load8_f32(vp + static_cast<long>(c0 + t) * DV + j0 + j, fv[u]);
+      }
+#pragma unroll
+      for (int u = 0; u < KI; ++u) {
+        const int i = tid + u * NT, t = i / (DK / 8), a = (i % (DK / 8)) * 8;
+        if (i >= C * DK / 8) continue;
+        const float w = t < Cv ? pw[Cv - 1 - t] : 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) sK[t * QS + a + e] = t < Cv ? w * feat_f32(fk[u][e], ident) : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < VI; ++u) {
+        const int i = tid + u * NT, t = i / (DVS / 8), j = (i % (DVS / 8)) * 8;
+        if (i >= C * DVS / 8) continue;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) sV[t * (DVS + 1) + j + e] = fv[u][e];
+      }
     }
     __syncthreads();
     const float gC = pw[Cv];
