@@ -362,9 +362,10 @@ def global_leg(lib, args, world, rank, stream, hbm):
 
 
 def seg_leg(lib, args, world, rank, stream, hbm):
-    """The causal_d64 workload (B=2, H=8, N=4096, d=64, bf16, no decay), which
-    the CUDA-core path serves with 32 CTAs: one sequential pass per head and
-    dv slice, against the segment-parallel form with its workspace."""
+    """The causal_d64 workload (B=2, H=8, N=4096, d=64, bf16, no decay): the
+    product path (the tensor-core kernel in its d_k = 64 mode, 16 CTAs), and
+    for comparison the CUDA-core kernel (forced) in one sequential pass per
+    head and dv slice and in the segment-parallel form with its workspace."""
     w = inputs.WORKLOADS["causal_d64"]
     B, H, N, d = w.B, w.H, w.N, w.d
     dev = torch.device("cuda")
@@ -373,18 +374,28 @@ def seg_leg(lib, args, world, rank, stream, hbm):
     out = torch.empty_like(v)
     S = torch.empty(B, H, d, d, device=dev)
     z = torch.empty(B, H, d, device=dev)
+    os.environ["LINATTN_CAUSAL_KERNEL"] = "simt"
     need = lib.linattn_fwd_causal_workspace(B, H, N, d, d, w.dtype)
+    del os.environ["LINATTN_CAUSAL_KERNEL"]
     ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
     res = {"workload": "causal_d64: B=2 x H=8 x N=4096, d=64, bf16, no decay",
            "workspace_bytes": need}
     alg = causal_bytes(B, H, N, d, d)
-    for name, fn in (("single_pass", lambda: lib.linattn_fwd_causal(q, k, v, None, w.eps, out, S,
-                                                                     z, stream)),
-                     ("segmented", lambda: lib.linattn_fwd_causal_ws(q, k, v, None, w.eps, None,
-                                                                     None, out, S, z, ws,
-                                                                     stream))):
-        with torch.cuda.stream(stream):
-            ms = time_steps(fn, args.steps, args.warmup, world, stream)
+    legs = (("tensor_core", None, lambda: lib.linattn_fwd_causal(q, k, v, None, w.eps, out, S, z,
+                                                                 stream)),
+            ("cuda_core_single_pass", "simt",
+             lambda: lib.linattn_fwd_causal(q, k, v, None, w.eps, out, S, z, stream)),
+            ("cuda_core_segmented", "simt",
+             lambda: lib.linattn_fwd_causal_ws(q, k, v, None, w.eps, None, None, out, S, z, ws,
+                                               stream)))
+    for name, kernel, fn in legs:
+        if kernel:
+            os.environ["LINATTN_CAUSAL_KERNEL"] = kernel
+        try:
+            with torch.cuda.stream(stream):
+                ms = time_steps(fn, args.steps, args.warmup, world, stream)
+        finally:
+            os.environ.pop("LINATTN_CAUSAL_KERNEL", None)
         per = ms / 1e3 / args.steps
         res[name] = {"value": B * N * world / per, "unit": "tokens/s", "ms_per_step": per * 1e3,
                      "roofline": {"bound": "hbm", "achieved": alg / per / 1e9, "peak": hbm,

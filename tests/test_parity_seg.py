@@ -29,9 +29,11 @@ def run_ws(lib, q, k, v, lam, eps, S0=None, z0=None, ws_bytes=None):
     return need, out, S, z
 
 
-def test_causal_d64_workload_segmented(cuda_lib):
-    """The causal_d64 workload (16 heads, 4096 tokens, d = 64, bf16): the
-    CUDA-core path cut into segments."""
+def test_causal_d64_workload_segmented(cuda_lib, monkeypatch):
+    """The causal_d64 workload (16 heads, 4096 tokens, d = 64, bf16) on the
+    CUDA-core path (forced: bf16 with d_k = 64 normally takes the tensor
+    cores), cut into segments."""
+    monkeypatch.setenv("LINATTN_CAUSAL_KERNEL", "simt")
     w = inputs.WORKLOADS["causal_d64"]
     q, k, v = inputs.causal_inputs(w)
     need, out, S, z = run_ws(cuda_lib, q, k, v, None, w.eps)
@@ -68,7 +70,8 @@ def test_small_decay_segments(cuda_lib):
     assert_close("S_final", S, S_o, 1e-4)
 
 
-def test_small_workspace_runs_the_single_pass(cuda_lib):
+def test_small_workspace_runs_the_single_pass(cuda_lib, monkeypatch):
+    monkeypatch.setenv("LINATTN_CAUSAL_KERNEL", "simt")
     w = inputs.WORKLOADS["causal_d64"]
     q, k, v = inputs.causal_inputs(w, B=1, H=2, N=1024)
     need, out, S, z = run_ws(cuda_lib, q, k, v, None, w.eps, ws_bytes=64)
@@ -78,10 +81,15 @@ def test_small_workspace_runs_the_single_pass(cuda_lib):
     assert_close("S_final", S, S_o, 2e-2)
 
 
-def test_workspace_query(cuda_lib):
+def test_workspace_query(cuda_lib, monkeypatch):
     ws = cuda_lib.linattn_fwd_causal_workspace
-    assert ws(2, 8, 4096, 64, 64, torch.bfloat16) > 0        # 16 heads: segmented
+    assert ws(2, 8, 4096, 64, 64, torch.bfloat16) == 0       # tensor-core path (d_k = 64)
     assert ws(4, 16, 16384, 128, 128, torch.bfloat16) == 0   # tensor-core path
+    assert ws(2, 8, 4096, 32, 32, torch.bfloat16) > 0        # 16 heads on CUDA cores: segmented
+    assert ws(2, 8, 4096, 64, 64, torch.float32) > 0         # likewise
+    monkeypatch.setenv("LINATTN_CAUSAL_KERNEL", "simt")
+    assert ws(2, 8, 4096, 64, 64, torch.bfloat16) > 0        # forced CUDA cores: segmented
+    monkeypatch.delenv("LINATTN_CAUSAL_KERNEL")
     assert ws(64, 64, 4096, 64, 64, torch.float32) == 0      # enough heads already
     assert ws(1, 1, 100, 64, 64, torch.float32) == 0         # too short to cut
     assert ws(1, 1, 4096, 48, 64, torch.float32) == 0        # unsupported: no plan

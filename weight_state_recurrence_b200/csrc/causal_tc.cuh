@@ -1,5 +1,8 @@
 // Chunked causal forward on the 5th-generation tensor cores (bf16 operands,
-// fp32 accumulators in TMEM), d_k = 128, dv sliced 64 columns per CTA.
+// fp32 accumulators in TMEM), d_k = 128 or 64, dv sliced 64 columns per CTA.
+// With d_k = 64 the operand tiles keep their 128-column shape: the second
+// d_k panel of q and k is zero (loaded never, transformed never), so the score
+// and O_x chains skip its K steps and the state rows 64-127 stay zero.
 //
 // The method (fast-weight article §2.1/§3.2/§4.2 recurrence, §3.1
 // triangular-mask form, §4.1 note and §5.2 "cut the sequence into blocks:
@@ -264,7 +267,7 @@ __global__ void __launch_bounds__(NT, 1)
                      const __grid_constant__ CUtensorMap tm_v, const float *__restrict__ lam,
                      float eps, const float *__restrict__ S_init, const float *__restrict__ z_init,
                      __nv_bfloat16 *__restrict__ out, float *__restrict__ S_final,
-                     float *__restrict__ z_final, int H, int N, int DV, bool ident) {
+                     float *__restrict__ z_final, int H, int N, int DV, int dk, bool ident) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *sm = smem_raw;
   const uint32_t sb = smem_u32(sm);
@@ -302,6 +305,8 @@ __global__ void __launch_bounds__(NT, 1)
   float *qf = reinterpret_cast<float *>(misc + kMiscQf);
   float *qt = reinterpret_cast<float *>(misc + kMiscQt);
   const bool factored = L >= kFactorMin;   // uniform over the CTA (and its peer)
+  const bool dk64 = dk == 64;              // only the first d_k panel holds data
+  const int kpanels = dk64 ? 1 : 2;
 
   // ------------------------------------------------------------ set-up
   if (tid == 0) {
@@ -327,6 +332,12 @@ __global__ void __launch_bounds__(NT, 1)
   }
   for (uint32_t o = tid * 16u; o < 2 * kPanel; o += NT * 16u)
     *reinterpret_cast<uint4 *>(sm + kOffA + o) = make_uint4(0, 0, 0, 0);
+  if (dk64)   // the second d_k panel of the q and k tiles of both stages stays zero
+    for (uint32_t o = tid * 16u; o < 4 * kPanel; o += NT * 16u) {
+      const uint32_t st = (o / (2 * kPanel)) * kStage, w = o % (2 * kPanel);
+      *reinterpret_cast<uint4 *>(sm + st + (w < kPanel ? kOffQ : kOffK - kPanel) + kPanel + w) =
+          make_uint4(0, 0, 0, 0);
+    }
   __syncthreads();
   if (tid < C) {
     *reinterpret_cast<__nv_bfloat16 *>(sm + kOffX + sw128_offset(tid, 0)) =
@@ -350,16 +361,17 @@ __global__ void __launch_bounds__(NT, 1)
   if (has_init) {
     if (warp >= 12 && warp < 16) {
       const int r = (warp - 12) * 32 + lane;   // d_k row
+      const bool live = r < dk;
       const uint32_t lane_field = static_cast<uint32_t>((warp - 12) * 32) << 16;
       const float g0 = pw[nchunks == 1 ? Ct : C];   // decay of the first chunk
-      const float4 *src =
-          reinterpret_cast<const float4 *>(S_init + (static_cast<long>(pair) * DK + r) * DV + j0);
+      const float4 *src = reinterpret_cast<const float4 *>(
+          S_init + (static_cast<long>(pair) * dk + (live ? r : 0)) * DV + j0);
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         uint32_t sv[32], pk[16];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          const float4 f = src[half * 8 + i];
+          const float4 f = live ? src[half * 8 + i] : make_float4(0.f, 0.f, 0.f, 0.f);
           sv[4 * i] = __float_as_uint(f.x * g0);
           sv[4 * i + 1] = __float_as_uint(f.y * g0);
           sv[4 * i + 2] = __float_as_uint(f.z * g0);
@@ -373,7 +385,7 @@ __global__ void __launch_bounds__(NT, 1)
           *reinterpret_cast<uint4 *>(sm + kOffS + sw128_offset(r, half * 64 + i * 16)) =
               make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
       }
-      const float z0 = z_init[static_cast<long>(pair) * DK + r];
+      const float z0 = live ? z_init[static_cast<long>(pair) * dk + r] : 0.f;
       uint32_t zcol[16];
       zcol[0] = __float_as_uint(z0 * g0);
 #pragma unroll
@@ -416,20 +428,24 @@ __global__ void __launch_bounds__(NT, 1)
           // this CTA's MMAs are done with the stage: the peer may write its rows into it
           if (kPair && c >= 2) mbar_arrive_remote(map_to_rank(bar(kPeerFree0 + s), peer));
           const uint32_t b = bar(kFullQK0 + s);
-          mbar_arrive_expect_tx(b, kPair ? kQKTxBytes / 2 : kQKTxBytes);
+          mbar_arrive_expect_tx(b, (kPair ? kQKTxBytes / 2 : kQKTxBytes) / (dk64 ? 2 : 1));
           const int y = c * C + row0;
           tma_load_3d(base + kOffQ + own_off, &tm_q, b, 0, y, pair);
           tma_load_3d(base + kOffK + own_off, &tm_k, b, 0, y, pair);
-          tma_load_3d(base + kOffQ + kPanel + own_off, &tm_q, b, 64, y, pair);
-          tma_load_3d(base + kOffK + kPanel + own_off, &tm_k, b, 64, y, pair);
+          if (!dk64) {
+            tma_load_3d(base + kOffQ + kPanel + own_off, &tm_q, b, 64, y, pair);
+            tma_load_3d(base + kOffK + kPanel + own_off, &tm_k, b, 64, y, pair);
+          }
           // the same rows two chunks ahead into L2, so that their load, issued
           // when this stage frees up again, does not wait on HBM
           if (c + kPrefetch < nchunks) {
             const int yp = y + kPrefetch * C;
             tma_prefetch_l2_3d(&tm_q, 0, yp, pair);
             tma_prefetch_l2_3d(&tm_k, 0, yp, pair);
-            tma_prefetch_l2_3d(&tm_q, 64, yp, pair);
-            tma_prefetch_l2_3d(&tm_k, 64, yp, pair);
+            if (!dk64) {
+              tma_prefetch_l2_3d(&tm_q, 64, yp, pair);
+              tma_prefetch_l2_3d(&tm_k, 64, yp, pair);
+            }
           }
           LINATTN_TRACE_EVENT(c, 0);
         } else {
@@ -461,6 +477,7 @@ __global__ void __launch_bounds__(NT, 1)
         const uint32_t st = sb + s * kStage;
 #pragma unroll
         for (int ks = 0; ks < DK / 16; ++ks) {
+          if (ks >= 4 * kpanels) break;   // the zero second panel adds nothing
           // d_k half 0 (ks < 4) and half 1 become ready separately
           if ((ks & 3) == 0) {
             if (!mbar_wait(bar((ks == 0 ? kPhi0 : kPhiB0) + s), (c >> 1) & 1)) return false;
@@ -505,6 +522,7 @@ __global__ void __launch_bounds__(NT, 1)
         LINATTN_TRACE_EVENT(c, 6);
 #pragma unroll
         for (int ks = 0; ks < DK / 16; ++ks) {
+          if (ks >= 4 * kpanels) break;
           const uint32_t off = (ks >> 2) * kPanel + (ks & 3) * 32;
           umma_bf16(tmem + kTmOX, sdesc_sw128(st + kOffQ + off, 16, 1024),
                     sdesc_sw128(sb + kOffS + ks * 2048, kOffX - kOffS, 1024), kIdN80, ks > 0);
@@ -553,7 +571,7 @@ __global__ void __launch_bounds__(NT, 1)
       if (tt == 0) LINATTN_TRACE_EVENT(c, 1);
       // this CTA's rows, one d_k half (q panel g and k panel g) at a time
       const bool tail = c == nchunks - 1;
-      for (int g = 0; g < 2; ++g) {
+      for (int g = 0; g < kpanels; ++g) {
         uint8_t *base = sm + s * kStage + kOffQ + g * kPanel;
         if (!rf && (factored || !ident))
           phi_pass<4>(base + own_off, own_bytes, 2 * kPanel, 2, row0, tail ? qt : qf,
@@ -697,9 +715,9 @@ __global__ void __launch_bounds__(NT, 1)
           tmem_ld_32x32b_x32(tmem + lane_field + kTmS + half * 32, sv);
           tmem_wait_ld();
           if (last) {
-            if (S_final) {
+            if (S_final && r < dk) {
               float4 *dst = reinterpret_cast<float4 *>(
-                  S_final + (static_cast<long>(pair) * DK + r) * DV + j0 + half * 32);
+                  S_final + (static_cast<long>(pair) * dk + r) * DV + j0 + half * 32);
 #pragma unroll
               for (int i = 0; i < 8; ++i)
                 dst[i] = make_float4(__uint_as_float(sv[4 * i]), __uint_as_float(sv[4 * i + 1]),
@@ -721,7 +739,7 @@ __global__ void __launch_bounds__(NT, 1)
         }
         const float zc = __uint_as_float(zz[0]);
         if (last) {
-          if (z_final && j0 == 0) z_final[static_cast<long>(pair) * DK + r] = zc;
+          if (z_final && j0 == 0 && r < dk) z_final[static_cast<long>(pair) * dk + r] = zc;
         } else {
           // z (decayed) back into column 64; the other side columns restart at 0
           uint32_t zcol[16];

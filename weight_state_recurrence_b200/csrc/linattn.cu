@@ -129,12 +129,12 @@ bool make_map_bf16(CUtensorMap *m, const void *ptr, int inner, int rows, int pla
 }
 
 // Which causal kernel: LINATTN_CAUSAL_KERNEL=simt forces the CUDA-core
-// kernel (a second opinion for tests); otherwise bf16 with d_k = 128 and dv
-// a multiple of 64 takes the tensor-core kernel.
+// kernel (a second opinion for tests); otherwise bf16 with d_k = 128 or 64
+// and dv a multiple of 64 takes the tensor-core kernel.
 bool use_tc_causal(const linattn_dims *d) {
   const char *e = std::getenv("LINATTN_CAUSAL_KERNEL");
   if (e && std::strcmp(e, "simt") == 0) return false;
-  return d->dtype == LINATTN_BF16 && d->dk == tc::DK && d->dv % tc::DVS == 0;
+  return d->dtype == LINATTN_BF16 && (d->dk == tc::DK || d->dk == 64) && d->dv % tc::DVS == 0;
 }
 
 // ------------------------------------------------------------ launchers
@@ -302,7 +302,7 @@ int launch_causal_tc(const linattn_dims *d, const void *q, const void *k, const 
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   if (cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, lam, eps, S_init, z_init,
-                         static_cast<bf16 *>(out), S_final, z_final, d->H, d->N, d->dv,
+                         static_cast<bf16 *>(out), S_final, z_final, d->H, d->N, d->dv, d->dk,
                          ident(d)) != cudaSuccess)
     return LINATTN_ERR_CUDA;
   return launch_status();
