@@ -260,14 +260,14 @@ __device__ __forceinline__ void phi_pass(uint8_t *p, uint32_t own_bytes, uint32_
   }
 }
 
-template <bool kPair>
+template <bool kPair, bool kDk64>
 __global__ void __launch_bounds__(NT, 1)
     causal_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                      const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const float *__restrict__ lam,
                      float eps, const float *__restrict__ S_init, const float *__restrict__ z_init,
                      __nv_bfloat16 *__restrict__ out, float *__restrict__ S_final,
-                     float *__restrict__ z_final, int H, int N, int DV, int dk, bool ident) {
+                     float *__restrict__ z_final, int H, int N, int DV, bool ident) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *sm = smem_raw;
   const uint32_t sb = smem_u32(sm);
@@ -305,8 +305,9 @@ __global__ void __launch_bounds__(NT, 1)
   float *qf = reinterpret_cast<float *>(misc + kMiscQf);
   float *qt = reinterpret_cast<float *>(misc + kMiscQt);
   const bool factored = L >= kFactorMin;   // uniform over the CTA (and its peer)
-  const bool dk64 = dk == 64;              // only the first d_k panel holds data
-  const int kpanels = dk64 ? 1 : 2;
+  constexpr bool dk64 = kDk64;             // only the first d_k panel holds data
+  constexpr int kpanels = kDk64 ? 1 : 2;
+  constexpr int dk = kDk64 ? 64 : DK;      // the caller's d_k (state layout)
 
   // ------------------------------------------------------------ set-up
   if (tid == 0) {
@@ -361,7 +362,7 @@ __global__ void __launch_bounds__(NT, 1)
   if (has_init) {
     if (warp >= 12 && warp < 16) {
       const int r = (warp - 12) * 32 + lane;   // d_k row
-      const bool live = r < dk;
+      const bool live = !kDk64 || r < dk;
       const uint32_t lane_field = static_cast<uint32_t>((warp - 12) * 32) << 16;
       const float g0 = pw[nchunks == 1 ? Ct : C];   // decay of the first chunk
       const float4 *src = reinterpret_cast<const float4 *>(
@@ -715,7 +716,7 @@ __global__ void __launch_bounds__(NT, 1)
           tmem_ld_32x32b_x32(tmem + lane_field + kTmS + half * 32, sv);
           tmem_wait_ld();
           if (last) {
-            if (S_final && r < dk) {
+            if (S_final && (!kDk64 || r < dk)) {
               float4 *dst = reinterpret_cast<float4 *>(
                   S_final + (static_cast<long>(pair) * dk + r) * DV + j0 + half * 32);
 #pragma unroll
@@ -739,7 +740,7 @@ __global__ void __launch_bounds__(NT, 1)
         }
         const float zc = __uint_as_float(zz[0]);
         if (last) {
-          if (z_final && j0 == 0 && r < dk) z_final[static_cast<long>(pair) * dk + r] = zc;
+          if (z_final && j0 == 0 && (!kDk64 || r < dk)) z_final[static_cast<long>(pair) * dk + r] = zc;
         } else {
           // z (decayed) back into column 64; the other side columns restart at 0
           uint32_t zcol[16];

@@ -287,7 +287,9 @@ int launch_causal_tc(const linattn_dims *d, const void *q, const void *k, const 
   if (!make_map_bf16(&mq, q, d->dk, d->N, BH, qk_rows) ||
       !make_map_bf16(&mk, k, d->dk, d->N, BH, qk_rows) || !make_map_bf16(&mv, v, d->dv, d->N, BH))
     return LINATTN_ERR_CUDA;
-  auto *kern = paired ? tc::causal_tc_kernel<true> : tc::causal_tc_kernel<false>;
+  const bool half = d->dk == 64;   // d_k = 64: the kernel's second d_k panel stays zero
+  auto *kern = paired ? (half ? tc::causal_tc_kernel<true, true> : tc::causal_tc_kernel<true, false>)
+                      : (half ? tc::causal_tc_kernel<false, true> : tc::causal_tc_kernel<false, false>);
   if (!set_smem(kern, static_cast<int>(tc::kSmemBytes))) return LINATTN_ERR_CUDA;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(BH * (d->dv / tc::DVS));
@@ -302,7 +304,7 @@ int launch_causal_tc(const linattn_dims *d, const void *q, const void *k, const 
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   if (cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, lam, eps, S_init, z_init,
-                         static_cast<bf16 *>(out), S_final, z_final, d->H, d->N, d->dv, d->dk,
+                         static_cast<bf16 *>(out), S_final, z_final, d->H, d->N, d->dv,
                          ident(d)) != cudaSuccess)
     return LINATTN_ERR_CUDA;
   return launch_status();
