@@ -102,6 +102,10 @@ enum {
  *   z_final [B, H, dk]     fp32 or NULL   normaliser after the last token
  * The starting state is zero ([FW] §4.1 init_state, [LN] §6 init_state).
  * N = 0 writes zero S_final / z_final and nothing else.
+ * Kernels: bf16 with dk in {64, 128} and dv a multiple of 64 runs on the
+ * tensor cores (bf16 operands, fp32 accumulators and state); everything else
+ * runs on CUDA cores in fp32 arithmetic, cut into sequence segments when there
+ * are too few heads to fill the GPU (linattn_fwd_causal_workspace).
  */
 LINATTN_API int linattn_fwd_causal(const linattn_dims *dims, const void *q, const void *k,
                        const void *v, const float *lambda, float eps, void *out,
@@ -142,7 +146,9 @@ LINATTN_API int linattn_fwd_causal_from(const linattn_dims *dims, const void *q,
  *
  * linattn_fwd_causal_workspace: the bytes of workspace the segmented form
  *   needs for these dims (0: the single pass is used; also for invalid dims).
- *   Only the CUDA-core path (fp32 inputs, or d_k != 128) is segmented.
+ *   Only the CUDA-core path is segmented: fp32 inputs, or d_k in {16, 32}, or d_v
+ *   not a multiple of 64.  bf16 with d_k in {64, 128} and d_v a multiple of 64 runs
+ *   on the tensor cores in one pass (workspace 0).
  * linattn_fwd_causal_ws: linattn_fwd_causal_from with a caller-owned device
  *   workspace (16-byte aligned, overlapping no other argument, contents
  *   irrelevant and overwritten); with workspace_bytes below the size above,
