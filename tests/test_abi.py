@@ -226,3 +226,48 @@ def test_performer_features_rejects_bad_arguments(lib):
 
 def test_performer_features_zero_rows_is_a_no_op(lib):
     assert feats(lib, rows=0, x=None, w=None, out=None) == linattn.LINATTN_OK
+
+
+def test_python_binding_checks_performer_shapes():
+    import torch
+    x = torch.zeros(3, 64, dtype=torch.bfloat16)
+    w = torch.zeros(32, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):      # omega's d differs from x's
+        linattn.linattn_performer_features(x, torch.zeros(32, 16, dtype=torch.bfloat16), 0,
+                                           torch.zeros(3, 64, dtype=torch.bfloat16))
+    with pytest.raises(ValueError):      # out must hold 2m features per row
+        linattn.linattn_performer_features(x, w, 0, torch.zeros(3, 32, dtype=torch.bfloat16))
+    with pytest.raises(ValueError):      # one dtype for x, omega and out
+        linattn.linattn_performer_features(x, w.float(), 0, torch.zeros(3, 64, dtype=torch.bfloat16))
+    with pytest.raises(ValueError):      # omega must be [m, d]
+        linattn.linattn_performer_features(x, torch.zeros(2, 32, 64, dtype=torch.bfloat16), 0,
+                                           torch.zeros(3, 64, dtype=torch.bfloat16))
+
+
+def test_python_binding_passes_phi_into_the_dims():
+    import torch
+    captured = {}
+
+    class FakeLib:
+        def linattn_fwd_causal(self, d, *args):
+            captured["phi"] = d._obj.phi
+            captured["dtype"] = d._obj.dtype
+            return linattn.LINATTN_OK
+
+    real = linattn._lib
+    try:
+        linattn._lib = FakeLib()
+        # tensors on the CPU never reach a kernel: the fake library records the dims
+        orig_ptr = linattn._ptr
+        linattn._ptr = lambda t: None
+        try:
+            q = torch.zeros(1, 2, 4, 64, dtype=torch.bfloat16)
+            linattn.linattn_fwd_causal(q, q, q, None, 1e-6, q, stream=0,
+                                       phi=linattn.LINATTN_PHI_IDENTITY)
+            assert captured == {"phi": 1, "dtype": linattn.LINATTN_BF16}
+            linattn.linattn_fwd_causal(q, q, q, None, 1e-6, q, stream=0)
+            assert captured["phi"] == linattn.LINATTN_PHI_ELU1
+        finally:
+            linattn._ptr = orig_ptr
+    finally:
+        linattn._lib = real
