@@ -320,6 +320,10 @@ __global__ void __launch_bounds__(256) causal_seg_combine_kernel(
     const float *__restrict__ lam, const float *__restrict__ S_init,
     const float *__restrict__ z_init, float *__restrict__ ws_S, float *__restrict__ ws_z, int H,
     int DK, int DV, int N, int seg_len, int G) {
+  // blockIdx.x: the (b, h) pair; blockIdx.y: a block of 256 of its DK*DV + DK
+  // state elements, one per thread.  Each element's G segment values are read
+  // eight at a time before any is overwritten, so a thread has eight loads in
+  // flight instead of one per step of its scan.
   __shared__ float decay[64];       // lambda^len_g
   const long pair = blockIdx.x;
   const float L = lam ? lam[pair % H] : 1.f;
@@ -327,17 +331,28 @@ __global__ void __launch_bounds__(256) causal_seg_combine_kernel(
     decay[gg] = pow_int(L, min(seg_len, N - gg * seg_len));
   __syncthreads();
   const long per = static_cast<long>(DK) * DV;
-  for (long e = threadIdx.x; e < per + DK; e += blockDim.x) {
-    const bool isz = e >= per;
-    const long ei = isz ? e - per : e;
-    float *base = isz ? ws_z + pair * G * static_cast<long>(DK) : ws_S + pair * G * per;
-    const long stride = isz ? DK : per;
-    const float *init = isz ? z_init : S_init;
-    float run = init ? init[pair * stride + ei] : 0.f;
-    for (int gg = 0; gg < G; ++gg) {
-      const float d = gg < G - 1 ? base[gg * stride + ei] : 0.f;
-      base[gg * stride + ei] = run;
-      run = fmaf(decay[gg], run, d);
+  const long e = static_cast<long>(blockIdx.y) * blockDim.x + threadIdx.x;
+  if (e >= per + DK) return;
+  const bool isz = e >= per;
+  const long ei = isz ? e - per : e;
+  float *base = isz ? ws_z + pair * G * static_cast<long>(DK) : ws_S + pair * G * per;
+  const long stride = isz ? DK : per;
+  const float *init = isz ? z_init : S_init;
+  float run = init ? init[pair * stride + ei] : 0.f;
+  for (int g0 = 0; g0 < G; g0 += 8) {
+    float d[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int gg = g0 + j;
+      d[j] = gg < G - 1 ? base[gg * stride + ei] : 0.f;
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int gg = g0 + j;
+      if (gg < G) {
+        base[gg * stride + ei] = run;
+        run = fmaf(decay[gg], run, d[j]);
+      }
     }
   }
 }

@@ -238,8 +238,9 @@ int launch_causal_simt(const linattn_dims *d, const void *q, const void *k, cons
         static_cast<const T *>(k), static_cast<const T *>(v), lam, wsS, wsz, d->H, d->N, d->dv,
         sg.len, sg.G, ident(d));
     if (cudaGetLastError() != cudaSuccess) return LINATTN_ERR_CUDA;
-    causal_seg_combine_kernel<<<d->B * d->H, 256, 0, s>>>(lam, S_init, z_init, wsS, wsz, d->H,
-                                                          d->dk, d->dv, d->N, sg.len, sg.G);
+    const int eblocks = (d->dk * d->dv + d->dk + 255) / 256;
+    causal_seg_combine_kernel<<<dim3(d->B * d->H, eblocks), 256, 0, s>>>(
+        lam, S_init, z_init, wsS, wsz, d->H, d->dk, d->dv, d->N, sg.len, sg.G);
     if (cudaGetLastError() != cudaSuccess) return LINATTN_ERR_CUDA;
   }
   kern<<<dim3(ctas, sg.G), 256, bytes, s>>>(
