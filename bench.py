@@ -67,15 +67,15 @@ def causal_bytes(B, H, N, dk, dv, es=2):
 
 
 def causal_mma_flops(B, H, N, dk, dv):
-    """MMA flops the tensor-core kernel executes per launch (C = 128, dv
-    sliced 64 per CTA).  Per 128-token chunk and slice: scores 128x128xdk;
-    O_in, O_x and the state update 128x64x128 each; row sums, phi(q).z and
-    dz 128x16x128 each."""
+    """MMA flops the segmented tensor-core causal kernel executes per launch
+    (C = 128 tokens per chunk, one CTA per head with the whole dv).  Per chunk
+    and head: the score tile 128x128xdk, the carried term 128xdvxdk, the state
+    update 128xdvx128 (its M is the 128 rows of d_k, zero-padded for
+    dk = 64) and the intra term 128xdvx128."""
     C = 128
     chunks = -(-N // C)
-    slices = dv // 64
-    per = 2 * (C * C * dk + 3 * C * 64 * 128 + 3 * C * 16 * 128)
-    return B * H * slices * chunks * per
+    per = 2 * C * (C * dk + dv * dk + dv * 128 + dv * C)
+    return B * H * chunks * per
 
 
 def decode_bytes(B, H, dk, dv, es=2):
@@ -232,29 +232,52 @@ def causal_leg(lib, args, world, rank, stream, hbm, tc_peak):
     S = torch.empty(B, H, d, d, device=dev)
     z = torch.empty(B, H, d, device=dev)
 
+    ws = None
+    seg_launches = 1
+    if args.segments:
+        # the segmented form asked for explicitly (state pass, combine scan,
+        # then all segments at once), through the workspace entry point
+        with lib.kernel_choice(lib.LINATTN_OP_CAUSAL, lib.LINATTN_KERNEL_AUTO, args.segments):
+            need = lib.linattn_fwd_causal_workspace(B, H, N, d, d, WL.dtype)
+        ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+        seg_launches = 3 if need > 0 else 1   # state pass, combine scan, forward
+
+    ops = wdist.LibraryOps(lib, stream)
+
     def step():
-        lib.linattn_fwd_causal(q, k, v, lam, WL.eps, out, S, z, stream)
+        if args.seq_parallel:
+            # this rank holds tokens [rank N, (rank + 1) N) of sequences of
+            # world * N tokens: own segment state, one all-gather, the scan,
+            # then the segment's forward from its starting state
+            wdist.seq_parallel_causal(q, k, v, lam, WL.eps, world=world, rank=rank, seg_len=N,
+                                      ops=ops)
+        elif ws is None:
+            lib.linattn_fwd_causal(q, k, v, lam, WL.eps, out, S, z, stream)
+        else:
+            lib.linattn_fwd_causal_ws(q, k, v, lam, WL.eps, None, None, out, S, z, ws, stream)
 
     with torch.cuda.stream(stream):
         with ClockSampler(torch.cuda.current_device()) as clk:
-            ms = time_steps(step, args.steps, args.warmup, world, stream)
+            with lib.kernel_choice(lib.LINATTN_OP_CAUSAL, lib.LINATTN_KERNEL_AUTO, args.segments):
+                ms = time_steps(step, args.steps, args.warmup, world, stream)
     assert lib.linattn_device_status(clear=True, stream=stream) == 0, "device error flag set"
     per_launch_s = ms / 1e3 / args.steps
     tokens = B * N * world * args.steps
     value = tokens / (ms / 1e3)
     alg = causal_bytes(B, H, N, d, d)
     flops = causal_mma_flops(B, H, N, d, d)
-    traffic = traffic_record("causal_tc_kernel")
+    traffic = traffic_record("causal_seg_tc_kernel")
     roof = {"bound": "hbm", "achieved": alg / per_launch_s / 1e9, "peak": hbm, "unit": "GB/s",
             "frac": alg / per_launch_s / 1e9 / hbm, "traffic": traffic,
-            "algorithmic_bytes_per_launch": alg, "kernel": "causal_tc_kernel",
+            "algorithmic_bytes_per_launch": alg, "kernel": "causal_seg_tc_kernel",
             "tensor": {"mma_tflops": flops / per_launch_s / 1e12, "peak": tc_peak,
                        "frac": flops / per_launch_s / 1e12 / tc_peak,
                        "mma_flops_per_launch": flops}}
+    launches = args.steps * (3 if args.seq_parallel else seg_launches)
     res = {"ms_per_step": ms / args.steps, "value": value, "roofline": roof,
-           "clocks": clk.summary(), "gpu_launches": args.steps}
+           "clocks": clk.summary(), "gpu_launches": launches}
 
-    if args.e2e:
+    if args.e2e and not args.seq_parallel:
         # through the public API with host buffers (fwd_causal_host): every
         # step copies q, k, v in from pinned host memory and y, S_final,
         # z_final back, four heads at a time on overlapping streams
@@ -363,9 +386,10 @@ def global_leg(lib, args, world, rank, stream, hbm):
 
 def seg_leg(lib, args, world, rank, stream, hbm):
     """The causal_d64 workload (B=2, H=8, N=4096, d=64, bf16, no decay): the
-    product path (the tensor-core kernel in its d_k = 64 mode, 16 CTAs), and
-    for comparison the CUDA-core kernel (forced) in one sequential pass per
-    head and dv slice and in the segment-parallel form with its workspace."""
+    product path (the tensor-core kernel cut into about one segment per SM,
+    with its state pass and combine scan, through linattn_fwd_causal_ws), the
+    same kernel in one pass (16 CTAs), and for comparison the CUDA-core kernel
+    in one pass and segmented."""
     w = inputs.WORKLOADS["causal_d64"]
     B, H, N, d = w.B, w.H, w.N, w.d
     dev = torch.device("cuda")
@@ -374,28 +398,28 @@ def seg_leg(lib, args, world, rank, stream, hbm):
     out = torch.empty_like(v)
     S = torch.empty(B, H, d, d, device=dev)
     z = torch.empty(B, H, d, device=dev)
-    os.environ["LINATTN_CAUSAL_KERNEL"] = "simt"
-    need = lib.linattn_fwd_causal_workspace(B, H, N, d, d, w.dtype)
-    del os.environ["LINATTN_CAUSAL_KERNEL"]
-    ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    need_tc = lib.linattn_fwd_causal_workspace(B, H, N, d, d, w.dtype)
+    with lib.kernel_choice(lib.LINATTN_OP_CAUSAL, lib.LINATTN_KERNEL_CUDA_CORES):
+        need_cc = lib.linattn_fwd_causal_workspace(B, H, N, d, d, w.dtype)
+    ws = torch.empty(max(need_tc, need_cc, 16), dtype=torch.uint8, device=dev)
     res = {"workload": "causal_d64: B=2 x H=8 x N=4096, d=64, bf16, no decay",
-           "workspace_bytes": need}
+           "workspace_bytes": need_tc}
     alg = causal_bytes(B, H, N, d, d)
-    legs = (("tensor_core", None, lambda: lib.linattn_fwd_causal(q, k, v, None, w.eps, out, S, z,
-                                                                 stream)),
-            ("cuda_core_single_pass", "simt",
+    auto, cc = lib.LINATTN_KERNEL_AUTO, lib.LINATTN_KERNEL_CUDA_CORES
+    legs = (("tensor_core", auto,
+             lambda: lib.linattn_fwd_causal_ws(q, k, v, None, w.eps, None, None, out, S, z, ws,
+                                               stream)),
+            ("tensor_core_single_pass", auto,
              lambda: lib.linattn_fwd_causal(q, k, v, None, w.eps, out, S, z, stream)),
-            ("cuda_core_segmented", "simt",
+            ("cuda_core_single_pass", cc,
+             lambda: lib.linattn_fwd_causal(q, k, v, None, w.eps, out, S, z, stream)),
+            ("cuda_core_segmented", cc,
              lambda: lib.linattn_fwd_causal_ws(q, k, v, None, w.eps, None, None, out, S, z, ws,
                                                stream)))
     for name, kernel, fn in legs:
-        if kernel:
-            os.environ["LINATTN_CAUSAL_KERNEL"] = kernel
-        try:
+        with lib.kernel_choice(lib.LINATTN_OP_CAUSAL, kernel):
             with torch.cuda.stream(stream):
                 ms = time_steps(fn, args.steps, args.warmup, world, stream)
-        finally:
-            os.environ.pop("LINATTN_CAUSAL_KERNEL", None)
         per = ms / 1e3 / args.steps
         res[name] = {"value": B * N * world / per, "unit": "tokens/s", "ms_per_step": per * 1e3,
                      "roofline": {"bound": "hbm", "achieved": alg / per / 1e9, "peak": hbm,
@@ -509,7 +533,7 @@ def performer_leg(lib, args, world, rank, stream, hbm):
                                      "unit": "GB/s", "frac": fb / per_f / 1e9 / hbm,
                                      "algorithmic_bytes_per_launch": fb,
                                      "traffic": traffic_record("performer_tc_kernel")}},
-           "attention": {"kernel": "causal_tc_kernel (identity features)",
+           "attention": {"kernel": "causal_seg_tc_kernel (identity features)",
                          "ms_per_launch": per_a * 1e3,
                          "roofline": {"bound": "hbm", "achieved": ab / per_a / 1e9, "peak": hbm,
                                       "unit": "GB/s", "frac": ab / per_a / 1e9 / hbm,
@@ -591,6 +615,12 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--segments", type=int, default=0,
+                    help="causal leg: ask for at most this many segments per sequence "
+                         "(0: the library's plan)")
+    ap.add_argument("--seq-parallel", action="store_true",
+                    help="causal leg: split each sequence by token position across the "
+                         "ranks (each rank N tokens; one all-gather of segment states)")
     ap.add_argument("--no-e2e", dest="e2e", action="store_false")
     ap.add_argument("--no-legs", dest="legs", action="store_false")
     ap.add_argument("--no-cpu-baseline", dest="cpu", action="store_false")
@@ -635,8 +665,13 @@ def main():
         "data": "synthetic (seeded torch RNG on the device, N(0,1)/sqrt(d))",
         "config": {"workload": f"causal_decay_d128: B={B} x H=16 x N=16384, d_k=d_v=128, bf16 "
                                "q/k/v, lambda_h=linspace(0.9,0.999,16), fp32 S/z, eps=1e-6",
-                   "global_batch": B * world, "seq_len": WL.N, "heads": WL.H, "d": WL.d,
-                   "parallelism": f"dp{world} (batch sharded, no data-path collective)",
+                   "global_batch": B if args.seq_parallel else B * world,
+                   "seq_len": WL.N * (world if args.seq_parallel else 1), "heads": WL.H,
+                   "d": WL.d,
+                   "parallelism": (f"sp{world} (each sequence split by token position, "
+                                   f"{WL.N} tokens per rank; one all-gather of segment "
+                                   "states)") if args.seq_parallel else
+                                  f"dp{world} (batch sharded, no data-path collective)",
                    "l2": f"inputs larger than L2 ({3 * B * WL.H * WL.N * WL.d * 2 / 1e6:.0f} MB "
                          "per step)"},
         "roofline": res["roofline"], "clocks": res["clocks"],

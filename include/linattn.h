@@ -102,10 +102,11 @@ enum {
  *   z_final [B, H, dk]     fp32 or NULL   normaliser after the last token
  * The starting state is zero ([FW] §4.1 init_state, [LN] §6 init_state).
  * N = 0 writes zero S_final / z_final and nothing else.
- * Kernels: bf16 with dk in {64, 128} and dv a multiple of 64 runs on the
- * tensor cores (bf16 operands, fp32 accumulators and state); everything else
- * runs on CUDA cores in fp32 arithmetic, cut into sequence segments when there
- * are too few heads to fill the GPU (linattn_fwd_causal_workspace).
+ * Kernels: bf16 with dk and dv in {64, 128} runs on the tensor cores (bf16
+ * operands, fp32 accumulators and state), one CTA per (b, h) with the whole
+ * dv; everything else runs on CUDA cores in fp32 arithmetic.  Both are cut
+ * into sequence segments when there are too few heads to fill the GPU and
+ * the caller supplies a workspace (linattn_fwd_causal_ws).
  */
 LINATTN_API int linattn_fwd_causal(const linattn_dims *dims, const void *q, const void *k,
                        const void *v, const float *lambda, float eps, void *out,
@@ -145,10 +146,12 @@ LINATTN_API int linattn_fwd_causal_from(const linattn_dims *dims, const void *q,
  * summation order.
  *
  * linattn_fwd_causal_workspace: the bytes of workspace the segmented form
- *   needs for these dims (0: the single pass is used; also for invalid dims).
- *   Only the CUDA-core path is segmented: fp32 inputs, or d_k in {16, 32}, or d_v
- *   not a multiple of 64.  bf16 with d_k in {64, 128} and d_v a multiple of 64 runs
- *   on the tensor cores in one pass (workspace 0).
+ *   needs for these dims on this device (0: the single pass is used; also for
+ *   invalid dims): B*H*G*(dk*dv + dk)*4 bytes for G segments.  G is chosen so
+ *   that B*H*G is about the number of SMs; with B*H above a third of them the
+ *   single pass is used.  On the tensor-core path the segment states come from
+ *   a tensor-core state pass that reads k and v of every segment but the last
+ *   once more.
  * linattn_fwd_causal_ws: linattn_fwd_causal_from with a caller-owned device
  *   workspace (16-byte aligned, overlapping no other argument, contents
  *   irrelevant and overwritten); with workspace_bytes below the size above,
@@ -162,16 +165,81 @@ LINATTN_API int linattn_fwd_causal_ws(const linattn_dims *dims, const void *q, c
                        size_t workspace_bytes, linattn_stream_t stream);
 
 /*
- * linattn_fwd_causal (zero starting state) without a caller workspace: the
- * segmented form uses a 16 MB device array that the library holds for every
- * device it is loaded on, and falls back to the single pass when the
- * workspace it needs is larger.  That array is shared by all calls of this
- * entry point on one device, so those calls must be ordered (one stream, or
- * streams ordered by events); it is the only memory the library owns.
+ * Kernel family choice, for tests and benchmarks that run the same call on
+ * two kernel families (not part of the method; the default is AUTO and
+ * nothing needs to call this).  Process-wide; set it only while no call of
+ * the library is being made from another thread.
+ *   op:       LINATTN_OP_CAUSAL (both causal forwards), LINATTN_OP_GLOBAL,
+ *             LINATTN_OP_PERFORMER (linattn_performer_features)
+ *   kernel:   LINATTN_KERNEL_AUTO (the library's choice),
+ *             LINATTN_KERNEL_CUDA_CORES (the fp32 CUDA-core kernels),
+ *             LINATTN_KERNEL_TC_PAIRED (causal only: the tensor-core kernel
+ *             with two CTAs per head, each owning 64 columns of dv; bf16,
+ *             dk in {64, 128}, dv a multiple of 64; never segmented)
+ *   segments: causal tensor-core path only: 0 lets the library choose G,
+ *             G >= 1 asks for at most G segments per sequence (used when the
+ *             call has a large enough workspace)
+ * Returns LINATTN_ERR_INVALID for an unknown op or kernel, a kernel the op
+ * does not have, or segments outside 0..64.
+ */
+enum { LINATTN_OP_CAUSAL = 0, LINATTN_OP_GLOBAL = 1, LINATTN_OP_PERFORMER = 2 };
+enum { LINATTN_KERNEL_AUTO = 0, LINATTN_KERNEL_CUDA_CORES = 1, LINATTN_KERNEL_TC_PAIRED = 2 };
+LINATTN_API int linattn_set_kernel_choice(int op, int kernel, int segments);
+
+/*
+ * linattn_fwd_causal (zero starting state) for callers that cannot allocate
+ * device memory themselves (no cudaMalloc: a host that hands out only fixed
+ * buffers, or code that runs where an allocation could block or fail): the
+ * segmented form takes its workspace from a 16 MB device array the library
+ * holds for every device it is loaded on (until the process exits), and the
+ * call falls back to the single pass when the workspace it needs is larger.
+ * The paper has no counterpart of this entry point.  It allocates nothing.
+ * The array's device address is looked up with cudaGetSymbolAddress on the
+ * first call on a device (and again if the device's context has changed), so
+ * make that first call before any stream capture.  The array is shared by
+ * all calls of this entry point on one device and keeps the last call's
+ * contents; calls that overlap on the GPU race on it, so order them (one
+ * stream, or streams ordered by events).  It is the only memory the library
+ * owns.  Arguments and errors as linattn_fwd_causal.
  */
 LINATTN_API int linattn_fwd_causal_noalloc(const linattn_dims *dims, const void *q, const void *k,
                        const void *v, const float *lambda, float eps, void *out,
                        float *S_final, float *z_final, linattn_stream_t stream);
+
+/*
+ * State-only causal pass: the fast weights a sequence leaves behind, without
+ * its outputs ([FW] §2.1 and §3.2 recurrence, §4.2 normaliser, from a zero
+ * start):
+ *   S = sum_j lambda^(N-1-j) phi(k_j) v_j^T      z = sum_j lambda^(N-1-j) phi(k_j)
+ *   k [B, H, N, dk] dtype, v [B, H, N, dv] dtype, lambda [H] fp32 or NULL
+ *   S [B, H, dk, dv] fp32, z [B, H, dk] fp32     written (N = 0: zeros)
+ * Equal to the S_final / z_final of linattn_fwd_causal up to fp32 summation
+ * order; it reads k and v only.  Its use: the state each segment of a
+ * sequence split across devices hands on (see linattn_combine_states).
+ * bf16 with dk and dv in {64, 128} runs on the tensor cores, the rest on CUDA
+ * cores.  S and z must not overlap k, v or each other.
+ */
+LINATTN_API int linattn_causal_state(const linattn_dims *dims, const void *k, const void *v,
+                       const float *lambda, float *S, float *z, linattn_stream_t stream);
+
+/*
+ * Scan of segment states into starting states: the step that joins the
+ * segments of the "parallel scan" form ([FW] §4.1 note and §5.2: blocks
+ * computed in parallel, the state carried across them).  A sequence is cut
+ * into G consecutive segments of dims->N tokens each (the last may be
+ * shorter: its length does not enter); dS [G, B, H, dk, dv] and
+ * dz [G, B, H, dk] (fp32, slot-major) hold each segment's own final state from
+ * zero (linattn_causal_state on that segment).  On return slot g holds the
+ * state at the start of segment g:
+ *   carry_0 = (S_init, z_init), or zero when both are NULL
+ *   carry_{g+1} = lambda^N carry_g + dS_g      (and likewise for z)
+ * so that linattn_fwd_causal_from on segment g from slot g continues the
+ * whole sequence.  dims.dtype, dims.phi are ignored; 0 <= G <= 64.  S_init,
+ * z_init must not overlap dS or dz.
+ */
+LINATTN_API int linattn_combine_states(const linattn_dims *dims, int G, const float *lambda,
+                       const float *S_init, const float *z_init, float *dS, float *dz,
+                       linattn_stream_t stream);
 
 /*
  * Backward of linattn_fwd_causal (zero starting state): the gradients of
@@ -222,6 +290,23 @@ LINATTN_API int linattn_fwd_global(const linattn_dims *dims, const void *q, cons
 LINATTN_API int linattn_fwd_global_cross(const linattn_dims *dims, int Nk, const void *q,
                        const void *k, const void *v, float eps, void *out, float *KV,
                        float *ksum, linattn_stream_t stream);
+
+/*
+ * The global / cross forward with a key padding mask ([LN] §6: the module's
+ * forward takes key_padding_mask and its example leaves it out; read here in
+ * the usual sense: a key marked as padding is not attended to, so it enters
+ * neither sum):
+ *   KV = sum_{n<Nk, mask[b][n] = 0} phi(k_n) v_n^T,   ksum likewise,
+ *   y_i = phi(q_i)^T KV / (phi(q_i)^T ksum + eps).
+ *   key_padding_mask [B, Nk] bytes, nonzero = padding (one row per sequence,
+ *   shared by its heads), device memory, not overlapping out, KV or ksum; NULL
+ *   means no padding (exactly linattn_fwd_global_cross).  A sequence whose
+ *   keys are all padding gets KV = 0, ksum = 0 and y = 0.  Other arguments as
+ *   linattn_fwd_global_cross.
+ */
+LINATTN_API int linattn_fwd_global_masked(const linattn_dims *dims, int Nk, const void *q,
+                       const void *k, const void *v, const unsigned char *key_padding_mask,
+                       float eps, void *out, float *KV, float *ksum, linattn_stream_t stream);
 
 /*
  * One decode step for every (b, h) ([FW] §4.1 forward_step, §3.1 constant

@@ -54,6 +54,9 @@ def _load():
         lib.oracle_global.restype = i
         lib.oracle_global_cross.argtypes = [i, i, i, i, i, i, _dp, _dp, _dp, d, _dp, _dp, _dp, i]
         lib.oracle_global_cross.restype = i
+        lib.oracle_global_masked.argtypes = [i, i, i, i, i, i, _dp, _dp, _dp,
+                                             ctypes.POINTER(ctypes.c_ubyte), d, _dp, _dp, _dp, i]
+        lib.oracle_global_masked.restype = i
         lib.oracle_feature_map.argtypes = [ctypes.c_long, _dp, _dp]
         lib.oracle_feature_map.restype = None
         lib.oracle_num_threads.argtypes = [i]
@@ -148,6 +151,33 @@ def global_cross(q, k, v, eps=1e-6, nthreads=0):
                                      float(eps), _ptr(y), _ptr(KV), _ptr(ks), int(nthreads))
     if rc != 0:
         raise ValueError("oracle_global_cross rejected its arguments")
+    return y, KV, ks
+
+
+def global_masked(q, k, v, key_padding_mask, eps=1e-6, nthreads=0):
+    """Cross form with a key padding mask ``[B, Nk]`` (nonzero: padding, left
+    out of both sums; None: no padding).  Returns ``(y, KV, ks)`` as
+    ``global_cross``."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, H, Nq, dk = q.shape
+    Nk, dv = k.shape[2], v.shape[-1]
+    pad = None
+    if key_padding_mask is not None:
+        m = key_padding_mask
+        if hasattr(m, "detach"):
+            m = m.detach().to("cpu").numpy()
+        pad = np.ascontiguousarray(np.asarray(m) != 0, dtype=np.uint8)
+        if pad.shape != (B, Nk):
+            raise ValueError("key_padding_mask must have shape [B, Nk]")
+    y = np.empty((B, H, Nq, dv))
+    KV = np.empty((B, H, dk, dv))
+    ks = np.empty((B, H, dk))
+    rc = _load().oracle_global_masked(
+        B, H, Nq, Nk, dk, dv, _ptr(q), _ptr(k), _ptr(v),
+        None if pad is None else pad.ctypes.data_as(ctypes.POINTER(ctypes.c_ubyte)), float(eps),
+        _ptr(y), _ptr(KV), _ptr(ks), int(nthreads))
+    if rc != 0:
+        raise ValueError("oracle_global_masked rejected its arguments")
     return y, KV, ks
 
 

@@ -199,6 +199,8 @@ typedef struct {
     const double *q, *k, *v;
     double eps;
     double *y, *KV, *ks;
+    const unsigned char *pad;   /* [B, Nk], nonzero: the key is padding, or NULL */
+    int H;
 } global_ctx;
 
 static void global_pair(void *vctx, long pair) {
@@ -211,7 +213,9 @@ static void global_pair(void *vctx, long pair) {
     double *ks = (double *)calloc((size_t)dk, sizeof(double));
     double *f = (double *)malloc(sizeof(double) * dk);
 
+    const unsigned char *pad = c->pad ? c->pad + (size_t)(pair / c->H) * Nk : NULL;
     for (int n = 0; n < Nk; ++n) {
+        if (pad && pad[n]) continue;   /* a padding key enters neither sum */
         const double *kn = k + (size_t)n * dk;
         const double *vn = v + (size_t)n * dv;
         for (int a = 0; a < dk; ++a) f[a] = phi(kn[a]);
@@ -250,7 +254,22 @@ int oracle_global_cross(int B, int H, int Nq, int Nk, int dk, int dv,
                         double *y, double *KV, double *ks, int nthreads) {
     if (B < 0 || H < 0 || Nq < 0 || Nk < 0 || dk <= 0 || dv <= 0) return -1;
     if ((Nq > 0 && !q) || (Nk > 0 && (!k || !v))) return -1;
-    global_ctx c = {Nq, Nk, dk, dv, q, k, v, eps, y, KV, ks};
+    global_ctx c = {Nq, Nk, dk, dv, q, k, v, eps, y, KV, ks, NULL, H};
+    for_each_pair((long)B * H, nthreads, global_pair, &c);
+    return 0;
+}
+
+/* Cross form with a key padding mask: the linear-attention note's module
+ * forward (§6) takes key_padding_mask (its example leaves it out); a key
+ * marked as padding (pad[b][n] != 0, one row per sequence b shared by its
+ * heads) is not attended to, so it is left out of both sums KV and ks. */
+int oracle_global_masked(int B, int H, int Nq, int Nk, int dk, int dv,
+                         const double *q, const double *k, const double *v,
+                         const unsigned char *pad, double eps,
+                         double *y, double *KV, double *ks, int nthreads) {
+    if (B < 0 || H <= 0 || Nq < 0 || Nk < 0 || dk <= 0 || dv <= 0) return -1;
+    if ((Nq > 0 && !q) || (Nk > 0 && (!k || !v))) return -1;
+    global_ctx c = {Nq, Nk, dk, dv, q, k, v, eps, y, KV, ks, pad, H};
     for_each_pair((long)B * H, nthreads, global_pair, &c);
     return 0;
 }

@@ -34,10 +34,16 @@ def test_algorithmic_bytes_match_the_workloads():
 
 
 def test_mma_flops_of_the_causal_kernel():
-    # per 128-token chunk and 64-column slice: scores 128x128x128, three
-    # N=64 products and three N=16 side products of K = 128, 2 flops each
-    per = 2 * (128 * 128 * 128 + 3 * 128 * 64 * 128 + 3 * 128 * 16 * 128)
-    assert bench.causal_mma_flops(4, 16, 16384, 128, 128) == 4 * 16 * 2 * 128 * per
+    # per 128-token chunk and head, the whole dv in one CTA: the score tile,
+    # the carried term, the state update and the intra term, each 128 x 128
+    # x 128 at d = 128, 2 flops per multiply-add
+    per = 4 * 2 * 128 * 128 * 128
+    assert bench.causal_mma_flops(4, 16, 16384, 128, 128) == 4 * 16 * 128 * per
+    # 137.4 GFLOP for the headline workload (the count at C = 128)
+    assert round(bench.causal_mma_flops(4, 16, 16384, 128, 128) / 1e9, 1) == 137.4
+    # d = 64: the state update keeps its 128 rows of d_k (zero-padded)
+    assert bench.causal_mma_flops(2, 8, 4096, 64, 64) == \
+        16 * 32 * 2 * 128 * (128 * 64 + 64 * 64 + 64 * 128 + 64 * 128)
 
 
 def test_traffic_record_checks_its_sources(tmp_path, monkeypatch):

@@ -196,6 +196,36 @@ def test_global_cross_brute_force():
     assert not y0.any() and not KV0.any() and not ks0.any()
 
 
+def test_global_masked_pins():
+    """Key padding mask ([LN] §6 key_padding_mask): the double sum over the
+    keys that are not padding; the same as the cross form on those keys alone
+    (per sequence); no padding gives the cross form; all padding gives
+    KV = ks = 0 and y = 0."""
+    q, _, _ = rand(23, 3, 2, 6, 5, 4)
+    _, k, v = rand(24, 3, 2, 13, 5, 4)
+    eps = 1e-3
+    pad = np.zeros((3, 13), dtype=np.uint8)
+    pad[0, [0, 4, 12]] = 1          # a few padding keys
+    pad[1, 7:] = 1                  # a padded tail
+    pad[2, :] = 1                   # all padding
+    y, KV, ks = oracle.global_masked(q, k, v, pad, eps)
+    fq, fk = phi_np(q), phi_np(k)
+    keep = (pad == 0).astype(np.float64)[:, None, :]          # [B, 1, Nk]
+    w = np.einsum("bhid,bhjd->bhij", fq, fk) * keep[:, :, None, :]
+    assert rel(y, np.einsum("bhij,bhjv->bhiv", w, v) / (w.sum(-1, keepdims=True) + eps)) < 1e-13
+    assert rel(KV, np.einsum("bhjd,bhjv->bhdv", fk * keep[..., None], v)) < 1e-13
+    assert rel(ks, (fk * keep[..., None]).sum(2)) < 1e-13
+    for b in range(2):
+        idx = np.nonzero(pad[b] == 0)[0]
+        yc, KVc, ksc = oracle.global_cross(q[b:b + 1], k[b:b + 1, :, idx], v[b:b + 1, :, idx], eps)
+        assert rel(y[b:b + 1], yc) < 1e-14 and rel(KV[b:b + 1], KVc) < 1e-14
+        assert rel(ks[b:b + 1], ksc) < 1e-14
+    assert not KV[2].any() and not ks[2].any() and not y[2].any()
+    y0, KV0, ks0 = oracle.global_masked(q, k, v, None, eps)
+    yx, KVx, ksx = oracle.global_cross(q, k, v, eps)
+    assert np.array_equal(y0, yx) and np.array_equal(KV0, KVx) and np.array_equal(ks0, ksx)
+
+
 def test_causal_last_token_equals_global_without_decay():
     q, k, v = rand(5, 1, 3, 40, 8, 8)
     y, S, z = oracle.causal(q, k, v, None, eps=1e-6)

@@ -13,6 +13,9 @@ import torch
 
 import oracle
 from weight_state_recurrence_b200 import inputs
+from weight_state_recurrence_b200.linattn import (LINATTN_KERNEL_CUDA_CORES,
+                                                   LINATTN_KERNEL_TC_PAIRED, LINATTN_OP_CAUSAL,
+                                                   LINATTN_OP_GLOBAL, kernel_choice)
 from tests._compare import assert_close
 
 pytestmark = pytest.mark.gpu
@@ -143,11 +146,15 @@ def test_decode_reduced_all_heads(cuda_lib):
     _decode_run(cuda_lib, W["decode_d128"], B=4, steps=48)
 
 
-def test_decode_full_size_sampled(cuda_lib):
-    # full 256 x 32 heads (the benchmark's launch configuration); a shorter
-    # prefix keeps input generation on the host quick
-    _decode_run(cuda_lib, W["decode_d128"], B=256, steps=8, N=64,
-                heads=[(0, 0), (17, 31), (128, 5), (255, 16)])
+def test_decode_d128_as_stated(cuda_lib):
+    """The decode workload exactly as stated: 256 sequences x 32 heads, the
+    state prefilled from 512 tokens through the causal forward, then 1024
+    decode steps, each launched over all 8192 heads (the benchmark's launch
+    configuration).  Every step's y of five sampled heads, and their S, z
+    after the last step, against the oracle."""
+    w = W["decode_d128"]
+    _decode_run(cuda_lib, w, B=w.B, steps=w.steps,
+                heads=[(0, 0), (17, 31), (128, 5), (200, 9), (255, 16)])
 
 
 # ------------------------------------------------------------ edge cases
@@ -169,19 +176,23 @@ def test_causal_shapes(cuda_lib, dk, dv, dtype):
     check_causal(cuda_lib, q, k, v, lam, 1e-6, tol)
 
 
-def test_causal_simt_second_opinion(cuda_lib, monkeypatch):
-    """The CUDA-core kernel on the tensor-core kernel's inputs."""
+def test_causal_other_kernels_second_opinion(cuda_lib):
+    """The CUDA-core kernel and the paired tensor-core kernel on the product
+    kernel's inputs."""
     w = W["causal_decay_d128"]
     q, k, v = inputs.causal_inputs(w, B=1, H=4, N=700)
     lam = inputs.decay(w, H=4)
     out_tc, S_tc, z_tc = run_causal(cuda_lib, q, k, v, lam, w.eps)
-    monkeypatch.setenv("LINATTN_CAUSAL_KERNEL", "simt")
-    out_s, S_s, z_s = run_causal(cuda_lib, q, k, v, lam, w.eps)
+    with kernel_choice(LINATTN_OP_CAUSAL, LINATTN_KERNEL_CUDA_CORES):
+        out_s, S_s, z_s = run_causal(cuda_lib, q, k, v, lam, w.eps)
+    with kernel_choice(LINATTN_OP_CAUSAL, LINATTN_KERNEL_TC_PAIRED):
+        out_p, S_p, z_p = run_causal(cuda_lib, q, k, v, lam, w.eps)
     y_o, S_o, z_o = oracle.causal(q, k, v, lam, w.eps)
-    assert_close("y simt", out_s, y_o, 2e-2)
-    assert_close("y tc", out_tc, y_o, 2e-2)
-    assert_close("S simt", S_s, S_o, 2e-2)
-    assert_close("S tc", S_tc, S_o, 2e-2)
+    for name, (y, S, z) in {"simt": (out_s, S_s, z_s), "tc": (out_tc, S_tc, z_tc),
+                            "paired": (out_p, S_p, z_p)}.items():
+        assert_close(f"y {name}", y, y_o, 2e-2)
+        assert_close(f"S {name}", S, S_o, 2e-2)
+        assert_close(f"z {name}", z, z_o, 2e-2)
 
 
 def test_causal_empty_and_zero_heads(cuda_lib):
@@ -278,11 +289,11 @@ def test_global_tc_edges(cuda_lib, N):
     assert_close("ksum", ks, ks_o, 2e-2)
 
 
-def test_global_simt_second_opinion(cuda_lib, monkeypatch):
+def test_global_simt_second_opinion(cuda_lib):
     q, k, v = inputs.random_case(17, 1, 6, 3000, 64, 64, torch.bfloat16, scale=0.125)
     out_tc, KV_tc, _ = cuda_lib.fwd_global(q.to(DEV), k.to(DEV), v.to(DEV), 1e-6)
-    monkeypatch.setenv("LINATTN_GLOBAL_KERNEL", "simt")
-    out_s, KV_s, _ = cuda_lib.fwd_global(q.to(DEV), k.to(DEV), v.to(DEV), 1e-6)
+    with kernel_choice(LINATTN_OP_GLOBAL, LINATTN_KERNEL_CUDA_CORES):
+        out_s, KV_s, _ = cuda_lib.fwd_global(q.to(DEV), k.to(DEV), v.to(DEV), 1e-6)
     torch.cuda.synchronize()
     y_o, KV_o, _ = oracle.global_attn(q, k, v, 1e-6)
     assert_close("y tc", out_tc, y_o, 2e-2)

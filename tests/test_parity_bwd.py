@@ -73,6 +73,15 @@ def test_bwd_decay_workload_shape(cuda_lib):
     check_bwd(cuda_lib, 1, 4, 300, 128, 128, torch.bfloat16, lam, 1500, 2e-2)
 
 
+@pytest.mark.parametrize("N,lam", [(4096, (0.9, 0.999)), (8192, (1.0,))])
+def test_bwd_long_sequence(cuda_lib, N, lam):
+    """Accumulation of the carried states over a long sequence: heads of the
+    decay workload's shape (d = 128, bf16) and lambda range, 32 and 64 chunks
+    of 128 tokens, against the gradient oracle's masked form."""
+    lam = torch.tensor(lam, dtype=torch.float32)
+    check_bwd(cuda_lib, 1, lam.numel(), N, 128, 128, torch.bfloat16, lam, 1600 + N, 2e-2)
+
+
 def test_bwd_empty_sequence(cuda_lib):
     q = torch.zeros(1, 2, 0, 32, device=DEV)
     dq, dk, dv, dl = cuda_lib.bwd_causal(q, q, q, q, torch.ones(2, device=DEV), 1e-6,

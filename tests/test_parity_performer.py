@@ -14,6 +14,8 @@ import torch
 
 from oracle import performer as P
 from weight_state_recurrence_b200 import inputs
+from weight_state_recurrence_b200.linattn import (LINATTN_KERNEL_AUTO, LINATTN_KERNEL_CUDA_CORES,
+                                                   LINATTN_OP_PERFORMER, kernel_choice)
 from tests._compare import assert_close
 
 pytestmark = pytest.mark.gpu
@@ -33,13 +35,12 @@ def draw(seed, shape, scale, dtype):
 
 
 # --------------------------------------------------------------- features
-def check_features(lib, rows, d, m, kernel, dtype, scale, seed, tol, simt=False,
-                   monkeypatch=None):
-    if simt:
-        monkeypatch.setenv("LINATTN_PERFORMER_KERNEL", "simt")
+def check_features(lib, rows, d, m, kernel, dtype, scale, seed, tol, simt=False):
     x = draw(seed, (rows, d), scale, dtype)
     w = inputs.performer_omega(m, d, seed + 1, True, dtype)
-    f = lib.performer_features(x.to(DEV), w.to(DEV), KERNELS[kernel])
+    with kernel_choice(LINATTN_OP_PERFORMER,
+                       LINATTN_KERNEL_CUDA_CORES if simt else LINATTN_KERNEL_AUTO):
+        f = lib.performer_features(x.to(DEV), w.to(DEV), KERNELS[kernel])
     torch.cuda.synchronize()
     assert f.shape == (rows, 2 * m) and f.dtype == dtype
     if rows:
@@ -76,9 +77,9 @@ def test_cuda_core_features(cuda_lib, d, m, dtype, tol):
     check_features(cuda_lib, 333, d, m, "gaussian", dtype, 1.0, 2400 + d + m, tol)
 
 
-def test_forced_cuda_core_features_bf16(cuda_lib, monkeypatch):
+def test_forced_cuda_core_features_bf16(cuda_lib):
     check_features(cuda_lib, 500, 128, 64, "softmax", torch.bfloat16, 0.5 / math.sqrt(128), 2500,
-                   BF16_FEAT_TOL, simt=True, monkeypatch=monkeypatch)
+                   BF16_FEAT_TOL, simt=True)
 
 
 def test_zero_rows(cuda_lib):

@@ -6,6 +6,8 @@ import torch
 
 import oracle
 from weight_state_recurrence_b200 import inputs
+from weight_state_recurrence_b200.linattn import (LINATTN_KERNEL_CUDA_CORES, LINATTN_OP_CAUSAL,
+                                                   kernel_choice)
 from tests._compare import assert_close
 
 pytestmark = pytest.mark.gpu
@@ -29,14 +31,14 @@ def run_ws(lib, q, k, v, lam, eps, S0=None, z0=None, ws_bytes=None):
     return need, out, S, z
 
 
-def test_causal_d64_workload_segmented(cuda_lib, monkeypatch):
+def test_causal_d64_workload_segmented_cuda_cores(cuda_lib):
     """The causal_d64 workload (16 heads, 4096 tokens, d = 64, bf16) on the
-    CUDA-core path (forced: bf16 with d_k = 64 normally takes the tensor
-    cores), cut into segments."""
-    monkeypatch.setenv("LINATTN_CAUSAL_KERNEL", "simt")
+    CUDA-core path (chosen explicitly: bf16 with d_k = 64 normally takes the
+    tensor cores), cut into segments."""
     w = inputs.WORKLOADS["causal_d64"]
     q, k, v = inputs.causal_inputs(w)
-    need, out, S, z = run_ws(cuda_lib, q, k, v, None, w.eps)
+    with kernel_choice(LINATTN_OP_CAUSAL, LINATTN_KERNEL_CUDA_CORES):
+        need, out, S, z = run_ws(cuda_lib, q, k, v, None, w.eps)
     assert need > 0
     y_o, S_o, z_o = oracle.causal(q, k, v, None, w.eps)
     assert_close("y", out, y_o, 2e-2)
@@ -70,26 +72,28 @@ def test_small_decay_segments(cuda_lib):
     assert_close("S_final", S, S_o, 1e-4)
 
 
-def test_small_workspace_runs_the_single_pass(cuda_lib, monkeypatch):
-    monkeypatch.setenv("LINATTN_CAUSAL_KERNEL", "simt")
+def test_small_workspace_runs_the_single_pass(cuda_lib):
     w = inputs.WORKLOADS["causal_d64"]
     q, k, v = inputs.causal_inputs(w, B=1, H=2, N=1024)
-    need, out, S, z = run_ws(cuda_lib, q, k, v, None, w.eps, ws_bytes=64)
+    with kernel_choice(LINATTN_OP_CAUSAL, LINATTN_KERNEL_CUDA_CORES):
+        need, out, S, z = run_ws(cuda_lib, q, k, v, None, w.eps, ws_bytes=64)
     assert need > 64
     y_o, S_o, _ = oracle.causal(q, k, v, None, w.eps)
     assert_close("y", out, y_o, 2e-2)
     assert_close("S_final", S, S_o, 2e-2)
 
 
-def test_workspace_query(cuda_lib, monkeypatch):
+def test_workspace_query(cuda_lib):
     ws = cuda_lib.linattn_fwd_causal_workspace
-    assert ws(2, 8, 4096, 64, 64, torch.bfloat16) == 0       # tensor-core path (d_k = 64)
-    assert ws(4, 16, 16384, 128, 128, torch.bfloat16) == 0   # tensor-core path
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    # tensor-core path, 16 heads: about one segment per SM, 128-token multiples
+    G = -(-32 // -(-32 // (sms // 16)))
+    assert ws(2, 8, 4096, 64, 64, torch.bfloat16) == 16 * G * (64 * 64 + 64) * 4
+    assert ws(4, 16, 16384, 128, 128, torch.bfloat16) == 0   # 64 heads: one pass
     assert ws(2, 8, 4096, 32, 32, torch.bfloat16) > 0        # 16 heads on CUDA cores: segmented
     assert ws(2, 8, 4096, 64, 64, torch.float32) > 0         # likewise
-    monkeypatch.setenv("LINATTN_CAUSAL_KERNEL", "simt")
-    assert ws(2, 8, 4096, 64, 64, torch.bfloat16) > 0        # forced CUDA cores: segmented
-    monkeypatch.delenv("LINATTN_CAUSAL_KERNEL")
+    with kernel_choice(LINATTN_OP_CAUSAL, LINATTN_KERNEL_CUDA_CORES):
+        assert ws(2, 8, 4096, 64, 64, torch.bfloat16) > 0    # CUDA cores chosen: segmented
     assert ws(64, 64, 4096, 64, 64, torch.float32) == 0      # enough heads already
     assert ws(1, 1, 100, 64, 64, torch.float32) == 0         # too short to cut
     assert ws(1, 1, 4096, 48, 64, torch.float32) == 0        # unsupported: no plan

@@ -43,15 +43,29 @@ def run(lib, q, k, v, lam, eps):
     return out, S, z
 
 
+SCRATCH_BYTES = 16 << 20   # the library's static scratch array
+
+
 @pytest.mark.gpu
-def test_no_alloc_segmented_workload(cuda_lib, monkeypatch):
-    # the CUDA-core path (forced: bf16 with d_k = 64 normally takes the tensor cores)
-    monkeypatch.setenv("LINATTN_CAUSAL_KERNEL", "simt")
+def test_no_alloc_segmented_workload(cuda_lib):
+    """causal_d64 (16 heads): the tensor-core path cuts it into segments
+    whose states fit the scratch.  The no-allocation call must give exactly
+    the bits of the same segmented call with a caller workspace, which differ
+    from the single pass (other summation order), so the scratch was used."""
     w = inputs.WORKLOADS["causal_d64"]
     q, k, v = inputs.causal_inputs(w)
-    assert cuda_lib.linattn_fwd_causal_workspace(w.B, w.H, w.N, w.d, w.d, w.dtype) > 0
+    need = cuda_lib.linattn_fwd_causal_workspace(w.B, w.H, w.N, w.d, w.d, w.dtype)
+    assert 0 < need <= SCRATCH_BYTES
     out, S, z = run(cuda_lib, q, k, v, None, w.eps)
+    ws = torch.empty(need, dtype=torch.uint8, device=DEV)
+    out_ws = torch.empty_like(out)
+    S_ws, z_ws = torch.empty_like(S), torch.empty_like(z)
+    cuda_lib.linattn_fwd_causal_ws(q.to(DEV), k.to(DEV), v.to(DEV), None, w.eps, None, None,
+                                   out_ws, S_ws, z_ws, ws)
+    out_1, S_1, _ = cuda_lib.fwd_causal(q.to(DEV), k.to(DEV), v.to(DEV), None, w.eps)
     torch.cuda.synchronize()
+    assert torch.equal(out, out_ws) and torch.equal(S, S_ws) and torch.equal(z, z_ws)
+    assert not torch.equal(S, S_1)
     y_o, S_o, z_o = oracle.causal(q, k, v, None, w.eps)
     assert_close("y", out, y_o, 2e-2)
     assert_close("S_final", S, S_o, 2e-2)

@@ -1,0 +1,868 @@
+// Chunked causal forward on the 5th-generation tensor cores, one CTA per
+// (head, segment of the sequence) with the head's whole d_v, plus the
+// tensor-core state pass that gives every segment after the first its
+// starting state.  bf16 operands, fp32 accumulators in TMEM, d_k and d_v in
+// {64, 128}.
+//
+// The method (fast-weight article §2.1/§3.2/§4.2 recurrence; §3.1 triangular
+// mask; §4.1 note and §5.2: cut the sequence into blocks, parallel inside a
+// block, carried across blocks; the "parallel scan" over segments of §5.2 is
+// the split into segments), per chunk of C = 128 tokens, t and s 0-based in
+// the chunk, Cv valid tokens, carried state (S, z):
+//
+//   P    = (phi(Q) phi(K)^T) o M,   M[t][s] = lambda^(t-s) for s <= t, else 0
+//   num  = P V + Lq phi(Q) S,       Lq = diag(lambda^(t+1))
+//   den  = P 1 + Lq phi(Q) z + eps
+//   y    = num / den
+//   S   <- lambda^Cv S + (Lk phi(K))^T V,   Lk = diag(lambda^(Cv-1-s))
+//   z   <- lambda^Cv z + (Lk phi(K))^T 1
+//
+// Tensor-core chains per chunk (M = 128, K = 16 per instruction, N = d_v):
+//   score   D_A   = phi(Q) phi(K)^T                       SMEM x SMEM
+//   carried D_O   = phi(Q) S'        (S' = bf16 state)    SMEM x SMEM
+//   state   D_S  += (Lk phi(K))^T V                       SMEM x SMEM (both MN-major)
+//   intra   D_O  += P V              (P = bf16 in TMEM)   TMEM x SMEM
+// One accumulator takes both halves of the numerator.  The denominator is
+// formed in fp32 on the CUDA cores: the feature-map warps keep z and take
+// phi(q_t).z while they transform q; the score epilogue adds the row sums of
+// the bf16 P tile (the weights the numerator uses).
+//
+// Decay.  For lambda >= kFactorMin the decay is factored into the operands:
+// phi(q_t) is scaled by lambda^(t+1-Cv) and phi(k_s) by lambda^(Cv-1-s)
+// while the feature map is applied, so the score MMA yields lambda^(t-s)
+// phi(q_t).phi(k_s), the state MMA gets its weights, and the carried term
+// needs the state scaled once by lambda^Cv (the state warps write the bf16
+// operand as lambda^Cv S).  Smaller lambda (down to 0): the score epilogue
+// multiplies by lambda^(t-s), and after the score MMA has read them the q
+// rows are rescaled by lambda^(t+1) and the k rows by lambda^(Cv-1-s).
+//
+// Warp roles (768 threads):
+//   warp 0      TMA producer of the q and k tiles
+//   warp 1      TMEM owner, the single MMA-issuing thread
+//   warp 2      TMA producer of the v tiles
+//   warps 4-7   score epilogue: D_A -> mask (and decay) -> bf16 P in TMEM, row sums
+//   warps 8-11  output: y = D_O / den -> global memory
+//   warps 12-15 state: D_S -> bf16 operand S' and D_S <- lambda^Cv D_S
+//   warps 16-23 feature map (in place, packed bf16x2), phi(q).z, z update
+// Every wait is bounded (sm100.cuh); a wait that runs out records an error
+// flag and every role leaves its loop.
+#pragma once
+#include "common.cuh"
+#include "sm100.cuh"
+#include "causal_tc.cuh"
+
+namespace linattn {
+namespace stc {
+
+using tc::mul_bf16x2;
+using tc::pack_bf16;
+using tc::phi_bf16x2;
+
+constexpr int C = 128;
+constexpr int NT = 768;
+constexpr int kPhiThreads = 256;
+constexpr int kBarPhi = 1, kBarP = 2, kBarOut = 3, kBarState = 4;   // named barriers
+constexpr float kFactorMin = 0.7f;
+
+constexpr uint32_t kPanel = 16384;              // 128 rows x 128 bytes (64 bf16)
+constexpr uint32_t kOffQ = 0;                   // per stage: q, 2 panels of d_k
+constexpr uint32_t kOffK = 2 * kPanel;          //            k, 2 panels of d_k
+constexpr uint32_t kOffV = 4 * kPanel;          //            v, 2 panels of d_v
+constexpr uint32_t kStage = 6 * kPanel;         // 96 KB
+constexpr uint32_t kOffSop = 2 * kStage;        // bf16 state operand: rows d_k, 2 panels of d_v
+constexpr uint32_t kOffMisc = kOffSop + 2 * kPanel;
+constexpr uint32_t kMiscTmem = 256, kMiscAbort = 260, kMiscRoleFail = 272;
+constexpr uint32_t kMiscPw = 320;               // lambda^i, i = 0..C        (129 floats)
+constexpr uint32_t kMiscZ = 848;                // z, fp32                   (128 floats)
+constexpr uint32_t kMiscDen = 1360;             // den[2][128]: phi(q).z + row sum of P
+constexpr uint32_t kMiscBytes = kMiscDen + 2 * 128 * 4;
+constexpr uint32_t kSmemBytes = kOffMisc + kMiscBytes;
+static_assert(kSmemBytes <= 232448, "exceeds the per-CTA shared memory of sm_100");
+
+enum Bar {
+  kFullQK0 = 0, kFullQK1, kFullV0, kFullV1, kFreeQK0, kFreeQK1, kFreeV0, kFreeV1,
+  kPhi0, kPhi1, kScore, kRescale, kState, kReadout, kPDone, kO0, kO1, kOut0, kOut1,
+  kDen0, kDen1, kFinal, kNumBars
+};
+static_assert(kNumBars * 8 <= 256, "barrier area overflow");
+
+// tensor memory columns (fp32, lane = row)
+constexpr uint32_t kTmS = 0;     // state D_S, lane = d_k row
+constexpr uint32_t kTmA = 128;   // score D_A; P (bf16 pairs) overwrites its first 64 columns
+constexpr uint32_t kTmO = 256;   // output accumulators D_O[0], D_O[1]
+constexpr uint32_t kTmCols = 512;
+
+__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// byte offset of 16-byte chunk j (0..15) of row `row` in a 2-panel K-major tile
+__device__ __forceinline__ uint32_t chunk_off(uint32_t row, uint32_t j) {
+  return (j >> 3) * kPanel + sw128_offset(row, (j & 7) * 16);
+}
+
+template <int DKP, int DVP>
+__global__ void __launch_bounds__(NT, 1)
+    causal_seg_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
+                         const __grid_constant__ CUtensorMap tm_k,
+                         const __grid_constant__ CUtensorMap tm_v, const float *__restrict__ lam,
+                         float eps, const float *__restrict__ S_init,
+                         const float *__restrict__ z_init, const float *__restrict__ ws_S,
+                         const float *__restrict__ ws_z, __nv_bfloat16 *__restrict__ out,
+                         float *__restrict__ S_final, float *__restrict__ z_final, int H, int N,
+                         int seg_len, int G, bool ident) {
+  constexpr int DK = 64 * DKP, DV = 64 * DVP;
+  constexpr int KCH = 8 * DKP;                  // 16-byte chunks per q/k row
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *sm = smem_raw;
+  const uint32_t sb = smem_u32(sm);
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  if (sb & 1023u) {
+    if (tid == 0) atomicOr(&g_status, kStatusWaitTimeout);
+    return;
+  }
+  const long pair = blockIdx.x / G;
+  const int g = blockIdx.x % G;
+  const int h = static_cast<int>(pair % H);
+  const float L = lam ? lam[h] : 1.f;
+  const int n0 = g * seg_len;
+  const int n1 = min(N, n0 + seg_len);
+  const int nchunks = (n1 - n0 + C - 1) / C;
+  const int Ct = (n1 - n0) - (nchunks - 1) * C;   // valid tokens of the last chunk
+  const bool last_seg = g == G - 1;
+  const float *S0 = g == 0 ? S_init : ws_S + (pair * G + g) * static_cast<long>(DK) * DV;
+  const float *z0 = g == 0 ? z_init : ws_z + (pair * G + g) * static_cast<long>(DK);
+  const bool has_init = S0 != nullptr;
+  const bool factored = L >= kFactorMin;
+
+  uint8_t *misc = sm + kOffMisc;
+  auto bar = [&](int i) { return sb + kOffMisc + 8u * static_cast<uint32_t>(i); };
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(misc + kMiscTmem);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(misc + kMiscAbort);
+  volatile int *role_fail = reinterpret_cast<volatile int *>(misc + kMiscRoleFail);
+  float *pw = reinterpret_cast<float *>(misc + kMiscPw);
+  float *zs = reinterpret_cast<float *>(misc + kMiscZ);
+  float *den = reinterpret_cast<float *>(misc + kMiscDen);
+  auto Cv_of = [&](int c) { return c == nchunks - 1 ? Ct : C; };
+
+  // ------------------------------------------------------------ set-up
+  if (tid == 0) {
+    for (int i = 0; i < kNumBars; ++i) mbar_init(bar(i), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+  }
+  if (tid < 4) role_fail[tid] = 0;
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), kTmCols);
+    tmem_relinquish();
+  }
+  if (tid <= C) pw[tid] = pow_int(L, tid);
+  if (tid < 128) zs[tid] = (z0 && tid < DK) ? z0[pair * DK + tid] : 0.f;
+  if (DKP == 1) {
+    // the second d_k panel of the q and k tiles stays zero (the state MMA
+    // reads it as rows 64-127 of phi(K)^T; the other chains never do)
+    for (uint32_t o = tid * 16u; o < 4 * kPanel; o += NT * 16u) {
+      const uint32_t st = (o / (2 * kPanel)) * kStage, w = o % (2 * kPanel);
+      *reinterpret_cast<uint4 *>(sm + st + (w < kPanel ? kOffQ : kOffK - kPanel) + kPanel + w) =
+          make_uint4(0, 0, 0, 0);
+    }
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  auto fail = [&]() { *abort_flag = 1; };
+
+  if (warp == 0 || warp == 2) {
+    // ------------------------------------------------------ TMA producers
+    if (lane == 0 && nchunks > 0) {
+      const bool qk = warp == 0;
+      int issued = 0;
+      for (int c = 0; c < nchunks && !*abort_flag; ++c) {
+        const int s = c & 1;
+        if (c >= 2 && !mbar_wait(bar((qk ? kFreeQK0 : kFreeV0) + s), ((c - 2) >> 1) & 1)) {
+          fail();
+          break;
+        }
+        const uint32_t base = sb + s * kStage;
+        const int y = n0 + c * C;
+        if (qk) {
+          const uint32_t b = bar(kFullQK0 + s);
+          mbar_arrive_expect_tx(b, 2 * DKP * kPanel);
+          for (int p = 0; p < DKP; ++p) {
+            tma_load_3d(base + kOffQ + p * kPanel, &tm_q, b, 64 * p, y, static_cast<int>(pair));
+            tma_load_3d(base + kOffK + p * kPanel, &tm_k, b, 64 * p, y, static_cast<int>(pair));
+          }
+          if (c + 2 < nchunks)
+            for (int p = 0; p < DKP; ++p) {
+              tma_prefetch_l2_3d(&tm_q, 64 * p, y + 2 * C, static_cast<int>(pair));
+              tma_prefetch_l2_3d(&tm_k, 64 * p, y + 2 * C, static_cast<int>(pair));
+            }
+        } else {
+          const uint32_t b = bar(kFullV0 + s);
+          mbar_arrive_expect_tx(b, DVP * kPanel);
+          for (int p = 0; p < DVP; ++p)
+            tma_load_3d(base + kOffV + p * kPanel, &tm_v, b, 64 * p, y, static_cast<int>(pair));
+          if (c + 2 < nchunks)
+            for (int p = 0; p < DVP; ++p)
+              tma_prefetch_l2_3d(&tm_v, 64 * p, y + 2 * C, static_cast<int>(pair));
+        }
+        issued = c + 1;
+      }
+      if (*abort_flag) {
+        // let the copies this thread started land before the CTA exits
+        for (int c = issued - 2 < 0 ? 0 : issued - 2; c < issued; ++c)
+          mbar_wait(bar((qk ? kFullQK0 : kFullV0) + (c & 1)), (c >> 1) & 1);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idA = idesc_bf16(128, 128, 0, 0);    // K-major x K-major
+      constexpr uint32_t idQS = idesc_bf16(128, DV, 0, 1);    // K-major x MN-major
+      constexpr uint32_t idS = idesc_bf16(128, DV, 1, 1);     // MN-major x MN-major
+      // descriptors of every operand tile, per stage; a K step adds its byte
+      // offset >> 4 to the start-address field (tiles stay below 256 KB, so
+      // the 14-bit field never carries)
+      uint64_t dQ[2], dK[2], dKmn[2], dV[2];
+#pragma unroll
+      for (int s = 0; s < 2; ++s) {
+        const uint32_t st = sb + s * kStage;
+        dQ[s] = sdesc_sw128(st + kOffQ, 16, 1024);
+        dK[s] = sdesc_sw128(st + kOffK, 16, 1024);
+        dKmn[s] = sdesc_sw128(st + kOffK, kPanel, 1024);
+        dV[s] = sdesc_sw128(st + kOffV, kPanel, 1024);
+      }
+      const uint64_t dSop = sdesc_sw128(sb + kOffSop, kPanel, 1024);
+      auto kofs = [](int ks) -> uint64_t { return ((ks >> 2) * kPanel + (ks & 3) * 32) >> 4; };
+      bool ok = true;
+      for (int c = 0; ok && c < nchunks; ++c) {
+        const int s = c & 1;
+        if (*abort_flag) break;
+        // score: D_A = phi(Q) phi(K)^T (the previous chunk's P V, issued
+        // before, has read D_A: the chains run in issue order)
+        if (!mbar_wait(bar(kPhi0 + s), (c >> 1) & 1)) { ok = false; break; }
+        tc_fence_after();
+        const uint64_t q0 = dQ[s], k0 = dK[s], kmn0 = dKmn[s], v0 = dV[s];
+#pragma unroll
+        for (int ks = 0; ks < 4 * DKP; ++ks)
+          umma_bf16(tmem + kTmA, q0 + kofs(ks), k0 + kofs(ks), idA, ks > 0);
+        umma_commit(bar(kScore));
+        // explicit decay: the q and k rows are rescaled once the score MMA has read them
+        if (!factored && !mbar_wait(bar(kRescale), c & 1)) { ok = false; break; }
+        // carried: D_O[s] = phi(Q) S'  (state before this chunk; D_O[s] drained)
+        if (!mbar_wait(bar(kReadout), c & 1) ||
+            (c >= 2 && !mbar_wait(bar(kOut0 + s), ((c - 2) >> 1) & 1)) ||
+            !mbar_wait(bar(kFullV0 + s), (c >> 1) & 1)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t dO = tmem + kTmO + s * 128;
+        const bool carried = c > 0 || has_init;
+        if (carried) {
+#pragma unroll
+          for (int ks = 0; ks < 4 * DKP; ++ks)
+            umma_bf16(dO, q0 + kofs(ks), dSop + ks * (2048 >> 4), idQS, ks > 0);
+        }
+        // state: D_S += (Lk phi(K))^T V   (onto the state decayed by lambda^Cv)
+#pragma unroll
+        for (int ks = 0; ks < C / 16; ++ks)
+          umma_bf16(tmem + kTmS, kmn0 + ks * (2048 >> 4), v0 + ks * (2048 >> 4), idS,
+                    (carried || ks > 0) ? 1u : 0u);
+        umma_commit(bar(kState));
+        umma_commit(bar(kFreeQK0 + s));   // q and k of this chunk fully read
+        // intra: D_O[s] += P V
+        if (!mbar_wait(bar(kPDone), c & 1)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < C / 16; ++ks)
+          umma_bf16_ts(dO, tmem + kTmA + ks * 8, v0 + ks * (2048 >> 4), idQS,
+                       (carried || ks > 0) ? 1u : 0u);
+        umma_commit(bar(kO0 + s));
+        umma_commit(bar(kFreeV0 + s));
+      }
+      if (!ok) fail();
+      umma_commit(bar(kFinal));
+      mbar_wait(bar(kFinal), 0);
+    }
+    __syncwarp();
+  } else if (warp >= 4 && warp < 8) {
+    // --------------------------------------- score epilogue: P into TMEM
+    const int wq = warp - 4;
+    const int t = wq * 32 + lane;
+    const uint32_t lf = static_cast<uint32_t>(wq * 32) << 16;
+    volatile int &rf = role_fail[0];
+    for (int c = 0; c < nchunks; ++c) {
+      const int s = c & 1;
+      // kPhi[s] (already complete) orders the feature-map warps' phi(q).z
+      // before this role's update of den[s]
+      if (*abort_flag || !mbar_wait(bar(kScore), c & 1) ||
+          !mbar_wait(bar(kPhi0 + s), (c >> 1) & 1)) {
+        rf = 1;
+        fail();
+      }
+      tc_fence_after();
+      float rs = 0.f;
+      if (!rf) {
+        // blocks of 32 keys; only blocks 0..wq hold s <= t
+#pragma unroll
+        for (int bk = 0; bk < 4; ++bk) {
+          uint32_t pk[16];
+          if (bk <= wq) {
+            uint32_t r[32];
+            tmem_ld_32x32b_x32(tmem + lf + kTmA + bk * 32, r);
+            tmem_wait_ld();
+            const int s0 = bk * 32;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const int s_a = s0 + 2 * i, s_b = s_a + 1;
+              float a = s_a <= t ? __uint_as_float(r[2 * i]) : 0.f;
+              float b = s_b <= t ? __uint_as_float(r[2 * i + 1]) : 0.f;
+              if (!factored) {
+                a *= s_a <= t ? pw[t - s_a] : 0.f;
+                b *= s_b <= t ? pw[t - s_b] : 0.f;
+              }
+              pk[i] = pack_bf16(a, b);
+              rs += bf_lo(pk[i]) + bf_hi(pk[i]);
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) pk[i] = 0u;
+          }
+          // bf16 pairs of keys 32 bk .. 32 bk + 31 into columns 16 bk .. 16 bk + 15,
+          // which the loads of this or an earlier block have already read
+          tmem_st_32x32b_x16(tmem + lf + kTmA + bk * 16, pk);
+        }
+        tmem_wait_st();
+        den[s * 128 + t] += rs;   // phi(q).z was written there by the feature-map warps
+      }
+      tc_fence_before();
+      named_bar_sync(kBarP, 128);
+      if (rf) break;
+      if (t == 0) {
+        mbar_arrive(bar(kPDone));
+        mbar_arrive(bar(kDen0 + s));
+      }
+    }
+  } else if (warp >= 8 && warp < 12) {
+    // ---------------------------------------------------------- output y
+    const int wq = warp - 8;
+    const int t = wq * 32 + lane;
+    const uint32_t lf = static_cast<uint32_t>(wq * 32) << 16;
+    volatile int &rf = role_fail[1];
+    for (int c = 0; c < nchunks; ++c) {
+      const int s = c & 1;
+      if (*abort_flag || !mbar_wait(bar(kO0 + s), (c >> 1) & 1) ||
+          !mbar_wait(bar(kDen0 + s), (c >> 1) & 1)) {
+        rf = 1;
+        fail();
+      }
+      tc_fence_after();
+      if (!rf) {
+        const float inv = 1.f / (den[s * 128 + t] + eps);
+        const bool live = t < Cv_of(c);
+        uint4 *dst = reinterpret_cast<uint4 *>(
+            out + (pair * N + n0 + static_cast<long>(c) * C + (live ? t : 0)) * DV);
+#pragma unroll
+        for (int blk = 0; blk < DV / 32; ++blk) {
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(tmem + lf + kTmO + s * 128 + blk * 32, r);
+          tmem_wait_ld();
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            pk[i] = pack_bf16(__uint_as_float(r[2 * i]) * inv, __uint_as_float(r[2 * i + 1]) * inv);
+          if (live) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              dst[blk * 4 + i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+          }
+        }
+      }
+      tc_fence_before();
+      named_bar_sync(kBarOut, 128);
+      if (rf) break;
+      if (t == 0) mbar_arrive(bar(kOut0 + s));
+    }
+  } else if (warp >= 12 && warp < 16) {
+    // ------------------------------------- state: operand S' and decay
+    const int wq = warp - 12;
+    const int r = wq * 32 + lane;             // d_k row
+    const bool live = r < DK;
+    const uint32_t lf = static_cast<uint32_t>(wq * 32) << 16;
+    volatile int &rf = role_fail[2];
+    // bf16 row of the MN-major operand (row = d_k, 64 d_v per panel)
+    auto put_op = [&](int blk, const uint32_t (&v32)[32], float f) {
+      uint32_t pk[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        pk[i] = pack_bf16(__uint_as_float(v32[2 * i]) * f, __uint_as_float(v32[2 * i + 1]) * f);
+      const uint32_t col = blk * 32;     // first d_v column of this block
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        *reinterpret_cast<uint4 *>(sm + kOffSop + (col >> 6) * kPanel +
+                                   sw128_offset(r, (col & 63) * 2 + i * 16)) =
+            make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+    };
+    // starting state: D_S = lambda^Cv0 S0, operand = S0 scaled as the carried term wants
+    if (has_init && nchunks > 0) {
+      const float g0 = pw[Cv_of(0)];
+      const float fop = factored ? g0 : 1.f;
+      const float *src = S0 + (pair * DK + (live ? r : 0)) * static_cast<long>(DV);
+#pragma unroll
+      for (int blk = 0; blk < DV / 32; ++blk) {
+        uint32_t v32[32], sv[32];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float4 f = live ? reinterpret_cast<const float4 *>(src)[blk * 8 + i]
+                                : make_float4(0.f, 0.f, 0.f, 0.f);
+          v32[4 * i] = __float_as_uint(f.x);
+          v32[4 * i + 1] = __float_as_uint(f.y);
+          v32[4 * i + 2] = __float_as_uint(f.z);
+          v32[4 * i + 3] = __float_as_uint(f.w);
+        }
+#pragma unroll
+        for (int i = 0; i < 32; ++i) sv[i] = __float_as_uint(__uint_as_float(v32[i]) * g0);
+        tmem_st_32x32b_x32(tmem + lf + kTmS + blk * 32, sv);
+        put_op(blk, v32, fop);
+      }
+      tmem_wait_st();
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    named_bar_sync(kBarState, 128);
+    if (r == 0) mbar_arrive(bar(kReadout));
+    for (int c = 0; c < nchunks; ++c) {
+      const bool last = c == nchunks - 1;
+      if (*abort_flag || !mbar_wait(bar(kState), c & 1)) {
+        rf = 1;
+        fail();
+      }
+      tc_fence_after();
+      if (!rf) {
+        const float gn = last ? 1.f : pw[Cv_of(c + 1)];
+        const float fop = factored ? gn : 1.f;
+#pragma unroll
+        for (int blk = 0; blk < DV / 32; ++blk) {
+          uint32_t sv[32];
+          tmem_ld_32x32b_x32(tmem + lf + kTmS + blk * 32, sv);
+          tmem_wait_ld();
+          if (last) {
+            if (last_seg && S_final && live) {
+              float4 *dst = reinterpret_cast<float4 *>(S_final + (pair * DK + r) * DV) + blk * 8;
+#pragma unroll
+              for (int i = 0; i < 8; ++i)
+                dst[i] = make_float4(__uint_as_float(sv[4 * i]), __uint_as_float(sv[4 * i + 1]),
+                                     __uint_as_float(sv[4 * i + 2]), __uint_as_float(sv[4 * i + 3]));
+            }
+          } else {
+            put_op(blk, sv, fop);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) sv[i] = __float_as_uint(__uint_as_float(sv[i]) * gn);
+            tmem_st_32x32b_x32(tmem + lf + kTmS + blk * 32, sv);
+          }
+        }
+        if (!last) tmem_wait_st();
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      named_bar_sync(kBarState, 128);
+      if (rf) break;
+      if (r == 0 && !last) mbar_arrive(bar(kReadout));
+    }
+  } else if (warp >= 16) {
+    // -------------------------------------------------------- feature map
+    const int tt = tid - 512;                 // 0..255
+    volatile int &rf = role_fail[3];
+    auto check = [&](bool ok_wait) {
+      if (!ok_wait || *abort_flag) {
+        rf = 1;
+        fail();
+      }
+    };
+    // q: thread (row tq, half hq of the row's 16-byte chunks)
+    const int tq = tt >> 1, hq = tt & 1;
+    constexpr int QCH = KCH / 2;
+    // k: thread (column group cg of 8 columns, row block rb)
+    constexpr int NCG = KCH;                  // 16 or 8 column groups
+    constexpr int RPB = NCG / 2;              // rows per row block (8 or 4)
+    const int cg = tt % NCG, rb = tt / NCG;
+    for (int c = 0; c < nchunks; ++c) {
+      const int s = c & 1;
+      const int Cv = Cv_of(c);
+      uint8_t *st = sm + s * kStage;
+      if (tt == 0) {
+        check(mbar_wait(bar(kFullQK0 + s), (c >> 1) & 1));
+        // den[s] was read by the output of chunk c - 2
+        if (c >= 2) check(mbar_wait(bar(kOut0 + s), ((c - 2) >> 1) & 1));
+      }
+      named_bar_sync(kBarPhi, kPhiThreads);
+      if (rf) break;
+      const float gC = pw[Cv];
+      // (1) factored: the carried term reads lambda^Cv z; scale z first
+      if (factored && tt < 128) zs[tt] *= gC;
+      named_bar_sync(kBarPhi, kPhiThreads);
+      // (2) q rows: feature map, decay scale, phi(q).z
+      {
+        float fq;
+        if (tq >= Cv) fq = 0.f;
+        else fq = factored ? 1.f / pw[Cv - 1 - tq] : 1.f;
+        const uint32_t f2 = pack_bf16(fq, fq);
+        float qz = 0.f;
+        uint4 w[QCH];
+#pragma unroll
+        for (int j = 0; j < QCH; ++j)
+          w[j] = *reinterpret_cast<const uint4 *>(st + kOffQ + chunk_off(tq, hq * QCH + j));
+#pragma unroll
+        for (int j = 0; j < QCH; ++j) {
+          uint32_t e[4] = {w[j].x, w[j].y, w[j].z, w[j].w};
+          const float4 za = *reinterpret_cast<const float4 *>(zs + (hq * QCH + j) * 8);
+          const float4 zb = *reinterpret_cast<const float4 *>(zs + (hq * QCH + j) * 8 + 4);
+          const float zz[8] = {za.x, za.y, za.z, za.w, zb.x, zb.y, zb.z, zb.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            if (!ident) e[i] = phi_bf16x2(e[i]);
+            e[i] = mul_bf16x2(e[i], f2);
+            qz = fmaf(bf_lo(e[i]), zz[2 * i], qz);
+            qz = fmaf(bf_hi(e[i]), zz[2 * i + 1], qz);
+          }
+          w[j] = make_uint4(e[0], e[1], e[2], e[3]);
+        }
+#pragma unroll
+        for (int j = 0; j < QCH; ++j)
+          *reinterpret_cast<uint4 *>(st + kOffQ + chunk_off(tq, hq * QCH + j)) = w[j];
+        qz += __shfl_xor_sync(0xffffffffu, qz, 1);
+        // explicit decay: the carried term of row t is lambda^(t+1) phi(q_t).z
+        if (!factored) qz *= tq < Cv ? pw[tq + 1] : 0.f;
+        if (hq == 0) den[s * 128 + tq] = qz;
+      }
+      named_bar_sync(kBarPhi, kPhiThreads);
+      if (!factored && tt < 128) zs[tt] *= gC;
+      if (!factored) named_bar_sync(kBarPhi, kPhiThreads);
+      // (3) k: feature map, decay weights (factored), column sums into z
+      {
+        float csum[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) csum[e] = 0.f;
+#pragma unroll
+        for (int i = 0; i < RPB; ++i) {
+          const int row = rb * RPB + i;
+          const float wk = row < Cv ? pw[Cv - 1 - row] : 0.f;
+          const uint32_t f2 = pack_bf16(factored ? wk : (row < Cv ? 1.f : 0.f),
+                                        factored ? wk : (row < Cv ? 1.f : 0.f));
+          uint8_t *p = st + kOffK + chunk_off(row, cg);
+          uint4 w = *reinterpret_cast<const uint4 *>(p);
+          uint32_t e[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            if (!ident) e[q4] = phi_bf16x2(e[q4]);
+            e[q4] = mul_bf16x2(e[q4], f2);
+            // the explicit path keeps phi(k) unweighted for the score MMA; the
+            // normaliser takes the weights here
+            const float m = factored ? 1.f : wk;
+            csum[2 * q4] = fmaf(bf_lo(e[q4]), m, csum[2 * q4]);
+            csum[2 * q4 + 1] = fmaf(bf_hi(e[q4]), m, csum[2 * q4 + 1]);
+          }
+          *reinterpret_cast<uint4 *>(p) = make_uint4(e[0], e[1], e[2], e[3]);
+        }
+        // reduce over the row blocks of this warp, then across warps
+#pragma unroll
+        for (int o = NCG; o < 32; o <<= 1)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) csum[e] += __shfl_xor_sync(0xffffffffu, csum[e], o);
+        if (lane < NCG) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) atomicAdd(zs + cg * 8 + e, csum[e]);
+        }
+      }
+      fence_proxy_async_smem();
+      named_bar_sync(kBarPhi, kPhiThreads);
+      if (tt == 0) mbar_arrive(bar(kPhi0 + s));
+      if (!factored) {
+        // after the score MMA: q rows times lambda^(t+1), k rows times lambda^(Cv-1-s)
+        if (tt == 0) check(mbar_wait(bar(kScore), c & 1));
+        named_bar_sync(kBarPhi, kPhiThreads);
+        if (rf) break;
+#pragma unroll
+        for (int which = 0; which < 2; ++which) {
+          const float f = which == 0 ? (tq < Cv ? pw[tq + 1] : 0.f)
+                                     : (tq < Cv ? pw[Cv - 1 - tq] : 0.f);
+          const uint32_t f2 = pack_bf16(f, f);
+          uint8_t *base = st + (which == 0 ? kOffQ : kOffK);
+#pragma unroll
+          for (int j = 0; j < QCH; ++j) {
+            uint4 *p = reinterpret_cast<uint4 *>(base + chunk_off(tq, hq * QCH + j));
+            uint4 w = *p;
+            *p = make_uint4(mul_bf16x2(w.x, f2), mul_bf16x2(w.y, f2), mul_bf16x2(w.z, f2),
+                            mul_bf16x2(w.w, f2));
+          }
+        }
+        fence_proxy_async_smem();
+        named_bar_sync(kBarPhi, kPhiThreads);
+        if (tt == 0) mbar_arrive(bar(kRescale));
+      }
+    }
+    named_bar_sync(kBarPhi, kPhiThreads);
+    if (!rf && last_seg && z_final && tt < DK) z_final[pair * DK + tt] = zs[tt];
+  }
+
+  // ------------------------------------------------------------ teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmCols);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// State pass: for segment g of each head (tokens [g len, min(N, (g+1) len))),
+// the segment's own final state from zero,
+//   dS_g = sum_s lambda^(n-1-s) phi(k_s) v_s^T,  dz_g = sum_s lambda^(n-1-s) phi(k_s)
+// (s and n counted inside the segment), written to slot pair * slots + g of
+// out_S / out_z.  The segmented forward runs it on its first G - 1 segments
+// (slots = G; the combine scan then turns the slots into starting states);
+// linattn_causal_state runs it on whole sequences (one segment, slots = 1).
+// Roles (512 threads): warp 0 TMA (k and v, 3 stages), warp 1 MMA issuer,
+// warps 4-7 decay of the TMEM state between chunks, warps 8-15 feature map.
+namespace sp {
+constexpr int NT = 512;
+constexpr int kStages = 3;
+constexpr uint32_t kOffK = 0, kOffV = 2 * kPanel;
+constexpr uint32_t kStage = 4 * kPanel;                  // 64 KB
+constexpr uint32_t kOffMisc = kStages * kStage;          // 192 KB
+constexpr uint32_t kMiscTmem = 256, kMiscAbort = 260, kMiscRoleFail = 272;
+constexpr uint32_t kMiscPw = 320, kMiscZ = 848;
+constexpr uint32_t kSmemBytes = kOffMisc + kMiscZ + 128 * 4;
+static_assert(kSmemBytes <= 232448, "exceeds the per-CTA shared memory of sm_100");
+enum Bar { kFull0 = 0, kFree0 = 3, kPhi0 = 6, kState = 9, kDecay, kFinal, kNumBars };
+constexpr int kBarPhi = 1, kBarDecay = 2;
+}  // namespace sp
+
+template <int DKP, int DVP>
+__global__ void __launch_bounds__(sp::NT, 1)
+    causal_seg_state_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
+                               const __grid_constant__ CUtensorMap tm_v,
+                               const float *__restrict__ lam, float *__restrict__ out_S,
+                               float *__restrict__ out_z, int H, int N, int seg_len, int nseg,
+                               int slots, bool ident) {
+  constexpr int DK = 64 * DKP, DV = 64 * DVP;
+  constexpr int KCH = 8 * DKP;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *sm = smem_raw;
+  const uint32_t sb = smem_u32(sm);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (sb & 1023u) {
+    if (tid == 0) atomicOr(&g_status, kStatusWaitTimeout);
+    return;
+  }
+  const long pair = blockIdx.x / nseg;
+  const int g = blockIdx.x % nseg;
+  const long slot = pair * slots + g;
+  const float L = lam ? lam[pair % H] : 1.f;
+  const int n0 = g * seg_len;
+  const int n1 = min(N, n0 + seg_len);
+  const int nchunks = (n1 - n0 + C - 1) / C;
+  const int Ct = (n1 - n0) - (nchunks - 1) * C;   // valid tokens of the last chunk
+  auto Cv_of = [&](int c) { return c == nchunks - 1 ? Ct : C; };
+  uint8_t *misc = sm + sp::kOffMisc;
+  auto bar = [&](int i) { return sb + sp::kOffMisc + 8u * static_cast<uint32_t>(i); };
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(misc + sp::kMiscTmem);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(misc + sp::kMiscAbort);
+  volatile int *role_fail = reinterpret_cast<volatile int *>(misc + sp::kMiscRoleFail);
+  float *pw = reinterpret_cast<float *>(misc + sp::kMiscPw);
+  float *zs = reinterpret_cast<float *>(misc + sp::kMiscZ);
+  if (tid == 0) {
+    for (int i = 0; i < sp::kNumBars; ++i) mbar_init(bar(i), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+  }
+  if (tid < 4) role_fail[tid] = 0;
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), 128);
+    tmem_relinquish();
+  }
+  if (tid <= C) pw[tid] = pow_int(L, tid);
+  if (tid < 128) zs[tid] = 0.f;
+  if (DKP == 1)
+    for (uint32_t o = tid * 16u; o < sp::kStages * kPanel; o += sp::NT * 16u)
+      *reinterpret_cast<uint4 *>(sm + (o / kPanel) * sp::kStage + sp::kOffK + kPanel + o % kPanel) =
+          make_uint4(0, 0, 0, 0);
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  auto fail = [&]() { *abort_flag = 1; };
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int issued = 0;
+      for (int c = 0; c < nchunks && !*abort_flag; ++c) {
+        const int s = c % sp::kStages;
+        if (c >= sp::kStages &&
+            !mbar_wait(bar(sp::kFree0 + s), ((c - sp::kStages) / sp::kStages) & 1)) {
+          fail();
+          break;
+        }
+        const uint32_t base = sb + s * sp::kStage;
+        const uint32_t b = bar(sp::kFull0 + s);
+        const int y = n0 + c * C;
+        mbar_arrive_expect_tx(b, (DKP + DVP) * kPanel);
+        for (int p = 0; p < DKP; ++p)
+          tma_load_3d(base + sp::kOffK + p * kPanel, &tm_k, b, 64 * p, y, static_cast<int>(pair));
+        for (int p = 0; p < DVP; ++p)
+          tma_load_3d(base + sp::kOffV + p * kPanel, &tm_v, b, 64 * p, y, static_cast<int>(pair));
+        if (c + sp::kStages < nchunks) {
+          for (int p = 0; p < DKP; ++p)
+            tma_prefetch_l2_3d(&tm_k, 64 * p, y + sp::kStages * C, static_cast<int>(pair));
+          for (int p = 0; p < DVP; ++p)
+            tma_prefetch_l2_3d(&tm_v, 64 * p, y + sp::kStages * C, static_cast<int>(pair));
+        }
+        issued = c + 1;
+      }
+      if (*abort_flag)
+        for (int c = issued - sp::kStages < 0 ? 0 : issued - sp::kStages; c < issued; ++c)
+          mbar_wait(bar(sp::kFull0 + c % sp::kStages), (c / sp::kStages) & 1);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc_bf16(128, DV, 1, 1);
+      bool ok = true;
+      for (int c = 0; ok && c < nchunks; ++c) {
+        const int s = c % sp::kStages;
+        const uint32_t st = sb + s * sp::kStage;
+        if (*abort_flag || !mbar_wait(bar(sp::kPhi0 + s), (c / sp::kStages) & 1) ||
+            (c >= 1 && !mbar_wait(bar(sp::kDecay), (c - 1) & 1))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint64_t k0 = sdesc_sw128(st + sp::kOffK, kPanel, 1024);
+        const uint64_t v0 = sdesc_sw128(st + sp::kOffV, kPanel, 1024);
+#pragma unroll
+        for (int ks = 0; ks < C / 16; ++ks)
+          umma_bf16(tmem, k0 + ks * (2048 >> 4), v0 + ks * (2048 >> 4), idS,
+                    (c > 0 || ks > 0) ? 1u : 0u);
+        umma_commit(bar(sp::kState));
+        umma_commit(bar(sp::kFree0 + s));
+      }
+      if (!ok) fail();
+      umma_commit(bar(sp::kFinal));
+      mbar_wait(bar(sp::kFinal), 0);
+    }
+    __syncwarp();
+  } else if (warp >= 4 && warp < 8) {
+    const int wq = warp - 4;
+    const int r = wq * 32 + lane;
+    const uint32_t lf = static_cast<uint32_t>(wq * 32) << 16;
+    volatile int &rf = role_fail[0];
+    for (int c = 0; c < nchunks; ++c) {
+      const bool last = c == nchunks - 1;
+      if (*abort_flag || !mbar_wait(bar(sp::kState), c & 1)) {
+        rf = 1;
+        fail();
+      }
+      tc_fence_after();
+      if (!rf) {
+        const float gC = last ? 1.f : pw[Cv_of(c + 1)];
+#pragma unroll
+        for (int blk = 0; blk < DV / 32; ++blk) {
+          uint32_t sv[32];
+          tmem_ld_32x32b_x32(tmem + lf + blk * 32, sv);
+          tmem_wait_ld();
+          if (last) {
+            if (r < DK) {
+              float4 *dst = reinterpret_cast<float4 *>(
+                                out_S + (slot * DK + r) * static_cast<long>(DV)) +
+                            blk * 8;
+#pragma unroll
+              for (int i = 0; i < 8; ++i)
+                dst[i] = make_float4(__uint_as_float(sv[4 * i]), __uint_as_float(sv[4 * i + 1]),
+                                     __uint_as_float(sv[4 * i + 2]), __uint_as_float(sv[4 * i + 3]));
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) sv[i] = __float_as_uint(__uint_as_float(sv[i]) * gC);
+            tmem_st_32x32b_x32(tmem + lf + blk * 32, sv);
+          }
+        }
+        if (!last) tmem_wait_st();
+      }
+      tc_fence_before();
+      named_bar_sync(sp::kBarDecay, 128);
+      if (rf) break;
+      if (r == 0 && !last) mbar_arrive(bar(sp::kDecay));
+    }
+  } else if (warp >= 8) {
+    const int tt = tid - 256;                 // 0..255
+    volatile int &rf = role_fail[1];
+    constexpr int NCG = KCH, RPB = NCG / 2;
+    const int cg = tt % NCG, rb = tt / NCG;
+    for (int c = 0; c < nchunks; ++c) {
+      const int s = c % sp::kStages;
+      uint8_t *st = sm + s * sp::kStage;
+      if (tt == 0 && (*abort_flag || !mbar_wait(bar(sp::kFull0 + s), (c / sp::kStages) & 1))) {
+        rf = 1;
+        fail();
+      }
+      named_bar_sync(sp::kBarPhi, 256);
+      if (rf) break;
+      const int Cv = Cv_of(c);
+      if (tt < 128) zs[tt] *= pw[Cv];
+      named_bar_sync(sp::kBarPhi, 256);
+      float csum[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) csum[e] = 0.f;
+#pragma unroll
+      for (int i = 0; i < RPB; ++i) {
+        const int row = rb * RPB + i;
+        const float wk = row < Cv ? pw[Cv - 1 - row] : 0.f;
+        const uint32_t f2 = pack_bf16(wk, wk);
+        uint8_t *p = st + sp::kOffK + chunk_off(row, cg);
+        uint4 w = *reinterpret_cast<const uint4 *>(p);
+        uint32_t e[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          if (!ident) e[q4] = phi_bf16x2(e[q4]);
+          e[q4] = mul_bf16x2(e[q4], f2);
+          csum[2 * q4] += bf_lo(e[q4]);
+          csum[2 * q4 + 1] += bf_hi(e[q4]);
+        }
+        *reinterpret_cast<uint4 *>(p) = make_uint4(e[0], e[1], e[2], e[3]);
+      }
+#pragma unroll
+      for (int o = NCG; o < 32; o <<= 1)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) csum[e] += __shfl_xor_sync(0xffffffffu, csum[e], o);
+      if (lane < NCG) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) atomicAdd(zs + cg * 8 + e, csum[e]);
+      }
+      fence_proxy_async_smem();
+      named_bar_sync(sp::kBarPhi, 256);
+      if (tt == 0) mbar_arrive(bar(sp::kPhi0 + s));
+    }
+    named_bar_sync(sp::kBarPhi, 256);
+    if (!rf && tt < DK) out_z[slot * DK + tt] = zs[tt];
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 128);
+  }
+}
+
+}  // namespace stc
+}  // namespace linattn

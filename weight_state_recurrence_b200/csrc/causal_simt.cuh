@@ -229,7 +229,7 @@ template <int DK, int DVS, typename T>
 __global__ void __launch_bounds__(256) causal_seg_state_kernel(
     const T *__restrict__ k, const T *__restrict__ v, const float *__restrict__ lam,
     float *__restrict__ ws_S, float *__restrict__ ws_z, int H, int N, int DV, int seg_len,
-    int G, bool ident) {
+    int slots, bool ident) {
   constexpr int C = kSimtChunk, NT = 256, QS = DK + 1;
   constexpr int NR = DK / 16, NCOL = DVS / 16;
   __shared__ float sK[C * QS];      // lambda^(Cv-1-s) phi(k_s)
@@ -306,20 +306,21 @@ __global__ void __launch_bounds__(256) causal_seg_state_kernel(
       for (int t = 0; t < Cv; ++t) zacc += sK[t * QS + tid];
     }
   }
-  float *Sg = ws_S + (pair * G + g) * static_cast<long>(DK) * DV;
+  float *Sg = ws_S + (pair * slots + g) * static_cast<long>(DK) * DV;
 #pragma unroll
   for (int r = 0; r < NR; ++r)
 #pragma unroll
     for (int m = 0; m < NCOL; ++m) Sg[(ty + 16 * r) * static_cast<long>(DV) + j0 + tx + 16 * m] = acc[r][m];
-  if (j0 == 0 && tid < DK) ws_z[(pair * G + g) * static_cast<long>(DK) + tid] = zacc;
+  if (j0 == 0 && tid < DK) ws_z[(pair * slots + g) * static_cast<long>(DK) + tid] = zacc;
 }
 
 // carry_0 = (S_init, z_init) or zero; carry_{g+1} = lambda^len_g carry_g + dS_g,
-// written over dS_g's slot; one CTA per (b, h), one element per thread step
+// written over dS_g's slot.  Grid: blockIdx.x is the (b, h) pair, blockIdx.y
+// a block of 256 of its DK*DV + DK state elements, one element per thread.
 __global__ void __launch_bounds__(256) causal_seg_combine_kernel(
     const float *__restrict__ lam, const float *__restrict__ S_init,
     const float *__restrict__ z_init, float *__restrict__ ws_S, float *__restrict__ ws_z, int H,
-    int DK, int DV, int N, int seg_len, int G) {
+    int DK, int DV, long N, int seg_len, int G, bool seg_major) {
   // blockIdx.x: the (b, h) pair; blockIdx.y: a block of 256 of its DK*DV + DK
   // state elements, one per thread.  Each element's G segment values are read
   // eight at a time before any is overwritten, so a thread has eight loads in
@@ -328,17 +329,21 @@ __global__ void __launch_bounds__(256) causal_seg_combine_kernel(
   const long pair = blockIdx.x;
   const float L = lam ? lam[pair % H] : 1.f;
   for (int gg = threadIdx.x; gg < G; gg += blockDim.x)
-    decay[gg] = pow_int(L, min(seg_len, N - gg * seg_len));
+    decay[gg] = pow_int(L, static_cast<int>(min(static_cast<long>(seg_len),
+                                                 N - static_cast<long>(gg) * seg_len)));
   __syncthreads();
   const long per = static_cast<long>(DK) * DV;
   const long e = static_cast<long>(blockIdx.y) * blockDim.x + threadIdx.x;
   if (e >= per + DK) return;
   const bool isz = e >= per;
   const long ei = isz ? e - per : e;
-  float *base = isz ? ws_z + pair * G * static_cast<long>(DK) : ws_S + pair * G * per;
-  const long stride = isz ? DK : per;
+  const long unit = isz ? DK : per;   // one state's elements
+  // [B*H][G] slots (the segmented forward's workspace) or [G][B*H] (segment
+  // states gathered from several devices)
+  float *base = (isz ? ws_z : ws_S) + (seg_major ? pair : pair * G) * unit;
+  const long stride = seg_major ? static_cast<long>(gridDim.x) * unit : unit;
   const float *init = isz ? z_init : S_init;
-  float run = init ? init[pair * stride + ei] : 0.f;
+  float run = init ? init[pair * unit + ei] : 0.f;
   for (int g0 = 0; g0 < G; g0 += 8) {
     float d[8];
 #pragma unroll

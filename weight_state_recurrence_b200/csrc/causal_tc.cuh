@@ -65,24 +65,6 @@
 #include "common.cuh"
 #include "sm100.cuh"
 
-// Optional per-chunk timeline (compiled out unless LINATTN_TRACE is defined):
-// one thread of each role records clock64() at the points below for the
-// first two CTAs, into a buffer the host installs in g_trace.
-#ifdef LINATTN_TRACE
-namespace linattn {
-__device__ unsigned long long *g_trace;
-}
-#define LINATTN_TRACE_EVENT(c, ev)                                                        \
-  do {                                                                                    \
-    if (blockIdx.x < 2 && ::linattn::g_trace && (c) < 256)                                \
-      ::linattn::g_trace[(blockIdx.x * 256 + (c)) * 16 + (ev)] = clock64();                \
-  } while (0)
-#else
-#define LINATTN_TRACE_EVENT(c, ev) \
-  do {                             \
-  } while (0)
-#endif
-
 namespace linattn {
 namespace tc {
 
@@ -448,7 +430,6 @@ __global__ void __launch_bounds__(NT, 1)
               tma_prefetch_l2_3d(&tm_k, 64, yp, pair);
             }
           }
-          LINATTN_TRACE_EVENT(c, 0);
         } else {
           const uint32_t b = bar(kFullV0 + s);
           mbar_arrive_expect_tx(b, kVTxBytes);
@@ -483,7 +464,6 @@ __global__ void __launch_bounds__(NT, 1)
           if ((ks & 3) == 0) {
             if (!mbar_wait(bar((ks == 0 ? kPhi0 : kPhiB0) + s), (c >> 1) & 1)) return false;
             tc_fence_after();
-            if (ks == 0) LINATTN_TRACE_EVENT(c, 5);
           }
           const uint32_t off = (ks >> 2) * kPanel + (ks & 3) * 32;
           umma_bf16(tmem + kTmA + s * 128, sdesc_sw128(st + kOffQ + off, 16, 1024),
@@ -507,7 +487,6 @@ __global__ void __launch_bounds__(NT, 1)
           break;
         }
         tc_fence_after();
-        LINATTN_TRACE_EVENT(c, 8);
 #pragma unroll
         for (int ks = 0; ks < C / 16; ++ks)
           umma_bf16(tmem + kTmS, sdesc_sw128(st + kOffK + ks * 2048, kPanel, 1024),
@@ -520,7 +499,6 @@ __global__ void __launch_bounds__(NT, 1)
           break;
         }
         tc_fence_after();
-        LINATTN_TRACE_EVENT(c, 6);
 #pragma unroll
         for (int ks = 0; ks < DK / 16; ++ks) {
           if (ks >= 4 * kpanels) break;
@@ -536,7 +514,6 @@ __global__ void __launch_bounds__(NT, 1)
           break;
         }
         tc_fence_after();
-        LINATTN_TRACE_EVENT(c, 7);
 #pragma unroll
         for (int ks = 0; ks < C / 16; ++ks)
           umma_bf16(tmem + kTmOV,
@@ -569,7 +546,6 @@ __global__ void __launch_bounds__(NT, 1)
       if (tt == 0) *consumed = c + 1;
       // the peer's MMAs must be done with its copy of this stage before we copy into it
       if (kPair && tt == 0 && c >= 2) check(mbar_wait(bar(kPeerFree0 + s), ((c - 2) >> 1) & 1));
-      if (tt == 0) LINATTN_TRACE_EVENT(c, 1);
       // this CTA's rows, one d_k half (q panel g and k panel g) at a time
       const bool tail = c == nchunks - 1;
       for (int g = 0; g < kpanels; ++g) {
@@ -581,7 +557,6 @@ __global__ void __launch_bounds__(NT, 1)
         named_bar_sync(kBarXform, kXformThreads);
         if (rf) return false;
         if (tt == 0) {
-          if (g == 1) LINATTN_TRACE_EVENT(c, 2);
           const uint32_t pb = bar((g == 0 ? kPhi0 : kPhiB0) + s);
           if (kPair) {
             const uint32_t src = sb + s * kStage + kOffQ + g * kPanel + own_off;
@@ -601,7 +576,6 @@ __global__ void __launch_bounds__(NT, 1)
     auto weight_k = [&](int c) -> bool {
       const int s = c & 1;
       check(mbar_wait(bar(kAFull0 + s), (c >> 1) & 1));   // the score MMA has read phi(K)
-      if (tt == 0) LINATTN_TRACE_EVENT(c, 3);
       const float *wk = c == nchunks - 1 ? kt : kf;
       if (!rf)
         tile_pass<4>(sm + s * kStage + kOffK, 2 * kPanel, 2 * kPanel, 1, tt, kXformThreads,
@@ -612,7 +586,6 @@ __global__ void __launch_bounds__(NT, 1)
       fence_proxy_async_smem();
       named_bar_sync(kBarXform, kXformThreads);
       if (rf) return false;
-      if (tt == 0) LINATTN_TRACE_EVENT(c, 4);
       if (tt == 0) mbar_arrive(bar(kKsDone));
       return true;
     };
@@ -637,7 +610,6 @@ __global__ void __launch_bounds__(NT, 1)
         fail();
       }
       tc_fence_after();
-      if (t == 0) LINATTN_TRACE_EVENT(c, 9);
       // only blocks at or below the diagonal change; the others stay zero
       for (int bk = 0; !rf && bk <= wq; ++bk) {
         uint32_t r[32];
@@ -682,7 +654,6 @@ __global__ void __launch_bounds__(NT, 1)
       fence_proxy_async_smem();
       named_bar_sync(kBarEpiA, 128);
       if (rf) break;
-      if (t == 0) LINATTN_TRACE_EVENT(c, 10);
       if (t == 0) {
         mbar_arrive(bar(kAFree0 + b));
         mbar_arrive(bar(kAbfFull));
@@ -705,7 +676,6 @@ __global__ void __launch_bounds__(NT, 1)
         fail();
       }
       tc_fence_after();
-      if (r == 0) LINATTN_TRACE_EVENT(c, 13);
       if (!rf) {
         uint32_t zz[2];
         tmem_ld_32x32b_x2(tmem + lane_field + kTmS + 64, zz);   // z, junk
@@ -760,7 +730,6 @@ __global__ void __launch_bounds__(NT, 1)
       tc_fence_before();
       named_bar_sync(kBarOut, 128);
       if (rf) break;
-      if (r == 0) LINATTN_TRACE_EVENT(c, 14);
       if (r == 0) mbar_arrive(bar(kStateDone));
       // -- y for the chunk's rows
       okw = !*abort_flag && mbar_wait(bar(kOvDone), c & 1);
@@ -769,7 +738,6 @@ __global__ void __launch_bounds__(NT, 1)
         fail();
       }
       tc_fence_after();
-      if (r == 0) LINATTN_TRACE_EVENT(c, 11);
       if (!rf) {
         uint32_t rs[2], qz[2];
         tmem_ld_32x32b_x2(tmem + lane_field + kTmOV + 64, rs);   // row sum, junk
@@ -804,7 +772,6 @@ __global__ void __launch_bounds__(NT, 1)
       tc_fence_before();
       named_bar_sync(kBarOut, 128);
       if (rf) break;
-      if (r == 0) LINATTN_TRACE_EVENT(c, 12);
       if (r == 0) mbar_arrive(bar(kOutDone));
     }
   }

@@ -1,7 +1,7 @@
 // Global (non-causal) form on CUDA cores, fp32 arithmetic.
-//   pass 1: KV = sum_n phi(k_n) v_n^T and ksum = sum_n phi(k_n), split over
-//           N across CTAs and accumulated with fp32 atomics into the
-//           caller's (zeroed) KV / ksum;
+//   pass 1: KV = sum_n phi(k_n) v_n^T and ksum = sum_n phi(k_n) over the keys
+//           that are not padding, split over N across CTAs and accumulated
+//           with fp32 atomics into the caller's (zeroed) KV / ksum;
 //   pass 2: y_i = phi(q_i)^T KV / (phi(q_i)^T ksum + eps).
 // Linear-attention note §3 (after the sum swap) and §6 forward; "Beyond
 // self-attention", linear-attention code (here with eps).
@@ -15,12 +15,15 @@ namespace linattn {
 constexpr int kGlobalTile = 32;     // tokens staged per iteration
 constexpr int kGlobalSplit = 512;   // tokens per pass-1 CTA
 
+// kpm: key padding mask [B, N] (nonzero: the key is padding and enters
+// neither sum) or NULL; H: heads per sequence (to find a pair's row of kpm).
 template <int DK, int DV, typename T>
 __global__ void __launch_bounds__(256) global_kv_simt_kernel(const T *__restrict__ k,
                                                              const T *__restrict__ v,
+                                                             const uint8_t *__restrict__ kpm,
                                                              float *__restrict__ KV,
                                                              float *__restrict__ ksum, int N,
-                                                             bool ident) {
+                                                             int H, bool ident) {
   constexpr int NT = 256, TT = kGlobalTile;
   constexpr int ENT = DK * DV;
   constexpr int PER = (ENT + NT - 1) / NT;
@@ -34,12 +37,14 @@ __global__ void __launch_bounds__(256) global_kv_simt_kernel(const T *__restrict
 #pragma unroll
   for (int i = 0; i < PER; ++i) acc[i] = 0.f;
   float ks = 0.f;
+  const uint8_t *mrow = kpm ? kpm + (pair / H) * static_cast<long>(N) : nullptr;
   for (int t0 = n0; t0 < n1; t0 += TT) {
     const int tv = min(TT, n1 - t0);
     __syncthreads();
     for (int i = tid; i < TT * DK; i += NT) {
       const int t = i / DK, a = i % DK;
-      sK[t][a] = t < tv ? feat_f32(to_f32(k[(pair * N + t0 + t) * DK + a]), ident) : 0.f;
+      const bool live = t < tv && !(mrow && mrow[t0 + t]);
+      sK[t][a] = live ? feat_f32(to_f32(k[(pair * N + t0 + t) * DK + a]), ident) : 0.f;
     }
     for (int i = tid; i < TT * DV; i += NT) {
       const int t = i / DV, b = i % DV;

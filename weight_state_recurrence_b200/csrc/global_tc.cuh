@@ -7,7 +7,8 @@
 // Two persistent kernels, each bound by HBM traffic (k and v are read once by
 // the first, q read and y written once by the second):
 //
-// global_kv_tc_kernel: two heads of one sequence share every MMA.  With the
+// global_kv_tc_kernel: two heads of one sequence share every MMA (keys marked
+//   as padding are zeroed with the feature map, so they enter neither sum).  With the
 //   phi(k) tiles of both heads stacked along M (2 x 64 = 128 rows, MN-major)
 //   and the v tiles side by side along N, D[128 x 128] += phi(K)^T V holds
 //   both heads' KV on its diagonal blocks (the off-diagonal blocks are
@@ -52,9 +53,12 @@ __device__ __forceinline__ uint32_t phi2(uint32_t x) {
 }
 
 // phi in place over `bytes` of swizzled tile rows (128 bytes per row); rows at
-// or past `valid` become 0 when zero_tail (rows the TMA filled with zeros).
+// or past `valid` become 0 when zero_tail (rows the TMA filled with zeros), and
+// so do rows whose byte in `pad` (the tile's 128 rows of the key padding
+// mask, or NULL) is nonzero.
 __device__ __forceinline__ void phi_tile(uint8_t *p, uint32_t bytes, int valid, bool zero_tail,
-                                         bool ident, int tid, int nthr) {
+                                         bool ident, int tid, int nthr,
+                                         const uint8_t *pad = nullptr) {
   const uint32_t step = static_cast<uint32_t>(nthr) * 16u;
   for (uint32_t o0 = static_cast<uint32_t>(tid) * 16u; o0 < bytes; o0 += 4 * step) {
     uint4 w[4];
@@ -64,7 +68,8 @@ __device__ __forceinline__ void phi_tile(uint8_t *p, uint32_t bytes, int valid, 
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const uint32_t o = o0 + i * step;
-      const bool dead = zero_tail && static_cast<int>((o % kPanel) >> 7) >= valid;
+      const int row = static_cast<int>((o % kPanel) >> 7);
+      const bool dead = (zero_tail && row >= valid) || (pad && row < valid && pad[row]);
       w[i].x = dead ? 0u : ident ? w[i].x : phi2(w[i].x);
       w[i].y = dead ? 0u : ident ? w[i].y : phi2(w[i].y);
       w[i].z = dead ? 0u : ident ? w[i].z : phi2(w[i].z);
@@ -114,8 +119,9 @@ constexpr uint32_t kMiscTmem = 128, kMiscFail = 132, kMiscRoleFail = 136;
 
 __global__ void __launch_bounds__(kv::NT, 1)
     global_kv_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
-                        const __grid_constant__ CUtensorMap tm_v, float *__restrict__ KV,
-                        float *__restrict__ ksum, int npairs, int N, bool ident) {
+                        const __grid_constant__ CUtensorMap tm_v,
+                        const uint8_t *__restrict__ kpm, float *__restrict__ KV,
+                        float *__restrict__ ksum, int npairs, int N, int H, bool ident) {
   using namespace kv;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *sm = smem_raw;
@@ -243,7 +249,11 @@ __global__ void __launch_bounds__(kv::NT, 1)
         *fail = 1;
       }
       const int valid = N - u.index * C;
-      if (!*rfail) phi_tile(sm + s * kStage, 2 * kPanel, valid, valid < C, ident, tt, kXform);
+      // the pair's two heads belong to one sequence: one row of the padding mask
+      const uint8_t *pad =
+          kpm ? kpm + (2L * u.group / H) * N + static_cast<long>(u.index) * C : nullptr;
+      if (!*rfail)
+        phi_tile(sm + s * kStage, 2 * kPanel, valid, valid < C, ident, tt, kXform, pad);
       fence_proxy_async_smem();
       named_bar_sync(1, kXform);
       if (*rfail) break;

@@ -9,6 +9,7 @@
 #include <cstdint>
 #include <cstdlib>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 #include <set>
 #include <utility>
@@ -19,6 +20,7 @@
 #include "decode.cuh"
 #include "causal_simt.cuh"
 #include "causal_tc.cuh"
+#include "causal_seg_tc.cuh"
 #include "causal_bwd.cuh"
 #include "global_simt.cuh"
 #include "global_tc.cuh"
@@ -128,13 +130,27 @@ bool make_map_bf16(CUtensorMap *m, const void *ptr, int inner, int rows, int pla
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Which causal kernel: LINATTN_CAUSAL_KERNEL=simt forces the CUDA-core
-// kernel (a second opinion for tests); otherwise bf16 with d_k = 128 or 64
-// and dv a multiple of 64 takes the tensor-core kernel.
-bool use_tc_causal(const linattn_dims *d) {
-  const char *e = std::getenv("LINATTN_CAUSAL_KERNEL");
-  if (e && std::strcmp(e, "simt") == 0) return false;
-  return d->dtype == LINATTN_BF16 && (d->dk == tc::DK || d->dk == 64) && d->dv % tc::DVS == 0;
+// Kernel family per operation, set by linattn_set_kernel_choice (tests and
+// benchmarks compare families on the same call); AUTO unless set.
+std::atomic<int> g_choice[3] = {{LINATTN_KERNEL_AUTO}, {LINATTN_KERNEL_AUTO}, {LINATTN_KERNEL_AUTO}};
+std::atomic<int> g_forced_segments{0};
+
+int choice(int op) { return g_choice[op].load(std::memory_order_relaxed); }
+
+bool tc_causal_shape(const linattn_dims *d) {
+  return d->dtype == LINATTN_BF16 && (d->dk == 128 || d->dk == 64) && (d->dv == 128 || d->dv == 64);
+}
+
+// Which causal kernel: bf16 with d_k and d_v in {64, 128} takes the
+// segmented tensor-core kernel (one CTA per head and segment, the head's
+// whole d_v); the paired kernel (two CTAs per head, d_v split) and the
+// CUDA-core kernel are there when chosen explicitly.
+enum class CausalPath { kSegTc, kPairedTc, kSimt };
+CausalPath causal_path(const linattn_dims *d) {
+  const int c = choice(LINATTN_OP_CAUSAL);
+  if (c == LINATTN_KERNEL_CUDA_CORES || !tc_causal_shape(d)) return CausalPath::kSimt;
+  if (c == LINATTN_KERNEL_TC_PAIRED) return CausalPath::kPairedTc;
+  return CausalPath::kSegTc;
 }
 
 // ------------------------------------------------------------ launchers
@@ -201,7 +217,7 @@ int simt_dv_slice(int dv) { return dv <= 16 ? 16 : 32; }
 Segments plan_segments(const linattn_dims *d) {
   Segments sg;
   sg.len = d->N;
-  if (use_tc_causal(d) || d->N < 256) return sg;
+  if (causal_path(d) != CausalPath::kSimt || d->N < 256) return sg;
   const long ctas = static_cast<long>(d->B) * d->H * (d->dv / simt_dv_slice(d->dv));
   const int sms = num_sms();
   if (sms <= 0 || ctas == 0 || ctas >= sms) return sg;
@@ -240,7 +256,7 @@ int launch_causal_simt(const linattn_dims *d, const void *q, const void *k, cons
     if (cudaGetLastError() != cudaSuccess) return LINATTN_ERR_CUDA;
     const int eblocks = (d->dk * d->dv + d->dk + 255) / 256;
     causal_seg_combine_kernel<<<dim3(d->B * d->H, eblocks), 256, 0, s>>>(
-        lam, S_init, z_init, wsS, wsz, d->H, d->dk, d->dv, d->N, sg.len, sg.G);
+        lam, S_init, z_init, wsS, wsz, d->H, d->dk, d->dv, d->N, sg.len, sg.G, false);
     if (cudaGetLastError() != cudaSuccess) return LINATTN_ERR_CUDA;
   }
   kern<<<dim3(ctas, sg.G), 256, bytes, s>>>(
@@ -274,6 +290,87 @@ int causal_simt_dispatch(const linattn_dims *d, const void *q, const void *k, co
     case 128: return causal_simt_dv<128, T>(d, q, k, v, lam, eps, S_init, z_init, out, S_final, z_final, sg, s);
   }
   return LINATTN_ERR_UNSUPPORTED;
+}
+
+// Segment plan of the tensor-core causal kernel: G segments of seg_len
+// tokens (whole chunks) when one CTA per head would leave most SMs idle.
+struct TcSegments {
+  int G = 1, len = 0;
+};
+
+TcSegments plan_tc_segments(const linattn_dims *d) {
+  TcSegments sg;
+  sg.len = d->N;
+  const long BH = static_cast<long>(d->B) * d->H;
+  const int nch = (d->N + stc::C - 1) / stc::C;
+  const int sms = num_sms();
+  if (BH <= 0 || nch < 2 || sms <= 0) return sg;
+  long gmax = g_forced_segments.load(std::memory_order_relaxed);
+  if (gmax <= 0) {
+    gmax = sms / BH;               // about one CTA per SM
+    if (gmax < 3) return sg;       // the state pass re-reads k and v: not worth it for 2
+  }
+  gmax = std::min<long>(gmax, std::min(nch, kMaxSegments));
+  if (gmax < 2) return sg;
+  const int len_ch = (nch + static_cast<int>(gmax) - 1) / static_cast<int>(gmax);
+  sg.G = (nch + len_ch - 1) / len_ch;
+  sg.len = len_ch * stc::C;
+  if (sg.G < 2) sg = TcSegments{1, d->N};
+  return sg;
+}
+
+size_t tc_segment_bytes(const linattn_dims *d, const TcSegments &sg) {
+  if (sg.G < 2) return 0;
+  return static_cast<size_t>(d->B) * d->H * sg.G * (static_cast<size_t>(d->dk) * d->dv + d->dk) * 4;
+}
+
+template <int DKP, int DVP>
+int launch_causal_seg_tc_t(const linattn_dims *d, const CUtensorMap &mq, const CUtensorMap &mk,
+                           const CUtensorMap &mv, const float *lam, float eps,
+                           const float *S_init, const float *z_init, void *out, float *S_final,
+                           float *z_final, const TcSegments &sg, float *ws, cudaStream_t s) {
+  auto *kern = stc::causal_seg_tc_kernel<DKP, DVP>;
+  if (!set_smem(kern, static_cast<int>(stc::kSmemBytes))) return LINATTN_ERR_CUDA;
+  const int BH = d->B * d->H;
+  float *wsS = nullptr, *wsz = nullptr;
+  if (sg.G > 1) {
+    wsS = ws;
+    wsz = ws + static_cast<long>(BH) * sg.G * d->dk * d->dv;
+    // (1) each segment's own final state from zero, (2) the starting states
+    auto *sk = stc::causal_seg_state_tc_kernel<DKP, DVP>;
+    if (!set_smem(sk, static_cast<int>(stc::sp::kSmemBytes))) return LINATTN_ERR_CUDA;
+    sk<<<BH * (sg.G - 1), stc::sp::NT, stc::sp::kSmemBytes, s>>>(
+        mk, mv, lam, wsS, wsz, d->H, d->N, sg.len, sg.G - 1, sg.G, ident(d));
+    if (cudaGetLastError() != cudaSuccess) return LINATTN_ERR_CUDA;
+    const int eblocks = (d->dk * d->dv + d->dk + 255) / 256;
+    causal_seg_combine_kernel<<<dim3(BH, eblocks), 256, 0, s>>>(
+        lam, S_init, z_init, wsS, wsz, d->H, d->dk, d->dv, d->N, sg.len, sg.G, false);
+    if (cudaGetLastError() != cudaSuccess) return LINATTN_ERR_CUDA;
+  }
+  kern<<<BH * sg.G, stc::NT, stc::kSmemBytes, s>>>(
+      mq, mk, mv, lam, eps, S_init, z_init, wsS, wsz, static_cast<bf16 *>(out), S_final, z_final,
+      d->H, d->N, sg.len, sg.G, ident(d));
+  return launch_status();
+}
+
+int launch_causal_seg_tc(const linattn_dims *d, const void *q, const void *k, const void *v,
+                         const float *lam, float eps, const float *S_init, const float *z_init,
+                         void *out, float *S_final, float *z_final, const TcSegments &sg,
+                         float *ws, cudaStream_t s) {
+  const int BH = d->B * d->H;
+  CUtensorMap mq, mk, mv;
+  if (!make_map_bf16(&mq, q, d->dk, d->N, BH) || !make_map_bf16(&mk, k, d->dk, d->N, BH) ||
+      !make_map_bf16(&mv, v, d->dv, d->N, BH))
+    return LINATTN_ERR_CUDA;
+  if (d->dk == 128)
+    return d->dv == 128 ? launch_causal_seg_tc_t<2, 2>(d, mq, mk, mv, lam, eps, S_init, z_init, out,
+                                                       S_final, z_final, sg, ws, s)
+                        : launch_causal_seg_tc_t<2, 1>(d, mq, mk, mv, lam, eps, S_init, z_init, out,
+                                                       S_final, z_final, sg, ws, s);
+  return d->dv == 128 ? launch_causal_seg_tc_t<1, 2>(d, mq, mk, mv, lam, eps, S_init, z_init, out,
+                                                     S_final, z_final, sg, ws, s)
+                      : launch_causal_seg_tc_t<1, 1>(d, mq, mk, mv, lam, eps, S_init, z_init, out,
+                                                     S_final, z_final, sg, ws, s);
 }
 
 int launch_causal_tc(const linattn_dims *d, const void *q, const void *k, const void *v,
@@ -313,14 +410,14 @@ int launch_causal_tc(const linattn_dims *d, const void *q, const void *k, const 
 
 template <int DK, int DV, typename T>
 int launch_global_simt(const linattn_dims *d, int Nk, const void *q, const void *k,
-                       const void *v, float eps, void *out, float *KV, float *ksum,
-                       cudaStream_t s) {
+                       const void *v, const uint8_t *kpm, float eps, void *out, float *KV,
+                       float *ksum, cudaStream_t s) {
   // KV, ksum over the Nk keys (none: they stay zero), then y for the d->N queries
   const int BH = d->B * d->H;
   if (Nk > 0) {
     dim3 g1(BH, (Nk + kGlobalSplit - 1) / kGlobalSplit);
     global_kv_simt_kernel<DK, DV, T><<<g1, 256, 0, s>>>(
-        static_cast<const T *>(k), static_cast<const T *>(v), KV, ksum, Nk, ident(d));
+        static_cast<const T *>(k), static_cast<const T *>(v), kpm, KV, ksum, Nk, d->H, ident(d));
     if (cudaGetLastError() != cudaSuccess) return LINATTN_ERR_CUDA;
   }
   if (d->N > 0) {
@@ -335,11 +432,10 @@ int launch_global_simt(const linattn_dims *d, int Nk, const void *q, const void 
 }
 
 // Tensor-core global path: bf16, d_k = d_v = 64, an even number of heads
-// (heads are paired in the KV kernel).  LINATTN_GLOBAL_KERNEL=simt forces the
-// CUDA-core kernels.
+// (heads are paired in the KV kernel).  LINATTN_KERNEL_CUDA_CORES chosen for
+// the global operation forces the CUDA-core kernels.
 bool use_tc_global(const linattn_dims *d) {
-  const char *e = std::getenv("LINATTN_GLOBAL_KERNEL");
-  if (e && std::strcmp(e, "simt") == 0) return false;
+  if (choice(LINATTN_OP_GLOBAL) == LINATTN_KERNEL_CUDA_CORES) return false;
   return d->dtype == LINATTN_BF16 && d->dk == gtc::D && d->dv == gtc::D && d->H % 2 == 0;
 }
 
@@ -374,8 +470,8 @@ int zero_kv(float *KV, size_t nS, float *ksum, size_t nz, cudaStream_t s) {
 }
 
 int launch_global_tc(const linattn_dims *d, int Nk, const void *q, const void *k,
-                     const void *v, float eps, void *out, float *KV, float *ksum,
-                     cudaStream_t s) {
+                     const void *v, const uint8_t *kpm, float eps, void *out, float *KV,
+                     float *ksum, cudaStream_t s) {
   // KV, ksum over the Nk keys (none: they stay zero), then y for the d->N queries
   const int BH = d->B * d->H;
   const int sms = num_sms();
@@ -392,8 +488,8 @@ int launch_global_tc(const linattn_dims *d, int Nk, const void *q, const void *k
     // being zeroed; it waits for that grid only before its first flush
     const ProgrammaticLaunch pl(static_cast<int>(u1 < sms ? u1 : sms), gtc::kv::NT,
                                 gtc::kv::kSmemBytes, s);
-    if (cudaLaunchKernelEx(&pl.cfg, gtc::global_kv_tc_kernel, mk, mv, KV, ksum, BH / 2, Nk,
-                           ident(d)) != cudaSuccess)
+    if (cudaLaunchKernelEx(&pl.cfg, gtc::global_kv_tc_kernel, mk, mv, kpm, KV, ksum, BH / 2, Nk,
+                           d->H, ident(d)) != cudaSuccess)
       return LINATTN_ERR_CUDA;
   }
   if (d->N > 0) {
@@ -415,24 +511,25 @@ int launch_global_tc(const linattn_dims *d, int Nk, const void *q, const void *k
 
 template <int DK, typename T>
 int global_dv(const linattn_dims *d, int Nk, const void *q, const void *k, const void *v,
-              float eps, void *out, float *KV, float *ksum, cudaStream_t s) {
+              const uint8_t *kpm, float eps, void *out, float *KV, float *ksum, cudaStream_t s) {
   switch (d->dv) {
-    case 16: return launch_global_simt<DK, 16, T>(d, Nk, q, k, v, eps, out, KV, ksum, s);
-    case 32: return launch_global_simt<DK, 32, T>(d, Nk, q, k, v, eps, out, KV, ksum, s);
-    case 64: return launch_global_simt<DK, 64, T>(d, Nk, q, k, v, eps, out, KV, ksum, s);
-    case 128: return launch_global_simt<DK, 128, T>(d, Nk, q, k, v, eps, out, KV, ksum, s);
+    case 16: return launch_global_simt<DK, 16, T>(d, Nk, q, k, v, kpm, eps, out, KV, ksum, s);
+    case 32: return launch_global_simt<DK, 32, T>(d, Nk, q, k, v, kpm, eps, out, KV, ksum, s);
+    case 64: return launch_global_simt<DK, 64, T>(d, Nk, q, k, v, kpm, eps, out, KV, ksum, s);
+    case 128: return launch_global_simt<DK, 128, T>(d, Nk, q, k, v, kpm, eps, out, KV, ksum, s);
   }
   return LINATTN_ERR_UNSUPPORTED;
 }
 
 template <typename T>
 int global_dispatch(const linattn_dims *d, int Nk, const void *q, const void *k, const void *v,
-                    float eps, void *out, float *KV, float *ksum, cudaStream_t s) {
+                    const uint8_t *kpm, float eps, void *out, float *KV, float *ksum,
+                    cudaStream_t s) {
   switch (d->dk) {
-    case 16: return global_dv<16, T>(d, Nk, q, k, v, eps, out, KV, ksum, s);
-    case 32: return global_dv<32, T>(d, Nk, q, k, v, eps, out, KV, ksum, s);
-    case 64: return global_dv<64, T>(d, Nk, q, k, v, eps, out, KV, ksum, s);
-    case 128: return global_dv<128, T>(d, Nk, q, k, v, eps, out, KV, ksum, s);
+    case 16: return global_dv<16, T>(d, Nk, q, k, v, kpm, eps, out, KV, ksum, s);
+    case 32: return global_dv<32, T>(d, Nk, q, k, v, kpm, eps, out, KV, ksum, s);
+    case 64: return global_dv<64, T>(d, Nk, q, k, v, kpm, eps, out, KV, ksum, s);
+    case 128: return global_dv<128, T>(d, Nk, q, k, v, kpm, eps, out, KV, ksum, s);
   }
   return LINATTN_ERR_UNSUPPORTED;
 }
@@ -529,18 +626,34 @@ int fwd_causal_impl(const linattn_dims *d, const void *q, const void *k, const v
     }
     return LINATTN_OK;
   }
-  if (use_tc_causal(d))
+  const CausalPath path = causal_path(d);
+  if (path == CausalPath::kPairedTc)
     return launch_causal_tc(d, q, k, v, lambda, eps, S_init, z_init, out, S_final, z_final, s);
   // the segment-parallel form when it pays and the workspace holds it
-  Segments sg = plan_segments(d);
-  const size_t need = segment_bytes(d, sg);
-  if (sg.G > 1 && ws && ws_bytes >= need) {
+  auto ws_ok = [&](size_t need) -> int {
     if (!aligned16(ws)) return LINATTN_ERR_INVALID;
     if (overlaps(ws, need, q, nq) || overlaps(ws, need, k, nq) || overlaps(ws, need, v, nv) ||
         overlaps(ws, need, out, nv) || overlaps(ws, need, S_final, nS) ||
         overlaps(ws, need, z_final, nz) || overlaps(ws, need, S_init, nS) ||
         overlaps(ws, need, z_init, nz))
       return LINATTN_ERR_INVALID;
+    return LINATTN_OK;
+  };
+  if (path == CausalPath::kSegTc) {
+    TcSegments tsg = plan_tc_segments(d);
+    const size_t need = tc_segment_bytes(d, tsg);
+    if (tsg.G > 1 && ws && ws_bytes >= need) {
+      if ((rc = ws_ok(need)) != LINATTN_OK) return rc;
+    } else {
+      tsg = TcSegments{1, d->N};
+    }
+    return launch_causal_seg_tc(d, q, k, v, lambda, eps, S_init, z_init, out, S_final, z_final,
+                                tsg, static_cast<float *>(tsg.G > 1 ? ws : nullptr), s);
+  }
+  Segments sg = plan_segments(d);
+  const size_t need = segment_bytes(d, sg);
+  if (sg.G > 1 && ws && ws_bytes >= need) {
+    if ((rc = ws_ok(need)) != LINATTN_OK) return rc;
     sg.ws = static_cast<float *>(ws);
   } else {
     sg = Segments{1, d->N, nullptr};
@@ -557,15 +670,40 @@ int fwd_causal_impl(const linattn_dims *d, const void *q, const void *k, const v
 constexpr size_t kScratchBytes = size_t(16) << 20;
 __device__ __align__(256) unsigned char g_causal_scratch[kScratchBytes];
 
+// The current context, through the driver entry point (nullptr if unknown).
+using CtxGetCurrent = CUresult (*)(CUcontext *);
+CUcontext current_context() {
+  static CtxGetCurrent fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrent>(p);
+  });
+  CUcontext c = nullptr;
+  if (!fn || fn(&c) != CUDA_SUCCESS) return nullptr;
+  return c;
+}
+
+// Looked up once per device and context: a context created anew on the
+// device (after cudaDeviceReset, say) loads the module again, and the array
+// may then sit at another address.
 void *scratch_address() {
   static void *addr[64] = {};
+  static CUcontext ctx[64] = {};
   static std::mutex mu;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
   std::lock_guard<std::mutex> lock(mu);
-  if (!addr[dev] && cudaGetSymbolAddress(&addr[dev], g_causal_scratch) != cudaSuccess)
-    addr[dev] = nullptr;
-  return addr[dev];
+  const CUcontext cur = current_context();
+  if (addr[dev] && cur && ctx[dev] == cur) return addr[dev];
+  void *a = nullptr;
+  if (cudaGetSymbolAddress(&a, g_causal_scratch) != cudaSuccess) a = nullptr;
+  addr[dev] = a;
+  ctx[dev] = current_context();   // the lookup makes the device's context current
+  return a;
 }
 
 }  // namespace
@@ -588,7 +726,22 @@ extern "C" int linattn_fwd_causal_from(const linattn_dims *d, const void *q, con
 
 extern "C" size_t linattn_fwd_causal_workspace(const linattn_dims *d) {
   if (check_dims(d, true) != LINATTN_OK || d->B == 0 || d->H == 0 || d->N == 0) return 0;
+  switch (causal_path(d)) {
+    case CausalPath::kSegTc: return tc_segment_bytes(d, plan_tc_segments(d));
+    case CausalPath::kPairedTc: return 0;
+    case CausalPath::kSimt: break;
+  }
   return segment_bytes(d, plan_segments(d));
+}
+
+extern "C" int linattn_set_kernel_choice(int op, int kernel, int segments) {
+  if (op < LINATTN_OP_CAUSAL || op > LINATTN_OP_PERFORMER) return LINATTN_ERR_INVALID;
+  if (kernel < LINATTN_KERNEL_AUTO || kernel > LINATTN_KERNEL_TC_PAIRED) return LINATTN_ERR_INVALID;
+  if (kernel == LINATTN_KERNEL_TC_PAIRED && op != LINATTN_OP_CAUSAL) return LINATTN_ERR_INVALID;
+  if (segments < 0 || segments > kMaxSegments) return LINATTN_ERR_INVALID;
+  g_choice[op].store(kernel, std::memory_order_relaxed);
+  if (op == LINATTN_OP_CAUSAL) g_forced_segments.store(segments, std::memory_order_relaxed);
+  return LINATTN_OK;
 }
 
 extern "C" int linattn_fwd_causal_ws(const linattn_dims *d, const void *q, const void *k,
@@ -607,6 +760,114 @@ extern "C" int linattn_fwd_causal_noalloc(const linattn_dims *d, const void *q, 
   void *ws = scratch_address();
   return fwd_causal_impl(d, q, k, v, lambda, eps, nullptr, nullptr, out, S_final, z_final, ws,
                          ws ? kScratchBytes : 0, reinterpret_cast<cudaStream_t>(stream));
+}
+
+namespace linattn {
+namespace {
+
+template <int DK, int DVS, typename T>
+int launch_state_simt(const linattn_dims *d, const void *k, const void *v, const float *lam,
+                      float *S, float *z, cudaStream_t s) {
+  const int ctas = d->B * d->H * (d->dv / DVS);
+  causal_seg_state_kernel<DK, DVS, T><<<dim3(ctas, 1), 256, 0, s>>>(
+      static_cast<const T *>(k), static_cast<const T *>(v), lam, S, z, d->H, d->N, d->dv, d->N,
+      1, ident(d));
+  return launch_status();
+}
+
+template <typename T>
+int state_simt_dispatch(const linattn_dims *d, const void *k, const void *v, const float *lam,
+                        float *S, float *z, cudaStream_t s) {
+  const bool narrow = d->dv == 16;
+#define LINATTN_STATE_CASE(DKV)                                                              \
+  case DKV:                                                                                 \
+    return narrow ? launch_state_simt<DKV, 16, T>(d, k, v, lam, S, z, s)                    \
+                  : launch_state_simt<DKV, 32, T>(d, k, v, lam, S, z, s);
+  switch (d->dk) {
+    LINATTN_STATE_CASE(16)
+    LINATTN_STATE_CASE(32)
+    LINATTN_STATE_CASE(64)
+    LINATTN_STATE_CASE(128)
+  }
+#undef LINATTN_STATE_CASE
+  return LINATTN_ERR_UNSUPPORTED;
+}
+
+template <int DKP, int DVP>
+int launch_state_tc(const linattn_dims *d, const CUtensorMap &mk, const CUtensorMap &mv,
+                    const float *lam, float *S, float *z, cudaStream_t s) {
+  auto *sk = stc::causal_seg_state_tc_kernel<DKP, DVP>;
+  if (!set_smem(sk, static_cast<int>(stc::sp::kSmemBytes))) return LINATTN_ERR_CUDA;
+  sk<<<d->B * d->H, stc::sp::NT, stc::sp::kSmemBytes, s>>>(mk, mv, lam, S, z, d->H, d->N, d->N,
+                                                            1, 1, ident(d));
+  return launch_status();
+}
+
+}  // namespace
+}  // namespace linattn
+
+extern "C" int linattn_causal_state(const linattn_dims *d, const void *k, const void *v,
+                                    const float *lambda, float *S, float *z,
+                                    linattn_stream_t stream) {
+  int rc = check_dims(d, true);
+  if (rc != LINATTN_OK) return rc;
+  const size_t BH = static_cast<size_t>(d->B) * d->H;
+  if (BH == 0) return LINATTN_OK;
+  const size_t es = elem_size(d->dtype);
+  const size_t nk = BH * d->N * d->dk * es, nv = BH * d->N * d->dv * es;
+  const size_t nS = BH * d->dk * d->dv * 4, nz = BH * d->dk * 4;
+  if (!S || !z || (d->N > 0 && (!k || !v))) return LINATTN_ERR_INVALID;
+  if (!aligned16(k) || !aligned16(v) || !aligned16(S) || !aligned16(z) || !aligned16(lambda))
+    return LINATTN_ERR_INVALID;
+  if (overlaps(S, nS, k, nk) || overlaps(S, nS, v, nv) || overlaps(z, nz, k, nk) ||
+      overlaps(z, nz, v, nv) || overlaps(S, nS, z, nz))
+    return LINATTN_ERR_INVALID;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (d->N == 0) {
+    if (cudaMemsetAsync(S, 0, nS, s) != cudaSuccess || cudaMemsetAsync(z, 0, nz, s) != cudaSuccess)
+      return LINATTN_ERR_CUDA;
+    return LINATTN_OK;
+  }
+  if (causal_path(d) != CausalPath::kSimt) {
+    const int BHi = d->B * d->H;
+    CUtensorMap mk, mv;
+    if (!make_map_bf16(&mk, k, d->dk, d->N, BHi) || !make_map_bf16(&mv, v, d->dv, d->N, BHi))
+      return LINATTN_ERR_CUDA;
+    if (d->dk == 128)
+      return d->dv == 128 ? launch_state_tc<2, 2>(d, mk, mv, lambda, S, z, s)
+                          : launch_state_tc<2, 1>(d, mk, mv, lambda, S, z, s);
+    return d->dv == 128 ? launch_state_tc<1, 2>(d, mk, mv, lambda, S, z, s)
+                        : launch_state_tc<1, 1>(d, mk, mv, lambda, S, z, s);
+  }
+  if (d->dtype == LINATTN_F32) return state_simt_dispatch<float>(d, k, v, lambda, S, z, s);
+  return state_simt_dispatch<bf16>(d, k, v, lambda, S, z, s);
+}
+
+extern "C" int linattn_combine_states(const linattn_dims *d, int G, const float *lambda,
+                                      const float *S_init, const float *z_init, float *dS,
+                                      float *dz, linattn_stream_t stream) {
+  if (!d || d->B < 0 || d->H < 0 || d->N < 0 || G < 0) return LINATTN_ERR_INVALID;
+  if (!supported_dim(d->dk) || !supported_dim(d->dv)) return LINATTN_ERR_UNSUPPORTED;
+  if (G > kMaxSegments) return LINATTN_ERR_UNSUPPORTED;
+  const size_t BH = static_cast<size_t>(d->B) * d->H;
+  if (BH == 0 || G == 0) return LINATTN_OK;
+  if (static_cast<long long>(BH) * G * d->dk * d->dv >= (1ll << 31)) return LINATTN_ERR_UNSUPPORTED;
+  if ((S_init == nullptr) != (z_init == nullptr) || !dS || !dz) return LINATTN_ERR_INVALID;
+  if (!aligned16(dS) || !aligned16(dz) || !aligned16(S_init) || !aligned16(z_init) ||
+      !aligned16(lambda))
+    return LINATTN_ERR_INVALID;
+  const size_t nS = BH * d->dk * d->dv * 4, nz = BH * d->dk * 4;
+  if (overlaps(dS, G * nS, dz, G * nz) || overlaps(S_init, nS, dS, G * nS) ||
+      overlaps(S_init, nS, dz, G * nz) || overlaps(z_init, nz, dS, G * nS) ||
+      overlaps(z_init, nz, dz, G * nz))
+    return LINATTN_ERR_INVALID;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int eblocks = (d->dk * d->dv + d->dk + 255) / 256;
+  // every segment is N tokens long here: the decay between slots is lambda^N
+  causal_seg_combine_kernel<<<dim3(static_cast<unsigned>(BH), eblocks), 256, 0, s>>>(
+      lambda, S_init, z_init, dS, dz, d->H, d->dk, d->dv, static_cast<long>(G) * d->N, d->N, G,
+      true);
+  return launch_status();
 }
 
 extern "C" int linattn_bwd_causal(const linattn_dims *d, const void *q, const void *k,
@@ -649,7 +910,8 @@ namespace {
 
 // Both global entry points: d->N queries against Nk keys/values.
 int fwd_global_impl(const linattn_dims *d, int Nk, const void *q, const void *k, const void *v,
-                    float eps, void *out, float *KV, float *ksum, cudaStream_t s) {
+                    const uint8_t *kpm, float eps, void *out, float *KV, float *ksum,
+                    cudaStream_t s) {
   int rc = check_dims(d, true);
   if (rc != LINATTN_OK) return rc;
   if (Nk < 0) return LINATTN_ERR_INVALID;
@@ -675,12 +937,16 @@ int fwd_global_impl(const linattn_dims *d, int Nk, const void *q, const void *k,
       overlaps(KV, nS, k, nk) || overlaps(KV, nS, v, nv) || overlaps(KV, nS, q, nq) ||
       overlaps(ksum, nz, q, nq) || overlaps(ksum, nz, k, nk) || overlaps(ksum, nz, v, nv))
     return LINATTN_ERR_INVALID;
+  // the padding mask is read while the outputs are written: no overlap
+  const size_t nm = kpm ? static_cast<size_t>(d->B) * Nk : 0;
+  if (overlaps(kpm, nm, out, ny) || overlaps(kpm, nm, KV, nS) || overlaps(kpm, nm, ksum, nz))
+    return LINATTN_ERR_INVALID;
   if ((rc = zero_kv(KV, nS, ksum, nz, s)) != LINATTN_OK) return rc;
   if (d->N == 0 && Nk == 0) return LINATTN_OK;
-  if (use_tc_global(d)) return launch_global_tc(d, Nk, q, k, v, eps, out, KV, ksum, s);
+  if (use_tc_global(d)) return launch_global_tc(d, Nk, q, k, v, kpm, eps, out, KV, ksum, s);
   if (d->dtype == LINATTN_F32)
-    return global_dispatch<float>(d, Nk, q, k, v, eps, out, KV, ksum, s);
-  return global_dispatch<bf16>(d, Nk, q, k, v, eps, out, KV, ksum, s);
+    return global_dispatch<float>(d, Nk, q, k, v, kpm, eps, out, KV, ksum, s);
+  return global_dispatch<bf16>(d, Nk, q, k, v, kpm, eps, out, KV, ksum, s);
 }
 
 }  // namespace
@@ -689,14 +955,23 @@ int fwd_global_impl(const linattn_dims *d, int Nk, const void *q, const void *k,
 extern "C" int linattn_fwd_global(const linattn_dims *d, const void *q, const void *k,
                                   const void *v, float eps, void *out, float *KV, float *ksum,
                                   linattn_stream_t stream) {
-  return fwd_global_impl(d, d ? d->N : 0, q, k, v, eps, out, KV, ksum,
+  return fwd_global_impl(d, d ? d->N : 0, q, k, v, nullptr, eps, out, KV, ksum,
                          reinterpret_cast<cudaStream_t>(stream));
 }
 
 extern "C" int linattn_fwd_global_cross(const linattn_dims *d, int Nk, const void *q,
                                         const void *k, const void *v, float eps, void *out,
                                         float *KV, float *ksum, linattn_stream_t stream) {
-  return fwd_global_impl(d, Nk, q, k, v, eps, out, KV, ksum,
+  return fwd_global_impl(d, Nk, q, k, v, nullptr, eps, out, KV, ksum,
+                         reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" int linattn_fwd_global_masked(const linattn_dims *d, int Nk, const void *q,
+                                         const void *k, const void *v,
+                                         const unsigned char *key_padding_mask, float eps,
+                                         void *out, float *KV, float *ksum,
+                                         linattn_stream_t stream) {
+  return fwd_global_impl(d, Nk, q, k, v, key_padding_mask, eps, out, KV, ksum,
                          reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -731,10 +1006,10 @@ namespace {
 bool supported_features(int m) { return m == 8 || m == 16 || m == 32 || m == 64; }
 
 // bf16 with d in {64, 128} and m in {32, 64} takes the tensor-core kernel;
-// LINATTN_PERFORMER_KERNEL=simt forces the CUDA-core kernel.
+// LINATTN_KERNEL_CUDA_CORES chosen for the feature map forces the CUDA-core
+// kernel.
 bool use_tc_features(int d, int m, int dtype) {
-  const char *e = std::getenv("LINATTN_PERFORMER_KERNEL");
-  if (e && std::strcmp(e, "simt") == 0) return false;
+  if (choice(LINATTN_OP_PERFORMER) == LINATTN_KERNEL_CUDA_CORES) return false;
   return dtype == LINATTN_BF16 && (d == 64 || d == 128) && (m == 32 || m == 64);
 }
 

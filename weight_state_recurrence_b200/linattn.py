@@ -27,12 +27,15 @@ LINATTN_ERR_CUDA = 3
 LINATTN_ERR_DEVICE = 4
 LINATTN_PHI_ELU1, LINATTN_PHI_IDENTITY = 0, 1
 LINATTN_PERFORMER_SOFTMAX, LINATTN_PERFORMER_GAUSSIAN = 0, 1
+LINATTN_OP_CAUSAL, LINATTN_OP_GLOBAL, LINATTN_OP_PERFORMER = 0, 1, 2
+LINATTN_KERNEL_AUTO, LINATTN_KERNEL_CUDA_CORES, LINATTN_KERNEL_TC_PAIRED = 0, 1, 2
 
 ENTRY_POINTS = ("linattn_fwd_causal", "linattn_fwd_causal_from", "linattn_fwd_causal_workspace",
                 "linattn_fwd_causal_ws", "linattn_fwd_causal_noalloc", "linattn_bwd_causal",
                 "linattn_fwd_global", "linattn_fwd_global_cross", "linattn_decode_step",
                 "linattn_performer_features", "linattn_status_string", "linattn_device_status",
-                "linattn_version")
+                "linattn_version", "linattn_set_kernel_choice", "linattn_causal_state",
+                "linattn_combine_states", "linattn_fwd_global_masked")
 
 
 class linattn_dims(ctypes.Structure):
@@ -95,8 +98,40 @@ def load(build_if_missing: bool = True):
     lib.linattn_device_status.restype = i
     lib.linattn_version.argtypes = []
     lib.linattn_version.restype = i
+    lib.linattn_set_kernel_choice.argtypes = [i, i, i]
+    lib.linattn_set_kernel_choice.restype = i
+    lib.linattn_causal_state.argtypes = [dp, vp, vp, fp, fp, fp, vp]
+    lib.linattn_causal_state.restype = i
+    lib.linattn_combine_states.argtypes = [dp, i, fp, fp, fp, fp, fp, vp]
+    lib.linattn_combine_states.restype = i
+    lib.linattn_fwd_global_masked.argtypes = [dp, i, vp, vp, vp, vp, f, vp, fp, fp, vp]
+    lib.linattn_fwd_global_masked.restype = i
     _lib = lib
     return lib
+
+
+def linattn_set_kernel_choice(op: int, kernel: int, segments: int = 0) -> None:
+    """Choose the kernel family of an operation (tests and benchmarks only;
+    see include/linattn.h)."""
+    _check(load().linattn_set_kernel_choice(int(op), int(kernel), int(segments)),
+           "linattn_set_kernel_choice")
+
+
+class kernel_choice:
+    """Context manager: ``with kernel_choice(LINATTN_OP_CAUSAL,
+    LINATTN_KERNEL_CUDA_CORES): ...`` runs the block with that kernel family
+    and restores the automatic choice afterwards."""
+
+    def __init__(self, op: int, kernel: int, segments: int = 0):
+        self.op, self.kernel, self.segments = op, kernel, segments
+
+    def __enter__(self):
+        linattn_set_kernel_choice(self.op, self.kernel, self.segments)
+        return self
+
+    def __exit__(self, *exc):
+        linattn_set_kernel_choice(self.op, LINATTN_KERNEL_AUTO, 0)
+        return False
 
 
 def status_string(code: int) -> str:
@@ -277,6 +312,31 @@ def linattn_fwd_global_cross(q, k, v, eps, out, KV, ksum, stream=None, *,
                                            _stream(stream)), "linattn_fwd_global_cross")
 
 
+def linattn_fwd_global_masked(q, k, v, key_padding_mask, eps, out, KV, ksum, stream=None, *,
+                              phi=LINATTN_PHI_ELU1):
+    """Cross global forward with a key padding mask [B, Nk] (bool or uint8,
+    nonzero = padding, on the device; None = no padding); the other arguments
+    as linattn_fwd_global_cross."""
+    B, H, Nq, dk = q.shape
+    Nk, dv = k.shape[2], v.shape[-1]
+    if (tuple(k.shape) != (B, H, Nk, dk) or tuple(v.shape) != (B, H, Nk, dv) or
+            tuple(out.shape) != (B, H, Nq, dv)):
+        raise ValueError("shape mismatch among q, k, v, out")
+    if not (q.dtype == k.dtype == v.dtype == out.dtype):
+        raise ValueError("q, k, v, out must share one dtype")
+    _f32(KV, (B, H, dk, dv), "KV")
+    _f32(ksum, (B, H, dk), "ksum")
+    m = key_padding_mask
+    if m is not None:
+        if tuple(m.shape) != (B, Nk) or m.dtype not in (torch.bool, torch.uint8):
+            raise ValueError(f"key_padding_mask must be bool/uint8 with shape {(B, Nk)}")
+        m = m.view(torch.uint8) if m.dtype == torch.bool else m
+    d = linattn_dims(B, H, Nq, dk, dv, _dtype_code(q.dtype), int(phi))
+    _check(load().linattn_fwd_global_masked(ctypes.byref(d), int(Nk), _ptr(q), _ptr(k), _ptr(v),
+                                            _ptr(m), float(eps), _ptr(out), _ptr(KV), _ptr(ksum),
+                                            _stream(stream)), "linattn_fwd_global_masked")
+
+
 def linattn_decode_step(q, k, v, lam, eps, S, z, out, stream=None, *, phi=LINATTN_PHI_ELU1):
     """One decode step: q, k [B,H,dk], v/out [B,H,dv]; S [B,H,dk,dv] and z
     [B,H,dk] fp32 are updated in place."""
@@ -312,6 +372,35 @@ def linattn_performer_features(x, omega, kernel, out, stream=None):
                                              _dtype_code(x.dtype), _ptr(x), _ptr(omega),
                                              _ptr(out), _stream(stream)),
            "linattn_performer_features")
+
+
+def linattn_causal_state(k, v, lam, S, z, stream=None, *, phi=LINATTN_PHI_ELU1):
+    """State-only pass: S [B,H,dk,dv], z [B,H,dk] fp32 (written) from
+    k [B,H,N,dk], v [B,H,N,dv] and lam [H] fp32 or None."""
+    B, H, N, dk = k.shape
+    dv = v.shape[-1]
+    if tuple(v.shape) != (B, H, N, dv) or k.dtype != v.dtype:
+        raise ValueError("k and v must agree in B, H, N and dtype")
+    _f32(lam, (H,), "lambda")
+    _f32(S, (B, H, dk, dv), "S")
+    _f32(z, (B, H, dk), "z")
+    d = linattn_dims(B, H, N, dk, dv, _dtype_code(k.dtype), int(phi))
+    _check(load().linattn_causal_state(ctypes.byref(d), _ptr(k), _ptr(v), _ptr(lam), _ptr(S),
+                                       _ptr(z), _stream(stream)), "linattn_causal_state")
+
+
+def linattn_combine_states(seg_len, lam, S_init, z_init, dS, dz, stream=None):
+    """In place: slots dS [G,B,H,dk,dv], dz [G,B,H,dk] fp32 holding segment
+    states become the states at the start of each segment of seg_len tokens."""
+    G, B, H, dk, dv = dS.shape
+    _f32(dz, (G, B, H, dk), "dz")
+    _f32(lam, (H,), "lambda")
+    _f32(S_init, (B, H, dk, dv), "S_init")
+    _f32(z_init, (B, H, dk), "z_init")
+    d = linattn_dims(B, H, int(seg_len), dk, dv, LINATTN_F32, LINATTN_PHI_ELU1)
+    _check(load().linattn_combine_states(ctypes.byref(d), int(G), _ptr(lam), _ptr(S_init),
+                                         _ptr(z_init), _ptr(dS), _ptr(dz), _stream(stream)),
+           "linattn_combine_states")
 
 
 def linattn_status_string(code: int) -> str:
@@ -366,6 +455,16 @@ def fwd_global_cross(q, k, v, eps=1e-6, stream=None, phi=LINATTN_PHI_ELU1):
     KV = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
     ks = torch.empty((B, H, dk), dtype=torch.float32, device=q.device)
     linattn_fwd_global_cross(q, k, v, eps, out, KV, ks, stream, phi=phi)
+    return out, KV, ks
+
+
+def fwd_global_masked(q, k, v, key_padding_mask, eps=1e-6, stream=None, phi=LINATTN_PHI_ELU1):
+    B, H, Nq, dk = q.shape
+    dv = v.shape[-1]
+    out = torch.empty((B, H, Nq, dv), dtype=v.dtype, device=v.device)
+    KV = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
+    ks = torch.empty((B, H, dk), dtype=torch.float32, device=q.device)
+    linattn_fwd_global_masked(q, k, v, key_padding_mask, eps, out, KV, ks, stream, phi=phi)
     return out, KV, ks
 
 
