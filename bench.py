@@ -384,6 +384,35 @@ def global_leg(lib, args, world, rank, stream, hbm):
     return res
 
 
+def tiny_leg(lib, args, world, rank, stream, hbm):
+    """The tiny_f32 workload (B=1, H=1, N=256, d=32, fp32, no decay) on its
+    kernel (the CUDA-core causal kernel: fp32 inputs).  A single head of 256
+    tokens is latency-bound; the time is reported as the workload asks, with
+    the HBM fraction for completeness."""
+    w = inputs.WORKLOADS["tiny_f32"]
+    B, H, N, d = w.B, w.H, w.N, w.d
+    dev = torch.device("cuda")
+    q, k, v = inputs.qkv((B, H, N, d), (B, H, N, d), w.seed * 1000 + rank, w.scale, w.dtype,
+                         device=dev)
+    out = torch.empty_like(v)
+    S = torch.empty(B, H, d, d, device=dev)
+    z = torch.empty(B, H, d, device=dev)
+
+    def step():
+        lib.linattn_fwd_causal(q, k, v, None, w.eps, out, S, z, stream)
+
+    with torch.cuda.stream(stream):
+        ms = time_steps(step, args.steps, args.warmup, world, stream)
+    per = ms / 1e3 / args.steps
+    alg = causal_bytes(B, H, N, d, d, es=4)
+    return {"workload": "tiny_f32: B=1 x H=1 x N=256, d=32, fp32, no decay",
+            "value": B * N * world / per, "unit": "tokens/s", "ms_per_step": per * 1e3,
+            "kernel": "causal_simt_kernel (fp32)",
+            "roofline": {"bound": "latency", "achieved": alg / per / 1e9, "peak": hbm,
+                         "unit": "GB/s", "frac": alg / per / 1e9 / hbm,
+                         "algorithmic_bytes_per_launch": alg}}
+
+
 def seg_leg(lib, args, world, rank, stream, hbm):
     """The causal_d64 workload (B=2, H=8, N=4096, d=64, bf16, no decay): the
     product path (the tensor-core kernel cut into about one segment per SM,
@@ -626,7 +655,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", dest="cpu", action="store_false")
     ap.add_argument("--only", default="all",
                     choices=["all", "causal", "decode", "global", "backward", "segmented",
-                             "performer"])
+                             "performer", "tiny"])
     ap.add_argument("--batch", type=int, default=0, help="causal leg batch (profiling)")
     ap.add_argument("--dec-batch", type=int, default=0, help="decode sequences (profiling)")
     ap.add_argument("--dec-steps", type=int, default=0, help="decode steps (profiling)")
@@ -642,8 +671,10 @@ def main():
     hbm, tcp, peak_src = peaks()
     stream = torch.cuda.Stream()
 
-    if args.only in ("decode", "global", "backward", "segmented", "performer"):
-        if args.only == "performer":
+    if args.only in ("decode", "global", "backward", "segmented", "performer", "tiny"):
+        if args.only == "tiny":
+            r = tiny_leg(lib, args, world, rank, stream, hbm)
+        elif args.only == "performer":
             r = performer_leg(lib, args, world, rank, stream, hbm)
         elif args.only == "backward":
             r = bwd_leg(lib, args, world, rank, stream, ALU_PEAK_TFLOPS)
@@ -685,6 +716,7 @@ def main():
         line["backward"] = bwd_leg(lib, args, world, rank, stream, ALU_PEAK_TFLOPS)
         line["segmented"] = seg_leg(lib, args, world, rank, stream, hbm)
         line["performer"] = performer_leg(lib, args, world, rank, stream, hbm)
+        line["tiny"] = tiny_leg(lib, args, world, rank, stream, hbm)
     if args.cpu and world == 1 and rank == 0:
         tok_s, cores, desc, _ = oracle_sample()
         line["cpu_baseline"] = {"value": tok_s, "unit": "tokens/s", "cores": cores,

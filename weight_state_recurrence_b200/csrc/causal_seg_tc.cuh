@@ -24,26 +24,31 @@
 //   intra   D_O  += P V              (P = bf16 in TMEM)   TMEM x SMEM
 // One accumulator takes both halves of the numerator.  The denominator is
 // formed in fp32 on the CUDA cores: the feature-map warps keep z and take
-// phi(q_t).z while they transform q; the score epilogue adds the row sums of
-// the bf16 P tile (the weights the numerator uses).
+// phi(q_t).z while they transform q; the score epilogue adds the fp32 row sums
+// of the masked score tile (the numerator uses the same weights rounded to
+// bf16, a relative difference below 2^-9).
 //
-// Decay.  For lambda >= kFactorMin the decay is factored into the operands:
-// phi(q_t) is scaled by lambda^(t+1-Cv) and phi(k_s) by lambda^(Cv-1-s)
-// while the feature map is applied, so the score MMA yields lambda^(t-s)
-// phi(q_t).phi(k_s), the state MMA gets its weights, and the carried term
-// needs the state scaled once by lambda^Cv (the state warps write the bf16
-// operand as lambda^Cv S).  Smaller lambda (down to 0): the score epilogue
-// multiplies by lambda^(t-s), and after the score MMA has read them the q
-// rows are rescaled by lambda^(t+1) and the k rows by lambda^(Cv-1-s).
+// Decay.  For lambda >= kFactorMin the decay is factored into the operands
+// relative to a frame of R chunks that starts at token n_f: the q row of
+// token p is scaled by lambda^(p+1-n_f) and the k row by lambda^(n_f-1-p)
+// while the feature map is applied.  The score MMA then yields lambda^(t-s)
+// phi(q_t).phi(k_s), the state MMA accumulates S~ = lambda^-(n-n_f) S with
+// no decay between chunks, and phi(q') S~ is the carried term itself; the
+// state warps only convert S~ to the bf16 operand, and once per frame
+// multiply it by lambda^(R C) (frame_chunks bounds the weights).  Smaller
+// lambda (down to 0): the score epilogue multiplies by lambda^(t-s), after
+// the score MMA has read them the q rows are rescaled by lambda^(t+1) and the
+// k rows by lambda^(Cv-1-s), and the state is decayed by lambda^Cv before
+// every state MMA.
 //
-// Warp roles (768 threads):
+// Warp roles (1024 threads):
 //   warp 0      TMA producer of the q and k tiles
 //   warp 1      TMEM owner, the single MMA-issuing thread
 //   warp 2      TMA producer of the v tiles
 //   warps 4-7   score epilogue: D_A -> mask (and decay) -> bf16 P in TMEM, row sums
 //   warps 8-11  output: y = D_O / den -> global memory
-//   warps 12-15 state: D_S -> bf16 operand S' and D_S <- lambda^Cv D_S
-//   warps 16-23 feature map (in place, packed bf16x2), phi(q).z, z update
+//   warps 12-15 state: D_S -> bf16 operand S' (and the decay or renormalisation of D_S)
+//   warps 16-31 feature map (in place, packed bf16x2), phi(q).z, z update
 // Every wait is bounded (sm100.cuh); a wait that runs out records an error
 // flag and every role leaves its loop.
 #pragma once
@@ -59,8 +64,8 @@ using tc::pack_bf16;
 using tc::phi_bf16x2;
 
 constexpr int C = 128;
-constexpr int NT = 768;
-constexpr int kPhiThreads = 256;
+constexpr int NT = 1024;
+constexpr int kPhiThreads = 512;
 constexpr int kBarPhi = 1, kBarP = 2, kBarOut = 3, kBarState = 4;   // named barriers
 constexpr float kFactorMin = 0.7f;
 
@@ -74,15 +79,19 @@ constexpr uint32_t kOffMisc = kOffSop + 2 * kPanel;
 constexpr uint32_t kMiscTmem = 256, kMiscAbort = 260, kMiscRoleFail = 272;
 constexpr uint32_t kMiscPw = 320;               // lambda^i, i = 0..C        (129 floats)
 constexpr uint32_t kMiscZ = 848;                // z, fp32                   (128 floats)
-constexpr uint32_t kMiscDen = 1360;             // den[2][128]: phi(q).z + row sum of P
-constexpr uint32_t kMiscBytes = kMiscDen + 2 * 128 * 4;
+constexpr uint32_t kMiscDen = 1360;             // den[3][128]: phi(q).z + row sum of P
+constexpr int kDenBufs = 3;
+constexpr uint32_t kMiscBytes = kMiscDen + kDenBufs * 128 * 4;
 constexpr uint32_t kSmemBytes = kOffMisc + kMiscBytes;
 static_assert(kSmemBytes <= 232448, "exceeds the per-CTA shared memory of sm_100");
 
 enum Bar {
   kFullQK0 = 0, kFullQK1, kFullV0, kFullV1, kFreeQK0, kFreeQK1, kFreeV0, kFreeV1,
   kPhi0, kPhi1, kScore, kRescale, kState, kReadout, kPDone, kO0, kO1, kOut0, kOut1,
-  kDen0, kDen1, kFinal, kNumBars
+  kSop,
+  // den buffer b (chunk c uses b = c % 3): phi(q).z written, row sums added, read by the output
+  kDenQz0, kDenQz1, kDenQz2, kDenRs0, kDenRs1, kDenRs2, kDenFree0, kDenFree1, kDenFree2,
+  kFinal, kNumBars
 };
 static_assert(kNumBars * 8 <= 256, "barrier area overflow");
 
@@ -95,9 +104,50 @@ constexpr uint32_t kTmCols = 512;
 __device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
+// Sums of 8 values over the 32 lanes of a warp in 9 shuffles: each round
+// keeps half of the values and trades the other half with the partner lane.
+// Lane L ends with the full sum of value ((L >> 4) & 1) * 4 + ((L >> 3) & 1) * 2
+// + ((L >> 2) & 1); lanes that differ only in bits 0-1 hold the same sum.
+__device__ __forceinline__ float warp_sum8_transposed(const float (&v)[8], int lane) {
+  float a[4], b[2];
+  const bool h16 = lane & 16, h8 = lane & 8, h4 = lane & 4;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float send = h16 ? v[i] : v[4 + i];
+    a[i] = (h16 ? v[4 + i] : v[i]) + __shfl_xor_sync(0xffffffffu, send, 16);
+  }
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const float send = h8 ? a[i] : a[2 + i];
+    b[i] = (h8 ? a[2 + i] : a[i]) + __shfl_xor_sync(0xffffffffu, send, 8);
+  }
+  const float send = h4 ? b[0] : b[1];
+  float c = (h4 ? b[1] : b[0]) + __shfl_xor_sync(0xffffffffu, send, 4);
+  c += __shfl_xor_sync(0xffffffffu, c, 2);
+  c += __shfl_xor_sync(0xffffffffu, c, 1);
+  return c;
+}
+__device__ __forceinline__ int warp_sum8_index(int lane) {
+  return ((lane >> 4) & 1) * 4 + ((lane >> 3) & 1) * 2 + ((lane >> 2) & 1);
+}
+
 // byte offset of 16-byte chunk j (0..15) of row `row` in a 2-panel K-major tile
 __device__ __forceinline__ uint32_t chunk_off(uint32_t row, uint32_t j) {
   return (j >> 3) * kPanel + sw128_offset(row, (j & 7) * 16);
+}
+
+// Chunks per frame of the factored decay.  Inside a frame that starts at
+// token n_f, the TMEM state is S~ = lambda^-(n - n_f) S (n = tokens seen), the
+// k row of token p carries lambda^(n_f - 1 - p) and the q row lambda^(p + 1 -
+// n_f), so the state MMA accumulates onto S~ with no decay between chunks
+// and the carried term phi(q') S~ is already lambda^(t+1) phi(q) S.  The
+// weights stay within 2^+-64 (one chunk at lambda = kFactorMin reaches
+// 2^66), so the frame spans at most 64 / (C log2(1/lambda)) chunks; at its end
+// the state is multiplied by lambda^(R C) once (a renormalisation).
+__device__ __forceinline__ int frame_chunks(float L) {
+  if (L >= 1.f) return 1 << 30;
+  const float f = 64.f / (static_cast<float>(C) * -log2f(L));
+  return f >= static_cast<float>(1 << 20) ? (1 << 20) : max(1, static_cast<int>(f));
 }
 
 template <int DKP, int DVP>
@@ -131,10 +181,16 @@ __global__ void __launch_bounds__(NT, 1)
   const int nchunks = (n1 - n0 + C - 1) / C;
   const int Ct = (n1 - n0) - (nchunks - 1) * C;   // valid tokens of the last chunk
   const bool last_seg = g == G - 1;
-  const float *S0 = g == 0 ? S_init : ws_S + (pair * G + g) * static_cast<long>(DK) * DV;
-  const float *z0 = g == 0 ? z_init : ws_z + (pair * G + g) * static_cast<long>(DK);
+  // this head's starting state: the caller's (first segment) or the scanned
+  // carry of slot g of the workspace
+  const float *S0 = g == 0 ? (S_init ? S_init + pair * DK * static_cast<long>(DV) : nullptr)
+                           : ws_S + (pair * G + g) * static_cast<long>(DK) * DV;
+  const float *z0 = g == 0 ? (z_init ? z_init + pair * static_cast<long>(DK) : nullptr)
+                           : ws_z + (pair * G + g) * static_cast<long>(DK);
   const bool has_init = S0 != nullptr;
   const bool factored = L >= kFactorMin;
+  // factored decay keeps the state in a frame of R chunks (see frame_chunks)
+  const int R = factored ? frame_chunks(L) : 1;
 
   uint8_t *misc = sm + kOffMisc;
   auto bar = [&](int i) { return sb + kOffMisc + 8u * static_cast<uint32_t>(i); };
@@ -161,7 +217,7 @@ __global__ void __launch_bounds__(NT, 1)
     tmem_relinquish();
   }
   if (tid <= C) pw[tid] = pow_int(L, tid);
-  if (tid < 128) zs[tid] = (z0 && tid < DK) ? z0[pair * DK + tid] : 0.f;
+  if (tid < 128) zs[tid] = (z0 && tid < DK) ? z0[tid] : 0.f;
   if (DKP == 1) {
     // the second d_k panel of the q and k tiles stays zero (the state MMA
     // reads it as rows 64-127 of phi(K)^T; the other chains never do)
@@ -230,15 +286,10 @@ __global__ void __launch_bounds__(NT, 1)
       // descriptors of every operand tile, per stage; a K step adds its byte
       // offset >> 4 to the start-address field (tiles stay below 256 KB, so
       // the 14-bit field never carries)
-      uint64_t dQ[2], dK[2], dKmn[2], dV[2];
-#pragma unroll
-      for (int s = 0; s < 2; ++s) {
-        const uint32_t st = sb + s * kStage;
-        dQ[s] = sdesc_sw128(st + kOffQ, 16, 1024);
-        dK[s] = sdesc_sw128(st + kOffK, 16, 1024);
-        dKmn[s] = sdesc_sw128(st + kOffK, kPanel, 1024);
-        dV[s] = sdesc_sw128(st + kOffV, kPanel, 1024);
-      }
+      const uint64_t dQ = sdesc_sw128(sb + kOffQ, 16, 1024);
+      const uint64_t dK = sdesc_sw128(sb + kOffK, 16, 1024);
+      const uint64_t dKmn = sdesc_sw128(sb + kOffK, kPanel, 1024);
+      const uint64_t dV = sdesc_sw128(sb + kOffV, kPanel, 1024);
       const uint64_t dSop = sdesc_sw128(sb + kOffSop, kPanel, 1024);
       auto kofs = [](int ks) -> uint64_t { return ((ks >> 2) * kPanel + (ks & 3) * 32) >> 4; };
       bool ok = true;
@@ -249,7 +300,8 @@ __global__ void __launch_bounds__(NT, 1)
         // before, has read D_A: the chains run in issue order)
         if (!mbar_wait(bar(kPhi0 + s), (c >> 1) & 1)) { ok = false; break; }
         tc_fence_after();
-        const uint64_t q0 = dQ[s], k0 = dK[s], kmn0 = dKmn[s], v0 = dV[s];
+        const uint64_t so = static_cast<uint64_t>(s) * (kStage >> 4);   // stage offset
+        const uint64_t q0 = dQ + so, k0 = dK + so, kmn0 = dKmn + so, v0 = dV + so;
 #pragma unroll
         for (int ks = 0; ks < 4 * DKP; ++ks)
           umma_bf16(tmem + kTmA, q0 + kofs(ks), k0 + kofs(ks), idA, ks > 0);
@@ -257,9 +309,8 @@ __global__ void __launch_bounds__(NT, 1)
         // explicit decay: the q and k rows are rescaled once the score MMA has read them
         if (!factored && !mbar_wait(bar(kRescale), c & 1)) { ok = false; break; }
         // carried: D_O[s] = phi(Q) S'  (state before this chunk; D_O[s] drained)
-        if (!mbar_wait(bar(kReadout), c & 1) ||
-            (c >= 2 && !mbar_wait(bar(kOut0 + s), ((c - 2) >> 1) & 1)) ||
-            !mbar_wait(bar(kFullV0 + s), (c >> 1) & 1)) {
+        if (!mbar_wait(bar(kSop), c & 1) ||
+            (c >= 2 && !mbar_wait(bar(kOut0 + s), ((c - 2) >> 1) & 1))) {
           ok = false;
           break;
         }
@@ -272,6 +323,11 @@ __global__ void __launch_bounds__(NT, 1)
             umma_bf16(dO, q0 + kofs(ks), dSop + ks * (2048 >> 4), idQS, ks > 0);
         }
         // state: D_S += (Lk phi(K))^T V   (onto the state decayed by lambda^Cv)
+        if (!mbar_wait(bar(kReadout), c & 1) || !mbar_wait(bar(kFullV0 + s), (c >> 1) & 1)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
 #pragma unroll
         for (int ks = 0; ks < C / 16; ++ks)
           umma_bf16(tmem + kTmS, kmn0 + ks * (2048 >> 4), v0 + ks * (2048 >> 4), idS,
@@ -301,18 +357,18 @@ __global__ void __launch_bounds__(NT, 1)
     volatile int &rf = role_fail[0];
     for (int c = 0; c < nchunks; ++c) {
       const int s = c & 1;
-      // kPhi[s] (already complete) orders the feature-map warps' phi(q).z
-      // before this role's update of den[s]
+      // kDenQz orders the feature-map warps' phi(q).z before this role's
+      // update of the chunk's den buffer
       if (*abort_flag || !mbar_wait(bar(kScore), c & 1) ||
-          !mbar_wait(bar(kPhi0 + s), (c >> 1) & 1)) {
+          !mbar_wait(bar(kDenQz0 + c % kDenBufs), (c / kDenBufs) & 1)) {
         rf = 1;
         fail();
       }
       tc_fence_after();
       float rs = 0.f;
       if (!rf) {
-        // blocks of 32 keys; only blocks 0..wq hold s <= t
-#pragma unroll
+        // blocks of 32 keys, one load each; only blocks 0..wq hold s <= t
+#pragma unroll 1
         for (int bk = 0; bk < 4; ++bk) {
           uint32_t pk[16];
           if (bk <= wq) {
@@ -320,17 +376,27 @@ __global__ void __launch_bounds__(NT, 1)
             tmem_ld_32x32b_x32(tmem + lf + kTmA + bk * 32, r);
             tmem_wait_ld();
             const int s0 = bk * 32;
+            if (factored && bk < wq) {
+              // below the diagonal block: every key s <= t, no mask
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const int s_a = s0 + 2 * i, s_b = s_a + 1;
-              float a = s_a <= t ? __uint_as_float(r[2 * i]) : 0.f;
-              float b = s_b <= t ? __uint_as_float(r[2 * i + 1]) : 0.f;
-              if (!factored) {
-                a *= s_a <= t ? pw[t - s_a] : 0.f;
-                b *= s_b <= t ? pw[t - s_b] : 0.f;
+              for (int i = 0; i < 16; ++i) {
+                const float a = __uint_as_float(r[2 * i]), b = __uint_as_float(r[2 * i + 1]);
+                pk[i] = pack_bf16(a, b);
+                rs += a + b;
               }
-              pk[i] = pack_bf16(a, b);
-              rs += bf_lo(pk[i]) + bf_hi(pk[i]);
+            } else {
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                const int s_a = s0 + 2 * i, s_b = s_a + 1;
+                float a = s_a <= t ? __uint_as_float(r[2 * i]) : 0.f;
+                float b = s_b <= t ? __uint_as_float(r[2 * i + 1]) : 0.f;
+                if (!factored) {
+                  a *= s_a <= t ? pw[t - s_a] : 0.f;
+                  b *= s_b <= t ? pw[t - s_b] : 0.f;
+                }
+                pk[i] = pack_bf16(a, b);
+                rs += a + b;
+              }
             }
           } else {
 #pragma unroll
@@ -341,14 +407,14 @@ __global__ void __launch_bounds__(NT, 1)
           tmem_st_32x32b_x16(tmem + lf + kTmA + bk * 16, pk);
         }
         tmem_wait_st();
-        den[s * 128 + t] += rs;   // phi(q).z was written there by the feature-map warps
+        den[(c % kDenBufs) * 128 + t] += rs;   // phi(q).z was written there by the feature-map warps
       }
       tc_fence_before();
       named_bar_sync(kBarP, 128);
       if (rf) break;
       if (t == 0) {
         mbar_arrive(bar(kPDone));
-        mbar_arrive(bar(kDen0 + s));
+        mbar_arrive(bar(kDenRs0 + c % kDenBufs));
       }
     }
   } else if (warp >= 8 && warp < 12) {
@@ -360,17 +426,17 @@ __global__ void __launch_bounds__(NT, 1)
     for (int c = 0; c < nchunks; ++c) {
       const int s = c & 1;
       if (*abort_flag || !mbar_wait(bar(kO0 + s), (c >> 1) & 1) ||
-          !mbar_wait(bar(kDen0 + s), (c >> 1) & 1)) {
+          !mbar_wait(bar(kDenRs0 + c % kDenBufs), (c / kDenBufs) & 1)) {
         rf = 1;
         fail();
       }
       tc_fence_after();
       if (!rf) {
-        const float inv = 1.f / (den[s * 128 + t] + eps);
+        const float inv = 1.f / (den[(c % kDenBufs) * 128 + t] + eps);
         const bool live = t < Cv_of(c);
         uint4 *dst = reinterpret_cast<uint4 *>(
             out + (pair * N + n0 + static_cast<long>(c) * C + (live ? t : 0)) * DV);
-#pragma unroll
+#pragma unroll 1
         for (int blk = 0; blk < DV / 32; ++blk) {
           uint32_t r[32];
           tmem_ld_32x32b_x32(tmem + lf + kTmO + s * 128 + blk * 32, r);
@@ -389,7 +455,10 @@ __global__ void __launch_bounds__(NT, 1)
       tc_fence_before();
       named_bar_sync(kBarOut, 128);
       if (rf) break;
-      if (t == 0) mbar_arrive(bar(kOut0 + s));
+      if (t == 0) {
+        mbar_arrive(bar(kOut0 + s));
+        mbar_arrive(bar(kDenFree0 + c % kDenBufs));
+      }
     }
   } else if (warp >= 12 && warp < 16) {
     // ------------------------------------- state: operand S' and decay
@@ -399,46 +468,53 @@ __global__ void __launch_bounds__(NT, 1)
     const uint32_t lf = static_cast<uint32_t>(wq * 32) << 16;
     volatile int &rf = role_fail[2];
     // bf16 row of the MN-major operand (row = d_k, 64 d_v per panel)
-    auto put_op = [&](int blk, const uint32_t (&v32)[32], float f) {
-      uint32_t pk[16];
+    // 16 columns (block blk) of this d_k row as bf16 into the operand
+    auto put_op = [&](int blk, const uint32_t (&v16)[16], float f) {
+      uint32_t pk[8];
 #pragma unroll
-      for (int i = 0; i < 16; ++i)
-        pk[i] = pack_bf16(__uint_as_float(v32[2 * i]) * f, __uint_as_float(v32[2 * i + 1]) * f);
-      const uint32_t col = blk * 32;     // first d_v column of this block
+      for (int i = 0; i < 8; ++i)
+        pk[i] = pack_bf16(__uint_as_float(v16[2 * i]) * f, __uint_as_float(v16[2 * i + 1]) * f);
+      const uint32_t col = blk * 16;     // first d_v column of this block
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
+      for (int i = 0; i < 2; ++i)
         *reinterpret_cast<uint4 *>(sm + kOffSop + (col >> 6) * kPanel +
                                    sw128_offset(r, (col & 63) * 2 + i * 16)) =
             make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
     };
-    // starting state: D_S = lambda^Cv0 S0, operand = S0 scaled as the carried term wants
+    // starting state, operand S' = S0.  Explicit decay: D_S = lambda^Cv0 S0
+    // (the state MMA adds chunk 0 onto the decayed state); factored: D_S = S0,
+    // the first frame starting at the segment's first token.
     if (has_init && nchunks > 0) {
-      const float g0 = pw[Cv_of(0)];
-      const float fop = factored ? g0 : 1.f;
-      const float *src = S0 + (pair * DK + (live ? r : 0)) * static_cast<long>(DV);
+      const float g0 = factored ? 1.f : pw[Cv_of(0)];
+      const float *src = S0 + (live ? r : 0) * static_cast<long>(DV);
+#pragma unroll 1
+      for (int blk = 0; blk < DV / 16; ++blk) {
+        uint32_t v16[16], sv[16];
 #pragma unroll
-      for (int blk = 0; blk < DV / 32; ++blk) {
-        uint32_t v32[32], sv[32];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const float4 f = live ? reinterpret_cast<const float4 *>(src)[blk * 8 + i]
+        for (int i = 0; i < 4; ++i) {
+          const float4 f = live ? reinterpret_cast<const float4 *>(src)[blk * 4 + i]
                                 : make_float4(0.f, 0.f, 0.f, 0.f);
-          v32[4 * i] = __float_as_uint(f.x);
-          v32[4 * i + 1] = __float_as_uint(f.y);
-          v32[4 * i + 2] = __float_as_uint(f.z);
-          v32[4 * i + 3] = __float_as_uint(f.w);
+          v16[4 * i] = __float_as_uint(f.x);
+          v16[4 * i + 1] = __float_as_uint(f.y);
+          v16[4 * i + 2] = __float_as_uint(f.z);
+          v16[4 * i + 3] = __float_as_uint(f.w);
         }
 #pragma unroll
-        for (int i = 0; i < 32; ++i) sv[i] = __float_as_uint(__uint_as_float(v32[i]) * g0);
-        tmem_st_32x32b_x32(tmem + lf + kTmS + blk * 32, sv);
-        put_op(blk, v32, fop);
+        for (int i = 0; i < 16; ++i) sv[i] = __float_as_uint(__uint_as_float(v16[i]) * g0);
+        tmem_st_32x32b_x16(tmem + lf + kTmS + blk * 16, sv);
+        put_op(blk, v16, 1.f);
       }
       tmem_wait_st();
     }
     fence_proxy_async_smem();
     tc_fence_before();
     named_bar_sync(kBarState, 128);
-    if (r == 0) mbar_arrive(bar(kReadout));
+    if (r == 0) {
+      mbar_arrive(bar(kSop));
+      mbar_arrive(bar(kReadout));
+    }
+    // lambda^(R C): the renormalisation at the end of a frame (factored)
+    const float gR = factored && R < nchunks ? pow_int(L, R * C) : 1.f;
     for (int c = 0; c < nchunks; ++c) {
       const bool last = c == nchunks - 1;
       if (*abort_flag || !mbar_wait(bar(kState), c & 1)) {
@@ -446,40 +522,76 @@ __global__ void __launch_bounds__(NT, 1)
         fail();
       }
       tc_fence_after();
-      if (!rf) {
-        const float gn = last ? 1.f : pw[Cv_of(c + 1)];
-        const float fop = factored ? gn : 1.f;
-#pragma unroll
-        for (int blk = 0; blk < DV / 32; ++blk) {
-          uint32_t sv[32];
-          tmem_ld_32x32b_x32(tmem + lf + kTmS + blk * 32, sv);
+      if (!rf && last && last_seg && S_final) {
+        // factored: S = lambda^(tokens since the frame start) S~
+        const float fin = factored ? pow_int(pw[C], c % R) * pw[Cv_of(c)] : 1.f;
+#pragma unroll 1
+        for (int blk = 0; blk < DV / 16; ++blk) {
+          uint32_t sv[16];
+          tmem_ld_32x32b_x16(tmem + lf + kTmS + blk * 16, sv);   // warp-wide load
           tmem_wait_ld();
-          if (last) {
-            if (last_seg && S_final && live) {
-              float4 *dst = reinterpret_cast<float4 *>(S_final + (pair * DK + r) * DV) + blk * 8;
+          if (live) {
+            float4 *dst = reinterpret_cast<float4 *>(S_final + (pair * DK + r) * DV) + blk * 4;
 #pragma unroll
-              for (int i = 0; i < 8; ++i)
-                dst[i] = make_float4(__uint_as_float(sv[4 * i]), __uint_as_float(sv[4 * i + 1]),
-                                     __uint_as_float(sv[4 * i + 2]), __uint_as_float(sv[4 * i + 3]));
-            }
-          } else {
-            put_op(blk, sv, fop);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) sv[i] = __float_as_uint(__uint_as_float(sv[i]) * gn);
-            tmem_st_32x32b_x32(tmem + lf + kTmS + blk * 32, sv);
+            for (int i = 0; i < 4; ++i)
+              dst[i] = make_float4(__uint_as_float(sv[4 * i]) * fin,
+                                   __uint_as_float(sv[4 * i + 1]) * fin,
+                                   __uint_as_float(sv[4 * i + 2]) * fin,
+                                   __uint_as_float(sv[4 * i + 3]) * fin);
           }
         }
-        if (!last) tmem_wait_st();
+      }
+      // explicit decay: D_S <- lambda^Cv(next) D_S before every state MMA, the
+      // operand unscaled; factored: only at the end of a frame, operand and
+      // D_S both renormalised
+      const bool decay = !last && (!factored || (c + 1) % R == 0);
+      const float gd = factored ? gR : (last ? 1.f : pw[Cv_of(c + 1)]);
+      const float fop = factored && decay ? gR : 1.f;
+      if (!rf && !last) {
+        // (1) the bf16 operand of the next chunk's carried product
+#pragma unroll 1
+        for (int blk = 0; blk < DV / 16; ++blk) {
+          uint32_t sv[16];
+          tmem_ld_32x32b_x16(tmem + lf + kTmS + blk * 16, sv);
+          tmem_wait_ld();
+          put_op(blk, sv, fop);
+        }
       }
       fence_proxy_async_smem();
-      tc_fence_before();
-      named_bar_sync(kBarState, 128);
-      if (rf) break;
-      if (r == 0 && !last) mbar_arrive(bar(kReadout));
+      if (decay) {
+        named_bar_sync(kBarState, 128);
+        if (rf) break;
+        if (r == 0) mbar_arrive(bar(kSop));
+        if (!rf) {
+          // (2) D_S <- gd D_S, before the next state MMA accumulates onto it
+#pragma unroll 1
+          for (int blk = 0; blk < DV / 16; ++blk) {
+            uint32_t sv[16];
+            tmem_ld_32x32b_x16(tmem + lf + kTmS + blk * 16, sv);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) sv[i] = __float_as_uint(__uint_as_float(sv[i]) * gd);
+            tmem_st_32x32b_x16(tmem + lf + kTmS + blk * 16, sv);
+          }
+          tmem_wait_st();
+        }
+        tc_fence_before();
+        named_bar_sync(kBarState, 128);
+        if (rf) break;
+        if (r == 0) mbar_arrive(bar(kReadout));
+      } else {
+        tc_fence_before();
+        named_bar_sync(kBarState, 128);
+        if (rf) break;
+        if (r == 0 && !last) {
+          mbar_arrive(bar(kSop));
+          mbar_arrive(bar(kReadout));
+        }
+      }
     }
   } else if (warp >= 16) {
     // -------------------------------------------------------- feature map
-    const int tt = tid - 512;                 // 0..255
+    const int tt = tid - 512;                 // 0..511
     volatile int &rf = role_fail[3];
     auto check = [&](bool ok_wait) {
       if (!ok_wait || *abort_flag) {
@@ -487,44 +599,64 @@ __global__ void __launch_bounds__(NT, 1)
         fail();
       }
     };
-    // q: thread (row tq, half hq of the row's 16-byte chunks)
-    const int tq = tt >> 1, hq = tt & 1;
-    constexpr int QCH = KCH / 2;
-    // k: thread (column group cg of 8 columns, row block rb)
+    const int fw = tt >> 5;                   // feature-map warp 0..15
+    // q: thread (row tq, quarter qq of the row's 16-byte chunks): a warp holds
+    // 8 rows x 4 quarters; at step j quarter qq takes chunk (j + qq) of its
+    // quarter, so the tile accesses and the reads of z spread over all banks.
+    // The quarters of a row meet by shuffles.
+    constexpr int QCH = KCH / 4;              // chunks per thread (4 or 2)
+    const int tq = fw * 8 + (lane & 7), qq = lane >> 3;
+    // k: a warp owns one column group of 8 columns over all 128 rows, so the
+    // column sums of z need no atomics; with d_k = 64 (8 groups) only the
+    // first 8 warps take k
     constexpr int NCG = KCH;                  // 16 or 8 column groups
-    constexpr int RPB = NCG / 2;              // rows per row block (8 or 4)
-    const int cg = tt % NCG, rb = tt / NCG;
+    constexpr int RPL = 128 / 32;             // rows per lane
+    const bool kwarp = fw < NCG;
+    const int cg = fw;
+    float ztot = 0.f;                         // this lane's share of the column sums
+    const int zcol = cg * 8 + warp_sum8_index(lane);
+    const bool zowner = kwarp && (lane & 3) == 0;
+    // factored: lambda^(tokens from the frame start to this chunk); explicit: unused
+    float Eq = 1.f;
+    const float gR = factored && R < nchunks ? pow_int(L, R * C) : 1.f;
     for (int c = 0; c < nchunks; ++c) {
       const int s = c & 1;
       const int Cv = Cv_of(c);
       uint8_t *st = sm + s * kStage;
+      const bool frame_start = c % R == 0;
+      if (factored) Eq = frame_start ? 1.f : Eq * pw[C];
+      // the previous chunk's column sums: explicit z_{c-1} = lambda^Cv z_{c-2} + sums;
+      // factored z~ += sums, renormalised with the state when a frame starts
+      if (c > 0 && zowner)
+        zs[zcol] = factored ? (frame_start ? gR : 1.f) * (zs[zcol] + ztot)
+                            : pw[Cv_of(c - 1)] * zs[zcol] + ztot;
       if (tt == 0) {
         check(mbar_wait(bar(kFullQK0 + s), (c >> 1) & 1));
-        // den[s] was read by the output of chunk c - 2
-        if (c >= 2) check(mbar_wait(bar(kOut0 + s), ((c - 2) >> 1) & 1));
+        // den[c % 3] was read by the output of chunk c - 3
+        if (c >= kDenBufs)
+          check(mbar_wait(bar(kDenFree0 + c % kDenBufs), ((c - kDenBufs) / kDenBufs) & 1));
       }
       named_bar_sync(kBarPhi, kPhiThreads);
       if (rf) break;
-      const float gC = pw[Cv];
-      // (1) factored: the carried term reads lambda^Cv z; scale z first
-      if (factored && tt < 128) zs[tt] *= gC;
-      named_bar_sync(kBarPhi, kPhiThreads);
-      // (2) q rows: feature map, decay scale, phi(q).z
+      // (1) q rows: feature map, decay scale, phi(q).z_{c-1}
       {
         float fq;
         if (tq >= Cv) fq = 0.f;
-        else fq = factored ? 1.f / pw[Cv - 1 - tq] : 1.f;
+        else fq = factored ? Eq * pw[tq + 1] : 1.f;
         const uint32_t f2 = pack_bf16(fq, fq);
         float qz = 0.f;
         uint4 w[QCH];
+        int ch[QCH];
 #pragma unroll
-        for (int j = 0; j < QCH; ++j)
-          w[j] = *reinterpret_cast<const uint4 *>(st + kOffQ + chunk_off(tq, hq * QCH + j));
+        for (int j = 0; j < QCH; ++j) {
+          ch[j] = qq * QCH + ((j + qq) & (QCH - 1));
+          w[j] = *reinterpret_cast<const uint4 *>(st + kOffQ + chunk_off(tq, ch[j]));
+        }
 #pragma unroll
         for (int j = 0; j < QCH; ++j) {
           uint32_t e[4] = {w[j].x, w[j].y, w[j].z, w[j].w};
-          const float4 za = *reinterpret_cast<const float4 *>(zs + (hq * QCH + j) * 8);
-          const float4 zb = *reinterpret_cast<const float4 *>(zs + (hq * QCH + j) * 8 + 4);
+          const float4 za = *reinterpret_cast<const float4 *>(zs + ch[j] * 8);
+          const float4 zb = *reinterpret_cast<const float4 *>(zs + ch[j] * 8 + 4);
           const float zz[8] = {za.x, za.y, za.z, za.w, zb.x, zb.y, zb.z, zb.w};
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
@@ -537,29 +669,32 @@ __global__ void __launch_bounds__(NT, 1)
         }
 #pragma unroll
         for (int j = 0; j < QCH; ++j)
-          *reinterpret_cast<uint4 *>(st + kOffQ + chunk_off(tq, hq * QCH + j)) = w[j];
-        qz += __shfl_xor_sync(0xffffffffu, qz, 1);
-        // explicit decay: the carried term of row t is lambda^(t+1) phi(q_t).z
-        if (!factored) qz *= tq < Cv ? pw[tq + 1] : 0.f;
-        if (hq == 0) den[s * 128 + tq] = qz;
+          *reinterpret_cast<uint4 *>(st + kOffQ + chunk_off(tq, ch[j])) = w[j];
+        qz += __shfl_xor_sync(0xffffffffu, qz, 8);
+        qz += __shfl_xor_sync(0xffffffffu, qz, 16);
+        // factored: phi(q') . z~; explicit: lambda^(t+1) phi(q) . z
+        if (qq == 0)
+          den[(c % kDenBufs) * 128 + tq] = qz * (factored ? 1.f : (tq < Cv ? pw[tq + 1] : 0.f));
       }
-      named_bar_sync(kBarPhi, kPhiThreads);
-      if (!factored && tt < 128) zs[tt] *= gC;
-      if (!factored) named_bar_sync(kBarPhi, kPhiThreads);
-      // (3) k: feature map, decay weights (factored), column sums into z
-      {
+      // (2) k: feature map, decay weights (factored), column sums for z
+      // factored k weight lambda^(n_f - 1 - p) = Fk lambda^(C - 1 - s)
+      const float Fk = factored ? 1.f / (Eq * pw[C]) : 1.f;
+      if (kwarp) {
         float csum[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) csum[e] = 0.f;
+        // every load of the thread's rows in flight before the first store
+        uint4 w[RPL];
 #pragma unroll
-        for (int i = 0; i < RPB; ++i) {
-          const int row = rb * RPB + i;
+        for (int i = 0; i < RPL; ++i)
+          w[i] = *reinterpret_cast<const uint4 *>(st + kOffK + chunk_off(lane + 32 * i, cg));
+#pragma unroll
+        for (int i = 0; i < RPL; ++i) {
+          const int row = lane + 32 * i;
           const float wk = row < Cv ? pw[Cv - 1 - row] : 0.f;
-          const uint32_t f2 = pack_bf16(factored ? wk : (row < Cv ? 1.f : 0.f),
-                                        factored ? wk : (row < Cv ? 1.f : 0.f));
-          uint8_t *p = st + kOffK + chunk_off(row, cg);
-          uint4 w = *reinterpret_cast<const uint4 *>(p);
-          uint32_t e[4] = {w.x, w.y, w.z, w.w};
+          const float fk = row < Cv ? (factored ? Fk * pw[C - 1 - row] : 1.f) : 0.f;
+          const uint32_t f2 = pack_bf16(fk, fk);
+          uint32_t e[4] = {w[i].x, w[i].y, w[i].z, w[i].w};
 #pragma unroll
           for (int q4 = 0; q4 < 4; ++q4) {
             if (!ident) e[q4] = phi_bf16x2(e[q4]);
@@ -570,21 +705,19 @@ __global__ void __launch_bounds__(NT, 1)
             csum[2 * q4] = fmaf(bf_lo(e[q4]), m, csum[2 * q4]);
             csum[2 * q4 + 1] = fmaf(bf_hi(e[q4]), m, csum[2 * q4 + 1]);
           }
-          *reinterpret_cast<uint4 *>(p) = make_uint4(e[0], e[1], e[2], e[3]);
+          w[i] = make_uint4(e[0], e[1], e[2], e[3]);
         }
-        // reduce over the row blocks of this warp, then across warps
 #pragma unroll
-        for (int o = NCG; o < 32; o <<= 1)
-#pragma unroll
-          for (int e = 0; e < 8; ++e) csum[e] += __shfl_xor_sync(0xffffffffu, csum[e], o);
-        if (lane < NCG) {
-#pragma unroll
-          for (int e = 0; e < 8; ++e) atomicAdd(zs + cg * 8 + e, csum[e]);
-        }
+        for (int i = 0; i < RPL; ++i)
+          *reinterpret_cast<uint4 *>(st + kOffK + chunk_off(lane + 32 * i, cg)) = w[i];
+        ztot = warp_sum8_transposed(csum, lane);
       }
       fence_proxy_async_smem();
       named_bar_sync(kBarPhi, kPhiThreads);
-      if (tt == 0) mbar_arrive(bar(kPhi0 + s));
+      if (tt == 0) {
+        mbar_arrive(bar(kPhi0 + s));
+        mbar_arrive(bar(kDenQz0 + c % kDenBufs));
+      }
       if (!factored) {
         // after the score MMA: q rows times lambda^(t+1), k rows times lambda^(Cv-1-s)
         if (tt == 0) check(mbar_wait(bar(kScore), c & 1));
@@ -598,7 +731,7 @@ __global__ void __launch_bounds__(NT, 1)
           uint8_t *base = st + (which == 0 ? kOffQ : kOffK);
 #pragma unroll
           for (int j = 0; j < QCH; ++j) {
-            uint4 *p = reinterpret_cast<uint4 *>(base + chunk_off(tq, hq * QCH + j));
+            uint4 *p = reinterpret_cast<uint4 *>(base + chunk_off(tq, qq * QCH + j));
             uint4 w = *p;
             *p = make_uint4(mul_bf16x2(w.x, f2), mul_bf16x2(w.y, f2), mul_bf16x2(w.z, f2),
                             mul_bf16x2(w.w, f2));
@@ -609,6 +742,10 @@ __global__ void __launch_bounds__(NT, 1)
         if (tt == 0) mbar_arrive(bar(kRescale));
       }
     }
+    // the last chunk's column sums; factored: z = lambda^(tokens since the frame start) z~
+    if (!rf && nchunks > 0 && zowner)
+      zs[zcol] = factored ? (zs[zcol] + ztot) * (Eq * pw[Cv_of(nchunks - 1)])
+                          : pw[Cv_of(nchunks - 1)] * zs[zcol] + ztot;
     named_bar_sync(kBarPhi, kPhiThreads);
     if (!rf && last_seg && z_final && tt < DK) z_final[pair * DK + tt] = zs[tt];
   }
@@ -630,10 +767,14 @@ __global__ void __launch_bounds__(NT, 1)
 // out_S / out_z.  The segmented forward runs it on its first G - 1 segments
 // (slots = G; the combine scan then turns the slots into starting states);
 // linattn_causal_state runs it on whole sequences (one segment, slots = 1).
-// Roles (512 threads): warp 0 TMA (k and v, 3 stages), warp 1 MMA issuer,
-// warps 4-7 decay of the TMEM state between chunks, warps 8-15 feature map.
+// Every k row is weighted by its own lambda^(n-1-s) (at most 1; weights below
+// the fp32 range flush to zero, far below the rounding of the kept terms), so
+// the state MMAs accumulate the whole segment with no decay step between
+// chunks.
+// Roles (768 threads): warp 0 TMA (k and v, 3 stages), warp 1 MMA issuer,
+// warps 4-7 store of the final state, warps 8-23 feature map.
 namespace sp {
-constexpr int NT = 512;
+constexpr int NT = 768;
 constexpr int kStages = 3;
 constexpr uint32_t kOffK = 0, kOffV = 2 * kPanel;
 constexpr uint32_t kStage = 4 * kPanel;                  // 64 KB
@@ -642,8 +783,9 @@ constexpr uint32_t kMiscTmem = 256, kMiscAbort = 260, kMiscRoleFail = 272;
 constexpr uint32_t kMiscPw = 320, kMiscZ = 848;
 constexpr uint32_t kSmemBytes = kOffMisc + kMiscZ + 128 * 4;
 static_assert(kSmemBytes <= 232448, "exceeds the per-CTA shared memory of sm_100");
-enum Bar { kFull0 = 0, kFree0 = 3, kPhi0 = 6, kState = 9, kDecay, kFinal, kNumBars };
-constexpr int kBarPhi = 1, kBarDecay = 2;
+enum Bar { kFull0 = 0, kFree0 = 3, kPhi0 = 6, kState = 9, kNumBars };
+constexpr int kBarPhi = 1, kBarStore = 2;
+constexpr int kPhiThreads = 512;
 }  // namespace sp
 
 template <int DKP, int DVP>
@@ -742,8 +884,7 @@ __global__ void __launch_bounds__(sp::NT, 1)
       for (int c = 0; ok && c < nchunks; ++c) {
         const int s = c % sp::kStages;
         const uint32_t st = sb + s * sp::kStage;
-        if (*abort_flag || !mbar_wait(bar(sp::kPhi0 + s), (c / sp::kStages) & 1) ||
-            (c >= 1 && !mbar_wait(bar(sp::kDecay), (c - 1) & 1))) {
+        if (*abort_flag || !mbar_wait(bar(sp::kPhi0 + s), (c / sp::kStages) & 1)) {
           ok = false;
           break;
         }
@@ -754,106 +895,102 @@ __global__ void __launch_bounds__(sp::NT, 1)
         for (int ks = 0; ks < C / 16; ++ks)
           umma_bf16(tmem, k0 + ks * (2048 >> 4), v0 + ks * (2048 >> 4), idS,
                     (c > 0 || ks > 0) ? 1u : 0u);
-        umma_commit(bar(sp::kState));
         umma_commit(bar(sp::kFree0 + s));
       }
       if (!ok) fail();
-      umma_commit(bar(sp::kFinal));
-      mbar_wait(bar(sp::kFinal), 0);
+      // every MMA done: the state is final (and TMEM idle before teardown)
+      umma_commit(bar(sp::kState));
+      mbar_wait(bar(sp::kState), 0);
     }
     __syncwarp();
   } else if (warp >= 4 && warp < 8) {
     const int wq = warp - 4;
     const int r = wq * 32 + lane;
     const uint32_t lf = static_cast<uint32_t>(wq * 32) << 16;
-    volatile int &rf = role_fail[0];
-    for (int c = 0; c < nchunks; ++c) {
-      const bool last = c == nchunks - 1;
-      if (*abort_flag || !mbar_wait(bar(sp::kState), c & 1)) {
-        rf = 1;
-        fail();
-      }
-      tc_fence_after();
-      if (!rf) {
-        const float gC = last ? 1.f : pw[Cv_of(c + 1)];
+    if (*abort_flag || !mbar_wait(bar(sp::kState), 0)) fail();
+    tc_fence_after();
+    if (!*abort_flag) {
+#pragma unroll 1
+      for (int blk = 0; blk < DV / 32; ++blk) {
+        uint32_t sv[32];
+        tmem_ld_32x32b_x32(tmem + lf + blk * 32, sv);   // warp-wide load
+        tmem_wait_ld();
+        if (r < DK) {
+          float4 *dst =
+              reinterpret_cast<float4 *>(out_S + (slot * DK + r) * static_cast<long>(DV)) + blk * 8;
 #pragma unroll
-        for (int blk = 0; blk < DV / 32; ++blk) {
-          uint32_t sv[32];
-          tmem_ld_32x32b_x32(tmem + lf + blk * 32, sv);
-          tmem_wait_ld();
-          if (last) {
-            if (r < DK) {
-              float4 *dst = reinterpret_cast<float4 *>(
-                                out_S + (slot * DK + r) * static_cast<long>(DV)) +
-                            blk * 8;
-#pragma unroll
-              for (int i = 0; i < 8; ++i)
-                dst[i] = make_float4(__uint_as_float(sv[4 * i]), __uint_as_float(sv[4 * i + 1]),
-                                     __uint_as_float(sv[4 * i + 2]), __uint_as_float(sv[4 * i + 3]));
-            }
-          } else {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) sv[i] = __float_as_uint(__uint_as_float(sv[i]) * gC);
-            tmem_st_32x32b_x32(tmem + lf + blk * 32, sv);
-          }
+          for (int i = 0; i < 8; ++i)
+            dst[i] = nchunks == 0 ? make_float4(0.f, 0.f, 0.f, 0.f)
+                                  : make_float4(__uint_as_float(sv[4 * i]),
+                                                __uint_as_float(sv[4 * i + 1]),
+                                                __uint_as_float(sv[4 * i + 2]),
+                                                __uint_as_float(sv[4 * i + 3]));
         }
-        if (!last) tmem_wait_st();
       }
-      tc_fence_before();
-      named_bar_sync(sp::kBarDecay, 128);
-      if (rf) break;
-      if (r == 0 && !last) mbar_arrive(bar(sp::kDecay));
     }
+    tc_fence_before();
   } else if (warp >= 8) {
-    const int tt = tid - 256;                 // 0..255
+    const int tt = tid - 256;                 // 0..511
+    const int fw = tt >> 5;                   // feature-map warp 0..15
     volatile int &rf = role_fail[1];
-    constexpr int NCG = KCH, RPB = NCG / 2;
-    const int cg = tt % NCG, rb = tt / NCG;
+    // a warp owns one column group of 8 columns over all 128 rows (the column
+    // sums of z need no atomics); with d_k = 64 only the first 8 warps work
+    constexpr int NCG = KCH, RPL = 128 / 32;
+    const bool kwarp = fw < NCG;
+    const int cg = fw;
+    float ztot = 0.f;
+    const int zcol = cg * 8 + warp_sum8_index(lane);
+    const bool zowner = kwarp && (lane & 3) == 0;
+    const float log2L = L > 0.f ? log2f(L) : 0.f;
     for (int c = 0; c < nchunks; ++c) {
       const int s = c % sp::kStages;
       uint8_t *st = sm + s * sp::kStage;
+      // the previous chunk's column sums (already weighted to the segment end)
+      if (c > 0 && zowner) zs[zcol] += ztot;
       if (tt == 0 && (*abort_flag || !mbar_wait(bar(sp::kFull0 + s), (c / sp::kStages) & 1))) {
         rf = 1;
         fail();
       }
-      named_bar_sync(sp::kBarPhi, 256);
+      named_bar_sync(sp::kBarPhi, sp::kPhiThreads);
       if (rf) break;
       const int Cv = Cv_of(c);
-      if (tt < 128) zs[tt] *= pw[Cv];
-      named_bar_sync(sp::kBarPhi, 256);
-      float csum[8];
+      // lambda^(tokens of the segment after this chunk)
+      const int after = (n1 - n0) - c * C - Cv;
+      const float Tc = after == 0 ? 1.f : (L > 0.f ? exp2f(static_cast<float>(after) * log2L) : 0.f);
+      if (kwarp) {
+        float csum[8];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) csum[e] = 0.f;
+        for (int e = 0; e < 8; ++e) csum[e] = 0.f;
+        uint4 w[RPL];
 #pragma unroll
-      for (int i = 0; i < RPB; ++i) {
-        const int row = rb * RPB + i;
-        const float wk = row < Cv ? pw[Cv - 1 - row] : 0.f;
-        const uint32_t f2 = pack_bf16(wk, wk);
-        uint8_t *p = st + sp::kOffK + chunk_off(row, cg);
-        uint4 w = *reinterpret_cast<const uint4 *>(p);
-        uint32_t e[4] = {w.x, w.y, w.z, w.w};
+        for (int i = 0; i < RPL; ++i)
+          w[i] = *reinterpret_cast<const uint4 *>(st + sp::kOffK + chunk_off(lane + 32 * i, cg));
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          if (!ident) e[q4] = phi_bf16x2(e[q4]);
-          e[q4] = mul_bf16x2(e[q4], f2);
-          csum[2 * q4] += bf_lo(e[q4]);
-          csum[2 * q4 + 1] += bf_hi(e[q4]);
+        for (int i = 0; i < RPL; ++i) {
+          const int row = lane + 32 * i;
+          const float wk = row < Cv ? Tc * pw[Cv - 1 - row] : 0.f;
+          const uint32_t f2 = pack_bf16(wk, wk);
+          uint32_t e[4] = {w[i].x, w[i].y, w[i].z, w[i].w};
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            if (!ident) e[q4] = phi_bf16x2(e[q4]);
+            e[q4] = mul_bf16x2(e[q4], f2);
+            csum[2 * q4] += bf_lo(e[q4]);
+            csum[2 * q4 + 1] += bf_hi(e[q4]);
+          }
+          w[i] = make_uint4(e[0], e[1], e[2], e[3]);
         }
-        *reinterpret_cast<uint4 *>(p) = make_uint4(e[0], e[1], e[2], e[3]);
-      }
 #pragma unroll
-      for (int o = NCG; o < 32; o <<= 1)
-#pragma unroll
-        for (int e = 0; e < 8; ++e) csum[e] += __shfl_xor_sync(0xffffffffu, csum[e], o);
-      if (lane < NCG) {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) atomicAdd(zs + cg * 8 + e, csum[e]);
+        for (int i = 0; i < RPL; ++i)
+          *reinterpret_cast<uint4 *>(st + sp::kOffK + chunk_off(lane + 32 * i, cg)) = w[i];
+        ztot = warp_sum8_transposed(csum, lane);
       }
       fence_proxy_async_smem();
-      named_bar_sync(sp::kBarPhi, 256);
+      named_bar_sync(sp::kBarPhi, sp::kPhiThreads);
       if (tt == 0) mbar_arrive(bar(sp::kPhi0 + s));
     }
-    named_bar_sync(sp::kBarPhi, 256);
+    if (!rf && nchunks > 0 && zowner) zs[zcol] += ztot;
+    named_bar_sync(sp::kBarPhi, sp::kPhiThreads);
     if (!rf && tt < DK) out_z[slot * DK + tt] = zs[tt];
   }
   tc_fence_before();

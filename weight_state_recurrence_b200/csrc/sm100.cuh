@@ -56,6 +56,22 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// As mbar_try_wait, but a thread whose phase is still open may be suspended
+// for up to kSuspendHintNs (it resumes as soon as the phase completes), so a
+// waiting warp takes no issue slots from the warps doing the work.
+constexpr uint32_t kSuspendHintNs = 1000000u;   // 1 ms
+__device__ __forceinline__ bool mbar_try_wait_suspend(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(kSuspendHintNs)
+      : "memory");
+  return ok != 0;
+}
+
 // Bounded wait for the phase with the given parity to complete.  Returns
 // false (and records kStatusWaitTimeout) if it did not complete within
 // kWaitLimitNs; the caller must then abandon its work in an orderly way.
@@ -63,7 +79,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = global_timer_ns();
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_suspend(bar, parity)) return true;
     if (global_timer_ns() - t0 > kWaitLimitNs) {
       atomicOr(&g_status, kStatusWaitTimeout);
       return false;
