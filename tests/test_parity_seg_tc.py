@@ -117,3 +117,21 @@ def test_headline_workload_two_segments_sampled(cuda_lib):
 
 def test_no_device_errors_recorded(cuda_lib):
     assert cuda_lib.linattn_device_status(True) == 0
+
+
+def test_output_16_byte_aligned_only(cuda_lib):
+    """y written to a buffer that is 16- but not 32-byte aligned (the
+    kernel's 32-byte stores need the wider alignment and fall back)."""
+    q, k, v = inputs.random_case(3300, 1, 2, 300, 128, 128, torch.bfloat16, scale=128 ** -0.5)
+    lam = torch.tensor([0.95, 1.0])
+    raw = torch.empty(q.numel() + 8, dtype=torch.bfloat16, device=DEV)
+    off = 8 if raw.data_ptr() % 32 == 0 else 0   # 8 bf16 = 16 bytes
+    out = raw[off:off + q.numel()].view(q.shape)
+    assert out.data_ptr() % 32 == 16
+    S = torch.empty(1, 2, 128, 128, device=DEV)
+    z = torch.empty(1, 2, 128, device=DEV)
+    cuda_lib.linattn_fwd_causal(q.to(DEV), k.to(DEV), v.to(DEV), lam.to(DEV), 1e-6, out, S, z)
+    torch.cuda.synchronize()
+    y_o, S_o, z_o = oracle.causal(q, k, v, lam, 1e-6)
+    assert_close("y", out, y_o, 2e-2)
+    assert_close("S_final", S, S_o, 2e-2)

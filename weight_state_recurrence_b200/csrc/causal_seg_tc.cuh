@@ -18,11 +18,14 @@
 //   z   <- lambda^Cv z + (Lk phi(K))^T 1
 //
 // Tensor-core chains per chunk (M = 128, K = 16 per instruction, N = d_v):
-//   score   D_A   = phi(Q) phi(K)^T                       SMEM x SMEM
-//   carried D_O   = phi(Q) S'        (S' = bf16 state)    SMEM x SMEM
+//   score   D_A   = phi(Q) phi(K)^T                       TMEM x SMEM
+//   carried D_O   = phi(Q) S'        (S' = bf16 state)    TMEM x SMEM
 //   state   D_S  += (Lk phi(K))^T V                       SMEM x SMEM (both MN-major)
 //   intra   D_O  += P V              (P = bf16 in TMEM)   TMEM x SMEM
-// One accumulator takes both halves of the numerator.  The denominator is
+// One accumulator takes both halves of the numerator.  phi(Q) is written to
+// TMEM by the feature-map warps, so three of the four chains read only their
+// B operand from shared memory: an MMA that reads both operands there takes
+// shared-memory bandwidth that the feature map needs.  The denominator is
 // formed in fp32 on the CUDA cores: the feature-map warps keep z and take
 // phi(q_t).z while they transform q; the score epilogue adds the fp32 row sums
 // of the masked score tile (the numerator uses the same weights rounded to
@@ -46,9 +49,11 @@
 //   warp 1      TMEM owner, the single MMA-issuing thread
 //   warp 2      TMA producer of the v tiles
 //   warps 4-7   score epilogue: D_A -> mask (and decay) -> bf16 P in TMEM, row sums
-//   warps 8-11  output: y = D_O / den -> global memory
+//   warps 8-11  output: y = D_O / den -> global memory (D_O single-buffered:
+//               the next carried product waits until it is drained)
 //   warps 12-15 state: D_S -> bf16 operand S' (and the decay or renormalisation of D_S)
-//   warps 16-31 feature map (in place, packed bf16x2), phi(q).z, z update
+//   warps 16-31 feature map (packed bf16x2): phi(q) into TMEM, phi(k) in place,
+//               phi(q).z, z update
 // Every wait is bounded (sm100.cuh); a wait that runs out records an error
 // flag and every role leaves its loop.
 #pragma once
@@ -87,18 +92,19 @@ static_assert(kSmemBytes <= 232448, "exceeds the per-CTA shared memory of sm_100
 
 enum Bar {
   kFullQK0 = 0, kFullQK1, kFullV0, kFullV1, kFreeQK0, kFreeQK1, kFreeV0, kFreeV1,
-  kPhi0, kPhi1, kScore, kRescale, kState, kReadout, kPDone, kO0, kO1, kOut0, kOut1,
-  kSop,
+  kPhi0, kPhi1, kScore, kRescale, kState, kReadout, kPDone, kO, kOut, kSop,
+  kQFree0, kQFree1,   // the score epilogue has read the phi(q).z parts left in q tile s
   // den buffer b (chunk c uses b = c % 3): phi(q).z written, row sums added, read by the output
   kDenQz0, kDenQz1, kDenQz2, kDenRs0, kDenRs1, kDenRs2, kDenFree0, kDenFree1, kDenFree2,
   kFinal, kNumBars
 };
 static_assert(kNumBars * 8 <= 256, "barrier area overflow");
 
-// tensor memory columns (fp32, lane = row)
+// tensor memory columns (32-bit, lane = row)
 constexpr uint32_t kTmS = 0;     // state D_S, lane = d_k row
 constexpr uint32_t kTmA = 128;   // score D_A; P (bf16 pairs) overwrites its first 64 columns
-constexpr uint32_t kTmO = 256;   // output accumulators D_O[0], D_O[1]
+constexpr uint32_t kTmO = 256;   // output accumulator D_O
+constexpr uint32_t kTmQ = 384;   // phi(Q') as bf16 pairs, 64 columns per stage (A of score, carried)
 constexpr uint32_t kTmCols = 512;
 
 __device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
@@ -241,7 +247,8 @@ __global__ void __launch_bounds__(NT, 1)
       int issued = 0;
       for (int c = 0; c < nchunks && !*abort_flag; ++c) {
         const int s = c & 1;
-        if (c >= 2 && !mbar_wait(bar((qk ? kFreeQK0 : kFreeV0) + s), ((c - 2) >> 1) & 1)) {
+        if (c >= 2 && (!mbar_wait(bar((qk ? kFreeQK0 : kFreeV0) + s), ((c - 2) >> 1) & 1) ||
+                       (qk && !mbar_wait(bar(kQFree0 + s), ((c - 2) >> 1) & 1)))) {
           fail();
           break;
         }
@@ -286,7 +293,6 @@ __global__ void __launch_bounds__(NT, 1)
       // descriptors of every operand tile, per stage; a K step adds its byte
       // offset >> 4 to the start-address field (tiles stay below 256 KB, so
       // the 14-bit field never carries)
-      const uint64_t dQ = sdesc_sw128(sb + kOffQ, 16, 1024);
       const uint64_t dK = sdesc_sw128(sb + kOffK, 16, 1024);
       const uint64_t dKmn = sdesc_sw128(sb + kOffK, kPanel, 1024);
       const uint64_t dV = sdesc_sw128(sb + kOffV, kPanel, 1024);
@@ -296,33 +302,34 @@ __global__ void __launch_bounds__(NT, 1)
       for (int c = 0; ok && c < nchunks; ++c) {
         const int s = c & 1;
         if (*abort_flag) break;
-        // score: D_A = phi(Q) phi(K)^T (the previous chunk's P V, issued
-        // before, has read D_A: the chains run in issue order)
+        // score: D_A = phi(Q') phi(K')^T, phi(Q') from TMEM (the previous
+        // chunk's P V, issued before, has read D_A: the chains run in issue order)
         if (!mbar_wait(bar(kPhi0 + s), (c >> 1) & 1)) { ok = false; break; }
         tc_fence_after();
         const uint64_t so = static_cast<uint64_t>(s) * (kStage >> 4);   // stage offset
-        const uint64_t q0 = dQ + so, k0 = dK + so, kmn0 = dKmn + so, v0 = dV + so;
+        const uint64_t k0 = dK + so, kmn0 = dKmn + so, v0 = dV + so;
+        const uint32_t qa = tmem + kTmQ + s * 64;
 #pragma unroll
         for (int ks = 0; ks < 4 * DKP; ++ks)
-          umma_bf16(tmem + kTmA, q0 + kofs(ks), k0 + kofs(ks), idA, ks > 0);
+          umma_bf16_ts(tmem + kTmA, qa + ks * 8, k0 + kofs(ks), idA, ks > 0);
         umma_commit(bar(kScore));
         // explicit decay: the q and k rows are rescaled once the score MMA has read them
         if (!factored && !mbar_wait(bar(kRescale), c & 1)) { ok = false; break; }
-        // carried: D_O[s] = phi(Q) S'  (state before this chunk; D_O[s] drained)
-        if (!mbar_wait(bar(kSop), c & 1) ||
-            (c >= 2 && !mbar_wait(bar(kOut0 + s), ((c - 2) >> 1) & 1))) {
+        // carried: D_O = phi(Q') S'  (state before this chunk; the previous
+        // chunk's output has drained D_O)
+        if (!mbar_wait(bar(kSop), c & 1) || (c >= 1 && !mbar_wait(bar(kOut), (c - 1) & 1))) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t dO = tmem + kTmO + s * 128;
+        const uint32_t dO = tmem + kTmO;
         const bool carried = c > 0 || has_init;
         if (carried) {
 #pragma unroll
           for (int ks = 0; ks < 4 * DKP; ++ks)
-            umma_bf16(dO, q0 + kofs(ks), dSop + ks * (2048 >> 4), idQS, ks > 0);
+            umma_bf16_ts(dO, qa + ks * 8, dSop + ks * (2048 >> 4), idQS, ks > 0);
         }
-        // state: D_S += (Lk phi(K))^T V   (onto the state decayed by lambda^Cv)
+        // state: D_S += (Lk phi(K))^T V
         if (!mbar_wait(bar(kReadout), c & 1) || !mbar_wait(bar(kFullV0 + s), (c >> 1) & 1)) {
           ok = false;
           break;
@@ -333,15 +340,15 @@ __global__ void __launch_bounds__(NT, 1)
           umma_bf16(tmem + kTmS, kmn0 + ks * (2048 >> 4), v0 + ks * (2048 >> 4), idS,
                     (carried || ks > 0) ? 1u : 0u);
         umma_commit(bar(kState));
-        umma_commit(bar(kFreeQK0 + s));   // q and k of this chunk fully read
-        // intra: D_O[s] += P V
+        umma_commit(bar(kFreeQK0 + s));   // q, k tiles and phi(Q') of this chunk fully read
+        // intra: D_O += P V
         if (!mbar_wait(bar(kPDone), c & 1)) { ok = false; break; }
         tc_fence_after();
 #pragma unroll
         for (int ks = 0; ks < C / 16; ++ks)
           umma_bf16_ts(dO, tmem + kTmA + ks * 8, v0 + ks * (2048 >> 4), idQS,
                        (carried || ks > 0) ? 1u : 0u);
-        umma_commit(bar(kO0 + s));
+        umma_commit(bar(kO));
         umma_commit(bar(kFreeV0 + s));
       }
       if (!ok) fail();
@@ -358,15 +365,25 @@ __global__ void __launch_bounds__(NT, 1)
     for (int c = 0; c < nchunks; ++c) {
       const int s = c & 1;
       // kDenQz orders the feature-map warps' phi(q).z before this role's
-      // update of the chunk's den buffer
-      if (*abort_flag || !mbar_wait(bar(kScore), c & 1) ||
-          !mbar_wait(bar(kDenQz0 + c % kDenBufs), (c / kDenBufs) & 1)) {
+      // update of the chunk's den buffer.  One thread polls; the others wait
+      // at the named barrier, which takes no issue slots.
+      if (t == 0 && (*abort_flag || !mbar_wait(bar(kScore), c & 1) ||
+                     !mbar_wait(bar(kDenQz0 + c % kDenBufs), (c / kDenBufs) & 1) ||
+                     (c >= kDenBufs && !mbar_wait(bar(kDenFree0 + c % kDenBufs),
+                                                  ((c - kDenBufs) / kDenBufs) & 1)))) {
         rf = 1;
         fail();
       }
+      named_bar_sync(kBarP, 128);
       tc_fence_after();
       float rs = 0.f;
       if (!rf) {
+        // phi(q').z of row t: the feature-map warps left one part per column
+        // block in q tile s, summed here in a fixed order
+        const uint8_t *qt = sm + (c & 1) * kStage + kOffQ;
+#pragma unroll
+        for (int cb = 0; cb < 4; ++cb)
+          rs += *reinterpret_cast<const float *>(qt + chunk_off(t, cb * (2 * DKP)));
         // blocks of 32 keys, one load each; only blocks 0..wq hold s <= t
 #pragma unroll 1
         for (int bk = 0; bk < 4; ++bk) {
@@ -407,7 +424,7 @@ __global__ void __launch_bounds__(NT, 1)
           tmem_st_32x32b_x16(tmem + lf + kTmA + bk * 16, pk);
         }
         tmem_wait_st();
-        den[(c % kDenBufs) * 128 + t] += rs;   // phi(q).z was written there by the feature-map warps
+        den[(c % kDenBufs) * 128 + t] = rs;
       }
       tc_fence_before();
       named_bar_sync(kBarP, 128);
@@ -415,6 +432,7 @@ __global__ void __launch_bounds__(NT, 1)
       if (t == 0) {
         mbar_arrive(bar(kPDone));
         mbar_arrive(bar(kDenRs0 + c % kDenBufs));
+        mbar_arrive(bar(kQFree0 + (c & 1)));
       }
     }
   } else if (warp >= 8 && warp < 12) {
@@ -423,13 +441,15 @@ __global__ void __launch_bounds__(NT, 1)
     const int t = wq * 32 + lane;
     const uint32_t lf = static_cast<uint32_t>(wq * 32) << 16;
     volatile int &rf = role_fail[1];
+    // rows are 128 or 256 bytes, so 32-byte stores need only the base aligned
+    const bool out32 = (reinterpret_cast<uintptr_t>(out) & 31u) == 0;
     for (int c = 0; c < nchunks; ++c) {
-      const int s = c & 1;
-      if (*abort_flag || !mbar_wait(bar(kO0 + s), (c >> 1) & 1) ||
-          !mbar_wait(bar(kDenRs0 + c % kDenBufs), (c / kDenBufs) & 1)) {
+      if (t == 0 && (*abort_flag || !mbar_wait(bar(kO), c & 1) ||
+                     !mbar_wait(bar(kDenRs0 + c % kDenBufs), (c / kDenBufs) & 1))) {
         rf = 1;
         fail();
       }
+      named_bar_sync(kBarOut, 128);
       tc_fence_after();
       if (!rf) {
         const float inv = 1.f / (den[(c % kDenBufs) * 128 + t] + eps);
@@ -439,16 +459,20 @@ __global__ void __launch_bounds__(NT, 1)
 #pragma unroll 1
         for (int blk = 0; blk < DV / 32; ++blk) {
           uint32_t r[32];
-          tmem_ld_32x32b_x32(tmem + lf + kTmO + s * 128 + blk * 32, r);
+          tmem_ld_32x32b_x32(tmem + lf + kTmO + blk * 32, r);
           tmem_wait_ld();
           uint32_t pk[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i)
             pk[i] = pack_bf16(__uint_as_float(r[2 * i]) * inv, __uint_as_float(r[2 * i + 1]) * inv);
           if (live) {
+            if (out32) {
+              st_global_na_v8(dst + blk * 4, pk);
+              st_global_na_v8(dst + blk * 4 + 2, pk + 8);
+            } else {
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-              dst[blk * 4 + i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+              for (int i = 0; i < 4; ++i) st_global_na_v4(dst + blk * 4 + i, pk + 4 * i);
+            }
           }
         }
       }
@@ -456,7 +480,7 @@ __global__ void __launch_bounds__(NT, 1)
       named_bar_sync(kBarOut, 128);
       if (rf) break;
       if (t == 0) {
-        mbar_arrive(bar(kOut0 + s));
+        mbar_arrive(bar(kOut));
         mbar_arrive(bar(kDenFree0 + c % kDenBufs));
       }
     }
@@ -517,10 +541,11 @@ __global__ void __launch_bounds__(NT, 1)
     const float gR = factored && R < nchunks ? pow_int(L, R * C) : 1.f;
     for (int c = 0; c < nchunks; ++c) {
       const bool last = c == nchunks - 1;
-      if (*abort_flag || !mbar_wait(bar(kState), c & 1)) {
+      if (r == 0 && (*abort_flag || !mbar_wait(bar(kState), c & 1))) {
         rf = 1;
         fail();
       }
+      named_bar_sync(kBarState, 128);
       tc_fence_after();
       if (!rf && last && last_seg && S_final) {
         // factored: S = lambda^(tokens since the frame start) S~
@@ -600,12 +625,14 @@ __global__ void __launch_bounds__(NT, 1)
       }
     };
     const int fw = tt >> 5;                   // feature-map warp 0..15
-    // q: thread (row tq, quarter qq of the row's 16-byte chunks): a warp holds
-    // 8 rows x 4 quarters; at step j quarter qq takes chunk (j + qq) of its
-    // quarter, so the tile accesses and the reads of z spread over all banks.
-    // The quarters of a row meet by shuffles.
-    constexpr int QCH = KCH / 4;              // chunks per thread (4 or 2)
-    const int tq = fw * 8 + (lane & 7), qq = lane >> 3;
+    // q: a thread owns row tq = 32 (warp % 4) + lane, its TMEM lane, and
+    // column block cb = fw / 4 (d_k / 4 columns); phi(q') goes to TMEM as the A
+    // operand of the score and carried products, and the block's part of
+    // phi(q').z is added to the chunk's den
+    constexpr int QCH = KCH / 4;              // 16-byte chunks per thread (4 or 2)
+    const int tq = (warp & 3) * 32 + lane, cb = fw >> 2;
+    const uint32_t lfq = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    auto tq_col = [&](int s) { return tmem + lfq + kTmQ + s * 64 + cb * 4 * QCH; };
     // k: a warp owns one column group of 8 columns over all 128 rows, so the
     // column sums of z need no atomics; with d_k = 64 (8 groups) only the
     // first 8 warps take k
@@ -630,12 +657,7 @@ __global__ void __launch_bounds__(NT, 1)
       if (c > 0 && zowner)
         zs[zcol] = factored ? (frame_start ? gR : 1.f) * (zs[zcol] + ztot)
                             : pw[Cv_of(c - 1)] * zs[zcol] + ztot;
-      if (tt == 0) {
-        check(mbar_wait(bar(kFullQK0 + s), (c >> 1) & 1));
-        // den[c % 3] was read by the output of chunk c - 3
-        if (c >= kDenBufs)
-          check(mbar_wait(bar(kDenFree0 + c % kDenBufs), ((c - kDenBufs) / kDenBufs) & 1));
-      }
+      if (tt == 0) check(mbar_wait(bar(kFullQK0 + s), (c >> 1) & 1));
       named_bar_sync(kBarPhi, kPhiThreads);
       if (rf) break;
       // (1) q rows: feature map, decay scale, phi(q).z_{c-1}
@@ -646,17 +668,15 @@ __global__ void __launch_bounds__(NT, 1)
         const uint32_t f2 = pack_bf16(fq, fq);
         float qz = 0.f;
         uint4 w[QCH];
-        int ch[QCH];
 #pragma unroll
-        for (int j = 0; j < QCH; ++j) {
-          ch[j] = qq * QCH + ((j + qq) & (QCH - 1));
-          w[j] = *reinterpret_cast<const uint4 *>(st + kOffQ + chunk_off(tq, ch[j]));
-        }
+        for (int j = 0; j < QCH; ++j)
+          w[j] = *reinterpret_cast<const uint4 *>(st + kOffQ + chunk_off(tq, cb * QCH + j));
+        uint32_t pk[4 * QCH];
 #pragma unroll
         for (int j = 0; j < QCH; ++j) {
           uint32_t e[4] = {w[j].x, w[j].y, w[j].z, w[j].w};
-          const float4 za = *reinterpret_cast<const float4 *>(zs + ch[j] * 8);
-          const float4 zb = *reinterpret_cast<const float4 *>(zs + ch[j] * 8 + 4);
+          const float4 za = *reinterpret_cast<const float4 *>(zs + (cb * QCH + j) * 8);
+          const float4 zb = *reinterpret_cast<const float4 *>(zs + (cb * QCH + j) * 8 + 4);
           const float zz[8] = {za.x, za.y, za.z, za.w, zb.x, zb.y, zb.z, zb.w};
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
@@ -664,17 +684,16 @@ __global__ void __launch_bounds__(NT, 1)
             e[i] = mul_bf16x2(e[i], f2);
             qz = fmaf(bf_lo(e[i]), zz[2 * i], qz);
             qz = fmaf(bf_hi(e[i]), zz[2 * i + 1], qz);
+            pk[4 * j + i] = e[i];
           }
-          w[j] = make_uint4(e[0], e[1], e[2], e[3]);
         }
-#pragma unroll
-        for (int j = 0; j < QCH; ++j)
-          *reinterpret_cast<uint4 *>(st + kOffQ + chunk_off(tq, ch[j])) = w[j];
-        qz += __shfl_xor_sync(0xffffffffu, qz, 8);
-        qz += __shfl_xor_sync(0xffffffffu, qz, 16);
-        // factored: phi(q') . z~; explicit: lambda^(t+1) phi(q) . z
-        if (qq == 0)
-          den[(c % kDenBufs) * 128 + tq] = qz * (factored ? 1.f : (tq < Cv ? pw[tq + 1] : 0.f));
+        if constexpr (QCH == 4) tmem_st_32x32b_x16(tq_col(s), pk);
+        else tmem_st_32x32b_x8(tq_col(s), pk);
+        // factored: phi(q') . z~; explicit: lambda^(t+1) phi(q) . z.  The
+        // part of this column block goes into the q bytes this thread alone
+        // has read (the score epilogue sums the four parts of the row).
+        *reinterpret_cast<float *>(st + kOffQ + chunk_off(tq, cb * QCH)) =
+            qz * (factored ? 1.f : (tq < Cv ? pw[tq + 1] : 0.f));
       }
       // (2) k: feature map, decay weights (factored), column sums for z
       // factored k weight lambda^(n_f - 1 - p) = Fk lambda^(C - 1 - s)
@@ -713,30 +732,45 @@ __global__ void __launch_bounds__(NT, 1)
         ztot = warp_sum8_transposed(csum, lane);
       }
       fence_proxy_async_smem();
+      tmem_wait_st();
+      tc_fence_before();
       named_bar_sync(kBarPhi, kPhiThreads);
       if (tt == 0) {
         mbar_arrive(bar(kPhi0 + s));
         mbar_arrive(bar(kDenQz0 + c % kDenBufs));
       }
       if (!factored) {
-        // after the score MMA: q rows times lambda^(t+1), k rows times lambda^(Cv-1-s)
+        // after the score MMA: q rows (TMEM) times lambda^(t+1), k rows (SMEM)
+        // times lambda^(Cv-1-s)
         if (tt == 0) check(mbar_wait(bar(kScore), c & 1));
         named_bar_sync(kBarPhi, kPhiThreads);
         if (rf) break;
-#pragma unroll
-        for (int which = 0; which < 2; ++which) {
-          const float f = which == 0 ? (tq < Cv ? pw[tq + 1] : 0.f)
-                                     : (tq < Cv ? pw[Cv - 1 - tq] : 0.f);
+        tc_fence_after();
+        {
+          const float f = tq < Cv ? pw[tq + 1] : 0.f;
           const uint32_t f2 = pack_bf16(f, f);
-          uint8_t *base = st + (which == 0 ? kOffQ : kOffK);
+          uint32_t pk[4 * QCH];
+          if constexpr (QCH == 4) tmem_ld_32x32b_x16(tq_col(s), pk);
+          else tmem_ld_32x32b_x8(tq_col(s), pk);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 4 * QCH; ++i) pk[i] = mul_bf16x2(pk[i], f2);
+          if constexpr (QCH == 4) tmem_st_32x32b_x16(tq_col(s), pk);
+          else tmem_st_32x32b_x8(tq_col(s), pk);
+        }
+        {
+          const float f = tq < Cv ? pw[Cv - 1 - tq] : 0.f;
+          const uint32_t f2 = pack_bf16(f, f);
 #pragma unroll
           for (int j = 0; j < QCH; ++j) {
-            uint4 *p = reinterpret_cast<uint4 *>(base + chunk_off(tq, qq * QCH + j));
+            uint4 *p = reinterpret_cast<uint4 *>(st + kOffK + chunk_off(tq, cb * QCH + j));
             uint4 w = *p;
             *p = make_uint4(mul_bf16x2(w.x, f2), mul_bf16x2(w.y, f2), mul_bf16x2(w.z, f2),
                             mul_bf16x2(w.w, f2));
           }
         }
+        tmem_wait_st();
+        tc_fence_before();
         fence_proxy_async_smem();
         named_bar_sync(kBarPhi, kPhiThreads);
         if (tt == 0) mbar_arrive(bar(kRescale));
@@ -907,7 +941,9 @@ __global__ void __launch_bounds__(sp::NT, 1)
     const int wq = warp - 4;
     const int r = wq * 32 + lane;
     const uint32_t lf = static_cast<uint32_t>(wq * 32) << 16;
-    if (*abort_flag || !mbar_wait(bar(sp::kState), 0)) fail();
+    // one thread polls for the whole pass; the others wait at the named barrier
+    if (r == 0 && (*abort_flag || !mbar_wait(bar(sp::kState), 0))) fail();
+    named_bar_sync(sp::kBarStore, 128);
     tc_fence_after();
     if (!*abort_flag) {
 #pragma unroll 1
