@@ -232,15 +232,13 @@ def causal_leg(lib, args, world, rank, stream, hbm, tc_peak):
     S = torch.empty(B, H, d, d, device=dev)
     z = torch.empty(B, H, d, device=dev)
 
-    ws = None
-    seg_launches = 1
-    if args.segments:
-        # the segmented form asked for explicitly (state pass, combine scan,
-        # then all segments at once), through the workspace entry point
-        with lib.kernel_choice(lib.LINATTN_OP_CAUSAL, lib.LINATTN_KERNEL_AUTO, args.segments):
-            need = lib.linattn_fwd_causal_workspace(B, H, N, d, d, WL.dtype)
-        ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
-        seg_launches = 3 if need > 0 else 1   # state pass, combine scan, forward
+    # the product call: linattn_fwd_causal_ws with the workspace the library
+    # asks for (the segment plan it picks, or --segments forced), i.e. the
+    # state pass and the forward launched as its dependent
+    with lib.kernel_choice(lib.LINATTN_OP_CAUSAL, lib.LINATTN_KERNEL_AUTO, args.segments):
+        need = lib.linattn_fwd_causal_workspace(B, H, N, d, d, WL.dtype)
+    ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    seg_launches = 2 if need > 0 else 1
 
     ops = wdist.LibraryOps(lib, stream)
 
@@ -251,8 +249,6 @@ def causal_leg(lib, args, world, rank, stream, hbm, tc_peak):
             # then the segment's forward from its starting state
             wdist.seq_parallel_causal(q, k, v, lam, WL.eps, world=world, rank=rank, seg_len=N,
                                       ops=ops)
-        elif ws is None:
-            lib.linattn_fwd_causal(q, k, v, lam, WL.eps, out, S, z, stream)
         else:
             lib.linattn_fwd_causal_ws(q, k, v, lam, WL.eps, None, None, out, S, z, ws, stream)
 
@@ -416,7 +412,7 @@ def tiny_leg(lib, args, world, rank, stream, hbm):
 def seg_leg(lib, args, world, rank, stream, hbm):
     """The causal_d64 workload (B=2, H=8, N=4096, d=64, bf16, no decay): the
     product path (the tensor-core kernel cut into about one segment per SM,
-    with its state pass and combine scan, through linattn_fwd_causal_ws), the
+    with its state pass, through linattn_fwd_causal_ws), the
     same kernel in one pass (16 CTAs), and for comparison the CUDA-core kernel
     in one pass and segmented."""
     w = inputs.WORKLOADS["causal_d64"]

@@ -91,7 +91,7 @@ constexpr uint32_t kSmemBytes = kOffMisc + kMiscBytes;
 static_assert(kSmemBytes <= 232448, "exceeds the per-CTA shared memory of sm_100");
 
 enum Bar {
-  kFullQK0 = 0, kFullQK1, kFullV0, kFullV1, kFreeQK0, kFreeQK1, kFreeV0, kFreeV1,
+  kFullQ0 = 0, kFullQ1, kFullK0, kFullK1, kFullV0, kFullV1, kFreeK0, kFreeK1, kFreeV0, kFreeV1,
   kPhi0, kPhi1, kScore, kRescale, kState, kReadout, kPDone, kO, kOut, kSop,
   kQFree0, kQFree1,   // the score epilogue has read the phi(q).z parts left in q tile s
   // den buffer b (chunk c uses b = c % 3): phi(q).z written, row sums added, read by the output
@@ -178,8 +178,11 @@ __global__ void __launch_bounds__(NT, 1)
     if (tid == 0) atomicOr(&g_status, kStatusWaitTimeout);
     return;
   }
-  const long pair = blockIdx.x / G;
-  const int g = blockIdx.x % G;
+  // segment-major: the first segments' CTAs come first, so they start
+  // while the state pass of the previous launch is still running
+  const long BH = gridDim.x / G;
+  const int g = static_cast<int>(blockIdx.x / BH);
+  const long pair = blockIdx.x % BH;
   const int h = static_cast<int>(pair % H);
   const float L = lam ? lam[h] : 1.f;
   const int n0 = g * seg_len;
@@ -187,13 +190,35 @@ __global__ void __launch_bounds__(NT, 1)
   const int nchunks = (n1 - n0 + C - 1) / C;
   const int Ct = (n1 - n0) - (nchunks - 1) * C;   // valid tokens of the last chunk
   const bool last_seg = g == G - 1;
-  // this head's starting state: the caller's (first segment) or the scanned
-  // carry of slot g of the workspace
-  const float *S0 = g == 0 ? (S_init ? S_init + pair * DK * static_cast<long>(DV) : nullptr)
-                           : ws_S + (pair * G + g) * static_cast<long>(DK) * DV;
-  const float *z0 = g == 0 ? (z_init ? z_init + pair * static_cast<long>(DK) : nullptr)
-                           : ws_z + (pair * G + g) * static_cast<long>(DK);
-  const bool has_init = S0 != nullptr;
+  // this head's starting state: the caller's (S_init, first segment) or the
+  // carry into segment g, summed here from the states of segments 0..g-1
+  // that the state pass left in slots pair G + j of the workspace:
+  //   S0_g = sum_j lambda^((g-1-j) len) dS_j + lambda^(g len) S_init
+  // (every segment before g holds len tokens).  Those CTAs wait for the
+  // state pass, which they may overlap when launched as its dependent.
+  const float *Sin = S_init ? S_init + pair * DK * static_cast<long>(DV) : nullptr;
+  const float *zin = z_init ? z_init + pair * static_cast<long>(DK) : nullptr;
+  const bool has_init = g > 0 || Sin != nullptr;
+  if (g > 0) grid_dependency_wait();
+  // four consecutive elements e..e+3 of the starting S (unit DK DV) or z
+  // (unit DK): the newest segment first, each older one lambda^len further back
+  const float Llen = g > 0 ? pow_int(L, seg_len) : 1.f;
+  auto carry4 = [&](const float *init, const float *slots, long unit, long e) {
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    float f = 1.f;
+    for (int j = g - 1; j >= 0; --j) {
+      const float4 v = *reinterpret_cast<const float4 *>(slots + (pair * G + j) * unit + e);
+      acc = make_float4(fmaf(f, v.x, acc.x), fmaf(f, v.y, acc.y), fmaf(f, v.z, acc.z),
+                        fmaf(f, v.w, acc.w));
+      f *= Llen;
+    }
+    if (init) {
+      const float4 v = *reinterpret_cast<const float4 *>(init + e);
+      acc = make_float4(fmaf(f, v.x, acc.x), fmaf(f, v.y, acc.y), fmaf(f, v.z, acc.z),
+                        fmaf(f, v.w, acc.w));
+    }
+    return acc;
+  };
   const bool factored = L >= kFactorMin;
   // factored decay keeps the state in a frame of R chunks (see frame_chunks)
   const int R = factored ? frame_chunks(L) : 1;
@@ -223,7 +248,14 @@ __global__ void __launch_bounds__(NT, 1)
     tmem_relinquish();
   }
   if (tid <= C) pw[tid] = pow_int(L, tid);
-  if (tid < 128) zs[tid] = (z0 && tid < DK) ? z0[tid] : 0.f;
+  if (tid < DK / 4) {
+    const float4 z4 = g > 0 ? carry4(zin, ws_z, DK, 4 * tid)
+                            : (zin ? reinterpret_cast<const float4 *>(zin)[tid]
+                                   : make_float4(0.f, 0.f, 0.f, 0.f));
+    reinterpret_cast<float4 *>(zs)[tid] = z4;
+  } else if (tid < 32) {
+    reinterpret_cast<float4 *>(zs)[tid] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
   if (DKP == 1) {
     // the second d_k panel of the q and k tiles stays zero (the state MMA
     // reads it as rows 64-127 of phi(K)^T; the other chains never do)
@@ -240,47 +272,91 @@ __global__ void __launch_bounds__(NT, 1)
   const uint32_t tmem = *tmem_slot;
   auto fail = [&]() { *abort_flag = 1; };
 
-  if (warp == 0 || warp == 2) {
-    // ------------------------------------------------------ TMA producers
+  // Starting state, written by every warp (warp w: TMEM lane quarter w % 4,
+  // d_v slice w / 4 of DV / 8 columns), so that the carry summed from the
+  // state pass's slots costs a few loads per thread: operand S' = S0;
+  // explicit decay: D_S = lambda^Cv0 S0 (the state MMA adds chunk 0 onto the
+  // decayed state); factored: D_S = S0, the first frame starting at the
+  // segment's first token.  Rows d_k..127 of D_S are zero.
+  if (has_init && nchunks > 0) {
+    constexpr int SC = DV / 8;                  // 16 or 8 columns
+    const int r = (warp & 3) * 32 + lane;       // d_k row, TMEM lane
+    const int c0 = (warp >> 2) * SC;
+    const bool live = r < DK;
+    const float g0 = factored ? 1.f : pw[Cv_of(0)];
+    uint32_t v[SC], sv[SC];
+#pragma unroll
+    for (int i = 0; i < SC / 4; ++i) {
+      float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (live) {
+        const long e = static_cast<long>(r) * DV + c0 + 4 * i;
+        f = g == 0 ? *reinterpret_cast<const float4 *>(Sin + e)
+                   : carry4(Sin, ws_S, static_cast<long>(DK) * DV, e);
+      }
+      v[4 * i] = __float_as_uint(f.x);
+      v[4 * i + 1] = __float_as_uint(f.y);
+      v[4 * i + 2] = __float_as_uint(f.z);
+      v[4 * i + 3] = __float_as_uint(f.w);
+    }
+#pragma unroll
+    for (int i = 0; i < SC; ++i) sv[i] = __float_as_uint(__uint_as_float(v[i]) * g0);
+    const uint32_t ta = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16) + kTmS + c0;
+    if constexpr (SC == 16) tmem_st_32x32b_x16(ta, sv);
+    else tmem_st_32x32b_x8(ta, sv);
+    uint32_t pk[SC / 2];
+#pragma unroll
+    for (int i = 0; i < SC / 2; ++i)
+      pk[i] = pack_bf16(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+#pragma unroll
+    for (int i = 0; i < SC / 8; ++i)
+      *reinterpret_cast<uint4 *>(sm + kOffSop + (c0 >> 6) * kPanel +
+                                 sw128_offset(r, (c0 & 63) * 2 + i * 16)) =
+          make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+    tmem_wait_st();
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+
+  if (warp == 0 || warp == 2 || warp == 3) {
+    // ------------------------------------------- TMA producers: q, v, k
+    // k is read by the score and state products, v by the state and P V
+    // products.  The q tile is read only by the feature map, but loading
+    // q(c + 2) lets the feature map overwrite phi(Q') of stage s in TMEM, so
+    // the q ring also waits for the MMAs of chunk c to be done with it (the
+    // k ring's release) and for the score epilogue to have taken the
+    // phi(q).z parts left in the tile.
     if (lane == 0 && nchunks > 0) {
-      const bool qk = warp == 0;
+      const int which = warp == 0 ? 0 : (warp == 3 ? 1 : 2);
+      const CUtensorMap *map = which == 0 ? &tm_q : (which == 1 ? &tm_k : &tm_v);
+      const uint32_t off = which == 0 ? kOffQ : (which == 1 ? kOffK : kOffV);
+      const int np = which == 2 ? DVP : DKP;
+      const int full0 = which == 0 ? kFullQ0 : (which == 1 ? kFullK0 : kFullV0);
+      const int free0 = which == 0 ? kQFree0 : (which == 1 ? kFreeK0 : kFreeV0);
       int issued = 0;
       for (int c = 0; c < nchunks && !*abort_flag; ++c) {
         const int s = c & 1;
-        if (c >= 2 && (!mbar_wait(bar((qk ? kFreeQK0 : kFreeV0) + s), ((c - 2) >> 1) & 1) ||
-                       (qk && !mbar_wait(bar(kQFree0 + s), ((c - 2) >> 1) & 1)))) {
+        if (c >= 2 && (!mbar_wait(bar(free0 + s), ((c - 2) >> 1) & 1) ||
+                       (which == 0 && !mbar_wait(bar(kFreeK0 + s), ((c - 2) >> 1) & 1)))) {
           fail();
           break;
         }
-        const uint32_t base = sb + s * kStage;
         const int y = n0 + c * C;
-        if (qk) {
-          const uint32_t b = bar(kFullQK0 + s);
-          mbar_arrive_expect_tx(b, 2 * DKP * kPanel);
-          for (int p = 0; p < DKP; ++p) {
-            tma_load_3d(base + kOffQ + p * kPanel, &tm_q, b, 64 * p, y, static_cast<int>(pair));
-            tma_load_3d(base + kOffK + p * kPanel, &tm_k, b, 64 * p, y, static_cast<int>(pair));
-          }
-          if (c + 2 < nchunks)
-            for (int p = 0; p < DKP; ++p) {
-              tma_prefetch_l2_3d(&tm_q, 64 * p, y + 2 * C, static_cast<int>(pair));
-              tma_prefetch_l2_3d(&tm_k, 64 * p, y + 2 * C, static_cast<int>(pair));
-            }
-        } else {
-          const uint32_t b = bar(kFullV0 + s);
-          mbar_arrive_expect_tx(b, DVP * kPanel);
-          for (int p = 0; p < DVP; ++p)
-            tma_load_3d(base + kOffV + p * kPanel, &tm_v, b, 64 * p, y, static_cast<int>(pair));
-          if (c + 2 < nchunks)
-            for (int p = 0; p < DVP; ++p)
-              tma_prefetch_l2_3d(&tm_v, 64 * p, y + 2 * C, static_cast<int>(pair));
-        }
+        const uint32_t b = bar(full0 + s);
+        mbar_arrive_expect_tx(b, np * kPanel);
+        for (int p = 0; p < np; ++p)
+          tma_load_3d(sb + s * kStage + off + p * kPanel, map, b, 64 * p, y,
+                      static_cast<int>(pair));
+        if (c + 2 < nchunks)
+          for (int p = 0; p < np; ++p)
+            tma_prefetch_l2_3d(map, 64 * p, y + 2 * C, static_cast<int>(pair));
         issued = c + 1;
       }
       if (*abort_flag) {
         // let the copies this thread started land before the CTA exits
         for (int c = issued - 2 < 0 ? 0 : issued - 2; c < issued; ++c)
-          mbar_wait(bar((qk ? kFullQK0 : kFullV0) + (c & 1)), (c >> 1) & 1);
+          mbar_wait(bar(full0 + (c & 1)), (c >> 1) & 1);
       }
     }
     __syncwarp();
@@ -340,7 +416,7 @@ __global__ void __launch_bounds__(NT, 1)
           umma_bf16(tmem + kTmS, kmn0 + ks * (2048 >> 4), v0 + ks * (2048 >> 4), idS,
                     (carried || ks > 0) ? 1u : 0u);
         umma_commit(bar(kState));
-        umma_commit(bar(kFreeQK0 + s));   // q, k tiles and phi(Q') of this chunk fully read
+        umma_commit(bar(kFreeK0 + s));    // k tile and phi(Q') of this chunk fully read
         // intra: D_O += P V
         if (!mbar_wait(bar(kPDone), c & 1)) { ok = false; break; }
         tc_fence_after();
@@ -505,31 +581,7 @@ __global__ void __launch_bounds__(NT, 1)
                                    sw128_offset(r, (col & 63) * 2 + i * 16)) =
             make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
     };
-    // starting state, operand S' = S0.  Explicit decay: D_S = lambda^Cv0 S0
-    // (the state MMA adds chunk 0 onto the decayed state); factored: D_S = S0,
-    // the first frame starting at the segment's first token.
-    if (has_init && nchunks > 0) {
-      const float g0 = factored ? 1.f : pw[Cv_of(0)];
-      const float *src = S0 + (live ? r : 0) * static_cast<long>(DV);
-#pragma unroll 1
-      for (int blk = 0; blk < DV / 16; ++blk) {
-        uint32_t v16[16], sv[16];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float4 f = live ? reinterpret_cast<const float4 *>(src)[blk * 4 + i]
-                                : make_float4(0.f, 0.f, 0.f, 0.f);
-          v16[4 * i] = __float_as_uint(f.x);
-          v16[4 * i + 1] = __float_as_uint(f.y);
-          v16[4 * i + 2] = __float_as_uint(f.z);
-          v16[4 * i + 3] = __float_as_uint(f.w);
-        }
-#pragma unroll
-        for (int i = 0; i < 16; ++i) sv[i] = __float_as_uint(__uint_as_float(v16[i]) * g0);
-        tmem_st_32x32b_x16(tmem + lf + kTmS + blk * 16, sv);
-        put_op(blk, v16, 1.f);
-      }
-      tmem_wait_st();
-    }
+    // the starting state (D_S and S') was written by every warp before the roles began
     fence_proxy_async_smem();
     tc_fence_before();
     named_bar_sync(kBarState, 128);
@@ -657,7 +709,7 @@ __global__ void __launch_bounds__(NT, 1)
       if (c > 0 && zowner)
         zs[zcol] = factored ? (frame_start ? gR : 1.f) * (zs[zcol] + ztot)
                             : pw[Cv_of(c - 1)] * zs[zcol] + ztot;
-      if (tt == 0) check(mbar_wait(bar(kFullQK0 + s), (c >> 1) & 1));
+      if (tt == 0) check(mbar_wait(bar(kFullQ0 + s), (c >> 1) & 1));
       named_bar_sync(kBarPhi, kPhiThreads);
       if (rf) break;
       // (1) q rows: feature map, decay scale, phi(q).z_{c-1}
@@ -698,6 +750,15 @@ __global__ void __launch_bounds__(NT, 1)
       // (2) k: feature map, decay weights (factored), column sums for z
       // factored k weight lambda^(n_f - 1 - p) = Fk lambda^(C - 1 - s)
       const float Fk = factored ? 1.f / (Eq * pw[C]) : 1.f;
+      // the k tile has its own ring: every warp checks that it has landed
+      {
+        bool okk = true;
+        if (lane == 0) okk = mbar_wait(bar(kFullK0 + s), (c >> 1) & 1);
+        if (!__shfl_sync(0xffffffffu, okk, 0)) {
+          rf = 1;
+          fail();
+        }
+      }
       if (kwarp) {
         float csum[8];
 #pragma unroll
@@ -839,6 +900,9 @@ __global__ void __launch_bounds__(sp::NT, 1)
     if (tid == 0) atomicOr(&g_status, kStatusWaitTimeout);
     return;
   }
+  // the forward launched after this grid as its dependent may start its
+  // first segments' CTAs now (they do not read this grid's output)
+  grid_launch_dependents();
   const long pair = blockIdx.x / nseg;
   const int g = blockIdx.x % nseg;
   const long slot = pair * slots + g;

@@ -211,6 +211,9 @@ struct Segments {
   float *ws = nullptr;
 };
 constexpr int kMaxSegments = 64;
+// time per token of the tensor-core state pass relative to the forward
+// (measured on the causal_decay_d128 workload); sets the split of two segments
+constexpr double kStatePassCost = 0.4;
 
 int simt_dv_slice(int dv) { return dv <= 16 ? 16 : 32; }
 
@@ -298,6 +301,24 @@ struct TcSegments {
   int G = 1, len = 0;
 };
 
+// Launch configuration with programmatic stream serialization: the grid may
+// begin before the previous grid of the stream has finished, and orders
+// itself after it with griddepcontrol.wait where it reads that grid's output.
+struct ProgrammaticLaunch {
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  ProgrammaticLaunch(int grid, int block, size_t smem, cudaStream_t s) {
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  }
+};
+
 TcSegments plan_tc_segments(const linattn_dims *d) {
   TcSegments sg;
   sg.len = d->N;
@@ -306,13 +327,19 @@ TcSegments plan_tc_segments(const linattn_dims *d) {
   const int sms = num_sms();
   if (BH <= 0 || nch < 2 || sms <= 0) return sg;
   long gmax = g_forced_segments.load(std::memory_order_relaxed);
-  if (gmax <= 0) {
-    gmax = sms / BH;               // about one CTA per SM
-    if (gmax < 3) return sg;       // the state pass re-reads k and v: not worth it for 2
-  }
+  if (gmax <= 0) gmax = sms / BH;   // about one CTA per SM
   gmax = std::min<long>(gmax, std::min(nch, kMaxSegments));
   if (gmax < 2) return sg;
-  const int len_ch = (nch + static_cast<int>(gmax) - 1) / static_cast<int>(gmax);
+  int len_ch;
+  if (gmax == 2) {
+    // Two segments: the first runs beside the state pass over itself, the
+    // second after it, so the first is longer by the state pass's share:
+    // len0 (1 - a) = len1 with a the state pass's cost per token relative
+    // to the forward's.
+    len_ch = static_cast<int>(std::ceil(nch / (2.0 - kStatePassCost)));
+  } else {
+    len_ch = (nch + static_cast<int>(gmax) - 1) / static_cast<int>(gmax);
+  }
   sg.G = (nch + len_ch - 1) / len_ch;
   sg.len = len_ch * stc::C;
   if (sg.G < 2) sg = TcSegments{1, d->N};
@@ -336,20 +363,26 @@ int launch_causal_seg_tc_t(const linattn_dims *d, const CUtensorMap &mq, const C
   if (sg.G > 1) {
     wsS = ws;
     wsz = ws + static_cast<long>(BH) * sg.G * d->dk * d->dv;
-    // (1) each segment's own final state from zero, (2) the starting states
+    // each of the first G - 1 segments' own final state from zero; the
+    // forward sums them into its starting states
     auto *sk = stc::causal_seg_state_tc_kernel<DKP, DVP>;
     if (!set_smem(sk, static_cast<int>(stc::sp::kSmemBytes))) return LINATTN_ERR_CUDA;
     sk<<<BH * (sg.G - 1), stc::sp::NT, stc::sp::kSmemBytes, s>>>(
         mk, mv, lam, wsS, wsz, d->H, d->N, sg.len, sg.G - 1, sg.G, ident(d));
     if (cudaGetLastError() != cudaSuccess) return LINATTN_ERR_CUDA;
-    const int eblocks = (d->dk * d->dv + d->dk + 255) / 256;
-    causal_seg_combine_kernel<<<dim3(BH, eblocks), 256, 0, s>>>(
-        lam, S_init, z_init, wsS, wsz, d->H, d->dk, d->dv, d->N, sg.len, sg.G, false);
-    if (cudaGetLastError() != cudaSuccess) return LINATTN_ERR_CUDA;
+    // the forward as the state pass's dependent: its first segment's CTAs
+    // run beside the state pass, the others wait for it (griddepcontrol)
+    ProgrammaticLaunch pl(BH * sg.G, stc::NT, stc::kSmemBytes, s);
+    if (cudaLaunchKernelEx(&pl.cfg, kern, mq, mk, mv, lam, eps, S_init, z_init,
+                           static_cast<const float *>(wsS), static_cast<const float *>(wsz),
+                           static_cast<bf16 *>(out), S_final, z_final, d->H, d->N, sg.len, sg.G,
+                           ident(d)) != cudaSuccess)
+      return LINATTN_ERR_CUDA;
+    return launch_status();
   }
-  kern<<<BH * sg.G, stc::NT, stc::kSmemBytes, s>>>(
-      mq, mk, mv, lam, eps, S_init, z_init, wsS, wsz, static_cast<bf16 *>(out), S_final, z_final,
-      d->H, d->N, sg.len, sg.G, ident(d));
+  kern<<<BH, stc::NT, stc::kSmemBytes, s>>>(
+      mq, mk, mv, lam, eps, S_init, z_init, nullptr, nullptr, static_cast<bf16 *>(out), S_final,
+      z_final, d->H, d->N, sg.len, 1, ident(d));
   return launch_status();
 }
 
@@ -438,24 +471,6 @@ bool use_tc_global(const linattn_dims *d) {
   if (choice(LINATTN_OP_GLOBAL) == LINATTN_KERNEL_CUDA_CORES) return false;
   return d->dtype == LINATTN_BF16 && d->dk == gtc::D && d->dv == gtc::D && d->H % 2 == 0;
 }
-
-// Launch configuration with programmatic stream serialization: the grid may
-// begin before the previous grid of the stream has finished, and orders
-// itself after it with griddepcontrol.wait where it reads that grid's output.
-struct ProgrammaticLaunch {
-  cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
-  ProgrammaticLaunch(int grid, int block, size_t smem, cudaStream_t s) {
-    cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(block);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = s;
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-  }
-};
 
 // KV and ksum to zero in one launch
 int zero_kv(float *KV, size_t nS, float *ksum, size_t nz, cudaStream_t s) {
