@@ -262,10 +262,16 @@ def causal_leg(lib, args, world, rank, stream, hbm, tc_peak):
     value = tokens / (ms / 1e3)
     alg = causal_bytes(B, H, N, d, d)
     flops = causal_mma_flops(B, H, N, d, d)
+    # DRAM bytes of one step: the forward, plus the state pass when the step has one
     traffic = traffic_record("causal_seg_tc_kernel")
+    if traffic is not None and seg_launches == 2:
+        sp = traffic_record("causal_seg_state_tc_kernel")
+        traffic = None if sp is None else traffic + sp
     roof = {"bound": "hbm", "achieved": alg / per_launch_s / 1e9, "peak": hbm, "unit": "GB/s",
             "frac": alg / per_launch_s / 1e9 / hbm, "traffic": traffic,
-            "algorithmic_bytes_per_launch": alg, "kernel": "causal_seg_tc_kernel",
+            "algorithmic_bytes_per_launch": alg,
+            "kernel": ("causal_seg_state_tc_kernel + causal_seg_tc_kernel (overlapped; timed as one step)"
+                       if seg_launches == 2 else "causal_seg_tc_kernel"),
             "tensor": {"mma_tflops": flops / per_launch_s / 1e12, "peak": tc_peak,
                        "frac": flops / per_launch_s / 1e12 / tc_peak,
                        "mma_flops_per_launch": flops}}
