@@ -12,10 +12,10 @@
 //   phi(k) tiles of both heads stacked along M (2 x 64 = 128 rows, MN-major)
 //   and the v tiles side by side along N, D[128 x 128] += phi(K)^T V holds
 //   both heads' KV on its diagonal blocks (the off-diagonal blocks are
-//   discarded); the feature-map threads keep the column sums of phi(k)
-//   (ksum) in registers.  Each CTA accumulates over a contiguous range of
-//   128-token chunks and adds its partial sums into the caller's (zeroed) KV /
-//   ksum with vector fp32 reductions whenever its range leaves a head pair.
+//   discarded), and D2[128 x 16] += phi(K)^T 1 holds both ksum.  Each CTA
+//   accumulates in TMEM over a contiguous range of 128-token chunks and adds
+//   its partial sums into the caller's (zeroed) KV / ksum with vector fp32
+//   reductions whenever its range leaves a head pair.
 //
 // global_out_tc_kernel: per 128-token tile of one head,
 //   [O | qz_hi, qz_lo] = phi(Q) [KV | ksum_hi, ksum_lo]   (N = 80, K = 64)
@@ -56,18 +56,17 @@ __device__ __forceinline__ uint32_t phi2(uint32_t x) {
 // or past `valid` become 0 when zero_tail (rows the TMA filled with zeros), and
 // so do rows whose byte in `pad` (the tile's 128 rows of the key padding
 // mask, or NULL) is nonzero.
-template <int U = 4>
 __device__ __forceinline__ void phi_tile(uint8_t *p, uint32_t bytes, int valid, bool zero_tail,
                                          bool ident, int tid, int nthr,
                                          const uint8_t *pad = nullptr) {
   const uint32_t step = static_cast<uint32_t>(nthr) * 16u;
-  for (uint32_t o0 = static_cast<uint32_t>(tid) * 16u; o0 < bytes; o0 += U * step) {
-    uint4 w[U];
+  for (uint32_t o0 = static_cast<uint32_t>(tid) * 16u; o0 < bytes; o0 += 4 * step) {
+    uint4 w[4];
 #pragma unroll
-    for (int i = 0; i < U; ++i)
+    for (int i = 0; i < 4; ++i)
       if (o0 + i * step < bytes) w[i] = *reinterpret_cast<const uint4 *>(p + o0 + i * step);
 #pragma unroll
-    for (int i = 0; i < U; ++i) {
+    for (int i = 0; i < 4; ++i) {
       const uint32_t o = o0 + i * step;
       const int row = static_cast<int>((o % kPanel) >> 7);
       const bool dead = (zero_tail && row >= valid) || (pad && row < valid && pad[row]);
@@ -77,7 +76,7 @@ __device__ __forceinline__ void phi_tile(uint8_t *p, uint32_t bytes, int valid, 
       w[i].w = dead ? 0u : ident ? w[i].w : phi2(w[i].w);
     }
 #pragma unroll
-    for (int i = 0; i < U; ++i)
+    for (int i = 0; i < 4; ++i)
       if (o0 + i * step < bytes) *reinterpret_cast<uint4 *>(p + o0 + i * step) = w[i];
   }
 }
@@ -107,11 +106,12 @@ struct UnitCursor {
 namespace kv {
 constexpr int kStages = 3;
 constexpr uint32_t kStage = 4 * kPanel;            // k head0, k head1, v head0, v head1
-constexpr uint32_t kOffMisc = kStages * kStage;
+constexpr uint32_t kOffW = kStages * kStage;       // [1; 0 ...] 16 x 128 K-major, 2 x 2 KB
+constexpr uint32_t kOffMisc = kOffW + 4096;
 constexpr uint32_t kSmemBytes = kOffMisc + 512;
 constexpr int NT = 384;                            // warp 0 TMA, 1 MMA, 4-11 phi + flush
 constexpr int kXform = 256;
-constexpr uint32_t kTmKV = 0, kTmCols = 128;
+constexpr uint32_t kTmKV = 0, kTmKS = 128, kTmCols = 256;
 enum { kFull = 0, kPhi = kStages, kEmpty = 2 * kStages, kFlushReady = 3 * kStages, kFlushDone,
        kFinal, kNumBars };
 constexpr uint32_t kMiscTmem = 128, kMiscFail = 132, kMiscRoleFail = 136;
@@ -155,6 +155,12 @@ __global__ void __launch_bounds__(kv::NT, 1)
     tmem_alloc(smem_u32(tmem_slot), kTmCols);
     tmem_relinquish();
   }
+  for (uint32_t o = tid * 16u; o < 4096u; o += NT * 16u) {
+    const bool row0 = ((o & 2047u) >> 7) == 0;
+    const uint32_t one2 = 0x3F803F80u;
+    *reinterpret_cast<uint4 *>(sm + kOffW + o) =
+        row0 ? make_uint4(one2, one2, one2, one2) : make_uint4(0, 0, 0, 0);
+  }
   fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
@@ -194,15 +200,12 @@ __global__ void __launch_bounds__(kv::NT, 1)
     __syncwarp();
   } else if (warp == 1) {
     if (lane == 0) {
-      const uint32_t idkv = idesc_bf16(128, 128, 1, 1);
-      // A = [phi(k) head0 | head1]^T (M = 128: d_k of both heads, MN-major) and
-      // B = [v head0 | head1] per stage; a K step of 16 tokens adds 2048 bytes
-      const uint64_t dA = sdesc_sw128(sb, kPanel, 1024);
-      const uint64_t dB = sdesc_sw128(sb + 2 * kPanel, kPanel, 1024);
+      const uint32_t idkv = idesc_bf16(128, 128, 1, 1), idks = idesc_bf16(128, 16, 1, 0);
       int seg = 0;
       bool first = true;
       UnitCursor u(u0, nchunks);
-      for (int i = 0, s = 0; i < nmine; ++i, u.next(), s = s + 1 == kStages ? 0 : s + 1) {
+      for (int i = 0; i < nmine; ++i, u.next()) {
+        const int s = i % kStages;
         if (*fail || !mbar_wait(bar(kPhi + s), (i / kStages) & 1)) {
           *fail = 1;
           break;
@@ -212,12 +215,17 @@ __global__ void __launch_bounds__(kv::NT, 1)
           break;
         }
         tc_fence_after();
-        const uint64_t so = static_cast<uint64_t>(s) * (kStage >> 4);   // stage offset
-        const uint64_t a0 = dA + so, b0 = dB + so;
+        const uint32_t st = sb + s * kStage;
 #pragma unroll
-        for (int ks = 0; ks < C / 16; ++ks)
-          umma_bf16(tmem + kTmKV, a0 + ks * (2048 >> 4), b0 + ks * (2048 >> 4), idkv,
+        for (int ks = 0; ks < C / 16; ++ks) {
+          // A = [phi(k) head0 | head1]^T: M = 128 (d_k of both heads), MN-major
+          const uint64_t a = sdesc_sw128(st + ks * 2048, kPanel, 1024);
+          umma_bf16(tmem + kTmKV, a, sdesc_sw128(st + 2 * kPanel + ks * 2048, kPanel, 1024), idkv,
                     (!first || ks > 0) ? 1u : 0u);
+          umma_bf16(tmem + kTmKS, a,
+                    sdesc_sw128(sb + kOffW + (ks >> 2) * 2048 + (ks & 3) * 32, 16, 1024), idks,
+                    (!first || ks > 0) ? 1u : 0u);
+        }
         umma_commit(bar(kEmpty + s));
         first = false;
         if (seg_end(i, u)) {
@@ -232,16 +240,10 @@ __global__ void __launch_bounds__(kv::NT, 1)
     __syncwarp();
   } else if (warp >= 4) {
     const int tt = tid - 128;   // 0..255
-    // thread (head p of the pair, 8-column group cg, block rb of 8 rows): it
-    // applies phi to its 8 rows x 8 columns of the k tile and keeps the column
-    // sums of those features over the segment's units (ksum, reduced at the flush)
-    const int hp = tt >> 7, cg = tt & 7, rb = (tt & 127) >> 3;
-    float csum[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) csum[e] = 0.f;
     int seg = 0;
     UnitCursor u(u0, nchunks);
-    for (int i = 0, s = 0; i < nmine; ++i, u.next(), s = s + 1 == kStages ? 0 : s + 1) {
+    for (int i = 0; i < nmine; ++i, u.next()) {
+      const int s = i % kStages;
       if (*fail || !mbar_wait(bar(kFull + s), (i / kStages) & 1)) {
         *rfail = 1;
         *fail = 1;
@@ -250,30 +252,8 @@ __global__ void __launch_bounds__(kv::NT, 1)
       // the pair's two heads belong to one sequence: one row of the padding mask
       const uint8_t *pad =
           kpm ? kpm + (2L * u.group / H) * N + static_cast<long>(u.index) * C : nullptr;
-      if (!*rfail) {
-        uint8_t *tile = sm + s * kStage + hp * kPanel;
-        // every load of the thread's 8 rows in flight before the first store
-        uint4 w[8];
-#pragma unroll
-        for (int r8 = 0; r8 < 8; ++r8)
-          w[r8] = *reinterpret_cast<const uint4 *>(tile + sw128_offset(rb * 8 + r8, cg * 16));
-#pragma unroll
-        for (int r8 = 0; r8 < 8; ++r8) {
-          const int row = rb * 8 + r8;
-          const bool dead = row >= valid || (pad && pad[row]);
-          uint32_t e4[4] = {w[r8].x, w[r8].y, w[r8].z, w[r8].w};
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            e4[j] = dead ? 0u : ident ? e4[j] : phi2(e4[j]);
-            csum[2 * j] += __uint_as_float(e4[j] << 16);
-            csum[2 * j + 1] += __uint_as_float(e4[j] & 0xffff0000u);
-          }
-          w[r8] = make_uint4(e4[0], e4[1], e4[2], e4[3]);
-        }
-#pragma unroll
-        for (int r8 = 0; r8 < 8; ++r8)
-          *reinterpret_cast<uint4 *>(tile + sw128_offset(rb * 8 + r8, cg * 16)) = w[r8];
-      }
+      if (!*rfail)
+        phi_tile(sm + s * kStage, 2 * kPanel, valid, valid < C, ident, tt, kXform, pad);
       fence_proxy_async_smem();
       named_bar_sync(1, kXform);
       if (*rfail) break;
@@ -290,39 +270,27 @@ __global__ void __launch_bounds__(kv::NT, 1)
         named_bar_sync(1, kXform);
         if (*rfail) break;
         tc_fence_after();
-        grid_dependency_wait();   // KV and ksum have been zeroed
         if (warp < 8) {
+          grid_dependency_wait();   // KV and ksum have been zeroed
           const int row = (warp - 4) * 32 + lane;
           const int hsel = row >> 6, kk = row & 63;
           const long bh = 2L * u.group + hsel;
           const uint32_t lf = static_cast<uint32_t>((warp - 4) * 32) << 16;
-          uint32_t a[32];
+          uint32_t a[32], ksv[2];
           float *dst = KV + (bh * D + kk) * D;
 #pragma unroll
           for (int half = 0; half < 2; ++half) {
             tmem_ld_32x32b_x32(tmem + lf + kTmKV + hsel * 64 + half * 32, a);
+            if (half == 0) tmem_ld_32x32b_x2(tmem + lf + kTmKS, ksv);
             tmem_wait_ld();
 #pragma unroll
             for (int j = 0; j < 8; ++j)
               red_add_v4(dst + half * 32 + 4 * j, __uint_as_float(a[4 * j]),
                          __uint_as_float(a[4 * j + 1]), __uint_as_float(a[4 * j + 2]),
                          __uint_as_float(a[4 * j + 3]));
+            if (half == 0) atomicAdd(ksum + bh * D + kk, __uint_as_float(ksv[0]));
           }
         }
-        // ksum: the column sums of the four row blocks of this warp, then one
-        // reduction per warp into the caller's ksum
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          csum[e] += __shfl_xor_sync(0xffffffffu, csum[e], 8);
-          csum[e] += __shfl_xor_sync(0xffffffffu, csum[e], 16);
-        }
-        if (lane < 8) {
-          float *kd = ksum + (2L * u.group + hp) * D + cg * 8;
-          red_add_v4(kd, csum[0], csum[1], csum[2], csum[3]);
-          red_add_v4(kd + 4, csum[4], csum[5], csum[6], csum[7]);
-        }
-#pragma unroll
-        for (int e = 0; e < 8; ++e) csum[e] = 0.f;
         tc_fence_before();
         named_bar_sync(1, kXform);
         if (*rfail) break;
@@ -348,14 +316,12 @@ constexpr uint32_t kOffX = kOffB + 8192;                // [ksum_hi, ksum_lo, 0 
 constexpr uint32_t kOffY = kOffX + 8192;                // 2 y staging tiles
 constexpr uint32_t kOffMisc = kOffY + 2 * kPanel;
 constexpr uint32_t kSmemBytes = kOffMisc + 512;
-// warp 0 TMA loads, 1 MMA, 2 TMA stores, 4-7 and 12-15 the two epilogue
-// warpgroups (even and odd tiles), 8-11 phi
-constexpr int NT = 512;
-constexpr int kXform = 128;
+constexpr int NT = 512;   // warp 0 TMA loads, 1 MMA, 2 TMA stores, 4-7 epilogue, 8-15 phi
+constexpr int kXform = 256;
 constexpr uint32_t kTmCols = 256;   // two 128-column accumulators (80 used each)
 enum { kFull = 0, kPhi = kStages, kEmpty = 2 * kStages, kDFull = 3 * kStages, kDEmpty = kDFull + 2,
        kBReady = kDEmpty + 2, kYFull, kYFree = kYFull + 2, kFinal = kYFree + 2, kNumBars };
-constexpr uint32_t kMiscTmem = 256, kMiscFail = 260, kMiscXFail = 264, kMiscEFail = 268;  // +4
+constexpr uint32_t kMiscTmem = 256, kMiscFail = 260, kMiscXFail = 264, kMiscEFail = 268;
 }  // namespace out
 
 __global__ void __launch_bounds__(out::NT, 1)
@@ -391,8 +357,7 @@ __global__ void __launch_bounds__(out::NT, 1)
     for (int i = 0; i < kNumBars; ++i) mbar_init(bar(i), 1);
     *fail = 0;
     *xfail = 0;
-    efail[0] = 0;
-    efail[1] = 0;
+    *efail = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_y);
@@ -477,7 +442,7 @@ __global__ void __launch_bounds__(out::NT, 1)
       tma_store_wait_all();
     }
     __syncwarp();
-  } else if (warp >= 8 && warp < 12) {
+  } else if (warp >= 8) {
     const int tt = tid - 256;
     for (int i = 0; i < nmine; ++i) {
       const int s = i % kStages;
@@ -485,42 +450,24 @@ __global__ void __launch_bounds__(out::NT, 1)
         *xfail = 1;
         *fail = 1;
       }
-      // the whole 16 KB tile in flight at once: 8 chunks per thread
-      if (!*xfail && !ident)
-        phi_tile<8>(sm + kOffQ + s * kPanel, kPanel, C, false, false, tt, kXform);
+      if (!*xfail && !ident) phi_tile(sm + kOffQ + s * kPanel, kPanel, C, false, false, tt, kXform);
       fence_proxy_async_smem();
       named_bar_sync(1, kXform);
       if (*xfail) break;
       if (tt == 0) mbar_arrive(bar(kPhi + s));
     }
   } else if (warp >= 4) {
-    // two epilogue warpgroups, one for the even and one for the odd tiles
-    // (each with its own accumulator and staging tile, so one group's waits
-    // overlap the other's work): the group whose tile starts a head (re)builds
-    // the [KV | ksum] operand, then each turns its accumulator tiles into y
-    const int eg = warp >= 12 ? 1 : 0;                 // group = tile parity = accumulator
-    const int r = (warp & 3) * 32 + lane;
-    const uint32_t lf = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const int ebar = 2 + eg;
-    volatile int *gfail = efail + eg;                  // the group's own verdict
+    // epilogue warpgroup: (re)builds the [KV | ksum] operand at the start of
+    // every head, then turns each accumulator tile into y
+    const int r = (warp - 4) * 32 + lane;
+    const uint32_t lf = static_cast<uint32_t>((warp - 4) * 32) << 16;
     UnitCursor u(u0, ntiles);
-    if (eg == 1) u.next();
-    for (int i = eg; i < nmine; i += 2, u.next(), u.next()) {
+    for (int i = 0; i < nmine; ++i, u.next()) {
       const int d = i & 1;
       if (seg_start(i, u)) {
-        // the operand can be rewritten once every earlier MMA has completed:
-        // the one of tile i - 1 (the other group's accumulator) is the last
-        if (i >= 1) {
-          const bool okp = !*fail && mbar_wait(bar(kDFull + (d ^ 1)), ((i - 1) >> 1) & 1);
-          if (!okp) {
-            *gfail = 1;
-            *fail = 1;
-          }
-          named_bar_sync(ebar, 128);
-          if (*gfail) break;
-        }
-        // KV rows = d_k (K), 64 columns (N); KV and ksum are complete once
-        // the KV grid has finished
+        // every earlier MMA has completed (its tile was consumed below), so
+        // the operand can be rewritten: KV rows = d_k (K), 64 columns (N);
+        // KV and ksum are complete once the KV grid has finished
         grid_dependency_wait();
         const long bh = u.group;
         if (r < D) {
@@ -539,7 +486,7 @@ __global__ void __launch_bounds__(out::NT, 1)
           *reinterpret_cast<__nv_bfloat16 *>(sm + kOffX + sw128_offset(r, 2)) = lo;
         }
         fence_proxy_async_smem();
-        named_bar_sync(ebar, 128);
+        named_bar_sync(2, 128);
         if (r == 0) mbar_arrive(bar(kBReady));
       }
       // every thread decides before the barrier and reads the verdict after
@@ -548,12 +495,12 @@ __global__ void __launch_bounds__(out::NT, 1)
       // staging tile d must be free: the store of tile i-2 has read it
       if (ok && i >= 2 && r == 0) ok = mbar_wait(bar(kYFree + d), ((i >> 1) - 1) & 1);
       if (!ok) {
-        *gfail = 1;
+        *efail = 1;
         *fail = 1;
       }
       tc_fence_after();
-      named_bar_sync(ebar, 128);
-      if (*gfail) break;
+      named_bar_sync(2, 128);
+      if (*efail) break;
       {
         uint32_t o[32], qz[2];
         tmem_ld_32x32b_x2(tmem + lf + d * 128 + 64, qz);
@@ -578,7 +525,7 @@ __global__ void __launch_bounds__(out::NT, 1)
       }
       tc_fence_before();
       fence_proxy_async_smem();
-      named_bar_sync(ebar, 128);
+      named_bar_sync(2, 128);
       if (r == 0) {
         mbar_arrive(bar(kDEmpty + d));
         mbar_arrive(bar(kYFull + d));
