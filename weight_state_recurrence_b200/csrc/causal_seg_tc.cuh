@@ -72,6 +72,12 @@ constexpr int C = 128;
 constexpr int NT = 1024;
 constexpr int kPhiThreads = 512;
 constexpr int kBarPhi = 1, kBarP = 2, kBarOut = 3, kBarState = 4;   // named barriers
+// The thread of each multi-warp role that polls its mbarriers (the others wait
+// at the role's named barrier), placed so that the four schedulers of the SM
+// (warp % 4) each carry about the same number of polling warps: TMA q 0,
+// MMA 1, TMA v 2, TMA k 3, score epilogue warp 4, feature map warp 17,
+// state warp 14, output warp 11.
+constexpr int kPollPhi = 32, kPollState = 64, kPollOut = 96;
 constexpr float kFactorMin = 0.7f;
 
 constexpr uint32_t kPanel = 16384;              // 128 rows x 128 bytes (64 bf16)
@@ -337,8 +343,9 @@ __global__ void __launch_bounds__(NT, 1)
       int issued = 0;
       for (int c = 0; c < nchunks && !*abort_flag; ++c) {
         const int s = c & 1;
-        if (c >= 2 && (!mbar_wait(bar(free0 + s), ((c - 2) >> 1) & 1) ||
-                       (which == 0 && !mbar_wait(bar(kFreeK0 + s), ((c - 2) >> 1) & 1)))) {
+        // the stage is needed a chunk from now: wait without taking issue slots
+        if (c >= 2 && (!mbar_wait_backoff(bar(free0 + s), ((c - 2) >> 1) & 1) ||
+                       (which == 0 && !mbar_wait_backoff(bar(kFreeK0 + s), ((c - 2) >> 1) & 1)))) {
           fail();
           break;
         }
@@ -520,7 +527,7 @@ __global__ void __launch_bounds__(NT, 1)
     // rows are 128 or 256 bytes, so 32-byte stores need only the base aligned
     const bool out32 = (reinterpret_cast<uintptr_t>(out) & 31u) == 0;
     for (int c = 0; c < nchunks; ++c) {
-      if (t == 0 && (*abort_flag || !mbar_wait(bar(kO), c & 1) ||
+      if (t == kPollOut && (*abort_flag || !mbar_wait(bar(kO), c & 1) ||
                      !mbar_wait(bar(kDenRs0 + c % kDenBufs), (c / kDenBufs) & 1))) {
         rf = 1;
         fail();
@@ -555,7 +562,7 @@ __global__ void __launch_bounds__(NT, 1)
       tc_fence_before();
       named_bar_sync(kBarOut, 128);
       if (rf) break;
-      if (t == 0) {
+      if (t == kPollOut) {
         mbar_arrive(bar(kOut));
         mbar_arrive(bar(kDenFree0 + c % kDenBufs));
       }
@@ -585,7 +592,7 @@ __global__ void __launch_bounds__(NT, 1)
     fence_proxy_async_smem();
     tc_fence_before();
     named_bar_sync(kBarState, 128);
-    if (r == 0) {
+    if (r == kPollState) {
       mbar_arrive(bar(kSop));
       mbar_arrive(bar(kReadout));
     }
@@ -593,7 +600,7 @@ __global__ void __launch_bounds__(NT, 1)
     const float gR = factored && R < nchunks ? pow_int(L, R * C) : 1.f;
     for (int c = 0; c < nchunks; ++c) {
       const bool last = c == nchunks - 1;
-      if (r == 0 && (*abort_flag || !mbar_wait(bar(kState), c & 1))) {
+      if (r == kPollState && (*abort_flag || !mbar_wait(bar(kState), c & 1))) {
         rf = 1;
         fail();
       }
@@ -638,7 +645,7 @@ __global__ void __launch_bounds__(NT, 1)
       if (decay) {
         named_bar_sync(kBarState, 128);
         if (rf) break;
-        if (r == 0) mbar_arrive(bar(kSop));
+        if (r == kPollState) mbar_arrive(bar(kSop));
         if (!rf) {
           // (2) D_S <- gd D_S, before the next state MMA accumulates onto it
 #pragma unroll 1
@@ -655,12 +662,12 @@ __global__ void __launch_bounds__(NT, 1)
         tc_fence_before();
         named_bar_sync(kBarState, 128);
         if (rf) break;
-        if (r == 0) mbar_arrive(bar(kReadout));
+        if (r == kPollState) mbar_arrive(bar(kReadout));
       } else {
         tc_fence_before();
         named_bar_sync(kBarState, 128);
         if (rf) break;
-        if (r == 0 && !last) {
+        if (r == kPollState && !last) {
           mbar_arrive(bar(kSop));
           mbar_arrive(bar(kReadout));
         }
@@ -709,7 +716,7 @@ __global__ void __launch_bounds__(NT, 1)
       if (c > 0 && zowner)
         zs[zcol] = factored ? (frame_start ? gR : 1.f) * (zs[zcol] + ztot)
                             : pw[Cv_of(c - 1)] * zs[zcol] + ztot;
-      if (tt == 0) check(mbar_wait(bar(kFullQ0 + s), (c >> 1) & 1));
+      if (tt == kPollPhi) check(mbar_wait(bar(kFullQ0 + s), (c >> 1) & 1));
       named_bar_sync(kBarPhi, kPhiThreads);
       if (rf) break;
       // (1) q rows: feature map, decay scale, phi(q).z_{c-1}
@@ -796,14 +803,14 @@ __global__ void __launch_bounds__(NT, 1)
       tmem_wait_st();
       tc_fence_before();
       named_bar_sync(kBarPhi, kPhiThreads);
-      if (tt == 0) {
+      if (tt == kPollPhi) {
         mbar_arrive(bar(kPhi0 + s));
         mbar_arrive(bar(kDenQz0 + c % kDenBufs));
       }
       if (!factored) {
         // after the score MMA: q rows (TMEM) times lambda^(t+1), k rows (SMEM)
         // times lambda^(Cv-1-s)
-        if (tt == 0) check(mbar_wait(bar(kScore), c & 1));
+        if (tt == kPollPhi) check(mbar_wait(bar(kScore), c & 1));
         named_bar_sync(kBarPhi, kPhiThreads);
         if (rf) break;
         tc_fence_after();
@@ -834,7 +841,7 @@ __global__ void __launch_bounds__(NT, 1)
         tc_fence_before();
         fence_proxy_async_smem();
         named_bar_sync(kBarPhi, kPhiThreads);
-        if (tt == 0) mbar_arrive(bar(kRescale));
+        if (tt == kPollPhi) mbar_arrive(bar(kRescale));
       }
     }
     // the last chunk's column sums; factored: z = lambda^(tokens since the frame start) z~
@@ -950,7 +957,7 @@ __global__ void __launch_bounds__(sp::NT, 1)
       for (int c = 0; c < nchunks && !*abort_flag; ++c) {
         const int s = c % sp::kStages;
         if (c >= sp::kStages &&
-            !mbar_wait(bar(sp::kFree0 + s), ((c - sp::kStages) / sp::kStages) & 1)) {
+            !mbar_wait_backoff(bar(sp::kFree0 + s), ((c - sp::kStages) / sp::kStages) & 1)) {
           fail();
           break;
         }
@@ -1005,8 +1012,10 @@ __global__ void __launch_bounds__(sp::NT, 1)
     const int wq = warp - 4;
     const int r = wq * 32 + lane;
     const uint32_t lf = static_cast<uint32_t>(wq * 32) << 16;
-    // one thread polls for the whole pass; the others wait at the named barrier
-    if (r == 0 && (*abort_flag || !mbar_wait(bar(sp::kState), 0))) fail();
+    // one thread polls for the whole pass, sleeping between tries (warp 7,
+    // away from the TMA and feature-map pollers' schedulers); the others wait
+    // at the named barrier
+    if (r == 96 && (*abort_flag || !mbar_wait_backoff(bar(sp::kState), 0, 512))) fail();
     named_bar_sync(sp::kBarStore, 128);
     tc_fence_after();
     if (!*abort_flag) {
@@ -1047,7 +1056,7 @@ __global__ void __launch_bounds__(sp::NT, 1)
       uint8_t *st = sm + s * sp::kStage;
       // the previous chunk's column sums (already weighted to the segment end)
       if (c > 0 && zowner) zs[zcol] += ztot;
-      if (tt == 0 && (*abort_flag || !mbar_wait(bar(sp::kFull0 + s), (c / sp::kStages) & 1))) {
+      if (tt == 32 && (*abort_flag || !mbar_wait(bar(sp::kFull0 + s), (c / sp::kStages) & 1))) {
         rf = 1;
         fail();
       }
@@ -1087,7 +1096,7 @@ __global__ void __launch_bounds__(sp::NT, 1)
       }
       fence_proxy_async_smem();
       named_bar_sync(sp::kBarPhi, sp::kPhiThreads);
-      if (tt == 0) mbar_arrive(bar(sp::kPhi0 + s));
+      if (tt == 32) mbar_arrive(bar(sp::kPhi0 + s));
     }
     if (!rf && nchunks > 0 && zowner) zs[zcol] += ztot;
     named_bar_sync(sp::kBarPhi, sp::kPhiThreads);
