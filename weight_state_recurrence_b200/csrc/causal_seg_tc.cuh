@@ -460,6 +460,7 @@ __global__ void __launch_bounds__(NT, 1)
       named_bar_sync(kBarP, 128);
       tc_fence_after();
       float rs = 0.f;
+      float2 rs2 = make_float2(0.f, 0.f);   // the row sum, even and odd keys
       if (!rf) {
         // phi(q').z of row t: the feature-map warps left one part per column
         // block in q tile s, summed here in a fixed order
@@ -482,7 +483,7 @@ __global__ void __launch_bounds__(NT, 1)
               for (int i = 0; i < 16; ++i) {
                 const float a = __uint_as_float(r[2 * i]), b = __uint_as_float(r[2 * i + 1]);
                 pk[i] = pack_bf16(a, b);
-                rs += a + b;
+                rs2 = fadd2(rs2, make_float2(a, b));
               }
             } else {
 #pragma unroll
@@ -495,7 +496,7 @@ __global__ void __launch_bounds__(NT, 1)
                   b *= s_b <= t ? pw[t - s_b] : 0.f;
                 }
                 pk[i] = pack_bf16(a, b);
-                rs += a + b;
+                rs2 = fadd2(rs2, make_float2(a, b));
               }
             }
           } else {
@@ -507,7 +508,7 @@ __global__ void __launch_bounds__(NT, 1)
           tmem_st_32x32b_x16(tmem + lf + kTmA + bk * 16, pk);
         }
         tmem_wait_st();
-        den[(c % kDenBufs) * 128 + t] = rs;
+        den[(c % kDenBufs) * 128 + t] = rs + (rs2.x + rs2.y);
       }
       tc_fence_before();
       named_bar_sync(kBarP, 128);
@@ -546,8 +547,12 @@ __global__ void __launch_bounds__(NT, 1)
           tmem_wait_ld();
           uint32_t pk[16];
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            pk[i] = pack_bf16(__uint_as_float(r[2 * i]) * inv, __uint_as_float(r[2 * i + 1]) * inv);
+          for (int i = 0; i < 16; ++i) {
+            const float2 y2 = fmul2(
+                make_float2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])),
+                make_float2(inv, inv));
+            pk[i] = pack_bf16(y2.x, y2.y);
+          }
           if (live) {
             if (out32) {
               st_global_na_v8(dst + blk * 4, pk);
@@ -578,9 +583,19 @@ __global__ void __launch_bounds__(NT, 1)
     // 16 columns (block blk) of this d_k row as bf16 into the operand
     auto put_op = [&](int blk, const uint32_t (&v16)[16], float f) {
       uint32_t pk[8];
+      if (f == 1.f) {   // no renormalisation at this chunk: convert only
 #pragma unroll
-      for (int i = 0; i < 8; ++i)
-        pk[i] = pack_bf16(__uint_as_float(v16[2 * i]) * f, __uint_as_float(v16[2 * i + 1]) * f);
+        for (int i = 0; i < 8; ++i)
+          pk[i] = pack_bf16(__uint_as_float(v16[2 * i]), __uint_as_float(v16[2 * i + 1]));
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float2 y2 = fmul2(
+              make_float2(__uint_as_float(v16[2 * i]), __uint_as_float(v16[2 * i + 1])),
+              make_float2(f, f));
+          pk[i] = pack_bf16(y2.x, y2.y);
+        }
+      }
       const uint32_t col = blk * 16;     // first d_v column of this block
 #pragma unroll
       for (int i = 0; i < 2; ++i)
@@ -725,7 +740,7 @@ __global__ void __launch_bounds__(NT, 1)
         if (tq >= Cv) fq = 0.f;
         else fq = factored ? Eq * pw[tq + 1] : 1.f;
         const uint32_t f2 = pack_bf16(fq, fq);
-        float qz = 0.f;
+        float2 qz2 = make_float2(0.f, 0.f);   // phi(q').z, even and odd columns
         uint4 w[QCH];
 #pragma unroll
         for (int j = 0; j < QCH; ++j)
@@ -741,8 +756,8 @@ __global__ void __launch_bounds__(NT, 1)
           for (int i = 0; i < 4; ++i) {
             if (!ident) e[i] = phi_bf16x2(e[i]);
             e[i] = mul_bf16x2(e[i], f2);
-            qz = fmaf(bf_lo(e[i]), zz[2 * i], qz);
-            qz = fmaf(bf_hi(e[i]), zz[2 * i + 1], qz);
+            qz2 = ffma2(make_float2(bf_lo(e[i]), bf_hi(e[i])), make_float2(zz[2 * i], zz[2 * i + 1]),
+                        qz2);
             pk[4 * j + i] = e[i];
           }
         }
@@ -752,7 +767,7 @@ __global__ void __launch_bounds__(NT, 1)
         // part of this column block goes into the q bytes this thread alone
         // has read (the score epilogue sums the four parts of the row).
         *reinterpret_cast<float *>(st + kOffQ + chunk_off(tq, cb * QCH)) =
-            qz * (factored ? 1.f : (tq < Cv ? pw[tq + 1] : 0.f));
+            (qz2.x + qz2.y) * (factored ? 1.f : (tq < Cv ? pw[tq + 1] : 0.f));
       }
       // (2) k: feature map, decay weights (factored), column sums for z
       // factored k weight lambda^(n_f - 1 - p) = Fk lambda^(C - 1 - s)
@@ -789,8 +804,10 @@ __global__ void __launch_bounds__(NT, 1)
             // the explicit path keeps phi(k) unweighted for the score MMA; the
             // normaliser takes the weights here
             const float m = factored ? 1.f : wk;
-            csum[2 * q4] = fmaf(bf_lo(e[q4]), m, csum[2 * q4]);
-            csum[2 * q4 + 1] = fmaf(bf_hi(e[q4]), m, csum[2 * q4 + 1]);
+            const float2 c2 = ffma2(make_float2(bf_lo(e[q4]), bf_hi(e[q4])), make_float2(m, m),
+                                    make_float2(csum[2 * q4], csum[2 * q4 + 1]));
+            csum[2 * q4] = c2.x;
+            csum[2 * q4 + 1] = c2.y;
           }
           w[i] = make_uint4(e[0], e[1], e[2], e[3]);
         }

@@ -326,6 +326,30 @@ __device__ __forceinline__ void tmem_st_32x32b_x8(uint32_t taddr, const uint32_t
                : "memory");
 }
 
+// Packed fp32 pairs (two lanes of arithmetic per instruction on sm_100).
+__device__ __forceinline__ unsigned long long f2_bits(float2 a) {
+  return (static_cast<unsigned long long>(__float_as_uint(a.y)) << 32) | __float_as_uint(a.x);
+}
+__device__ __forceinline__ float2 f2_val(unsigned long long b) {
+  return make_float2(__uint_as_float(static_cast<uint32_t>(b)),
+                     __uint_as_float(static_cast<uint32_t>(b >> 32)));
+}
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
+  unsigned long long d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2_bits(a)), "l"(f2_bits(b)));
+  return f2_val(d);
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+  unsigned long long d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2_bits(a)), "l"(f2_bits(b)));
+  return f2_val(d);
+}
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  unsigned long long d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(f2_bits(a)), "l"(f2_bits(b)), "l"(f2_bits(c)));
+  return f2_val(d);
+}
+
 // Global stores that do not allocate in L1: 32 bytes (address 32-byte aligned)
 // or 16 bytes per thread.  Wide, non-allocating stores keep a warp that
 // writes 32 different rows from flooding the load/store pipe the rest of the
