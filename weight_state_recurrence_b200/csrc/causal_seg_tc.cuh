@@ -717,15 +717,24 @@ __global__ void __launch_bounds__(NT, 1)
     float ztot = 0.f;                         // this lane's share of the column sums
     const int zcol = cg * 8 + warp_sum8_index(lane);
     const bool zowner = kwarp && (lane & 3) == 0;
-    // factored: lambda^(tokens from the frame start to this chunk); explicit: unused
+    // factored: Eq = lambda^(tokens from the frame start to this chunk) and
+    // Fk = lambda^-(those tokens + C), both stepped by one factor per chunk
+    // (no division on the chunk's path; the product Eq Fk lambda^C stays
+    // within ~1e-5 of 1 over a frame, far below the bf16 rounding of the
+    // operands); explicit: unused
     float Eq = 1.f;
+    const float ipwC = factored ? 1.f / pw[C] : 1.f;
+    float Fk = ipwC;
     const float gR = factored && R < nchunks ? pow_int(L, R * C) : 1.f;
     for (int c = 0; c < nchunks; ++c) {
       const int s = c & 1;
       const int Cv = Cv_of(c);
       uint8_t *st = sm + s * kStage;
       const bool frame_start = c % R == 0;
-      if (factored) Eq = frame_start ? 1.f : Eq * pw[C];
+      if (factored) {
+        Eq = frame_start ? 1.f : Eq * pw[C];
+        Fk = frame_start ? ipwC : Fk * ipwC;
+      }
       // the previous chunk's column sums: explicit z_{c-1} = lambda^Cv z_{c-2} + sums;
       // factored z~ += sums, renormalised with the state when a frame starts
       if (c > 0 && zowner)
@@ -771,7 +780,6 @@ __global__ void __launch_bounds__(NT, 1)
       }
       // (2) k: feature map, decay weights (factored), column sums for z
       // factored k weight lambda^(n_f - 1 - p) = Fk lambda^(C - 1 - s)
-      const float Fk = factored ? 1.f / (Eq * pw[C]) : 1.f;
       // the k tile has its own ring: every warp checks that it has landed
       {
         bool okk = true;
