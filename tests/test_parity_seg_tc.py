@@ -138,3 +138,23 @@ def test_output_16_byte_aligned_only(cuda_lib):
     y_o, S_o, z_o = oracle.causal(q, k, v, lam, 1e-6)
     assert_close("y", out, y_o, 2e-2)
     assert_close("S_final", S, S_o, 2e-2)
+
+
+@pytest.mark.parametrize("G", [1, 2, 3])
+@pytest.mark.parametrize("with_init", [False, True])
+def test_factored_frames(cuda_lib, G, with_init):
+    """Factored decay keeps the state relative to a frame of
+    R = floor(64 / (128 log2(1/lambda))) chunks and renormalises at its end:
+    lambda = 0.7 (R = 1: every chunk, k weights near 2^66), 0.75 (R = 1),
+    0.85 (R = 2), 0.9 (R = 3), 0.99 (R = 34: one frame here), 0.9999; ten
+    chunks with a ragged last one, in one pass or cut into segments."""
+    N = 128 * 9 + 37
+    q, k, v = inputs.random_case(3400 + G + 10 * with_init, 1, 6, N, 128, 128, torch.bfloat16,
+                                 scale=128 ** -0.5)
+    lam = torch.tensor([0.7, 0.75, 0.85, 0.9, 0.99, 0.9999])
+    S0 = z0 = None
+    if with_init:
+        gen = torch.Generator().manual_seed(3450 + G)
+        S0 = torch.randn(1, 6, 128, 128, generator=gen) * 0.05
+        z0 = torch.rand(1, 6, 128, generator=gen) + 0.5
+    check(cuda_lib, q, k, v, lam, 1e-6, G, S0=S0, z0=z0)
