@@ -317,6 +317,9 @@ constexpr uint32_t kOffY = kOffX + 8192;                // 2 y staging tiles
 constexpr uint32_t kOffMisc = kOffY + 2 * kPanel;
 constexpr uint32_t kSmemBytes = kOffMisc + 512;
 constexpr int NT = 512;   // warp 0 TMA loads, 1 MMA, 2 TMA stores, 4-7 epilogue, 8-15 phi
+// Two CTAs share an SM (64 registers a thread, 2 x 115.2 KB of shared memory,
+// 2 x 256 TMEM columns), so one CTA's epilogue chain overlaps the other's.
+constexpr int kCtasPerSm = 2;
 constexpr int kXform = 256;
 constexpr uint32_t kTmCols = 256;   // two 128-column accumulators (80 used each)
 enum { kFull = 0, kPhi = kStages, kEmpty = 2 * kStages, kDFull = 3 * kStages, kDEmpty = kDFull + 2,
@@ -324,7 +327,7 @@ enum { kFull = 0, kPhi = kStages, kEmpty = 2 * kStages, kDFull = 3 * kStages, kD
 constexpr uint32_t kMiscTmem = 256, kMiscFail = 260, kMiscXFail = 264, kMiscEFail = 268;
 }  // namespace out
 
-__global__ void __launch_bounds__(out::NT, 1)
+__global__ void __launch_bounds__(out::NT, out::kCtasPerSm)
     global_out_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                          const __grid_constant__ CUtensorMap tm_y, const float *__restrict__ KV,
                          const float *__restrict__ ksum, float eps, int BH, int N,

@@ -491,8 +491,11 @@ int launch_global_tc(const linattn_dims *d, int Nk, const void *q, const void *k
   const int BH = d->B * d->H;
   const int sms = num_sms();
   if (sms <= 0) return LINATTN_ERR_CUDA;
+  // the output kernel runs two CTAs per SM: the largest shared-memory carveout
   if (!set_smem(gtc::global_kv_tc_kernel, static_cast<int>(gtc::kv::kSmemBytes)) ||
-      !set_smem(gtc::global_out_tc_kernel, static_cast<int>(gtc::out::kSmemBytes)))
+      !set_smem(gtc::global_out_tc_kernel, static_cast<int>(gtc::out::kSmemBytes)) ||
+      cudaFuncSetAttribute(gtc::global_out_tc_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                           cudaSharedmemCarveoutMaxShared) != cudaSuccess)
     return LINATTN_ERR_CUDA;
   if (Nk > 0) {
     CUtensorMap mk, mv;
@@ -514,7 +517,9 @@ int launch_global_tc(const linattn_dims *d, int Nk, const void *q, const void *k
     const long u2 = static_cast<long>(BH) * ((d->N + gtc::C - 1) / gtc::C);
     // the output grid loads q and applies phi while the KV grid drains; it
     // waits for that grid only before reading KV and ksum
-    const ProgrammaticLaunch pl(static_cast<int>(u2 < sms ? u2 : sms), gtc::out::NT,
+    // two persistent CTAs per SM (64 registers, 115 KB of shared memory each)
+    const int cap2 = gtc::out::kCtasPerSm * sms;
+    const ProgrammaticLaunch pl(static_cast<int>(u2 < cap2 ? u2 : cap2), gtc::out::NT,
                                 gtc::out::kSmemBytes, s);
     if (cudaLaunchKernelEx(&pl.cfg, gtc::global_out_tc_kernel, mq, my,
                            static_cast<const float *>(KV), static_cast<const float *>(ksum), eps,
