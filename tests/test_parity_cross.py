@@ -84,12 +84,16 @@ def test_cuda_core_path_masked(cuda_lib, dk, dv, dtype):
 
 
 def test_masked_without_mask_is_cross(cuda_lib):
+    """No mask: the same kernels as the cross form.  The KV kernel's CTAs add
+    their partial sums with float atomics, so the order of those adds (and the
+    last bits) may differ between calls: equal up to that rounding."""
     q, k, v = inputs.random_case(2100, 2, 4, 200, 64, 64, torch.bfloat16, scale=0.125)
     a = cuda_lib.fwd_global_masked(q.to(DEV), k.to(DEV), v.to(DEV), None, 1e-6)
     b = cuda_lib.fwd_global_cross(q.to(DEV), k.to(DEV), v.to(DEV), 1e-6)
     torch.cuda.synchronize()
-    for x, y in zip(a, b):
-        assert torch.equal(x, y)
+    # KV and ksum (fp32) to rounding; y (bf16) to a bf16 step or two
+    for name, x, y, tol in zip(("y", "KV", "ksum"), a, b, (8e-3, 1e-5, 1e-5)):
+        assert_close(f"masked vs cross {name}", x, y.double().cpu().numpy(), tol)
 
 
 def test_no_device_errors_recorded(cuda_lib):

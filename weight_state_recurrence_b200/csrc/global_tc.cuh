@@ -58,7 +58,8 @@ __device__ __forceinline__ uint32_t phi2(uint32_t x) {
 // mask, or NULL) is nonzero.
 __device__ __forceinline__ void phi_tile(uint8_t *p, uint32_t bytes, int valid, bool zero_tail,
                                          bool ident, int tid, int nthr,
-                                         const uint8_t *pad = nullptr) {
+                                         const uint8_t *pad = nullptr,
+                                         uint32_t panel = kPanel) {
   const uint32_t step = static_cast<uint32_t>(nthr) * 16u;
   for (uint32_t o0 = static_cast<uint32_t>(tid) * 16u; o0 < bytes; o0 += 4 * step) {
     uint4 w[4];
@@ -68,7 +69,7 @@ __device__ __forceinline__ void phi_tile(uint8_t *p, uint32_t bytes, int valid, 
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const uint32_t o = o0 + i * step;
-      const int row = static_cast<int>((o % kPanel) >> 7);
+      const int row = static_cast<int>((o % panel) >> 7);   // panels of `panel` bytes
       const bool dead = (zero_tail && row >= valid) || (pad && row < valid && pad[row]);
       w[i].x = dead ? 0u : ident ? w[i].x : phi2(w[i].x);
       w[i].y = dead ? 0u : ident ? w[i].y : phi2(w[i].y);
@@ -104,8 +105,14 @@ struct UnitCursor {
 
 // ============================================================= KV, ksum
 namespace kv {
+// Units of CK = 64 tokens of a head pair, so that the 3-deep ring (96 KB)
+// leaves room for two CTAs per SM (80 registers a thread, 2 x 256 TMEM
+// columns): one CTA's feature map and MMA chain overlap the other's.
+constexpr int CK = 64;
+constexpr uint32_t kPanelK = CK * 128;              // one head's [64 tokens x 64] bf16 tile, 8 KB
+constexpr int kCtasPerSm = 2;
 constexpr int kStages = 3;
-constexpr uint32_t kStage = 4 * kPanel;            // k head0, k head1, v head0, v head1
+constexpr uint32_t kStage = 4 * kPanelK;           // k head0, k head1, v head0, v head1
 constexpr uint32_t kOffW = kStages * kStage;       // [1; 0 ...] 16 x 128 K-major, 2 x 2 KB
 constexpr uint32_t kOffMisc = kOffW + 4096;
 constexpr uint32_t kSmemBytes = kOffMisc + 512;
@@ -117,7 +124,7 @@ enum { kFull = 0, kPhi = kStages, kEmpty = 2 * kStages, kFlushReady = 3 * kStage
 constexpr uint32_t kMiscTmem = 128, kMiscFail = 132, kMiscRoleFail = 136;
 }  // namespace kv
 
-__global__ void __launch_bounds__(kv::NT, 1)
+__global__ void __launch_bounds__(kv::NT, kv::kCtasPerSm)
     global_kv_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v,
                         const uint8_t *__restrict__ kpm, float *__restrict__ KV,
@@ -138,7 +145,7 @@ __global__ void __launch_bounds__(kv::NT, 1)
   // threads of the role take the same exit
   volatile int *rfail = reinterpret_cast<volatile int *>(sm + kOffMisc + kMiscRoleFail);
 
-  const int nchunks = (N + C - 1) / C;
+  const int nchunks = (N + CK - 1) / CK;
   const long units = static_cast<long>(npairs) * nchunks;
   const long u0 = units * blockIdx.x / gridDim.x, u1 = units * (blockIdx.x + 1) / gridDim.x;
   const int nmine = static_cast<int>(u1 - u0);
@@ -187,10 +194,10 @@ __global__ void __launch_bounds__(kv::NT, 1)
         const int p = u.group, c = u.index;
         const uint32_t st = sb + s * kStage, b = bar(kFull + s);
         mbar_arrive_expect_tx(b, kStage);
-        tma_load_3d(st, &tm_k, b, 0, c * C, 2 * p);
-        tma_load_3d(st + kPanel, &tm_k, b, 0, c * C, 2 * p + 1);
-        tma_load_3d(st + 2 * kPanel, &tm_v, b, 0, c * C, 2 * p);
-        tma_load_3d(st + 3 * kPanel, &tm_v, b, 0, c * C, 2 * p + 1);
+        tma_load_3d(st, &tm_k, b, 0, c * CK, 2 * p);
+        tma_load_3d(st + kPanelK, &tm_k, b, 0, c * CK, 2 * p + 1);
+        tma_load_3d(st + 2 * kPanelK, &tm_v, b, 0, c * CK, 2 * p);
+        tma_load_3d(st + 3 * kPanelK, &tm_v, b, 0, c * CK, 2 * p + 1);
         issued = i + 1;
       }
       if (*fail)   // let the copies still in flight land before the CTA exits
@@ -217,10 +224,10 @@ __global__ void __launch_bounds__(kv::NT, 1)
         tc_fence_after();
         const uint32_t st = sb + s * kStage;
 #pragma unroll
-        for (int ks = 0; ks < C / 16; ++ks) {
+        for (int ks = 0; ks < CK / 16; ++ks) {
           // A = [phi(k) head0 | head1]^T: M = 128 (d_k of both heads), MN-major
-          const uint64_t a = sdesc_sw128(st + ks * 2048, kPanel, 1024);
-          umma_bf16(tmem + kTmKV, a, sdesc_sw128(st + 2 * kPanel + ks * 2048, kPanel, 1024), idkv,
+          const uint64_t a = sdesc_sw128(st + ks * 2048, kPanelK, 1024);
+          umma_bf16(tmem + kTmKV, a, sdesc_sw128(st + 2 * kPanelK + ks * 2048, kPanelK, 1024), idkv,
                     (!first || ks > 0) ? 1u : 0u);
           umma_bf16(tmem + kTmKS, a,
                     sdesc_sw128(sb + kOffW + (ks >> 2) * 2048 + (ks & 3) * 32, 16, 1024), idks,
@@ -248,12 +255,12 @@ __global__ void __launch_bounds__(kv::NT, 1)
         *rfail = 1;
         *fail = 1;
       }
-      const int valid = N - u.index * C;
+      const int valid = N - u.index * CK;
       // the pair's two heads belong to one sequence: one row of the padding mask
       const uint8_t *pad =
-          kpm ? kpm + (2L * u.group / H) * N + static_cast<long>(u.index) * C : nullptr;
+          kpm ? kpm + (2L * u.group / H) * N + static_cast<long>(u.index) * CK : nullptr;
       if (!*rfail)
-        phi_tile(sm + s * kStage, 2 * kPanel, valid, valid < C, ident, tt, kXform, pad);
+        phi_tile(sm + s * kStage, 2 * kPanelK, valid, valid < CK, ident, tt, kXform, pad, kPanelK);
       fence_proxy_async_smem();
       named_bar_sync(1, kXform);
       if (*rfail) break;

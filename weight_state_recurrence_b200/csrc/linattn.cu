@@ -491,20 +491,26 @@ int launch_global_tc(const linattn_dims *d, int Nk, const void *q, const void *k
   const int BH = d->B * d->H;
   const int sms = num_sms();
   if (sms <= 0) return LINATTN_ERR_CUDA;
-  // the output kernel runs two CTAs per SM: the largest shared-memory carveout
+  // both kernels run two CTAs per SM: the largest shared-memory carveout
   if (!set_smem(gtc::global_kv_tc_kernel, static_cast<int>(gtc::kv::kSmemBytes)) ||
       !set_smem(gtc::global_out_tc_kernel, static_cast<int>(gtc::out::kSmemBytes)) ||
       cudaFuncSetAttribute(gtc::global_out_tc_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                           cudaSharedmemCarveoutMaxShared) != cudaSuccess ||
+      cudaFuncSetAttribute(gtc::global_kv_tc_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
                            cudaSharedmemCarveoutMaxShared) != cudaSuccess)
     return LINATTN_ERR_CUDA;
   if (Nk > 0) {
     CUtensorMap mk, mv;
-    if (!make_map_bf16(&mk, k, d->dk, Nk, BH) || !make_map_bf16(&mv, v, d->dv, Nk, BH))
+    // 64-token boxes: the KV kernel's units are 64 tokens of a head pair
+    if (!make_map_bf16(&mk, k, d->dk, Nk, BH, gtc::kv::CK) ||
+        !make_map_bf16(&mv, v, d->dv, Nk, BH, gtc::kv::CK))
       return LINATTN_ERR_CUDA;
-    const long u1 = static_cast<long>(BH / 2) * ((Nk + gtc::C - 1) / gtc::C);
+    const long u1 = static_cast<long>(BH / 2) * ((Nk + gtc::kv::CK - 1) / gtc::kv::CK);
     // programmatic dependent launch: the KV grid may start while KV / ksum are
-    // being zeroed; it waits for that grid only before its first flush
-    const ProgrammaticLaunch pl(static_cast<int>(u1 < sms ? u1 : sms), gtc::kv::NT,
+    // being zeroed; it waits for that grid only before its first flush.  Two
+    // persistent CTAs per SM.
+    const int cap1 = gtc::kv::kCtasPerSm * sms;
+    const ProgrammaticLaunch pl(static_cast<int>(u1 < cap1 ? u1 : cap1), gtc::kv::NT,
                                 gtc::kv::kSmemBytes, s);
     if (cudaLaunchKernelEx(&pl.cfg, gtc::global_kv_tc_kernel, mk, mv, kpm, KV, ksum, BH / 2, Nk,
                            d->H, ident(d)) != cudaSuccess)
