@@ -170,7 +170,8 @@ LINATTN_API int linattn_fwd_causal_ws(const linattn_dims *dims, const void *q, c
  * nothing needs to call this).  Process-wide; set it only while no call of
  * the library is being made from another thread.
  *   op:       LINATTN_OP_CAUSAL (both causal forwards), LINATTN_OP_GLOBAL,
- *             LINATTN_OP_PERFORMER (linattn_performer_features)
+ *             LINATTN_OP_PERFORMER (linattn_performer_features),
+ *             LINATTN_OP_BACKWARD (linattn_bwd_causal)
  *   kernel:   LINATTN_KERNEL_AUTO (the library's choice),
  *             LINATTN_KERNEL_CUDA_CORES (the fp32 CUDA-core kernels),
  *             LINATTN_KERNEL_TC_PAIRED (causal only: the tensor-core kernel
@@ -182,7 +183,8 @@ LINATTN_API int linattn_fwd_causal_ws(const linattn_dims *dims, const void *q, c
  * Returns LINATTN_ERR_INVALID for an unknown op or kernel, a kernel the op
  * does not have, or segments outside 0..64.
  */
-enum { LINATTN_OP_CAUSAL = 0, LINATTN_OP_GLOBAL = 1, LINATTN_OP_PERFORMER = 2 };
+enum { LINATTN_OP_CAUSAL = 0, LINATTN_OP_GLOBAL = 1, LINATTN_OP_PERFORMER = 2,
+       LINATTN_OP_BACKWARD = 3 };
 enum { LINATTN_KERNEL_AUTO = 0, LINATTN_KERNEL_CUDA_CORES = 1, LINATTN_KERNEL_TC_PAIRED = 2 };
 LINATTN_API int linattn_set_kernel_choice(int op, int kernel, int segments);
 
@@ -253,11 +255,16 @@ LINATTN_API int linattn_combine_states(const linattn_dims *dims, int G, const fl
  *   dlambda [H] fp32 or NULL        written (summed over the batch); with
  *                                   lambda = NULL it is the gradient at 1
  * Every output must overlap no input and no other output.  The forward is
- * recomputed inside (nothing from it is needed).  fp32 arithmetic for both
- * dtypes; dlambda is a sum of per-(b, h) fp32 atomics, so its last bits may
- * vary from run to run.  Between its two passes the kernel keeps two fp32
- * numbers per token in the first 8 bytes of that token's dk row, which it
- * overwrites afterwards: dk must not be read before the call completes.
+ * recomputed inside (nothing from it is needed).  bf16 with dk = dv = 128
+ * runs on the tensor cores (bf16 operands, fp32 accumulation, chunks of 128
+ * tokens: a forward pass for dq, a pass for dlambda when it is wanted, a
+ * reverse pass for dk and dv); every other shape, fp32, and the CUDA-core
+ * choice of linattn_set_kernel_choice(LINATTN_OP_BACKWARD, ...) use fp32
+ * arithmetic on CUDA cores.  dlambda is a sum of per-(b, h) fp32 atomics, so
+ * its last bits may vary from run to run; dq, dk, dv do not.  Between its
+ * passes the call keeps two fp32 numbers per token in the first 8 bytes of
+ * that token's dk row, which it overwrites afterwards: dk must not be read
+ * before the call completes.
  */
 LINATTN_API int linattn_bwd_causal(const linattn_dims *dims, const void *q, const void *k,
                        const void *v, const float *lambda, float eps, const void *dy,

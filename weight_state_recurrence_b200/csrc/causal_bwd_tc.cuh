@@ -1,0 +1,1060 @@
+// Backward of the chunked causal forward on the 5th-generation tensor cores:
+// bf16 operands, fp32 accumulators in TMEM, d_k = d_v = 128, chunks of C = 128
+// tokens.  Three passes, each one CTA per (b, h) walking the chunks:
+//
+// The loss is L = sum_i dy_i . y_i with y_i = num_i / den_i (fast-weight
+// article §2.1, §3.2, §4.2: S_i = lambda S_(i-1) + phi(k_i) v_i^T, z likewise,
+// num_i = phi(q_i)^T S_i, den_i = phi(q_i)^T z_i + eps).  Per token
+//   dnum_i = dy_i / den_i,   dden_i = -(dy_i . num_i) / den_i^2 = -dnum_i . y_i
+// (formed here from the bf16 dnum_i the products use, so that the key weight
+// dnum_i . v_j + dden_i = dnum_i . (v_j - y_i) stays exact where it cancels)
+// and the three gradients are linear attentions of their own:
+//   dphi(q_i) = S_i dnum_i + z_i dden_i                       (causal, keys j <= i)
+//   dphi(k_j) = sum_{i>=j} lambda^(i-j) phi(q_i) (dnum_i . v_j + dden_i)
+//   dv_j      = sum_{i>=j} lambda^(i-j) (phi(q_i) . phi(k_j)) dnum_i
+// (the last two anti-causal), dq = dphi(q) phi'(q), dk = dphi(k) phi'(k) with
+// phi'(x) = 1 for x > 0 and e^x = phi(x) otherwise, i.e. min(phi(x), 1).
+//
+// Per chunk (t, s local token indices, Q = phi(q) rows, K = phi(k) rows,
+// M[t][s] = lambda^(t-s) for s <= t, P = Q K^T, w_t = dnum_t):
+//   pass F (chunks in order; state S, z at the chunk start):
+//     A = P o M,  num = diag(lambda^(t+1)) Q S + A V,  den = lambda^(t+1) Q z + A 1 + eps
+//     W = w V^T,  B = (W + dden 1^T) o M
+//     dphi(Q) = diag(lambda^(t+1)) (w S^T + dden z^T) + B K
+//     S <- lambda^C S + (Lk K)^T V,  Lk = diag(lambda^(C-1-s))     (z on CUDA cores)
+//   pass R (chunks in reverse; R, r = the adjoint of every later token,
+//   R = sum_{later t} lambda^(t - chunk end) Q_t w_t^T):
+//     dv      = A^T w + Lk K R
+//     dphi(K) = B^T Q + Lk (V R^T + 1 r^T)
+//     R <- lambda^C R + (Lq Q)^T w,  Lq = diag(lambda^(t+1))           (r likewise)
+//   The per-token den_t and dden_t pass from F to R in the first 8 bytes of
+//   that token's dk row, which R overwrites with the gradient afterwards.
+//
+// dlambda = sum_{s<t} (t-s) lambda^(t-s-1) (Q_t . K_s)(w_t . v_s + dden_t)
+// is split by where the pair (t, s) lies.  Both in the chunk: the tile
+// A' = P o M', M'[t][s] = (t-s) lambda^(t-s-1), against W + dden (pass F).
+// Key before the chunk: the chunk-start state enters token t as
+// lambda^(t+1) S, whose lambda-derivative is (t+1) lambda^t S + lambda^(t+1) S'
+// with S' = dS/dlambda.  The first part is (t+1) lambda^t Q_t . (S w_t + z dden_t),
+// read off pass F's own S w product; the second needs S' and is pass L
+// (dlambda only):
+//     Ms = (Lq Q)^T w,   dlambda += <S', Ms> + sum_t dden_t lambda^(t+1) Q_t . z'
+//     S' <- lambda^C S' + C lambda^(C-1) S + (Lk' K)^T V,  Lk' = diag((C-1-s) lambda^(C-2-s))
+// Every power is a table entry lambda^m or m lambda^(m-1) formed directly, so
+// lambda = 0 and lambda = 1 need no special case.
+//
+// Each pass is one warpgroup (thread = row of the token tile or of the state)
+// issuing its MMAs from thread 0 in program order: the role split and the
+// deep pipelines of the forward are not used here.  Waits are bounded: thread
+// 0 polls, the verdict goes through shared memory to a block barrier, and on
+// a timeout every thread leaves the chunk loop together.
+#pragma once
+#include "common.cuh"
+#include "sm100.cuh"
+#include "causal_tc.cuh"
+
+namespace linattn {
+namespace btc {
+
+using tc::mul_bf16x2;
+using tc::pack_bf16;
+using tc::phi_bf16x2;
+
+constexpr int C = 128;     // tokens per chunk
+constexpr int D = 128;     // d_k = d_v
+constexpr int NT = 128;    // one warpgroup
+constexpr uint32_t kPanel = 128u * 128u;   // 128 rows x 128 bytes (64 bf16)
+constexpr uint32_t kTile = 2u * kPanel;    // 128 x 128 bf16 in two 64-column panels
+
+// byte offset of 16-byte chunk j (0..15) of row r in a tile (128-byte swizzle)
+__device__ __forceinline__ uint32_t toff(uint32_t r, uint32_t j) {
+  return (j >> 3) * kPanel + sw128_offset(r, (j & 7u) * 16u);
+}
+__device__ __forceinline__ float blo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bhi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// Operand descriptors.  K-major: rows are M (or N), K runs along the row
+// (across the two panels).  MN-major: rows are K, M (or N) runs along the row.
+__device__ __forceinline__ uint64_t kdesc(uint32_t a) { return sdesc_sw128(a, 16, 1024); }
+__device__ __forceinline__ uint64_t mdesc(uint32_t a) { return sdesc_sw128(a, kPanel, 1024); }
+__device__ __forceinline__ uint64_t kstep(int ks) {
+  return static_cast<uint64_t>((ks >> 2) * kPanel + (ks & 3) * 32) >> 4;
+}
+__device__ __forceinline__ uint64_t mstep(int ks) { return static_cast<uint64_t>(ks * 2048) >> 4; }
+
+constexpr uint32_t kIdKK = idesc_bf16(128, 128, 0, 0);
+constexpr uint32_t kIdKM = idesc_bf16(128, 128, 0, 1);
+constexpr uint32_t kIdMM = idesc_bf16(128, 128, 1, 1);
+
+// D (+)= A B, K = 128 in 8 steps, both operands in shared memory
+__device__ __forceinline__ void mma_ss(uint32_t d, uint64_t a, bool a_mn, uint64_t b, bool b_mn,
+                                       bool acc) {
+  const uint32_t id = a_mn ? kIdMM : (b_mn ? kIdKM : kIdKK);
+#pragma unroll
+  for (int ks = 0; ks < 8; ++ks)
+    umma_bf16(d, a + (a_mn ? mstep(ks) : kstep(ks)), b + (b_mn ? mstep(ks) : kstep(ks)), id,
+              (acc || ks > 0) ? 1u : 0u);
+}
+// D (+)= A B, A in tensor memory (bf16 pairs, lane = row), B in shared memory
+__device__ __forceinline__ void mma_ts(uint32_t d, uint32_t a, uint64_t b, bool b_mn, bool acc) {
+  const uint32_t id = b_mn ? kIdKM : kIdKK;
+#pragma unroll
+  for (int ks = 0; ks < 8; ++ks)
+    umma_bf16_ts(d, a + ks * 8, b + (b_mn ? mstep(ks) : kstep(ks)), id,
+                 (acc || ks > 0) ? 1u : 0u);
+}
+
+// Row r of a bf16 tile through the feature map in place (nothing with
+// `ident`); returns phi(row) . vec (fp32) when vec is given and adds the row's
+// sum to *sum when sum is given.
+__device__ __forceinline__ float phi_row(uint8_t *tile, int r, bool ident, const float *vec,
+                                         float *sum = nullptr) {
+  float acc = 0.f, rs = 0.f;
+#pragma unroll 4
+  for (int j = 0; j < 16; ++j) {
+    uint4 *p = reinterpret_cast<uint4 *>(tile + toff(r, j));
+    uint4 w = *p;
+    if (!ident) {
+      w.x = phi_bf16x2(w.x);
+      w.y = phi_bf16x2(w.y);
+      w.z = phi_bf16x2(w.z);
+      w.w = phi_bf16x2(w.w);
+      *p = w;
+    }
+    const uint32_t e[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      if (vec) acc += blo(e[m]) * vec[8 * j + 2 * m] + bhi(e[m]) * vec[8 * j + 2 * m + 1];
+      rs += blo(e[m]) + bhi(e[m]);
+    }
+  }
+  if (sum) *sum += rs;
+  return acc;
+}
+
+// elu(x) = phi(x) - 1, in fp32 (e^x - 1 from the fast exponential: its
+// absolute error is far below the bf16 rounding that follows)
+__device__ __forceinline__ float elu_f32(float x) { return x > 0.f ? x : __expf(x) - 1.f; }
+
+// Row r of a bf16 k tile -> elu(k) in place (nothing with `ident`).  The key
+// side of every product is carried as elu(k) = phi(k) - 1 plus exact rank-one
+// terms for the 1: for small k, phi(k) is 1 plus a small part that bf16 near 1
+// would resolve to only ~2^-8, and the gradient of q lives in that part.
+__device__ __forceinline__ void elu_row(uint8_t *tile, int r, bool ident) {
+  if (ident) return;
+#pragma unroll 4
+  for (int j = 0; j < 16; ++j) {
+    uint4 *p = reinterpret_cast<uint4 *>(tile + toff(r, j));
+    uint4 w = *p;
+    w.x = pack_bf16(elu_f32(blo(w.x)), elu_f32(bhi(w.x)));
+    w.y = pack_bf16(elu_f32(blo(w.y)), elu_f32(bhi(w.y)));
+    w.z = pack_bf16(elu_f32(blo(w.z)), elu_f32(bhi(w.z)));
+    w.w = pack_bf16(elu_f32(blo(w.w)), elu_f32(bhi(w.w)));
+    *p = w;
+  }
+}
+
+// dst row r = src row r * f (bf16 product), dst may be src
+__device__ __forceinline__ void scale_row(uint8_t *dst, const uint8_t *src, int r, float f) {
+  const uint32_t f2 = pack_bf16(f, f);
+#pragma unroll 4
+  for (int j = 0; j < 16; ++j) {
+    uint4 w = *reinterpret_cast<const uint4 *>(src + toff(r, j));
+    w.x = mul_bf16x2(w.x, f2);
+    w.y = mul_bf16x2(w.y, f2);
+    w.z = mul_bf16x2(w.z, f2);
+    w.w = mul_bf16x2(w.w, f2);
+    *reinterpret_cast<uint4 *>(dst + toff(r, j)) = w;
+  }
+}
+
+// Column k of a bf16 tile summed over its 128 rows (fp32), optionally
+// weighted per row.
+__device__ __forceinline__ float col_sum(const uint8_t *tile, int k, const float *wrow) {
+  float acc = 0.f;
+  const uint32_t j = static_cast<uint32_t>(k) >> 3, b = (static_cast<uint32_t>(k) & 7u) * 2u;
+#pragma unroll 8
+  for (int r = 0; r < C; ++r) {
+    const uint16_t h = *reinterpret_cast<const uint16_t *>(tile + toff(r, j) + b);
+    const float x = __uint_as_float(static_cast<uint32_t>(h) << 16);
+    acc += wrow ? x * wrow[r] : x;
+  }
+  return acc;
+}
+
+// Row r of the fp32 state in TMEM (this warp's lanes) -> bf16 row r of the
+// operand tile, and the state multiplied by `f` written back.
+__device__ __forceinline__ void state_to_operand(uint32_t t, uint8_t *tile, int r, float f) {
+#pragma unroll 1
+  for (int blk = 0; blk < 4; ++blk) {
+    uint32_t v[32];
+    tmem_ld_32x32b_x32(t + blk * 32, v);
+    tmem_wait_ld();
+    uint32_t pk[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      pk[i] = pack_bf16(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+#pragma unroll
+    for (int m = 0; m < 4; ++m)
+      *reinterpret_cast<uint4 *>(tile + toff(r, blk * 4 + m)) =
+          make_uint4(pk[4 * m], pk[4 * m + 1], pk[4 * m + 2], pk[4 * m + 3]);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * f);
+    tmem_st_32x32b_x32(t + blk * 32, v);
+  }
+  tmem_wait_st();
+}
+
+// tab[m] for 0 <= m (m < 0: 0); the load index stays in the table either way
+__device__ __forceinline__ float tab(const float *t, int m) {
+  const float x = t[m < 0 ? 0 : m];
+  return m < 0 ? 0.f : x;
+}
+
+__device__ __forceinline__ float block_sum(float x, float *red) {
+  x = warp_sum(x);
+  const int w = threadIdx.x >> 5;
+  if ((threadIdx.x & 31) == 0) red[w] = x;
+  __syncthreads();
+  const float s = red[0] + red[1] + red[2] + red[3];
+  __syncthreads();
+  return s;
+}
+
+// ============================================================== pass F
+// The key side in the elu form (o = 1; o = 0 and elu(k) -> k with `ident`):
+// K = Kt + o 1 1^T with Kt = elu(K), so
+//   P = Q Kt^T + o rq 1^T,  rq = Q 1 (row sums of phi(Q))
+//   B K = B Kt + o (B 1) 1^T
+// and the state S = St + o 1 s^T, z = zt + o zeta 1 with
+//   St = sum_s w_s Kt_s v_s^T,  s = sum_s w_s v_s,  zt = sum_s w_s Kt_s,  zeta = sum_s w_s
+// (w_s the decay weight of key s), so that
+//   Q S = Q St + o rq s^T,   Q z = Q zt + o rq zeta,
+//   S w_t + z dden_t = St w_t + zt dden_t + o (s . w_t + zeta dden_t) 1.
+namespace pf {
+constexpr uint32_t kOffQ = 0, kOffK = kTile, kOffV = 2 * kTile, kOffG = 3 * kTile,
+                   kOffSb = 4 * kTile, kOffAp = 5 * kTile, kOffMisc = 6 * kTile;
+enum { kFullQ = 0, kFullK, kFullV, kFullG, kMma, kFinal, kNumBars };
+constexpr uint32_t kMiscTmem = 64, kMiscFlag = 68, kMiscPw = 128;
+constexpr uint32_t kMiscDpw = kMiscPw + 132 * 4, kMiscPwr = kMiscDpw + 132 * 4;
+constexpr uint32_t kMiscZ = kMiscPwr + 128 * 4, kMiscS = kMiscZ + 128 * 4;
+constexpr uint32_t kMiscGs = kMiscS + 128 * 4, kMiscRed = kMiscGs + 128 * 4;
+constexpr uint32_t kSmemBytes = kOffMisc + kMiscRed + 64;
+static_assert(kSmemBytes <= 232448, "exceeds the per-CTA shared memory of sm_100");
+// tensor memory columns
+constexpr uint32_t kTmS = 0, kTmT1 = 128, kTmT2 = 256, kTmA = 384, kTmW = 448;
+}  // namespace pf
+
+__global__ void __launch_bounds__(NT, 1)
+    bwd_tc_f_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
+                    const float *__restrict__ lam, float eps, __nv_bfloat16 *__restrict__ dq,
+                    __nv_bfloat16 *__restrict__ dk, float *__restrict__ dlam, int H, int N,
+                    bool ident) {
+  using namespace pf;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *sm = smem_raw;
+  const uint32_t sb = smem_u32(sm);
+  const int tid = threadIdx.x, warp = tid >> 5;
+  if (sb & 1023u) {
+    if (tid == 0) atomicOr(&g_status, kStatusWaitTimeout);
+    return;
+  }
+  const long bh = blockIdx.x;
+  const int h = static_cast<int>(bh % H);
+  const float L = lam ? lam[h] : 1.f;
+  const float o = ident ? 0.f : 1.f;
+  const int nch = (N + C - 1) / C;
+  uint8_t *misc = sm + kOffMisc;
+  auto bar = [&](int i) { return sb + kOffMisc + 8u * static_cast<uint32_t>(i); };
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(misc + kMiscTmem);
+  volatile int *flag = reinterpret_cast<volatile int *>(misc + kMiscFlag);
+  float *pw = reinterpret_cast<float *>(misc + kMiscPw);     // lambda^m, m = 0..C
+  float *dpw = reinterpret_cast<float *>(misc + kMiscDpw);   // m lambda^(m-1)
+  float *pwr = reinterpret_cast<float *>(misc + kMiscPwr);   // lambda^(C-1-s)
+  float *zt = reinterpret_cast<float *>(misc + kMiscZ);
+  float *sv = reinterpret_cast<float *>(misc + kMiscS);
+  float *gs = reinterpret_cast<float *>(misc + kMiscGs);     // sum_{m<=t} lambda^m
+  float *red = reinterpret_cast<float *>(misc + kMiscRed);
+  const CUtensorMap *maps[4] = {&tm_q, &tm_k, &tm_v, &tm_g};
+  const uint32_t offs[4] = {kOffQ, kOffK, kOffV, kOffG};
+  int issued[4] = {0, 0, 0, 0}, waited[4] = {0, 0, 0, 0};   // thread 0: copies per tile
+  auto load = [&](int which, int c) {
+    const uint32_t b = bar(kFullQ + which);
+    mbar_arrive_expect_tx(b, kTile);
+    tma_load_3d(sb + offs[which], maps[which], b, 0, c * C, static_cast<int>(bh));
+    tma_load_3d(sb + offs[which] + kPanel, maps[which], b, 64, c * C, static_cast<int>(bh));
+    if (c + 1 < nch) tma_prefetch_l2_3d(maps[which], 0, (c + 1) * C, static_cast<int>(bh));
+    if (c + 1 < nch) tma_prefetch_l2_3d(maps[which], 64, (c + 1) * C, static_cast<int>(bh));
+    ++issued[which];
+  };
+  if (tid == 0) {
+    for (int i = 0; i < kNumBars; ++i) mbar_init(bar(i), 1);
+    *flag = 0;
+    fence_mbar_init();
+    for (int i = 0; i < 4; ++i) tma_prefetch_desc(maps[i]);
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  pw[tid] = pow_int(L, tid);
+  dpw[tid] = tid == 0 ? 0.f : static_cast<float>(tid) * pow_int(L, tid - 1);
+  pwr[tid] = pow_int(L, C - 1 - tid);
+  if (tid == 0) {
+    pw[C] = pow_int(L, C);
+    dpw[C] = static_cast<float>(C) * pow_int(L, C - 1);
+  }
+  zt[tid] = 0.f;
+  sv[tid] = 0.f;
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t lf = static_cast<uint32_t>(warp * 32) << 16;
+  if (tid == 0 && nch > 0)
+    for (int i = 0; i < 4; ++i) load(i, 0);
+  // thread 0 waits (bounded); every thread learns the verdict at the barrier
+  auto poll = [&](int b, int parity) {
+    if (tid == 0 && !*flag) {
+      if (!mbar_wait(bar(b), static_cast<uint32_t>(parity) & 1u)) *flag = 1;
+      else if (b <= kFullG) ++waited[b];
+    }
+  };
+  auto meet = [&]() -> bool {
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    return *flag == 0;
+  };
+  int mph = 0;   // completed phases of the MMA barrier
+  auto mma_done = [&]() { poll(kMma, mph); ++mph; };
+
+  const uint64_t dQ = kdesc(sb + kOffQ), dK = kdesc(sb + kOffK), dKm = mdesc(sb + kOffK);
+  const uint64_t dV = kdesc(sb + kOffV), dVm = mdesc(sb + kOffV);
+  const uint64_t dSb = kdesc(sb + kOffSb), dSbm = mdesc(sb + kOffSb);
+  const int i = tid;            // token row of the chunk (and d_k, d_v row of the state)
+  float dl = 0.f;               // this thread's share of dlambda
+  float zeta = 0.f;             // sum of the decay weights of the keys before the chunk
+  float geo = 0.f;              // sum_s lambda^(C-1-s) over a chunk
+  for (int m = 0; m < C; ++m) geo += pwr[m];
+  {
+    float g = 0.f;
+    for (int m = 0; m <= tid; ++m) g += pw[m];
+    gs[tid] = g;
+  }
+  __syncthreads();
+  uint8_t *ap_row = sm + kOffAp + static_cast<uint32_t>(i) * 256u;   // A' row, thread-private
+  const float lf_i = pw[i + 1];
+
+  for (int c = 0; c < nch; ++c) {
+    const int row0 = c * C, Cv = min(C, N - row0);
+    const bool carried = c > 0, last = c == nch - 1;
+    // ---- the state before this chunk: bf16 operand, and lambda^C St kept for the update
+    if (carried) state_to_operand(tmem + kTmS + lf, sm + kOffSb, i, pw[C]);
+    poll(kFullQ, c);
+    if (!meet()) break;
+    float rq = 0.f;
+    const float qzt = phi_row(sm + kOffQ, i, ident, zt, &rq);   // phi(q_i) . zt, row sum
+    const float qz = qzt + o * rq * zeta;                       // phi(q_i) . z
+    poll(kFullK, c);
+    if (!meet()) break;
+    elu_row(sm + kOffK, i, ident);
+    fence_proxy_async_smem();
+    if (!meet()) break;
+    if (tid == 0) {
+      mma_ss(tmem + kTmT1, dQ, false, dK, false, false);                 // Q Kt^T
+      if (carried) mma_ss(tmem + kTmT2, dQ, false, dSbm, true, false);   // Q St
+      umma_commit(bar(kMma));
+    }
+    mma_done();
+    if (!meet()) break;
+    // ---- the score weights A = (o rq 1^T + Q Kt^T) o M: the small part
+    // At = (Q Kt^T) o M into TMEM (bf16), At' = (Q Kt^T) o M' into shared
+    // memory; the o rq part stays exact (row sum o rq g_t here, its products
+    // with V and w through the masked row sums of W below)
+    float rs = o * rq * gs[i];
+#pragma unroll 1
+    for (int blk = 0; blk < 4; ++blk) {
+      uint32_t v[32];
+      tmem_ld_32x32b_x32(tmem + lf + kTmT1 + blk * 32, v);
+      tmem_wait_ld();
+      uint32_t pa[16], pp[16];
+#pragma unroll
+      for (int e = 0; e < 32; e += 2) {
+        const int s0 = blk * 32 + e, s1 = s0 + 1;
+        const float p0 = __uint_as_float(v[e]), p1 = __uint_as_float(v[e + 1]);
+        pa[e / 2] = pack_bf16(p0 * tab(pw, i - s0), p1 * tab(pw, i - s1));
+        rs += blo(pa[e / 2]) + bhi(pa[e / 2]);
+        pp[e / 2] = pack_bf16(p0 * tab(dpw, i - s0), p1 * tab(dpw, i - s1));
+      }
+      tmem_st_32x32b_x16(tmem + lf + kTmA + blk * 16, pa);
+#pragma unroll
+      for (int m = 0; m < 4; ++m)
+        *reinterpret_cast<uint4 *>(ap_row + (((blk * 4 + m) ^ (i & 15)) << 4)) =
+            make_uint4(pp[4 * m], pp[4 * m + 1], pp[4 * m + 2], pp[4 * m + 3]);
+    }
+    tmem_wait_st();
+    poll(kFullV, c);
+    if (!meet()) break;
+    if (tid == 0) {
+      mma_ts(tmem + kTmT1, tmem + kTmA, dVm, true, false);   // At V
+      umma_commit(bar(kMma));
+    }
+    mma_done();
+    poll(kFullG, c);
+    if (!meet()) break;
+    // ---- den, dnum (bf16 into TMEM) and dnum . num but for its o rq part
+    const float den = lf_i * qz + rs + eps, inv = 1.f / den;
+    float gn = 0.f, sd = 0.f;   // dnum . (At V + carried part), dnum . s
+#pragma unroll 1
+    for (int blk = 0; blk < 4; ++blk) {
+      uint32_t av[32], xv[32];
+      tmem_ld_32x32b_x32(tmem + lf + kTmT1 + blk * 32, av);
+      if (carried) tmem_ld_32x32b_x32(tmem + lf + kTmT2 + blk * 32, xv);
+      tmem_wait_ld();
+      uint32_t pk[16];
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const uint4 g4 = *reinterpret_cast<const uint4 *>(sm + kOffG + toff(i, blk * 4 + m));
+        const uint32_t g[4] = {g4.x, g4.y, g4.z, g4.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int e = 8 * m + 2 * u, v0 = blk * 32 + e;
+          float n0 = __uint_as_float(av[e]), n1 = __uint_as_float(av[e + 1]);
+          if (carried) {
+            n0 += lf_i * (__uint_as_float(xv[e]) + o * rq * sv[v0]);
+            n1 += lf_i * (__uint_as_float(xv[e + 1]) + o * rq * sv[v0 + 1]);
+          }
+          // dden from the bf16 dnum the MMAs use, so that dnum . v + dden (the
+          // weight of every key) is exact up to the fp32 sums even where the
+          // two terms nearly cancel
+          pk[4 * m + u] = pack_bf16(blo(g[u]) * inv, bhi(g[u]) * inv);
+          const float d0 = blo(pk[4 * m + u]), d1 = bhi(pk[4 * m + u]);
+          gn += d0 * n0 + d1 * n1;
+          sd += d0 * sv[v0] + d1 * sv[v0 + 1];
+        }
+      }
+      tmem_st_32x32b_x16(tmem + lf + kTmW + blk * 16, pk);
+    }
+    tmem_wait_st();
+    if (!meet()) break;
+    if (tid == 0) {
+      if (!last) load(3, c + 1);                                   // dy tile is free
+      mma_ts(tmem + kTmT1, tmem + kTmW, dV, false, false);        // W = w V^T
+      if (carried) mma_ts(tmem + kTmT2, tmem + kTmW, dSb, false, false);   // U = w St^T
+      umma_commit(bar(kMma));
+    }
+    mma_done();
+    if (!meet()) break;
+    // ---- dden = -dnum . num / den, the o rq part from the masked row sum of
+    // W = w V^T; den and dden kept for pass R
+    float gw = 0.f;
+#pragma unroll 1
+    for (int blk = 0; blk < 4; ++blk) {
+      uint32_t v[32];
+      tmem_ld_32x32b_x32(tmem + lf + kTmT1 + blk * 32, v);
+      tmem_wait_ld();
+#pragma unroll
+      for (int e = 0; e < 32; ++e) gw += __uint_as_float(v[e]) * tab(pw, i - blk * 32 - e);
+    }
+    const float dden = -(gn + o * rq * gw) * inv;
+    if (i < Cv)
+      *reinterpret_cast<float2 *>(dk + (bh * N + row0 + i) * static_cast<long>(D)) =
+          make_float2(den, dden);
+    // ---- B = (W + dden) o M into TMEM, its fp32 row sum; dlambda, pairs inside the chunk
+    float rb = 0.f;
+#pragma unroll 1
+    for (int blk = 0; blk < 4; ++blk) {
+      uint32_t v[32];
+      tmem_ld_32x32b_x32(tmem + lf + kTmT1 + blk * 32, v);
+      tmem_wait_ld();
+      uint32_t pb[16];
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const uint4 a4 = *reinterpret_cast<const uint4 *>(ap_row + (((blk * 4 + m) ^ (i & 15)) << 4));
+        const uint32_t ap[4] = {a4.x, a4.y, a4.z, a4.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int e = 8 * m + 2 * u;
+          const int s0 = blk * 32 + e, s1 = s0 + 1;
+          const float w0 = __uint_as_float(v[e]) + dden, w1 = __uint_as_float(v[e + 1]) + dden;
+          dl += (blo(ap[u]) + o * rq * tab(dpw, i - s0)) * w0 +
+                (bhi(ap[u]) + o * rq * tab(dpw, i - s1)) * w1;
+          const float b0 = w0 * tab(pw, i - s0), b1 = w1 * tab(pw, i - s1);
+          rb += b0 + b1;
+          pb[4 * m + u] = pack_bf16(b0, b1);
+        }
+      }
+      tmem_st_32x32b_x16(tmem + lf + kTmA + blk * 16, pb);
+    }
+    tmem_wait_st();
+    if (!meet()) break;
+    if (tid == 0) {
+      mma_ts(tmem + kTmT1, tmem + kTmA, dKm, true, false);   // B Kt
+      umma_commit(bar(kMma));
+    }
+    mma_done();
+    if (!meet()) break;
+    // ---- dq = (B Kt + o B1 + lambda^(t+1) (U + zt dden + o (s.w + zeta dden))) phi'(q);
+    //      dlambda, keys before the chunk (the lambda^(t+1) factor's derivative)
+    {
+      float qu = 0.f;
+      const float one = o * (rb + (carried ? lf_i * (sd + zeta * dden) : 0.f));
+      __nv_bfloat16 *dst = dq + (bh * N + row0 + i) * static_cast<long>(D);
+#pragma unroll 1
+      for (int blk = 0; blk < 4; ++blk) {
+        uint32_t bk[32], uv[32];
+        tmem_ld_32x32b_x32(tmem + lf + kTmT1 + blk * 32, bk);
+        if (carried) tmem_ld_32x32b_x32(tmem + lf + kTmT2 + blk * 32, uv);
+        tmem_wait_ld();
+        uint32_t pk[16];
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          const uint4 q4 = *reinterpret_cast<const uint4 *>(sm + kOffQ + toff(i, blk * 4 + m));
+          const uint32_t qw[4] = {q4.x, q4.y, q4.z, q4.w};
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int e = 8 * m + 2 * u, k0 = blk * 32 + e;
+            const float u0 = carried ? __uint_as_float(uv[e]) : 0.f;
+            const float u1 = carried ? __uint_as_float(uv[e + 1]) : 0.f;
+            const float q0 = blo(qw[u]), q1 = bhi(qw[u]);
+            qu += q0 * u0 + q1 * u1;
+            float g0 = __uint_as_float(bk[e]) + one + lf_i * (u0 + dden * zt[k0]);
+            float g1 = __uint_as_float(bk[e + 1]) + one + lf_i * (u1 + dden * zt[k0 + 1]);
+            if (!ident) {
+              g0 *= fminf(q0, 1.f);
+              g1 *= fminf(q1, 1.f);
+            }
+            pk[4 * m + u] = pack_bf16(g0, g1);
+          }
+        }
+        if (i < Cv)
+#pragma unroll
+          for (int m = 0; m < 4; ++m)
+            reinterpret_cast<uint4 *>(dst + blk * 32)[m] =
+                make_uint4(pk[4 * m], pk[4 * m + 1], pk[4 * m + 2], pk[4 * m + 3]);
+      }
+      if (carried) dl += dpw[i + 1] * (qu + dden * qzt + o * rq * (sd + zeta * dden));
+    }
+    if (last) break;
+    // ---- state update: key rows weighted lambda^(C-1-s): St += (Lk Kt)^T V, zt, s, zeta likewise
+    scale_row(sm + kOffK, sm + kOffK, i, pwr[i]);
+    fence_proxy_async_smem();
+    if (!meet()) break;
+    if (tid == 0) {
+      mma_ss(tmem + kTmS, dKm, true, dVm, true, carried);
+      umma_commit(bar(kMma));
+      load(0, c + 1);   // the q tile is free
+    }
+    zt[i] = pw[C] * zt[i] + col_sum(sm + kOffK, i, nullptr);
+    sv[i] = pw[C] * sv[i] + col_sum(sm + kOffV, i, pwr);
+    zeta = pw[C] * zeta + geo;
+    mma_done();
+    if (!meet()) break;
+    if (tid == 0) {
+      load(1, c + 1);
+      load(2, c + 1);
+    }
+  }
+  // dlambda: pairs inside a chunk and the carried-state part of pairs across chunks
+  if (dlam) {
+    const float tot = block_sum(dl, red);
+    if (tid == 0 && !*flag) atomicAdd(dlam + h, tot);
+  }
+  // leave with no copy and no MMA in flight
+  if (tid == 0) {
+    for (int b = 0; b < 4; ++b)
+      for (int n = waited[b]; n < issued[b]; ++n) mbar_wait(bar(kFullQ + b), n & 1);
+    umma_commit(bar(kFinal));
+    mbar_wait(bar(kFinal), 0);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ============================================================== pass R
+namespace pr {
+constexpr uint32_t kOffQ = 0, kOffK = kTile, kOffKd = 2 * kTile, kOffV = 3 * kTile,
+                   kOffVd = 4 * kTile, kOffG = 5 * kTile, kOffRb = 6 * kTile, kOffMisc = 7 * kTile;
+enum { kFullQ = 0, kFullK, kFullV, kFullG, kMma, kFinal, kNumBars };
+constexpr uint32_t kMiscTmem = 64, kMiscFlag = 68, kMiscPw = 128;
+constexpr uint32_t kMiscDden = kMiscPw + 132 * 4, kMiscR = kMiscDden + 128 * 4;
+constexpr uint32_t kSmemBytes = kOffMisc + kMiscR + 128 * 4;
+static_assert(kSmemBytes <= 232448, "exceeds the per-CTA shared memory of sm_100");
+constexpr uint32_t kTmR = 0, kTmT1 = 128, kTmT2 = 256, kTmAt = 384, kTmBt = 448;
+}  // namespace pr
+
+__global__ void __launch_bounds__(NT, 1)
+    bwd_tc_r_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
+                    const float *__restrict__ lam, __nv_bfloat16 *__restrict__ dk,
+                    __nv_bfloat16 *__restrict__ dv, int H, int N, bool ident) {
+  using namespace pr;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *sm = smem_raw;
+  const uint32_t sb = smem_u32(sm);
+  const int tid = threadIdx.x, warp = tid >> 5;
+  if (sb & 1023u) {
+    if (tid == 0) atomicOr(&g_status, kStatusWaitTimeout);
+    return;
+  }
+  const long bh = blockIdx.x;
+  const int h = static_cast<int>(bh % H);
+  const float L = lam ? lam[h] : 1.f;
+  const int nch = (N + C - 1) / C;
+  uint8_t *misc = sm + kOffMisc;
+  auto bar = [&](int i) { return sb + kOffMisc + 8u * static_cast<uint32_t>(i); };
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(misc + kMiscTmem);
+  volatile int *flag = reinterpret_cast<volatile int *>(misc + kMiscFlag);
+  float *pw = reinterpret_cast<float *>(misc + kMiscPw);
+  float *sdd = reinterpret_cast<float *>(misc + kMiscDden);   // dden of the chunk's tokens
+  float *rv = reinterpret_cast<float *>(misc + kMiscR);       // r, the normaliser's adjoint
+  const CUtensorMap *maps[4] = {&tm_q, &tm_k, &tm_v, &tm_g};
+  const uint32_t offs[4] = {kOffQ, kOffK, kOffV, kOffG};
+  int issued[4] = {0, 0, 0, 0}, waited[4] = {0, 0, 0, 0};
+  auto load = [&](int which, int c) {
+    const uint32_t b = bar(kFullQ + which);
+    mbar_arrive_expect_tx(b, kTile);
+    tma_load_3d(sb + offs[which], maps[which], b, 0, c * C, static_cast<int>(bh));
+    tma_load_3d(sb + offs[which] + kPanel, maps[which], b, 64, c * C, static_cast<int>(bh));
+    if (c > 0) tma_prefetch_l2_3d(maps[which], 0, (c - 1) * C, static_cast<int>(bh));
+    if (c > 0) tma_prefetch_l2_3d(maps[which], 64, (c - 1) * C, static_cast<int>(bh));
+    ++issued[which];
+  };
+  if (tid == 0) {
+    for (int i = 0; i < kNumBars; ++i) mbar_init(bar(i), 1);
+    *flag = 0;
+    fence_mbar_init();
+    for (int i = 0; i < 4; ++i) tma_prefetch_desc(maps[i]);
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  pw[tid] = pow_int(L, tid);
+  if (tid == 0) pw[C] = pow_int(L, C);
+  rv[tid] = 0.f;
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t lf = static_cast<uint32_t>(warp * 32) << 16;
+  if (tid == 0 && nch > 0)
+    for (int i = 0; i < 4; ++i) load(i, nch - 1);
+  auto poll = [&](int b, int parity) {
+    if (tid == 0 && !*flag) {
+      if (!mbar_wait(bar(b), static_cast<uint32_t>(parity) & 1u)) *flag = 1;
+      else if (b <= kFullG) ++waited[b];
+    }
+  };
+  auto meet = [&]() -> bool {
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    return *flag == 0;
+  };
+  int mph = 0;
+  auto mma_done = [&]() { poll(kMma, mph); ++mph; };
+
+  const uint64_t dQ = kdesc(sb + kOffQ), dQm = mdesc(sb + kOffQ), dK = kdesc(sb + kOffK);
+  const uint64_t dKd = kdesc(sb + kOffKd), dV = kdesc(sb + kOffV), dVd = kdesc(sb + kOffVd);
+  const uint64_t dG = kdesc(sb + kOffG), dGm = mdesc(sb + kOffG);
+  const uint64_t dRb = kdesc(sb + kOffRb), dRbm = mdesc(sb + kOffRb);
+  const int i = tid;   // token row (key j of the formulas) and d_k row of R
+
+  for (int cc = 0; cc < nch; ++cc) {
+    const int c = nch - 1 - cc, row0 = c * C, Cv = min(C, N - row0);
+    const bool carried = cc > 0;   // later tokens exist: R, r nonzero
+    // den, dden of this token from pass F (tokens past the end: no gradient)
+    float den = 1.f, dden = 0.f;
+    if (i < Cv) {
+      const float2 st =
+          *reinterpret_cast<const float2 *>(dk + (bh * N + row0 + i) * static_cast<long>(D));
+      den = st.x;
+      dden = st.y;
+    }
+    sdd[i] = dden;
+    if (carried) state_to_operand(tmem + kTmR + lf, sm + kOffRb, i, pw[C]);
+    poll(kFullQ, cc);
+    poll(kFullK, cc);
+    poll(kFullV, cc);
+    poll(kFullG, cc);
+    if (!meet()) break;
+    phi_row(sm + kOffQ, i, ident, nullptr);
+    phi_row(sm + kOffK, i, ident, nullptr);
+    if (carried) {
+      scale_row(sm + kOffKd, sm + kOffK, i, pw[C - 1 - i]);
+      scale_row(sm + kOffVd, sm + kOffV, i, pw[C - 1 - i]);
+    }
+    {
+      // w = dnum = dy / den in place of dy
+      const float inv = 1.f / den;
+#pragma unroll 4
+      for (int j = 0; j < 16; ++j) {
+        uint4 *p = reinterpret_cast<uint4 *>(sm + kOffG + toff(i, j));
+        uint4 g = *p;
+        g.x = pack_bf16(blo(g.x) * inv, bhi(g.x) * inv);
+        g.y = pack_bf16(blo(g.y) * inv, bhi(g.y) * inv);
+        g.z = pack_bf16(blo(g.z) * inv, bhi(g.z) * inv);
+        g.w = pack_bf16(blo(g.w) * inv, bhi(g.w) * inv);
+        *p = g;
+      }
+    }
+    fence_proxy_async_smem();
+    if (!meet()) break;
+    if (tid == 0) {
+      mma_ss(tmem + kTmT1, dK, false, dQ, false, false);   // P^T = K Q^T
+      mma_ss(tmem + kTmT2, dV, false, dG, false, false);   // W^T = V w^T
+      umma_commit(bar(kMma));
+    }
+    mma_done();
+    if (!meet()) break;
+    if (tid == 0 && c > 0) load(2, c - 1);   // v has been read (its weighted copy is made)
+    // ---- A^T and B^T rows (key i, queries s >= i) into TMEM
+#pragma unroll 1
+    for (int blk = 0; blk < 4; ++blk) {
+      uint32_t pv[32], wv[32];
+      tmem_ld_32x32b_x32(tmem + lf + kTmT1 + blk * 32, pv);
+      tmem_ld_32x32b_x32(tmem + lf + kTmT2 + blk * 32, wv);
+      tmem_wait_ld();
+      uint32_t pa[16], pb[16];
+#pragma unroll
+      for (int e = 0; e < 32; e += 2) {
+        const int s0 = blk * 32 + e, s1 = s0 + 1;
+        const float m0 = tab(pw, s0 - i), m1 = tab(pw, s1 - i);
+        pa[e / 2] = pack_bf16(__uint_as_float(pv[e]) * m0, __uint_as_float(pv[e + 1]) * m1);
+        pb[e / 2] = pack_bf16((__uint_as_float(wv[e]) + sdd[s0]) * m0,
+                              (__uint_as_float(wv[e + 1]) + sdd[s1]) * m1);
+      }
+      tmem_st_32x32b_x16(tmem + lf + kTmAt + blk * 16, pa);
+      tmem_st_32x32b_x16(tmem + lf + kTmBt + blk * 16, pb);
+    }
+    tmem_wait_st();
+    if (!meet()) break;
+    if (tid == 0) {
+      mma_ts(tmem + kTmT1, tmem + kTmAt, dGm, true, false);                 // A^T w
+      if (carried) mma_ss(tmem + kTmT1, dKd, false, dRbm, true, true);     // + Lk K R
+      mma_ts(tmem + kTmT2, tmem + kTmBt, dQm, true, false);                 // B^T Q
+      if (carried) mma_ss(tmem + kTmT2, dVd, false, dRb, false, true);     // + Lk V R^T
+      umma_commit(bar(kMma));
+    }
+    mma_done();
+    if (!meet()) break;
+    // ---- dv and dk = (dphi(k) + Lk r) phi'(k)
+    {
+      const float kf = carried ? pw[C - 1 - i] : 0.f;
+      __nv_bfloat16 *vd = dv + (bh * N + row0 + i) * static_cast<long>(D);
+      __nv_bfloat16 *kd = dk + (bh * N + row0 + i) * static_cast<long>(D);
+#pragma unroll 1
+      for (int blk = 0; blk < 4; ++blk) {
+        uint32_t a[32], b[32];
+        tmem_ld_32x32b_x32(tmem + lf + kTmT1 + blk * 32, a);
+        tmem_ld_32x32b_x32(tmem + lf + kTmT2 + blk * 32, b);
+        tmem_wait_ld();
+        uint32_t pv[16], pk[16];
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          const uint4 k4 = *reinterpret_cast<const uint4 *>(sm + kOffK + toff(i, blk * 4 + m));
+          const uint32_t kw[4] = {k4.x, k4.y, k4.z, k4.w};
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int e = 8 * m + 2 * u, k0 = blk * 32 + e;
+            pv[4 * m + u] = pack_bf16(__uint_as_float(a[e]), __uint_as_float(a[e + 1]));
+            float g0 = __uint_as_float(b[e]) + kf * rv[k0];
+            float g1 = __uint_as_float(b[e + 1]) + kf * rv[k0 + 1];
+            if (!ident) {
+              g0 *= fminf(blo(kw[u]), 1.f);
+              g1 *= fminf(bhi(kw[u]), 1.f);
+            }
+            pk[4 * m + u] = pack_bf16(g0, g1);
+          }
+        }
+        if (i < Cv)
+#pragma unroll
+          for (int m = 0; m < 4; ++m) {
+            reinterpret_cast<uint4 *>(vd + blk * 32)[m] =
+                make_uint4(pv[4 * m], pv[4 * m + 1], pv[4 * m + 2], pv[4 * m + 3]);
+            reinterpret_cast<uint4 *>(kd + blk * 32)[m] =
+                make_uint4(pk[4 * m], pk[4 * m + 1], pk[4 * m + 2], pk[4 * m + 3]);
+          }
+      }
+    }
+    if (c == 0) break;
+    // ---- R += (Lq Q)^T w, r likewise: q rows weighted lambda^(t+1)
+    scale_row(sm + kOffQ, sm + kOffQ, i, pw[i + 1]);
+    fence_proxy_async_smem();
+    if (!meet()) break;
+    if (tid == 0) {
+      mma_ss(tmem + kTmR, dQm, true, dGm, true, carried);
+      umma_commit(bar(kMma));
+      load(1, c - 1);   // k has been read
+    }
+    rv[i] = pw[C] * rv[i] + col_sum(sm + kOffQ, i, sdd);
+    mma_done();
+    if (!meet()) break;
+    if (tid == 0) {
+      load(0, c - 1);
+      load(3, c - 1);
+    }
+  }
+  if (tid == 0) {
+    for (int b = 0; b < 4; ++b)
+      for (int n = waited[b]; n < issued[b]; ++n) mbar_wait(bar(kFullQ + b), n & 1);
+    umma_commit(bar(kFinal));
+    mbar_wait(bar(kFinal), 0);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ============================================================== pass L
+// dlambda's part from the derivative state S' = dS/dlambda (keys before the
+// chunk), in the elu form of pass F: S' = St' + o 1 s'^T, z' = zt' + o zeta' 1,
+//   <S', Ms> = <St', Ms> + o s' . (1^T Ms),   1^T Ms = sum_t lambda^(t+1) rq_t w_t
+//   sum_t dden_t lambda^(t+1) Q_t . z' = sum_t dden_t lambda^(t+1) (Q_t . zt' + o rq_t zeta')
+// and every part of (St, s, zt, zeta) and of its derivative steps per chunk as
+//   X' <- lambda^C X' + C lambda^(C-1) X + (chunk term with (C-1-s) lambda^(C-2-s))
+//   X  <- lambda^C X  + (chunk term with lambda^(C-1-s)).
+namespace pl {
+constexpr uint32_t kOffQ = 0, kOffK = kTile, kOffKp = 2 * kTile, kOffV = 3 * kTile,
+                   kOffG = 4 * kTile, kOffMisc = 5 * kTile;
+enum { kFullQ = 0, kFullK, kFullV, kFullG, kMma, kFinal, kNumBars };
+constexpr uint32_t kMiscTmem = 64, kMiscFlag = 68, kMiscPw = 128;
+constexpr uint32_t kMiscDpw = kMiscPw + 132 * 4, kMiscPwr = kMiscDpw + 132 * 4;
+constexpr uint32_t kMiscDpwr = kMiscPwr + 128 * 4, kMiscZ = kMiscDpwr + 128 * 4;
+constexpr uint32_t kMiscZp = kMiscZ + 128 * 4, kMiscS = kMiscZp + 128 * 4;
+constexpr uint32_t kMiscSp = kMiscS + 128 * 4, kMiscWq = kMiscSp + 128 * 4;
+constexpr uint32_t kMiscRed = kMiscWq + 128 * 4;
+constexpr uint32_t kSmemBytes = kOffMisc + kMiscRed + 64;
+static_assert(kSmemBytes <= 232448, "exceeds the per-CTA shared memory of sm_100");
+constexpr uint32_t kTmS = 0, kTmSp = 128, kTmM = 256;
+}  // namespace pl
+
+__global__ void __launch_bounds__(NT, 1)
+    bwd_tc_l_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
+                    const float *__restrict__ lam, const __nv_bfloat16 *__restrict__ dk,
+                    float *__restrict__ dlam, int H, int N, bool ident) {
+  using namespace pl;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *sm = smem_raw;
+  const uint32_t sb = smem_u32(sm);
+  const int tid = threadIdx.x, warp = tid >> 5;
+  if (sb & 1023u) {
+    if (tid == 0) atomicOr(&g_status, kStatusWaitTimeout);
+    return;
+  }
+  const long bh = blockIdx.x;
+  const int h = static_cast<int>(bh % H);
+  const float L = lam ? lam[h] : 1.f;
+  const float o = ident ? 0.f : 1.f;
+  const int nch = (N + C - 1) / C;
+  uint8_t *misc = sm + kOffMisc;
+  auto bar = [&](int i) { return sb + kOffMisc + 8u * static_cast<uint32_t>(i); };
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(misc + kMiscTmem);
+  volatile int *flag = reinterpret_cast<volatile int *>(misc + kMiscFlag);
+  float *pw = reinterpret_cast<float *>(misc + kMiscPw);
+  float *dpw = reinterpret_cast<float *>(misc + kMiscDpw);
+  float *pwr = reinterpret_cast<float *>(misc + kMiscPwr);     // lambda^(C-1-s)
+  float *dpwr = reinterpret_cast<float *>(misc + kMiscDpwr);   // (C-1-s) lambda^(C-2-s)
+  float *zt = reinterpret_cast<float *>(misc + kMiscZ);
+  float *ztp = reinterpret_cast<float *>(misc + kMiscZp);
+  float *sv = reinterpret_cast<float *>(misc + kMiscS);
+  float *svp = reinterpret_cast<float *>(misc + kMiscSp);
+  float *wq = reinterpret_cast<float *>(misc + kMiscWq);       // lambda^(t+1) rq_t
+  float *red = reinterpret_cast<float *>(misc + kMiscRed);
+  const CUtensorMap *maps[4] = {&tm_q, &tm_k, &tm_v, &tm_g};
+  const uint32_t offs[4] = {kOffQ, kOffK, kOffV, kOffG};
+  int issued[4] = {0, 0, 0, 0}, waited[4] = {0, 0, 0, 0};
+  auto load = [&](int which, int c) {
+    const uint32_t b = bar(kFullQ + which);
+    mbar_arrive_expect_tx(b, kTile);
+    tma_load_3d(sb + offs[which], maps[which], b, 0, c * C, static_cast<int>(bh));
+    tma_load_3d(sb + offs[which] + kPanel, maps[which], b, 64, c * C, static_cast<int>(bh));
+    if (c + 1 < nch) tma_prefetch_l2_3d(maps[which], 0, (c + 1) * C, static_cast<int>(bh));
+    if (c + 1 < nch) tma_prefetch_l2_3d(maps[which], 64, (c + 1) * C, static_cast<int>(bh));
+    ++issued[which];
+  };
+  if (tid == 0) {
+    for (int i = 0; i < kNumBars; ++i) mbar_init(bar(i), 1);
+    *flag = 0;
+    fence_mbar_init();
+    for (int i = 0; i < 4; ++i) tma_prefetch_desc(maps[i]);
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  pw[tid] = pow_int(L, tid);
+  dpw[tid] = tid == 0 ? 0.f : static_cast<float>(tid) * pow_int(L, tid - 1);
+  pwr[tid] = pow_int(L, C - 1 - tid);
+  dpwr[tid] = tid == C - 1 ? 0.f : static_cast<float>(C - 1 - tid) * pow_int(L, C - 2 - tid);
+  if (tid == 0) {
+    pw[C] = pow_int(L, C);
+    dpw[C] = static_cast<float>(C) * pow_int(L, C - 1);
+  }
+  zt[tid] = 0.f;
+  ztp[tid] = 0.f;
+  sv[tid] = 0.f;
+  svp[tid] = 0.f;
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t lf = static_cast<uint32_t>(warp * 32) << 16;
+  if (tid == 0 && nch > 0)
+    for (int i = 0; i < 4; ++i) load(i, 0);
+  auto poll = [&](int b, int parity) {
+    if (tid == 0 && !*flag) {
+      if (!mbar_wait(bar(b), static_cast<uint32_t>(parity) & 1u)) *flag = 1;
+      else if (b <= kFullG) ++waited[b];
+    }
+  };
+  auto meet = [&]() -> bool {
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    return *flag == 0;
+  };
+  int mph = 0;
+  auto mma_done = [&]() { poll(kMma, mph); ++mph; };
+
+  const uint64_t dQm = mdesc(sb + kOffQ), dKm = mdesc(sb + kOffK), dKpm = mdesc(sb + kOffKp);
+  const uint64_t dVm = mdesc(sb + kOffV), dGm = mdesc(sb + kOffG);
+  const int i = tid;
+  float dl = 0.f;
+  float zeta = 0.f, zetap = 0.f;
+  float geo = 0.f, dgeo = 0.f;
+  for (int m = 0; m < C; ++m) {
+    geo += pwr[m];
+    dgeo += dpwr[m];
+  }
+
+  for (int c = 0; c < nch; ++c) {
+    const int row0 = c * C, Cv = min(C, N - row0);
+    const bool carried = c > 0, last = c == nch - 1;
+    float den = 1.f, dden = 0.f;
+    if (i < Cv) {
+      const float2 st =
+          *reinterpret_cast<const float2 *>(dk + (bh * N + row0 + i) * static_cast<long>(D));
+      den = st.x;
+      dden = st.y;
+    }
+    poll(kFullQ, c);
+    poll(kFullK, c);
+    poll(kFullG, c);
+    if (!meet()) break;
+    // q rows weighted lambda^(t+1); the z' part of dlambda
+    float rq = 0.f;
+    const float qztp = phi_row(sm + kOffQ, i, ident, ztp, &rq);
+    dl += dden * pw[i + 1] * (qztp + o * rq * zetap);
+    wq[i] = pw[i + 1] * rq;
+    scale_row(sm + kOffQ, sm + kOffQ, i, pw[i + 1]);
+    {
+      const float inv = 1.f / den;
+#pragma unroll 4
+      for (int j = 0; j < 16; ++j) {
+        uint4 *p = reinterpret_cast<uint4 *>(sm + kOffG + toff(i, j));
+        uint4 g = *p;
+        g.x = pack_bf16(blo(g.x) * inv, bhi(g.x) * inv);
+        g.y = pack_bf16(blo(g.y) * inv, bhi(g.y) * inv);
+        g.z = pack_bf16(blo(g.z) * inv, bhi(g.z) * inv);
+        g.w = pack_bf16(blo(g.w) * inv, bhi(g.w) * inv);
+        *p = g;
+      }
+    }
+    if (!last) {
+      // key rows as elu(k), weighted lambda^(C-1-s) (state) and (C-1-s) lambda^(C-2-s) (derivative)
+      elu_row(sm + kOffK, i, ident);
+      scale_row(sm + kOffKp, sm + kOffK, i, dpwr[i]);
+      scale_row(sm + kOffK, sm + kOffK, i, pwr[i]);
+    }
+    fence_proxy_async_smem();
+    if (!meet()) break;
+    if (tid == 0) {
+      mma_ss(tmem + kTmM, dQm, true, dGm, true, false);   // Ms = (Lq Q)^T w
+      umma_commit(bar(kMma));
+    }
+    // o s' . (1^T Ms) on this thread's d_v column (s' of the chunk start)
+    dl += o * svp[i] * col_sum(sm + kOffG, i, wq);
+    mma_done();
+    if (!meet()) break;
+    if (tid == 0 && !last) {
+      load(0, c + 1);
+      load(3, c + 1);
+    }
+    // <St', Ms> on this thread's d_k row; then St' <- lambda^C St' + C lambda^(C-1) St, St <- lambda^C St
+    if (carried) {
+#pragma unroll 1
+      for (int blk = 0; blk < 4; ++blk) {
+        uint32_t sp[32], mv[32], sq[32];
+        tmem_ld_32x32b_x32(tmem + lf + kTmSp + blk * 32, sp);
+        tmem_ld_32x32b_x32(tmem + lf + kTmM + blk * 32, mv);
+        tmem_ld_32x32b_x32(tmem + lf + kTmS + blk * 32, sq);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const float s1 = __uint_as_float(sp[e]), s0 = __uint_as_float(sq[e]);
+          dl += s1 * __uint_as_float(mv[e]);
+          sp[e] = __float_as_uint(pw[C] * s1 + dpw[C] * s0);
+          sq[e] = __float_as_uint(pw[C] * s0);
+        }
+        if (!last) {
+          tmem_st_32x32b_x32(tmem + lf + kTmSp + blk * 32, sp);
+          tmem_st_32x32b_x32(tmem + lf + kTmS + blk * 32, sq);
+        }
+      }
+      tmem_wait_st();
+    }
+    if (last) break;
+    // the vector parts of the state and of its derivative (this thread's d_k / d_v index)
+    ztp[i] = pw[C] * ztp[i] + dpw[C] * zt[i] + col_sum(sm + kOffKp, i, nullptr);
+    zt[i] = pw[C] * zt[i] + col_sum(sm + kOffK, i, nullptr);
+    svp[i] = pw[C] * svp[i] + dpw[C] * sv[i] + col_sum(sm + kOffV, i, dpwr);
+    sv[i] = pw[C] * sv[i] + col_sum(sm + kOffV, i, pwr);
+    zetap = pw[C] * zetap + dpw[C] * zeta + dgeo;
+    zeta = pw[C] * zeta + geo;
+    poll(kFullV, c);
+    if (!meet()) break;
+    if (tid == 0) {
+      mma_ss(tmem + kTmS, dKm, true, dVm, true, carried);
+      mma_ss(tmem + kTmSp, dKpm, true, dVm, true, carried);
+      umma_commit(bar(kMma));
+    }
+    mma_done();
+    if (!meet()) break;
+    if (tid == 0) {
+      load(1, c + 1);
+      load(2, c + 1);
+    }
+  }
+  const float tot = block_sum(dl, red);
+  if (tid == 0 && !*flag) atomicAdd(dlam + h, tot);
+  if (tid == 0) {
+    for (int b = 0; b < 4; ++b)
+      for (int n = waited[b]; n < issued[b]; ++n) mbar_wait(bar(kFullQ + b), n & 1);
+    umma_commit(bar(kFinal));
+    mbar_wait(bar(kFinal), 0);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace btc
+}  // namespace linattn

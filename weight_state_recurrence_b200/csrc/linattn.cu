@@ -22,6 +22,7 @@
 #include "causal_tc.cuh"
 #include "causal_seg_tc.cuh"
 #include "causal_bwd.cuh"
+#include "causal_bwd_tc.cuh"
 #include "global_simt.cuh"
 #include "global_tc.cuh"
 #include "performer.cuh"
@@ -132,7 +133,8 @@ bool make_map_bf16(CUtensorMap *m, const void *ptr, int inner, int rows, int pla
 
 // Kernel family per operation, set by linattn_set_kernel_choice (tests and
 // benchmarks compare families on the same call); AUTO unless set.
-std::atomic<int> g_choice[3] = {{LINATTN_KERNEL_AUTO}, {LINATTN_KERNEL_AUTO}, {LINATTN_KERNEL_AUTO}};
+std::atomic<int> g_choice[4] = {{LINATTN_KERNEL_AUTO}, {LINATTN_KERNEL_AUTO}, {LINATTN_KERNEL_AUTO},
+                                {LINATTN_KERNEL_AUTO}};
 std::atomic<int> g_forced_segments{0};
 
 int choice(int op) { return g_choice[op].load(std::memory_order_relaxed); }
@@ -588,6 +590,43 @@ int causal_bwd_dv(const linattn_dims *d, const void *q, const void *k, const voi
   return LINATTN_ERR_UNSUPPORTED;
 }
 
+// The tensor-core backward: bf16, d_k = d_v = 128.  Pass F (dq, and den,
+// dden per token into dk), pass L (dlambda's carried-derivative part, only
+// when dlambda is wanted), pass R (dk, dv), in stream order.
+bool use_tc_bwd(const linattn_dims *d) {
+  return choice(LINATTN_OP_BACKWARD) != LINATTN_KERNEL_CUDA_CORES && d->dtype == LINATTN_BF16 &&
+         d->dk == 128 && d->dv == 128;
+}
+
+int launch_bwd_tc(const linattn_dims *d, const void *q, const void *k, const void *v,
+                  const float *lam, float eps, const void *dy, void *dq, void *dk, void *dv,
+                  float *dlam, cudaStream_t s) {
+  const int BH = d->B * d->H;
+  CUtensorMap mq, mk, mv, mg;
+  if (!make_map_bf16(&mq, q, 128, d->N, BH) || !make_map_bf16(&mk, k, 128, d->N, BH) ||
+      !make_map_bf16(&mv, v, 128, d->N, BH) || !make_map_bf16(&mg, dy, 128, d->N, BH))
+    return LINATTN_ERR_CUDA;
+  if (!set_smem(btc::bwd_tc_f_kernel, static_cast<int>(btc::pf::kSmemBytes)) ||
+      !set_smem(btc::bwd_tc_l_kernel, static_cast<int>(btc::pl::kSmemBytes)) ||
+      !set_smem(btc::bwd_tc_r_kernel, static_cast<int>(btc::pr::kSmemBytes)))
+    return LINATTN_ERR_CUDA;
+  auto *bq = static_cast<bf16 *>(dq);
+  auto *bk = static_cast<bf16 *>(dk);
+  auto *bv = static_cast<bf16 *>(dv);
+  btc::bwd_tc_f_kernel<<<BH, btc::NT, btc::pf::kSmemBytes, s>>>(mq, mk, mv, mg, lam, eps, bq, bk,
+                                                                 dlam, d->H, d->N, ident(d));
+  int rc = launch_status();
+  if (rc != LINATTN_OK) return rc;
+  if (dlam) {
+    btc::bwd_tc_l_kernel<<<BH, btc::NT, btc::pl::kSmemBytes, s>>>(mq, mk, mv, mg, lam, bk, dlam,
+                                                                   d->H, d->N, ident(d));
+    if ((rc = launch_status()) != LINATTN_OK) return rc;
+  }
+  btc::bwd_tc_r_kernel<<<BH, btc::NT, btc::pr::kSmemBytes, s>>>(mq, mk, mv, mg, lam, bk, bv, d->H,
+                                                                 d->N, ident(d));
+  return launch_status();
+}
+
 template <typename T>
 int causal_bwd_dispatch(const linattn_dims *d, const void *q, const void *k, const void *v,
                         const float *lam, float eps, const void *dy, void *dq, void *dk, void *dv,
@@ -761,7 +800,7 @@ extern "C" size_t linattn_fwd_causal_workspace(const linattn_dims *d) {
 }
 
 extern "C" int linattn_set_kernel_choice(int op, int kernel, int segments) {
-  if (op < LINATTN_OP_CAUSAL || op > LINATTN_OP_PERFORMER) return LINATTN_ERR_INVALID;
+  if (op < LINATTN_OP_CAUSAL || op > LINATTN_OP_BACKWARD) return LINATTN_ERR_INVALID;
   if (kernel < LINATTN_KERNEL_AUTO || kernel > LINATTN_KERNEL_TC_PAIRED) return LINATTN_ERR_INVALID;
   if (kernel == LINATTN_KERNEL_TC_PAIRED && op != LINATTN_OP_CAUSAL) return LINATTN_ERR_INVALID;
   if (segments < 0 || segments > kMaxSegments) return LINATTN_ERR_INVALID;
@@ -926,6 +965,7 @@ extern "C" int linattn_bwd_causal(const linattn_dims *d, const void *q, const vo
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (dlambda && cudaMemsetAsync(dlambda, 0, nl, s) != cudaSuccess) return LINATTN_ERR_CUDA;
   if (BH == 0 || d->N == 0) return LINATTN_OK;
+  if (use_tc_bwd(d)) return launch_bwd_tc(d, q, k, v, lambda, eps, dy, dq, dk, dv, dlambda, s);
   if (d->dtype == LINATTN_F32)
     return causal_bwd_dispatch<float>(d, q, k, v, lambda, eps, dy, dq, dk, dv, dlambda, s);
   return causal_bwd_dispatch<bf16>(d, q, k, v, lambda, eps, dy, dq, dk, dv, dlambda, s);

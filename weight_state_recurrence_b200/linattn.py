@@ -27,7 +27,7 @@ LINATTN_ERR_CUDA = 3
 LINATTN_ERR_DEVICE = 4
 LINATTN_PHI_ELU1, LINATTN_PHI_IDENTITY = 0, 1
 LINATTN_PERFORMER_SOFTMAX, LINATTN_PERFORMER_GAUSSIAN = 0, 1
-LINATTN_OP_CAUSAL, LINATTN_OP_GLOBAL, LINATTN_OP_PERFORMER = 0, 1, 2
+LINATTN_OP_CAUSAL, LINATTN_OP_GLOBAL, LINATTN_OP_PERFORMER, LINATTN_OP_BACKWARD = 0, 1, 2, 3
 LINATTN_KERNEL_AUTO, LINATTN_KERNEL_CUDA_CORES, LINATTN_KERNEL_TC_PAIRED = 0, 1, 2
 
 ENTRY_POINTS = ("linattn_fwd_causal", "linattn_fwd_causal_from", "linattn_fwd_causal_workspace",
