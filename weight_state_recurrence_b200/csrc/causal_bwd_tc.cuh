@@ -27,8 +27,10 @@
 //     dv      = A^T w + Lk K R
 //     dphi(K) = B^T Q + Lk (V R^T + 1 r^T)
 //     R <- lambda^C R + (Lq Q)^T w,  Lq = diag(lambda^(t+1))           (r likewise)
-//   The per-token den_t and dden_t pass from F to R in the first 8 bytes of
-//   that token's dk row, which R overwrites with the gradient afterwards.
+//   The per-token den_t and dden_t pass from F to L and R through a stash:
+//   two floats per token at a caller-given stride (a workspace, or the first
+//   8 bytes of the token's dk row, which R overwrites afterwards; then L must
+//   finish before R starts).
 //
 // dlambda = sum_{s<t} (t-s) lambda^(t-s-1) (Q_t . K_s)(w_t . v_s + dden_t)
 // is split by where the pair (t, s) lies.  Both in the chunk: the tile
@@ -249,8 +251,8 @@ __global__ void __launch_bounds__(NT, 1)
     bwd_tc_f_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
                     const float *__restrict__ lam, float eps, __nv_bfloat16 *__restrict__ dq,
-                    __nv_bfloat16 *__restrict__ dk, float *__restrict__ dlam, int H, int N,
-                    bool ident) {
+                    float *__restrict__ stash, long stash_stride, float *__restrict__ dlam, int H,
+                    int N, bool ident) {
   using namespace pf;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *sm = smem_raw;
@@ -461,7 +463,7 @@ __global__ void __launch_bounds__(NT, 1)
     }
     const float dden = -(gn + o * rq * gw) * inv;
     if (i < Cv)
-      *reinterpret_cast<float2 *>(dk + (bh * N + row0 + i) * static_cast<long>(D)) =
+      *reinterpret_cast<float2 *>(stash + (bh * N + row0 + i) * stash_stride) =
           make_float2(den, dden);
     // ---- B = (W + dden) o M into TMEM, its fp32 row sum; dlambda, pairs inside the chunk
     float rb = 0.f;
@@ -593,8 +595,9 @@ constexpr uint32_t kTmR = 0, kTmT1 = 128, kTmT2 = 256, kTmAt = 384, kTmBt = 448;
 __global__ void __launch_bounds__(NT, 1)
     bwd_tc_r_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
-                    const float *__restrict__ lam, __nv_bfloat16 *__restrict__ dk,
-                    __nv_bfloat16 *__restrict__ dv, int H, int N, bool ident) {
+                    const float *__restrict__ lam, const float *stash, long stash_stride,
+                    __nv_bfloat16 *__restrict__ dk, __nv_bfloat16 *__restrict__ dv, int H, int N,
+                    bool ident) {
   using namespace pr;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *sm = smem_raw;
@@ -675,8 +678,7 @@ __global__ void __launch_bounds__(NT, 1)
     // den, dden of this token from pass F (tokens past the end: no gradient)
     float den = 1.f, dden = 0.f;
     if (i < Cv) {
-      const float2 st =
-          *reinterpret_cast<const float2 *>(dk + (bh * N + row0 + i) * static_cast<long>(D));
+      const float2 st = *reinterpret_cast<const float2 *>(stash + (bh * N + row0 + i) * stash_stride);
       den = st.x;
       dden = st.y;
     }
@@ -844,8 +846,8 @@ constexpr uint32_t kTmS = 0, kTmSp = 128, kTmM = 256;
 __global__ void __launch_bounds__(NT, 1)
     bwd_tc_l_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
-                    const float *__restrict__ lam, const __nv_bfloat16 *__restrict__ dk,
-                    float *__restrict__ dlam, int H, int N, bool ident) {
+                    const float *__restrict__ lam, const float *__restrict__ stash,
+                    long stash_stride, float *__restrict__ dlam, int H, int N, bool ident) {
   using namespace pl;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *sm = smem_raw;
@@ -916,6 +918,9 @@ __global__ void __launch_bounds__(NT, 1)
   const uint32_t lf = static_cast<uint32_t>(warp * 32) << 16;
   if (tid == 0 && nch > 0)
     for (int i = 0; i < 4; ++i) load(i, 0);
+  // the reverse pass (launched after this one as its programmatic dependent,
+  // when the stash is not in dk) reads nothing this pass writes: let it start
+  grid_launch_dependents();
   auto poll = [&](int b, int parity) {
     if (tid == 0 && !*flag) {
       if (!mbar_wait(bar(b), static_cast<uint32_t>(parity) & 1u)) *flag = 1;
@@ -947,8 +952,7 @@ __global__ void __launch_bounds__(NT, 1)
     const bool carried = c > 0, last = c == nch - 1;
     float den = 1.f, dden = 0.f;
     if (i < Cv) {
-      const float2 st =
-          *reinterpret_cast<const float2 *>(dk + (bh * N + row0 + i) * static_cast<long>(D));
+      const float2 st = *reinterpret_cast<const float2 *>(stash + (bh * N + row0 + i) * stash_stride);
       den = st.x;
       dden = st.y;
     }

@@ -591,11 +591,23 @@ int causal_bwd_dv(const linattn_dims *d, const void *q, const void *k, const voi
 }
 
 // The tensor-core backward: bf16, d_k = d_v = 128.  Pass F (dq, and den,
-// dden per token into dk), pass L (dlambda's carried-derivative part, only
-// when dlambda is wanted), pass R (dk, dv), in stream order.
+// dden per token into the stash), pass L (dlambda's carried-derivative part,
+// only when dlambda is wanted), pass R (dk, dv).  The stash is a stream-ordered
+// allocation of 8 bytes per token, so R (which writes dk) runs beside L as its
+// programmatic dependent; without it the stash lives in the dk rows and R
+// follows L.
 bool use_tc_bwd(const linattn_dims *d) {
   return choice(LINATTN_OP_BACKWARD) != LINATTN_KERNEL_CUDA_CORES && d->dtype == LINATTN_BF16 &&
          d->dk == 128 && d->dv == 128;
+}
+
+template <typename... KArgs, typename... Args>
+int launch_pdl(void (*kern)(KArgs...), int grid, int block, size_t smem, cudaStream_t s,
+               bool programmatic, Args... args) {
+  ProgrammaticLaunch pl(grid, block, smem, s);
+  if (!programmatic) pl.cfg.numAttrs = 0;
+  return cudaLaunchKernelEx(&pl.cfg, kern, args...) == cudaSuccess ? LINATTN_OK
+                                                                   : LINATTN_ERR_CUDA;
 }
 
 int launch_bwd_tc(const linattn_dims *d, const void *q, const void *k, const void *v,
@@ -613,18 +625,26 @@ int launch_bwd_tc(const linattn_dims *d, const void *q, const void *k, const voi
   auto *bq = static_cast<bf16 *>(dq);
   auto *bk = static_cast<bf16 *>(dk);
   auto *bv = static_cast<bf16 *>(dv);
-  btc::bwd_tc_f_kernel<<<BH, btc::NT, btc::pf::kSmemBytes, s>>>(mq, mk, mv, mg, lam, eps, bq, bk,
-                                                                 dlam, d->H, d->N, ident(d));
-  int rc = launch_status();
-  if (rc != LINATTN_OK) return rc;
-  if (dlam) {
-    btc::bwd_tc_l_kernel<<<BH, btc::NT, btc::pl::kSmemBytes, s>>>(mq, mk, mv, mg, lam, bk, dlam,
-                                                                   d->H, d->N, ident(d));
-    if ((rc = launch_status()) != LINATTN_OK) return rc;
+  const bool id = ident(d);
+  float *ws = nullptr;
+  const size_t stash_bytes = static_cast<size_t>(BH) * d->N * 2 * sizeof(float);
+  if (cudaMallocAsync(reinterpret_cast<void **>(&ws), stash_bytes, s) != cudaSuccess) {
+    cudaGetLastError();   // fall back to the stash in the dk rows
+    ws = nullptr;
   }
-  btc::bwd_tc_r_kernel<<<BH, btc::NT, btc::pr::kSmemBytes, s>>>(mq, mk, mv, mg, lam, bk, bv, d->H,
-                                                                 d->N, ident(d));
-  return launch_status();
+  float *stash = ws ? ws : reinterpret_cast<float *>(dk);
+  const long stride = ws ? 2 : btc::D / 2;
+  int rc = launch_pdl(btc::bwd_tc_f_kernel, BH, btc::NT, btc::pf::kSmemBytes, s, false, mq, mk,
+                      mv, mg, lam, eps, bq, stash, stride, dlam, d->H, d->N, id);
+  if (rc == LINATTN_OK && dlam)
+    rc = launch_pdl(btc::bwd_tc_l_kernel, BH, btc::NT, btc::pl::kSmemBytes, s, false, mq, mk, mv,
+                    mg, lam, static_cast<const float *>(stash), stride, dlam, d->H, d->N, id);
+  if (rc == LINATTN_OK)
+    rc = launch_pdl(btc::bwd_tc_r_kernel, BH, btc::NT, btc::pr::kSmemBytes, s,
+                    ws != nullptr && dlam != nullptr, mq, mk, mv, mg, lam,
+                    static_cast<const float *>(stash), stride, bk, bv, d->H, d->N, id);
+  if (ws && cudaFreeAsync(ws, s) != cudaSuccess && rc == LINATTN_OK) rc = LINATTN_ERR_CUDA;
+  return rc;
 }
 
 template <typename T>
