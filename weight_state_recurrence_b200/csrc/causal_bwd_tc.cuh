@@ -45,11 +45,13 @@
 // Every power is a table entry lambda^m or m lambda^(m-1) formed directly, so
 // lambda = 0 and lambda = 1 need no special case.
 //
-// Each pass is one warpgroup (thread = row of the token tile or of the state)
-// issuing its MMAs from thread 0 in program order: the role split and the
-// deep pipelines of the forward are not used here.  Waits are bounded: thread
-// 0 polls, the verdict goes through shared memory to a block barrier, and on
-// a timeout every thread leaves the chunk loop together.
+// Each pass is two warpgroups that own the same rows (thread = row of the token
+// tile or of the state, TMEM lane = row) and split each row's 128 columns in
+// halves; row sums meet through shared memory at the block barriers.  Thread
+// 0 issues the MMAs in program order: the role split and the deep pipelines
+// of the forward are not used here.  Waits are bounded: thread 0 polls, the
+// verdict goes through shared memory to a block barrier, and on a timeout
+// every thread leaves the chunk loop together.
 #pragma once
 #include "common.cuh"
 #include "sm100.cuh"
@@ -64,7 +66,7 @@ using tc::phi_bf16x2;
 
 constexpr int C = 128;     // tokens per chunk
 constexpr int D = 128;     // d_k = d_v
-constexpr int NT = 128;    // one warpgroup
+constexpr int NT = 256;    // two warpgroups: thread (h, r) owns columns [64h, 64h + 64) of row r
 constexpr uint32_t kPanel = 128u * 128u;   // 128 rows x 128 bytes (64 bf16)
 constexpr uint32_t kTile = 2u * kPanel;    // 128 x 128 bf16 in two 64-column panels
 
@@ -106,14 +108,17 @@ __device__ __forceinline__ void mma_ts(uint32_t d, uint32_t a, uint64_t b, bool 
                  (acc || ks > 0) ? 1u : 0u);
 }
 
-// Row r of a bf16 tile through the feature map in place (nothing with
-// `ident`); returns phi(row) . vec (fp32) when vec is given and adds the row's
-// sum to *sum when sum is given.
-__device__ __forceinline__ float phi_row(uint8_t *tile, int r, bool ident, const float *vec,
+// The row helpers below work on this thread's half h of row r: 16-byte
+// chunks [8h, 8h + 8), i.e. columns [64h, 64h + 64).
+
+// The half row through the feature map in place (nothing with `ident`);
+// returns phi(row) . vec over the half (fp32) when vec is given and adds the
+// half row's sum to *sum when sum is given.
+__device__ __forceinline__ float phi_row(uint8_t *tile, int r, int h, bool ident, const float *vec,
                                          float *sum = nullptr) {
   float acc = 0.f, rs = 0.f;
 #pragma unroll 4
-  for (int j = 0; j < 16; ++j) {
+  for (int j = 8 * h; j < 8 * h + 8; ++j) {
     uint4 *p = reinterpret_cast<uint4 *>(tile + toff(r, j));
     uint4 w = *p;
     if (!ident) {
@@ -138,14 +143,15 @@ __device__ __forceinline__ float phi_row(uint8_t *tile, int r, bool ident, const
 // absolute error is far below the bf16 rounding that follows)
 __device__ __forceinline__ float elu_f32(float x) { return x > 0.f ? x : __expf(x) - 1.f; }
 
-// Row r of a bf16 k tile -> elu(k) in place (nothing with `ident`).  The key
-// side of every product is carried as elu(k) = phi(k) - 1 plus exact rank-one
-// terms for the 1: for small k, phi(k) is 1 plus a small part that bf16 near 1
-// would resolve to only ~2^-8, and the gradient of q lives in that part.
-__device__ __forceinline__ void elu_row(uint8_t *tile, int r, bool ident) {
+// The half row of a bf16 k tile -> elu(k) in place (nothing with `ident`).
+// The key side of every product is carried as elu(k) = phi(k) - 1 plus exact
+// rank-one terms for the 1: for small k, phi(k) is 1 plus a small part that
+// bf16 near 1 would resolve to only ~2^-8, and the gradient of q lives in
+// that part.
+__device__ __forceinline__ void elu_row(uint8_t *tile, int r, int h, bool ident) {
   if (ident) return;
 #pragma unroll 4
-  for (int j = 0; j < 16; ++j) {
+  for (int j = 8 * h; j < 8 * h + 8; ++j) {
     uint4 *p = reinterpret_cast<uint4 *>(tile + toff(r, j));
     uint4 w = *p;
     w.x = pack_bf16(elu_f32(blo(w.x)), elu_f32(bhi(w.x)));
@@ -156,11 +162,11 @@ __device__ __forceinline__ void elu_row(uint8_t *tile, int r, bool ident) {
   }
 }
 
-// dst row r = src row r * f (bf16 product), dst may be src
-__device__ __forceinline__ void scale_row(uint8_t *dst, const uint8_t *src, int r, float f) {
+// dst half row = src half row * f (bf16 product), dst may be src
+__device__ __forceinline__ void scale_row(uint8_t *dst, const uint8_t *src, int r, int h, float f) {
   const uint32_t f2 = pack_bf16(f, f);
 #pragma unroll 4
-  for (int j = 0; j < 16; ++j) {
+  for (int j = 8 * h; j < 8 * h + 8; ++j) {
     uint4 w = *reinterpret_cast<const uint4 *>(src + toff(r, j));
     w.x = mul_bf16x2(w.x, f2);
     w.y = mul_bf16x2(w.y, f2);
@@ -170,25 +176,43 @@ __device__ __forceinline__ void scale_row(uint8_t *dst, const uint8_t *src, int 
   }
 }
 
-// Column k of a bf16 tile summed over its 128 rows (fp32), optionally
-// weighted per row.
-__device__ __forceinline__ float col_sum(const uint8_t *tile, int k, const float *wrow) {
-  float acc = 0.f;
-  const uint32_t j = static_cast<uint32_t>(k) >> 3, b = (static_cast<uint32_t>(k) & 7u) * 2u;
-#pragma unroll 8
-  for (int r = 0; r < C; ++r) {
-    const uint16_t h = *reinterpret_cast<const uint16_t *>(tile + toff(r, j) + b);
-    const float x = __uint_as_float(static_cast<uint32_t>(h) << 16);
-    acc += wrow ? x * wrow[r] : x;
+// The half row of dy -> dnum = dy * inv in place (fp32 product, one rounding)
+__device__ __forceinline__ void dnum_row(uint8_t *tile, int r, int h, float inv) {
+#pragma unroll 4
+  for (int j = 8 * h; j < 8 * h + 8; ++j) {
+    uint4 *p = reinterpret_cast<uint4 *>(tile + toff(r, j));
+    uint4 g = *p;
+    g.x = pack_bf16(blo(g.x) * inv, bhi(g.x) * inv);
+    g.y = pack_bf16(blo(g.y) * inv, bhi(g.y) * inv);
+    g.z = pack_bf16(blo(g.z) * inv, bhi(g.z) * inv);
+    g.w = pack_bf16(blo(g.w) * inv, bhi(g.w) * inv);
+    *p = g;
   }
-  return acc;
 }
 
-// Row r of the fp32 state in TMEM (this warp's lanes) -> bf16 row r of the
-// operand tile, and the state multiplied by `f` written back.
-__device__ __forceinline__ void state_to_operand(uint32_t t, uint8_t *tile, int r, float f) {
+// Column k of a bf16 tile summed over rows [64h, 64h + 64) (fp32),
+// optionally weighted per row.
+__device__ __forceinline__ float col_sum(const uint8_t *tile, int k, int h, const float *wrow) {
+  float a0 = 0.f, a1 = 0.f;
+  const uint32_t j = static_cast<uint32_t>(k) >> 3, b = (static_cast<uint32_t>(k) & 7u) * 2u;
+#pragma unroll 8
+  for (int r = 64 * h; r < 64 * h + 64; r += 2) {
+    const float x0 = __uint_as_float(
+        static_cast<uint32_t>(*reinterpret_cast<const uint16_t *>(tile + toff(r, j) + b)) << 16);
+    const float x1 = __uint_as_float(
+        static_cast<uint32_t>(*reinterpret_cast<const uint16_t *>(tile + toff(r + 1, j) + b)) << 16);
+    a0 += wrow ? x0 * wrow[r] : x0;
+    a1 += wrow ? x1 * wrow[r + 1] : x1;
+  }
+  return a0 + a1;
+}
+
+// The half row r of the fp32 state in TMEM (this warp's lanes; t already
+// holds the lane offset) -> bf16 row r of the operand tile, and the state
+// multiplied by `f` written back.
+__device__ __forceinline__ void state_to_operand(uint32_t t, uint8_t *tile, int r, int h, float f) {
 #pragma unroll 1
-  for (int blk = 0; blk < 4; ++blk) {
+  for (int blk = 2 * h; blk < 2 * h + 2; ++blk) {
     uint32_t v[32];
     tmem_ld_32x32b_x32(t + blk * 32, v);
     tmem_wait_ld();
@@ -218,10 +242,22 @@ __device__ __forceinline__ float block_sum(float x, float *red) {
   const int w = threadIdx.x >> 5;
   if ((threadIdx.x & 31) == 0) red[w] = x;
   __syncthreads();
-  const float s = red[0] + red[1] + red[2] + red[3];
+  float s = 0.f;
+#pragma unroll
+  for (int k = 0; k < NT / 32; ++k) s += red[k];
   __syncthreads();
   return s;
 }
+
+// Per-row sums of the two halves: slot x holds [2][128] floats.
+struct Halves {
+  float *base;
+  int h, r;
+  __device__ __forceinline__ void put(int x, float v) const { base[(2 * x + h) * 128 + r] = v; }
+  __device__ __forceinline__ float get(int x) const {
+    return base[(2 * x) * 128 + r] + base[(2 * x + 1) * 128 + r];
+  }
+};
 
 // ============================================================== pass F
 // The key side in the elu form (o = 1; o = 0 and elu(k) -> k with `ident`):
@@ -233,6 +269,10 @@ __device__ __forceinline__ float block_sum(float x, float *red) {
 // (w_s the decay weight of key s), so that
 //   Q S = Q St + o rq s^T,   Q z = Q zt + o rq zeta,
 //   S w_t + z dden_t = St w_t + zt dden_t + o (s . w_t + zeta dden_t) 1.
+// The score weights A = (o rq 1^T + Q Kt^T) o M keep their o rq part exact
+// too: its row sum is o rq_t g_t (g_t = sum_{m<=t} lambda^m) and its product
+// with V, dotted with w_t, is o rq_t times the masked row sum of W = w V^T;
+// only At = (Q Kt^T) o M goes through bf16.
 namespace pf {
 constexpr uint32_t kOffQ = 0, kOffK = kTile, kOffV = 2 * kTile, kOffG = 3 * kTile,
                    kOffSb = 4 * kTile, kOffAp = 5 * kTile, kOffMisc = 6 * kTile;
@@ -241,7 +281,9 @@ constexpr uint32_t kMiscTmem = 64, kMiscFlag = 68, kMiscPw = 128;
 constexpr uint32_t kMiscDpw = kMiscPw + 132 * 4, kMiscPwr = kMiscDpw + 132 * 4;
 constexpr uint32_t kMiscZ = kMiscPwr + 128 * 4, kMiscS = kMiscZ + 128 * 4;
 constexpr uint32_t kMiscGs = kMiscS + 128 * 4, kMiscRed = kMiscGs + 128 * 4;
-constexpr uint32_t kSmemBytes = kOffMisc + kMiscRed + 64;
+constexpr uint32_t kMiscX = kMiscRed + 64;
+enum { kXQz = 0, kXRq, kXRs, kXGn, kXSd, kXGw, kXRb, kXZt, kXSv, kNumX };
+constexpr uint32_t kSmemBytes = kOffMisc + kMiscX + kNumX * 2 * 128 * 4;
 static_assert(kSmemBytes <= 232448, "exceeds the per-CTA shared memory of sm_100");
 // tensor memory columns
 constexpr uint32_t kTmS = 0, kTmT1 = 128, kTmT2 = 256, kTmA = 384, kTmW = 448;
@@ -278,6 +320,8 @@ __global__ void __launch_bounds__(NT, 1)
   float *sv = reinterpret_cast<float *>(misc + kMiscS);
   float *gs = reinterpret_cast<float *>(misc + kMiscGs);     // sum_{m<=t} lambda^m
   float *red = reinterpret_cast<float *>(misc + kMiscRed);
+  const int hf = tid >> 7, i = tid & 127;   // column half, row
+  const Halves X{reinterpret_cast<float *>(misc + kMiscX), hf, i};
   const CUtensorMap *maps[4] = {&tm_q, &tm_k, &tm_v, &tm_g};
   const uint32_t offs[4] = {kOffQ, kOffK, kOffV, kOffG};
   int issued[4] = {0, 0, 0, 0}, waited[4] = {0, 0, 0, 0};   // thread 0: copies per tile
@@ -291,32 +335,41 @@ __global__ void __launch_bounds__(NT, 1)
     ++issued[which];
   };
   if (tid == 0) {
-    for (int i = 0; i < kNumBars; ++i) mbar_init(bar(i), 1);
+    for (int b = 0; b < kNumBars; ++b) mbar_init(bar(b), 1);
     *flag = 0;
     fence_mbar_init();
-    for (int i = 0; i < 4; ++i) tma_prefetch_desc(maps[i]);
+    for (int b = 0; b < 4; ++b) tma_prefetch_desc(maps[b]);
   }
   if (warp == 0) {
     tmem_alloc(smem_u32(tmem_slot), 512);
     tmem_relinquish();
   }
-  pw[tid] = pow_int(L, tid);
-  dpw[tid] = tid == 0 ? 0.f : static_cast<float>(tid) * pow_int(L, tid - 1);
-  pwr[tid] = pow_int(L, C - 1 - tid);
+  if (tid < 128) {
+    pw[tid] = pow_int(L, tid);
+    dpw[tid] = tid == 0 ? 0.f : static_cast<float>(tid) * pow_int(L, tid - 1);
+    pwr[tid] = pow_int(L, C - 1 - tid);
+    zt[tid] = 0.f;
+    sv[tid] = 0.f;
+  }
   if (tid == 0) {
     pw[C] = pow_int(L, C);
     dpw[C] = static_cast<float>(C) * pow_int(L, C - 1);
   }
-  zt[tid] = 0.f;
-  sv[tid] = 0.f;
   fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t lf = static_cast<uint32_t>(warp * 32) << 16;
+  const uint32_t lf = static_cast<uint32_t>((warp & 3) * 32) << 16;
   if (tid == 0 && nch > 0)
-    for (int i = 0; i < 4; ++i) load(i, 0);
+    for (int b = 0; b < 4; ++b) load(b, 0);
+  float geo = 0.f;   // sum_s lambda^(C-1-s) over a chunk
+  for (int m = 0; m < C; ++m) geo += pwr[m];
+  if (tid < 128) {
+    float g = 0.f;
+    for (int m = 0; m <= tid; ++m) g += pw[m];
+    gs[tid] = g;
+  }
   // thread 0 waits (bounded); every thread learns the verdict at the barrier
   auto poll = [&](int b, int parity) {
     if (tid == 0 && !*flag) {
@@ -336,33 +389,29 @@ __global__ void __launch_bounds__(NT, 1)
   const uint64_t dQ = kdesc(sb + kOffQ), dK = kdesc(sb + kOffK), dKm = mdesc(sb + kOffK);
   const uint64_t dV = kdesc(sb + kOffV), dVm = mdesc(sb + kOffV);
   const uint64_t dSb = kdesc(sb + kOffSb), dSbm = mdesc(sb + kOffSb);
-  const int i = tid;            // token row of the chunk (and d_k, d_v row of the state)
-  float dl = 0.f;               // this thread's share of dlambda
-  float zeta = 0.f;             // sum of the decay weights of the keys before the chunk
-  float geo = 0.f;              // sum_s lambda^(C-1-s) over a chunk
-  for (int m = 0; m < C; ++m) geo += pwr[m];
-  {
-    float g = 0.f;
-    for (int m = 0; m <= tid; ++m) g += pw[m];
-    gs[tid] = g;
-  }
-  __syncthreads();
-  uint8_t *ap_row = sm + kOffAp + static_cast<uint32_t>(i) * 256u;   // A' row, thread-private
+  float dl = 0.f;      // this thread's share of dlambda
+  float zeta = 0.f;    // sum of the decay weights of the keys before the chunk
+  uint8_t *ap_row = sm + kOffAp + static_cast<uint32_t>(i) * 256u;   // At' row (its two halves)
+  const int b0 = 2 * hf;   // this half's first 32-column block
   const float lf_i = pw[i + 1];
 
   for (int c = 0; c < nch; ++c) {
     const int row0 = c * C, Cv = min(C, N - row0);
     const bool carried = c > 0, last = c == nch - 1;
     // ---- the state before this chunk: bf16 operand, and lambda^C St kept for the update
-    if (carried) state_to_operand(tmem + kTmS + lf, sm + kOffSb, i, pw[C]);
+    if (carried) state_to_operand(tmem + kTmS + lf, sm + kOffSb, i, hf, pw[C]);
     poll(kFullQ, c);
     if (!meet()) break;
-    float rq = 0.f;
-    const float qzt = phi_row(sm + kOffQ, i, ident, zt, &rq);   // phi(q_i) . zt, row sum
-    const float qz = qzt + o * rq * zeta;                       // phi(q_i) . z
+    {
+      float rqh = 0.f;
+      X.put(kXQz, phi_row(sm + kOffQ, i, hf, ident, zt, &rqh));   // phi(q_i) . zt, half
+      X.put(kXRq, rqh);
+    }
     poll(kFullK, c);
     if (!meet()) break;
-    elu_row(sm + kOffK, i, ident);
+    const float rq = X.get(kXRq), qzt = X.get(kXQz);
+    const float qz = qzt + o * rq * zeta;   // phi(q_i) . z
+    elu_row(sm + kOffK, i, hf, ident);
     fence_proxy_async_smem();
     if (!meet()) break;
     if (tid == 0) {
@@ -372,30 +421,30 @@ __global__ void __launch_bounds__(NT, 1)
     }
     mma_done();
     if (!meet()) break;
-    // ---- the score weights A = (o rq 1^T + Q Kt^T) o M: the small part
-    // At = (Q Kt^T) o M into TMEM (bf16), At' = (Q Kt^T) o M' into shared
-    // memory; the o rq part stays exact (row sum o rq g_t here, its products
-    // with V and w through the masked row sums of W below)
-    float rs = o * rq * gs[i];
+    // ---- At = (Q Kt^T) o M into TMEM (bf16), At' = (Q Kt^T) o M' into shared memory
+    {
+      float rsh = 0.f;
 #pragma unroll 1
-    for (int blk = 0; blk < 4; ++blk) {
-      uint32_t v[32];
-      tmem_ld_32x32b_x32(tmem + lf + kTmT1 + blk * 32, v);
-      tmem_wait_ld();
-      uint32_t pa[16], pp[16];
+      for (int blk = b0; blk < b0 + 2; ++blk) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tmem + lf + kTmT1 + blk * 32, v);
+        tmem_wait_ld();
+        uint32_t pa[16], pp[16];
 #pragma unroll
-      for (int e = 0; e < 32; e += 2) {
-        const int s0 = blk * 32 + e, s1 = s0 + 1;
-        const float p0 = __uint_as_float(v[e]), p1 = __uint_as_float(v[e + 1]);
-        pa[e / 2] = pack_bf16(p0 * tab(pw, i - s0), p1 * tab(pw, i - s1));
-        rs += blo(pa[e / 2]) + bhi(pa[e / 2]);
-        pp[e / 2] = pack_bf16(p0 * tab(dpw, i - s0), p1 * tab(dpw, i - s1));
+        for (int e = 0; e < 32; e += 2) {
+          const int s0 = blk * 32 + e, s1 = s0 + 1;
+          const float p0 = __uint_as_float(v[e]), p1 = __uint_as_float(v[e + 1]);
+          pa[e / 2] = pack_bf16(p0 * tab(pw, i - s0), p1 * tab(pw, i - s1));
+          rsh += blo(pa[e / 2]) + bhi(pa[e / 2]);
+          pp[e / 2] = pack_bf16(p0 * tab(dpw, i - s0), p1 * tab(dpw, i - s1));
+        }
+        tmem_st_32x32b_x16(tmem + lf + kTmA + blk * 16, pa);
+#pragma unroll
+        for (int m = 0; m < 4; ++m)
+          *reinterpret_cast<uint4 *>(ap_row + (((blk * 4 + m) ^ (i & 15)) << 4)) =
+              make_uint4(pp[4 * m], pp[4 * m + 1], pp[4 * m + 2], pp[4 * m + 3]);
       }
-      tmem_st_32x32b_x16(tmem + lf + kTmA + blk * 16, pa);
-#pragma unroll
-      for (int m = 0; m < 4; ++m)
-        *reinterpret_cast<uint4 *>(ap_row + (((blk * 4 + m) ^ (i & 15)) << 4)) =
-            make_uint4(pp[4 * m], pp[4 * m + 1], pp[4 * m + 2], pp[4 * m + 3]);
+      X.put(kXRs, rsh);
     }
     tmem_wait_st();
     poll(kFullV, c);
@@ -408,37 +457,41 @@ __global__ void __launch_bounds__(NT, 1)
     poll(kFullG, c);
     if (!meet()) break;
     // ---- den, dnum (bf16 into TMEM) and dnum . num but for its o rq part
-    const float den = lf_i * qz + rs + eps, inv = 1.f / den;
-    float gn = 0.f, sd = 0.f;   // dnum . (At V + carried part), dnum . s
+    const float den = lf_i * qz + o * rq * gs[i] + X.get(kXRs) + eps, inv = 1.f / den;
+    {
+      float gnh = 0.f, sdh = 0.f;   // dnum . (At V + carried part), dnum . s
 #pragma unroll 1
-    for (int blk = 0; blk < 4; ++blk) {
-      uint32_t av[32], xv[32];
-      tmem_ld_32x32b_x32(tmem + lf + kTmT1 + blk * 32, av);
-      if (carried) tmem_ld_32x32b_x32(tmem + lf + kTmT2 + blk * 32, xv);
-      tmem_wait_ld();
-      uint32_t pk[16];
+      for (int blk = b0; blk < b0 + 2; ++blk) {
+        uint32_t av[32], xv[32];
+        tmem_ld_32x32b_x32(tmem + lf + kTmT1 + blk * 32, av);
+        if (carried) tmem_ld_32x32b_x32(tmem + lf + kTmT2 + blk * 32, xv);
+        tmem_wait_ld();
+        uint32_t pk[16];
 #pragma unroll
-      for (int m = 0; m < 4; ++m) {
-        const uint4 g4 = *reinterpret_cast<const uint4 *>(sm + kOffG + toff(i, blk * 4 + m));
-        const uint32_t g[4] = {g4.x, g4.y, g4.z, g4.w};
+        for (int m = 0; m < 4; ++m) {
+          const uint4 g4 = *reinterpret_cast<const uint4 *>(sm + kOffG + toff(i, blk * 4 + m));
+          const uint32_t g[4] = {g4.x, g4.y, g4.z, g4.w};
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int e = 8 * m + 2 * u, v0 = blk * 32 + e;
-          float n0 = __uint_as_float(av[e]), n1 = __uint_as_float(av[e + 1]);
-          if (carried) {
-            n0 += lf_i * (__uint_as_float(xv[e]) + o * rq * sv[v0]);
-            n1 += lf_i * (__uint_as_float(xv[e + 1]) + o * rq * sv[v0 + 1]);
+          for (int u = 0; u < 4; ++u) {
+            const int e = 8 * m + 2 * u, v0 = blk * 32 + e;
+            float n0 = __uint_as_float(av[e]), n1 = __uint_as_float(av[e + 1]);
+            if (carried) {
+              n0 += lf_i * (__uint_as_float(xv[e]) + o * rq * sv[v0]);
+              n1 += lf_i * (__uint_as_float(xv[e + 1]) + o * rq * sv[v0 + 1]);
+            }
+            // dden from the bf16 dnum the MMAs use, so that dnum . v + dden (the
+            // weight of every key) is exact up to the fp32 sums even where the
+            // two terms nearly cancel
+            pk[4 * m + u] = pack_bf16(blo(g[u]) * inv, bhi(g[u]) * inv);
+            const float d0 = blo(pk[4 * m + u]), d1 = bhi(pk[4 * m + u]);
+            gnh += d0 * n0 + d1 * n1;
+            sdh += d0 * sv[v0] + d1 * sv[v0 + 1];
           }
-          // dden from the bf16 dnum the MMAs use, so that dnum . v + dden (the
-          // weight of every key) is exact up to the fp32 sums even where the
-          // two terms nearly cancel
-          pk[4 * m + u] = pack_bf16(blo(g[u]) * inv, bhi(g[u]) * inv);
-          const float d0 = blo(pk[4 * m + u]), d1 = bhi(pk[4 * m + u]);
-          gn += d0 * n0 + d1 * n1;
-          sd += d0 * sv[v0] + d1 * sv[v0 + 1];
         }
+        tmem_st_32x32b_x16(tmem + lf + kTmW + blk * 16, pk);
       }
-      tmem_st_32x32b_x16(tmem + lf + kTmW + blk * 16, pk);
+      X.put(kXGn, gnh);
+      X.put(kXSd, sdh);
     }
     tmem_wait_st();
     if (!meet()) break;
@@ -450,46 +503,54 @@ __global__ void __launch_bounds__(NT, 1)
     }
     mma_done();
     if (!meet()) break;
-    // ---- dden = -dnum . num / den, the o rq part from the masked row sum of
-    // W = w V^T; den and dden kept for pass R
-    float gw = 0.f;
+    const float gn = X.get(kXGn), sd = X.get(kXSd);
+    // ---- dden = -dnum . num / den, the o rq part from the masked row sum of W
+    {
+      float gwh = 0.f;
 #pragma unroll 1
-    for (int blk = 0; blk < 4; ++blk) {
-      uint32_t v[32];
-      tmem_ld_32x32b_x32(tmem + lf + kTmT1 + blk * 32, v);
-      tmem_wait_ld();
+      for (int blk = b0; blk < b0 + 2; ++blk) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tmem + lf + kTmT1 + blk * 32, v);
+        tmem_wait_ld();
 #pragma unroll
-      for (int e = 0; e < 32; ++e) gw += __uint_as_float(v[e]) * tab(pw, i - blk * 32 - e);
+        for (int e = 0; e < 32; ++e) gwh += __uint_as_float(v[e]) * tab(pw, i - blk * 32 - e);
+      }
+      X.put(kXGw, gwh);
     }
-    const float dden = -(gn + o * rq * gw) * inv;
-    if (i < Cv)
+    __syncthreads();
+    const float dden = -(gn + o * rq * X.get(kXGw)) * inv;
+    if (hf == 0 && i < Cv)
       *reinterpret_cast<float2 *>(stash + (bh * N + row0 + i) * stash_stride) =
           make_float2(den, dden);
     // ---- B = (W + dden) o M into TMEM, its fp32 row sum; dlambda, pairs inside the chunk
-    float rb = 0.f;
+    {
+      float rbh = 0.f;
 #pragma unroll 1
-    for (int blk = 0; blk < 4; ++blk) {
-      uint32_t v[32];
-      tmem_ld_32x32b_x32(tmem + lf + kTmT1 + blk * 32, v);
-      tmem_wait_ld();
-      uint32_t pb[16];
+      for (int blk = b0; blk < b0 + 2; ++blk) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tmem + lf + kTmT1 + blk * 32, v);
+        tmem_wait_ld();
+        uint32_t pb[16];
 #pragma unroll
-      for (int m = 0; m < 4; ++m) {
-        const uint4 a4 = *reinterpret_cast<const uint4 *>(ap_row + (((blk * 4 + m) ^ (i & 15)) << 4));
-        const uint32_t ap[4] = {a4.x, a4.y, a4.z, a4.w};
+        for (int m = 0; m < 4; ++m) {
+          const uint4 a4 =
+              *reinterpret_cast<const uint4 *>(ap_row + (((blk * 4 + m) ^ (i & 15)) << 4));
+          const uint32_t ap[4] = {a4.x, a4.y, a4.z, a4.w};
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int e = 8 * m + 2 * u;
-          const int s0 = blk * 32 + e, s1 = s0 + 1;
-          const float w0 = __uint_as_float(v[e]) + dden, w1 = __uint_as_float(v[e + 1]) + dden;
-          dl += (blo(ap[u]) + o * rq * tab(dpw, i - s0)) * w0 +
-                (bhi(ap[u]) + o * rq * tab(dpw, i - s1)) * w1;
-          const float b0 = w0 * tab(pw, i - s0), b1 = w1 * tab(pw, i - s1);
-          rb += b0 + b1;
-          pb[4 * m + u] = pack_bf16(b0, b1);
+          for (int u = 0; u < 4; ++u) {
+            const int e = 8 * m + 2 * u;
+            const int s0 = blk * 32 + e, s1 = s0 + 1;
+            const float w0 = __uint_as_float(v[e]) + dden, w1 = __uint_as_float(v[e + 1]) + dden;
+            dl += (blo(ap[u]) + o * rq * tab(dpw, i - s0)) * w0 +
+                  (bhi(ap[u]) + o * rq * tab(dpw, i - s1)) * w1;
+            const float bb0 = w0 * tab(pw, i - s0), bb1 = w1 * tab(pw, i - s1);
+            rbh += bb0 + bb1;
+            pb[4 * m + u] = pack_bf16(bb0, bb1);
+          }
         }
+        tmem_st_32x32b_x16(tmem + lf + kTmA + blk * 16, pb);
       }
-      tmem_st_32x32b_x16(tmem + lf + kTmA + blk * 16, pb);
+      X.put(kXRb, rbh);
     }
     tmem_wait_st();
     if (!meet()) break;
@@ -502,11 +563,11 @@ __global__ void __launch_bounds__(NT, 1)
     // ---- dq = (B Kt + o B1 + lambda^(t+1) (U + zt dden + o (s.w + zeta dden))) phi'(q);
     //      dlambda, keys before the chunk (the lambda^(t+1) factor's derivative)
     {
-      float qu = 0.f;
-      const float one = o * (rb + (carried ? lf_i * (sd + zeta * dden) : 0.f));
+      float quh = 0.f;
+      const float one = o * (X.get(kXRb) + (carried ? lf_i * (sd + zeta * dden) : 0.f));
       __nv_bfloat16 *dst = dq + (bh * N + row0 + i) * static_cast<long>(D);
 #pragma unroll 1
-      for (int blk = 0; blk < 4; ++blk) {
+      for (int blk = b0; blk < b0 + 2; ++blk) {
         uint32_t bk[32], uv[32];
         tmem_ld_32x32b_x32(tmem + lf + kTmT1 + blk * 32, bk);
         if (carried) tmem_ld_32x32b_x32(tmem + lf + kTmT2 + blk * 32, uv);
@@ -522,7 +583,7 @@ __global__ void __launch_bounds__(NT, 1)
             const float u0 = carried ? __uint_as_float(uv[e]) : 0.f;
             const float u1 = carried ? __uint_as_float(uv[e + 1]) : 0.f;
             const float q0 = blo(qw[u]), q1 = bhi(qw[u]);
-            qu += q0 * u0 + q1 * u1;
+            quh += q0 * u0 + q1 * u1;
             float g0 = __uint_as_float(bk[e]) + one + lf_i * (u0 + dden * zt[k0]);
             float g1 = __uint_as_float(bk[e + 1]) + one + lf_i * (u1 + dden * zt[k0 + 1]);
             if (!ident) {
@@ -538,11 +599,13 @@ __global__ void __launch_bounds__(NT, 1)
             reinterpret_cast<uint4 *>(dst + blk * 32)[m] =
                 make_uint4(pk[4 * m], pk[4 * m + 1], pk[4 * m + 2], pk[4 * m + 3]);
       }
-      if (carried) dl += dpw[i + 1] * (qu + dden * qzt + o * rq * (sd + zeta * dden));
+      if (carried)
+        dl += dpw[i + 1] *
+              (quh + (hf == 0 ? dden * qzt + o * rq * (sd + zeta * dden) : 0.f));
     }
     if (last) break;
     // ---- state update: key rows weighted lambda^(C-1-s): St += (Lk Kt)^T V, zt, s, zeta likewise
-    scale_row(sm + kOffK, sm + kOffK, i, pwr[i]);
+    scale_row(sm + kOffK, sm + kOffK, i, hf, pwr[i]);
     fence_proxy_async_smem();
     if (!meet()) break;
     if (tid == 0) {
@@ -550,11 +613,15 @@ __global__ void __launch_bounds__(NT, 1)
       umma_commit(bar(kMma));
       load(0, c + 1);   // the q tile is free
     }
-    zt[i] = pw[C] * zt[i] + col_sum(sm + kOffK, i, nullptr);
-    sv[i] = pw[C] * sv[i] + col_sum(sm + kOffV, i, pwr);
+    X.put(kXZt, col_sum(sm + kOffK, i, hf, nullptr));
+    X.put(kXSv, col_sum(sm + kOffV, i, hf, pwr));
     zeta = pw[C] * zeta + geo;
     mma_done();
     if (!meet()) break;
+    if (tid < 128) {
+      zt[i] = pw[C] * zt[i] + X.get(kXZt);
+      sv[i] = pw[C] * sv[i] + X.get(kXSv);
+    }
     if (tid == 0) {
       load(1, c + 1);
       load(2, c + 1);
@@ -587,7 +654,8 @@ constexpr uint32_t kOffQ = 0, kOffK = kTile, kOffKd = 2 * kTile, kOffV = 3 * kTi
 enum { kFullQ = 0, kFullK, kFullV, kFullG, kMma, kFinal, kNumBars };
 constexpr uint32_t kMiscTmem = 64, kMiscFlag = 68, kMiscPw = 128;
 constexpr uint32_t kMiscDden = kMiscPw + 132 * 4, kMiscR = kMiscDden + 128 * 4;
-constexpr uint32_t kSmemBytes = kOffMisc + kMiscR + 128 * 4;
+constexpr uint32_t kMiscX = kMiscR + 128 * 4;
+constexpr uint32_t kSmemBytes = kOffMisc + kMiscX + 2 * 128 * 4;
 static_assert(kSmemBytes <= 232448, "exceeds the per-CTA shared memory of sm_100");
 constexpr uint32_t kTmR = 0, kTmT1 = 128, kTmT2 = 256, kTmAt = 384, kTmBt = 448;
 }  // namespace pr
@@ -618,6 +686,8 @@ __global__ void __launch_bounds__(NT, 1)
   float *pw = reinterpret_cast<float *>(misc + kMiscPw);
   float *sdd = reinterpret_cast<float *>(misc + kMiscDden);   // dden of the chunk's tokens
   float *rv = reinterpret_cast<float *>(misc + kMiscR);       // r, the normaliser's adjoint
+  const int hf = tid >> 7, i = tid & 127;
+  const Halves X{reinterpret_cast<float *>(misc + kMiscX), hf, i};
   const CUtensorMap *maps[4] = {&tm_q, &tm_k, &tm_v, &tm_g};
   const uint32_t offs[4] = {kOffQ, kOffK, kOffV, kOffG};
   int issued[4] = {0, 0, 0, 0}, waited[4] = {0, 0, 0, 0};
@@ -631,26 +701,28 @@ __global__ void __launch_bounds__(NT, 1)
     ++issued[which];
   };
   if (tid == 0) {
-    for (int i = 0; i < kNumBars; ++i) mbar_init(bar(i), 1);
+    for (int b = 0; b < kNumBars; ++b) mbar_init(bar(b), 1);
     *flag = 0;
     fence_mbar_init();
-    for (int i = 0; i < 4; ++i) tma_prefetch_desc(maps[i]);
+    for (int b = 0; b < 4; ++b) tma_prefetch_desc(maps[b]);
   }
   if (warp == 0) {
     tmem_alloc(smem_u32(tmem_slot), 512);
     tmem_relinquish();
   }
-  pw[tid] = pow_int(L, tid);
+  if (tid < 128) {
+    pw[tid] = pow_int(L, tid);
+    rv[tid] = 0.f;
+  }
   if (tid == 0) pw[C] = pow_int(L, C);
-  rv[tid] = 0.f;
   fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t lf = static_cast<uint32_t>(warp * 32) << 16;
+  const uint32_t lf = static_cast<uint32_t>((warp & 3) * 32) << 16;
   if (tid == 0 && nch > 0)
-    for (int i = 0; i < 4; ++i) load(i, nch - 1);
+    for (int b = 0; b < 4; ++b) load(b, nch - 1);
   auto poll = [&](int b, int parity) {
     if (tid == 0 && !*flag) {
       if (!mbar_wait(bar(b), static_cast<uint32_t>(parity) & 1u)) *flag = 1;
@@ -670,7 +742,7 @@ __global__ void __launch_bounds__(NT, 1)
   const uint64_t dKd = kdesc(sb + kOffKd), dV = kdesc(sb + kOffV), dVd = kdesc(sb + kOffVd);
   const uint64_t dG = kdesc(sb + kOffG), dGm = mdesc(sb + kOffG);
   const uint64_t dRb = kdesc(sb + kOffRb), dRbm = mdesc(sb + kOffRb);
-  const int i = tid;   // token row (key j of the formulas) and d_k row of R
+  const int b0 = 2 * hf;
 
   for (int cc = 0; cc < nch; ++cc) {
     const int c = nch - 1 - cc, row0 = c * C, Cv = min(C, N - row0);
@@ -682,33 +754,20 @@ __global__ void __launch_bounds__(NT, 1)
       den = st.x;
       dden = st.y;
     }
-    sdd[i] = dden;
-    if (carried) state_to_operand(tmem + kTmR + lf, sm + kOffRb, i, pw[C]);
+    if (hf == 0) sdd[i] = dden;
+    if (carried) state_to_operand(tmem + kTmR + lf, sm + kOffRb, i, hf, pw[C]);
     poll(kFullQ, cc);
     poll(kFullK, cc);
     poll(kFullV, cc);
     poll(kFullG, cc);
     if (!meet()) break;
-    phi_row(sm + kOffQ, i, ident, nullptr);
-    phi_row(sm + kOffK, i, ident, nullptr);
+    phi_row(sm + kOffQ, i, hf, ident, nullptr);
+    phi_row(sm + kOffK, i, hf, ident, nullptr);
     if (carried) {
-      scale_row(sm + kOffKd, sm + kOffK, i, pw[C - 1 - i]);
-      scale_row(sm + kOffVd, sm + kOffV, i, pw[C - 1 - i]);
+      scale_row(sm + kOffKd, sm + kOffK, i, hf, pw[C - 1 - i]);
+      scale_row(sm + kOffVd, sm + kOffV, i, hf, pw[C - 1 - i]);
     }
-    {
-      // w = dnum = dy / den in place of dy
-      const float inv = 1.f / den;
-#pragma unroll 4
-      for (int j = 0; j < 16; ++j) {
-        uint4 *p = reinterpret_cast<uint4 *>(sm + kOffG + toff(i, j));
-        uint4 g = *p;
-        g.x = pack_bf16(blo(g.x) * inv, bhi(g.x) * inv);
-        g.y = pack_bf16(blo(g.y) * inv, bhi(g.y) * inv);
-        g.z = pack_bf16(blo(g.z) * inv, bhi(g.z) * inv);
-        g.w = pack_bf16(blo(g.w) * inv, bhi(g.w) * inv);
-        *p = g;
-      }
-    }
+    dnum_row(sm + kOffG, i, hf, 1.f / den);   // w = dnum in place of dy
     fence_proxy_async_smem();
     if (!meet()) break;
     if (tid == 0) {
@@ -721,7 +780,7 @@ __global__ void __launch_bounds__(NT, 1)
     if (tid == 0 && c > 0) load(2, c - 1);   // v has been read (its weighted copy is made)
     // ---- A^T and B^T rows (key i, queries s >= i) into TMEM
 #pragma unroll 1
-    for (int blk = 0; blk < 4; ++blk) {
+    for (int blk = b0; blk < b0 + 2; ++blk) {
       uint32_t pv[32], wv[32];
       tmem_ld_32x32b_x32(tmem + lf + kTmT1 + blk * 32, pv);
       tmem_ld_32x32b_x32(tmem + lf + kTmT2 + blk * 32, wv);
@@ -755,7 +814,7 @@ __global__ void __launch_bounds__(NT, 1)
       __nv_bfloat16 *vd = dv + (bh * N + row0 + i) * static_cast<long>(D);
       __nv_bfloat16 *kd = dk + (bh * N + row0 + i) * static_cast<long>(D);
 #pragma unroll 1
-      for (int blk = 0; blk < 4; ++blk) {
+      for (int blk = b0; blk < b0 + 2; ++blk) {
         uint32_t a[32], b[32];
         tmem_ld_32x32b_x32(tmem + lf + kTmT1 + blk * 32, a);
         tmem_ld_32x32b_x32(tmem + lf + kTmT2 + blk * 32, b);
@@ -790,7 +849,7 @@ __global__ void __launch_bounds__(NT, 1)
     }
     if (c == 0) break;
     // ---- R += (Lq Q)^T w, r likewise: q rows weighted lambda^(t+1)
-    scale_row(sm + kOffQ, sm + kOffQ, i, pw[i + 1]);
+    scale_row(sm + kOffQ, sm + kOffQ, i, hf, pw[i + 1]);
     fence_proxy_async_smem();
     if (!meet()) break;
     if (tid == 0) {
@@ -798,9 +857,10 @@ __global__ void __launch_bounds__(NT, 1)
       umma_commit(bar(kMma));
       load(1, c - 1);   // k has been read
     }
-    rv[i] = pw[C] * rv[i] + col_sum(sm + kOffQ, i, sdd);
+    X.put(0, col_sum(sm + kOffQ, i, hf, sdd));
     mma_done();
     if (!meet()) break;
+    if (tid < 128) rv[i] = pw[C] * rv[i] + X.get(0);
     if (tid == 0) {
       load(0, c - 1);
       load(3, c - 1);
@@ -837,8 +897,9 @@ constexpr uint32_t kMiscDpw = kMiscPw + 132 * 4, kMiscPwr = kMiscDpw + 132 * 4;
 constexpr uint32_t kMiscDpwr = kMiscPwr + 128 * 4, kMiscZ = kMiscDpwr + 128 * 4;
 constexpr uint32_t kMiscZp = kMiscZ + 128 * 4, kMiscS = kMiscZp + 128 * 4;
 constexpr uint32_t kMiscSp = kMiscS + 128 * 4, kMiscWq = kMiscSp + 128 * 4;
-constexpr uint32_t kMiscRed = kMiscWq + 128 * 4;
-constexpr uint32_t kSmemBytes = kOffMisc + kMiscRed + 64;
+constexpr uint32_t kMiscRed = kMiscWq + 128 * 4, kMiscX = kMiscRed + 64;
+enum { kXQz = 0, kXRq, kXZt, kXZtp, kXSv, kXSvp, kNumX };
+constexpr uint32_t kSmemBytes = kOffMisc + kMiscX + kNumX * 2 * 128 * 4;
 static_assert(kSmemBytes <= 232448, "exceeds the per-CTA shared memory of sm_100");
 constexpr uint32_t kTmS = 0, kTmSp = 128, kTmM = 256;
 }  // namespace pl
@@ -876,6 +937,8 @@ __global__ void __launch_bounds__(NT, 1)
   float *svp = reinterpret_cast<float *>(misc + kMiscSp);
   float *wq = reinterpret_cast<float *>(misc + kMiscWq);       // lambda^(t+1) rq_t
   float *red = reinterpret_cast<float *>(misc + kMiscRed);
+  const int hf = tid >> 7, i = tid & 127;
+  const Halves X{reinterpret_cast<float *>(misc + kMiscX), hf, i};
   const CUtensorMap *maps[4] = {&tm_q, &tm_k, &tm_v, &tm_g};
   const uint32_t offs[4] = {kOffQ, kOffK, kOffV, kOffG};
   int issued[4] = {0, 0, 0, 0}, waited[4] = {0, 0, 0, 0};
@@ -889,35 +952,37 @@ __global__ void __launch_bounds__(NT, 1)
     ++issued[which];
   };
   if (tid == 0) {
-    for (int i = 0; i < kNumBars; ++i) mbar_init(bar(i), 1);
+    for (int b = 0; b < kNumBars; ++b) mbar_init(bar(b), 1);
     *flag = 0;
     fence_mbar_init();
-    for (int i = 0; i < 4; ++i) tma_prefetch_desc(maps[i]);
+    for (int b = 0; b < 4; ++b) tma_prefetch_desc(maps[b]);
   }
   if (warp == 0) {
     tmem_alloc(smem_u32(tmem_slot), 512);
     tmem_relinquish();
   }
-  pw[tid] = pow_int(L, tid);
-  dpw[tid] = tid == 0 ? 0.f : static_cast<float>(tid) * pow_int(L, tid - 1);
-  pwr[tid] = pow_int(L, C - 1 - tid);
-  dpwr[tid] = tid == C - 1 ? 0.f : static_cast<float>(C - 1 - tid) * pow_int(L, C - 2 - tid);
+  if (tid < 128) {
+    pw[tid] = pow_int(L, tid);
+    dpw[tid] = tid == 0 ? 0.f : static_cast<float>(tid) * pow_int(L, tid - 1);
+    pwr[tid] = pow_int(L, C - 1 - tid);
+    dpwr[tid] = tid == C - 1 ? 0.f : static_cast<float>(C - 1 - tid) * pow_int(L, C - 2 - tid);
+    zt[tid] = 0.f;
+    ztp[tid] = 0.f;
+    sv[tid] = 0.f;
+    svp[tid] = 0.f;
+  }
   if (tid == 0) {
     pw[C] = pow_int(L, C);
     dpw[C] = static_cast<float>(C) * pow_int(L, C - 1);
   }
-  zt[tid] = 0.f;
-  ztp[tid] = 0.f;
-  sv[tid] = 0.f;
-  svp[tid] = 0.f;
   fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t lf = static_cast<uint32_t>(warp * 32) << 16;
+  const uint32_t lf = static_cast<uint32_t>((warp & 3) * 32) << 16;
   if (tid == 0 && nch > 0)
-    for (int i = 0; i < 4; ++i) load(i, 0);
+    for (int b = 0; b < 4; ++b) load(b, 0);
   // the reverse pass (launched after this one as its programmatic dependent,
   // when the stash is not in dk) reads nothing this pass writes: let it start
   grid_launch_dependents();
@@ -938,7 +1003,7 @@ __global__ void __launch_bounds__(NT, 1)
 
   const uint64_t dQm = mdesc(sb + kOffQ), dKm = mdesc(sb + kOffK), dKpm = mdesc(sb + kOffKp);
   const uint64_t dVm = mdesc(sb + kOffV), dGm = mdesc(sb + kOffG);
-  const int i = tid;
+  const int b0 = 2 * hf;
   float dl = 0.f;
   float zeta = 0.f, zetap = 0.f;
   float geo = 0.f, dgeo = 0.f;
@@ -958,32 +1023,22 @@ __global__ void __launch_bounds__(NT, 1)
     }
     poll(kFullQ, c);
     poll(kFullK, c);
+    poll(kFullV, c);
     poll(kFullG, c);
     if (!meet()) break;
-    // q rows weighted lambda^(t+1); the z' part of dlambda
-    float rq = 0.f;
-    const float qztp = phi_row(sm + kOffQ, i, ident, ztp, &rq);
-    dl += dden * pw[i + 1] * (qztp + o * rq * zetap);
-    wq[i] = pw[i + 1] * rq;
-    scale_row(sm + kOffQ, sm + kOffQ, i, pw[i + 1]);
+    // q rows weighted lambda^(t+1); the half sums of phi(q) . zt' and of phi(q)
     {
-      const float inv = 1.f / den;
-#pragma unroll 4
-      for (int j = 0; j < 16; ++j) {
-        uint4 *p = reinterpret_cast<uint4 *>(sm + kOffG + toff(i, j));
-        uint4 g = *p;
-        g.x = pack_bf16(blo(g.x) * inv, bhi(g.x) * inv);
-        g.y = pack_bf16(blo(g.y) * inv, bhi(g.y) * inv);
-        g.z = pack_bf16(blo(g.z) * inv, bhi(g.z) * inv);
-        g.w = pack_bf16(blo(g.w) * inv, bhi(g.w) * inv);
-        *p = g;
-      }
+      float rqh = 0.f;
+      X.put(kXQz, phi_row(sm + kOffQ, i, hf, ident, ztp, &rqh));
+      X.put(kXRq, rqh);
     }
+    scale_row(sm + kOffQ, sm + kOffQ, i, hf, pw[i + 1]);
+    dnum_row(sm + kOffG, i, hf, 1.f / den);
     if (!last) {
       // key rows as elu(k), weighted lambda^(C-1-s) (state) and (C-1-s) lambda^(C-2-s) (derivative)
-      elu_row(sm + kOffK, i, ident);
-      scale_row(sm + kOffKp, sm + kOffK, i, dpwr[i]);
-      scale_row(sm + kOffK, sm + kOffK, i, pwr[i]);
+      elu_row(sm + kOffK, i, hf, ident);
+      scale_row(sm + kOffKp, sm + kOffK, i, hf, dpwr[i]);
+      scale_row(sm + kOffK, sm + kOffK, i, hf, pwr[i]);
     }
     fence_proxy_async_smem();
     if (!meet()) break;
@@ -991,8 +1046,17 @@ __global__ void __launch_bounds__(NT, 1)
       mma_ss(tmem + kTmM, dQm, true, dGm, true, false);   // Ms = (Lq Q)^T w
       umma_commit(bar(kMma));
     }
-    // o s' . (1^T Ms) on this thread's d_v column (s' of the chunk start)
-    dl += o * svp[i] * col_sum(sm + kOffG, i, wq);
+    {
+      // the z' part of dlambda (once per row), and lambda^(t+1) rq_t for 1^T Ms
+      const float rq = X.get(kXRq);
+      if (hf == 0) {
+        dl += dden * pw[i + 1] * (X.get(kXQz) + o * rq * zetap);
+        wq[i] = pw[i + 1] * rq;
+      }
+    }
+    __syncthreads();
+    // o s' . (1^T Ms) on this thread's d_v column (s' of the chunk start), half of the rows
+    dl += o * svp[i] * col_sum(sm + kOffG, i, hf, wq);
     mma_done();
     if (!meet()) break;
     if (tid == 0 && !last) {
@@ -1002,7 +1066,7 @@ __global__ void __launch_bounds__(NT, 1)
     // <St', Ms> on this thread's d_k row; then St' <- lambda^C St' + C lambda^(C-1) St, St <- lambda^C St
     if (carried) {
 #pragma unroll 1
-      for (int blk = 0; blk < 4; ++blk) {
+      for (int blk = b0; blk < b0 + 2; ++blk) {
         uint32_t sp[32], mv[32], sq[32];
         tmem_ld_32x32b_x32(tmem + lf + kTmSp + blk * 32, sp);
         tmem_ld_32x32b_x32(tmem + lf + kTmM + blk * 32, mv);
@@ -1023,20 +1087,25 @@ __global__ void __launch_bounds__(NT, 1)
       tmem_wait_st();
     }
     if (last) break;
-    // the vector parts of the state and of its derivative (this thread's d_k / d_v index)
-    ztp[i] = pw[C] * ztp[i] + dpw[C] * zt[i] + col_sum(sm + kOffKp, i, nullptr);
-    zt[i] = pw[C] * zt[i] + col_sum(sm + kOffK, i, nullptr);
-    svp[i] = pw[C] * svp[i] + dpw[C] * sv[i] + col_sum(sm + kOffV, i, dpwr);
-    sv[i] = pw[C] * sv[i] + col_sum(sm + kOffV, i, pwr);
-    zetap = pw[C] * zetap + dpw[C] * zeta + dgeo;
-    zeta = pw[C] * zeta + geo;
-    poll(kFullV, c);
+    // the vector parts of the state and of its derivative: half sums over the chunk's rows
+    X.put(kXZtp, col_sum(sm + kOffKp, i, hf, nullptr));
+    X.put(kXZt, col_sum(sm + kOffK, i, hf, nullptr));
+    X.put(kXSvp, col_sum(sm + kOffV, i, hf, dpwr));
+    X.put(kXSv, col_sum(sm + kOffV, i, hf, pwr));
     if (!meet()) break;
     if (tid == 0) {
       mma_ss(tmem + kTmS, dKm, true, dVm, true, carried);
       mma_ss(tmem + kTmSp, dKpm, true, dVm, true, carried);
       umma_commit(bar(kMma));
     }
+    if (tid < 128) {
+      ztp[i] = pw[C] * ztp[i] + dpw[C] * zt[i] + X.get(kXZtp);
+      zt[i] = pw[C] * zt[i] + X.get(kXZt);
+      svp[i] = pw[C] * svp[i] + dpw[C] * sv[i] + X.get(kXSvp);
+      sv[i] = pw[C] * sv[i] + X.get(kXSv);
+    }
+    zetap = pw[C] * zetap + dpw[C] * zeta + dgeo;
+    zeta = pw[C] * zeta + geo;
     mma_done();
     if (!meet()) break;
     if (tid == 0) {
