@@ -190,21 +190,75 @@ __device__ __forceinline__ void dnum_row(uint8_t *tile, int r, int h, float inv)
   }
 }
 
-// Column k of a bf16 tile summed over rows [64h, 64h + 64) (fp32),
-// optionally weighted per row.
-__device__ __forceinline__ float col_sum(const uint8_t *tile, int k, int h, const float *wrow) {
-  float a0 = 0.f, a1 = 0.f;
-  const uint32_t j = static_cast<uint32_t>(k) >> 3, b = (static_cast<uint32_t>(k) & 7u) * 2u;
-#pragma unroll 8
-  for (int r = 64 * h; r < 64 * h + 64; r += 2) {
-    const float x0 = __uint_as_float(
-        static_cast<uint32_t>(*reinterpret_cast<const uint16_t *>(tile + toff(r, j) + b)) << 16);
-    const float x1 = __uint_as_float(
-        static_cast<uint32_t>(*reinterpret_cast<const uint16_t *>(tile + toff(r + 1, j) + b)) << 16);
-    a0 += wrow ? x0 * wrow[r] : x0;
-    a1 += wrow ? x1 * wrow[r + 1] : x1;
+// Column sums of one or two bf16 tiles over all 128 rows, each optionally
+// weighted per row, by all 256 threads together; thread k < 128 receives the
+// sums of column k in sa and sb.  Thread t reads 16-byte chunk t % 16 of rows
+// t / 16 + 16 m; partial sums meet through `scratch` (2 x 8 x 128 floats, in
+// no live tile).  Holds two block barriers: every thread calls it.
+__device__ __forceinline__ void col_sums(const uint8_t *ta, const float *wa, const uint8_t *tb,
+                                         const float *wb, float *scratch, float &sa, float &sb) {
+  const int t = threadIdx.x, j = t & 15, g = t >> 4, lane = t & 31, w = t >> 5;
+  float a[8], b[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) a[e] = b[e] = 0.f;
+#pragma unroll
+  for (int m = 0; m < 8; ++m) {
+    const int r = g + 16 * m;
+    const uint4 x = *reinterpret_cast<const uint4 *>(ta + toff(r, j));
+    const float fa = wa ? wa[r] : 1.f;
+    const uint32_t xs[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      a[2 * u] += blo(xs[u]) * fa;
+      a[2 * u + 1] += bhi(xs[u]) * fa;
+    }
+    if (tb) {
+      const uint4 y = *reinterpret_cast<const uint4 *>(tb + toff(r, j));
+      const float fb = wb ? wb[r] : 1.f;
+      const uint32_t ys[4] = {y.x, y.y, y.z, y.w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        b[2 * u] += blo(ys[u]) * fb;
+        b[2 * u + 1] += bhi(ys[u]) * fb;
+      }
+    }
   }
-  return a0 + a1;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    a[e] += __shfl_xor_sync(0xffffffffu, a[e], 16);
+    b[e] += __shfl_xor_sync(0xffffffffu, b[e], 16);
+  }
+  if (lane < 16)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      scratch[w * 128 + 8 * j + e] = a[e];
+      scratch[1024 + w * 128 + 8 * j + e] = b[e];
+    }
+  __syncthreads();
+  if (t < 128) {
+    float x = 0.f, y = 0.f;
+#pragma unroll
+    for (int k = 0; k < NT / 32; ++k) {
+      x += scratch[k * 128 + t];
+      y += scratch[1024 + k * 128 + t];
+    }
+    sa = x;
+    sb = y;
+  }
+  __syncthreads();
+}
+
+// Masked power tables with an offset, so that a masked decay factor is one
+// load: lower[127 - t + s] = lambda^(t-s) for s <= t, else 0 (and likewise
+// (t-s) lambda^(t-s-1) in the derivative table); upper[127 - t + s] =
+// lambda^(s-t) for s >= t, else 0.  256 entries each, filled by thread m.
+__device__ __forceinline__ void fill_masked_tables(float L, int m, float *lower, float *dlower,
+                                                   float *upper) {
+  if (m >= 256) return;
+  const int x = 127 - m;   // t - s for lower, -(s - t) for upper
+  if (lower) lower[m] = x >= 0 ? pow_int(L, x) : 0.f;
+  if (dlower) dlower[m] = x >= 1 ? static_cast<float>(x) * pow_int(L, x - 1) : 0.f;
+  if (upper) upper[m] = x <= 0 ? pow_int(L, -x) : 0.f;
 }
 
 // The half row r of the fp32 state in TMEM (this warp's lanes; t already
@@ -229,12 +283,6 @@ __device__ __forceinline__ void state_to_operand(uint32_t t, uint8_t *tile, int 
     tmem_st_32x32b_x32(t + blk * 32, v);
   }
   tmem_wait_st();
-}
-
-// tab[m] for 0 <= m (m < 0: 0); the load index stays in the table either way
-__device__ __forceinline__ float tab(const float *t, int m) {
-  const float x = t[m < 0 ? 0 : m];
-  return m < 0 ? 0.f : x;
 }
 
 __device__ __forceinline__ float block_sum(float x, float *red) {
@@ -281,8 +329,9 @@ constexpr uint32_t kMiscTmem = 64, kMiscFlag = 68, kMiscPw = 128;
 constexpr uint32_t kMiscDpw = kMiscPw + 132 * 4, kMiscPwr = kMiscDpw + 132 * 4;
 constexpr uint32_t kMiscZ = kMiscPwr + 128 * 4, kMiscS = kMiscZ + 128 * 4;
 constexpr uint32_t kMiscGs = kMiscS + 128 * 4, kMiscRed = kMiscGs + 128 * 4;
-constexpr uint32_t kMiscX = kMiscRed + 64;
-enum { kXQz = 0, kXRq, kXRs, kXGn, kXSd, kXGw, kXRb, kXZt, kXSv, kNumX };
+constexpr uint32_t kMiscLo = kMiscRed + 64, kMiscDlo = kMiscLo + 256 * 4;
+constexpr uint32_t kMiscX = kMiscDlo + 256 * 4;
+enum { kXQz = 0, kXRq, kXRs, kXGn, kXSd, kXGw, kXRb, kNumX };
 constexpr uint32_t kSmemBytes = kOffMisc + kMiscX + kNumX * 2 * 128 * 4;
 static_assert(kSmemBytes <= 232448, "exceeds the per-CTA shared memory of sm_100");
 // tensor memory columns
@@ -320,6 +369,8 @@ __global__ void __launch_bounds__(NT, 1)
   float *sv = reinterpret_cast<float *>(misc + kMiscS);
   float *gs = reinterpret_cast<float *>(misc + kMiscGs);     // sum_{m<=t} lambda^m
   float *red = reinterpret_cast<float *>(misc + kMiscRed);
+  float *lo = reinterpret_cast<float *>(misc + kMiscLo);     // masked lambda^(t-s), offset
+  float *dlo = reinterpret_cast<float *>(misc + kMiscDlo);   // masked (t-s) lambda^(t-s-1)
   const int hf = tid >> 7, i = tid & 127;   // column half, row
   const Halves X{reinterpret_cast<float *>(misc + kMiscX), hf, i};
   const CUtensorMap *maps[4] = {&tm_q, &tm_k, &tm_v, &tm_g};
@@ -355,6 +406,7 @@ __global__ void __launch_bounds__(NT, 1)
     pw[C] = pow_int(L, C);
     dpw[C] = static_cast<float>(C) * pow_int(L, C - 1);
   }
+  fill_masked_tables(L, tid, lo, dlo, nullptr);
   fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
@@ -394,6 +446,7 @@ __global__ void __launch_bounds__(NT, 1)
   uint8_t *ap_row = sm + kOffAp + static_cast<uint32_t>(i) * 256u;   // At' row (its two halves)
   const int b0 = 2 * hf;   // this half's first 32-column block
   const float lf_i = pw[i + 1];
+  const float *mk = lo + 127 - i, *dmk = dlo + 127 - i;   // mk[s] = lambda^(i-s) (s <= i) or 0
 
   for (int c = 0; c < nch; ++c) {
     const int row0 = c * C, Cv = min(C, N - row0);
@@ -434,9 +487,9 @@ __global__ void __launch_bounds__(NT, 1)
         for (int e = 0; e < 32; e += 2) {
           const int s0 = blk * 32 + e, s1 = s0 + 1;
           const float p0 = __uint_as_float(v[e]), p1 = __uint_as_float(v[e + 1]);
-          pa[e / 2] = pack_bf16(p0 * tab(pw, i - s0), p1 * tab(pw, i - s1));
+          pa[e / 2] = pack_bf16(p0 * mk[s0], p1 * mk[s1]);
           rsh += blo(pa[e / 2]) + bhi(pa[e / 2]);
-          pp[e / 2] = pack_bf16(p0 * tab(dpw, i - s0), p1 * tab(dpw, i - s1));
+          pp[e / 2] = pack_bf16(p0 * dmk[s0], p1 * dmk[s1]);
         }
         tmem_st_32x32b_x16(tmem + lf + kTmA + blk * 16, pa);
 #pragma unroll
@@ -513,7 +566,7 @@ __global__ void __launch_bounds__(NT, 1)
         tmem_ld_32x32b_x32(tmem + lf + kTmT1 + blk * 32, v);
         tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 32; ++e) gwh += __uint_as_float(v[e]) * tab(pw, i - blk * 32 - e);
+        for (int e = 0; e < 32; ++e) gwh += __uint_as_float(v[e]) * mk[blk * 32 + e];
       }
       X.put(kXGw, gwh);
     }
@@ -541,9 +594,8 @@ __global__ void __launch_bounds__(NT, 1)
             const int e = 8 * m + 2 * u;
             const int s0 = blk * 32 + e, s1 = s0 + 1;
             const float w0 = __uint_as_float(v[e]) + dden, w1 = __uint_as_float(v[e + 1]) + dden;
-            dl += (blo(ap[u]) + o * rq * tab(dpw, i - s0)) * w0 +
-                  (bhi(ap[u]) + o * rq * tab(dpw, i - s1)) * w1;
-            const float bb0 = w0 * tab(pw, i - s0), bb1 = w1 * tab(pw, i - s1);
+            dl += (blo(ap[u]) + o * rq * dmk[s0]) * w0 + (bhi(ap[u]) + o * rq * dmk[s1]) * w1;
+            const float bb0 = w0 * mk[s0], bb1 = w1 * mk[s1];
             rbh += bb0 + bb1;
             pb[4 * m + u] = pack_bf16(bb0, bb1);
           }
@@ -613,15 +665,19 @@ __global__ void __launch_bounds__(NT, 1)
       umma_commit(bar(kMma));
       load(0, c + 1);   // the q tile is free
     }
-    X.put(kXZt, col_sum(sm + kOffK, i, hf, nullptr));
-    X.put(kXSv, col_sum(sm + kOffV, i, hf, pwr));
+    {
+      // the At' tile is done with: its space holds the column-sum partials
+      float zc = 0.f, sc = 0.f;
+      col_sums(sm + kOffK, nullptr, sm + kOffV, pwr, reinterpret_cast<float *>(sm + kOffAp), zc,
+               sc);
+      if (tid < 128) {
+        zt[i] = pw[C] * zt[i] + zc;
+        sv[i] = pw[C] * sv[i] + sc;
+      }
+    }
     zeta = pw[C] * zeta + geo;
     mma_done();
     if (!meet()) break;
-    if (tid < 128) {
-      zt[i] = pw[C] * zt[i] + X.get(kXZt);
-      sv[i] = pw[C] * sv[i] + X.get(kXSv);
-    }
     if (tid == 0) {
       load(1, c + 1);
       load(2, c + 1);
@@ -652,10 +708,9 @@ namespace pr {
 constexpr uint32_t kOffQ = 0, kOffK = kTile, kOffKd = 2 * kTile, kOffV = 3 * kTile,
                    kOffVd = 4 * kTile, kOffG = 5 * kTile, kOffRb = 6 * kTile, kOffMisc = 7 * kTile;
 enum { kFullQ = 0, kFullK, kFullV, kFullG, kMma, kFinal, kNumBars };
-constexpr uint32_t kMiscTmem = 64, kMiscFlag = 68, kMiscPw = 128;
-constexpr uint32_t kMiscDden = kMiscPw + 132 * 4, kMiscR = kMiscDden + 128 * 4;
-constexpr uint32_t kMiscX = kMiscR + 128 * 4;
-constexpr uint32_t kSmemBytes = kOffMisc + kMiscX + 2 * 128 * 4;
+constexpr uint32_t kMiscTmem = 64, kMiscFlag = 68, kMiscUp = 128;
+constexpr uint32_t kMiscDden = kMiscUp + 256 * 4, kMiscR = kMiscDden + 128 * 4;
+constexpr uint32_t kSmemBytes = kOffMisc + kMiscR + 128 * 4;
 static_assert(kSmemBytes <= 232448, "exceeds the per-CTA shared memory of sm_100");
 constexpr uint32_t kTmR = 0, kTmT1 = 128, kTmT2 = 256, kTmAt = 384, kTmBt = 448;
 }  // namespace pr
@@ -683,11 +738,12 @@ __global__ void __launch_bounds__(NT, 1)
   auto bar = [&](int i) { return sb + kOffMisc + 8u * static_cast<uint32_t>(i); };
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(misc + kMiscTmem);
   volatile int *flag = reinterpret_cast<volatile int *>(misc + kMiscFlag);
-  float *pw = reinterpret_cast<float *>(misc + kMiscPw);
+  // up[127 - t + s] = lambda^(s-t) for s >= t, else 0; up[127 + m] = lambda^m for m = 0..128
+  float *up = reinterpret_cast<float *>(misc + kMiscUp);
+  const float *pw = up + 127;
   float *sdd = reinterpret_cast<float *>(misc + kMiscDden);   // dden of the chunk's tokens
   float *rv = reinterpret_cast<float *>(misc + kMiscR);       // r, the normaliser's adjoint
   const int hf = tid >> 7, i = tid & 127;
-  const Halves X{reinterpret_cast<float *>(misc + kMiscX), hf, i};
   const CUtensorMap *maps[4] = {&tm_q, &tm_k, &tm_v, &tm_g};
   const uint32_t offs[4] = {kOffQ, kOffK, kOffV, kOffG};
   int issued[4] = {0, 0, 0, 0}, waited[4] = {0, 0, 0, 0};
@@ -710,11 +766,8 @@ __global__ void __launch_bounds__(NT, 1)
     tmem_alloc(smem_u32(tmem_slot), 512);
     tmem_relinquish();
   }
-  if (tid < 128) {
-    pw[tid] = pow_int(L, tid);
-    rv[tid] = 0.f;
-  }
-  if (tid == 0) pw[C] = pow_int(L, C);
+  fill_masked_tables(L, tid, nullptr, nullptr, up);
+  if (tid < 128) rv[tid] = 0.f;
   fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
@@ -743,6 +796,7 @@ __global__ void __launch_bounds__(NT, 1)
   const uint64_t dG = kdesc(sb + kOffG), dGm = mdesc(sb + kOffG);
   const uint64_t dRb = kdesc(sb + kOffRb), dRbm = mdesc(sb + kOffRb);
   const int b0 = 2 * hf;
+  const float *mk = up + 127 - i;   // mk[s] = lambda^(s-i) for s >= i, else 0
 
   for (int cc = 0; cc < nch; ++cc) {
     const int c = nch - 1 - cc, row0 = c * C, Cv = min(C, N - row0);
@@ -789,7 +843,7 @@ __global__ void __launch_bounds__(NT, 1)
 #pragma unroll
       for (int e = 0; e < 32; e += 2) {
         const int s0 = blk * 32 + e, s1 = s0 + 1;
-        const float m0 = tab(pw, s0 - i), m1 = tab(pw, s1 - i);
+        const float m0 = mk[s0], m1 = mk[s1];
         pa[e / 2] = pack_bf16(__uint_as_float(pv[e]) * m0, __uint_as_float(pv[e + 1]) * m1);
         pb[e / 2] = pack_bf16((__uint_as_float(wv[e]) + sdd[s0]) * m0,
                               (__uint_as_float(wv[e + 1]) + sdd[s1]) * m1);
@@ -857,10 +911,15 @@ __global__ void __launch_bounds__(NT, 1)
       umma_commit(bar(kMma));
       load(1, c - 1);   // k has been read
     }
-    X.put(0, col_sum(sm + kOffQ, i, hf, sdd));
+    {
+      // the weighted k tile is done with: its space holds the column-sum partials
+      float rc = 0.f, unused = 0.f;
+      col_sums(sm + kOffQ, sdd, nullptr, nullptr, reinterpret_cast<float *>(sm + kOffKd), rc,
+               unused);
+      if (tid < 128) rv[i] = pw[C] * rv[i] + rc;
+    }
     mma_done();
     if (!meet()) break;
-    if (tid < 128) rv[i] = pw[C] * rv[i] + X.get(0);
     if (tid == 0) {
       load(0, c - 1);
       load(3, c - 1);
@@ -898,8 +957,9 @@ constexpr uint32_t kMiscDpwr = kMiscPwr + 128 * 4, kMiscZ = kMiscDpwr + 128 * 4;
 constexpr uint32_t kMiscZp = kMiscZ + 128 * 4, kMiscS = kMiscZp + 128 * 4;
 constexpr uint32_t kMiscSp = kMiscS + 128 * 4, kMiscWq = kMiscSp + 128 * 4;
 constexpr uint32_t kMiscRed = kMiscWq + 128 * 4, kMiscX = kMiscRed + 64;
-enum { kXQz = 0, kXRq, kXZt, kXZtp, kXSv, kXSvp, kNumX };
-constexpr uint32_t kSmemBytes = kOffMisc + kMiscX + kNumX * 2 * 128 * 4;
+enum { kXQz = 0, kXRq, kNumX };
+constexpr uint32_t kMiscScr = kMiscX + kNumX * 2 * 128 * 4;   // column-sum partials
+constexpr uint32_t kSmemBytes = kOffMisc + kMiscScr + 2 * 8 * 128 * 4;
 static_assert(kSmemBytes <= 232448, "exceeds the per-CTA shared memory of sm_100");
 constexpr uint32_t kTmS = 0, kTmSp = 128, kTmM = 256;
 }  // namespace pl
@@ -937,6 +997,7 @@ __global__ void __launch_bounds__(NT, 1)
   float *svp = reinterpret_cast<float *>(misc + kMiscSp);
   float *wq = reinterpret_cast<float *>(misc + kMiscWq);       // lambda^(t+1) rq_t
   float *red = reinterpret_cast<float *>(misc + kMiscRed);
+  float *scr = reinterpret_cast<float *>(misc + kMiscScr);
   const int hf = tid >> 7, i = tid & 127;
   const Halves X{reinterpret_cast<float *>(misc + kMiscX), hf, i};
   const CUtensorMap *maps[4] = {&tm_q, &tm_k, &tm_v, &tm_g};
@@ -1054,9 +1115,13 @@ __global__ void __launch_bounds__(NT, 1)
         wq[i] = pw[i + 1] * rq;
       }
     }
-    __syncthreads();
-    // o s' . (1^T Ms) on this thread's d_v column (s' of the chunk start), half of the rows
-    dl += o * svp[i] * col_sum(sm + kOffG, i, hf, wq);
+    __syncthreads();   // wq is complete
+    {
+      // o s' . (1^T Ms) on this thread's d_v column (s' of the chunk start)
+      float cs = 0.f, unused = 0.f;
+      col_sums(sm + kOffG, wq, nullptr, nullptr, scr, cs, unused);
+      if (tid < 128) dl += o * svp[i] * cs;
+    }
     mma_done();
     if (!meet()) break;
     if (tid == 0 && !last) {
@@ -1088,21 +1153,22 @@ __global__ void __launch_bounds__(NT, 1)
     }
     if (last) break;
     // the vector parts of the state and of its derivative: half sums over the chunk's rows
-    X.put(kXZtp, col_sum(sm + kOffKp, i, hf, nullptr));
-    X.put(kXZt, col_sum(sm + kOffK, i, hf, nullptr));
-    X.put(kXSvp, col_sum(sm + kOffV, i, hf, dpwr));
-    X.put(kXSv, col_sum(sm + kOffV, i, hf, pwr));
     if (!meet()) break;
     if (tid == 0) {
       mma_ss(tmem + kTmS, dKm, true, dVm, true, carried);
       mma_ss(tmem + kTmSp, dKpm, true, dVm, true, carried);
       umma_commit(bar(kMma));
     }
-    if (tid < 128) {
-      ztp[i] = pw[C] * ztp[i] + dpw[C] * zt[i] + X.get(kXZtp);
-      zt[i] = pw[C] * zt[i] + X.get(kXZt);
-      svp[i] = pw[C] * svp[i] + dpw[C] * sv[i] + X.get(kXSvp);
-      sv[i] = pw[C] * sv[i] + X.get(kXSv);
+    {
+      float zpc = 0.f, zc = 0.f, spc = 0.f, sc = 0.f;
+      col_sums(sm + kOffKp, nullptr, sm + kOffK, nullptr, scr, zpc, zc);
+      col_sums(sm + kOffV, dpwr, sm + kOffV, pwr, scr, spc, sc);
+      if (tid < 128) {
+        ztp[i] = pw[C] * ztp[i] + dpw[C] * zt[i] + zpc;
+        zt[i] = pw[C] * zt[i] + zc;
+        svp[i] = pw[C] * svp[i] + dpw[C] * sv[i] + spc;
+        sv[i] = pw[C] * sv[i] + sc;
+      }
     }
     zetap = pw[C] * zetap + dpw[C] * zeta + dgeo;
     zeta = pw[C] * zeta + geo;
