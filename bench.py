@@ -46,11 +46,6 @@ WL_DEC = inputs.WORKLOADS["decode_d128"]
 WL_GLB = inputs.WORKLOADS["global_d64"]
 
 
-# fp32 FMA peak of the CUDA cores: 148 SMs x 128 FMA lanes x 2 flops x 1.965 GHz
-# (the nominal maximum SM clock), for kernels bound by plain ALU arithmetic
-ALU_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
-
-
 def peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -462,23 +457,32 @@ def seg_leg(lib, args, world, rank, stream, hbm):
     return res
 
 
-def bwd_flops(B, H, N, dk, dv, with_dlam=True):
-    """fp32 FMA work of the backward kernel as written, 2 flops each: per
-    chunk of C = 32 tokens and head, both sweeps' score tiles (lower
-    triangle), the per-token forward rebuild, dphi(q), dphi(k), dv and the
-    state / reverse-state updates (plus S' and its use for dlambda)."""
-    C = 32
-    tri = C * (C + 1) / 2
-    per_chunk = (2 * tri * dk + 2 * tri * dv + C * (tri / C + dk) + C * dv * (tri / C + dk) +
-                 C * dk * (dv + tri / C) * 2 + C * dv * (dk + tri / C) + 2 * dk * dv * C)
-    if with_dlam:
-        per_chunk += C * dk * dv + dk * dv * C
-    return 2 * per_chunk * B * H * N / C
+def bwd_mma_flops(B, H, N, d, with_dlam=True):
+    """MMA flops of the tensor-core backward (bf16, d_k = d_v = d = 128, chunks
+    of C = 128 tokens), each group a 128 x 128 x 128 product (2 * 128^3):
+    pass F per chunk P, At V, W, B Kt (and Q St, w St^T after the first
+    chunk, the state update before the last); pass L (dlambda) Ms (and the
+    two state updates before the last); pass R P^T, W^T, A^T w, B^T Q (and
+    Lk K R, Lk V R^T after the last chunk, the R update before the first)."""
+    C = 128
+    n = -(-N // C)
+    g = 2 * C * C * d
+    f = 4 * n + 2 * (n - 1) + (n - 1)
+    lpass = (n + 2 * (n - 1)) if with_dlam else 0
+    r = 4 * n + 2 * (n - 1) + (n - 1)
+    return B * H * g * (f + lpass + r)
 
 
-def bwd_leg(lib, args, world, rank, stream, alu_peak):
+def bwd_bytes(B, H, N, d, es=2):
+    """Algorithmic HBM bytes of one backward: q, k, v, dy read once and dq,
+    dk, dv written once (the per-token den, dden stash and dlambda aside)."""
+    return 7 * B * H * N * d * es
+
+
+def bwd_leg(lib, args, world, rank, stream, tensor_peak, hbm_peak):
     """Backward (dq, dk, dv, dlambda) of the causal forward on the
-    causal_decay_d128 workload, a few steps (CUDA cores, fp32 arithmetic)."""
+    causal_decay_d128 workload, a few steps: the tensor-core passes (bf16,
+    d = 128)."""
     B, H, N, d = args.batch or WL.B, WL.H, WL.N, WL.d
     dev = torch.device("cuda")
     q, k, v = inputs.qkv((B, H, N, d), (B, H, N, d), WL.seed * 1000 + rank, WL.scale,
@@ -493,18 +497,22 @@ def bwd_leg(lib, args, world, rank, stream, alu_peak):
     def step():
         lib.linattn_bwd_causal(q, k, v, lam, WL.eps, dy, dq, dk, dv, dl, stream)
 
-    steps = max(1, min(args.steps, 3))
+    steps = max(1, min(args.steps, 10))
     with torch.cuda.stream(stream):
         ms = time_steps(step, steps, args.warmup, world, stream)
     assert lib.linattn_device_status(clear=True, stream=stream) == 0
     per = ms / 1e3 / steps
-    fl = bwd_flops(B, H, N, d, d)
+    fl = bwd_mma_flops(B, H, N, d)
+    by = bwd_bytes(B, H, N, d)
     res = {"value": B * N * world / per, "unit": "tokens/s", "ms_per_step": per * 1e3,
            "steps": steps, "ctas": B * H,
-           "roofline": {"bound": "alu", "achieved": fl / per / 1e12, "peak": alu_peak,
-                        "unit": "TFLOP/s", "frac": fl / per / 1e12 / alu_peak,
-                        "flops_per_launch": fl, "kernel": "causal_bwd_kernel",
-                        "traffic": None}}
+           "roofline": {"bound": "tensor", "achieved": fl / per / 1e12, "peak": tensor_peak,
+                        "unit": "TFLOP/s", "frac": fl / per / 1e12 / tensor_peak,
+                        "flops_per_launch": fl,
+                        "kernel": "bwd_tc_f_kernel + bwd_tc_l_kernel + bwd_tc_r_kernel",
+                        "traffic": None},
+           "hbm": {"algorithmic_bytes": by, "achieved": by / per / 1e9, "peak": hbm_peak,
+                   "unit": "GB/s", "frac": by / per / 1e9 / hbm_peak}}
     del q, k, v, dy, dq, dk, dv
     torch.cuda.empty_cache()
     return res
@@ -684,7 +692,7 @@ def main():
         elif args.only == "performer":
             r = performer_leg(lib, args, world, rank, stream, hbm)
         elif args.only == "backward":
-            r = bwd_leg(lib, args, world, rank, stream, ALU_PEAK_TFLOPS)
+            r = bwd_leg(lib, args, world, rank, stream, tcp, hbm)
         elif args.only == "segmented":
             r = seg_leg(lib, args, world, rank, stream, hbm)
         else:
@@ -720,7 +728,7 @@ def main():
     if args.legs and args.only == "all":
         line["decode"] = decode_leg(lib, args, world, rank, stream, hbm)
         line["global"] = global_leg(lib, args, world, rank, stream, hbm)
-        line["backward"] = bwd_leg(lib, args, world, rank, stream, ALU_PEAK_TFLOPS)
+        line["backward"] = bwd_leg(lib, args, world, rank, stream, tcp, hbm)
         line["segmented"] = seg_leg(lib, args, world, rank, stream, hbm)
         line["performer"] = performer_leg(lib, args, world, rank, stream, hbm)
         line["tiny"] = tiny_leg(lib, args, world, rank, stream, hbm)

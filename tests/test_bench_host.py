@@ -46,6 +46,18 @@ def test_mma_flops_of_the_causal_kernel():
         16 * 32 * 2 * 128 * (128 * 64 + 64 * 64 + 64 * 128 + 64 * 128)
 
 
+def test_backward_mma_count():
+    g = 2 * 128 ** 3
+    # one chunk: F has P, At V, W, B Kt; L has Ms; R has P^T, W^T, A^T w, B^T Q
+    assert bench.bwd_mma_flops(1, 1, 128, 128) == 9 * g
+    assert bench.bwd_mma_flops(1, 1, 100, 128, with_dlam=False) == 8 * g
+    # two chunks: F 4n + 2(n-1) + (n-1) = 11, L n + 2(n-1) = 4, R 11
+    assert bench.bwd_mma_flops(1, 1, 256, 128) == 26 * g
+    # the headline workload: 2168 groups per head, 581.9 GFLOP
+    assert bench.bwd_mma_flops(4, 16, 16384, 128) == 64 * 2168 * g
+    assert bench.bwd_bytes(4, 16, 16384, 128) == 7 * 64 * 16384 * 128 * 2
+
+
 def test_traffic_record_checks_its_sources(tmp_path, monkeypatch):
     src = tmp_path / "k.cuh"
     src.write_text("kernel v1\n")

@@ -324,7 +324,7 @@ struct Halves {
 namespace pf {
 constexpr uint32_t kOffQ = 0, kOffK = kTile, kOffV = 2 * kTile, kOffG = 3 * kTile,
                    kOffSb = 4 * kTile, kOffAp = 5 * kTile, kOffMisc = 6 * kTile;
-enum { kFullQ = 0, kFullK, kFullV, kFullG, kMma, kFinal, kNumBars };
+enum { kFullQ = 0, kFullK, kFullV, kFullG, kMma, kMma2, kFinal, kNumBars };
 constexpr uint32_t kMiscTmem = 64, kMiscFlag = 68, kMiscPw = 128;
 constexpr uint32_t kMiscDpw = kMiscPw + 132 * 4, kMiscPwr = kMiscDpw + 132 * 4;
 constexpr uint32_t kMiscZ = kMiscPwr + 128 * 4, kMiscS = kMiscZ + 128 * 4;
@@ -437,6 +437,8 @@ __global__ void __launch_bounds__(NT, 1)
   };
   int mph = 0;   // completed phases of the MMA barrier
   auto mma_done = [&]() { poll(kMma, mph); ++mph; };
+  int mph2 = 0;  // completed phases of the second MMA barrier (a product an epilogue needs later)
+  auto mma2_done = [&]() { poll(kMma2, mph2); ++mph2; };
 
   const uint64_t dQ = kdesc(sb + kOffQ), dK = kdesc(sb + kOffK), dKm = mdesc(sb + kOffK);
   const uint64_t dV = kdesc(sb + kOffV), dVm = mdesc(sb + kOffV);
@@ -469,8 +471,11 @@ __global__ void __launch_bounds__(NT, 1)
     if (!meet()) break;
     if (tid == 0) {
       mma_ss(tmem + kTmT1, dQ, false, dK, false, false);                 // Q Kt^T
-      if (carried) mma_ss(tmem + kTmT2, dQ, false, dSbm, true, false);   // Q St
       umma_commit(bar(kMma));
+      if (carried) {
+        mma_ss(tmem + kTmT2, dQ, false, dSbm, true, false);   // Q St, read after the next product
+        umma_commit(bar(kMma2));
+      }
     }
     mma_done();
     if (!meet()) break;
@@ -507,6 +512,7 @@ __global__ void __launch_bounds__(NT, 1)
       umma_commit(bar(kMma));
     }
     mma_done();
+    if (carried) mma2_done();
     poll(kFullG, c);
     if (!meet()) break;
     // ---- den, dnum (bf16 into TMEM) and dnum . num but for its o rq part
@@ -551,8 +557,11 @@ __global__ void __launch_bounds__(NT, 1)
     if (tid == 0) {
       if (!last) load(3, c + 1);                                   // dy tile is free
       mma_ts(tmem + kTmT1, tmem + kTmW, dV, false, false);        // W = w V^T
-      if (carried) mma_ts(tmem + kTmT2, tmem + kTmW, dSb, false, false);   // U = w St^T
       umma_commit(bar(kMma));
+      if (carried) {
+        mma_ts(tmem + kTmT2, tmem + kTmW, dSb, false, false);   // U = w St^T, read in the dq epilogue
+        umma_commit(bar(kMma2));
+      }
     }
     mma_done();
     if (!meet()) break;
@@ -611,6 +620,7 @@ __global__ void __launch_bounds__(NT, 1)
       umma_commit(bar(kMma));
     }
     mma_done();
+    if (carried) mma2_done();
     if (!meet()) break;
     // ---- dq = (B Kt + o B1 + lambda^(t+1) (U + zt dden + o (s.w + zeta dden))) phi'(q);
     //      dlambda, keys before the chunk (the lambda^(t+1) factor's derivative)
@@ -707,7 +717,7 @@ __global__ void __launch_bounds__(NT, 1)
 namespace pr {
 constexpr uint32_t kOffQ = 0, kOffK = kTile, kOffKd = 2 * kTile, kOffV = 3 * kTile,
                    kOffVd = 4 * kTile, kOffG = 5 * kTile, kOffRb = 6 * kTile, kOffMisc = 7 * kTile;
-enum { kFullQ = 0, kFullK, kFullV, kFullG, kMma, kFinal, kNumBars };
+enum { kFullQ = 0, kFullK, kFullV, kFullG, kMma, kMma2, kFinal, kNumBars };
 constexpr uint32_t kMiscTmem = 64, kMiscFlag = 68, kMiscUp = 128;
 constexpr uint32_t kMiscDden = kMiscUp + 256 * 4, kMiscR = kMiscDden + 128 * 4;
 constexpr uint32_t kSmemBytes = kOffMisc + kMiscR + 128 * 4;
@@ -790,6 +800,8 @@ __global__ void __launch_bounds__(NT, 1)
   };
   int mph = 0;
   auto mma_done = [&]() { poll(kMma, mph); ++mph; };
+  int mph2 = 0;  // completed phases of the second MMA barrier (a product an epilogue needs later)
+  auto mma2_done = [&]() { poll(kMma2, mph2); ++mph2; };
 
   const uint64_t dQ = kdesc(sb + kOffQ), dQm = mdesc(sb + kOffQ), dK = kdesc(sb + kOffK);
   const uint64_t dKd = kdesc(sb + kOffKd), dV = kdesc(sb + kOffV), dVd = kdesc(sb + kOffVd);
@@ -797,17 +809,16 @@ __global__ void __launch_bounds__(NT, 1)
   const uint64_t dRb = kdesc(sb + kOffRb), dRbm = mdesc(sb + kOffRb);
   const int b0 = 2 * hf;
   const float *mk = up + 127 - i;   // mk[s] = lambda^(s-i) for s >= i, else 0
+  // den, dden of this thread's token in the chunk being processed (tokens past
+  // the end: no gradient); the next chunk's pair is loaded a chunk ahead
+  float2 st = make_float2(1.f, 0.f);
+  if (nch > 0 && i < N - (nch - 1) * C)
+    st = *reinterpret_cast<const float2 *>(stash + (bh * N + (nch - 1) * C + i) * stash_stride);
 
   for (int cc = 0; cc < nch; ++cc) {
     const int c = nch - 1 - cc, row0 = c * C, Cv = min(C, N - row0);
     const bool carried = cc > 0;   // later tokens exist: R, r nonzero
-    // den, dden of this token from pass F (tokens past the end: no gradient)
-    float den = 1.f, dden = 0.f;
-    if (i < Cv) {
-      const float2 st = *reinterpret_cast<const float2 *>(stash + (bh * N + row0 + i) * stash_stride);
-      den = st.x;
-      dden = st.y;
-    }
+    const float den = st.x, dden = st.y;
     if (hf == 0) sdd[i] = dden;
     if (carried) state_to_operand(tmem + kTmR + lf, sm + kOffRb, i, hf, pw[C]);
     poll(kFullQ, cc);
@@ -826,29 +837,43 @@ __global__ void __launch_bounds__(NT, 1)
     if (!meet()) break;
     if (tid == 0) {
       mma_ss(tmem + kTmT1, dK, false, dQ, false, false);   // P^T = K Q^T
-      mma_ss(tmem + kTmT2, dV, false, dG, false, false);   // W^T = V w^T
       umma_commit(bar(kMma));
+      mma_ss(tmem + kTmT2, dV, false, dG, false, false);   // W^T = V w^T
+      umma_commit(bar(kMma2));
     }
+    // the next chunk's den, dden, while the products run
+    if (c > 0)
+      st = *reinterpret_cast<const float2 *>(stash + (bh * N + row0 - C + i) * stash_stride);
     mma_done();
     if (!meet()) break;
-    if (tid == 0 && c > 0) load(2, c - 1);   // v has been read (its weighted copy is made)
     // ---- A^T and B^T rows (key i, queries s >= i) into TMEM
 #pragma unroll 1
     for (int blk = b0; blk < b0 + 2; ++blk) {
-      uint32_t pv[32], wv[32];
+      uint32_t pv[32];
       tmem_ld_32x32b_x32(tmem + lf + kTmT1 + blk * 32, pv);
+      tmem_wait_ld();
+      uint32_t pa[16];
+#pragma unroll
+      for (int e = 0; e < 32; e += 2)
+        pa[e / 2] = pack_bf16(__uint_as_float(pv[e]) * mk[blk * 32 + e],
+                              __uint_as_float(pv[e + 1]) * mk[blk * 32 + e + 1]);
+      tmem_st_32x32b_x16(tmem + lf + kTmAt + blk * 16, pa);
+    }
+    mma2_done();
+    if (!meet()) break;
+    if (tid == 0 && c > 0) load(2, c - 1);   // v has been read (its weighted copy is made)
+#pragma unroll 1
+    for (int blk = b0; blk < b0 + 2; ++blk) {
+      uint32_t wv[32];
       tmem_ld_32x32b_x32(tmem + lf + kTmT2 + blk * 32, wv);
       tmem_wait_ld();
-      uint32_t pa[16], pb[16];
+      uint32_t pb[16];
 #pragma unroll
       for (int e = 0; e < 32; e += 2) {
         const int s0 = blk * 32 + e, s1 = s0 + 1;
-        const float m0 = mk[s0], m1 = mk[s1];
-        pa[e / 2] = pack_bf16(__uint_as_float(pv[e]) * m0, __uint_as_float(pv[e + 1]) * m1);
-        pb[e / 2] = pack_bf16((__uint_as_float(wv[e]) + sdd[s0]) * m0,
-                              (__uint_as_float(wv[e + 1]) + sdd[s1]) * m1);
+        pb[e / 2] = pack_bf16((__uint_as_float(wv[e]) + sdd[s0]) * mk[s0],
+                              (__uint_as_float(wv[e + 1]) + sdd[s1]) * mk[s1]);
       }
-      tmem_st_32x32b_x16(tmem + lf + kTmAt + blk * 16, pa);
       tmem_st_32x32b_x16(tmem + lf + kTmBt + blk * 16, pb);
     }
     tmem_wait_st();
@@ -856,24 +881,43 @@ __global__ void __launch_bounds__(NT, 1)
     if (tid == 0) {
       mma_ts(tmem + kTmT1, tmem + kTmAt, dGm, true, false);                 // A^T w
       if (carried) mma_ss(tmem + kTmT1, dKd, false, dRbm, true, true);     // + Lk K R
+      umma_commit(bar(kMma));
       mma_ts(tmem + kTmT2, tmem + kTmBt, dQm, true, false);                 // B^T Q
       if (carried) mma_ss(tmem + kTmT2, dVd, false, dRb, false, true);     // + Lk V R^T
-      umma_commit(bar(kMma));
+      umma_commit(bar(kMma2));
     }
     mma_done();
     if (!meet()) break;
-    // ---- dv and dk = (dphi(k) + Lk r) phi'(k)
+    // ---- dv (while the dk product runs), then dk = (dphi(k) + Lk r) phi'(k)
+    {
+      __nv_bfloat16 *vd = dv + (bh * N + row0 + i) * static_cast<long>(D);
+#pragma unroll 1
+      for (int blk = b0; blk < b0 + 2; ++blk) {
+        uint32_t a[32];
+        tmem_ld_32x32b_x32(tmem + lf + kTmT1 + blk * 32, a);
+        tmem_wait_ld();
+        uint32_t pv[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2)
+          pv[e / 2] = pack_bf16(__uint_as_float(a[e]), __uint_as_float(a[e + 1]));
+        if (i < Cv)
+#pragma unroll
+          for (int m = 0; m < 4; ++m)
+            reinterpret_cast<uint4 *>(vd + blk * 32)[m] =
+                make_uint4(pv[4 * m], pv[4 * m + 1], pv[4 * m + 2], pv[4 * m + 3]);
+      }
+    }
+    mma2_done();
+    if (!meet()) break;
     {
       const float kf = carried ? pw[C - 1 - i] : 0.f;
-      __nv_bfloat16 *vd = dv + (bh * N + row0 + i) * static_cast<long>(D);
       __nv_bfloat16 *kd = dk + (bh * N + row0 + i) * static_cast<long>(D);
 #pragma unroll 1
       for (int blk = b0; blk < b0 + 2; ++blk) {
-        uint32_t a[32], b[32];
-        tmem_ld_32x32b_x32(tmem + lf + kTmT1 + blk * 32, a);
+        uint32_t b[32];
         tmem_ld_32x32b_x32(tmem + lf + kTmT2 + blk * 32, b);
         tmem_wait_ld();
-        uint32_t pv[16], pk[16];
+        uint32_t pk[16];
 #pragma unroll
         for (int m = 0; m < 4; ++m) {
           const uint4 k4 = *reinterpret_cast<const uint4 *>(sm + kOffK + toff(i, blk * 4 + m));
@@ -881,7 +925,6 @@ __global__ void __launch_bounds__(NT, 1)
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
             const int e = 8 * m + 2 * u, k0 = blk * 32 + e;
-            pv[4 * m + u] = pack_bf16(__uint_as_float(a[e]), __uint_as_float(a[e + 1]));
             float g0 = __uint_as_float(b[e]) + kf * rv[k0];
             float g1 = __uint_as_float(b[e + 1]) + kf * rv[k0 + 1];
             if (!ident) {
@@ -893,12 +936,9 @@ __global__ void __launch_bounds__(NT, 1)
         }
         if (i < Cv)
 #pragma unroll
-          for (int m = 0; m < 4; ++m) {
-            reinterpret_cast<uint4 *>(vd + blk * 32)[m] =
-                make_uint4(pv[4 * m], pv[4 * m + 1], pv[4 * m + 2], pv[4 * m + 3]);
+          for (int m = 0; m < 4; ++m)
             reinterpret_cast<uint4 *>(kd + blk * 32)[m] =
                 make_uint4(pk[4 * m], pk[4 * m + 1], pk[4 * m + 2], pk[4 * m + 3]);
-          }
       }
     }
     if (c == 0) break;
@@ -950,7 +990,7 @@ __global__ void __launch_bounds__(NT, 1)
 namespace pl {
 constexpr uint32_t kOffQ = 0, kOffK = kTile, kOffKp = 2 * kTile, kOffV = 3 * kTile,
                    kOffG = 4 * kTile, kOffMisc = 5 * kTile;
-enum { kFullQ = 0, kFullK, kFullV, kFullG, kMma, kFinal, kNumBars };
+enum { kFullQ = 0, kFullK, kFullV, kFullG, kMma, kMma2, kFinal, kNumBars };
 constexpr uint32_t kMiscTmem = 64, kMiscFlag = 68, kMiscPw = 128;
 constexpr uint32_t kMiscDpw = kMiscPw + 132 * 4, kMiscPwr = kMiscDpw + 132 * 4;
 constexpr uint32_t kMiscDpwr = kMiscPwr + 128 * 4, kMiscZ = kMiscDpwr + 128 * 4;
@@ -1073,15 +1113,16 @@ __global__ void __launch_bounds__(NT, 1)
     dgeo += dpwr[m];
   }
 
+  // den, dden of this thread's token in the chunk (past the end: no
+  // gradient); the next chunk's pair is loaded a chunk ahead
+  float2 st = make_float2(1.f, 0.f);
+  if (nch > 0 && i < min(C, N))
+    st = *reinterpret_cast<const float2 *>(stash + (bh * N + i) * stash_stride);
+
   for (int c = 0; c < nch; ++c) {
-    const int row0 = c * C, Cv = min(C, N - row0);
+    const int row0 = c * C;
     const bool carried = c > 0, last = c == nch - 1;
-    float den = 1.f, dden = 0.f;
-    if (i < Cv) {
-      const float2 st = *reinterpret_cast<const float2 *>(stash + (bh * N + row0 + i) * stash_stride);
-      den = st.x;
-      dden = st.y;
-    }
+    const float den = st.x, dden = st.y;
     poll(kFullQ, c);
     poll(kFullK, c);
     poll(kFullV, c);
@@ -1107,6 +1148,9 @@ __global__ void __launch_bounds__(NT, 1)
       mma_ss(tmem + kTmM, dQm, true, dGm, true, false);   // Ms = (Lq Q)^T w
       umma_commit(bar(kMma));
     }
+    st = make_float2(1.f, 0.f);   // the next chunk's den, dden
+    if (!last && i < N - row0 - C)
+      st = *reinterpret_cast<const float2 *>(stash + (bh * N + row0 + C + i) * stash_stride);
     {
       // the z' part of dlambda (once per row), and lambda^(t+1) rq_t for 1^T Ms
       const float rq = X.get(kXRq);
