@@ -70,6 +70,15 @@ def test_batch_heads_and_no_dlambda(cuda_lib):
     check(cuda_lib, 1, 2, 200, None, 4302, want_dlam=False)
 
 
+def test_split_and_unsplit_forward_pass(cuda_lib):
+    """The forward pass runs as two CTAs per head (the second from the state
+    the state pass leaves at the split point) while the heads leave SMs
+    idle, and as one CTA per head once they fill the GPU: an odd split point
+    (5 chunks), and 160 heads over 3 chunks (no split)."""
+    check(cuda_lib, 1, 2, 600, torch.tensor([0.95, 1.0]), 4350)
+    check(cuda_lib, 10, 16, 300, inputs.decay(inputs.WORKLOADS["causal_decay_d128"], H=16), 4360)
+
+
 def test_identity_features(cuda_lib):
     """phi = identity on positive feature vectors (phi' = 1)."""
     B, H, N = 1, 2, 300

@@ -307,6 +307,169 @@ struct Halves {
   }
 };
 
+// ============================================================== state pass for split F
+// Pass F can run as two CTAs per head: chunks [0, H0) and [H0, nch).  The
+// second needs the state at token T = H0 C in pass F's elu form (see below):
+//   St = sum_{s<T} lambda^(T-1-s) Kt_s v_s^T,  s = sum_{s<T} lambda^(T-1-s) v_s,
+//   zt = sum_{s<T} lambda^(T-1-s) Kt_s,        zeta = sum_{s<T} lambda^(T-1-s).
+// This pass walks the first H0 chunks of each head once, weighting key row s
+// of chunk c by lambda^((H0-1-c) C) lambda^(C-1-s) (a weight relative to T,
+// so no decay pass over the accumulator is needed; weights below the bf16
+// range are negligible against the others), and writes the state to `mid`:
+// per head St [128][128] fp32, then s [128], zt [128], zeta.
+constexpr int kMidFloats = D * D + 2 * D + 4;
+
+namespace ps {
+constexpr uint32_t kOffK = 0, kOffV = kTile, kOffMisc = 2 * kTile;
+enum { kFullK = 0, kFullV, kMma, kFinal, kNumBars };
+constexpr uint32_t kMiscTmem = 64, kMiscFlag = 68, kMiscPw = 128;
+constexpr uint32_t kMiscW = kMiscPw + 132 * 4, kMiscScr = kMiscW + 128 * 4;
+constexpr uint32_t kSmemBytes = kOffMisc + kMiscScr + 2 * 8 * 128 * 4;
+static_assert(kSmemBytes <= 232448, "exceeds the per-CTA shared memory of sm_100");
+}  // namespace ps
+
+__global__ void __launch_bounds__(NT, 1)
+    bwd_tc_s_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                    const float *__restrict__ lam, float *__restrict__ mid, int H, int N, int H0,
+                    bool ident) {
+  using namespace ps;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *sm = smem_raw;
+  const uint32_t sb = smem_u32(sm);
+  const int tid = threadIdx.x, warp = tid >> 5;
+  if (sb & 1023u) {
+    if (tid == 0) atomicOr(&g_status, kStatusWaitTimeout);
+    return;
+  }
+  // pass F (launched next as this pass's programmatic dependent) starts its
+  // first halves at once; its second halves wait for this grid
+  grid_launch_dependents();
+  const long bh = blockIdx.x;
+  const int h = static_cast<int>(bh % H);
+  const float L = lam ? lam[h] : 1.f;
+  uint8_t *misc = sm + kOffMisc;
+  auto bar = [&](int i) { return sb + kOffMisc + 8u * static_cast<uint32_t>(i); };
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(misc + kMiscTmem);
+  volatile int *flag = reinterpret_cast<volatile int *>(misc + kMiscFlag);
+  float *pw = reinterpret_cast<float *>(misc + kMiscPw);   // lambda^m, m = 0..C
+  float *wr = reinterpret_cast<float *>(misc + kMiscW);    // this chunk's row weights
+  float *scr = reinterpret_cast<float *>(misc + kMiscScr);
+  const int hf = tid >> 7, i = tid & 127;
+  const CUtensorMap *maps[2] = {&tm_k, &tm_v};
+  const uint32_t offs[2] = {kOffK, kOffV};
+  int issued[2] = {0, 0}, waited[2] = {0, 0};
+  auto load = [&](int which, int c) {
+    const uint32_t b = bar(kFullK + which);
+    mbar_arrive_expect_tx(b, kTile);
+    tma_load_3d(sb + offs[which], maps[which], b, 0, c * C, static_cast<int>(bh));
+    tma_load_3d(sb + offs[which] + kPanel, maps[which], b, 64, c * C, static_cast<int>(bh));
+    if (c + 1 < H0) tma_prefetch_l2_3d(maps[which], 0, (c + 1) * C, static_cast<int>(bh));
+    if (c + 1 < H0) tma_prefetch_l2_3d(maps[which], 64, (c + 1) * C, static_cast<int>(bh));
+    ++issued[which];
+  };
+  if (tid == 0) {
+    for (int b = 0; b < kNumBars; ++b) mbar_init(bar(b), 1);
+    *flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_slot), 128);
+    tmem_relinquish();
+  }
+  if (tid < 128) pw[tid] = pow_int(L, tid);
+  if (tid == 0) pw[C] = pow_int(L, C);
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t lf = static_cast<uint32_t>((warp & 3) * 32) << 16;
+  if (tid == 0 && H0 > 0) {
+    load(0, 0);
+    load(1, 0);
+  }
+  auto poll = [&](int b, int parity) {
+    if (tid == 0 && !*flag) {
+      if (!mbar_wait(bar(b), static_cast<uint32_t>(parity) & 1u)) *flag = 1;
+      else if (b <= kFullV) ++waited[b];
+    }
+  };
+  auto meet = [&]() -> bool {
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    return *flag == 0;
+  };
+  int mph = 0;
+  const uint64_t dKm = mdesc(sb + kOffK), dVm = mdesc(sb + kOffV);
+  float zt_acc = 0.f, s_acc = 0.f, zeta = 0.f;   // thread i < 128: column i of zt and s
+
+  for (int c = 0; c < H0; ++c) {
+    const float tc = pow_int(L, (H0 - 1 - c) * C);   // lambda^((H0-1-c) C)
+    if (tid < 128) wr[i] = tc * pw[C - 1 - i];
+    poll(kFullK, c);
+    poll(kFullV, c);
+    if (!meet()) break;
+    elu_row(sm + kOffK, i, hf, ident);
+    scale_row(sm + kOffK, sm + kOffK, i, hf, wr[i]);
+    fence_proxy_async_smem();
+    if (!meet()) break;
+    if (tid == 0) {
+      mma_ss(tmem, dKm, true, dVm, true, c > 0);   // St += (W Kt)^T V
+      umma_commit(bar(kMma));
+    }
+    {
+      float zc = 0.f, sc = 0.f;
+      col_sums(sm + kOffK, nullptr, sm + kOffV, wr, scr, zc, sc);
+      if (tid < 128) {
+        zt_acc += zc;
+        s_acc += sc;
+      }
+    }
+    for (int m = 0; m < C; ++m) zeta += wr[m];
+    poll(kMma, mph);
+    ++mph;
+    if (!meet()) break;
+    if (tid == 0 && c + 1 < H0) {
+      load(0, c + 1);
+      load(1, c + 1);
+    }
+  }
+  if (!*flag && H0 > 0) {
+    float *m = mid + bh * kMidFloats;
+#pragma unroll 1
+    for (int blk = 2 * hf; blk < 2 * hf + 2; ++blk) {
+      uint32_t v[32];
+      tmem_ld_32x32b_x32(tmem + lf + blk * 32, v);
+      tmem_wait_ld();
+      float4 *dst = reinterpret_cast<float4 *>(m + i * D + blk * 32);
+#pragma unroll
+      for (int e = 0; e < 8; ++e)
+        dst[e] = make_float4(__uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]),
+                             __uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3]));
+    }
+    if (tid < 128) {
+      m[D * D + i] = s_acc;
+      m[D * D + D + i] = zt_acc;
+    }
+    if (tid == 0) m[D * D + 2 * D] = zeta;
+  }
+  if (tid == 0) {
+    for (int b = 0; b < 2; ++b)
+      for (int n = waited[b]; n < issued[b]; ++n) mbar_wait(bar(kFullK + b), n & 1);
+    umma_commit(bar(kFinal));
+    mbar_wait(bar(kFinal), 0);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 128);
+  }
+}
+
 // ============================================================== pass F
 // The key side in the elu form (o = 1; o = 0 and elu(k) -> k with `ident`):
 // K = Kt + o 1 1^T with Kt = elu(K), so
@@ -342,8 +505,8 @@ __global__ void __launch_bounds__(NT, 1)
     bwd_tc_f_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
                     const float *__restrict__ lam, float eps, __nv_bfloat16 *__restrict__ dq,
-                    float *__restrict__ stash, long stash_stride, float *__restrict__ dlam, int H,
-                    int N, bool ident) {
+                    float *__restrict__ stash, long stash_stride, float *__restrict__ dlam,
+                    const float *__restrict__ mid, int H0, int H, int N, bool ident) {
   using namespace pf;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *sm = smem_raw;
@@ -353,11 +516,17 @@ __global__ void __launch_bounds__(NT, 1)
     if (tid == 0) atomicOr(&g_status, kStatusWaitTimeout);
     return;
   }
-  const long bh = blockIdx.x;
+  // H0 > 0: two CTAs per head, chunks [0, H0) and [H0, nch); the second
+  // starts from the state the state pass leaves in `mid`
+  const int G = H0 > 0 ? 2 : 1;
+  const long BH = gridDim.x / G;
+  const int half = static_cast<int>(blockIdx.x / BH);
+  const long bh = blockIdx.x % BH;
   const int h = static_cast<int>(bh % H);
   const float L = lam ? lam[h] : 1.f;
   const float o = ident ? 0.f : 1.f;
   const int nch = (N + C - 1) / C;
+  const int c0 = half ? H0 : 0, c1 = (G == 2 && half == 0) ? H0 : nch;
   uint8_t *misc = sm + kOffMisc;
   auto bar = [&](int i) { return sb + kOffMisc + 8u * static_cast<uint32_t>(i); };
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(misc + kMiscTmem);
@@ -413,8 +582,8 @@ __global__ void __launch_bounds__(NT, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t lf = static_cast<uint32_t>((warp & 3) * 32) << 16;
-  if (tid == 0 && nch > 0)
-    for (int b = 0; b < 4; ++b) load(b, 0);
+  if (tid == 0 && c0 < c1)
+    for (int b = 0; b < 4; ++b) load(b, c0);
   float geo = 0.f;   // sum_s lambda^(C-1-s) over a chunk
   for (int m = 0; m < C; ++m) geo += pwr[m];
   if (tid < 128) {
@@ -445,24 +614,52 @@ __global__ void __launch_bounds__(NT, 1)
   const uint64_t dSb = kdesc(sb + kOffSb), dSbm = mdesc(sb + kOffSb);
   float dl = 0.f;      // this thread's share of dlambda
   float zeta = 0.f;    // sum of the decay weights of the keys before the chunk
+  if (half == 1) {
+    // the state at token H0 C, from the state pass (this grid's prerequisite)
+    grid_dependency_wait();
+    const float *m = mid + bh * kMidFloats;
+#pragma unroll 1
+    for (int blk = 2 * hf; blk < 2 * hf + 2; ++blk) {
+      uint32_t v[32];
+      const float4 *src = reinterpret_cast<const float4 *>(m + i * D + blk * 32);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float4 x = src[e];
+        v[4 * e] = __float_as_uint(x.x);
+        v[4 * e + 1] = __float_as_uint(x.y);
+        v[4 * e + 2] = __float_as_uint(x.z);
+        v[4 * e + 3] = __float_as_uint(x.w);
+      }
+      tmem_st_32x32b_x32(tmem + kTmS + lf + blk * 32, v);
+    }
+    tmem_wait_st();
+    if (tid < 128) {
+      sv[i] = m[D * D + i];
+      zt[i] = m[D * D + D + i];
+    }
+    zeta = m[D * D + 2 * D];
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+  }
   uint8_t *ap_row = sm + kOffAp + static_cast<uint32_t>(i) * 256u;   // At' row (its two halves)
   const int b0 = 2 * hf;   // this half's first 32-column block
   const float lf_i = pw[i + 1];
   const float *mk = lo + 127 - i, *dmk = dlo + 127 - i;   // mk[s] = lambda^(i-s) (s <= i) or 0
 
-  for (int c = 0; c < nch; ++c) {
+  for (int c = c0; c < c1; ++c) {
     const int row0 = c * C, Cv = min(C, N - row0);
-    const bool carried = c > 0, last = c == nch - 1;
+    const bool carried = c > c0 || half == 1, last = c == c1 - 1;
     // ---- the state before this chunk: bf16 operand, and lambda^C St kept for the update
     if (carried) state_to_operand(tmem + kTmS + lf, sm + kOffSb, i, hf, pw[C]);
-    poll(kFullQ, c);
+    poll(kFullQ, c - c0);
     if (!meet()) break;
     {
       float rqh = 0.f;
       X.put(kXQz, phi_row(sm + kOffQ, i, hf, ident, zt, &rqh));   // phi(q_i) . zt, half
       X.put(kXRq, rqh);
     }
-    poll(kFullK, c);
+    poll(kFullK, c - c0);
     if (!meet()) break;
     const float rq = X.get(kXRq), qzt = X.get(kXQz);
     const float qz = qzt + o * rq * zeta;   // phi(q_i) . z
@@ -505,7 +702,7 @@ __global__ void __launch_bounds__(NT, 1)
       X.put(kXRs, rsh);
     }
     tmem_wait_st();
-    poll(kFullV, c);
+    poll(kFullV, c - c0);
     if (!meet()) break;
     if (tid == 0) {
       mma_ts(tmem + kTmT1, tmem + kTmA, dVm, true, false);   // At V
@@ -513,7 +710,7 @@ __global__ void __launch_bounds__(NT, 1)
     }
     mma_done();
     if (carried) mma2_done();
-    poll(kFullG, c);
+    poll(kFullG, c - c0);
     if (!meet()) break;
     // ---- den, dnum (bf16 into TMEM) and dnum . num but for its o rq part
     const float den = lf_i * qz + o * rq * gs[i] + X.get(kXRs) + eps, inv = 1.f / den;

@@ -620,22 +620,41 @@ int launch_bwd_tc(const linattn_dims *d, const void *q, const void *k, const voi
     return LINATTN_ERR_CUDA;
   if (!set_smem(btc::bwd_tc_f_kernel, static_cast<int>(btc::pf::kSmemBytes)) ||
       !set_smem(btc::bwd_tc_l_kernel, static_cast<int>(btc::pl::kSmemBytes)) ||
-      !set_smem(btc::bwd_tc_r_kernel, static_cast<int>(btc::pr::kSmemBytes)))
+      !set_smem(btc::bwd_tc_r_kernel, static_cast<int>(btc::pr::kSmemBytes)) ||
+      !set_smem(btc::bwd_tc_s_kernel, static_cast<int>(btc::ps::kSmemBytes)))
     return LINATTN_ERR_CUDA;
   auto *bq = static_cast<bf16 *>(dq);
   auto *bk = static_cast<bf16 *>(dk);
   auto *bv = static_cast<bf16 *>(dv);
   const bool id = ident(d);
-  float *ws = nullptr;
+  // Pass F in two halves per head when the heads alone leave SMs idle: the
+  // first half from the start, the second from the state at token H0 C
+  // (written by the state pass, which runs beside the first halves).  The
+  // split point balances the first half against the state pass plus the
+  // second half (the state pass costs ~0.15 of pass F per chunk).
+  const int nch = (d->N + btc::C - 1) / btc::C;
+  const int sms = num_sms();
+  int H0 = (nch >= 2 && sms > 0 && BH < sms) ? (nch * 54 + 99) / 100 : 0;
+  if (H0 >= nch) H0 = 0;
+  const size_t mid_bytes = H0 ? static_cast<size_t>(BH) * btc::kMidFloats * sizeof(float) : 0;
   const size_t stash_bytes = static_cast<size_t>(BH) * d->N * 2 * sizeof(float);
-  if (cudaMallocAsync(reinterpret_cast<void **>(&ws), stash_bytes, s) != cudaSuccess) {
-    cudaGetLastError();   // fall back to the stash in the dk rows
+  char *ws = nullptr;
+  if (cudaMallocAsync(reinterpret_cast<void **>(&ws), mid_bytes + stash_bytes, s) != cudaSuccess) {
+    cudaGetLastError();   // fall back to the stash in the dk rows, unsplit
     ws = nullptr;
+    H0 = 0;
   }
-  float *stash = ws ? ws : reinterpret_cast<float *>(dk);
+  float *mid = ws ? reinterpret_cast<float *>(ws) : nullptr;
+  float *stash = ws ? reinterpret_cast<float *>(ws + mid_bytes) : reinterpret_cast<float *>(dk);
   const long stride = ws ? 2 : btc::D / 2;
-  int rc = launch_pdl(btc::bwd_tc_f_kernel, BH, btc::NT, btc::pf::kSmemBytes, s, false, mq, mk,
-                      mv, mg, lam, eps, bq, stash, stride, dlam, d->H, d->N, id);
+  int rc = LINATTN_OK;
+  if (H0)
+    rc = launch_pdl(btc::bwd_tc_s_kernel, BH, btc::NT, btc::ps::kSmemBytes, s, false, mk, mv, lam,
+                    mid, d->H, d->N, H0, id);
+  if (rc == LINATTN_OK)
+    rc = launch_pdl(btc::bwd_tc_f_kernel, H0 ? 2 * BH : BH, btc::NT, btc::pf::kSmemBytes, s,
+                    H0 != 0, mq, mk, mv, mg, lam, eps, bq, stash, stride, dlam,
+                    static_cast<const float *>(mid), H0, d->H, d->N, id);
   if (rc == LINATTN_OK && dlam)
     rc = launch_pdl(btc::bwd_tc_l_kernel, BH, btc::NT, btc::pl::kSmemBytes, s, false, mq, mk, mv,
                     mg, lam, static_cast<const float *>(stash), stride, dlam, d->H, d->N, id);
