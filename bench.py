@@ -493,9 +493,13 @@ def bwd_leg(lib, args, world, rank, stream, tensor_peak, hbm_peak):
     lam = inputs.decay(WL).to(dev)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     dl = torch.empty(H, device=dev)
+    # the product call with its workspace (the split point's states and the
+    # per-token stash), allocated once like the forward leg's
+    need = lib.linattn_bwd_causal_workspace(B, H, N, d, d, WL.dtype)
+    ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
 
     def step():
-        lib.linattn_bwd_causal(q, k, v, lam, WL.eps, dy, dq, dk, dv, dl, stream)
+        lib.linattn_bwd_causal(q, k, v, lam, WL.eps, dy, dq, dk, dv, dl, stream, workspace=ws)
 
     steps = max(1, min(args.steps, 10))
     with torch.cuda.stream(stream):
@@ -505,15 +509,16 @@ def bwd_leg(lib, args, world, rank, stream, tensor_peak, hbm_peak):
     fl = bwd_mma_flops(B, H, N, d)
     by = bwd_bytes(B, H, N, d)
     res = {"value": B * N * world / per, "unit": "tokens/s", "ms_per_step": per * 1e3,
-           "steps": steps, "ctas": B * H,
+           "steps": steps, "ctas": B * H, "workspace_bytes": need,
            "roofline": {"bound": "tensor", "achieved": fl / per / 1e12, "peak": tensor_peak,
                         "unit": "TFLOP/s", "frac": fl / per / 1e12 / tensor_peak,
                         "flops_per_launch": fl,
-                        "kernel": "bwd_tc_f_kernel + bwd_tc_l_kernel + bwd_tc_r_kernel",
+                        "kernel": "bwd_tc_s_kernel + bwd_tc_f_kernel + bwd_tc_l_kernel + "
+                                  "bwd_tc_r_kernel",
                         "traffic": None},
            "hbm": {"algorithmic_bytes": by, "achieved": by / per / 1e9, "peak": hbm_peak,
                    "unit": "GB/s", "frac": by / per / 1e9 / hbm_peak}}
-    del q, k, v, dy, dq, dk, dv
+    del q, k, v, dy, dq, dk, dv, ws
     torch.cuda.empty_cache()
     return res
 

@@ -261,15 +261,41 @@ LINATTN_API int linattn_combine_states(const linattn_dims *dims, int G, const fl
  * reverse pass for dk and dv); every other shape, fp32, and the CUDA-core
  * choice of linattn_set_kernel_choice(LINATTN_OP_BACKWARD, ...) use fp32
  * arithmetic on CUDA cores.  dlambda is a sum of per-(b, h) fp32 atomics, so
- * its last bits may vary from run to run; dq, dk, dv do not.  Between its
- * passes the call keeps two fp32 numbers per token in the first 8 bytes of
- * that token's dk row, which it overwrites afterwards: dk must not be read
- * before the call completes.
+ * its last bits may vary from run to run; dq, dk, dv do not.  The
+ * tensor-core passes keep two fp32 numbers per token between them (and, when
+ * the forward pass is split, each head's state at the split point) in a
+ * stream-ordered allocation made inside the call; if that allocation fails
+ * the numbers live in the first 8 bytes of each token's dk row, which is
+ * overwritten afterwards.  Either way dk must not be read before the call
+ * completes.
  */
 LINATTN_API int linattn_bwd_causal(const linattn_dims *dims, const void *q, const void *k,
                        const void *v, const float *lambda, float eps, const void *dy,
                        void *dq, void *dk, void *dv, float *dlambda,
                        linattn_stream_t stream);
+
+/*
+ * linattn_bwd_causal_workspace: the bytes of workspace with which
+ * linattn_bwd_causal_ws runs its fastest form (0 when the call takes the
+ * CUDA-core kernel, which needs none): per-token den, dden (8 bytes per
+ * token) and, when the forward pass is split in two halves per head, the
+ * state at the split point of every head (66,576 bytes per head).
+ *
+ * linattn_bwd_causal_ws: linattn_bwd_causal with a caller-owned device
+ * workspace instead of a stream-ordered allocation inside the call.
+ *   workspace, workspace_bytes: 16-byte aligned, overlapping no input or
+ *     output; used from launch to completion of the call on `stream`.  With
+ *     fewer bytes than the query returns but at least 8 per token the call
+ *     runs unsplit; with fewer than that (or NULL, 0) the per-token numbers
+ *     live in the dk rows and the passes run in order (nothing is allocated).
+ *   Everything else as linattn_bwd_causal.  NULL with nonzero bytes:
+ *   LINATTN_ERR_INVALID.
+ */
+LINATTN_API size_t linattn_bwd_causal_workspace(const linattn_dims *dims);
+LINATTN_API int linattn_bwd_causal_ws(const linattn_dims *dims, const void *q, const void *k,
+                       const void *v, const float *lambda, float eps, const void *dy,
+                       void *dq, void *dk, void *dv, float *dlambda, void *workspace,
+                       size_t workspace_bytes, linattn_stream_t stream);
 
 /*
  * Global (non-causal) forward ([LN] §3 after the sum swap and §6 forward;

@@ -124,6 +124,27 @@ def test_bwd_rejects_bad_arguments(lib):
     assert bw(dl=MIS) == linattn.LINATTN_ERR_INVALID
 
 
+def test_bwd_workspace_entry_points_on_the_host(lib):
+    DY, DQ, DK, DV = (P(0x7F0000500000), P(0x7F0000600000), P(0x7F0000700000),
+                      P(0x7F0000800000))
+    WS = P(0x7F0000900000)
+    bw = lambda **kw: lib.linattn_bwd_causal_ws(
+        ctypes.byref(kw.get("d", D())), FAKE, FAKE2, FAKE3, None, 1e-6, DY, DQ, DK, DV, None,
+        kw.get("ws", WS), kw.get("nb", 1 << 20), None)
+    assert bw(ws=None, nb=64) == linattn.LINATTN_ERR_INVALID     # NULL with bytes
+    assert bw(ws=MIS) == linattn.LINATTN_ERR_INVALID             # unaligned
+    assert bw(ws=DQ) == linattn.LINATTN_ERR_INVALID              # over an output
+    assert bw(ws=FAKE) == linattn.LINATTN_ERR_INVALID            # over an input
+    assert bw(d=D(dv=24)) == linattn.LINATTN_ERR_UNSUPPORTED
+    # the CUDA-core kernel (fp32, or d != 128) needs no workspace
+    wsq = lambda d: lib.linattn_bwd_causal_workspace(ctypes.byref(d))
+    assert wsq(D()) == 0
+    bf = linattn.linattn_dims(2, 3, 300, 128, 128, linattn.LINATTN_BF16, 0)
+    # the tensor-core passes: at least the 8-byte stash of every token
+    assert wsq(bf) >= 2 * 3 * 300 * 8
+    assert wsq(linattn.linattn_dims(2, 3, 0, 128, 128, linattn.LINATTN_BF16, 0)) == 0
+
+
 def test_global_cross_rejects_bad_arguments(lib):
     KV, ks = P(0x7F0000500000), P(0x7F0000600000)
     gc = lambda **kw: lib.linattn_fwd_global_cross(

@@ -7,6 +7,8 @@ Gate per gradient tensor: max|gpu - oracle| / max|oracle| <= 2e-2, the bf16
 tolerance of the forward: the operands of every product are bf16 (phi(q),
 phi(k), v, dnum, the score tiles and the carried states rounded once, relative
 2^-9 each) and every sum is accumulated in fp32."""
+import ctypes
+
 import pytest
 import torch
 
@@ -77,6 +79,41 @@ def test_split_and_unsplit_forward_pass(cuda_lib):
     (5 chunks), and 160 heads over 3 chunks (no split)."""
     check(cuda_lib, 1, 2, 600, torch.tensor([0.95, 1.0]), 4350)
     check(cuda_lib, 10, 16, 300, inputs.decay(inputs.WORKLOADS["causal_decay_d128"], H=16), 4360)
+
+
+@pytest.mark.parametrize("room", ["full", "stash", "none"])
+def test_workspace_entry_point(cuda_lib, room):
+    """linattn_bwd_causal_ws: with the queried workspace (split forward pass),
+    with only the per-token stash (unsplit), and with none (the stash in the
+    dk rows, the passes in order) the gradients are the same."""
+    from weight_state_recurrence_b200 import linattn as L
+    B, H, N = 1, 3, 700
+    q, k, v = inputs.random_case(4700, B, H, N, D, D, torch.bfloat16, scale=D ** -0.5)
+    dy = torch.randn(B, H, N, D, generator=torch.Generator().manual_seed(4701)).to(torch.bfloat16)
+    lam = torch.tensor([0.9, 0.99, 1.0])
+    need = L.linattn_bwd_causal_workspace(B, H, N, D, D, torch.bfloat16)
+    assert need >= B * H * N * 8
+    nbytes = {"full": need, "stash": B * H * N * 8, "none": 0}[room]
+    ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=DEV)[:nbytes] if nbytes else None
+    args = (q.to(DEV), k.to(DEV), v.to(DEV), dy.to(DEV), lam.to(DEV), 1e-6)
+    if ws is None:
+        # the ws entry point with (NULL, 0)
+        d = L.linattn_dims(B, H, N, D, D, L.LINATTN_BF16, 0)
+        dq, dk, dv = (torch.empty_like(args[0]), torch.empty_like(args[1]),
+                      torch.empty_like(args[2]))
+        dl = torch.empty(H, device=DEV)
+        rc = L.load().linattn_bwd_causal_ws(ctypes.byref(d), *(L._ptr(t) for t in args[:3]),
+                                            L._ptr(args[4]), 1e-6, L._ptr(args[3]), L._ptr(dq),
+                                            L._ptr(dk), L._ptr(dv), L._ptr(dl), None, 0, None)
+        assert rc == 0
+    else:
+        dq, dk, dv, dl = cuda_lib.bwd_causal(*args[:4], args[4], 1e-6, want_dlam=True,
+                                             workspace=ws)
+    torch.cuda.synchronize()
+    _, dq_o, dk_o, dv_o, dl_o = og.causal_grad(q, k, v, lam, 1e-6, dy)
+    errs = {n: max_rel(a, b) for n, a, b in
+            (("dq", dq, dq_o), ("dk", dk, dk_o), ("dv", dv, dv_o), ("dlambda", dl, dl_o))}
+    assert max(errs.values()) <= TOL, errs
 
 
 def test_identity_features(cuda_lib):

@@ -320,8 +320,9 @@ struct Halves {
 constexpr int kMidFloats = D * D + 2 * D + 4;
 
 namespace ps {
-constexpr uint32_t kOffK = 0, kOffV = kTile, kOffMisc = 2 * kTile;
-enum { kFullK = 0, kFullV, kMma, kFinal, kNumBars };
+// two stages of (k, v) tiles: the copies of chunk c + 2 are issued once chunk c is done
+constexpr uint32_t kOffK0 = 0, kOffV0 = kTile, kStage = 2 * kTile, kOffMisc = 2 * kStage;
+enum { kFullK0 = 0, kFullV0, kFullK1, kFullV1, kMma, kFinal, kNumBars };
 constexpr uint32_t kMiscTmem = 64, kMiscFlag = 68, kMiscPw = 128;
 constexpr uint32_t kMiscW = kMiscPw + 132 * 4, kMiscScr = kMiscW + 128 * 4;
 constexpr uint32_t kSmemBytes = kOffMisc + kMiscScr + 2 * 8 * 128 * 4;
@@ -355,17 +356,20 @@ __global__ void __launch_bounds__(NT, 1)
   float *wr = reinterpret_cast<float *>(misc + kMiscW);    // this chunk's row weights
   float *scr = reinterpret_cast<float *>(misc + kMiscScr);
   const int hf = tid >> 7, i = tid & 127;
-  const CUtensorMap *maps[2] = {&tm_k, &tm_v};
-  const uint32_t offs[2] = {kOffK, kOffV};
-  int issued[2] = {0, 0}, waited[2] = {0, 0};
-  auto load = [&](int which, int c) {
-    const uint32_t b = bar(kFullK + which);
-    mbar_arrive_expect_tx(b, kTile);
-    tma_load_3d(sb + offs[which], maps[which], b, 0, c * C, static_cast<int>(bh));
-    tma_load_3d(sb + offs[which] + kPanel, maps[which], b, 64, c * C, static_cast<int>(bh));
-    if (c + 1 < H0) tma_prefetch_l2_3d(maps[which], 0, (c + 1) * C, static_cast<int>(bh));
-    if (c + 1 < H0) tma_prefetch_l2_3d(maps[which], 64, (c + 1) * C, static_cast<int>(bh));
-    ++issued[which];
+  int issued[4] = {0, 0, 0, 0}, waited[4] = {0, 0, 0, 0};   // per barrier kFullK0..kFullV1
+  auto load = [&](int c) {
+    const int st = c & 1;
+    for (int which = 0; which < 2; ++which) {
+      const CUtensorMap *map = which ? &tm_v : &tm_k;
+      const int b = 2 * st + which;
+      const uint32_t dst = sb + st * kStage + (which ? kOffV0 : kOffK0);
+      mbar_arrive_expect_tx(bar(b), kTile);
+      tma_load_3d(dst, map, bar(b), 0, c * C, static_cast<int>(bh));
+      tma_load_3d(dst + kPanel, map, bar(b), 64, c * C, static_cast<int>(bh));
+      if (c + 2 < H0) tma_prefetch_l2_3d(map, 0, (c + 2) * C, static_cast<int>(bh));
+      if (c + 2 < H0) tma_prefetch_l2_3d(map, 64, (c + 2) * C, static_cast<int>(bh));
+      ++issued[b];
+    }
   };
   if (tid == 0) {
     for (int b = 0; b < kNumBars; ++b) mbar_init(bar(b), 1);
@@ -386,14 +390,12 @@ __global__ void __launch_bounds__(NT, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t lf = static_cast<uint32_t>((warp & 3) * 32) << 16;
-  if (tid == 0 && H0 > 0) {
-    load(0, 0);
-    load(1, 0);
-  }
+  if (tid == 0)
+    for (int c = 0; c < min(H0, 2); ++c) load(c);
   auto poll = [&](int b, int parity) {
     if (tid == 0 && !*flag) {
       if (!mbar_wait(bar(b), static_cast<uint32_t>(parity) & 1u)) *flag = 1;
-      else if (b <= kFullV) ++waited[b];
+      else if (b <= kFullV1) ++waited[b];
     }
   };
   auto meet = [&]() -> bool {
@@ -403,39 +405,39 @@ __global__ void __launch_bounds__(NT, 1)
     return *flag == 0;
   };
   int mph = 0;
-  const uint64_t dKm = mdesc(sb + kOffK), dVm = mdesc(sb + kOffV);
+  float geo = 0.f;   // sum_s lambda^(C-1-s)
+  for (int m = 0; m < C; ++m) geo += pw[m];
   float zt_acc = 0.f, s_acc = 0.f, zeta = 0.f;   // thread i < 128: column i of zt and s
 
   for (int c = 0; c < H0; ++c) {
+    const int st = c & 1;
+    uint8_t *tk = sm + st * kStage + kOffK0, *tv = sm + st * kStage + kOffV0;
     const float tc = pow_int(L, (H0 - 1 - c) * C);   // lambda^((H0-1-c) C)
     if (tid < 128) wr[i] = tc * pw[C - 1 - i];
-    poll(kFullK, c);
-    poll(kFullV, c);
+    poll(2 * st, c >> 1);
+    poll(2 * st + 1, c >> 1);
     if (!meet()) break;
-    elu_row(sm + kOffK, i, hf, ident);
-    scale_row(sm + kOffK, sm + kOffK, i, hf, wr[i]);
+    elu_row(tk, i, hf, ident);
+    scale_row(tk, tk, i, hf, wr[i]);
     fence_proxy_async_smem();
     if (!meet()) break;
     if (tid == 0) {
-      mma_ss(tmem, dKm, true, dVm, true, c > 0);   // St += (W Kt)^T V
+      mma_ss(tmem, mdesc(smem_u32(tk)), true, mdesc(smem_u32(tv)), true, c > 0);   // St += (W Kt)^T V
       umma_commit(bar(kMma));
     }
     {
       float zc = 0.f, sc = 0.f;
-      col_sums(sm + kOffK, nullptr, sm + kOffV, wr, scr, zc, sc);
+      col_sums(tk, nullptr, tv, wr, scr, zc, sc);
       if (tid < 128) {
         zt_acc += zc;
         s_acc += sc;
       }
     }
-    for (int m = 0; m < C; ++m) zeta += wr[m];
+    zeta += tc * geo;
     poll(kMma, mph);
     ++mph;
     if (!meet()) break;
-    if (tid == 0 && c + 1 < H0) {
-      load(0, c + 1);
-      load(1, c + 1);
-    }
+    if (tid == 0 && c + 2 < H0) load(c + 2);   // this stage is free
   }
   if (!*flag && H0 > 0) {
     float *m = mid + bh * kMidFloats;
@@ -457,8 +459,8 @@ __global__ void __launch_bounds__(NT, 1)
     if (tid == 0) m[D * D + 2 * D] = zeta;
   }
   if (tid == 0) {
-    for (int b = 0; b < 2; ++b)
-      for (int n = waited[b]; n < issued[b]; ++n) mbar_wait(bar(kFullK + b), n & 1);
+    for (int b = 0; b < 4; ++b)
+      for (int n = waited[b]; n < issued[b]; ++n) mbar_wait(bar(b), n & 1);
     umma_commit(bar(kFinal));
     mbar_wait(bar(kFinal), 0);
   }

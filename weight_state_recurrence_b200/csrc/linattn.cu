@@ -610,9 +610,31 @@ int launch_pdl(void (*kern)(KArgs...), int grid, int block, size_t smem, cudaStr
                                                                    : LINATTN_ERR_CUDA;
 }
 
+// Split point of pass F (0: one CTA per head), see launch_bwd_tc.
+int bwd_split(const linattn_dims *d) {
+  const int BH = d->B * d->H;
+  const int nch = (d->N + btc::C - 1) / btc::C;
+  const int sms = num_sms();
+  const int H0 = (nch >= 2 && sms > 0 && BH < sms) ? (nch * 100 + 179) / 180 : 0;
+  return H0 >= nch ? 0 : H0;
+}
+
+// Workspace of the tensor-core backward: the mid-sequence states (when pass
+// F is split) and the per-token den, dden stash.
+size_t bwd_tc_bytes(const linattn_dims *d, int H0) {
+  const size_t BH = static_cast<size_t>(d->B) * d->H;
+  return (H0 ? BH * btc::kMidFloats * sizeof(float) : 0) +
+         BH * static_cast<size_t>(d->N) * 2 * sizeof(float);
+}
+
+// user_ws: the caller's workspace, used when it holds the split form or at
+// least the stash; otherwise, with may_alloc, one is allocated on the stream;
+// with neither, the stash lives in the dk rows and the passes run in order,
+// unsplit.
 int launch_bwd_tc(const linattn_dims *d, const void *q, const void *k, const void *v,
                   const float *lam, float eps, const void *dy, void *dq, void *dk, void *dv,
-                  float *dlam, cudaStream_t s) {
+                  float *dlam, void *user_ws, size_t user_bytes, bool may_alloc,
+                  cudaStream_t s) {
   const int BH = d->B * d->H;
   CUtensorMap mq, mk, mv, mg;
   if (!make_map_bf16(&mq, q, 128, d->N, BH) || !make_map_bf16(&mk, k, 128, d->N, BH) ||
@@ -631,19 +653,26 @@ int launch_bwd_tc(const linattn_dims *d, const void *q, const void *k, const voi
   // first half from the start, the second from the state at token H0 C
   // (written by the state pass, which runs beside the first halves).  The
   // split point balances the first half against the state pass plus the
-  // second half (the state pass costs ~0.15 of pass F per chunk).
-  const int nch = (d->N + btc::C - 1) / btc::C;
-  const int sms = num_sms();
-  int H0 = (nch >= 2 && sms > 0 && BH < sms) ? (nch * 54 + 99) / 100 : 0;
-  if (H0 >= nch) H0 = 0;
-  const size_t mid_bytes = H0 ? static_cast<size_t>(BH) * btc::kMidFloats * sizeof(float) : 0;
-  const size_t stash_bytes = static_cast<size_t>(BH) * d->N * 2 * sizeof(float);
+  // second half: with the state pass at a fraction a of pass F's time per
+  // chunk, H0 = nch / (2 - a); a is ~0.2.
+  int H0 = bwd_split(d);
   char *ws = nullptr;
-  if (cudaMallocAsync(reinterpret_cast<void **>(&ws), mid_bytes + stash_bytes, s) != cudaSuccess) {
-    cudaGetLastError();   // fall back to the stash in the dk rows, unsplit
-    ws = nullptr;
+  bool owned = false;
+  if (user_ws && user_bytes >= bwd_tc_bytes(d, H0)) {
+    ws = static_cast<char *>(user_ws);
+  } else if (user_ws && user_bytes >= bwd_tc_bytes(d, 0)) {
+    ws = static_cast<char *>(user_ws);
     H0 = 0;
+  } else if (may_alloc) {
+    if (cudaMallocAsync(reinterpret_cast<void **>(&ws), bwd_tc_bytes(d, H0), s) == cudaSuccess) {
+      owned = true;
+    } else {
+      cudaGetLastError();
+      ws = nullptr;
+    }
   }
+  if (!ws) H0 = 0;   // the stash in the dk rows, unsplit
+  const size_t mid_bytes = bwd_tc_bytes(d, H0) - bwd_tc_bytes(d, 0);
   float *mid = ws ? reinterpret_cast<float *>(ws) : nullptr;
   float *stash = ws ? reinterpret_cast<float *>(ws + mid_bytes) : reinterpret_cast<float *>(dk);
   const long stride = ws ? 2 : btc::D / 2;
@@ -662,7 +691,7 @@ int launch_bwd_tc(const linattn_dims *d, const void *q, const void *k, const voi
     rc = launch_pdl(btc::bwd_tc_r_kernel, BH, btc::NT, btc::pr::kSmemBytes, s,
                     ws != nullptr && dlam != nullptr, mq, mk, mv, mg, lam,
                     static_cast<const float *>(stash), stride, bk, bv, d->H, d->N, id);
-  if (ws && cudaFreeAsync(ws, s) != cudaSuccess && rc == LINATTN_OK) rc = LINATTN_ERR_CUDA;
+  if (owned && cudaFreeAsync(ws, s) != cudaSuccess && rc == LINATTN_OK) rc = LINATTN_ERR_CUDA;
   return rc;
 }
 
@@ -974,10 +1003,12 @@ extern "C" int linattn_combine_states(const linattn_dims *d, int G, const float 
   return launch_status();
 }
 
-extern "C" int linattn_bwd_causal(const linattn_dims *d, const void *q, const void *k,
-                                  const void *v, const float *lambda, float eps, const void *dy,
-                                  void *dq, void *dk, void *dv, float *dlambda,
-                                  linattn_stream_t stream) {
+namespace linattn {
+namespace {
+
+int bwd_causal_impl(const linattn_dims *d, const void *q, const void *k, const void *v,
+                    const float *lambda, float eps, const void *dy, void *dq, void *dk, void *dv,
+                    float *dlambda, void *ws, size_t ws_bytes, bool may_alloc, cudaStream_t s) {
   int rc = check_dims(d, true);
   if (rc != LINATTN_OK) return rc;
   if (bad_eps(eps)) return LINATTN_ERR_INVALID;
@@ -988,26 +1019,56 @@ extern "C" int linattn_bwd_causal(const linattn_dims *d, const void *q, const vo
   if (BH > 0 && d->N > 0 && (!q || !k || !v || !dy || !dq || !dk || !dv))
     return LINATTN_ERR_INVALID;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dy) || !aligned16(dq) ||
-      !aligned16(dk) || !aligned16(dv) || !aligned16(lambda) || !aligned16(dlambda))
+      !aligned16(dk) || !aligned16(dv) || !aligned16(lambda) || !aligned16(dlambda) ||
+      !aligned16(ws))
     return LINATTN_ERR_INVALID;
-  // every output overlaps no input and no other output
+  // every output (and the workspace) overlaps no input and no other output
   const void *in[5] = {q, k, v, dy, lambda};
   const size_t nin[5] = {nq, nq, nv, nv, nl};
-  const void *outp[4] = {dq, dk, dv, dlambda};
-  const size_t nout[4] = {nq, nq, nv, nl};
-  for (int o = 0; o < 4; ++o) {
+  const void *outp[5] = {dq, dk, dv, dlambda, ws};
+  const size_t nout[5] = {nq, nq, nv, nl, ws ? ws_bytes : 0};
+  for (int o = 0; o < 5; ++o) {
     for (int i = 0; i < 5; ++i)
       if (overlaps(outp[o], nout[o], in[i], nin[i])) return LINATTN_ERR_INVALID;
-    for (int o2 = o + 1; o2 < 4; ++o2)
+    for (int o2 = o + 1; o2 < 5; ++o2)
       if (overlaps(outp[o], nout[o], outp[o2], nout[o2])) return LINATTN_ERR_INVALID;
   }
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (dlambda && cudaMemsetAsync(dlambda, 0, nl, s) != cudaSuccess) return LINATTN_ERR_CUDA;
   if (BH == 0 || d->N == 0) return LINATTN_OK;
-  if (use_tc_bwd(d)) return launch_bwd_tc(d, q, k, v, lambda, eps, dy, dq, dk, dv, dlambda, s);
+  if (use_tc_bwd(d))
+    return launch_bwd_tc(d, q, k, v, lambda, eps, dy, dq, dk, dv, dlambda, ws, ws_bytes,
+                         may_alloc, s);
   if (d->dtype == LINATTN_F32)
     return causal_bwd_dispatch<float>(d, q, k, v, lambda, eps, dy, dq, dk, dv, dlambda, s);
   return causal_bwd_dispatch<bf16>(d, q, k, v, lambda, eps, dy, dq, dk, dv, dlambda, s);
+}
+
+}  // namespace
+}  // namespace linattn
+
+extern "C" int linattn_bwd_causal(const linattn_dims *d, const void *q, const void *k,
+                                  const void *v, const float *lambda, float eps, const void *dy,
+                                  void *dq, void *dk, void *dv, float *dlambda,
+                                  linattn_stream_t stream) {
+  return bwd_causal_impl(d, q, k, v, lambda, eps, dy, dq, dk, dv, dlambda, nullptr, 0, true,
+                         reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" size_t linattn_bwd_causal_workspace(const linattn_dims *d) {
+  if (!d || check_dims(d, true) != LINATTN_OK || !use_tc_bwd(d)) return 0;
+  if (static_cast<size_t>(d->B) * d->H == 0 || d->N == 0) return 0;
+  return bwd_tc_bytes(d, bwd_split(d));
+}
+
+extern "C" int linattn_bwd_causal_ws(const linattn_dims *d, const void *q, const void *k,
+                                     const void *v, const float *lambda, float eps,
+                                     const void *dy, void *dq, void *dk, void *dv,
+                                     float *dlambda, void *workspace, size_t workspace_bytes,
+                                     linattn_stream_t stream) {
+  if (!workspace && workspace_bytes) return LINATTN_ERR_INVALID;
+  return bwd_causal_impl(d, q, k, v, lambda, eps, dy, dq, dk, dv, dlambda, workspace,
+                         workspace ? workspace_bytes : 0, false,
+                         reinterpret_cast<cudaStream_t>(stream));
 }
 
 namespace linattn {

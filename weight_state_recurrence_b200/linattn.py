@@ -35,7 +35,8 @@ ENTRY_POINTS = ("linattn_fwd_causal", "linattn_fwd_causal_from", "linattn_fwd_ca
                 "linattn_fwd_global", "linattn_fwd_global_cross", "linattn_decode_step",
                 "linattn_performer_features", "linattn_status_string", "linattn_device_status",
                 "linattn_version", "linattn_set_kernel_choice", "linattn_causal_state",
-                "linattn_combine_states", "linattn_fwd_global_masked")
+                "linattn_combine_states", "linattn_fwd_global_masked",
+                "linattn_bwd_causal_workspace", "linattn_bwd_causal_ws")
 
 
 class linattn_dims(ctypes.Structure):
@@ -84,6 +85,11 @@ def load(build_if_missing: bool = True):
     lib.linattn_fwd_causal_noalloc.restype = i
     lib.linattn_bwd_causal.argtypes = [dp, vp, vp, vp, fp, f, vp, vp, vp, vp, fp, vp]
     lib.linattn_bwd_causal.restype = i
+    lib.linattn_bwd_causal_workspace.argtypes = [dp]
+    lib.linattn_bwd_causal_workspace.restype = ctypes.c_size_t
+    lib.linattn_bwd_causal_ws.argtypes = [dp, vp, vp, vp, fp, f, vp, vp, vp, vp, fp, vp,
+                                          ctypes.c_size_t, vp]
+    lib.linattn_bwd_causal_ws.restype = i
     lib.linattn_fwd_global.argtypes = [dp, vp, vp, vp, f, vp, fp, fp, vp]
     lib.linattn_fwd_global.restype = i
     lib.linattn_fwd_global_cross.argtypes = [dp, i, vp, vp, vp, f, vp, fp, fp, vp]
@@ -257,10 +263,16 @@ def linattn_fwd_causal_noalloc(q, k, v, lam, eps, out, S_final=None, z_final=Non
            "linattn_fwd_causal_noalloc")
 
 
+def linattn_bwd_causal_workspace(B, H, N, dk, dv, dtype, phi=LINATTN_PHI_ELU1) -> int:
+    d = linattn_dims(B, H, N, dk, dv, _dtype_code(dtype), int(phi))
+    return int(load().linattn_bwd_causal_workspace(ctypes.byref(d)))
+
+
 def linattn_bwd_causal(q, k, v, lam, eps, dy, dq, dk, dv, dlam=None, stream=None, *,
-                       phi=LINATTN_PHI_ELU1):
+                       phi=LINATTN_PHI_ELU1, workspace=None):
     """Backward of the causal forward: dy like v; dq, dk like q; dv like v;
-    dlam [H] fp32 or None."""
+    dlam [H] fp32 or None; workspace: a uint8 device tensor for
+    linattn_bwd_causal_ws (None: linattn_bwd_causal)."""
     B, H, N, dk_ = q.shape
     dv_ = v.shape[-1]
     if (k.shape != q.shape or tuple(v.shape) != (B, H, N, dv_) or dy.shape != v.shape or
@@ -271,6 +283,13 @@ def linattn_bwd_causal(q, k, v, lam, eps, dy, dq, dk, dv, dlam=None, stream=None
     _f32(lam, (H,), "lambda")
     _f32(dlam, (H,), "dlambda")
     d = linattn_dims(B, H, N, dk_, dv_, _dtype_code(q.dtype), int(phi))
+    if workspace is not None:
+        _check(load().linattn_bwd_causal_ws(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), _ptr(lam),
+                                            float(eps), _ptr(dy), _ptr(dq), _ptr(dk), _ptr(dv),
+                                            _ptr(dlam), _ptr(workspace),
+                                            workspace.numel() * workspace.element_size(),
+                                            _stream(stream)), "linattn_bwd_causal_ws")
+        return
     _check(load().linattn_bwd_causal(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), _ptr(lam),
                                      float(eps), _ptr(dy), _ptr(dq), _ptr(dk), _ptr(dv),
                                      _ptr(dlam), _stream(stream)), "linattn_bwd_causal")
@@ -431,10 +450,11 @@ def fwd_causal(q, k, v, lam=None, eps=1e-6, want_state=True, S_init=None, z_init
 
 
 def bwd_causal(q, k, v, dy, lam=None, eps=1e-6, want_dlam=False, stream=None,
-               phi=LINATTN_PHI_ELU1):
+               phi=LINATTN_PHI_ELU1, workspace=None):
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     dlam = (torch.empty(q.shape[1], dtype=torch.float32, device=q.device) if want_dlam else None)
-    linattn_bwd_causal(q, k, v, lam, eps, dy, dq, dk, dv, dlam, stream, phi=phi)
+    linattn_bwd_causal(q, k, v, lam, eps, dy, dq, dk, dv, dlam, stream, phi=phi,
+                       workspace=workspace)
     return dq, dk, dv, dlam
 
 
