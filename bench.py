@@ -501,15 +501,21 @@ def bwd_leg(lib, args, world, rank, stream, tensor_peak, hbm_peak):
     def step():
         lib.linattn_bwd_causal(q, k, v, lam, WL.eps, dy, dq, dk, dv, dl, stream, workspace=ws)
 
+    def step_no_dlam():
+        lib.linattn_bwd_causal(q, k, v, lam, WL.eps, dy, dq, dk, dv, None, stream, workspace=ws)
+
     steps = max(1, min(args.steps, 10))
     with torch.cuda.stream(stream):
         ms = time_steps(step, steps, args.warmup, world, stream)
+        ms_nd = time_steps(step_no_dlam, steps, args.warmup, world, stream)
     assert lib.linattn_device_status(clear=True, stream=stream) == 0
     per = ms / 1e3 / steps
     fl = bwd_mma_flops(B, H, N, d)
     by = bwd_bytes(B, H, N, d)
     res = {"value": B * N * world / per, "unit": "tokens/s", "ms_per_step": per * 1e3,
            "steps": steps, "ctas": B * H, "workspace_bytes": need,
+           "without_dlambda": {"ms_per_step": ms_nd / steps,
+                               "flops_per_launch": bwd_mma_flops(B, H, N, d, with_dlam=False)},
            "roofline": {"bound": "tensor", "achieved": fl / per / 1e12, "peak": tensor_peak,
                         "unit": "TFLOP/s", "frac": fl / per / 1e12 / tensor_peak,
                         "flops_per_launch": fl,

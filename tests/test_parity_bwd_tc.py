@@ -79,6 +79,10 @@ def test_split_and_unsplit_forward_pass(cuda_lib):
     (5 chunks), and 160 heads over 3 chunks (no split)."""
     check(cuda_lib, 1, 2, 600, torch.tensor([0.95, 1.0]), 4350)
     check(cuda_lib, 10, 16, 300, inputs.decay(inputs.WORKLOADS["causal_decay_d128"], H=16), 4360)
+    # without dlambda the reverse pass is split too (its earlier half from the
+    # reverse state pass's adjoint): odd and even split points
+    check(cuda_lib, 1, 2, 600, torch.tensor([0.95, 1.0]), 4370, want_dlam=False)
+    check(cuda_lib, 1, 3, 1100, torch.tensor([0.5, 0.9, 0.999]), 4380, want_dlam=False)
 
 
 @pytest.mark.parametrize("room", ["full", "stash", "none"])

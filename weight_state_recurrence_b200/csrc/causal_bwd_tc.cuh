@@ -912,6 +912,163 @@ __global__ void __launch_bounds__(NT, 1)
   }
 }
 
+// ============================================================== reverse state pass for split R
+// Pass R can run as two CTAs per head: chunks [H1, nch) and [0, H1), each
+// walked in reverse.  The second starts from the adjoint of every token at or
+// after T = H1 C:
+//   R = sum_{t>=T} lambda^(t-T+1) phi(q_t) w_t^T,   r = sum_{t>=T} lambda^(t-T+1) phi(q_t) dden_t
+// which this pass sums over chunks [H1, nch) (q row t of chunk c weighted
+// lambda^((c-H1) C) lambda^(t+1), no decay pass) and writes to `mid`: per
+// head R [128][128] fp32, then r [128].
+namespace pt {
+constexpr uint32_t kOffQ0 = 0, kOffG0 = kTile, kStage = 2 * kTile, kOffMisc = 2 * kStage;
+enum { kFullQ0 = 0, kFullG0, kFullQ1, kFullG1, kMma, kFinal, kNumBars };
+constexpr uint32_t kMiscTmem = 64, kMiscFlag = 68, kMiscPw = 128;
+constexpr uint32_t kMiscDd = kMiscPw + 132 * 4, kMiscScr = kMiscDd + 128 * 4;
+constexpr uint32_t kSmemBytes = kOffMisc + kMiscScr + 2 * 8 * 128 * 4;
+static_assert(kSmemBytes <= 232448, "exceeds the per-CTA shared memory of sm_100");
+}  // namespace pt
+
+__global__ void __launch_bounds__(NT, 1)
+    bwd_tc_t_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_g,
+                    const float *__restrict__ lam, const float *__restrict__ stash,
+                    long stash_stride, float *__restrict__ mid, int H, int N, int H1, bool ident) {
+  using namespace pt;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *sm = smem_raw;
+  const uint32_t sb = smem_u32(sm);
+  const int tid = threadIdx.x, warp = tid >> 5;
+  if (sb & 1023u) {
+    if (tid == 0) atomicOr(&g_status, kStatusWaitTimeout);
+    return;
+  }
+  // pass R (launched next as this pass's programmatic dependent) starts its
+  // later halves at once; its earlier halves wait for this grid
+  grid_launch_dependents();
+  const long bh = blockIdx.x;
+  const int h = static_cast<int>(bh % H);
+  const float L = lam ? lam[h] : 1.f;
+  const int nch = (N + C - 1) / C, n = nch - H1;   // chunks H1 .. nch-1
+  uint8_t *misc = sm + kOffMisc;
+  auto bar = [&](int i) { return sb + kOffMisc + 8u * static_cast<uint32_t>(i); };
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(misc + kMiscTmem);
+  volatile int *flag = reinterpret_cast<volatile int *>(misc + kMiscFlag);
+  float *pw = reinterpret_cast<float *>(misc + kMiscPw);   // lambda^m, m = 0..C
+  float *dd = reinterpret_cast<float *>(misc + kMiscDd);   // dden of the chunk's tokens
+  float *scr = reinterpret_cast<float *>(misc + kMiscScr);
+  const int hf = tid >> 7, i = tid & 127;
+  int issued[4] = {0, 0, 0, 0}, waited[4] = {0, 0, 0, 0};
+  auto load = [&](int j) {   // j-th chunk of the walk: chunk H1 + j
+    const int st = j & 1, c = H1 + j;
+    for (int which = 0; which < 2; ++which) {
+      const CUtensorMap *map = which ? &tm_g : &tm_q;
+      const int b = 2 * st + which;
+      const uint32_t dst = sb + st * kStage + (which ? kOffG0 : kOffQ0);
+      mbar_arrive_expect_tx(bar(b), kTile);
+      tma_load_3d(dst, map, bar(b), 0, c * C, static_cast<int>(bh));
+      tma_load_3d(dst + kPanel, map, bar(b), 64, c * C, static_cast<int>(bh));
+      if (j + 2 < n) tma_prefetch_l2_3d(map, 0, (c + 2) * C, static_cast<int>(bh));
+      if (j + 2 < n) tma_prefetch_l2_3d(map, 64, (c + 2) * C, static_cast<int>(bh));
+      ++issued[b];
+    }
+  };
+  if (tid == 0) {
+    for (int b = 0; b < kNumBars; ++b) mbar_init(bar(b), 1);
+    *flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_g);
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_slot), 128);
+    tmem_relinquish();
+  }
+  if (tid < 128) pw[tid] = pow_int(L, tid);
+  if (tid == 0) pw[C] = pow_int(L, C);
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t lf = static_cast<uint32_t>((warp & 3) * 32) << 16;
+  if (tid == 0)
+    for (int j = 0; j < min(n, 2); ++j) load(j);
+  auto poll = [&](int b, int parity) {
+    if (tid == 0 && !*flag) {
+      if (!mbar_wait(bar(b), static_cast<uint32_t>(parity) & 1u)) *flag = 1;
+      else if (b <= kFullG1) ++waited[b];
+    }
+  };
+  auto meet = [&]() -> bool {
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    return *flag == 0;
+  };
+  int mph = 0;
+  float r_acc = 0.f;   // thread i < 128: column i of r
+
+  for (int j = 0; j < n; ++j) {
+    const int st = j & 1, c = H1 + j, row0 = c * C, Cv = min(C, N - row0);
+    uint8_t *tq = sm + st * kStage + kOffQ0, *tg = sm + st * kStage + kOffG0;
+    float den = 1.f, dden = 0.f;   // tokens past the end: no gradient
+    if (i < Cv) {
+      const float2 sv = *reinterpret_cast<const float2 *>(stash + (bh * N + row0 + i) * stash_stride);
+      den = sv.x;
+      dden = sv.y;
+    }
+    if (hf == 0) dd[i] = dden;
+    poll(2 * st, j >> 1);
+    poll(2 * st + 1, j >> 1);
+    if (!meet()) break;
+    phi_row(tq, i, hf, ident, nullptr);
+    scale_row(tq, tq, i, hf, pow_int(L, j * C) * pw[i + 1]);
+    dnum_row(tg, i, hf, 1.f / den);
+    fence_proxy_async_smem();
+    if (!meet()) break;
+    if (tid == 0) {
+      mma_ss(tmem, mdesc(smem_u32(tq)), true, mdesc(smem_u32(tg)), true, j > 0);   // R += (Lq Q)^T w
+      umma_commit(bar(kMma));
+    }
+    {
+      float rc = 0.f, unused = 0.f;
+      col_sums(tq, dd, nullptr, nullptr, scr, rc, unused);
+      if (tid < 128) r_acc += rc;
+    }
+    poll(kMma, mph);
+    ++mph;
+    if (!meet()) break;
+    if (tid == 0 && j + 2 < n) load(j + 2);   // this stage is free
+  }
+  if (!*flag && n > 0) {
+    float *m = mid + bh * kMidFloats;
+#pragma unroll 1
+    for (int blk = 2 * hf; blk < 2 * hf + 2; ++blk) {
+      uint32_t v[32];
+      tmem_ld_32x32b_x32(tmem + lf + blk * 32, v);
+      tmem_wait_ld();
+      float4 *dst = reinterpret_cast<float4 *>(m + i * D + blk * 32);
+#pragma unroll
+      for (int e = 0; e < 8; ++e)
+        dst[e] = make_float4(__uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]),
+                             __uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3]));
+    }
+    if (tid < 128) m[D * D + i] = r_acc;
+  }
+  if (tid == 0) {
+    for (int b = 0; b < 4; ++b)
+      for (int k = waited[b]; k < issued[b]; ++k) mbar_wait(bar(b), k & 1);
+    umma_commit(bar(kFinal));
+    mbar_wait(bar(kFinal), 0);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 128);
+  }
+}
+
 // ============================================================== pass R
 namespace pr {
 constexpr uint32_t kOffQ = 0, kOffK = kTile, kOffKd = 2 * kTile, kOffV = 3 * kTile,
@@ -928,8 +1085,8 @@ __global__ void __launch_bounds__(NT, 1)
     bwd_tc_r_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
                     const float *__restrict__ lam, const float *stash, long stash_stride,
-                    __nv_bfloat16 *__restrict__ dk, __nv_bfloat16 *__restrict__ dv, int H, int N,
-                    bool ident) {
+                    __nv_bfloat16 *__restrict__ dk, __nv_bfloat16 *__restrict__ dv,
+                    const float *__restrict__ rmid, int H1, int H, int N, bool ident) {
   using namespace pr;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *sm = smem_raw;
@@ -939,10 +1096,16 @@ __global__ void __launch_bounds__(NT, 1)
     if (tid == 0) atomicOr(&g_status, kStatusWaitTimeout);
     return;
   }
-  const long bh = blockIdx.x;
+  // H1 > 0: two CTAs per head, chunks [H1, nch) and [0, H1), each walked in
+  // reverse; the second starts from the adjoint the reverse state pass leaves in `rmid`
+  const int G = H1 > 0 ? 2 : 1;
+  const long BH = gridDim.x / G;
+  const int half = static_cast<int>(blockIdx.x / BH);
+  const long bh = blockIdx.x % BH;
   const int h = static_cast<int>(bh % H);
   const float L = lam ? lam[h] : 1.f;
   const int nch = (N + C - 1) / C;
+  const int c_lo = half ? 0 : H1, c_hi = half ? H1 : nch;   // chunks [c_lo, c_hi)
   uint8_t *misc = sm + kOffMisc;
   auto bar = [&](int i) { return sb + kOffMisc + 8u * static_cast<uint32_t>(i); };
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(misc + kMiscTmem);
@@ -983,8 +1146,8 @@ __global__ void __launch_bounds__(NT, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t lf = static_cast<uint32_t>((warp & 3) * 32) << 16;
-  if (tid == 0 && nch > 0)
-    for (int b = 0; b < 4; ++b) load(b, nch - 1);
+  if (tid == 0 && c_lo < c_hi)
+    for (int b = 0; b < 4; ++b) load(b, c_hi - 1);
   auto poll = [&](int b, int parity) {
     if (tid == 0 && !*flag) {
       if (!mbar_wait(bar(b), static_cast<uint32_t>(parity) & 1u)) *flag = 1;
@@ -1011,12 +1174,37 @@ __global__ void __launch_bounds__(NT, 1)
   // den, dden of this thread's token in the chunk being processed (tokens past
   // the end: no gradient); the next chunk's pair is loaded a chunk ahead
   float2 st = make_float2(1.f, 0.f);
-  if (nch > 0 && i < N - (nch - 1) * C)
-    st = *reinterpret_cast<const float2 *>(stash + (bh * N + (nch - 1) * C + i) * stash_stride);
+  if (c_lo < c_hi && i < N - (c_hi - 1) * C)
+    st = *reinterpret_cast<const float2 *>(stash + (bh * N + (c_hi - 1) * C + i) * stash_stride);
+  if (half == 1) {
+    // the adjoint of the tokens from H1 C on, from the reverse state pass
+    // (this grid's prerequisite)
+    grid_dependency_wait();
+    const float *m = rmid + bh * kMidFloats;
+#pragma unroll 1
+    for (int blk = 2 * hf; blk < 2 * hf + 2; ++blk) {
+      uint32_t v[32];
+      const float4 *src = reinterpret_cast<const float4 *>(m + i * D + blk * 32);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float4 x = src[e];
+        v[4 * e] = __float_as_uint(x.x);
+        v[4 * e + 1] = __float_as_uint(x.y);
+        v[4 * e + 2] = __float_as_uint(x.z);
+        v[4 * e + 3] = __float_as_uint(x.w);
+      }
+      tmem_st_32x32b_x32(tmem + kTmR + lf + blk * 32, v);
+    }
+    tmem_wait_st();
+    if (tid < 128) rv[i] = m[D * D + i];
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+  }
 
-  for (int cc = 0; cc < nch; ++cc) {
-    const int c = nch - 1 - cc, row0 = c * C, Cv = min(C, N - row0);
-    const bool carried = cc > 0;   // later tokens exist: R, r nonzero
+  for (int cc = 0; cc < c_hi - c_lo; ++cc) {
+    const int c = c_hi - 1 - cc, row0 = c * C, Cv = min(C, N - row0);
+    const bool carried = cc > 0 || half == 1;   // later tokens exist: R, r nonzero
     const float den = st.x, dden = st.y;
     if (hf == 0) sdd[i] = dden;
     if (carried) state_to_operand(tmem + kTmR + lf, sm + kOffRb, i, hf, pw[C]);
@@ -1041,7 +1229,7 @@ __global__ void __launch_bounds__(NT, 1)
       umma_commit(bar(kMma2));
     }
     // the next chunk's den, dden, while the products run
-    if (c > 0)
+    if (c > c_lo)
       st = *reinterpret_cast<const float2 *>(stash + (bh * N + row0 - C + i) * stash_stride);
     mma_done();
     if (!meet()) break;
@@ -1060,7 +1248,7 @@ __global__ void __launch_bounds__(NT, 1)
     }
     mma2_done();
     if (!meet()) break;
-    if (tid == 0 && c > 0) load(2, c - 1);   // v has been read (its weighted copy is made)
+    if (tid == 0 && c > c_lo) load(2, c - 1);   // v has been read (its weighted copy is made)
 #pragma unroll 1
     for (int blk = b0; blk < b0 + 2; ++blk) {
       uint32_t wv[32];
@@ -1140,7 +1328,7 @@ __global__ void __launch_bounds__(NT, 1)
                 make_uint4(pk[4 * m], pk[4 * m + 1], pk[4 * m + 2], pk[4 * m + 3]);
       }
     }
-    if (c == 0) break;
+    if (c == c_lo) break;   // the adjoint before the range is not needed here
     // ---- R += (Lq Q)^T w, r likewise: q rows weighted lambda^(t+1)
     scale_row(sm + kOffQ, sm + kOffQ, i, hf, pw[i + 1]);
     fence_proxy_async_smem();

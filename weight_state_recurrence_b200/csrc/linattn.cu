@@ -619,11 +619,11 @@ int bwd_split(const linattn_dims *d) {
   return H0 >= nch ? 0 : H0;
 }
 
-// Workspace of the tensor-core backward: the mid-sequence states (when pass
-// F is split) and the per-token den, dden stash.
+// Workspace of the tensor-core backward: the split-point states of passes F
+// and R (when they are split) and the per-token den, dden stash.
 size_t bwd_tc_bytes(const linattn_dims *d, int H0) {
   const size_t BH = static_cast<size_t>(d->B) * d->H;
-  return (H0 ? BH * btc::kMidFloats * sizeof(float) : 0) +
+  return (H0 ? 2 * BH * btc::kMidFloats * sizeof(float) : 0) +
          BH * static_cast<size_t>(d->N) * 2 * sizeof(float);
 }
 
@@ -643,7 +643,8 @@ int launch_bwd_tc(const linattn_dims *d, const void *q, const void *k, const voi
   if (!set_smem(btc::bwd_tc_f_kernel, static_cast<int>(btc::pf::kSmemBytes)) ||
       !set_smem(btc::bwd_tc_l_kernel, static_cast<int>(btc::pl::kSmemBytes)) ||
       !set_smem(btc::bwd_tc_r_kernel, static_cast<int>(btc::pr::kSmemBytes)) ||
-      !set_smem(btc::bwd_tc_s_kernel, static_cast<int>(btc::ps::kSmemBytes)))
+      !set_smem(btc::bwd_tc_s_kernel, static_cast<int>(btc::ps::kSmemBytes)) ||
+      !set_smem(btc::bwd_tc_t_kernel, static_cast<int>(btc::pt::kSmemBytes)))
     return LINATTN_ERR_CUDA;
   auto *bq = static_cast<bf16 *>(dq);
   auto *bk = static_cast<bf16 *>(dk);
@@ -672,8 +673,17 @@ int launch_bwd_tc(const linattn_dims *d, const void *q, const void *k, const voi
     }
   }
   if (!ws) H0 = 0;   // the stash in the dk rows, unsplit
+  // pass R splits at H1 = nch - H0 when no dlambda is asked for: its later
+  // half (from the end, walked first with no carried adjoint) matches F's
+  // first, and the reverse state pass over that half supplies the earlier
+  // half's starting adjoint.  With dlambda, R stays one CTA per head beside
+  // the dlambda pass: the 64 + 128 + 64 CTAs of L, split R and the reverse
+  // state pass leave a tail wave on 148 SMs (3.1 ms against 2.7).
+  const int nch = (d->N + btc::C - 1) / btc::C;
+  const int H1 = (H0 && !dlam) ? nch - H0 : 0;
   const size_t mid_bytes = bwd_tc_bytes(d, H0) - bwd_tc_bytes(d, 0);
   float *mid = ws ? reinterpret_cast<float *>(ws) : nullptr;
+  float *rmid = H0 ? mid + static_cast<size_t>(BH) * btc::kMidFloats : nullptr;
   float *stash = ws ? reinterpret_cast<float *>(ws + mid_bytes) : reinterpret_cast<float *>(dk);
   const long stride = ws ? 2 : btc::D / 2;
   int rc = LINATTN_OK;
@@ -687,10 +697,16 @@ int launch_bwd_tc(const linattn_dims *d, const void *q, const void *k, const voi
   if (rc == LINATTN_OK && dlam)
     rc = launch_pdl(btc::bwd_tc_l_kernel, BH, btc::NT, btc::pl::kSmemBytes, s, false, mq, mk, mv,
                     mg, lam, static_cast<const float *>(stash), stride, dlam, d->H, d->N, id);
+  // R (and the reverse state pass before it) read nothing that L writes: with
+  // the stash out of the dk rows they start beside L as programmatic dependents
+  const bool beside_l = ws != nullptr && dlam != nullptr;
+  if (rc == LINATTN_OK && H1)
+    rc = launch_pdl(btc::bwd_tc_t_kernel, BH, btc::NT, btc::pt::kSmemBytes, s, beside_l, mq, mg,
+                    lam, static_cast<const float *>(stash), stride, rmid, d->H, d->N, H1, id);
   if (rc == LINATTN_OK)
-    rc = launch_pdl(btc::bwd_tc_r_kernel, BH, btc::NT, btc::pr::kSmemBytes, s,
-                    ws != nullptr && dlam != nullptr, mq, mk, mv, mg, lam,
-                    static_cast<const float *>(stash), stride, bk, bv, d->H, d->N, id);
+    rc = launch_pdl(btc::bwd_tc_r_kernel, H1 ? 2 * BH : BH, btc::NT, btc::pr::kSmemBytes, s,
+                    beside_l || H1 != 0, mq, mk, mv, mg, lam, static_cast<const float *>(stash),
+                    stride, bk, bv, static_cast<const float *>(rmid), H1, d->H, d->N, id);
   if (owned && cudaFreeAsync(ws, s) != cudaSuccess && rc == LINATTN_OK) rc = LINATTN_ERR_CUDA;
   return rc;
 }
