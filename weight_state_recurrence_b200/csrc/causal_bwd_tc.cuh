@@ -1117,13 +1117,22 @@ __global__ void __launch_bounds__(NT, 1)
   float *rv = reinterpret_cast<float *>(misc + kMiscR);       // r, the normaliser's adjoint
   const int hf = tid >> 7, i = tid & 127;
   const CUtensorMap *maps[4] = {&tm_q, &tm_k, &tm_v, &tm_g};
-  const uint32_t offs[4] = {kOffQ, kOffK, kOffV, kOffG};
   int issued[4] = {0, 0, 0, 0}, waited[4] = {0, 0, 0, 0};
-  auto load = [&](int which, int c) {
+  // Tile roles alternate between chunks: the q and dy tiles of the next chunk
+  // are loaded into this chunk's weighted k and v buffers once the dv and dk
+  // products have read them, and the next chunk weights k and v into this
+  // chunk's q and dy buffers.  With parity 0 the roles sit in the buffers
+  // named for them; with parity 1 q and weighted k trade buffers, and so do
+  // dy and weighted v.
+  auto off_q = [](int p) { return p ? kOffKd : kOffQ; };
+  auto off_g = [](int p) { return p ? kOffVd : kOffG; };
+  auto off_kd = [](int p) { return p ? kOffQ : kOffKd; };
+  auto off_vd = [](int p) { return p ? kOffG : kOffVd; };
+  auto load = [&](int which, int c, uint32_t off) {
     const uint32_t b = bar(kFullQ + which);
     mbar_arrive_expect_tx(b, kTile);
-    tma_load_3d(sb + offs[which], maps[which], b, 0, c * C, static_cast<int>(bh));
-    tma_load_3d(sb + offs[which] + kPanel, maps[which], b, 64, c * C, static_cast<int>(bh));
+    tma_load_3d(sb + off, maps[which], b, 0, c * C, static_cast<int>(bh));
+    tma_load_3d(sb + off + kPanel, maps[which], b, 64, c * C, static_cast<int>(bh));
     if (c > 0) tma_prefetch_l2_3d(maps[which], 0, (c - 1) * C, static_cast<int>(bh));
     if (c > 0) tma_prefetch_l2_3d(maps[which], 64, (c - 1) * C, static_cast<int>(bh));
     ++issued[which];
@@ -1146,8 +1155,12 @@ __global__ void __launch_bounds__(NT, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t lf = static_cast<uint32_t>((warp & 3) * 32) << 16;
-  if (tid == 0 && c_lo < c_hi)
-    for (int b = 0; b < 4; ++b) load(b, c_hi - 1);
+  if (tid == 0 && c_lo < c_hi) {
+    load(0, c_hi - 1, off_q(0));
+    load(1, c_hi - 1, kOffK);
+    load(2, c_hi - 1, kOffV);
+    load(3, c_hi - 1, off_g(0));
+  }
   auto poll = [&](int b, int parity) {
     if (tid == 0 && !*flag) {
       if (!mbar_wait(bar(b), static_cast<uint32_t>(parity) & 1u)) *flag = 1;
@@ -1165,9 +1178,7 @@ __global__ void __launch_bounds__(NT, 1)
   int mph2 = 0;  // completed phases of the second MMA barrier (a product an epilogue needs later)
   auto mma2_done = [&]() { poll(kMma2, mph2); ++mph2; };
 
-  const uint64_t dQ = kdesc(sb + kOffQ), dQm = mdesc(sb + kOffQ), dK = kdesc(sb + kOffK);
-  const uint64_t dKd = kdesc(sb + kOffKd), dV = kdesc(sb + kOffV), dVd = kdesc(sb + kOffVd);
-  const uint64_t dG = kdesc(sb + kOffG), dGm = mdesc(sb + kOffG);
+  const uint64_t dK = kdesc(sb + kOffK), dV = kdesc(sb + kOffV);
   const uint64_t dRb = kdesc(sb + kOffRb), dRbm = mdesc(sb + kOffRb);
   const int b0 = 2 * hf;
   const float *mk = up + 127 - i;   // mk[s] = lambda^(s-i) for s >= i, else 0
@@ -1205,6 +1216,10 @@ __global__ void __launch_bounds__(NT, 1)
   for (int cc = 0; cc < c_hi - c_lo; ++cc) {
     const int c = c_hi - 1 - cc, row0 = c * C, Cv = min(C, N - row0);
     const bool carried = cc > 0 || half == 1;   // later tokens exist: R, r nonzero
+    const int par = cc & 1;
+    const uint32_t oQ = off_q(par), oG = off_g(par), oKd = off_kd(par), oVd = off_vd(par);
+    const uint64_t dQ = kdesc(sb + oQ), dQm = mdesc(sb + oQ), dG = kdesc(sb + oG),
+                   dGm = mdesc(sb + oG), dKd = kdesc(sb + oKd), dVd = kdesc(sb + oVd);
     const float den = st.x, dden = st.y;
     if (hf == 0) sdd[i] = dden;
     if (carried) state_to_operand(tmem + kTmR + lf, sm + kOffRb, i, hf, pw[C]);
@@ -1213,13 +1228,13 @@ __global__ void __launch_bounds__(NT, 1)
     poll(kFullV, cc);
     poll(kFullG, cc);
     if (!meet()) break;
-    phi_row(sm + kOffQ, i, hf, ident, nullptr);
+    phi_row(sm + oQ, i, hf, ident, nullptr);
     phi_row(sm + kOffK, i, hf, ident, nullptr);
     if (carried) {
-      scale_row(sm + kOffKd, sm + kOffK, i, hf, pw[C - 1 - i]);
-      scale_row(sm + kOffVd, sm + kOffV, i, hf, pw[C - 1 - i]);
+      scale_row(sm + oKd, sm + kOffK, i, hf, pw[C - 1 - i]);
+      scale_row(sm + oVd, sm + kOffV, i, hf, pw[C - 1 - i]);
     }
-    dnum_row(sm + kOffG, i, hf, 1.f / den);   // w = dnum in place of dy
+    dnum_row(sm + oG, i, hf, 1.f / den);   // w = dnum in place of dy
     fence_proxy_async_smem();
     if (!meet()) break;
     if (tid == 0) {
@@ -1248,7 +1263,7 @@ __global__ void __launch_bounds__(NT, 1)
     }
     mma2_done();
     if (!meet()) break;
-    if (tid == 0 && c > c_lo) load(2, c - 1);   // v has been read (its weighted copy is made)
+    if (tid == 0 && c > c_lo) load(2, c - 1, kOffV);   // v has been read (its weighted copy is made)
 #pragma unroll 1
     for (int blk = b0; blk < b0 + 2; ++blk) {
       uint32_t wv[32];
@@ -1296,6 +1311,11 @@ __global__ void __launch_bounds__(NT, 1)
     }
     mma2_done();
     if (!meet()) break;
+    if (tid == 0 && c > c_lo) {
+      // the weighted k and v tiles have been read: the next chunk's q and dy go there
+      load(0, c - 1, off_q(par ^ 1));
+      load(3, c - 1, off_g(par ^ 1));
+    }
     {
       const float kf = carried ? pw[C - 1 - i] : 0.f;
       __nv_bfloat16 *kd = dk + (bh * N + row0 + i) * static_cast<long>(D);
@@ -1330,27 +1350,23 @@ __global__ void __launch_bounds__(NT, 1)
     }
     if (c == c_lo) break;   // the adjoint before the range is not needed here
     // ---- R += (Lq Q)^T w, r likewise: q rows weighted lambda^(t+1)
-    scale_row(sm + kOffQ, sm + kOffQ, i, hf, pw[i + 1]);
+    scale_row(sm + oQ, sm + oQ, i, hf, pw[i + 1]);
     fence_proxy_async_smem();
     if (!meet()) break;
     if (tid == 0) {
       mma_ss(tmem + kTmR, dQm, true, dGm, true, carried);
       umma_commit(bar(kMma));
-      load(1, c - 1);   // k has been read
+      load(1, c - 1, kOffK);   // k has been read
     }
     {
-      // the weighted k tile is done with: its space holds the column-sum partials
+      // the bf16 R operand is done with until the next chunk: its space holds
+      // the column-sum partials
       float rc = 0.f, unused = 0.f;
-      col_sums(sm + kOffQ, sdd, nullptr, nullptr, reinterpret_cast<float *>(sm + kOffKd), rc,
-               unused);
+      col_sums(sm + oQ, sdd, nullptr, nullptr, reinterpret_cast<float *>(sm + kOffRb), rc, unused);
       if (tid < 128) rv[i] = pw[C] * rv[i] + rc;
     }
     mma_done();
     if (!meet()) break;
-    if (tid == 0) {
-      load(0, c - 1);
-      load(3, c - 1);
-    }
   }
   if (tid == 0) {
     for (int b = 0; b < 4; ++b)
