@@ -108,17 +108,20 @@ __device__ __forceinline__ void mma_ts(uint32_t d, uint32_t a, uint64_t b, bool 
                  (acc || ks > 0) ? 1u : 0u);
 }
 
-// The row helpers below work on this thread's half h of row r: 16-byte
-// chunks [8h, 8h + 8), i.e. columns [64h, 64h + 64).
+// The row helpers below work on this thread's part h of row r when the row's
+// 128 columns are cut into P parts (P = 2: the two warpgroups of most passes;
+// P = 4: the reverse pass's four): 16-byte chunks [h 16/P, (h + 1) 16/P).
 
 // The half row through the feature map in place (nothing with `ident`);
 // returns phi(row) . vec over the half (fp32) when vec is given and adds the
 // half row's sum to *sum when sum is given.
+template <int P = 2>
 __device__ __forceinline__ float phi_row(uint8_t *tile, int r, int h, bool ident, const float *vec,
                                          float *sum = nullptr) {
+  constexpr int CH = 16 / P;
   float acc = 0.f, rs = 0.f;
 #pragma unroll 4
-  for (int j = 8 * h; j < 8 * h + 8; ++j) {
+  for (int j = CH * h; j < CH * h + CH; ++j) {
     uint4 *p = reinterpret_cast<uint4 *>(tile + toff(r, j));
     uint4 w = *p;
     if (!ident) {
@@ -148,10 +151,12 @@ __device__ __forceinline__ float elu_f32(float x) { return x > 0.f ? x : __expf(
 // rank-one terms for the 1: for small k, phi(k) is 1 plus a small part that
 // bf16 near 1 would resolve to only ~2^-8, and the gradient of q lives in
 // that part.
+template <int P = 2>
 __device__ __forceinline__ void elu_row(uint8_t *tile, int r, int h, bool ident) {
+  constexpr int CH = 16 / P;
   if (ident) return;
 #pragma unroll 4
-  for (int j = 8 * h; j < 8 * h + 8; ++j) {
+  for (int j = CH * h; j < CH * h + CH; ++j) {
     uint4 *p = reinterpret_cast<uint4 *>(tile + toff(r, j));
     uint4 w = *p;
     w.x = pack_bf16(elu_f32(blo(w.x)), elu_f32(bhi(w.x)));
@@ -163,10 +168,12 @@ __device__ __forceinline__ void elu_row(uint8_t *tile, int r, int h, bool ident)
 }
 
 // dst half row = src half row * f (bf16 product), dst may be src
+template <int P = 2>
 __device__ __forceinline__ void scale_row(uint8_t *dst, const uint8_t *src, int r, int h, float f) {
+  constexpr int CH = 16 / P;
   const uint32_t f2 = pack_bf16(f, f);
 #pragma unroll 4
-  for (int j = 8 * h; j < 8 * h + 8; ++j) {
+  for (int j = CH * h; j < CH * h + CH; ++j) {
     uint4 w = *reinterpret_cast<const uint4 *>(src + toff(r, j));
     w.x = mul_bf16x2(w.x, f2);
     w.y = mul_bf16x2(w.y, f2);
@@ -177,9 +184,11 @@ __device__ __forceinline__ void scale_row(uint8_t *dst, const uint8_t *src, int 
 }
 
 // The half row of dy -> dnum = dy * inv in place (fp32 product, one rounding)
+template <int P = 2>
 __device__ __forceinline__ void dnum_row(uint8_t *tile, int r, int h, float inv) {
+  constexpr int CH = 16 / P;
 #pragma unroll 4
-  for (int j = 8 * h; j < 8 * h + 8; ++j) {
+  for (int j = CH * h; j < CH * h + CH; ++j) {
     uint4 *p = reinterpret_cast<uint4 *>(tile + toff(r, j));
     uint4 g = *p;
     g.x = pack_bf16(blo(g.x) * inv, bhi(g.x) * inv);
@@ -191,19 +200,22 @@ __device__ __forceinline__ void dnum_row(uint8_t *tile, int r, int h, float inv)
 }
 
 // Column sums of one or two bf16 tiles over all 128 rows, each optionally
-// weighted per row, by all 256 threads together; thread k < 128 receives the
-// sums of column k in sa and sb.  Thread t reads 16-byte chunk t % 16 of rows
-// t / 16 + 16 m; partial sums meet through `scratch` (2 x 8 x 128 floats, in
-// no live tile).  Holds two block barriers: every thread calls it.
+// weighted per row, by all T threads of the block together; thread k < 128
+// receives the sums of column k in sa and sb.  Thread t reads 16-byte chunk
+// t % 16 of rows t / 16 + (T / 16) m; partial sums meet through `scratch`
+// (2 x T/32 x 128 floats, in no live tile).  Holds two block barriers: every
+// thread calls it.
+template <int T = NT>
 __device__ __forceinline__ void col_sums(const uint8_t *ta, const float *wa, const uint8_t *tb,
                                          const float *wb, float *scratch, float &sa, float &sb) {
+  constexpr int RG = T / 16, NW = T / 32;   // row groups, warps
   const int t = threadIdx.x, j = t & 15, g = t >> 4, lane = t & 31, w = t >> 5;
   float a[8], b[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) a[e] = b[e] = 0.f;
 #pragma unroll
-  for (int m = 0; m < 8; ++m) {
-    const int r = g + 16 * m;
+  for (int m = 0; m < 128 / RG; ++m) {
+    const int r = g + RG * m;
     const uint4 x = *reinterpret_cast<const uint4 *>(ta + toff(r, j));
     const float fa = wa ? wa[r] : 1.f;
     const uint32_t xs[4] = {x.x, x.y, x.z, x.w};
@@ -232,15 +244,15 @@ __device__ __forceinline__ void col_sums(const uint8_t *ta, const float *wa, con
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
       scratch[w * 128 + 8 * j + e] = a[e];
-      scratch[1024 + w * 128 + 8 * j + e] = b[e];
+      scratch[NW * 128 + w * 128 + 8 * j + e] = b[e];
     }
   __syncthreads();
   if (t < 128) {
     float x = 0.f, y = 0.f;
 #pragma unroll
-    for (int k = 0; k < NT / 32; ++k) {
+    for (int k = 0; k < NW; ++k) {
       x += scratch[k * 128 + t];
-      y += scratch[1024 + k * 128 + t];
+      y += scratch[NW * 128 + k * 128 + t];
     }
     sa = x;
     sb = y;
@@ -264,9 +276,11 @@ __device__ __forceinline__ void fill_masked_tables(float L, int m, float *lower,
 // The half row r of the fp32 state in TMEM (this warp's lanes; t already
 // holds the lane offset) -> bf16 row r of the operand tile, and the state
 // multiplied by `f` written back.
+template <int P = 2>
 __device__ __forceinline__ void state_to_operand(uint32_t t, uint8_t *tile, int r, int h, float f) {
+  constexpr int BL = 4 / P;
 #pragma unroll 1
-  for (int blk = 2 * h; blk < 2 * h + 2; ++blk) {
+  for (int blk = BL * h; blk < BL * h + BL; ++blk) {
     uint32_t v[32];
     tmem_ld_32x32b_x32(t + blk * 32, v);
     tmem_wait_ld();
@@ -285,25 +299,30 @@ __device__ __forceinline__ void state_to_operand(uint32_t t, uint8_t *tile, int 
   tmem_wait_st();
 }
 
+// Sum over the block (at most 16 warps; red holds 16 floats).
 __device__ __forceinline__ float block_sum(float x, float *red) {
   x = warp_sum(x);
-  const int w = threadIdx.x >> 5;
+  const int w = threadIdx.x >> 5, nw = blockDim.x >> 5;
   if ((threadIdx.x & 31) == 0) red[w] = x;
   __syncthreads();
   float s = 0.f;
-#pragma unroll
-  for (int k = 0; k < NT / 32; ++k) s += red[k];
+  for (int k = 0; k < nw; ++k) s += red[k];
   __syncthreads();
   return s;
 }
 
-// Per-row sums of the two halves: slot x holds [2][128] floats.
+// Per-row sums of a row's parts: slot x holds [parts][128] floats.
 struct Halves {
   float *base;
   int h, r;
-  __device__ __forceinline__ void put(int x, float v) const { base[(2 * x + h) * 128 + r] = v; }
+  int parts = 2;
+  __device__ __forceinline__ void put(int x, float v) const {
+    base[(parts * x + h) * 128 + r] = v;
+  }
   __device__ __forceinline__ float get(int x) const {
-    return base[(2 * x) * 128 + r] + base[(2 * x + 1) * 128 + r];
+    float s = 0.f;
+    for (int p = 0; p < parts; ++p) s += base[(parts * x + p) * 128 + r];
+    return s;
   }
 };
 
@@ -325,11 +344,12 @@ constexpr uint32_t kOffK0 = 0, kOffV0 = kTile, kStage = 2 * kTile, kOffMisc = 2 
 enum { kFullK0 = 0, kFullV0, kFullK1, kFullV1, kMma, kFinal, kNumBars };
 constexpr uint32_t kMiscTmem = 64, kMiscFlag = 68, kMiscPw = 128;
 constexpr uint32_t kMiscW = kMiscPw + 132 * 4, kMiscScr = kMiscW + 128 * 4;
-constexpr uint32_t kSmemBytes = kOffMisc + kMiscScr + 2 * 8 * 128 * 4;
+constexpr int kNT = 512, kParts = 4;   // four warpgroups, a quarter of each row each
+constexpr uint32_t kSmemBytes = kOffMisc + kMiscScr + 2 * (kNT / 32) * 128 * 4;
 static_assert(kSmemBytes <= 232448, "exceeds the per-CTA shared memory of sm_100");
 }  // namespace ps
 
-__global__ void __launch_bounds__(NT, 1)
+__global__ void __launch_bounds__(ps::kNT, 1)
     bwd_tc_s_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                     const float *__restrict__ lam, float *__restrict__ mid, int H, int N, int H0,
                     bool ident) {
@@ -417,8 +437,8 @@ __global__ void __launch_bounds__(NT, 1)
     poll(2 * st, c >> 1);
     poll(2 * st + 1, c >> 1);
     if (!meet()) break;
-    elu_row(tk, i, hf, ident);
-    scale_row(tk, tk, i, hf, wr[i]);
+    elu_row<kParts>(tk, i, hf, ident);
+    scale_row<kParts>(tk, tk, i, hf, wr[i]);
     fence_proxy_async_smem();
     if (!meet()) break;
     if (tid == 0) {
@@ -427,7 +447,7 @@ __global__ void __launch_bounds__(NT, 1)
     }
     {
       float zc = 0.f, sc = 0.f;
-      col_sums(tk, nullptr, tv, wr, scr, zc, sc);
+      col_sums<kNT>(tk, nullptr, tv, wr, scr, zc, sc);
       if (tid < 128) {
         zt_acc += zc;
         s_acc += sc;
@@ -442,7 +462,7 @@ __global__ void __launch_bounds__(NT, 1)
   if (!*flag && H0 > 0) {
     float *m = mid + bh * kMidFloats;
 #pragma unroll 1
-    for (int blk = 2 * hf; blk < 2 * hf + 2; ++blk) {
+    for (int blk = hf; blk < hf + 1; ++blk) {
       uint32_t v[32];
       tmem_ld_32x32b_x32(tmem + lf + blk * 32, v);
       tmem_wait_ld();
@@ -496,14 +516,17 @@ constexpr uint32_t kMiscZ = kMiscPwr + 128 * 4, kMiscS = kMiscZ + 128 * 4;
 constexpr uint32_t kMiscGs = kMiscS + 128 * 4, kMiscRed = kMiscGs + 128 * 4;
 constexpr uint32_t kMiscLo = kMiscRed + 64, kMiscDlo = kMiscLo + 256 * 4;
 constexpr uint32_t kMiscX = kMiscDlo + 256 * 4;
+// four warpgroups: thread (h, r) owns the 32 columns [32h, 32h + 32) of row r;
+// the row sums of the parts meet in the exchange slots below
+constexpr int kNT = 512, kParts = 4;
 enum { kXQz = 0, kXRq, kXRs, kXGn, kXSd, kXGw, kXRb, kNumX };
-constexpr uint32_t kSmemBytes = kOffMisc + kMiscX + kNumX * 2 * 128 * 4;
+constexpr uint32_t kSmemBytes = kOffMisc + kMiscX + kNumX * kParts * 128 * 4;
 static_assert(kSmemBytes <= 232448, "exceeds the per-CTA shared memory of sm_100");
 // tensor memory columns
 constexpr uint32_t kTmS = 0, kTmT1 = 128, kTmT2 = 256, kTmA = 384, kTmW = 448;
 }  // namespace pf
 
-__global__ void __launch_bounds__(NT, 1)
+__global__ void __launch_bounds__(pf::kNT, 1)
     bwd_tc_f_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
                     const float *__restrict__ lam, float eps, __nv_bfloat16 *__restrict__ dq,
@@ -542,8 +565,8 @@ __global__ void __launch_bounds__(NT, 1)
   float *red = reinterpret_cast<float *>(misc + kMiscRed);
   float *lo = reinterpret_cast<float *>(misc + kMiscLo);     // masked lambda^(t-s), offset
   float *dlo = reinterpret_cast<float *>(misc + kMiscDlo);   // masked (t-s) lambda^(t-s-1)
-  const int hf = tid >> 7, i = tid & 127;   // column half, row
-  const Halves X{reinterpret_cast<float *>(misc + kMiscX), hf, i};
+  const int hf = tid >> 7, i = tid & 127;   // column part, row
+  const Halves X{reinterpret_cast<float *>(misc + kMiscX), hf, i, kParts};
   const CUtensorMap *maps[4] = {&tm_q, &tm_k, &tm_v, &tm_g};
   const uint32_t offs[4] = {kOffQ, kOffK, kOffV, kOffG};
   int issued[4] = {0, 0, 0, 0}, waited[4] = {0, 0, 0, 0};   // thread 0: copies per tile
@@ -621,7 +644,7 @@ __global__ void __launch_bounds__(NT, 1)
     grid_dependency_wait();
     const float *m = mid + bh * kMidFloats;
 #pragma unroll 1
-    for (int blk = 2 * hf; blk < 2 * hf + 2; ++blk) {
+    for (int blk = hf; blk < hf + 1; ++blk) {
       uint32_t v[32];
       const float4 *src = reinterpret_cast<const float4 *>(m + i * D + blk * 32);
 #pragma unroll
@@ -645,7 +668,7 @@ __global__ void __launch_bounds__(NT, 1)
     tc_fence_after();
   }
   uint8_t *ap_row = sm + kOffAp + static_cast<uint32_t>(i) * 256u;   // At' row (its two halves)
-  const int b0 = 2 * hf;   // this half's first 32-column block
+  const int b0 = hf;   // this part's 32-column block
   const float lf_i = pw[i + 1];
   const float *mk = lo + 127 - i, *dmk = dlo + 127 - i;   // mk[s] = lambda^(i-s) (s <= i) or 0
 
@@ -653,19 +676,19 @@ __global__ void __launch_bounds__(NT, 1)
     const int row0 = c * C, Cv = min(C, N - row0);
     const bool carried = c > c0 || half == 1, last = c == c1 - 1;
     // ---- the state before this chunk: bf16 operand, and lambda^C St kept for the update
-    if (carried) state_to_operand(tmem + kTmS + lf, sm + kOffSb, i, hf, pw[C]);
+    if (carried) state_to_operand<kParts>(tmem + kTmS + lf, sm + kOffSb, i, hf, pw[C]);
     poll(kFullQ, c - c0);
     if (!meet()) break;
     {
       float rqh = 0.f;
-      X.put(kXQz, phi_row(sm + kOffQ, i, hf, ident, zt, &rqh));   // phi(q_i) . zt, half
+      X.put(kXQz, phi_row<kParts>(sm + kOffQ, i, hf, ident, zt, &rqh));   // phi(q_i) . zt, part
       X.put(kXRq, rqh);
     }
     poll(kFullK, c - c0);
     if (!meet()) break;
     const float rq = X.get(kXRq), qzt = X.get(kXQz);
     const float qz = qzt + o * rq * zeta;   // phi(q_i) . z
-    elu_row(sm + kOffK, i, hf, ident);
+    elu_row<kParts>(sm + kOffK, i, hf, ident);
     fence_proxy_async_smem();
     if (!meet()) break;
     if (tid == 0) {
@@ -680,25 +703,26 @@ __global__ void __launch_bounds__(NT, 1)
     if (!meet()) break;
     // ---- At = (Q Kt^T) o M into TMEM (bf16), At' = (Q Kt^T) o M' into shared memory
     {
+      // this part's 32 columns in steps of 16 (x = the step's first column)
       float rsh = 0.f;
 #pragma unroll 1
-      for (int blk = b0; blk < b0 + 2; ++blk) {
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(tmem + lf + kTmT1 + blk * 32, v);
+      for (int x = 32 * b0; x < 32 * b0 + 32; x += 16) {
+        uint32_t v[16];
+        tmem_ld_32x32b_x16(tmem + lf + kTmT1 + x, v);
         tmem_wait_ld();
-        uint32_t pa[16], pp[16];
+        uint32_t pa[8], pp[8];
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          const int s0 = blk * 32 + e, s1 = s0 + 1;
+        for (int e = 0; e < 16; e += 2) {
+          const int s0 = x + e, s1 = s0 + 1;
           const float p0 = __uint_as_float(v[e]), p1 = __uint_as_float(v[e + 1]);
           pa[e / 2] = pack_bf16(p0 * mk[s0], p1 * mk[s1]);
           rsh += blo(pa[e / 2]) + bhi(pa[e / 2]);
           pp[e / 2] = pack_bf16(p0 * dmk[s0], p1 * dmk[s1]);
         }
-        tmem_st_32x32b_x16(tmem + lf + kTmA + blk * 16, pa);
+        tmem_st_32x32b_x8(tmem + lf + kTmA + x / 2, pa);
 #pragma unroll
-        for (int m = 0; m < 4; ++m)
-          *reinterpret_cast<uint4 *>(ap_row + (((blk * 4 + m) ^ (i & 15)) << 4)) =
+        for (int m = 0; m < 2; ++m)
+          *reinterpret_cast<uint4 *>(ap_row + (((x / 8 + m) ^ (i & 15)) << 4)) =
               make_uint4(pp[4 * m], pp[4 * m + 1], pp[4 * m + 2], pp[4 * m + 3]);
       }
       X.put(kXRs, rsh);
@@ -719,19 +743,19 @@ __global__ void __launch_bounds__(NT, 1)
     {
       float gnh = 0.f, sdh = 0.f;   // dnum . (At V + carried part), dnum . s
 #pragma unroll 1
-      for (int blk = b0; blk < b0 + 2; ++blk) {
-        uint32_t av[32], xv[32];
-        tmem_ld_32x32b_x32(tmem + lf + kTmT1 + blk * 32, av);
-        if (carried) tmem_ld_32x32b_x32(tmem + lf + kTmT2 + blk * 32, xv);
+      for (int x = 32 * b0; x < 32 * b0 + 32; x += 16) {
+        uint32_t av[16], xv[16];
+        tmem_ld_32x32b_x16(tmem + lf + kTmT1 + x, av);
+        if (carried) tmem_ld_32x32b_x16(tmem + lf + kTmT2 + x, xv);
         tmem_wait_ld();
-        uint32_t pk[16];
+        uint32_t pk[8];
 #pragma unroll
-        for (int m = 0; m < 4; ++m) {
-          const uint4 g4 = *reinterpret_cast<const uint4 *>(sm + kOffG + toff(i, blk * 4 + m));
+        for (int m = 0; m < 2; ++m) {
+          const uint4 g4 = *reinterpret_cast<const uint4 *>(sm + kOffG + toff(i, x / 8 + m));
           const uint32_t g[4] = {g4.x, g4.y, g4.z, g4.w};
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
-            const int e = 8 * m + 2 * u, v0 = blk * 32 + e;
+            const int e = 8 * m + 2 * u, v0 = x + e;
             float n0 = __uint_as_float(av[e]), n1 = __uint_as_float(av[e + 1]);
             if (carried) {
               n0 += lf_i * (__uint_as_float(xv[e]) + o * rq * sv[v0]);
@@ -746,7 +770,7 @@ __global__ void __launch_bounds__(NT, 1)
             sdh += d0 * sv[v0] + d1 * sv[v0 + 1];
           }
         }
-        tmem_st_32x32b_x16(tmem + lf + kTmW + blk * 16, pk);
+        tmem_st_32x32b_x8(tmem + lf + kTmW + x / 2, pk);
       }
       X.put(kXGn, gnh);
       X.put(kXSd, sdh);
@@ -769,7 +793,7 @@ __global__ void __launch_bounds__(NT, 1)
     {
       float gwh = 0.f;
 #pragma unroll 1
-      for (int blk = b0; blk < b0 + 2; ++blk) {
+      for (int blk = b0; blk < b0 + 1; ++blk) {
         uint32_t v[32];
         tmem_ld_32x32b_x32(tmem + lf + kTmT1 + blk * 32, v);
         tmem_wait_ld();
@@ -787,20 +811,19 @@ __global__ void __launch_bounds__(NT, 1)
     {
       float rbh = 0.f;
 #pragma unroll 1
-      for (int blk = b0; blk < b0 + 2; ++blk) {
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(tmem + lf + kTmT1 + blk * 32, v);
+      for (int x = 32 * b0; x < 32 * b0 + 32; x += 16) {
+        uint32_t v[16];
+        tmem_ld_32x32b_x16(tmem + lf + kTmT1 + x, v);
         tmem_wait_ld();
-        uint32_t pb[16];
+        uint32_t pb[8];
 #pragma unroll
-        for (int m = 0; m < 4; ++m) {
-          const uint4 a4 =
-              *reinterpret_cast<const uint4 *>(ap_row + (((blk * 4 + m) ^ (i & 15)) << 4));
+        for (int m = 0; m < 2; ++m) {
+          const uint4 a4 = *reinterpret_cast<const uint4 *>(ap_row + (((x / 8 + m) ^ (i & 15)) << 4));
           const uint32_t ap[4] = {a4.x, a4.y, a4.z, a4.w};
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
             const int e = 8 * m + 2 * u;
-            const int s0 = blk * 32 + e, s1 = s0 + 1;
+            const int s0 = x + e, s1 = s0 + 1;
             const float w0 = __uint_as_float(v[e]) + dden, w1 = __uint_as_float(v[e + 1]) + dden;
             dl += (blo(ap[u]) + o * rq * dmk[s0]) * w0 + (bhi(ap[u]) + o * rq * dmk[s1]) * w1;
             const float bb0 = w0 * mk[s0], bb1 = w1 * mk[s1];
@@ -808,7 +831,7 @@ __global__ void __launch_bounds__(NT, 1)
             pb[4 * m + u] = pack_bf16(bb0, bb1);
           }
         }
-        tmem_st_32x32b_x16(tmem + lf + kTmA + blk * 16, pb);
+        tmem_st_32x32b_x8(tmem + lf + kTmA + x / 2, pb);
       }
       X.put(kXRb, rbh);
     }
@@ -828,19 +851,19 @@ __global__ void __launch_bounds__(NT, 1)
       const float one = o * (X.get(kXRb) + (carried ? lf_i * (sd + zeta * dden) : 0.f));
       __nv_bfloat16 *dst = dq + (bh * N + row0 + i) * static_cast<long>(D);
 #pragma unroll 1
-      for (int blk = b0; blk < b0 + 2; ++blk) {
-        uint32_t bk[32], uv[32];
-        tmem_ld_32x32b_x32(tmem + lf + kTmT1 + blk * 32, bk);
-        if (carried) tmem_ld_32x32b_x32(tmem + lf + kTmT2 + blk * 32, uv);
+      for (int x = 32 * b0; x < 32 * b0 + 32; x += 16) {
+        uint32_t bk[16], uv[16];
+        tmem_ld_32x32b_x16(tmem + lf + kTmT1 + x, bk);
+        if (carried) tmem_ld_32x32b_x16(tmem + lf + kTmT2 + x, uv);
         tmem_wait_ld();
-        uint32_t pk[16];
+        uint32_t pk[8];
 #pragma unroll
-        for (int m = 0; m < 4; ++m) {
-          const uint4 q4 = *reinterpret_cast<const uint4 *>(sm + kOffQ + toff(i, blk * 4 + m));
+        for (int m = 0; m < 2; ++m) {
+          const uint4 q4 = *reinterpret_cast<const uint4 *>(sm + kOffQ + toff(i, x / 8 + m));
           const uint32_t qw[4] = {q4.x, q4.y, q4.z, q4.w};
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
-            const int e = 8 * m + 2 * u, k0 = blk * 32 + e;
+            const int e = 8 * m + 2 * u, k0 = x + e;
             const float u0 = carried ? __uint_as_float(uv[e]) : 0.f;
             const float u1 = carried ? __uint_as_float(uv[e + 1]) : 0.f;
             const float q0 = blo(qw[u]), q1 = bhi(qw[u]);
@@ -856,8 +879,8 @@ __global__ void __launch_bounds__(NT, 1)
         }
         if (i < Cv)
 #pragma unroll
-          for (int m = 0; m < 4; ++m)
-            reinterpret_cast<uint4 *>(dst + blk * 32)[m] =
+          for (int m = 0; m < 2; ++m)
+            reinterpret_cast<uint4 *>(dst + x)[m] =
                 make_uint4(pk[4 * m], pk[4 * m + 1], pk[4 * m + 2], pk[4 * m + 3]);
       }
       if (carried)
@@ -866,7 +889,7 @@ __global__ void __launch_bounds__(NT, 1)
     }
     if (last) break;
     // ---- state update: key rows weighted lambda^(C-1-s): St += (Lk Kt)^T V, zt, s, zeta likewise
-    scale_row(sm + kOffK, sm + kOffK, i, hf, pwr[i]);
+    scale_row<kParts>(sm + kOffK, sm + kOffK, i, hf, pwr[i]);
     fence_proxy_async_smem();
     if (!meet()) break;
     if (tid == 0) {
@@ -877,8 +900,8 @@ __global__ void __launch_bounds__(NT, 1)
     {
       // the At' tile is done with: its space holds the column-sum partials
       float zc = 0.f, sc = 0.f;
-      col_sums(sm + kOffK, nullptr, sm + kOffV, pwr, reinterpret_cast<float *>(sm + kOffAp), zc,
-               sc);
+      col_sums<kNT>(sm + kOffK, nullptr, sm + kOffV, pwr, reinterpret_cast<float *>(sm + kOffAp),
+                    zc, sc);
       if (tid < 128) {
         zt[i] = pw[C] * zt[i] + zc;
         sv[i] = pw[C] * sv[i] + sc;
@@ -925,11 +948,12 @@ constexpr uint32_t kOffQ0 = 0, kOffG0 = kTile, kStage = 2 * kTile, kOffMisc = 2 
 enum { kFullQ0 = 0, kFullG0, kFullQ1, kFullG1, kMma, kFinal, kNumBars };
 constexpr uint32_t kMiscTmem = 64, kMiscFlag = 68, kMiscPw = 128;
 constexpr uint32_t kMiscDd = kMiscPw + 132 * 4, kMiscScr = kMiscDd + 128 * 4;
-constexpr uint32_t kSmemBytes = kOffMisc + kMiscScr + 2 * 8 * 128 * 4;
+constexpr int kNT = 512, kParts = 4;   // four warpgroups, a quarter of each row each
+constexpr uint32_t kSmemBytes = kOffMisc + kMiscScr + 2 * (kNT / 32) * 128 * 4;
 static_assert(kSmemBytes <= 232448, "exceeds the per-CTA shared memory of sm_100");
 }  // namespace pt
 
-__global__ void __launch_bounds__(NT, 1)
+__global__ void __launch_bounds__(pt::kNT, 1)
     bwd_tc_t_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_g,
                     const float *__restrict__ lam, const float *__restrict__ stash,
                     long stash_stride, float *__restrict__ mid, int H, int N, int H1, bool ident) {
@@ -1021,9 +1045,9 @@ __global__ void __launch_bounds__(NT, 1)
     poll(2 * st, j >> 1);
     poll(2 * st + 1, j >> 1);
     if (!meet()) break;
-    phi_row(tq, i, hf, ident, nullptr);
-    scale_row(tq, tq, i, hf, pow_int(L, j * C) * pw[i + 1]);
-    dnum_row(tg, i, hf, 1.f / den);
+    phi_row<kParts>(tq, i, hf, ident, nullptr);
+    scale_row<kParts>(tq, tq, i, hf, pow_int(L, j * C) * pw[i + 1]);
+    dnum_row<kParts>(tg, i, hf, 1.f / den);
     fence_proxy_async_smem();
     if (!meet()) break;
     if (tid == 0) {
@@ -1032,7 +1056,7 @@ __global__ void __launch_bounds__(NT, 1)
     }
     {
       float rc = 0.f, unused = 0.f;
-      col_sums(tq, dd, nullptr, nullptr, scr, rc, unused);
+      col_sums<kNT>(tq, dd, nullptr, nullptr, scr, rc, unused);
       if (tid < 128) r_acc += rc;
     }
     poll(kMma, mph);
@@ -1043,7 +1067,7 @@ __global__ void __launch_bounds__(NT, 1)
   if (!*flag && n > 0) {
     float *m = mid + bh * kMidFloats;
 #pragma unroll 1
-    for (int blk = 2 * hf; blk < 2 * hf + 2; ++blk) {
+    for (int blk = hf; blk < hf + 1; ++blk) {
       uint32_t v[32];
       tmem_ld_32x32b_x32(tmem + lf + blk * 32, v);
       tmem_wait_ld();
@@ -1079,9 +1103,13 @@ constexpr uint32_t kMiscDden = kMiscUp + 256 * 4, kMiscR = kMiscDden + 128 * 4;
 constexpr uint32_t kSmemBytes = kOffMisc + kMiscR + 128 * 4;
 static_assert(kSmemBytes <= 232448, "exceeds the per-CTA shared memory of sm_100");
 constexpr uint32_t kTmR = 0, kTmT1 = 128, kTmT2 = 256, kTmAt = 384, kTmBt = 448;
+// four warpgroups: thread (h, r) owns the 32 columns [32h, 32h + 32) of row r
+// (the reverse pass has no row sums to join, so more warps only add latency
+// hiding)
+constexpr int kNT = 512, kParts = 4;
 }  // namespace pr
 
-__global__ void __launch_bounds__(NT, 1)
+__global__ void __launch_bounds__(pr::kNT, 1)
     bwd_tc_r_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
                     const float *__restrict__ lam, const float *stash, long stash_stride,
@@ -1180,7 +1208,7 @@ __global__ void __launch_bounds__(NT, 1)
 
   const uint64_t dK = kdesc(sb + kOffK), dV = kdesc(sb + kOffV);
   const uint64_t dRb = kdesc(sb + kOffRb), dRbm = mdesc(sb + kOffRb);
-  const int b0 = 2 * hf;
+  const int b0 = hf;   // this part's 32-column block
   const float *mk = up + 127 - i;   // mk[s] = lambda^(s-i) for s >= i, else 0
   // den, dden of this thread's token in the chunk being processed (tokens past
   // the end: no gradient); the next chunk's pair is loaded a chunk ahead
@@ -1193,7 +1221,7 @@ __global__ void __launch_bounds__(NT, 1)
     grid_dependency_wait();
     const float *m = rmid + bh * kMidFloats;
 #pragma unroll 1
-    for (int blk = 2 * hf; blk < 2 * hf + 2; ++blk) {
+    for (int blk = hf; blk < hf + 1; ++blk) {
       uint32_t v[32];
       const float4 *src = reinterpret_cast<const float4 *>(m + i * D + blk * 32);
 #pragma unroll
@@ -1222,19 +1250,19 @@ __global__ void __launch_bounds__(NT, 1)
                    dGm = mdesc(sb + oG), dKd = kdesc(sb + oKd), dVd = kdesc(sb + oVd);
     const float den = st.x, dden = st.y;
     if (hf == 0) sdd[i] = dden;
-    if (carried) state_to_operand(tmem + kTmR + lf, sm + kOffRb, i, hf, pw[C]);
+    if (carried) state_to_operand<kParts>(tmem + kTmR + lf, sm + kOffRb, i, hf, pw[C]);
     poll(kFullQ, cc);
     poll(kFullK, cc);
     poll(kFullV, cc);
     poll(kFullG, cc);
     if (!meet()) break;
-    phi_row(sm + oQ, i, hf, ident, nullptr);
-    phi_row(sm + kOffK, i, hf, ident, nullptr);
+    phi_row<kParts>(sm + oQ, i, hf, ident, nullptr);
+    phi_row<kParts>(sm + kOffK, i, hf, ident, nullptr);
     if (carried) {
-      scale_row(sm + oKd, sm + kOffK, i, hf, pw[C - 1 - i]);
-      scale_row(sm + oVd, sm + kOffV, i, hf, pw[C - 1 - i]);
+      scale_row<kParts>(sm + oKd, sm + kOffK, i, hf, pw[C - 1 - i]);
+      scale_row<kParts>(sm + oVd, sm + kOffV, i, hf, pw[C - 1 - i]);
     }
-    dnum_row(sm + oG, i, hf, 1.f / den);   // w = dnum in place of dy
+    dnum_row<kParts>(sm + oG, i, hf, 1.f / den);   // w = dnum in place of dy
     fence_proxy_async_smem();
     if (!meet()) break;
     if (tid == 0) {
@@ -1250,7 +1278,7 @@ __global__ void __launch_bounds__(NT, 1)
     if (!meet()) break;
     // ---- A^T and B^T rows (key i, queries s >= i) into TMEM
 #pragma unroll 1
-    for (int blk = b0; blk < b0 + 2; ++blk) {
+    for (int blk = b0; blk < b0 + 1; ++blk) {
       uint32_t pv[32];
       tmem_ld_32x32b_x32(tmem + lf + kTmT1 + blk * 32, pv);
       tmem_wait_ld();
@@ -1265,7 +1293,7 @@ __global__ void __launch_bounds__(NT, 1)
     if (!meet()) break;
     if (tid == 0 && c > c_lo) load(2, c - 1, kOffV);   // v has been read (its weighted copy is made)
 #pragma unroll 1
-    for (int blk = b0; blk < b0 + 2; ++blk) {
+    for (int blk = b0; blk < b0 + 1; ++blk) {
       uint32_t wv[32];
       tmem_ld_32x32b_x32(tmem + lf + kTmT2 + blk * 32, wv);
       tmem_wait_ld();
@@ -1294,7 +1322,7 @@ __global__ void __launch_bounds__(NT, 1)
     {
       __nv_bfloat16 *vd = dv + (bh * N + row0 + i) * static_cast<long>(D);
 #pragma unroll 1
-      for (int blk = b0; blk < b0 + 2; ++blk) {
+      for (int blk = b0; blk < b0 + 1; ++blk) {
         uint32_t a[32];
         tmem_ld_32x32b_x32(tmem + lf + kTmT1 + blk * 32, a);
         tmem_wait_ld();
@@ -1320,7 +1348,7 @@ __global__ void __launch_bounds__(NT, 1)
       const float kf = carried ? pw[C - 1 - i] : 0.f;
       __nv_bfloat16 *kd = dk + (bh * N + row0 + i) * static_cast<long>(D);
 #pragma unroll 1
-      for (int blk = b0; blk < b0 + 2; ++blk) {
+      for (int blk = b0; blk < b0 + 1; ++blk) {
         uint32_t b[32];
         tmem_ld_32x32b_x32(tmem + lf + kTmT2 + blk * 32, b);
         tmem_wait_ld();
@@ -1350,7 +1378,7 @@ __global__ void __launch_bounds__(NT, 1)
     }
     if (c == c_lo) break;   // the adjoint before the range is not needed here
     // ---- R += (Lq Q)^T w, r likewise: q rows weighted lambda^(t+1)
-    scale_row(sm + oQ, sm + oQ, i, hf, pw[i + 1]);
+    scale_row<kParts>(sm + oQ, sm + oQ, i, hf, pw[i + 1]);
     fence_proxy_async_smem();
     if (!meet()) break;
     if (tid == 0) {
@@ -1362,7 +1390,8 @@ __global__ void __launch_bounds__(NT, 1)
       // the bf16 R operand is done with until the next chunk: its space holds
       // the column-sum partials
       float rc = 0.f, unused = 0.f;
-      col_sums(sm + oQ, sdd, nullptr, nullptr, reinterpret_cast<float *>(sm + kOffRb), rc, unused);
+      col_sums<kNT>(sm + oQ, sdd, nullptr, nullptr, reinterpret_cast<float *>(sm + kOffRb), rc,
+                    unused);
       if (tid < 128) rv[i] = pw[C] * rv[i] + rc;
     }
     mma_done();
@@ -1399,15 +1428,17 @@ constexpr uint32_t kMiscDpw = kMiscPw + 132 * 4, kMiscPwr = kMiscDpw + 132 * 4;
 constexpr uint32_t kMiscDpwr = kMiscPwr + 128 * 4, kMiscZ = kMiscDpwr + 128 * 4;
 constexpr uint32_t kMiscZp = kMiscZ + 128 * 4, kMiscS = kMiscZp + 128 * 4;
 constexpr uint32_t kMiscSp = kMiscS + 128 * 4, kMiscWq = kMiscSp + 128 * 4;
+// four warpgroups: thread (h, r) owns the 32 columns [32h, 32h + 32) of row r
+constexpr int kNT = 512, kParts = 4;
 constexpr uint32_t kMiscRed = kMiscWq + 128 * 4, kMiscX = kMiscRed + 64;
 enum { kXQz = 0, kXRq, kNumX };
-constexpr uint32_t kMiscScr = kMiscX + kNumX * 2 * 128 * 4;   // column-sum partials
-constexpr uint32_t kSmemBytes = kOffMisc + kMiscScr + 2 * 8 * 128 * 4;
+constexpr uint32_t kMiscScr = kMiscX + kNumX * kParts * 128 * 4;   // column-sum partials
+constexpr uint32_t kSmemBytes = kOffMisc + kMiscScr + 2 * (kNT / 32) * 128 * 4;
 static_assert(kSmemBytes <= 232448, "exceeds the per-CTA shared memory of sm_100");
 constexpr uint32_t kTmS = 0, kTmSp = 128, kTmM = 256;
 }  // namespace pl
 
-__global__ void __launch_bounds__(NT, 1)
+__global__ void __launch_bounds__(pl::kNT, 1)
     bwd_tc_l_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
                     const float *__restrict__ lam, const float *__restrict__ stash,
@@ -1442,7 +1473,7 @@ __global__ void __launch_bounds__(NT, 1)
   float *red = reinterpret_cast<float *>(misc + kMiscRed);
   float *scr = reinterpret_cast<float *>(misc + kMiscScr);
   const int hf = tid >> 7, i = tid & 127;
-  const Halves X{reinterpret_cast<float *>(misc + kMiscX), hf, i};
+  const Halves X{reinterpret_cast<float *>(misc + kMiscX), hf, i, kParts};
   const CUtensorMap *maps[4] = {&tm_q, &tm_k, &tm_v, &tm_g};
   const uint32_t offs[4] = {kOffQ, kOffK, kOffV, kOffG};
   int issued[4] = {0, 0, 0, 0}, waited[4] = {0, 0, 0, 0};
@@ -1507,7 +1538,7 @@ __global__ void __launch_bounds__(NT, 1)
 
   const uint64_t dQm = mdesc(sb + kOffQ), dKm = mdesc(sb + kOffK), dKpm = mdesc(sb + kOffKp);
   const uint64_t dVm = mdesc(sb + kOffV), dGm = mdesc(sb + kOffG);
-  const int b0 = 2 * hf;
+  const int b0 = hf;   // this part's 32-column block
   float dl = 0.f;
   float zeta = 0.f, zetap = 0.f;
   float geo = 0.f, dgeo = 0.f;
@@ -1534,16 +1565,16 @@ __global__ void __launch_bounds__(NT, 1)
     // q rows weighted lambda^(t+1); the half sums of phi(q) . zt' and of phi(q)
     {
       float rqh = 0.f;
-      X.put(kXQz, phi_row(sm + kOffQ, i, hf, ident, ztp, &rqh));
+      X.put(kXQz, phi_row<kParts>(sm + kOffQ, i, hf, ident, ztp, &rqh));
       X.put(kXRq, rqh);
     }
-    scale_row(sm + kOffQ, sm + kOffQ, i, hf, pw[i + 1]);
-    dnum_row(sm + kOffG, i, hf, 1.f / den);
+    scale_row<kParts>(sm + kOffQ, sm + kOffQ, i, hf, pw[i + 1]);
+    dnum_row<kParts>(sm + kOffG, i, hf, 1.f / den);
     if (!last) {
       // key rows as elu(k), weighted lambda^(C-1-s) (state) and (C-1-s) lambda^(C-2-s) (derivative)
-      elu_row(sm + kOffK, i, hf, ident);
-      scale_row(sm + kOffKp, sm + kOffK, i, hf, dpwr[i]);
-      scale_row(sm + kOffK, sm + kOffK, i, hf, pwr[i]);
+      elu_row<kParts>(sm + kOffK, i, hf, ident);
+      scale_row<kParts>(sm + kOffKp, sm + kOffK, i, hf, dpwr[i]);
+      scale_row<kParts>(sm + kOffK, sm + kOffK, i, hf, pwr[i]);
     }
     fence_proxy_async_smem();
     if (!meet()) break;
@@ -1566,7 +1597,7 @@ __global__ void __launch_bounds__(NT, 1)
     {
       // o s' . (1^T Ms) on this thread's d_v column (s' of the chunk start)
       float cs = 0.f, unused = 0.f;
-      col_sums(sm + kOffG, wq, nullptr, nullptr, scr, cs, unused);
+      col_sums<kNT>(sm + kOffG, wq, nullptr, nullptr, scr, cs, unused);
       if (tid < 128) dl += o * svp[i] * cs;
     }
     mma_done();
@@ -1577,23 +1608,24 @@ __global__ void __launch_bounds__(NT, 1)
     }
     // <St', Ms> on this thread's d_k row; then St' <- lambda^C St' + C lambda^(C-1) St, St <- lambda^C St
     if (carried) {
+      // this part's 32 columns in two steps of 16 (three values live per column)
 #pragma unroll 1
-      for (int blk = b0; blk < b0 + 2; ++blk) {
-        uint32_t sp[32], mv[32], sq[32];
-        tmem_ld_32x32b_x32(tmem + lf + kTmSp + blk * 32, sp);
-        tmem_ld_32x32b_x32(tmem + lf + kTmM + blk * 32, mv);
-        tmem_ld_32x32b_x32(tmem + lf + kTmS + blk * 32, sq);
+      for (int col = 32 * b0; col < 32 * b0 + 32; col += 16) {
+        uint32_t sp[16], mv[16], sq[16];
+        tmem_ld_32x32b_x16(tmem + lf + kTmSp + col, sp);
+        tmem_ld_32x32b_x16(tmem + lf + kTmM + col, mv);
+        tmem_ld_32x32b_x16(tmem + lf + kTmS + col, sq);
         tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
+        for (int e = 0; e < 16; ++e) {
           const float s1 = __uint_as_float(sp[e]), s0 = __uint_as_float(sq[e]);
           dl += s1 * __uint_as_float(mv[e]);
           sp[e] = __float_as_uint(pw[C] * s1 + dpw[C] * s0);
           sq[e] = __float_as_uint(pw[C] * s0);
         }
         if (!last) {
-          tmem_st_32x32b_x32(tmem + lf + kTmSp + blk * 32, sp);
-          tmem_st_32x32b_x32(tmem + lf + kTmS + blk * 32, sq);
+          tmem_st_32x32b_x16(tmem + lf + kTmSp + col, sp);
+          tmem_st_32x32b_x16(tmem + lf + kTmS + col, sq);
         }
       }
       tmem_wait_st();
@@ -1608,8 +1640,8 @@ __global__ void __launch_bounds__(NT, 1)
     }
     {
       float zpc = 0.f, zc = 0.f, spc = 0.f, sc = 0.f;
-      col_sums(sm + kOffKp, nullptr, sm + kOffK, nullptr, scr, zpc, zc);
-      col_sums(sm + kOffV, dpwr, sm + kOffV, pwr, scr, spc, sc);
+      col_sums<kNT>(sm + kOffKp, nullptr, sm + kOffK, nullptr, scr, zpc, zc);
+      col_sums<kNT>(sm + kOffV, dpwr, sm + kOffV, pwr, scr, spc, sc);
       if (tid < 128) {
         ztp[i] = pw[C] * ztp[i] + dpw[C] * zt[i] + zpc;
         zt[i] = pw[C] * zt[i] + zc;

@@ -615,7 +615,7 @@ int bwd_split(const linattn_dims *d) {
   const int BH = d->B * d->H;
   const int nch = (d->N + btc::C - 1) / btc::C;
   const int sms = num_sms();
-  const int H0 = (nch >= 2 && sms > 0 && BH < sms) ? (nch * 100 + 179) / 180 : 0;
+  const int H0 = (nch >= 2 && sms > 0 && BH < sms) ? (nch * 100 + 169) / 170 : 0;
   return H0 >= nch ? 0 : H0;
 }
 
@@ -655,7 +655,8 @@ int launch_bwd_tc(const linattn_dims *d, const void *q, const void *k, const voi
   // (written by the state pass, which runs beside the first halves).  The
   // split point balances the first half against the state pass plus the
   // second half: with the state pass at a fraction a of pass F's time per
-  // chunk, H0 = nch / (2 - a); a is ~0.2.
+  // chunk, H0 = nch / (2 - a); a is ~0.3 (nch / 1.7 timed best against
+  // nch / 1.8 at the full-size workload).
   int H0 = bwd_split(d);
   char *ws = nullptr;
   bool owned = false;
@@ -688,23 +689,23 @@ int launch_bwd_tc(const linattn_dims *d, const void *q, const void *k, const voi
   const long stride = ws ? 2 : btc::D / 2;
   int rc = LINATTN_OK;
   if (H0)
-    rc = launch_pdl(btc::bwd_tc_s_kernel, BH, btc::NT, btc::ps::kSmemBytes, s, false, mk, mv, lam,
+    rc = launch_pdl(btc::bwd_tc_s_kernel, BH, btc::ps::kNT, btc::ps::kSmemBytes, s, false, mk, mv, lam,
                     mid, d->H, d->N, H0, id);
   if (rc == LINATTN_OK)
-    rc = launch_pdl(btc::bwd_tc_f_kernel, H0 ? 2 * BH : BH, btc::NT, btc::pf::kSmemBytes, s,
+    rc = launch_pdl(btc::bwd_tc_f_kernel, H0 ? 2 * BH : BH, btc::pf::kNT, btc::pf::kSmemBytes, s,
                     H0 != 0, mq, mk, mv, mg, lam, eps, bq, stash, stride, dlam,
                     static_cast<const float *>(mid), H0, d->H, d->N, id);
   if (rc == LINATTN_OK && dlam)
-    rc = launch_pdl(btc::bwd_tc_l_kernel, BH, btc::NT, btc::pl::kSmemBytes, s, false, mq, mk, mv,
+    rc = launch_pdl(btc::bwd_tc_l_kernel, BH, btc::pl::kNT, btc::pl::kSmemBytes, s, false, mq, mk, mv,
                     mg, lam, static_cast<const float *>(stash), stride, dlam, d->H, d->N, id);
   // R (and the reverse state pass before it) read nothing that L writes: with
   // the stash out of the dk rows they start beside L as programmatic dependents
   const bool beside_l = ws != nullptr && dlam != nullptr;
   if (rc == LINATTN_OK && H1)
-    rc = launch_pdl(btc::bwd_tc_t_kernel, BH, btc::NT, btc::pt::kSmemBytes, s, beside_l, mq, mg,
+    rc = launch_pdl(btc::bwd_tc_t_kernel, BH, btc::pt::kNT, btc::pt::kSmemBytes, s, beside_l, mq, mg,
                     lam, static_cast<const float *>(stash), stride, rmid, d->H, d->N, H1, id);
   if (rc == LINATTN_OK)
-    rc = launch_pdl(btc::bwd_tc_r_kernel, H1 ? 2 * BH : BH, btc::NT, btc::pr::kSmemBytes, s,
+    rc = launch_pdl(btc::bwd_tc_r_kernel, H1 ? 2 * BH : BH, btc::pr::kNT, btc::pr::kSmemBytes, s,
                     beside_l || H1 != 0, mq, mk, mv, mg, lam, static_cast<const float *>(stash),
                     stride, bk, bv, static_cast<const float *>(rmid), H1, d->H, d->N, id);
   if (owned && cudaFreeAsync(ws, s) != cudaSuccess && rc == LINATTN_OK) rc = LINATTN_ERR_CUDA;
