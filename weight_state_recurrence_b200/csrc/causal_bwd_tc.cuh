@@ -425,6 +425,12 @@ __global__ void __launch_bounds__(ps::kNT, 1)
     return *flag == 0;
   };
   int mph = 0;
+  // every thread waits for the MMA phase itself (see pass F)
+  auto mma_wait_all = [&](int b, int &ph) {
+    if (!*flag && !mbar_wait(bar(b), static_cast<uint32_t>(ph) & 1u)) *flag = 1;
+    ++ph;
+    tc_fence_after();
+  };
   float geo = 0.f;   // sum_s lambda^(C-1-s)
   for (int m = 0; m < C; ++m) geo += pw[m];
   float zt_acc = 0.f, s_acc = 0.f, zeta = 0.f;   // thread i < 128: column i of zt and s
@@ -454,9 +460,7 @@ __global__ void __launch_bounds__(ps::kNT, 1)
       }
     }
     zeta += tc * geo;
-    poll(kMma, mph);
-    ++mph;
-    if (!meet()) break;
+    mma_wait_all(kMma, mph);
     if (tid == 0 && c + 2 < H0) load(c + 2);   // this stage is free
   }
   if (!*flag && H0 > 0) {
@@ -633,6 +637,15 @@ __global__ void __launch_bounds__(pf::kNT, 1)
   auto mma_done = [&]() { poll(kMma, mph); ++mph; };
   int mph2 = 0;  // completed phases of the second MMA barrier (a product an epilogue needs later)
   auto mma2_done = [&]() { poll(kMma2, mph2); ++mph2; };
+  // Every thread waits for an MMA phase itself (no block barrier): a thread
+  // whose wait runs out sets the flag and goes on to the next block barrier,
+  // where all threads leave together.  A block barrier lies between any two
+  // phases of each MMA barrier, so no thread is ever two phases behind.
+  auto mma_wait_all = [&](int b, int &ph) {
+    if (!*flag && !mbar_wait(bar(b), static_cast<uint32_t>(ph) & 1u)) *flag = 1;
+    ++ph;
+    tc_fence_after();
+  };
 
   const uint64_t dQ = kdesc(sb + kOffQ), dK = kdesc(sb + kOffK), dKm = mdesc(sb + kOffK);
   const uint64_t dV = kdesc(sb + kOffV), dVm = mdesc(sb + kOffV);
@@ -699,8 +712,7 @@ __global__ void __launch_bounds__(pf::kNT, 1)
         umma_commit(bar(kMma2));
       }
     }
-    mma_done();
-    if (!meet()) break;
+    mma_wait_all(kMma, mph);
     // ---- At = (Q Kt^T) o M into TMEM (bf16), At' = (Q Kt^T) o M' into shared memory
     {
       // this part's 32 columns in steps of 16 (x = the step's first column)
@@ -786,8 +798,7 @@ __global__ void __launch_bounds__(pf::kNT, 1)
         umma_commit(bar(kMma2));
       }
     }
-    mma_done();
-    if (!meet()) break;
+    mma_wait_all(kMma, mph);
     const float gn = X.get(kXGn), sd = X.get(kXSd);
     // ---- dden = -dnum . num / den, the o rq part from the masked row sum of W
     {
@@ -841,9 +852,8 @@ __global__ void __launch_bounds__(pf::kNT, 1)
       mma_ts(tmem + kTmT1, tmem + kTmA, dKm, true, false);   // B Kt
       umma_commit(bar(kMma));
     }
-    mma_done();
-    if (carried) mma2_done();
-    if (!meet()) break;
+    mma_wait_all(kMma, mph);
+    if (carried) mma_wait_all(kMma2, mph2);
     // ---- dq = (B Kt + o B1 + lambda^(t+1) (U + zt dden + o (s.w + zeta dden))) phi'(q);
     //      dlambda, keys before the chunk (the lambda^(t+1) factor's derivative)
     {
@@ -908,8 +918,7 @@ __global__ void __launch_bounds__(pf::kNT, 1)
       }
     }
     zeta = pw[C] * zeta + geo;
-    mma_done();
-    if (!meet()) break;
+    mma_wait_all(kMma, mph);
     if (tid == 0) {
       load(1, c + 1);
       load(2, c + 1);
@@ -1030,6 +1039,12 @@ __global__ void __launch_bounds__(pt::kNT, 1)
     return *flag == 0;
   };
   int mph = 0;
+  // every thread waits for the MMA phase itself (see pass F)
+  auto mma_wait_all = [&](int b, int &ph) {
+    if (!*flag && !mbar_wait(bar(b), static_cast<uint32_t>(ph) & 1u)) *flag = 1;
+    ++ph;
+    tc_fence_after();
+  };
   float r_acc = 0.f;   // thread i < 128: column i of r
 
   for (int j = 0; j < n; ++j) {
@@ -1059,9 +1074,7 @@ __global__ void __launch_bounds__(pt::kNT, 1)
       col_sums<kNT>(tq, dd, nullptr, nullptr, scr, rc, unused);
       if (tid < 128) r_acc += rc;
     }
-    poll(kMma, mph);
-    ++mph;
-    if (!meet()) break;
+    mma_wait_all(kMma, mph);
     if (tid == 0 && j + 2 < n) load(j + 2);   // this stage is free
   }
   if (!*flag && n > 0) {
@@ -1201,10 +1214,17 @@ __global__ void __launch_bounds__(pr::kNT, 1)
     tc_fence_after();
     return *flag == 0;
   };
-  int mph = 0;
-  auto mma_done = [&]() { poll(kMma, mph); ++mph; };
+  int mph = 0;   // completed phases of the MMA barrier
   int mph2 = 0;  // completed phases of the second MMA barrier (a product an epilogue needs later)
-  auto mma2_done = [&]() { poll(kMma2, mph2); ++mph2; };
+  // Every thread waits for an MMA phase itself (no block barrier): a thread
+  // whose wait runs out sets the flag and goes on to the next block barrier,
+  // where all threads leave together.  A block barrier lies between any two
+  // phases of each MMA barrier, so no thread is ever two phases behind.
+  auto mma_wait_all = [&](int b, int &ph) {
+    if (!*flag && !mbar_wait(bar(b), static_cast<uint32_t>(ph) & 1u)) *flag = 1;
+    ++ph;
+    tc_fence_after();
+  };
 
   const uint64_t dK = kdesc(sb + kOffK), dV = kdesc(sb + kOffV);
   const uint64_t dRb = kdesc(sb + kOffRb), dRbm = mdesc(sb + kOffRb);
@@ -1274,8 +1294,7 @@ __global__ void __launch_bounds__(pr::kNT, 1)
     // the next chunk's den, dden, while the products run
     if (c > c_lo)
       st = *reinterpret_cast<const float2 *>(stash + (bh * N + row0 - C + i) * stash_stride);
-    mma_done();
-    if (!meet()) break;
+    mma_wait_all(kMma, mph);
     // ---- A^T and B^T rows (key i, queries s >= i) into TMEM
 #pragma unroll 1
     for (int blk = b0; blk < b0 + 1; ++blk) {
@@ -1289,8 +1308,7 @@ __global__ void __launch_bounds__(pr::kNT, 1)
                               __uint_as_float(pv[e + 1]) * mk[blk * 32 + e + 1]);
       tmem_st_32x32b_x16(tmem + lf + kTmAt + blk * 16, pa);
     }
-    mma2_done();
-    if (!meet()) break;
+    mma_wait_all(kMma2, mph2);
     if (tid == 0 && c > c_lo) load(2, c - 1, kOffV);   // v has been read (its weighted copy is made)
 #pragma unroll 1
     for (int blk = b0; blk < b0 + 1; ++blk) {
@@ -1316,8 +1334,7 @@ __global__ void __launch_bounds__(pr::kNT, 1)
       if (carried) mma_ss(tmem + kTmT2, dVd, false, dRb, false, true);     // + Lk V R^T
       umma_commit(bar(kMma2));
     }
-    mma_done();
-    if (!meet()) break;
+    mma_wait_all(kMma, mph);
     // ---- dv (while the dk product runs), then dk = (dphi(k) + Lk r) phi'(k)
     {
       __nv_bfloat16 *vd = dv + (bh * N + row0 + i) * static_cast<long>(D);
@@ -1337,8 +1354,7 @@ __global__ void __launch_bounds__(pr::kNT, 1)
                 make_uint4(pv[4 * m], pv[4 * m + 1], pv[4 * m + 2], pv[4 * m + 3]);
       }
     }
-    mma2_done();
-    if (!meet()) break;
+    mma_wait_all(kMma2, mph2);
     if (tid == 0 && c > c_lo) {
       // the weighted k and v tiles have been read: the next chunk's q and dy go there
       load(0, c - 1, off_q(par ^ 1));
@@ -1394,8 +1410,7 @@ __global__ void __launch_bounds__(pr::kNT, 1)
                     unused);
       if (tid < 128) rv[i] = pw[C] * rv[i] + rc;
     }
-    mma_done();
-    if (!meet()) break;
+    mma_wait_all(kMma, mph);
   }
   if (tid == 0) {
     for (int b = 0; b < 4; ++b)
@@ -1533,8 +1548,16 @@ __global__ void __launch_bounds__(pl::kNT, 1)
     tc_fence_after();
     return *flag == 0;
   };
-  int mph = 0;
-  auto mma_done = [&]() { poll(kMma, mph); ++mph; };
+  int mph = 0;   // completed phases of the MMA barrier
+  // Every thread waits for an MMA phase itself (no block barrier): a thread
+  // whose wait runs out sets the flag and goes on to the next block barrier,
+  // where all threads leave together.  A block barrier lies between any two
+  // phases of each MMA barrier, so no thread is ever two phases behind.
+  auto mma_wait_all = [&](int b, int &ph) {
+    if (!*flag && !mbar_wait(bar(b), static_cast<uint32_t>(ph) & 1u)) *flag = 1;
+    ++ph;
+    tc_fence_after();
+  };
 
   const uint64_t dQm = mdesc(sb + kOffQ), dKm = mdesc(sb + kOffK), dKpm = mdesc(sb + kOffKp);
   const uint64_t dVm = mdesc(sb + kOffV), dGm = mdesc(sb + kOffG);
@@ -1600,8 +1623,7 @@ __global__ void __launch_bounds__(pl::kNT, 1)
       col_sums<kNT>(sm + kOffG, wq, nullptr, nullptr, scr, cs, unused);
       if (tid < 128) dl += o * svp[i] * cs;
     }
-    mma_done();
-    if (!meet()) break;
+    mma_wait_all(kMma, mph);
     if (tid == 0 && !last) {
       load(0, c + 1);
       load(3, c + 1);
@@ -1651,8 +1673,7 @@ __global__ void __launch_bounds__(pl::kNT, 1)
     }
     zetap = pw[C] * zetap + dpw[C] * zeta + dgeo;
     zeta = pw[C] * zeta + geo;
-    mma_done();
-    if (!meet()) break;
+    mma_wait_all(kMma, mph);
     if (tid == 0) {
       load(1, c + 1);
       load(2, c + 1);
