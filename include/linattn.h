@@ -31,9 +31,12 @@
  *     (each token then sees only itself: lambda^0 = 1).
  *   - eps >= 0 is added to the denominator ([FW] §4.2, [LN] §4.1 1e-6).
  *   - Every pointer is a device pointer, 16-byte aligned.  The caller owns
- *     every buffer.  The library allocates no memory, keeps no per-call state
- *     and never synchronises; work is queued on `stream` (NULL: the legacy
- *     default stream).  Inputs must not alias outputs.
+ *     every buffer.  The library keeps no per-call state and never
+ *     synchronises; it allocates no memory, except that linattn_bwd_causal
+ *     takes its tensor-core workspace as a stream-ordered allocation on
+ *     `stream` (linattn_bwd_causal_ws takes the caller's instead).  Work is
+ *     queued on `stream` (NULL: the legacy default stream).  Inputs must not
+ *     alias outputs.
  *   - Supported sizes: dk and dv in {16, 32, 64, 128}; B, H, N >= 0 with
  *     B*H*N*max(dk,dv) < 2^31.  dtype LINATTN_BF16 or LINATTN_F32.
  *
