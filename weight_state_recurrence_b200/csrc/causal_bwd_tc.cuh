@@ -45,13 +45,14 @@
 // Every power is a table entry lambda^m or m lambda^(m-1) formed directly, so
 // lambda = 0 and lambda = 1 need no special case.
 //
-// Each pass is two warpgroups that own the same rows (thread = row of the token
-// tile or of the state, TMEM lane = row) and split each row's 128 columns in
-// halves; row sums meet through shared memory at the block barriers.  Thread
-// 0 issues the MMAs in program order: the role split and the deep pipelines
-// of the forward are not used here.  Waits are bounded: thread 0 polls, the
-// verdict goes through shared memory to a block barrier, and on a timeout
-// every thread leaves the chunk loop together.
+// Each pass is four warpgroups (512 threads) that own the same rows (thread =
+// row of the token tile or of the state, TMEM lane = row) and split each row's
+// 128 columns in quarters; row sums meet through shared memory at the block
+// barriers.  Thread 0 issues the MMAs in program order: the role split and the
+// deep pipelines of the forward are not used here.  Waits are bounded: thread
+// 0 polls the copy barriers and every thread the MMA barriers; a wait that
+// runs out sets a shared flag, and every thread leaves the chunk loop together
+// at the next block barrier.
 #pragma once
 #include "common.cuh"
 #include "sm100.cuh"
@@ -66,7 +67,6 @@ using tc::phi_bf16x2;
 
 constexpr int C = 128;     // tokens per chunk
 constexpr int D = 128;     // d_k = d_v
-constexpr int NT = 256;    // two warpgroups: thread (h, r) owns columns [64h, 64h + 64) of row r
 constexpr uint32_t kPanel = 128u * 128u;   // 128 rows x 128 bytes (64 bf16)
 constexpr uint32_t kTile = 2u * kPanel;    // 128 x 128 bf16 in two 64-column panels
 
@@ -109,13 +109,13 @@ __device__ __forceinline__ void mma_ts(uint32_t d, uint32_t a, uint64_t b, bool 
 }
 
 // The row helpers below work on this thread's part h of row r when the row's
-// 128 columns are cut into P parts (P = 2: the two warpgroups of most passes;
-// P = 4: the reverse pass's four): 16-byte chunks [h 16/P, (h + 1) 16/P).
+// 128 columns are cut into P parts (the passes use P = 4, one per
+// warpgroup): 16-byte chunks [h 16/P, (h + 1) 16/P).
 
 // The half row through the feature map in place (nothing with `ident`);
 // returns phi(row) . vec over the half (fp32) when vec is given and adds the
 // half row's sum to *sum when sum is given.
-template <int P = 2>
+template <int P>
 __device__ __forceinline__ float phi_row(uint8_t *tile, int r, int h, bool ident, const float *vec,
                                          float *sum = nullptr) {
   constexpr int CH = 16 / P;
@@ -151,7 +151,7 @@ __device__ __forceinline__ float elu_f32(float x) { return x > 0.f ? x : __expf(
 // rank-one terms for the 1: for small k, phi(k) is 1 plus a small part that
 // bf16 near 1 would resolve to only ~2^-8, and the gradient of q lives in
 // that part.
-template <int P = 2>
+template <int P>
 __device__ __forceinline__ void elu_row(uint8_t *tile, int r, int h, bool ident) {
   constexpr int CH = 16 / P;
   if (ident) return;
@@ -168,7 +168,7 @@ __device__ __forceinline__ void elu_row(uint8_t *tile, int r, int h, bool ident)
 }
 
 // dst half row = src half row * f (bf16 product), dst may be src
-template <int P = 2>
+template <int P>
 __device__ __forceinline__ void scale_row(uint8_t *dst, const uint8_t *src, int r, int h, float f) {
   constexpr int CH = 16 / P;
   const uint32_t f2 = pack_bf16(f, f);
@@ -184,7 +184,7 @@ __device__ __forceinline__ void scale_row(uint8_t *dst, const uint8_t *src, int 
 }
 
 // The half row of dy -> dnum = dy * inv in place (fp32 product, one rounding)
-template <int P = 2>
+template <int P>
 __device__ __forceinline__ void dnum_row(uint8_t *tile, int r, int h, float inv) {
   constexpr int CH = 16 / P;
 #pragma unroll 4
@@ -205,7 +205,7 @@ __device__ __forceinline__ void dnum_row(uint8_t *tile, int r, int h, float inv)
 // t % 16 of rows t / 16 + (T / 16) m; partial sums meet through `scratch`
 // (2 x T/32 x 128 floats, in no live tile).  Holds two block barriers: every
 // thread calls it.
-template <int T = NT>
+template <int T>
 __device__ __forceinline__ void col_sums(const uint8_t *ta, const float *wa, const uint8_t *tb,
                                          const float *wb, float *scratch, float &sa, float &sb) {
   constexpr int RG = T / 16, NW = T / 32;   // row groups, warps
@@ -276,7 +276,7 @@ __device__ __forceinline__ void fill_masked_tables(float L, int m, float *lower,
 // The half row r of the fp32 state in TMEM (this warp's lanes; t already
 // holds the lane offset) -> bf16 row r of the operand tile, and the state
 // multiplied by `f` written back.
-template <int P = 2>
+template <int P>
 __device__ __forceinline__ void state_to_operand(uint32_t t, uint8_t *tile, int r, int h, float f) {
   constexpr int BL = 4 / P;
 #pragma unroll 1
